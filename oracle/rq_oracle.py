@@ -1,0 +1,450 @@
+"""CPU oracle for the ResidualQuant hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+arm of ``bench.py`` may import this module.  The product path (the CUDA
+library and its Python binding) never imports it, and this module imports
+nothing from the product path: the two share no code, constant or table.
+
+What it computes follows "ResidualQuant: KV Cache Quantization for Looped
+Transformers with 2-Bit Residuals" (Kim et al., 2026), cited below as [RQ]:
+
+* abstract: the final loop's KV states are the reference; the other loops are
+  stored as low-precision residuals, with least-squares scaling, rotations
+  applied to the residuals and loop-wise mixed precision;
+* Figure 1, steps (1)-(5): direct INT2 quantisation, Last-loop residual,
+  least-square scaling, rotation, mixed precision;
+* Figure 2 caption: the residual ``K_2 - alpha_2 K_1``;
+* Figure 3 caption: "alpha = 1" is the no-LS ablation;
+* Table 5 caption: INT2 group size 16/32, INT4 group size 32;
+* Table 8 caption: the effective bitwidth counts quantised values, scales,
+  offsets and LS coefficients.
+
+The pages print no equations, so the encoder's arithmetic is fixed by a written
+specification that this module follows step for step (all in IEEE binary32
+with round-to-nearest-even, each operation rounded separately):
+
+  alpha  (per vector of 128, separately for K and V)
+      lane j (0..15) owns elements 8j..8j+7; p_j = +0, then p_j += x_e * r_e
+      for e in order; then p_j += p_{j xor o} for o = 8, 4, 2, 1;
+      alpha = num / den (den == 0 -> 0), stored as fp16 (RNE).
+      alpha mode "one" stores 1, mode "zero" stores 0.
+  residual  r_e = x_e - (alpha_hat * ref_e)
+  rotation  (if enabled) unnormalised fast Walsh-Hadamard transform, strides
+      h = 1, 2, ..., 64, butterfly (a, b) -> (a + b, a - b) with a the lower
+      index; then each element times fl32(1/sqrt(128)).  The rotation is the
+      orthonormal Sylvester Hadamard matrix (the pages' OptR-H is not defined
+      on them; this build uses the plain Hadamard it is built on).
+  quantiser per group of g contiguous (rotated) coordinates, b bits:
+      mn = min + 0, mx = max + 0 (the "+ 0" makes a zero unsigned),
+      s = (mx - mn) / (2^b - 1); s_hat = fp16(s); z_hat = fp16(mn);
+      code = clamp(rint((y - z_hat) / s_hat), 0, 2^b - 1), code = 0 if s_hat == 0.
+  INT4 anchor: the reference loop is group-quantised directly (4 bits, g = 32,
+      no alpha, no rotation); the other loops take their alpha and residual
+      against its dequantised value  ref_hat = z_hat + (code * s_hat)  (fp32).
+
+Reconstruction and decode attention are computed in float64 from the stored
+codes and metadata.  The rotation there is an explicit 128x128 matrix built
+from its definition, not a fast transform.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against facts
+that do not come from this module (closed forms, brute force, a library
+Hadamard, the bitwidths printed on the pages).  Parity unpinned: none of the
+functions below; the pages' accuracy and NMSE tables need model weights and
+are out of scope.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+D = 128
+F32 = np.float32
+F16 = np.float16
+INV_SQRT_D_F32 = np.float32(1.0 / np.sqrt(128.0))
+FP16_MAX = 65504.0
+
+ALPHA_LS, ALPHA_ONE, ALPHA_ZERO = 0, 1, 2
+
+
+# ---------------------------------------------------------------------------
+# Rotation
+# ---------------------------------------------------------------------------
+
+def hadamard_pm1(n: int = D) -> np.ndarray:
+    """Sylvester Hadamard matrix with entries (-1)^popcount(i & j), float64."""
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    x = np.bitwise_and(i, j)
+    parity = np.zeros_like(x)
+    while np.any(x):
+        parity ^= x & 1
+        x = x >> 1
+    return np.where(parity == 0, 1.0, -1.0)
+
+
+def hadamard_orthonormal(n: int = D) -> np.ndarray:
+    """H / sqrt(n): orthonormal and symmetric, so it is its own inverse."""
+    return hadamard_pm1(n) / np.sqrt(float(n))
+
+
+def fwht_fp32(x: np.ndarray) -> np.ndarray:
+    """The encoder's rotation in binary32: butterflies at strides 1..64, then
+    the fl32(1/sqrt(128)) scale.  ``x``: float32 [..., 128]."""
+    y = np.asarray(x, dtype=F32).copy()
+    lead = y.shape[:-1]
+    h = 1
+    while h < D:
+        y = y.reshape(lead + (D // (2 * h), 2, h))
+        a = y[..., 0, :]
+        b = y[..., 1, :]
+        y = np.stack([a + b, a - b], axis=-2).reshape(lead + (D,))
+        h *= 2
+    return (y * INV_SQRT_D_F32).astype(F32)
+
+
+# ---------------------------------------------------------------------------
+# Least-squares scale ([RQ] Figure 1 step (3); Figure 2 caption)
+# ---------------------------------------------------------------------------
+
+def lane_tree_dot_fp32(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """<a, b> over the last axis (128) in the specified binary32 order."""
+    prod = (np.asarray(a, F32) * np.asarray(b, F32)).astype(F32)
+    prod = prod.reshape(prod.shape[:-1] + (16, 8))
+    p = np.zeros(prod.shape[:-1], dtype=F32)
+    for e in range(8):
+        p = (p + prod[..., e]).astype(F32)
+    lane = np.arange(16)
+    for o in (8, 4, 2, 1):
+        p = (p + p[..., lane ^ o]).astype(F32)
+    return p[..., 0]
+
+
+def ls_alpha_fp32(x: np.ndarray, ref: np.ndarray, mode: int = ALPHA_LS) -> np.ndarray:
+    """Stored (fp16) scale alpha_hat per vector; x, ref float32 [..., 128].
+
+    LS mode: alpha = <x, ref> / <ref, ref>, the minimiser of ||x - a ref||^2.
+    """
+    lead = np.asarray(x).shape[:-1]
+    if mode == ALPHA_ONE:
+        return np.ones(lead, dtype=F16)
+    if mode == ALPHA_ZERO:
+        return np.zeros(lead, dtype=F16)
+    num = lane_tree_dot_fp32(x, ref)
+    den = lane_tree_dot_fp32(ref, ref)
+    with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+        alpha = np.where(den == 0, F32(0), num / np.where(den == 0, F32(1), den)).astype(F32)
+        return alpha.astype(F16)
+
+
+# ---------------------------------------------------------------------------
+# Asymmetric group quantiser ([RQ] Table 5 caption: INT2 g = 16/32, INT4 g = 32;
+# Table 8 caption: scales and offsets per group)
+# ---------------------------------------------------------------------------
+
+@dataclass
+class QuantGroups:
+    codes: np.ndarray      # uint8 [..., 128]
+    scale: np.ndarray      # float16 [..., 128 // g]
+    zero: np.ndarray       # float16 [..., 128 // g]
+    near_tie: np.ndarray   # bool [..., 128]: within 1 fp32 ulp of a rounding midpoint
+
+
+def quantize_groups_fp32(y: np.ndarray, bits: int, g: int) -> QuantGroups:
+    """Min-max asymmetric quantiser of float32 ``y`` [..., 128] in groups of g."""
+    y = np.asarray(y, dtype=F32)
+    lead = y.shape[:-1]
+    ng = D // g
+    yg = y.reshape(lead + (ng, g))
+    qmax = F32((1 << bits) - 1)
+    mn = (yg.min(axis=-1) + F32(0)).astype(F32)
+    mx = (yg.max(axis=-1) + F32(0)).astype(F32)
+    with np.errstate(over="ignore", invalid="ignore", divide="ignore"):
+        s = ((mx - mn).astype(F32) / qmax).astype(F32)
+        s_hat = s.astype(F16)
+        z_hat = mn.astype(F16)
+        sf = s_hat.astype(F32)[..., None]
+        zf = z_hat.astype(F32)[..., None]
+        ok = sf > 0
+        u = ((yg - zf).astype(F32) / np.where(ok, sf, F32(1))).astype(F32)
+        c = np.clip(np.rint(u), 0, qmax)
+        c = np.where(ok, c, 0).astype(np.uint8)
+        # exact quotient from the same binary32 operands: flag near-midpoints
+        u64 = (yg.astype(np.float64) - zf.astype(np.float64)) / np.where(ok, sf, F32(1)).astype(np.float64)
+        mid = np.floor(u64) + 0.5
+        ulp = np.spacing(np.abs(mid).astype(F32)).astype(np.float64)
+        near = ok & (np.abs(u64 - mid) <= ulp)
+    return QuantGroups(codes=c.reshape(lead + (D,)), scale=s_hat, zero=z_hat,
+                       near_tie=near.reshape(lead + (D,)))
+
+
+def dequant_fp32(q: QuantGroups, g: int) -> np.ndarray:
+    """z_hat + (code * s_hat) in binary32 (the encoder's view of an INT4 anchor)."""
+    lead = q.codes.shape[:-1]
+    c = q.codes.reshape(lead + (D // g, g)).astype(F32)
+    v = (q.zero.astype(F32)[..., None] + (c * q.scale.astype(F32)[..., None]).astype(F32)).astype(F32)
+    return v.reshape(lead + (D,))
+
+
+def dequant_f64(codes: np.ndarray, scale: np.ndarray, zero: np.ndarray, g: int) -> np.ndarray:
+    """z_hat + code * s_hat in float64."""
+    lead = codes.shape[:-1]
+    c = codes.reshape(lead + (D // g, g)).astype(np.float64)
+    v = zero.astype(np.float64)[..., None] + c * scale.astype(np.float64)[..., None]
+    return v.reshape(lead + (D,))
+
+
+# ---------------------------------------------------------------------------
+# Encode ([RQ] abstract; Figure 1 steps (2)-(5))
+# ---------------------------------------------------------------------------
+
+@dataclass
+class CacheConfig:
+    num_loops: int
+    bits: Sequence[int]        # per loop; last = reference: 16 (bf16) or 4 (INT4 g=32)
+    group: Sequence[int]
+    rotate: Sequence[int]
+    alpha_mode: Sequence[int]
+
+    @staticmethod
+    def from_dict(d: dict) -> "CacheConfig":
+        return CacheConfig(d["num_loops"], list(d["bits"]), list(d["group"]),
+                           list(d["rotate"]), list(d["alpha_mode"]))
+
+    @property
+    def ref(self) -> int:
+        return self.num_loops - 1
+
+
+@dataclass
+class EncodedPlane:
+    """One loop's K or V as stored: codes/meta (+ alpha for residual loops)."""
+    codes: np.ndarray
+    scale: np.ndarray
+    zero: np.ndarray
+    alpha: Optional[np.ndarray]
+    near_tie: np.ndarray
+    bits: int
+    group: int
+    rotate: int
+
+
+@dataclass
+class Encoded:
+    cfg: CacheConfig
+    ref_bf16: Dict[str, np.ndarray] = field(default_factory=dict)      # 'k','v' float32 values
+    ref_q: Dict[str, EncodedPlane] = field(default_factory=dict)       # INT4 anchor
+    ref_hat32: Dict[str, np.ndarray] = field(default_factory=dict)     # encoder's fp32 view of ref
+    loops: List[Dict[str, EncodedPlane]] = field(default_factory=list)
+    error: bool = False
+
+
+def _check_range(x: np.ndarray) -> bool:
+    return bool(np.all(np.isfinite(x)) and np.all(np.abs(x) <= FP16_MAX))
+
+
+def encode_fp32emu(K: np.ndarray, V: np.ndarray, cfg: CacheConfig) -> Encoded:
+    """Encode every loop of the cached tokens.
+
+    K, V: float32 [L, ..., 128] holding bf16 values (any leading shape after
+    the loop axis, e.g. [B, H, T]).  The last loop is the reference.
+    """
+    L = cfg.num_loops
+    assert K.shape[0] == L and V.shape == K.shape
+    enc = Encoded(cfg=cfg)
+    enc.error = not (_check_range(K) and _check_range(V))
+    rb = cfg.bits[cfg.ref]
+    for name, X in (("k", K), ("v", V)):
+        ref = np.asarray(X[cfg.ref], dtype=F32)
+        if rb == 16:
+            enc.ref_bf16[name] = ref
+            enc.ref_hat32[name] = ref
+        elif rb == 4:
+            qg = quantize_groups_fp32(ref, 4, 32)
+            enc.ref_q[name] = EncodedPlane(qg.codes, qg.scale, qg.zero, None, qg.near_tie, 4, 32, 0)
+            enc.ref_hat32[name] = dequant_fp32(qg, 32)
+        else:
+            raise ValueError("reference bits must be 16 or 4")
+    for l in range(L - 1):
+        planes = {}
+        for name, X in (("k", K), ("v", V)):
+            x = np.asarray(X[l], dtype=F32)
+            ref = enc.ref_hat32[name]
+            a_hat = ls_alpha_fp32(x, ref, cfg.alpha_mode[l])
+            if not np.all(np.isfinite(a_hat.astype(np.float64))):
+                enc.error = True
+            a32 = a_hat.astype(F32)[..., None]
+            r = (x - (a32 * ref).astype(F32)).astype(F32)
+            y = fwht_fp32(r) if cfg.rotate[l] else r
+            qg = quantize_groups_fp32(y, cfg.bits[l], cfg.group[l])
+            if not (np.all(np.isfinite(qg.scale.astype(np.float64))) and
+                    np.all(np.isfinite(qg.zero.astype(np.float64)))):
+                enc.error = True
+            planes[name] = EncodedPlane(qg.codes, qg.scale, qg.zero, a_hat, qg.near_tie,
+                                        cfg.bits[l], cfg.group[l], cfg.rotate[l])
+        enc.loops.append(planes)
+    return enc
+
+
+# ---------------------------------------------------------------------------
+# Reconstruction (float64)
+# ---------------------------------------------------------------------------
+
+def reference_f64(enc: Encoded, name: str) -> np.ndarray:
+    """The decoder's reference: exact bf16 values, or the INT4 anchor dequantised in float64."""
+    if enc.cfg.bits[enc.cfg.ref] == 16:
+        return enc.ref_bf16[name].astype(np.float64)
+    p = enc.ref_q[name]
+    return dequant_f64(p.codes, p.scale, p.zero, 32)
+
+
+def residual_f64(p: EncodedPlane) -> np.ndarray:
+    """Dequantised residual in the original (unrotated) domain, float64."""
+    y = dequant_f64(p.codes, p.scale, p.zero, p.group)
+    if p.rotate:
+        y = y @ hadamard_orthonormal(D)  # H symmetric: row-vector form of H y
+    return y
+
+
+def reconstruct_f64(enc: Encoded, loop: int):
+    """(K_hat, V_hat) float64 of one loop: alpha_hat * ref + H^T deq(codes)."""
+    if loop == enc.cfg.ref:
+        return reference_f64(enc, "k"), reference_f64(enc, "v")
+    out = []
+    for name in ("k", "v"):
+        p = enc.loops[loop][name]
+        ref = reference_f64(enc, name)
+        out.append(p.alpha.astype(np.float64)[..., None] * ref + residual_f64(p))
+    return out[0], out[1]
+
+
+# ---------------------------------------------------------------------------
+# Decode attention (float64)
+# ---------------------------------------------------------------------------
+
+def _softmax_combine(scores: List[np.ndarray]):
+    s = np.concatenate(scores)
+    if s.size == 0:
+        return None, None
+    m = s.max()
+    p = np.exp(s - m)
+    return p, p.sum()
+
+
+def decode_attention_f64(enc: Encoded, loop: int, q: np.ndarray, ctx_len: np.ndarray,
+                         k_tail: Optional[np.ndarray] = None, v_tail: Optional[np.ndarray] = None,
+                         scale: float = 1.0 / np.sqrt(128.0)) -> np.ndarray:
+    """Decode attention of one loop, scored in the rotated domain.
+
+    q: [B, Hq, 128]; ctx_len: [B]; k_tail/v_tail: [B, Hkv, n_tail, 128] (bf16
+    values of the current token(s), attended unquantised).  For a residual loop
+    each cached token's score is
+        scale * (alpha_K (q . ref_k) + (H q) . deq(codes_K))
+    and the output is
+        (sum_t p_t alpha_V,t ref_v,t + H^T sum_t p_t deq(codes_V,t) + sum_tail p v) / sum p.
+    Returns float64 [B, Hq, 128].
+    """
+    cfg = enc.cfg
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, _ = q.shape
+    refk = reference_f64(enc, "k")
+    refv = reference_f64(enc, "v")
+    Hkv = refk.shape[1]
+    G = Hq // Hkv
+    Hn = hadamard_orthonormal(D)
+    out = np.zeros((B, Hq, D))
+    is_ref = loop == cfg.ref
+    if not is_ref:
+        pk, pv = enc.loops[loop]["k"], enc.loops[loop]["v"]
+        yk = dequant_f64(pk.codes, pk.scale, pk.zero, pk.group)
+        yv = dequant_f64(pv.codes, pv.scale, pv.zero, pv.group)
+    for b in range(B):
+        n = int(ctx_len[b])
+        for qh in range(Hq):
+            h = qh // G
+            qv = q[b, qh]
+            scores = []
+            if is_ref:
+                scores.append(scale * (refk[b, h, :n] @ qv))
+            else:
+                qr = Hn @ qv if pk.rotate else qv
+                ak = pk.alpha[b, h, :n].astype(np.float64)
+                scores.append(scale * (ak * (refk[b, h, :n] @ qv) + yk[b, h, :n] @ qr))
+            if k_tail is not None and k_tail.shape[2] > 0:
+                scores.append(scale * (np.asarray(k_tail[b, h], np.float64) @ qv))
+            p, lsum = _softmax_combine(scores)
+            if p is None:
+                continue
+            pc, pt = p[:n], p[n:]
+            if is_ref:
+                o = pc @ refv[b, h, :n]
+            else:
+                av = pv.alpha[b, h, :n].astype(np.float64)
+                acc_res = pc @ yv[b, h, :n]
+                if pv.rotate:
+                    acc_res = Hn @ acc_res
+                o = (pc * av) @ refv[b, h, :n] + acc_res
+            if pt.size:
+                o = o + pt @ np.asarray(v_tail[b, h], np.float64)
+            out[b, qh] = o / lsum
+    return out
+
+
+def attention_f64(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, ctx_len: np.ndarray,
+                  k_tail: Optional[np.ndarray] = None, v_tail: Optional[np.ndarray] = None,
+                  scale: float = 1.0 / np.sqrt(128.0)) -> np.ndarray:
+    """Brute-force softmax(q K^T * scale) V over given (reconstructed or bf16)
+    caches Kc, Vc [B, Hkv, T, 128] followed by the tail tokens."""
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, _ = q.shape
+    Hkv = Kc.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, D))
+    for b in range(B):
+        n = int(ctx_len[b])
+        for qh in range(Hq):
+            h = qh // G
+            Kb = np.asarray(Kc[b, h, :n], np.float64)
+            Vb = np.asarray(Vc[b, h, :n], np.float64)
+            if k_tail is not None and k_tail.shape[2] > 0:
+                Kb = np.concatenate([Kb, np.asarray(k_tail[b, h], np.float64)])
+                Vb = np.concatenate([Vb, np.asarray(v_tail[b, h], np.float64)])
+            if Kb.shape[0] == 0:
+                continue
+            s = scale * (Kb @ q[b, qh])
+            w = np.exp(s - s.max())
+            out[b, qh] = (w @ Vb) / w.sum()
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Effective bitwidth ([RQ] Table 5, Table 8 and Table 10 captions: values,
+# scales, offsets and LS coefficients are counted)
+# ---------------------------------------------------------------------------
+
+def effective_bitwidth(blocks: Sequence[Sequence[int]], group: int, head_dim: int = 128,
+                       residual: bool = True, meta_bits: int = 16, alpha_bits: int = 16,
+                       anchor_group: int = 32) -> float:
+    """Average stored bits per KV element over all loops.
+
+    ``blocks``: one list of per-loop bit widths per anchor interval; the last
+    entry of each list is that interval's anchor (reference) loop.  A loop
+    quantised to b bits with group g costs b + meta_bits/g per element (g is
+    ``group`` for 2-bit loops and ``anchor_group`` for 4-bit loops); a bf16
+    loop costs 16.  In residual mode every non-anchor loop also stores one
+    LS coefficient of ``alpha_bits`` per head_dim-element vector.
+    """
+    total, n = 0.0, 0
+    for blk in blocks:
+        for i, b in enumerate(blk):
+            if b == 16:
+                cost = 16.0
+            else:
+                g = group if b == 2 else anchor_group
+                cost = b + meta_bits / g
+            if residual and i != len(blk) - 1:
+                cost += alpha_bits / head_dim
+            total += cost
+            n += 1
+    return total / n

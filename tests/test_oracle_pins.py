@@ -1,0 +1,320 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle.
+
+Source of the method: "ResidualQuant: KV Cache Quantization for Looped
+Transformers with 2-Bit Residuals" (Kim et al., 2026), cited as [RQ].
+
+Each pin is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong sign, a transposed operand, an off-by-one group) fails at least one of
+them; ``test_oracle_mutations.py`` plants such slips and checks that they do.
+"""
+import math
+import os
+from decimal import ROUND_HALF_UP, Decimal
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle.rq_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16_values(rng, shape, scale=1.0):
+    """float32 arrays whose values are exactly representable in bf16."""
+    x = (rng.standard_normal(shape) * scale).astype(np.float32)
+    u = x.view(np.uint32)
+    # round to nearest even on the 16 dropped bits
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return u.view(np.float32)
+
+
+# ---------------------------------------------------------------- P1: alpha
+
+def brute_force_ls_scale(x, r):
+    """argmin_a ||x - a r||^2 by a grid scan then golden-section refinement."""
+    x = x.astype(np.float64)
+    r = r.astype(np.float64)
+
+    def f(a):
+        d = x - a * r
+        return float(d @ d)
+
+    grid = np.linspace(-4.0, 4.0, 8001)
+    vals = np.array([f(a) for a in grid])
+    i = int(np.argmin(vals))
+    lo, hi = grid[max(i - 1, 0)], grid[min(i + 1, len(grid) - 1)]
+    phi = (math.sqrt(5) - 1) / 2
+    for _ in range(200):
+        a1 = hi - phi * (hi - lo)
+        a2 = lo + phi * (hi - lo)
+        if f(a1) < f(a2):
+            hi = a2
+        else:
+            lo = a1
+    return 0.5 * (lo + hi)
+
+
+def test_p1_alpha_minimises_squared_error():
+    rng = np.random.default_rng(11)
+    for _ in range(12):
+        ref = bf16_values(rng, (128,), scale=rng.uniform(0.5, 3))
+        x = bf16_values(rng, (128,)) * np.float32(0.3) + np.float32(rng.uniform(-2, 2)) * ref
+        a_star = brute_force_ls_scale(x, ref)
+        a_hat = float(O.ls_alpha_fp32(x, ref))
+        # fp16 storage: within half an fp16 ulp (plus fp32 noise) of the minimiser
+        ulp16 = float(np.spacing(np.float16(abs(a_star))))
+        assert abs(a_hat - a_star) <= 0.5 * ulp16 + 1e-6 * abs(a_star) + 1e-9
+
+
+def test_p1_tree_dot_matches_float64_within_rounding():
+    rng = np.random.default_rng(12)
+    a = rng.standard_normal((64, 128)).astype(np.float32)
+    b = rng.standard_normal((64, 128)).astype(np.float32)
+    got = O.lane_tree_dot_fp32(a, b).astype(np.float64)
+    exact = np.einsum("nd,nd->n", a.astype(np.float64), b.astype(np.float64))
+    bound = 20 * 2.0 ** -24 * np.einsum("nd,nd->n", np.abs(a), np.abs(b))
+    assert np.all(np.abs(got - exact) <= bound)
+
+
+def test_p1_alpha_modes_and_zero_reference():
+    rng = np.random.default_rng(13)
+    x = bf16_values(rng, (4, 128))
+    ref = bf16_values(rng, (4, 128))
+    assert np.all(O.ls_alpha_fp32(x, ref, O.ALPHA_ONE) == 1)
+    assert np.all(O.ls_alpha_fp32(x, ref, O.ALPHA_ZERO) == 0)
+    assert np.all(O.ls_alpha_fp32(x, np.zeros_like(ref)) == 0)
+
+
+# ---------------------------------------------------------- P2: zero residual
+
+@pytest.mark.parametrize("c", [1.0, -1.0, 2.0, -2.0, 0.5, -0.5])
+@pytest.mark.parametrize("rotate", [0, 1])
+def test_p2_scaled_copy_has_zero_residual(c, rotate):
+    rng = np.random.default_rng(21)
+    B, H, T = 1, 2, 9
+    ref = bf16_values(rng, (B, H, T, 128), scale=1.5)
+    K = np.stack([np.float32(c) * ref, ref]).astype(np.float32)
+    V = np.stack([np.float32(-c) * ref, ref]).astype(np.float32)
+    cfg = O.CacheConfig(2, [2, 16], [32, 32], [rotate, 0], [O.ALPHA_LS, O.ALPHA_LS])
+    enc = O.encode_fp32emu(K, V, cfg)
+    pk = enc.loops[0]["k"]
+    assert np.all(pk.alpha.astype(np.float64) == c)
+    assert np.all(pk.codes == 0) and np.all(pk.scale == 0) and np.all(pk.zero == 0)
+    kh, vh = O.reconstruct_f64(enc, 0)
+    assert np.array_equal(kh, K[0].astype(np.float64))
+    assert np.array_equal(vh, V[0].astype(np.float64))
+
+
+# ------------------------------------------------ P3: direct quantisation
+
+def nearest_level_codes(x, scale, zero, bits, g):
+    """Textbook rounding: the level z + c*s (c in 0..2^b-1) nearest to x."""
+    lead = x.shape[:-1]
+    xs = x.reshape(lead + (128 // g, g)).astype(np.float64)
+    levels = zero.astype(np.float64)[..., None, None] + \
+        np.arange(1 << bits)[None, :] * scale.astype(np.float64)[..., None, None]
+    # levels: [..., ng, 1, 2^b]; distances [..., ng, g, 2^b]
+    d = np.abs(xs[..., None] - levels)
+    return np.argmin(d, axis=-1).reshape(lead + (128,))
+
+
+@pytest.mark.parametrize("bits,g", [(2, 32), (2, 16), (4, 32), (4, 16)])
+def test_p3_alpha_zero_without_rotation_is_plain_group_quantisation(bits, g):
+    rng = np.random.default_rng(31 + bits + g)
+    B, H, T = 2, 2, 33
+    K = bf16_values(rng, (2, B, H, T, 128), scale=2.0)
+    V = bf16_values(rng, (2, B, H, T, 128), scale=0.7)
+    cfg = O.CacheConfig(2, [bits, 16], [g, 32], [0, 0], [O.ALPHA_ZERO, O.ALPHA_LS])
+    enc = O.encode_fp32emu(K, V, cfg)
+    for name, X in (("k", K), ("v", V)):
+        p = enc.loops[0][name]
+        x = X[0]
+        assert np.all(p.alpha == 0)
+        xs = x.reshape(x.shape[:-1] + (128 // g, g)).astype(np.float64)
+        mn, mx = xs.min(-1), xs.max(-1)
+        # the stored offset is the fp16 value nearest the group minimum
+        assert np.all(np.abs(p.zero.astype(np.float64) - mn) <= 0.5 * np.spacing(np.abs(mn).astype(np.float16)).astype(np.float64))
+        # the stored scale is within one fp16 ulp of (max - min) / (2^b - 1)
+        s = (mx - mn) / ((1 << bits) - 1)
+        assert np.all(np.abs(p.scale.astype(np.float64) - s) <= np.spacing(s.astype(np.float16)).astype(np.float64))
+        want = nearest_level_codes(x, p.scale, p.zero, bits, g)
+        ok = ~p.near_tie
+        assert np.array_equal(p.codes[ok], want[ok])
+        # reconstruction is the textbook z + c * s
+        kh, vh = O.reconstruct_f64(enc, 0)
+        got = kh if name == "k" else vh
+        c = p.codes.reshape(x.shape[:-1] + (128 // g, g)).astype(np.float64)
+        want_rec = (p.zero.astype(np.float64)[..., None] + c * p.scale.astype(np.float64)[..., None])
+        assert np.array_equal(got, want_rec.reshape(x.shape))
+
+
+# --------------------------------------------------------------- P4: Hadamard
+
+def test_p4_hadamard_matches_library_and_is_orthogonal():
+    H = O.hadamard_pm1(128)
+    assert np.array_equal(H, scipy.linalg.hadamard(128).astype(np.float64))
+    Hi = H.astype(np.int64)
+    assert np.array_equal(Hi @ Hi.T, 128 * np.eye(128, dtype=np.int64))
+    Hn = O.hadamard_orthonormal(128)
+    assert np.allclose(Hn @ Hn, np.eye(128), atol=1e-14)
+
+
+def test_p4_fast_transform_equals_matrix():
+    rng = np.random.default_rng(41)
+    x = rng.standard_normal((50, 128)).astype(np.float32)
+    got = O.fwht_fp32(x).astype(np.float64)
+    want = x.astype(np.float64) @ scipy.linalg.hadamard(128).T / np.sqrt(128.0)
+    err = np.abs(got - want).max(axis=1)
+    assert np.all(err <= 16 * 2.0 ** -24 * np.abs(x).sum(axis=1) / np.sqrt(128))
+    # basis vectors map to columns of H scaled by fl32(1/sqrt(128)) exactly
+    eye = np.eye(128, dtype=np.float32)
+    cols = O.fwht_fp32(eye)
+    assert np.array_equal(cols, (scipy.linalg.hadamard(128).T * np.float32(1 / np.sqrt(128.0))).astype(np.float32))
+    assert np.float32(1 / np.sqrt(128.0)).view(np.uint32) == 0x3DB504F3
+
+
+# --------------------------------------------------------- P5: quantiser bounds
+
+@pytest.mark.parametrize("bits,g", [(2, 32), (2, 16), (4, 32)])
+def test_p5_quantiser_error_bound(bits, g):
+    rng = np.random.default_rng(51)
+    y = (rng.standard_normal((400, 128)) * rng.uniform(0.01, 5, (400, 1))).astype(np.float32)
+    q = O.quantize_groups_fp32(y, bits, g)
+    qmax = (1 << bits) - 1
+    assert q.codes.max() <= qmax
+    deq = O.dequant_f64(q.codes, q.scale, q.zero, g)
+    ys = y.reshape(400, 128 // g, g).astype(np.float64)
+    mn = ys.min(-1)
+    s = (ys.max(-1) - mn) / qmax
+    sh = q.scale.astype(np.float64)
+    zh = q.zero.astype(np.float64)
+    bound = 0.5 * sh + qmax * np.abs(sh - s) + np.abs(zh - mn) + 1e-7 * np.abs(ys).max(-1)
+    err = np.abs(deq.reshape(ys.shape) - ys).max(-1)
+    assert np.all(err <= bound)
+
+
+# ------------------------------------------------------------- P6: decode
+
+def _small_case(seed, B=2, Hkv=2, G=2, T=23, bits=(2, 16), group=(32, 32), rotate=(1, 0), n_tail=1,
+                lens=None):
+    rng = np.random.default_rng(seed)
+    L = len(bits)
+    ref = bf16_values(rng, (B, Hkv, T, 128), scale=1.3)
+    K = [bf16_values(rng, (B, Hkv, T, 128), scale=0.2) + np.float32(0.9) * ref for _ in range(L - 1)]
+    K = np.stack(K + [ref]).astype(np.float32)
+    vref = bf16_values(rng, (B, Hkv, T, 128))
+    V = [bf16_values(rng, (B, Hkv, T, 128), scale=0.3) + np.float32(1.1) * vref for _ in range(L - 1)]
+    V = np.stack(V + [vref]).astype(np.float32)
+    cfg = O.CacheConfig(L, list(bits), list(group), list(rotate), [0] * L)
+    enc = O.encode_fp32emu(K, V, cfg)
+    q = bf16_values(rng, (B, Hkv * G, 128))
+    kt = bf16_values(rng, (B, Hkv, n_tail, 128))
+    vt = bf16_values(rng, (B, Hkv, n_tail, 128))
+    ctx = np.array(lens if lens is not None else [T] * B)
+    return enc, q, ctx, kt, vt
+
+
+@pytest.mark.parametrize("bits,rotate", [((2, 16), (1, 0)), ((4, 4), (1, 0)), ((2, 4), (0, 0))])
+def test_p6_rotated_domain_decode_equals_brute_force(bits, rotate):
+    enc, q, ctx, kt, vt = _small_case(61, bits=bits, rotate=rotate, lens=[23, 7])
+    for loop in range(2):
+        got = O.decode_attention_f64(enc, loop, q, ctx, kt, vt)
+        Kh, Vh = O.reconstruct_f64(enc, loop)
+        want = O.attention_f64(q, Kh, Vh, ctx, kt, vt)
+        assert np.abs(got - want).max() <= 1e-12 * max(1.0, np.abs(want).max())
+
+
+def test_p6_two_token_softmax_by_hand():
+    enc, q, ctx, kt, vt = _small_case(62, B=1, Hkv=1, G=1, T=2, n_tail=0)
+    Kh, Vh = O.reconstruct_f64(enc, 0)
+    got = O.decode_attention_f64(enc, 0, q, ctx, kt[:, :, :0], vt[:, :, :0])[0, 0]
+    tau = 1 / math.sqrt(128)
+    s1 = tau * float(np.dot(q[0, 0].astype(np.float64), Kh[0, 0, 0]))
+    s2 = tau * float(np.dot(q[0, 0].astype(np.float64), Kh[0, 0, 1]))
+    w1 = 1.0 / (1.0 + math.exp(s2 - s1))
+    want = w1 * Vh[0, 0, 0] + (1 - w1) * Vh[0, 0, 1]
+    assert np.abs(got - want).max() <= 1e-12
+
+
+def test_p6_empty_context_and_tail_only():
+    enc, q, ctx, kt, vt = _small_case(63, lens=[0, 5])
+    got = O.decode_attention_f64(enc, 0, q, ctx, kt, vt)
+    # sequence 0 attends only to its single tail token: output == that token's value
+    G = q.shape[1] // kt.shape[1]
+    for qh in range(q.shape[1]):
+        assert np.array_equal(got[0, qh], vt[0, qh // G, 0].astype(np.float64))
+    none = O.decode_attention_f64(enc, 0, q, np.array([0, 0]), kt[:, :, :0], vt[:, :, :0])
+    assert np.all(none == 0)
+
+
+# ------------------------------------------------------------- P7: LS <= alpha=1
+
+def test_p7_ls_scaling_never_worse_than_unit_scale():
+    rng = np.random.default_rng(71)
+    ref = bf16_values(rng, (500, 128), scale=1.0)
+    x = (np.float32(0.7) * ref + bf16_values(rng, (500, 128), scale=0.3)).astype(np.float32)
+    a = O.ls_alpha_fp32(x, ref).astype(np.float64)[:, None]
+    e_ls = ((x - a * ref) ** 2).sum(1)
+    e_one = ((x - ref) ** 2).sum(1)
+    # fp16 storage of alpha can cost at most (0.5 ulp16)^2 * ||ref||^2 over the optimum
+    slack = (0.5 * np.spacing(np.abs(a[:, 0]).astype(np.float16)).astype(np.float64)) ** 2 * (ref.astype(np.float64) ** 2).sum(1)
+    assert np.all(e_ls <= e_one + slack + 1e-9)
+    assert np.mean(e_ls) < 0.8 * np.mean(e_one)
+
+
+# -------------------------------------------------------- P8: rotation is undone
+
+@pytest.mark.parametrize("rotate", [0, 1])
+def test_p8_full_precision_residual_reconstructs(rotate):
+    rng = np.random.default_rng(81)
+    ref = bf16_values(rng, (64, 128), scale=1.2)
+    x = (np.float32(0.95) * ref + bf16_values(rng, (64, 128), scale=0.25)).astype(np.float32)
+    a = O.ls_alpha_fp32(x, ref)
+    r = (x - (a.astype(np.float32)[:, None] * ref).astype(np.float32)).astype(np.float32)
+    y = O.fwht_fp32(r) if rotate else r
+    # undo with the float64 machinery that reconstruction uses (no quantisation)
+    back = y.astype(np.float64) @ O.hadamard_orthonormal(128) if rotate else y.astype(np.float64)
+    xr = a.astype(np.float64)[:, None] * ref.astype(np.float64) + back
+    assert np.abs(xr - x).max() <= 1e-6 * np.abs(x).max()
+
+
+# --------------------------------------------------- P9: bitwidths on the pages
+
+def _parse_blocks(s):
+    s = s.strip()
+    if "*" in s:
+        n, blk = s.split("*", 1)
+        blk = [int(v) for v in blk.strip("() ").split(",")]
+        return [blk] * int(n)
+    return [[int(v) for v in s.split(",")]]
+
+
+def _round_printed(x, printed):
+    places = len(printed.split(".")[1]) if "." in printed else 0
+    q = Decimal(1).scaleb(-places)
+    return Decimal(repr(x)).quantize(q, rounding=ROUND_HALF_UP)
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield [c.strip() for c in line.split("|")]
+
+
+def test_p9_effective_bitwidth_matches_pages():
+    n = 0
+    for where, mode, blocks, g, hd, printed in _rows("beff_pages.txt"):
+        b = O.effective_bitwidth(_parse_blocks(blocks), int(g), head_dim=int(hd),
+                                 residual=(mode == "residual"))
+        assert _round_printed(b, printed) == Decimal(printed), (where, b, printed)
+        n += 1
+    assert n == 13
+
+
+def test_p9_storage_reduction_matches_abstract():
+    for printed, blocks, g, hd in _rows("storage_reduction_pages.txt"):
+        b = O.effective_bitwidth(_parse_blocks(blocks), int(g), head_dim=int(hd))
+        assert _round_printed(100 * (1 - b / 16), printed) == Decimal(printed)
