@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the ResidualQuant hot path on B200.
+
+One step = one decode step of a 4-loop looped model's attention layer over a
+synthetic Ouro-1.4B-shaped cache (16 KV heads, head_dim 128, batch 16, 8192
+cached tokens): decode attention of every loop (three INT2 residual loops and
+the bf16 reference loop, each with the current token as a bf16 tail), then the
+encode of the new token into every loop's cache.  ``value`` is decode tokens/s
+(sequences x steps / s) over all ranks; the same step over a plain bf16 cache
+(same library, same kernels without the residual) is reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rq|reference]
+                    [--workload ouro8k|mixed|gqa|tiny] [--batch B]
+
+Multi-GPU (torchrun) runs independent replicas, one per rank (the path has no
+exchange step); timing is the max over ranks.  ``--impl reference`` times the
+CPU oracle (the reference arm for this method) on bounded samples.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from looped_transformer_decode_rq_b200 import synth  # noqa: E402
+
+METRIC = "RQ decode-attn tokens/s & HBM GB/s (% of B200 peak) at 8k ctx vs BF16 cache"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "rq_decode_split_ouro8k_traffic.txt")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["rq", "reference"], default="rq")
+    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "tiny"], default="ouro8k")
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-bf16", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def make_workload(args) -> synth.Workload:
+    if args.workload == "ouro8k":
+        return synth.ouro_8k(batch=args.batch or 16)
+    if args.workload == "mixed":
+        return synth.mixed_int4_anchor(batch=args.batch or 8)
+    if args.workload == "gqa":
+        return synth.gqa_long(batch=args.batch or 8)
+    return synth.tiny()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ---------------------------------------------------------------------------
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self):
+        self.proc = None
+        self.path = None
+        sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        self.sel = sel
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *self.sel, f"--query-gpu={CLOCK_FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# workload bytes (algorithmic: each record read once per call)
+# ---------------------------------------------------------------------------
+
+def record_bytes(lay, cfgd, loop):
+    L = cfgd["num_loops"]
+    ref = 2 * lay.ref_record_bytes + 2 * lay.ref_meta_record_bytes
+    if loop == L - 1:
+        return ref
+    res = 2 * lay.codes_record_bytes[loop] + 2 * lay.meta_record_bytes[loop]
+    if cfgd["alpha_mode"][loop] == 2:
+        return res
+    return ref + res + 4
+
+
+def call_bytes(lay, cfgd, loop, tokens_total, B, Hq, Hkv, n_tail):
+    return (tokens_total * Hkv * record_bytes(lay, cfgd, loop) + B * Hq * 128 * (2 + 4) +
+            B * Hkv * n_tail * 512)
+
+
+def source_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_profile_traffic(kernel_hash):
+    """Per-launch DRAM bytes of the split kernel from the committed ncu summary,
+    if it was taken on the current kernel source."""
+    if not os.path.exists(PROFILE_TRAFFIC):
+        return None
+    vals = {}
+    for line in open(PROFILE_TRAFFIC):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_hash:
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch_scaled"])
+    except (KeyError, ValueError):
+        return None
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """One (sequence, kv-head) slab of the workload, encoded by the oracle.
+    A sample step = decode attention of every loop for that slab's G q-heads
+    plus the encode of its new token; the full step is B*Hkv such samples."""
+
+    def __init__(self, wl, inp, b=0, h=0):
+        import oracle.rq_oracle as O
+        self.O = O
+        self.wl = wl
+        G = wl.gqa
+        sl = lambda t: t[:, b:b + 1, h:h + 1].float().cpu().numpy()  # noqa: E731
+        self.K, self.V = sl(inp["k"]), sl(inp["v"])
+        self.kt, self.vt = sl(inp["k_tail"]), sl(inp["v_tail"])
+        self.q = inp["q"][:, b:b + 1, h * G:(h + 1) * G].float().cpu().numpy()
+        self.ctx = np.array([int(inp["ctx_len"][b])])
+        self.cfg = O.CacheConfig.from_dict(synth.cache_config_dict(wl))
+        self.enc = O.encode_fp32emu(self.K, self.V, self.cfg)
+        self.b, self.h = b, h
+
+    def step(self):
+        O = self.O
+        outs = [O.decode_attention_f64(self.enc, l, self.q[l], self.ctx, self.kt[l], self.vt[l])
+                for l in range(self.wl.num_loops)]
+        O.encode_fp32emu(self.kt, self.vt, self.cfg)
+        return outs
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(sample, wl, seconds, min_reps=1):
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        sample.step()
+        reps += 1
+        el = time.perf_counter() - t0
+        if reps >= min_reps and el >= seconds:
+            break
+    per_sample = el / reps
+    full_step = per_sample * wl.batch * wl.kv_heads
+    return wl.batch / full_step, per_sample, reps
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+def run_rq(args, world, rank):
+    from looped_transformer_decode_rq_b200 import rq
+
+    wl = make_workload(args).with_(seed=make_workload(args).seed + 1000 * rank)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = synth.make_inputs(wl, dev)
+    L, B, Hkv, Hq, T = wl.num_loops, wl.batch, wl.kv_heads, wl.q_heads, wl.context
+    cfgd = synth.cache_config_dict(wl, capacity=T + 1)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
+    cache.encode(inp["k"], inp["v"])
+    ctx = inp["ctx_len"]
+    tokens_total = int(ctx.sum().item())
+    pos = ctx.clone()  # the new token goes to position ctx_len[b]
+    k_new = inp["k_tail"][:, :, :, :1].contiguous()
+    v_new = inp["v_tail"][:, :, :, :1].contiguous()
+    q = inp["q"]
+    outs = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
+    lay = cache.layout
+    stream = torch.cuda.current_stream()
+    n_tail = 1
+
+    ev_pairs = []
+
+    def step(record=False):
+        for l in range(L):
+            if record and l < L - 1:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
+            if record and l < L - 1:
+                e1.record(stream)
+                ev_pairs.append((e0, e1))
+        cache.encode(k_new, v_new, positions=pos)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flags = cache.get_error()
+
+    # parity spot check of the timed launch configuration (rank 0: sequence 0, kv-head 0)
+    parity = None
+    sample = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(wl, inp, 0, 0)
+        want = sample.step()
+        G = wl.gqa
+        errs = []
+        for l in range(L):
+            got = outs[l, 0, :G].cpu().numpy()
+            w = want[l][0]
+            errs.append(float((np.abs(got - w).max(-1) / np.abs(w).max(-1)).max()))
+        parity = {"max_rel_err": max(errs), "tol": 2e-3, "sampled": f"b=0, q-heads 0..{G - 1}, all {L} loops"}
+
+    clocks = ClockSampler()
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    ms = max_over_ranks(ms, world)
+    call_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_pairs)
+    flags |= cache.get_error()
+
+    res_bytes = call_bytes(lay, cfgd, 0, tokens_total, B, Hq, Hkv, n_tail)
+    step_bytes = sum(call_bytes(lay, cfgd, l, tokens_total, B, Hq, Hkv, n_tail) for l in range(L))
+    step_bytes += L * B * Hkv * 512 + B * Hkv * (sum(record_bytes(lay, cfgd, l) for l in range(L)))
+    peak, peak_kind = load_peaks()
+    kernel_hash = source_hash([os.path.join(ROOT, "looped_transformer_decode_rq_b200", "csrc", f)
+                               for f in ("rq_decode.cu", "rq_common.cuh")])
+    achieved = res_bytes / (call_ms * 1e-3) / 1e9
+    traffic = read_profile_traffic(kernel_hash)
+    value = B * world / (ms * 1e-3)
+
+    # ---- e2e through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q.cpu())
+        hk = torch.empty(k_new.shape, dtype=k_new.dtype, pin_memory=True).copy_(k_new.cpu())
+        hv = torch.empty(v_new.shape, dtype=v_new.dtype, pin_memory=True).copy_(v_new.cpu())
+        hout = torch.empty(outs.shape, dtype=outs.dtype, pin_memory=True)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            for l in range(L):
+                cache.decode_attention(l, dq[l], ctx, dk[l], dv[l], out=outs[l])
+            cache.encode(dk, dv, positions=pos)
+            hout.copy_(outs, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier(world)
+        torch.cuda.synchronize()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b2.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ems = max_over_ranks(a.elapsed_time(b2) / args.steps, world)
+        e2e = {"value": round(B * world / (ems * 1e-3), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
+               "d2h_bytes_per_step": int(hout.numel() * 4)}
+
+    # ---- the same step over a bf16 cache (same library)
+    bf16 = None
+    if not args.no_bf16:
+        kc = [inp["k"][l] for l in range(L)]
+        vc = [inp["v"][l] for l in range(L)]
+        ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+
+        def bf16_step():
+            for l in range(L):
+                rq.bf16_decode_attention(kc[l], vc[l], q[l], ctx, k_new[l], v_new[l], workspace=ws, out=outs[l])
+
+        for _ in range(args.warmup):
+            bf16_step()
+        barrier(world)
+        torch.cuda.synchronize()
+        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            bf16_step()
+        b2.record(stream)
+        torch.cuda.synchronize()
+        bms = max_over_ranks(a.elapsed_time(b2) / args.steps, world)
+        bf_bytes = L * (tokens_total * Hkv * 512 + B * Hq * 128 * 6 + B * Hkv * n_tail * 512)
+        bf16 = {"tokens_per_s": round(B * world / (bms * 1e-3), 1), "ms_per_step": round(bms, 4),
+                "hbm_gbs": round(bf_bytes / (bms * 1e-3) / 1e9, 1),
+                "bytes_per_step": bf_bytes, "rq_speedup": round(bms / ms, 3)}
+
+    # ---- CPU oracle on a bounded sample (rank 0, N = 1 only)
+    cpu = None
+    if sample is not None:
+        v, per, reps = time_oracle(sample, wl, args.cpu_seconds)
+        cpu = {"value": round(v, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": (f"float64 NumPy oracle: decode of all {L} loops for sequence 0, kv-head 0 "
+                          f"({wl.gqa} q-head(s), {int(ctx[0])} cached tokens + 1 tail) plus the encode "
+                          f"of its new token, {reps} reps of {per:.3f} s; scaled by B*Hkv={B * Hkv}")}
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+int2 (fp32 math)",
+        "data": "synthetic (seeded generator; Ouro-1.4B-shaped caches, random values)",
+        "config": {"workload": wl.name, "global_batch": B * world, "seq_len": T, "loops": L,
+                   "kv_heads": Hkv, "q_heads": Hq, "head_dim": 128, "bits": list(wl.bits),
+                   "group": list(wl.group), "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (>= 1 GB read per call), no flush"},
+        "hbm_gbs_step": round(step_bytes / (ms * 1e-3) / 1e9, 1),
+        "bytes_per_step": step_bytes,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "kernel": "rq_decode_attention on a residual loop (split + combine kernels)",
+                     "algorithmic_bytes_per_launch": res_bytes, "launch_ms": round(call_ms, 4),
+                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
+                     "frac_of_8tbs": round(achieved / 8000.0, 4)},
+        "cpu_baseline": cpu, "e2e": e2e, "bf16_cache": bf16, "parity": parity,
+        "gpu_launches": args.steps * (2 * L + 1), "clocks": clk, "device_flags": flags,
+    }
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    wl = make_workload(args)
+    inp = synth.make_inputs(wl.with_(context=wl.context), "cuda" if torch.cuda.is_available() else "cpu")
+    sample = OracleSample(wl, inp, 0, 0)
+    for _ in range(args.warmup):
+        sample.step()
+    t = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        sample.step()
+        t.append(time.perf_counter() - t0)
+    per = statistics.mean(t)
+    full = per * wl.batch * wl.kv_heads
+    value = wl.batch / full
+    cpu = {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+           "sample": (f"one (sequence, kv-head) slab per step: decode of all {wl.num_loops} loops over "
+                      f"{wl.context} tokens + encode of the new token; scaled by B*Hkv={wl.batch * wl.kv_heads}")}
+    out = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(full * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+           "config": {"workload": wl.name, "global_batch": wl.batch, "seq_len": wl.context},
+           "impl": "reference", "cpu_baseline": cpu,
+           "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out))
+
+
+def main():
+    args = parse_args()
+    world, rank = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_rq(args, world, rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

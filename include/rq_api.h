@@ -1,0 +1,236 @@
+/*
+ * rq_api.h -- C ABI of the B200 ResidualQuant hot path (librq_b200.so).
+ *
+ * Method: "ResidualQuant: KV Cache Quantization for Looped Transformers with
+ * 2-Bit Residuals" (Kim et al., 2026), cited below as [RQ].  A looped
+ * Transformer writes one KV cache per loop.  The final loop's keys/values are
+ * kept as the reference (bf16, or an INT4 "anchor"); every other loop l is
+ * stored as a least-squares scaled, Hadamard-rotated, group-quantised residual
+ *      K_l  ~  alpha_l * K_ref  +  H^T deq(codes_l)        (likewise V)
+ * ([RQ] abstract; Figure 1 steps 2-5; Figure 2 caption).  Decode attention
+ * scores each cached token as  alpha (q . K_ref) + (H q) . deq(codes)  and
+ * never materialises a bf16 copy of loop l.
+ *
+ * Conventions shared by every entry point:
+ *  - Memory: the caller owns all device memory and streams.  The library
+ *    allocates nothing on the device; a cache handle holds only host metadata.
+ *  - Asynchrony: calls that take a cudaStream_t enqueue work on that stream and
+ *    return without synchronising (rq_get_error is the one exception).
+ *  - Errors: argument errors are detected on the host before anything is
+ *    enqueued and are returned as RQ_ERR_INVALID_ARG / RQ_ERR_UNSUPPORTED /
+ *    RQ_ERR_CAPACITY / RQ_ERR_WORKSPACE; a failed launch returns RQ_ERR_CUDA.
+ *    Conditions only the device can see (non-finite inputs, a length beyond
+ *    capacity, a pipeline wait that timed out) set bits of the cache's device
+ *    status word, read by rq_get_error.  rq_last_error_message() returns a
+ *    human-readable reason for the calling thread's last non-OK status.
+ *  - Loop index is 0-based; loop num_loops-1 is the reference loop.
+ *  - head_dim is 128 everywhere (the rotation is the order-128 Hadamard).
+ *  - All tensors are row-major and contiguous unless strides are passed.
+ */
+#ifndef RQ_API_H
+#define RQ_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of this header are the library's only exported names. */
+#if defined(__GNUC__)
+#define RQ_API __attribute__((visibility("default")))
+#else
+#define RQ_API
+#endif
+
+/* A CUDA stream handle (cudaStream_t); 0 is the legacy default stream. */
+typedef void* rq_stream_t;
+
+#define RQ_MAX_LOOPS 16
+#define RQ_HEAD_DIM 128
+/* Cache planes are laid out in pages of this many tokens: capacity is rounded
+ * up to a multiple of it, and decode attention streams whole pages. */
+#define RQ_PAGE_TOKENS 64
+/* Largest batch a decode call accepts (per-sequence page offsets live in
+ * shared memory). */
+#define RQ_MAX_BATCH 1024
+
+typedef enum rq_status {
+  RQ_OK = 0,
+  RQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size or misaligned buffer */
+  RQ_ERR_UNSUPPORTED = 2,  /* a valid but unimplemented configuration */
+  RQ_ERR_CAPACITY = 3,     /* tokens would land beyond the cache capacity */
+  RQ_ERR_WORKSPACE = 4,    /* workspace smaller than *_workspace_size says */
+  RQ_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed */
+  RQ_ERR_DEVICE_FLAG = 6   /* rq_get_error: the device status word is set */
+} rq_status;
+
+/* Bits of the device status word (rq_get_error's *flags_out). */
+#define RQ_FLAG_BAD_INPUT 1u      /* encode saw a non-finite value or |x| > 65504 */
+#define RQ_FLAG_POSITION 2u       /* encode position + n_tokens beyond capacity (tokens dropped) */
+#define RQ_FLAG_CTX_LEN 4u        /* decode ctx_len outside [0, capacity] (clamped) */
+#define RQ_FLAG_PIPE_TIMEOUT 8u   /* a decode pipeline wait exceeded its limit (output invalid) */
+#define RQ_FLAG_META_OVERFLOW 16u /* an alpha, scale or offset overflowed fp16 */
+
+/* Least-squares scale: [RQ] Figure 1 step 3 ("LS"); Figure 3 caption ("alpha = 1"
+ * ablation); Figure 1 step 1 (direct quantisation = alpha 0, no rotation). */
+typedef enum rq_alpha_mode { RQ_ALPHA_LS = 0, RQ_ALPHA_ONE = 1, RQ_ALPHA_ZERO = 2 } rq_alpha_mode;
+
+/* Cache configuration ([RQ] Table 5 caption: loop-wise precision, INT2 with
+ * g = 16 or 32, INT4 with g = 32; Figure 1 step 5: mixed precision such as
+ * [2,2,2,4]).  Per-loop arrays use entries [0, num_loops). */
+typedef struct rq_config {
+  int32_t num_loops;  /* L in [2, 16]; loop L-1 is the reference */
+  int32_t batch;      /* B >= 1 sequences */
+  int32_t kv_heads;   /* Hkv >= 1 */
+  int32_t q_heads;    /* Hq = G * Hkv with G in {1, 2, 4, 8} */
+  int32_t head_dim;   /* must be RQ_HEAD_DIM */
+  int32_t capacity;   /* maximum cached tokens per sequence, >= 1 */
+  int32_t bits[RQ_MAX_LOOPS];  /* residual loops: 2 or 4; reference loop: 16 (bf16) or 4 (INT4) */
+  int32_t group[RQ_MAX_LOOPS]; /* residual loops: 16 or 32; reference loop: 32 (ignored for bf16) */
+  int32_t rotate[RQ_MAX_LOOPS];      /* residual loops: 1 = Hadamard-128 rotation, 0 = none; ref: 0 */
+  int32_t alpha_mode[RQ_MAX_LOOPS];  /* residual loops: rq_alpha_mode; ref: ignored */
+} rq_config;
+
+/* Where each plane lives inside the caller's cache buffer.  Every plane is
+ * indexed [b][h][t] with t < capacity_padded, one fixed-size record per
+ * (b, h, t), and starts on a 1024-byte boundary.  Offsets are bytes from the
+ * start of the buffer; -1 marks a plane the configuration does not have.
+ *
+ *  reference, bf16:  ref[k|v]   128 bf16 per record (256 B)
+ *  reference, INT4:  ref[k|v]   128 4-bit codes (64 B; element d in bits 4*(d%8)
+ *                               of little-endian 32-bit word d/8), ref_meta[k|v]
+ *                               4 groups x (fp16 scale, fp16 offset) = 16 B
+ *  residual loop l:  codes[l][k|v]  128 b-bit codes, rotated domain (INT2: element
+ *                               d in bits 2*(d%16) of word d/16, 32 B; INT4 as above)
+ *                    meta[l][k|v]   (128/g) x (fp16 scale, fp16 offset)
+ *                    alpha[l]       (fp16 alpha_K, fp16 alpha_V) = 4 B
+ *  status:           one 32-bit device status word (256 B reserved)
+ */
+typedef struct rq_layout {
+  int64_t capacity_padded;
+  int64_t total_bytes;
+  int64_t status_offset;
+  int64_t ref_offset[2];
+  int64_t ref_meta_offset[2];
+  int64_t ref_record_bytes;
+  int64_t ref_meta_record_bytes;
+  int64_t codes_offset[RQ_MAX_LOOPS][2];
+  int64_t meta_offset[RQ_MAX_LOOPS][2];
+  int64_t alpha_offset[RQ_MAX_LOOPS];
+  int64_t codes_record_bytes[RQ_MAX_LOOPS];
+  int64_t meta_record_bytes[RQ_MAX_LOOPS];
+} rq_layout;
+
+typedef struct rq_cache rq_cache;
+
+/* Validates cfg and fills *out.  Host only, pure.  RQ_ERR_INVALID_ARG for a
+ * null pointer or an out-of-range field; RQ_ERR_UNSUPPORTED for head_dim != 128
+ * or a bits/group/G combination this build does not implement. */
+RQ_API rq_status rq_cache_layout(const rq_config* cfg, rq_layout* out);
+
+/* Binds a cache handle to the caller's device buffer (>= layout.total_bytes,
+ * 1024-byte aligned) on the current device and zeroes its status word
+ * (a synchronous 256-byte cudaMemset).  The buffer stays caller-owned and must
+ * outlive the handle.  *out receives a heap-allocated host handle. */
+RQ_API rq_status rq_cache_create(const rq_config* cfg, void* device_buffer, int64_t buffer_bytes,
+                          rq_cache** out);
+
+/* Frees the host handle only (never the device buffer).  Null is a no-op. */
+RQ_API void rq_cache_destroy(rq_cache* cache);
+
+/* Copies the handle's configuration and layout out (either pointer may be null). */
+RQ_API rq_status rq_cache_info(const rq_cache* cache, rq_config* cfg_out, rq_layout* layout_out);
+
+/* Encode ([RQ] abstract; Figure 1 steps 2-5): for every loop, sequence b,
+ * kv-head h and the n_tokens tokens at positions [pos_b, pos_b + n_tokens):
+ * store the reference loop (bf16 copy or direct INT4 g=32), then for each
+ * other loop the fp16 LS scale alpha = <x, ref>/<ref, ref> (per 128-vector,
+ * K and V separately; 0 if <ref, ref> = 0), the residual x - alpha*ref, its
+ * Hadamard-128 rotation and asymmetric min-max group quantisation.  The INT4
+ * anchor's dequantised value is the reference the residuals are taken against.
+ *
+ *  k, v        device bf16, element [l][b][h][i][d] at
+ *              l*strides[0] + b*strides[1] + h*strides[2] + i*strides[3] + d
+ *              (strides in elements; d is unit-stride; all strides >= 0)
+ *  positions   device int32 [B] start positions, or NULL to use start_pos for
+ *              every sequence.  With NULL, start_pos + n_tokens > capacity is
+ *              RQ_ERR_CAPACITY; with device positions, tokens past capacity are
+ *              skipped and RQ_FLAG_POSITION is set.
+ *  n_tokens    >= 0 (0 enqueues nothing).
+ * Arithmetic is binary32 with round-to-nearest-even in a fixed order, so codes,
+ * scales and offsets are reproducible bit for bit.  Non-finite inputs or
+ * |x| > 65504 set RQ_FLAG_BAD_INPUT (their records are then unspecified). */
+RQ_API rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const int64_t* strides,
+                    int32_t start_pos, const int32_t* positions, int32_t n_tokens,
+                    rq_stream_t stream);
+
+/* Bytes of workspace rq_decode_attention needs for this cache on the current
+ * device (split-K partials; independent of context length). */
+RQ_API rq_status rq_decode_workspace_size(const rq_cache* cache, int64_t* bytes_out);
+
+/* Fused decode attention of one loop over the compact cache
+ * ([RQ] abstract: "reduced KV memory traffic"; Figure 1).  For a residual loop
+ * each cached token t < ctx_len[b] scores
+ *     s_t = softmax_scale * ( alpha_K,t (q . ref_k,t) + (H q) . deq(codes_K,t) )
+ * and the output is
+ *     ( sum_t p_t alpha_V,t ref_v,t  +  H^T sum_t p_t deq(codes_V,t)
+ *       + sum_tail p_j v_tail,j ) / sum p
+ * with one inverse rotation per (b, q-head).  The reference loop is plain
+ * attention over its bf16 or INT4 reference.  n_tail current tokens (bf16,
+ * not yet encoded) join the softmax.  Split-K over 64-token pages with an
+ * online softmax, merged by a second kernel.
+ *
+ *  q          device bf16 [B][Hq][128]
+ *  ctx_len    device int32 [B], each in [0, capacity] (clamped, RQ_FLAG_CTX_LEN)
+ *  k_tail/v_tail  device bf16 [B][Hkv][n_tail][128] (NULL allowed when n_tail == 0)
+ *  softmax_scale  e.g. 1/sqrt(128)
+ *  out        device fp32 [B][Hq][128]; kv-head of q-head j is j / G
+ *  workspace  device, >= rq_decode_workspace_size bytes, 256-byte aligned */
+RQ_API rq_status rq_decode_attention(const rq_cache* cache, int32_t loop, const void* q,
+                              const int32_t* ctx_len, const void* k_tail, const void* v_tail,
+                              int32_t n_tail, float softmax_scale, float* out, void* workspace,
+                              int64_t workspace_bytes, rq_stream_t stream);
+
+/* Workspace bytes for rq_bf16_decode_attention with these sizes. */
+RQ_API rq_status rq_bf16_decode_workspace_size(int32_t batch, int32_t kv_heads, int32_t q_heads,
+                                        int64_t* bytes_out);
+
+/* Decode attention over a plain bf16 KV cache (the BF16-cache baseline the
+ * [RQ] abstract compares against; same kernels with no residual):
+ *  k_cache/v_cache  device bf16, element [b][h][t][d] at b*strides[0] +
+ *                   h*strides[1] + t*strides[2] + d (strides in elements,
+ *                   multiples of 8, base 16-byte aligned), t < capacity
+ *  other arguments as rq_decode_attention; status flags go to *status_word if
+ *  it is non-null (device int32), else are dropped. */
+RQ_API rq_status rq_bf16_decode_attention(int32_t batch, int32_t kv_heads, int32_t q_heads,
+                                   const void* k_cache, const void* v_cache,
+                                   const int64_t* strides, int32_t capacity, const void* q,
+                                   const int32_t* ctx_len, const void* k_tail, const void* v_tail,
+                                   int32_t n_tail, float softmax_scale, float* out,
+                                   void* workspace, int64_t workspace_bytes, int32_t* status_word,
+                                   rq_stream_t stream);
+
+/* Reconstruction (test support): fp32 K_hat, V_hat of loop `loop` for tokens
+ * [t0, t0 + n) of every (b, h), written to k_out/v_out [B][Hkv][n][128]:
+ * alpha * ref + H^T deq(codes) for a residual loop, the (dequantised)
+ * reference for the reference loop. */
+RQ_API rq_status rq_reconstruct(const rq_cache* cache, int32_t loop, int32_t t0, int32_t n, float* k_out,
+                         float* v_out, rq_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the device status word.  Returns
+ * RQ_OK if it was zero, else RQ_ERR_DEVICE_FLAG with the bits in *flags_out
+ * (may be null). */
+RQ_API rq_status rq_get_error(const rq_cache* cache, rq_stream_t stream, uint32_t* flags_out);
+
+/* Static string naming a status code. */
+RQ_API const char* rq_status_string(rq_status status);
+
+/* Detail of the calling thread's most recent non-OK status ("" if none). */
+RQ_API const char* rq_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RQ_API_H */

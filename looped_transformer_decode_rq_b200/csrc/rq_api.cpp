@@ -1,0 +1,491 @@
+// rq_api.cpp -- host side of the C ABI declared in include/rq_api.h: argument
+// validation, cache layout, tensor-map construction and kernel dispatch.  All
+// device memory belongs to the caller; nothing here allocates on the device.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+
+#include "../../include/rq_api.h"
+#include "rq_internal.h"
+
+struct rq_cache {
+  rq_config cfg;
+  rq_layout lay;
+  uint8_t* base;
+  int device;
+  int num_ctas;
+  bool tmaps_ready;
+  CUtensorMap tm_ref[2];
+};
+
+namespace {
+
+thread_local std::string g_msg;
+
+rq_status fail(rq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_msg = buf;
+  return s;
+}
+
+rq_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(RQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 plane [B][H][T][128] with element strides (sb, sh, st); tiles of
+// 64 tokens x 64 dims with the 128-byte swizzle.
+rq_status make_plane_map(CUtensorMap* map, const void* base, int B, int H, int64_t T, int64_t sb,
+                         int64_t sh, int64_t st) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return fail(RQ_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(RQ_HEAD_DIM), static_cast<cuuint64_t>(T),
+                        static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(st * 2), static_cast<cuuint64_t>(sh * 2),
+                           static_cast<cuuint64_t>(sb * 2)};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(RQ_PAGE_TOKENS), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(RQ_ERR_INVALID_ARG, "tensor map rejected (CUresult %d)", static_cast<int>(r));
+  return RQ_OK;
+}
+
+rq_status validate_config(const rq_config* c) {
+  if (c == nullptr) return fail(RQ_ERR_INVALID_ARG, "config is null");
+  if (c->num_loops < 2 || c->num_loops > RQ_MAX_LOOPS)
+    return fail(RQ_ERR_INVALID_ARG, "num_loops %d outside [2, %d]", c->num_loops, RQ_MAX_LOOPS);
+  if (c->batch < 1) return fail(RQ_ERR_INVALID_ARG, "batch %d < 1", c->batch);
+  if (c->kv_heads < 1) return fail(RQ_ERR_INVALID_ARG, "kv_heads %d < 1", c->kv_heads);
+  if (c->q_heads < 1 || c->q_heads % c->kv_heads != 0)
+    return fail(RQ_ERR_INVALID_ARG, "q_heads %d not a multiple of kv_heads %d", c->q_heads, c->kv_heads);
+  const int G = c->q_heads / c->kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(RQ_ERR_UNSUPPORTED, "q_heads / kv_heads = %d (supported: 1, 2, 4, 8)", G);
+  if (c->head_dim != RQ_HEAD_DIM) return fail(RQ_ERR_UNSUPPORTED, "head_dim %d != 128", c->head_dim);
+  if (c->capacity < 1) return fail(RQ_ERR_INVALID_ARG, "capacity %d < 1", c->capacity);
+  const int ref = c->num_loops - 1;
+  if (c->bits[ref] != 16 && c->bits[ref] != 4)
+    return fail(RQ_ERR_UNSUPPORTED, "reference loop bits %d (supported: 16, 4)", c->bits[ref]);
+  if (c->bits[ref] == 4 && c->group[ref] != 32)
+    return fail(RQ_ERR_UNSUPPORTED, "INT4 reference group %d (supported: 32)", c->group[ref]);
+  for (int l = 0; l < ref; ++l) {
+    if (c->bits[l] != 2 && c->bits[l] != 4)
+      return fail(RQ_ERR_UNSUPPORTED, "loop %d bits %d (supported: 2, 4)", l, c->bits[l]);
+    if (c->group[l] != 16 && c->group[l] != 32)
+      return fail(RQ_ERR_UNSUPPORTED, "loop %d group %d (supported: 16, 32)", l, c->group[l]);
+    if (c->rotate[l] != 0 && c->rotate[l] != 1)
+      return fail(RQ_ERR_INVALID_ARG, "loop %d rotate %d", l, c->rotate[l]);
+    if (c->alpha_mode[l] < RQ_ALPHA_LS || c->alpha_mode[l] > RQ_ALPHA_ZERO)
+      return fail(RQ_ERR_INVALID_ARG, "loop %d alpha_mode %d", l, c->alpha_mode[l]);
+  }
+  return RQ_OK;
+}
+
+int ref_kind_for(const rq_config& c, int loop) {
+  const int ref = c.num_loops - 1;
+  if (loop != ref && c.alpha_mode[loop] == RQ_ALPHA_ZERO) return rq::kRefNone;
+  return c.bits[ref] == 16 ? rq::kRefBf16 : rq::kRefInt4;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rq_status_string(rq_status s) {
+  switch (s) {
+    case RQ_OK: return "RQ_OK";
+    case RQ_ERR_INVALID_ARG: return "RQ_ERR_INVALID_ARG";
+    case RQ_ERR_UNSUPPORTED: return "RQ_ERR_UNSUPPORTED";
+    case RQ_ERR_CAPACITY: return "RQ_ERR_CAPACITY";
+    case RQ_ERR_WORKSPACE: return "RQ_ERR_WORKSPACE";
+    case RQ_ERR_CUDA: return "RQ_ERR_CUDA";
+    case RQ_ERR_DEVICE_FLAG: return "RQ_ERR_DEVICE_FLAG";
+  }
+  return "RQ_UNKNOWN_STATUS";
+}
+
+const char* rq_last_error_message(void) { return g_msg.c_str(); }
+
+rq_status rq_cache_layout(const rq_config* cfg, rq_layout* out) {
+  if (out == nullptr) return fail(RQ_ERR_INVALID_ARG, "layout output is null");
+  rq_status st = validate_config(cfg);
+  if (st != RQ_OK) return st;
+  rq_layout L;
+  std::memset(&L, 0, sizeof(L));
+  const int ref = cfg->num_loops - 1;
+  const int64_t cap_pad = align_up(cfg->capacity, RQ_PAGE_TOKENS);
+  const int64_t recs = static_cast<int64_t>(cfg->batch) * cfg->kv_heads * cap_pad;
+  int64_t off = 0;
+  auto place = [&](int64_t bytes) {
+    const int64_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  L.capacity_padded = cap_pad;
+  L.status_offset = place(256);
+  L.ref_record_bytes = cfg->bits[ref] == 16 ? 256 : 64;
+  L.ref_meta_record_bytes = cfg->bits[ref] == 16 ? 0 : 16;
+  for (int kv = 0; kv < 2; ++kv) L.ref_offset[kv] = place(recs * L.ref_record_bytes);
+  for (int kv = 0; kv < 2; ++kv)
+    L.ref_meta_offset[kv] = L.ref_meta_record_bytes ? place(recs * L.ref_meta_record_bytes) : -1;
+  for (int l = 0; l < RQ_MAX_LOOPS; ++l) {
+    L.codes_offset[l][0] = L.codes_offset[l][1] = -1;
+    L.meta_offset[l][0] = L.meta_offset[l][1] = -1;
+    L.alpha_offset[l] = -1;
+  }
+  for (int l = 0; l < ref; ++l) {
+    L.codes_record_bytes[l] = cfg->bits[l] * RQ_HEAD_DIM / 8;
+    L.meta_record_bytes[l] = 4 * (RQ_HEAD_DIM / cfg->group[l]);
+    for (int kv = 0; kv < 2; ++kv) L.codes_offset[l][kv] = place(recs * L.codes_record_bytes[l]);
+    for (int kv = 0; kv < 2; ++kv) L.meta_offset[l][kv] = place(recs * L.meta_record_bytes[l]);
+    L.alpha_offset[l] = place(recs * 4);
+  }
+  L.total_bytes = off;
+  *out = L;
+  return RQ_OK;
+}
+
+rq_status rq_cache_create(const rq_config* cfg, void* device_buffer, int64_t buffer_bytes,
+                          rq_cache** out) {
+  if (out == nullptr) return fail(RQ_ERR_INVALID_ARG, "handle output is null");
+  *out = nullptr;
+  rq_layout L;
+  rq_status st = rq_cache_layout(cfg, &L);
+  if (st != RQ_OK) return st;
+  if (device_buffer == nullptr) return fail(RQ_ERR_INVALID_ARG, "device buffer is null");
+  if (!aligned(device_buffer, 1024)) return fail(RQ_ERR_INVALID_ARG, "device buffer not 1024-byte aligned");
+  if (buffer_bytes < L.total_bytes)
+    return fail(RQ_ERR_INVALID_ARG, "buffer has %lld bytes, layout needs %lld",
+                static_cast<long long>(buffer_bytes), static_cast<long long>(L.total_bytes));
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  e = cudaMemset(static_cast<uint8_t*>(device_buffer) + L.status_offset, 0, 256);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  rq_cache* c = new (std::nothrow) rq_cache;
+  if (c == nullptr) return fail(RQ_ERR_INVALID_ARG, "out of host memory");
+  c->cfg = *cfg;
+  c->lay = L;
+  c->base = static_cast<uint8_t*>(device_buffer);
+  c->device = dev;
+  c->num_ctas = rq::decode_grid_ctas(dev);
+  c->tmaps_ready = false;
+  *out = c;
+  return RQ_OK;
+}
+
+void rq_cache_destroy(rq_cache* cache) { delete cache; }
+
+rq_status rq_cache_info(const rq_cache* cache, rq_config* cfg_out, rq_layout* layout_out) {
+  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  if (cfg_out) *cfg_out = cache->cfg;
+  if (layout_out) *layout_out = cache->lay;
+  return RQ_OK;
+}
+
+rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const int64_t* strides,
+                    int32_t start_pos, const int32_t* positions, int32_t n_tokens,
+                    rq_stream_t stream) {
+  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  if (n_tokens < 0) return fail(RQ_ERR_INVALID_ARG, "n_tokens %d < 0", n_tokens);
+  if (n_tokens == 0) return RQ_OK;
+  if (k == nullptr || v == nullptr || strides == nullptr) return fail(RQ_ERR_INVALID_ARG, "k, v or strides is null");
+  if (!aligned(k, 16) || !aligned(v, 16)) return fail(RQ_ERR_INVALID_ARG, "k/v not 16-byte aligned");
+  for (int i = 0; i < 4; ++i)
+    if (strides[i] < 0 || strides[i] % 8 != 0)
+      return fail(RQ_ERR_INVALID_ARG, "stride[%d] = %lld must be a non-negative multiple of 8", i,
+                  static_cast<long long>(strides[i]));
+  const rq_config& c = cache->cfg;
+  if (positions == nullptr) {
+    if (start_pos < 0) return fail(RQ_ERR_INVALID_ARG, "start_pos %d < 0", start_pos);
+    if (static_cast<int64_t>(start_pos) + n_tokens > c.capacity)
+      return fail(RQ_ERR_CAPACITY, "start_pos %d + n_tokens %d > capacity %d", start_pos, n_tokens, c.capacity);
+  }
+  if (static_cast<int64_t>(c.batch) * c.kv_heads * n_tokens > (int64_t(1) << 31) - 8)
+    return fail(RQ_ERR_UNSUPPORTED, "too many vectors in one encode call");
+  rq::EncodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.L = c.num_loops;
+  p.B = c.batch;
+  p.Hkv = c.kv_heads;
+  p.cap_pad = cache->lay.capacity_padded;
+  p.capacity = c.capacity;
+  p.n_tokens = n_tokens;
+  p.start_pos = start_pos;
+  p.positions = positions;
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.s_l = strides[0];
+  p.s_b = strides[1];
+  p.s_h = strides[2];
+  p.s_t = strides[3];
+  const int ref = c.num_loops - 1;
+  p.ref_bits = c.bits[ref];
+  for (int kv = 0; kv < 2; ++kv) {
+    p.ref_plane[kv] = cache->base + cache->lay.ref_offset[kv];
+    p.ref_meta[kv] = cache->lay.ref_meta_offset[kv] >= 0 ? cache->base + cache->lay.ref_meta_offset[kv] : nullptr;
+  }
+  for (int l = 0; l < ref; ++l) {
+    for (int kv = 0; kv < 2; ++kv) {
+      p.codes[l][kv] = cache->base + cache->lay.codes_offset[l][kv];
+      p.meta[l][kv] = cache->base + cache->lay.meta_offset[l][kv];
+    }
+    p.alpha[l] = cache->base + cache->lay.alpha_offset[l];
+    p.bits[l] = c.bits[l];
+    p.group[l] = c.group[l];
+    p.rotate[l] = c.rotate[l];
+    p.alpha_mode[l] = c.alpha_mode[l];
+  }
+  p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
+  cudaError_t e = rq::launch_encode(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "encode launch");
+  return RQ_OK;
+}
+
+rq_status rq_decode_workspace_size(const rq_cache* cache, int64_t* bytes_out) {
+  if (cache == nullptr || bytes_out == nullptr) return fail(RQ_ERR_INVALID_ARG, "null argument");
+  const int G = cache->cfg.q_heads / cache->cfg.kv_heads;
+  *bytes_out = rq::decode_workspace_bytes(cache->cfg.batch, cache->cfg.kv_heads, G, cache->num_ctas);
+  return RQ_OK;
+}
+
+rq_status rq_bf16_decode_workspace_size(int32_t batch, int32_t kv_heads, int32_t q_heads,
+                                        int64_t* bytes_out) {
+  if (bytes_out == nullptr) return fail(RQ_ERR_INVALID_ARG, "null argument");
+  if (batch < 1 || kv_heads < 1 || q_heads < 1 || q_heads % kv_heads)
+    return fail(RQ_ERR_INVALID_ARG, "bad sizes");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  *bytes_out = rq::decode_workspace_bytes(batch, kv_heads, q_heads / kv_heads, rq::decode_grid_ctas(dev));
+  return RQ_OK;
+}
+
+namespace {
+
+rq_status check_decode_common(int B, int Hkv, int Hq, const void* q, const int32_t* ctx_len,
+                              const void* k_tail, const void* v_tail, int32_t n_tail, float scale,
+                              const float* out, const void* ws, int64_t ws_bytes, int64_t need) {
+  if (B > RQ_MAX_BATCH) return fail(RQ_ERR_UNSUPPORTED, "batch %d > %d", B, RQ_MAX_BATCH);
+  if (q == nullptr || ctx_len == nullptr || out == nullptr) return fail(RQ_ERR_INVALID_ARG, "q, ctx_len or out is null");
+  if (!aligned(q, 16) || !aligned(out, 16)) return fail(RQ_ERR_INVALID_ARG, "q/out not 16-byte aligned");
+  if (n_tail < 0) return fail(RQ_ERR_INVALID_ARG, "n_tail %d < 0", n_tail);
+  if (n_tail > 0 && (k_tail == nullptr || v_tail == nullptr)) return fail(RQ_ERR_INVALID_ARG, "tail is null");
+  if (n_tail > 0 && (!aligned(k_tail, 8) || !aligned(v_tail, 8))) return fail(RQ_ERR_INVALID_ARG, "tail misaligned");
+  if (!(scale > 0.f) || !(scale < 1e30f)) return fail(RQ_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+  if (ws == nullptr || !aligned(ws, 256)) return fail(RQ_ERR_WORKSPACE, "workspace null or not 256-byte aligned");
+  if (ws_bytes < need)
+    return fail(RQ_ERR_WORKSPACE, "workspace %lld bytes < %lld needed", static_cast<long long>(ws_bytes),
+                static_cast<long long>(need));
+  (void)Hkv; (void)Hq;
+  return RQ_OK;
+}
+
+}  // namespace
+
+rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void* q,
+                              const int32_t* ctx_len, const void* k_tail, const void* v_tail,
+                              int32_t n_tail, float softmax_scale, float* out, void* workspace,
+                              int64_t workspace_bytes, rq_stream_t stream) {
+  if (cache_c == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  rq_cache* cache = const_cast<rq_cache*>(cache_c);
+  const rq_config& c = cache->cfg;
+  if (loop < 0 || loop >= c.num_loops) return fail(RQ_ERR_INVALID_ARG, "loop %d outside [0, %d)", loop, c.num_loops);
+  const int G = c.q_heads / c.kv_heads;
+  int64_t need = 0;
+  rq_decode_workspace_size(cache, &need);
+  rq_status st = check_decode_common(c.batch, c.kv_heads, c.q_heads, q, ctx_len, k_tail, v_tail, n_tail,
+                                     softmax_scale, out, workspace, workspace_bytes, need);
+  if (st != RQ_OK) return st;
+  const int ref = c.num_loops - 1;
+  const int ref_kind = ref_kind_for(c, loop);
+  const int res_bits = loop == ref ? 0 : c.bits[loop];
+  const int res_group = loop == ref ? 32 : c.group[loop];
+  if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G))
+    return fail(RQ_ERR_UNSUPPORTED, "no decode kernel for this loop format");
+  if (ref_kind == rq::kRefBf16 && !cache->tmaps_ready) {
+    const int64_t cp = cache->lay.capacity_padded;
+    for (int kv = 0; kv < 2; ++kv) {
+      st = make_plane_map(&cache->tm_ref[kv], cache->base + cache->lay.ref_offset[kv], c.batch, c.kv_heads, cp,
+                          static_cast<int64_t>(c.kv_heads) * cp * RQ_HEAD_DIM, cp * RQ_HEAD_DIM, RQ_HEAD_DIM);
+      if (st != RQ_OK) return st;
+    }
+    cache->tmaps_ready = true;
+  }
+  rq::DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = c.batch;
+  p.Hkv = c.kv_heads;
+  p.G = G;
+  p.capacity = c.capacity;
+  p.plane_tokens = cache->lay.capacity_padded;
+  if (ref_kind == rq::kRefInt4) {
+    for (int kv = 0; kv < 2; ++kv) {
+      p.ref_codes[kv] = cache->base + cache->lay.ref_offset[kv];
+      p.ref_meta[kv] = cache->base + cache->lay.ref_meta_offset[kv];
+    }
+  }
+  if (res_bits) {
+    for (int kv = 0; kv < 2; ++kv) {
+      p.res_codes[kv] = cache->base + cache->lay.codes_offset[loop][kv];
+      p.res_meta[kv] = cache->base + cache->lay.meta_offset[loop][kv];
+    }
+    p.alpha = cache->base + cache->lay.alpha_offset[loop];
+    p.rotate = c.rotate[loop];
+  }
+  p.q = static_cast<const uint16_t*>(q);
+  p.ctx_len = ctx_len;
+  p.k_tail = static_cast<const uint16_t*>(k_tail);
+  p.v_tail = static_cast<const uint16_t*>(v_tail);
+  p.n_tail = n_tail;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  p.partials = static_cast<float*>(workspace);
+  p.num_ctas = cache->num_ctas;
+  p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
+  cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, &cache->tm_ref[0], &cache->tm_ref[1],
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return RQ_OK;
+}
+
+rq_status rq_bf16_decode_attention(int32_t batch, int32_t kv_heads, int32_t q_heads,
+                                   const void* k_cache, const void* v_cache,
+                                   const int64_t* strides, int32_t capacity, const void* q,
+                                   const int32_t* ctx_len, const void* k_tail, const void* v_tail,
+                                   int32_t n_tail, float softmax_scale, float* out,
+                                   void* workspace, int64_t workspace_bytes, int32_t* status_word,
+                                   rq_stream_t stream) {
+  if (batch < 1 || kv_heads < 1 || q_heads < 1 || q_heads % kv_heads)
+    return fail(RQ_ERR_INVALID_ARG, "bad sizes");
+  const int G = q_heads / kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(RQ_ERR_UNSUPPORTED, "q_heads / kv_heads = %d", G);
+  if (k_cache == nullptr || v_cache == nullptr || strides == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(RQ_ERR_INVALID_ARG, "cache not 16-byte aligned");
+  for (int i = 0; i < 3; ++i)
+    if (strides[i] <= 0 || strides[i] % 8 != 0)
+      return fail(RQ_ERR_INVALID_ARG, "stride[%d] must be a positive multiple of 8", i);
+  if (capacity < 1) return fail(RQ_ERR_INVALID_ARG, "capacity %d < 1", capacity);
+  int64_t need = 0;
+  rq_status st = rq_bf16_decode_workspace_size(batch, kv_heads, q_heads, &need);
+  if (st != RQ_OK) return st;
+  st = check_decode_common(batch, kv_heads, q_heads, q, ctx_len, k_tail, v_tail, n_tail, softmax_scale, out,
+                           workspace, workspace_bytes, need);
+  if (st != RQ_OK) return st;
+  CUtensorMap tk, tv;
+  st = make_plane_map(&tk, k_cache, batch, kv_heads, capacity, strides[0], strides[1], strides[2]);
+  if (st != RQ_OK) return st;
+  st = make_plane_map(&tv, v_cache, batch, kv_heads, capacity, strides[0], strides[1], strides[2]);
+  if (st != RQ_OK) return st;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  rq::DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = batch;
+  p.Hkv = kv_heads;
+  p.G = G;
+  p.capacity = capacity;
+  p.plane_tokens = 0;
+  p.q = static_cast<const uint16_t*>(q);
+  p.ctx_len = ctx_len;
+  p.k_tail = static_cast<const uint16_t*>(k_tail);
+  p.v_tail = static_cast<const uint16_t*>(v_tail);
+  p.n_tail = n_tail;
+  p.scale_log2 = softmax_scale * 1.4426950408889634f;
+  p.out = out;
+  p.partials = static_cast<float*>(workspace);
+  p.num_ctas = rq::decode_grid_ctas(dev);
+  p.status = status_word;
+  cudaError_t e = rq::launch_decode(p, rq::kRefBf16, 0, 32, &tk, &tv, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return RQ_OK;
+}
+
+rq_status rq_reconstruct(const rq_cache* cache, int32_t loop, int32_t t0, int32_t n, float* k_out,
+                         float* v_out, rq_stream_t stream) {
+  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  const rq_config& c = cache->cfg;
+  if (loop < 0 || loop >= c.num_loops) return fail(RQ_ERR_INVALID_ARG, "loop %d outside [0, %d)", loop, c.num_loops);
+  if (t0 < 0 || n < 0 || static_cast<int64_t>(t0) + n > c.capacity)
+    return fail(RQ_ERR_INVALID_ARG, "token range [%d, %d) outside the capacity %d", t0, t0 + n, c.capacity);
+  if (n == 0) return RQ_OK;
+  if (k_out == nullptr || v_out == nullptr || !aligned(k_out, 16) || !aligned(v_out, 16))
+    return fail(RQ_ERR_INVALID_ARG, "outputs null or not 16-byte aligned");
+  const int ref = c.num_loops - 1;
+  rq::ReconstructParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = c.batch;
+  p.Hkv = c.kv_heads;
+  p.cap_pad = cache->lay.capacity_padded;
+  p.t0 = t0;
+  p.n = n;
+  p.ref_bits = c.bits[ref];
+  for (int kv = 0; kv < 2; ++kv) {
+    p.ref_plane[kv] = cache->base + cache->lay.ref_offset[kv];
+    p.ref_meta[kv] = cache->lay.ref_meta_offset[kv] >= 0 ? cache->base + cache->lay.ref_meta_offset[kv] : nullptr;
+  }
+  p.is_ref = loop == ref;
+  if (!p.is_ref) {
+    for (int kv = 0; kv < 2; ++kv) {
+      p.codes[kv] = cache->base + cache->lay.codes_offset[loop][kv];
+      p.meta[kv] = cache->base + cache->lay.meta_offset[loop][kv];
+    }
+    p.alpha = cache->base + cache->lay.alpha_offset[loop];
+    p.bits = c.bits[loop];
+    p.group = c.group[loop];
+    p.rotate = c.rotate[loop];
+  }
+  p.out[0] = k_out;
+  p.out[1] = v_out;
+  cudaError_t e = rq::launch_reconstruct(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "reconstruct launch");
+  return RQ_OK;
+}
+
+rq_status rq_get_error(const rq_cache* cache, rq_stream_t stream, uint32_t* flags_out) {
+  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t w = 0;
+  void* dev = cache->base + cache->lay.status_offset;
+  e = cudaMemcpy(&w, dev, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  if (w != 0) {
+    e = cudaMemset(dev, 0, sizeof(w));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  }
+  if (flags_out) *flags_out = w;
+  if (w != 0) return fail(RQ_ERR_DEVICE_FLAG, "device status word 0x%x", w);
+  return RQ_OK;
+}
+
+}  // extern "C"

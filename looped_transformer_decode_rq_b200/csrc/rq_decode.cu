@@ -1,0 +1,854 @@
+// rq_decode.cu -- fused dequantise-and-reconstruct split-K decode attention
+// for sm_100a.
+//
+// "ResidualQuant: KV Cache Quantization for Looped Transformers with 2-Bit
+// Residuals" stores loop l's keys as K_l ~ alpha K_ref + H^T deq(R_l) (abstract,
+// Figure 1, Figure 2 caption) and credits its decode speed-up to the reduced
+// KV memory traffic (abstract).  Here each cached token is scored directly from
+// the compact cache:
+//     q . K_l,t = alpha_t (q . K_ref,t) + (H q) . deq(R_l,t)
+// and the value side accumulates sum p_t alpha_V,t V_ref,t in the original
+// domain and sum p_t deq(R^V_l,t) in the rotated domain; the rotated sum is
+// brought back with a single inverse Hadamard per (sequence, q-head) in the
+// combine kernel.  No bf16 copy of loop l is ever formed.
+//
+// Split kernel (persistent, one CTA per SM):
+//   * the flattened sequence of 64-token pages over all (b, kv-head) pairs is
+//     cut into num_ctas contiguous ranges of equal length, so ragged batches
+//     balance to within one page; a CTA emits one partial (m, l, acc) per
+//     (b, kv-head) segment it touches;
+//   * warp 8 is a producer: one lane streams pages into a ring of shared
+//     memory stages with the Tensor Memory Accelerator -- tiled tensor copies
+//     with the 128-byte swizzle for bf16 reference tiles, bulk copies for
+//     code, metadata and alpha records -- completing on mbarriers;
+//   * warps 0-7 consume each page in three phases: scores (4G threads per
+//     token, warp-shuffle reduction), softmax weights (one thread per
+//     (token, head)), value accumulation (16 threads per token row);
+//   * packed codes become floats with one LOP3 each (1 + c*2^(p-23)), the
+//     2^(p-23) factor being folded into the query once per segment and into
+//     the accumulators once per flush; fp32 pairs use FFMA2.
+// Combine kernel: one warp per (b, q-head) merges the CTA partials with the
+// max-rescale rule, adds the bf16 tail tokens, applies the inverse rotation and
+// normalises.
+#include "rq_common.cuh"
+#include "rq_internal.h"
+
+namespace rq {
+namespace {
+
+constexpr int kTT = kPage;   // tokens per page / tile
+constexpr int kNCW = 8;      // consumer warps
+constexpr int kNCT = kNCW * 32;
+constexpr int kNT = kNCT + 32;
+constexpr int kConsumerBar = 1;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+template <int REF, int RB, int RG, int G>
+struct Cfg {
+  static constexpr int TPT = 4 * G;       // phase-1 threads per token
+  static constexpr int D1 = 32 / G;       // phase-1 dims per thread
+  static constexpr int TOK_PASS = kNCT / TPT;
+  static constexpr int PASSES = kTT / TOK_PASS;
+  static constexpr int D2 = (G >= 8) ? 4 : 8;  // phase-2 dims per thread
+  static constexpr int TPR2 = kD / D2;          // phase-2 threads per token row
+  static constexpr int SLICES = kNCT / TPR2;
+  static constexpr int TOK2 = kTT / SLICES;     // tokens per phase-2 thread per tile
+  // per-record bytes
+  static constexpr int REF_REC = REF == kRefBf16 ? 256 : (REF == kRefInt4 ? 64 : 0);
+  static constexpr int REFM_REC = REF == kRefInt4 ? 16 : 0;
+  static constexpr int CB = RB * 16;
+  static constexpr int MB = RB ? 4 * (kD / RG) : 0;
+  static constexpr bool HAS_ALPHA = (REF != kRefNone) && (RB != 0);
+  static constexpr int AL_REC = HAS_ALPHA ? 4 : 0;
+  // stage layout (each piece 1024-byte aligned)
+  static constexpr int al(int x) { return (x + 1023) & ~1023; }
+  static constexpr int O_REFK = 0;
+  static constexpr int O_REFV = O_REFK + al(kTT * REF_REC);
+  static constexpr int O_REFMK = O_REFV + al(kTT * REF_REC);
+  static constexpr int O_REFMV = O_REFMK + al(kTT * REFM_REC);
+  static constexpr int O_RESK = O_REFMV + al(kTT * REFM_REC);
+  static constexpr int O_RESV = O_RESK + al(kTT * CB);
+  static constexpr int O_RESMK = O_RESV + al(kTT * CB);
+  static constexpr int O_RESMV = O_RESMK + al(kTT * MB);
+  static constexpr int O_AL = O_RESMV + al(kTT * MB);
+  static constexpr int STAGE_BYTES = O_AL + al(kTT * AL_REC);
+  static constexpr int TX_BYTES = kTT * (2 * REF_REC + 2 * REFM_REC + 2 * CB + 2 * MB + AL_REC);
+  // non-stage shared memory
+  static constexpr int O_S = 0;                      // scores   [G][kTT]
+  static constexpr int O_P = O_S + 4 * G * kTT;      // weights  [G][kTT]  (p)
+  static constexpr int O_PA = O_P + 4 * G * kTT;     // weights  [G][kTT]  (p * alpha_V)
+  static constexpr int O_WM = O_PA + 4 * G * kTT;    // warp max [G][kNCW]
+  static constexpr int O_ACC = O_WM + 4 * G * kNCW;  // [G][256]
+  static constexpr int O_L = O_ACC + 4 * G * 2 * kD; // [G]
+  static constexpr int O_QS = O_L + 4 * 8;           // [G][128]
+  static constexpr int O_QT = O_QS + 4 * G * kD;     // [G][128]
+  static constexpr int O_PRE = O_QT + 4 * G * kD;    // [RQ_MAX_BATCH + 1]
+  static constexpr int O_NT = O_PRE + 4 * (RQ_MAX_BATCH + 1);
+  static constexpr int O_MISC = O_NT + 4 * RQ_MAX_BATCH;  // abort flag
+  static constexpr int O_BAR = (O_MISC + 16 + 7) & ~7;
+  static constexpr int MISC_BYTES = O_BAR + 16 * 8;
+  static constexpr int kSmemLimit = 227 * 1024;
+  static constexpr int STAGES_MAX = (kSmemLimit - 1024 - MISC_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_MAX >= 4 ? 4 : STAGES_MAX;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
+  static_assert(STAGES >= 2, "stage ring does not fit in shared memory");
+  static_assert(PASSES * TOK_PASS == kTT, "phase-1 mapping");
+  static_assert(TOK2 * SLICES == kTT, "phase-2 mapping");
+};
+
+// ---------------------------------------------------------------------------
+// page walk over the flattened (b, h, page) sequence
+// ---------------------------------------------------------------------------
+struct PageIter {
+  int b, h, page;
+  __device__ __forceinline__ void seek(int64_t x, const int* pre, const int* nt, int B, int Hkv) {
+    int lo = 0, hi = B - 1;  // largest b with pre[b]*Hkv <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (static_cast<int64_t>(pre[mid]) * Hkv <= x) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    const int64_t r = x - static_cast<int64_t>(pre[b]) * Hkv;
+    h = static_cast<int>(r / nt[b]);
+    page = static_cast<int>(r % nt[b]);
+  }
+  __device__ __forceinline__ void next(const int* nt, int B, int Hkv) {
+    if (++page < nt[b]) return;
+    page = 0;
+    if (++h < Hkv) return;
+    h = 0;
+    do { ++b; } while (b < B && nt[b] == 0);
+  }
+};
+
+// ---------------------------------------------------------------------------
+// code unpacking helpers
+// ---------------------------------------------------------------------------
+// Load `NB` bytes (1, 2, 4, 8 or 16) of packed codes into 32-bit words.
+template <int NB>
+__device__ __forceinline__ void load_codes(const uint8_t* p, uint32_t (&w)[(NB + 3) / 4]) {
+  if constexpr (NB == 16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p);
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  } else if constexpr (NB == 8) {
+    const uint2 v = *reinterpret_cast<const uint2*>(p);
+    w[0] = v.x; w[1] = v.y;
+  } else if constexpr (NB == 4) {
+    w[0] = *reinterpret_cast<const uint32_t*>(p);
+  } else if constexpr (NB == 2) {
+    w[0] = *reinterpret_cast<const uint16_t*>(p);
+  } else {
+    w[0] = *p;
+  }
+}
+
+// code e of a thread's unit (bits per code BITS) as 1 + c*2^(p_e - 23)
+template <int BITS>
+__device__ __forceinline__ float code_f(const uint32_t* w, int e) {
+  const int bit = e * BITS;
+  const uint32_t word = w[bit >> 5];
+  const int b32 = bit & 31;
+  const uint32_t src = (b32 >= 16) ? (word >> 16) : word;
+  const int p = b32 & 15;
+  return code_float(src, ((1u << BITS) - 1u) << p);
+}
+
+template <int BITS>
+__device__ __forceinline__ int code_pos(int e) { return (e * BITS) & 15; }
+
+__device__ __forceinline__ float2 f2sub1(float2 f) { return __fadd2_rn(f, make_float2(-1.f, -1.f)); }
+
+// ---------------------------------------------------------------------------
+// split kernel
+// ---------------------------------------------------------------------------
+template <int REF, int RB, int RG, int G>
+__global__ void __launch_bounds__(kNT, 1)
+    decode_split_kernel(const __grid_constant__ DecodeParams P,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV) {
+  using C = Cfg<REF, RB, RG, G>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = base;
+  uint8_t* misc = base + C::STAGES * C::STAGE_BYTES;
+  float* sS = reinterpret_cast<float*>(misc + C::O_S);
+  float* sP = reinterpret_cast<float*>(misc + C::O_P);
+  float* sPA = reinterpret_cast<float*>(misc + C::O_PA);
+  float* sWM = reinterpret_cast<float*>(misc + C::O_WM);
+  float* sACC = reinterpret_cast<float*>(misc + C::O_ACC);
+  float* sL = reinterpret_cast<float*>(misc + C::O_L);
+  float* sQS = reinterpret_cast<float*>(misc + C::O_QS);
+  float* sQT = reinterpret_cast<float*>(misc + C::O_QT);
+  int* sPre = reinterpret_cast<int*>(misc + C::O_PRE);
+  int* sNt = reinterpret_cast<int*>(misc + C::O_NT);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(misc + C::O_MISC);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + C::O_BAR);
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int B = P.B, Hkv = P.Hkv;
+
+  // ---- page counts and prefix over sequences
+  for (int b = tid; b < B; b += kNT) {
+    int len = P.ctx_len[b];
+    if (len < 0 || len > P.capacity) {
+      if (blockIdx.x == 0) set_flag(P.status, RQ_FLAG_CTX_LEN);
+      len = len < 0 ? 0 : P.capacity;
+    }
+    sNt[b] = (len + kTT - 1) / kTT;
+  }
+  for (int i = tid; i < G * 2 * kD; i += kNT) sACC[i] = 0.f;
+  if (tid < 8) sL[tid] = 0.f;
+  if (tid == 0) *sAbort = 0;
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int b = b0 + lane;
+      const int v = b < B ? sNt[b] : 0;
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (b < B) sPre[b] = carry + x - v;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) sPre[B] = carry;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);                // full
+      mbar_init(smem_u32(&bars[C::STAGES + s]), kNCW);  // empty
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int64_t total = static_cast<int64_t>(sPre[B]) * Hkv;
+  const int64_t P_eff = total < P.num_ctas ? total : P.num_ctas;
+  if (static_cast<int64_t>(blockIdx.x) >= P_eff) return;
+  const int64_t x0 = static_cast<int64_t>(blockIdx.x) * total / P_eff;
+  const int64_t x1 = static_cast<int64_t>(blockIdx.x + 1) * total / P_eff;
+  const int n_pages = static_cast<int>(x1 - x0);
+
+  // ========================= producer warp =========================
+  if (warp == kNCW) {
+    if (lane == 0) {
+      if constexpr (REF == kRefBf16) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+      }
+      PageIter it;
+      it.seek(x0, sPre, sNt, B, Hkv);
+      int k = 0;
+      for (; k < n_pages; ++k) {
+        const int s = k % C::STAGES;
+        const uint32_t full = smem_u32(&bars[s]);
+        const uint32_t empty = smem_u32(&bars[C::STAGES + s]);
+        if (!mbar_wait_bounded(empty, ((k / C::STAGES) & 1) ^ 1)) {
+          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+          *sAbort = 1;
+          break;
+        }
+        if (*sAbort) break;
+        mbar_arrive_expect_tx(full, C::TX_BYTES);
+        uint8_t* st = stages + s * C::STAGE_BYTES;
+        const int t0 = it.page * kTT;
+        const int64_t rec0 = static_cast<int64_t>(it.b * Hkv + it.h) * P.plane_tokens + t0;
+        if constexpr (REF == kRefBf16) {
+          tma_load_4d(smem_u32(st + C::O_REFK), &tmK, 0, t0, it.h, it.b, full);
+          tma_load_4d(smem_u32(st + C::O_REFK + kTT * 128), &tmK, 64, t0, it.h, it.b, full);
+          tma_load_4d(smem_u32(st + C::O_REFV), &tmV, 0, t0, it.h, it.b, full);
+          tma_load_4d(smem_u32(st + C::O_REFV + kTT * 128), &tmV, 64, t0, it.h, it.b, full);
+        } else if constexpr (REF == kRefInt4) {
+          bulk_g2s(smem_u32(st + C::O_REFK), P.ref_codes[0] + rec0 * 64, kTT * 64, full);
+          bulk_g2s(smem_u32(st + C::O_REFV), P.ref_codes[1] + rec0 * 64, kTT * 64, full);
+          bulk_g2s(smem_u32(st + C::O_REFMK), P.ref_meta[0] + rec0 * 16, kTT * 16, full);
+          bulk_g2s(smem_u32(st + C::O_REFMV), P.ref_meta[1] + rec0 * 16, kTT * 16, full);
+        }
+        if constexpr (RB != 0) {
+          bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0] + rec0 * C::CB, kTT * C::CB, full);
+          bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[1] + rec0 * C::CB, kTT * C::CB, full);
+          bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0] + rec0 * C::MB, kTT * C::MB, full);
+          bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[1] + rec0 * C::MB, kTT * C::MB, full);
+        }
+        if constexpr (C::HAS_ALPHA) {
+          bulk_g2s(smem_u32(st + C::O_AL), P.alpha + rec0 * 4, kTT * 4, full);
+        }
+        it.next(sNt, B, Hkv);
+      }
+      // Drain: no copy this CTA issued may still be landing when it exits.
+      for (int kk = (k > C::STAGES ? k - C::STAGES : 0); kk < k; ++kk) {
+        if (!mbar_wait_bounded(smem_u32(&bars[kk % C::STAGES]), (kk / C::STAGES) & 1)) {
+          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+          break;
+        }
+      }
+    }
+    return;
+  }
+
+  // ========================= consumer warps =========================
+  // phase-1 mapping: token (within pass) and dim-slice index j
+  int tok1, j1;
+  if constexpr (G <= 2) {
+    const int jj = lane & (2 * G - 1);
+    const int tsub = (lane >> (G == 1 ? 1 : 2)) & ((4 / G) - 1);
+    const int box = (lane >> 3) & 1;
+    const int thi = lane >> 4;
+    tok1 = warp * (8 / G) + thi * (4 / G) + tsub;
+    j1 = box * (2 * G) + jj;
+  } else {
+    tok1 = warp * (8 / G) + lane / C::TPT;
+    j1 = lane % C::TPT;
+  }
+  const int d1 = C::D1 * j1;
+  // phase-2 mapping
+  const int slice = tid / C::TPR2;
+  const int j2 = tid % C::TPR2;
+  const int d2 = C::D2 * j2;
+
+  PageIter it;
+  it.seek(x0, sPre, sNt, B, Hkv);
+  int k = 0;
+  bool aborted = false;
+  while (k < n_pages) {
+    const int b = it.b, h = it.h;
+    const int seg_pages = min(sNt[b] - it.page, n_pages - k);
+    int len_b = P.ctx_len[b];
+    len_b = len_b < 0 ? 0 : (len_b > P.capacity ? P.capacity : len_b);
+
+    // ---- segment set-up: query (and its rotation) for the G heads of (b, h)
+    if (warp < G) {
+      const int qh = h * G + warp;
+      const uint2 raw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hkv * G + qh) * kD + 4 * lane);
+      const float2 a01 = bf16x2_to_f2(raw.x), a23 = bf16x2_to_f2(raw.y);
+      float x[4] = {a01.x, a01.y, a23.x, a23.y};
+      *reinterpret_cast<float4*>(&sQS[warp * kD + 4 * lane]) = make_float4(x[0], x[1], x[2], x[3]);
+      if (RB != 0 && P.rotate) {
+        float t0 = x[0] + x[1], t1 = x[0] - x[1], t2 = x[2] + x[3], t3 = x[2] - x[3];
+        x[0] = t0 + t2; x[2] = t0 - t2; x[1] = t1 + t3; x[3] = t1 - t3;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+          const bool up = (lane & m) != 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
+            x[e] = up ? (o - x[e]) : (x[e] + o);
+          }
+        }
+        const float c = 0.08838834764831845f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] *= c;
+      }
+      *reinterpret_cast<float4*>(&sQT[warp * kD + 4 * lane]) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+    named_bar_sync(kConsumerBar, kNCT);
+
+    // phase-1 registers: reference-side and residual-side query slices
+    float2 qref[G][C::D1 / 2];
+    float2 qres[G][C::D1 / 2];
+    constexpr int NG1 = RB ? ((C::D1 >= RG) ? C::D1 / RG : 1) : 1;
+    float qsum_res[G][NG1];
+    float qsum_ref[G];
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      qsum_ref[gi] = 0.f;
+#pragma unroll
+      for (int n = 0; n < NG1; ++n) qsum_res[gi][n] = 0.f;
+#pragma unroll
+      for (int e = 0; e < C::D1; e += 2) {
+        float r0 = sQS[gi * kD + d1 + e], r1 = sQS[gi * kD + d1 + e + 1];
+        qsum_ref[gi] += r0 + r1;
+        if constexpr (REF == kRefInt4) {
+          r0 *= pow2i(23 - code_pos<4>(e));
+          r1 *= pow2i(23 - code_pos<4>(e + 1));
+        }
+        qref[gi][e / 2] = make_float2(r0, r1);
+        if constexpr (RB != 0) {
+          float t0 = sQT[gi * kD + d1 + e], t1 = sQT[gi * kD + d1 + e + 1];
+          qsum_res[gi][(C::D1 >= RG) ? e / RG : 0] += t0 + t1;
+          qres[gi][e / 2] = make_float2(t0 * pow2i(23 - code_pos<RB>(e)),
+                                        t1 * pow2i(23 - code_pos<RB>(e + 1)));
+        }
+      }
+    }
+
+    // running softmax state and accumulators
+    float m_run[G], l_thr[G];
+    float2 acc_ref[G][C::D2 / 2];
+    float2 acc_res[G][C::D2 / 2];
+    float z_ref[G], z_res[G];
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+      m_run[gi] = -INFINITY;
+      l_thr[gi] = 0.f;
+      z_ref[gi] = 0.f;
+      z_res[gi] = 0.f;
+#pragma unroll
+      for (int e = 0; e < C::D2 / 2; ++e) {
+        acc_ref[gi][e] = make_float2(0.f, 0.f);
+        acc_res[gi][e] = make_float2(0.f, 0.f);
+      }
+    }
+
+    for (int sp = 0; sp < seg_pages; ++sp, ++k) {
+      const int s = k % C::STAGES;
+      const uint8_t* st = stages + s * C::STAGE_BYTES;
+      if (!*sAbort) {
+        if (!mbar_wait_bounded(smem_u32(&bars[s]), (k / C::STAGES) & 1)) {
+          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+          *sAbort = 1;
+          aborted = true;
+        }
+      }
+      const int t0 = it.page * kTT;
+      const int n_valid = min(kTT, len_b - t0);
+
+      // ---------------- phase 1: scores
+      float wmax[G];
+#pragma unroll
+      for (int gi = 0; gi < G; ++gi) wmax[gi] = -INFINITY;
+#pragma unroll
+      for (int ps = 0; ps < C::PASSES; ++ps) {
+        const int t = ps * C::TOK_PASS + tok1;
+        float part[G];
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) part[gi] = 0.f;
+        // reference side
+        float refdot[G];
+        if constexpr (REF == kRefBf16) {
+          float2 acc2[G];
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) acc2[gi] = make_float2(0.f, 0.f);
+          const uint8_t* rowK = st + C::O_REFK + (d1 >> 6) * (kTT * 128) + t * 128;
+          if constexpr (C::D1 >= 8) {
+#pragma unroll
+            for (int c = 0; c < C::D1 / 8; ++c) {
+              const int chunk = ((d1 & 63) >> 3) + c;
+              const uint4 v = *reinterpret_cast<const uint4*>(rowK + ((chunk ^ (t & 7)) << 4));
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float2 kv2 = bf16x2_to_f2(w4[u]);
+#pragma unroll
+                for (int gi = 0; gi < G; ++gi) acc2[gi] = __ffma2_rn(qref[gi][c * 4 + u], kv2, acc2[gi]);
+              }
+            }
+          } else {
+            const int chunk = (d1 & 63) >> 3;
+            const uint2 v = *reinterpret_cast<const uint2*>(rowK + ((chunk ^ (t & 7)) << 4) + ((d1 & 7) << 1));
+            const uint32_t w2[2] = {v.x, v.y};
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const float2 kv2 = bf16x2_to_f2(w2[u]);
+#pragma unroll
+              for (int gi = 0; gi < G; ++gi) acc2[gi] = __ffma2_rn(qref[gi][u], kv2, acc2[gi]);
+            }
+          }
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) refdot[gi] = acc2[gi].x + acc2[gi].y;
+        } else if constexpr (REF == kRefInt4) {
+          uint32_t cw[(C::D1 / 2 + 3) / 4];
+          load_codes<C::D1 / 2>(st + C::O_REFK + t * 64 + (d1 >> 1), cw);
+          const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMK + t * 16 + 4 * (d1 >> 5)));
+          float2 acc2[G];
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) acc2[gi] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int e = 0; e < C::D1; e += 2) {
+            const float2 f = f2sub1(make_float2(code_f<4>(cw, e), code_f<4>(cw, e + 1)));
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi) acc2[gi] = __ffma2_rn(qref[gi][e / 2], f, acc2[gi]);
+          }
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi)
+            refdot[gi] = fmaf(sz.x, acc2[gi].x + acc2[gi].y, sz.y * qsum_ref[gi]);
+        }
+        if constexpr (REF != kRefNone) {
+          float aK = 1.f;
+          if constexpr (C::HAS_ALPHA) aK = __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4));
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) part[gi] = aK * refdot[gi];
+        }
+        // residual side
+        if constexpr (RB != 0) {
+          constexpr int NBYTES = C::D1 * RB / 8;
+          uint32_t cw[(NBYTES + 3) / 4];
+          load_codes<NBYTES>(st + C::O_RESK + t * C::CB + (d1 * RB >> 3), cw);
+#pragma unroll
+          for (int n = 0; n < NG1; ++n) {
+            constexpr int EPG = (C::D1 >= RG) ? RG : C::D1;  // elements of this thread per group
+            const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(
+                st + C::O_RESMK + t * C::MB + 4 * (d1 / RG + n)));
+            float2 acc2[G];
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi) acc2[gi] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int e = n * EPG; e < (n + 1) * EPG; e += 2) {
+              const float2 f = f2sub1(make_float2(code_f<RB>(cw, e), code_f<RB>(cw, e + 1)));
+#pragma unroll
+              for (int gi = 0; gi < G; ++gi) acc2[gi] = __ffma2_rn(qres[gi][e / 2], f, acc2[gi]);
+            }
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi)
+              part[gi] += fmaf(sz.x, acc2[gi].x + acc2[gi].y, sz.y * qsum_res[gi][n]);
+          }
+        }
+        // reduce over the TPT threads of this token
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) {
+          float v = part[gi];
+          if constexpr (G <= 2) {
+#pragma unroll
+            for (int o = 1; o < 2 * G; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+          } else {
+#pragma unroll
+            for (int o = 1; o < C::TPT; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+          }
+          const float sc = (t < n_valid) ? v * P.scale_log2 : -INFINITY;
+          wmax[gi] = fmaxf(wmax[gi], sc);
+          if (j1 == 0) sS[gi * kTT + t] = sc;
+        }
+      }
+#pragma unroll
+      for (int gi = 0; gi < G; ++gi) {
+        float v = wmax[gi];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) sWM[gi * kNCW + warp] = v;
+      }
+      named_bar_sync(kConsumerBar, kNCT);
+
+      // ---------------- phase 1.5: softmax weights
+      float corr[G];
+#pragma unroll
+      for (int gi = 0; gi < G; ++gi) {
+        const float4 a = *reinterpret_cast<const float4*>(&sWM[gi * kNCW]);
+        const float4 c = *reinterpret_cast<const float4*>(&sWM[gi * kNCW + 4]);
+        const float mt = fmaxf(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)), fmaxf(fmaxf(c.x, c.y), fmaxf(c.z, c.w)));
+        const float mn = fmaxf(m_run[gi], mt);
+        corr[gi] = exp2f(m_run[gi] - mn);
+        m_run[gi] = mn;
+        l_thr[gi] *= corr[gi];
+      }
+#pragma unroll
+      for (int r = 0; r < (G * kTT + kNCT - 1) / kNCT; ++r) {
+        const int idx = tid + r * kNCT;
+        if (idx < G * kTT) {
+          const int t = idx % kTT, gi = idx / kTT;
+          float mg = m_run[0];
+#pragma unroll
+          for (int g2 = 1; g2 < G; ++g2) if (gi == g2) mg = m_run[g2];
+          float p = 0.f, pa = 0.f;
+          if (t < n_valid) {
+            p = exp2f(sS[gi * kTT + t] - mg);
+            pa = p;
+            if constexpr (C::HAS_ALPHA) pa = p * __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4 + 2));
+          }
+          sP[gi * kTT + t] = p;
+          sPA[gi * kTT + t] = pa;
+#pragma unroll
+          for (int g2 = 0; g2 < G; ++g2) if (gi == g2) l_thr[g2] += p;
+        }
+      }
+      named_bar_sync(kConsumerBar, kNCT);
+
+      // ---------------- phase 2: value accumulation
+#pragma unroll
+      for (int gi = 0; gi < G; ++gi) {
+        const float2 c2 = make_float2(corr[gi], corr[gi]);
+#pragma unroll
+        for (int e = 0; e < C::D2 / 2; ++e) {
+          acc_ref[gi][e] = __fmul2_rn(acc_ref[gi][e], c2);
+          acc_res[gi][e] = __fmul2_rn(acc_res[gi][e], c2);
+        }
+        z_ref[gi] *= corr[gi];
+        z_res[gi] *= corr[gi];
+      }
+#pragma unroll
+      for (int i = 0; i < C::TOK2; ++i) {
+        const int t = slice + i * C::SLICES;
+        if (t >= n_valid) break;
+        float pp[G], pa[G];
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) {
+          pp[gi] = sP[gi * kTT + t];
+          pa[gi] = sPA[gi * kTT + t];
+        }
+        if constexpr (REF == kRefBf16) {
+          const uint8_t* rowV = st + C::O_REFV + (d2 >> 6) * (kTT * 128) + t * 128;
+          const int chunk = (d2 & 63) >> 3;
+          if constexpr (C::D2 == 8) {
+            const uint4 v = *reinterpret_cast<const uint4*>(rowV + ((chunk ^ (t & 7)) << 4));
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 vv = bf16x2_to_f2(w4[u]);
+#pragma unroll
+              for (int gi = 0; gi < G; ++gi)
+                acc_ref[gi][u] = __ffma2_rn(make_float2(pa[gi], pa[gi]), vv, acc_ref[gi][u]);
+            }
+          } else {
+            const uint2 v = *reinterpret_cast<const uint2*>(rowV + ((chunk ^ (t & 7)) << 4) + ((d2 & 7) << 1));
+            const uint32_t w2[2] = {v.x, v.y};
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const float2 vv = bf16x2_to_f2(w2[u]);
+#pragma unroll
+              for (int gi = 0; gi < G; ++gi)
+                acc_ref[gi][u] = __ffma2_rn(make_float2(pa[gi], pa[gi]), vv, acc_ref[gi][u]);
+            }
+          }
+        } else if constexpr (REF == kRefInt4) {
+          uint32_t cw[1];
+          load_codes<C::D2 / 2>(st + C::O_REFV + t * 64 + (d2 >> 1), cw);
+          const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMV + t * 16 + 4 * (d2 >> 5)));
+#pragma unroll
+          for (int e = 0; e < C::D2; e += 2) {
+            const float2 f = f2sub1(make_float2(code_f<4>(cw, e), code_f<4>(cw, e + 1)));
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi) {
+              const float w = pa[gi] * sz.x;
+              acc_ref[gi][e / 2] = __ffma2_rn(make_float2(w, w), f, acc_ref[gi][e / 2]);
+            }
+          }
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) z_ref[gi] = fmaf(pa[gi], sz.y, z_ref[gi]);
+        }
+        if constexpr (RB != 0) {
+          uint32_t cw[1];
+          load_codes<C::D2 * RB / 8>(st + C::O_RESV + t * C::CB + (d2 * RB >> 3), cw);
+          const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_RESMV + t * C::MB + 4 * (d2 / RG)));
+#pragma unroll
+          for (int e = 0; e < C::D2; e += 2) {
+            const float2 f = f2sub1(make_float2(code_f<RB>(cw, e), code_f<RB>(cw, e + 1)));
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi) {
+              const float w = pp[gi] * sz.x;
+              acc_res[gi][e / 2] = __ffma2_rn(make_float2(w, w), f, acc_res[gi][e / 2]);
+            }
+          }
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) z_res[gi] = fmaf(pp[gi], sz.y, z_res[gi]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars[C::STAGES + s]));
+      it.next(sNt, B, Hkv);
+    }
+
+    // ---- flush this (b, h) segment: reduce over slices, write the partial
+#pragma unroll
+    for (int gi = 0; gi < G; ++gi) {
+#pragma unroll
+      for (int e = 0; e < C::D2; ++e) {
+        const float2 ar = acc_ref[gi][e / 2];
+        float vr = (e & 1) ? ar.y : ar.x;
+        if constexpr (REF == kRefInt4) vr = fmaf(vr, pow2i(23 - code_pos<4>(e)), z_ref[gi]);
+        atomicAdd(&sACC[gi * 2 * kD + d2 + e], vr);
+        if constexpr (RB != 0) {
+          const float2 as = acc_res[gi][e / 2];
+          const float vs = fmaf((e & 1) ? as.y : as.x, pow2i(23 - code_pos<RB>(e)), z_res[gi]);
+          atomicAdd(&sACC[gi * 2 * kD + kD + d2 + e], vs);
+        }
+      }
+      if (l_thr[gi] != 0.f) atomicAdd(&sL[gi], l_thr[gi]);
+    }
+    named_bar_sync(kConsumerBar, kNCT);
+    {
+      const int pair = b * Hkv + h;
+      float* rec = P.partials + static_cast<int64_t>(pair + blockIdx.x) * G * kPartialFloats;
+      for (int i = tid; i < G * (2 * kD / 4); i += kNCT) {
+        const int gi = i / (2 * kD / 4), f4 = i % (2 * kD / 4);
+        float4* src = reinterpret_cast<float4*>(&sACC[gi * 2 * kD]) + f4;
+        reinterpret_cast<float4*>(rec + gi * kPartialFloats + 4)[f4] = *src;
+        *src = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      if (tid < G) {
+        float mg = m_run[0];
+#pragma unroll
+        for (int g2 = 1; g2 < G; ++g2) if (tid == g2) mg = m_run[g2];
+        reinterpret_cast<float4*>(rec + tid * kPartialFloats)[0] = make_float4(mg, sL[tid], 0.f, 0.f);
+        sL[tid] = 0.f;
+      }
+    }
+  }
+  (void)aborted;
+}
+
+// ---------------------------------------------------------------------------
+// combine kernel: one warp per (b, q-head)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams P, int G, int rotate_res) {
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int Hq = P.Hkv * G;
+  if (wid >= P.B * Hq) return;
+  const int b = wid / Hq, qh = wid % Hq, h = qh / G, gi = qh % G;
+  auto clamp_len = [&](int len) { return len < 0 ? 0 : (len > P.capacity ? P.capacity : len); };
+  // page offsets (same arithmetic as the split kernel)
+  int64_t pre = 0, tot = 0;
+  for (int b2 = lane; b2 < P.B; b2 += 32) {
+    const int nt = (clamp_len(P.ctx_len[b2]) + kTT - 1) / kTT;
+    tot += nt;
+    if (b2 < b) pre += nt;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    pre += __shfl_xor_sync(0xffffffffu, pre, o);
+  }
+  const int nt_b = (clamp_len(P.ctx_len[b]) + kTT - 1) / kTT;
+  const int64_t total = tot * P.Hkv;
+  const int64_t P_eff = total < P.num_ctas ? total : P.num_ctas;
+
+  float m = -INFINITY, l = 0.f;
+  float4 ar = make_float4(0.f, 0.f, 0.f, 0.f), as = ar;
+  if (nt_b > 0) {
+    const int64_t ts = pre * P.Hkv + static_cast<int64_t>(h) * nt_b;
+    const int64_t te = ts + nt_b;
+    const int64_t c0 = ((ts + 1) * P_eff - 1) / total;
+    const int64_t c1 = (te * P_eff - 1) / total;
+    const int pair = b * P.Hkv + h;
+    for (int64_t c = c0; c <= c1; ++c) {
+      const float* rec = P.partials + ((pair + c) * G + gi) * kPartialFloats;
+      const float4 ml = reinterpret_cast<const float4*>(rec)[0];
+      const float4 r = reinterpret_cast<const float4*>(rec + 4)[lane];
+      const float4 s = reinterpret_cast<const float4*>(rec + 4 + kD)[lane];
+      const float mn = fmaxf(m, ml.x);
+      const float a = exp2f(m - mn), bb = exp2f(ml.x - mn);
+      l = l * a + ml.y * bb;
+      ar = make_float4(ar.x * a + r.x * bb, ar.y * a + r.y * bb, ar.z * a + r.z * bb, ar.w * a + r.w * bb);
+      as = make_float4(as.x * a + s.x * bb, as.y * a + s.y * bb, as.z * a + s.z * bb, as.w * a + s.w * bb);
+      m = mn;
+    }
+  }
+  // current (tail) tokens in bf16
+  if (P.n_tail > 0) {
+    const uint2 qraw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hq + qh) * kD + 4 * lane);
+    const float2 q01 = bf16x2_to_f2(qraw.x), q23 = bf16x2_to_f2(qraw.y);
+    for (int j = 0; j < P.n_tail; ++j) {
+      const int64_t off = ((static_cast<int64_t>(b) * P.Hkv + h) * P.n_tail + j) * kD + 4 * lane;
+      const uint2 kr = *reinterpret_cast<const uint2*>(P.k_tail + off);
+      const uint2 vr = *reinterpret_cast<const uint2*>(P.v_tail + off);
+      const float2 k01 = bf16x2_to_f2(kr.x), k23 = bf16x2_to_f2(kr.y);
+      float d = q01.x * k01.x + q01.y * k01.y + q23.x * k23.x + q23.y * k23.y;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+      const float sc = d * P.scale_log2;
+      const float mn = fmaxf(m, sc);
+      const float a = exp2f(m - mn), p = exp2f(sc - mn);
+      const float2 v01 = bf16x2_to_f2(vr.x), v23 = bf16x2_to_f2(vr.y);
+      l = l * a + p;
+      ar = make_float4(ar.x * a + p * v01.x, ar.y * a + p * v01.y, ar.z * a + p * v23.x, ar.w * a + p * v23.y);
+      as = make_float4(as.x * a, as.y * a, as.z * a, as.w * a);
+      m = mn;
+    }
+  }
+  if (rotate_res) {
+    float x[4] = {as.x, as.y, as.z, as.w};
+    float t0 = x[0] + x[1], t1 = x[0] - x[1], t2 = x[2] + x[3], t3 = x[2] - x[3];
+    x[0] = t0 + t2; x[2] = t0 - t2; x[1] = t1 + t3; x[3] = t1 - t3;
+#pragma unroll
+    for (int mm = 1; mm < 32; mm <<= 1) {
+      const bool up = (lane & mm) != 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float o = __shfl_xor_sync(0xffffffffu, x[e], mm);
+        x[e] = up ? (o - x[e]) : (x[e] + o);
+      }
+    }
+    const float c = 0.08838834764831845f;
+    as = make_float4(x[0] * c, x[1] * c, x[2] * c, x[3] * c);
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  float4 o = make_float4((ar.x + as.x) * inv, (ar.y + as.y) * inv, (ar.z + as.z) * inv, (ar.w + as.w) * inv);
+  reinterpret_cast<float4*>(P.out + (static_cast<int64_t>(b) * Hq + qh) * kD)[lane] = o;
+}
+
+// ---------------------------------------------------------------------------
+// dispatch
+// ---------------------------------------------------------------------------
+template <int REF, int RB, int RG, int G>
+cudaError_t launch_split(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
+                         cudaStream_t s) {
+  using C = Cfg<REF, RB, RG, G>;
+  auto kern = decode_split_kernel<REF, RB, RG, G>;
+  static bool attr_done = false;  // per instantiation; set once per process
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  kern<<<p.num_ctas, kNT, C::SMEM_BYTES, s>>>(p, *tk, *tv);
+  return cudaGetLastError();
+}
+
+using SplitFn = cudaError_t (*)(const DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);
+
+template <int REF, int RB, int RG>
+SplitFn pick_g(int G) {
+  switch (G) {
+    case 1: return launch_split<REF, RB, RG, 1>;
+    case 2: return launch_split<REF, RB, RG, 2>;
+    case 4: return launch_split<REF, RB, RG, 4>;
+    case 8: return launch_split<REF, RB, RG, 8>;
+    default: return nullptr;
+  }
+}
+
+SplitFn pick(int ref_kind, int res_bits, int res_group, int G) {
+  if (ref_kind == kRefBf16) {
+    if (res_bits == 0) return pick_g<kRefBf16, 0, 32>(G);
+    if (res_bits == 2) return res_group == 16 ? pick_g<kRefBf16, 2, 16>(G) : pick_g<kRefBf16, 2, 32>(G);
+    if (res_bits == 4) return res_group == 16 ? pick_g<kRefBf16, 4, 16>(G) : pick_g<kRefBf16, 4, 32>(G);
+  } else if (ref_kind == kRefInt4) {
+    if (res_bits == 0) return pick_g<kRefInt4, 0, 32>(G);
+    if (res_bits == 2) return res_group == 16 ? pick_g<kRefInt4, 2, 16>(G) : pick_g<kRefInt4, 2, 32>(G);
+    if (res_bits == 4) return res_group == 16 ? pick_g<kRefInt4, 4, 16>(G) : pick_g<kRefInt4, 4, 32>(G);
+  } else if (ref_kind == kRefNone) {
+    if (res_bits == 2) return res_group == 16 ? pick_g<kRefNone, 2, 16>(G) : pick_g<kRefNone, 2, 32>(G);
+    if (res_bits == 4) return res_group == 16 ? pick_g<kRefNone, 4, 16>(G) : pick_g<kRefNone, 4, 32>(G);
+  }
+  return nullptr;
+}
+
+}  // namespace
+
+bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G) {
+  if (res_bits != 0 && res_group != 16 && res_group != 32) return false;
+  return pick(ref_kind, res_bits, res_group, G) != nullptr;
+}
+
+int decode_grid_ctas(int device) {
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0) sms = 148;
+  return sms;  // one persistent CTA per SM
+}
+
+int64_t decode_workspace_bytes(int B, int Hkv, int G, int num_ctas) {
+  const int64_t slots = static_cast<int64_t>(B) * Hkv + num_ctas;
+  return slots * G * kPartialFloats * static_cast<int64_t>(sizeof(float));
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int ref_kind, int res_bits, int res_group,
+                          const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s) {
+  SplitFn fn = pick(ref_kind, res_bits, res_group, p.G);
+  if (fn == nullptr) return cudaErrorInvalidValue;
+  cudaError_t e = fn(p, tmap_k, tmap_v, s);
+  if (e != cudaSuccess) return e;
+  const int warps = p.B * p.Hkv * p.G;
+  if (warps == 0) return cudaSuccess;
+  decode_combine_kernel<<<(warps + 3) / 4, 128, 0, s>>>(p, p.G, (res_bits != 0 && p.rotate) ? 1 : 0);
+  return cudaGetLastError();
+}
+
+}  // namespace rq

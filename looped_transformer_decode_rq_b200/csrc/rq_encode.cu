@@ -1,0 +1,324 @@
+// rq_encode.cu -- ResidualQuant encode and (test-support) reconstruction on
+// sm_100a.
+//
+// Encode follows "ResidualQuant: KV Cache Quantization for Looped Transformers
+// with 2-Bit Residuals" (abstract; Figure 1 steps 2-5; Figure 2 caption): the
+// final loop is the reference, every other loop is stored as the LS-scaled
+// residual, rotated by the order-128 Hadamard, quantised per group to INT2 or
+// INT4 with an fp16 scale and offset.
+//
+// One warp handles one (b, h, token) for all loops: lanes 0-15 the key,
+// lanes 16-31 the value; lane j of a half owns elements 8j..8j+7 and loads
+// them with one 16-byte access.  The arithmetic order is fixed so that codes,
+// scales, offsets and alphas are reproducible bit for bit:
+//   dot products: per lane, +0 then += x_e*r_e in element order (each product
+//     and sum rounded separately, no FMA contraction), then a butterfly over
+//     lane distances 8, 4, 2, 1;
+//   rotation: butterflies at strides 1..64 in increasing order, then one
+//     multiply by fl32(1/sqrt(128));
+//   quantiser: min/max made unsigned-zero, s = (mx - mn)/(2^b - 1), fp16 RNE
+//     scale and offset, code = clamp(rint((y - z)/s), 0, 2^b - 1), code 0 when
+//     the fp16 scale is 0.
+#include "rq_common.cuh"
+#include "rq_internal.h"
+
+namespace rq {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+// fl32(1/sqrt(128)) = 0x3DB504F3
+__device__ __forceinline__ float inv_sqrt_d() { return __int_as_float(0x3DB504F3); }
+
+__device__ __forceinline__ void load8_bf16(const uint16_t* src, float (&x)[8]) {
+  const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
+  float2 a = bf16x2_to_f2(raw.x), b = bf16x2_to_f2(raw.y), c = bf16x2_to_f2(raw.z),
+         d = bf16x2_to_f2(raw.w);
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  x[4] = c.x; x[5] = c.y; x[6] = d.x; x[7] = d.y;
+}
+
+__device__ __forceinline__ bool in_range8(const float (&x)[8]) {
+  bool ok = true;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ok &= (fabsf(x[e]) <= 65504.f);  // false for NaN
+  return ok;
+}
+
+// <a, b> over a half-warp's 128 elements in the fixed order.
+__device__ __forceinline__ float tree_dot(const float (&a)[8], const float (&b)[8]) {
+  float p = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) p = __fadd_rn(p, __fmul_rn(a[e], b[e]));
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(kFull, p, o));
+  return p;
+}
+
+// In-place rotation of a half-warp's 128 elements (lane j holds 8j..8j+7).
+__device__ __forceinline__ void fwht128(float (&x)[8], int j) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if ((e & h) == 0) {
+        const float a = x[e], b = x[e + h];
+        x[e] = __fadd_rn(a, b);
+        x[e + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < 16; m <<= 1) {
+    const bool upper = (j & m) != 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float o = __shfl_xor_sync(kFull, x[e], m);
+      x[e] = upper ? __fsub_rn(o, x[e]) : __fadd_rn(x[e], o);
+    }
+  }
+  const float c = inv_sqrt_d();
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = __fmul_rn(x[e], c);
+}
+
+// Group min-max quantiser.  lanes_per_group = g / 8 (2 or 4).  Returns the
+// 8 codes of this lane and the group's fp16 scale/offset.
+__device__ __forceinline__ void quantize8(const float (&y)[8], int bits, int lanes_per_group,
+                                          uint32_t (&c)[8], __half& s_h, __half& z_h) {
+  float mn = y[0], mx = y[0];
+#pragma unroll
+  for (int e = 1; e < 8; ++e) {
+    mn = fminf(mn, y[e]);
+    mx = fmaxf(mx, y[e]);
+  }
+  for (int o = 1; o < lanes_per_group; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+  }
+  mn = __fadd_rn(mn, 0.f);  // an exact zero becomes +0 in every lane
+  mx = __fadd_rn(mx, 0.f);
+  const float qmax = static_cast<float>((1 << bits) - 1);
+  const float s = __fdiv_rn(__fsub_rn(mx, mn), qmax);
+  s_h = __float2half_rn(s);
+  z_h = __float2half_rn(mn);
+  const float sf = __half2float(s_h), zf = __half2float(z_h);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    float u = 0.f;
+    if (sf > 0.f) u = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(y[e], zf), sf)), 0.f), qmax);
+    c[e] = static_cast<uint32_t>(u);
+  }
+}
+
+__device__ __forceinline__ uint32_t half2_bits(__half s, __half z) {
+  return static_cast<uint32_t>(__half_as_ushort(s)) |
+         (static_cast<uint32_t>(__half_as_ushort(z)) << 16);
+}
+
+__device__ __forceinline__ bool half_finite(__half h) {
+  return (__half_as_ushort(h) & 0x7C00u) != 0x7C00u;
+}
+
+__global__ void __launch_bounds__(256) encode_kernel(const EncodeParams P) {
+  const int warp = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int total = P.B * P.Hkv * P.n_tokens;
+  if (warp >= total) return;
+  const int lane = threadIdx.x & 31;
+  const int kv = lane >> 4;  // 0: key, 1: value
+  const int j = lane & 15;
+  const int i = warp % P.n_tokens;
+  const int bh = warp / P.n_tokens;
+  const int h = bh % P.Hkv;
+  const int b = bh / P.Hkv;
+  const int pos = (P.positions ? P.positions[b] : P.start_pos) + i;
+  if (pos < 0 || pos >= P.capacity) {  // warp-uniform
+    if (lane == 0) set_flag(P.status, RQ_FLAG_POSITION);
+    return;
+  }
+  const uint16_t* X = kv ? P.v : P.k;
+  const int64_t src0 = b * P.s_b + h * P.s_h + static_cast<int64_t>(i) * P.s_t + 8 * j;
+  const int64_t rec = static_cast<int64_t>(b * P.Hkv + h) * P.cap_pad + pos;
+  bool bad = false, overflow = false;
+
+  // ---- reference loop
+  float ref[8];
+  {
+    const uint16_t* src = X + static_cast<int64_t>(P.L - 1) * P.s_l + src0;
+    load8_bf16(src, ref);
+    bad |= !in_range8(ref);
+    if (P.ref_bits == 16) {
+      *reinterpret_cast<uint4*>(P.ref_plane[kv] + rec * 256 + 16 * j) =
+          __ldg(reinterpret_cast<const uint4*>(src));
+    } else {
+      uint32_t c[8];
+      __half s_h, z_h;
+      quantize8(ref, 4, 4, c, s_h, z_h);
+      uint32_t w = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w |= c[e] << (4 * e);
+      *reinterpret_cast<uint32_t*>(P.ref_plane[kv] + rec * 64 + 4 * j) = w;
+      if ((j & 3) == 0)
+        *reinterpret_cast<uint32_t*>(P.ref_meta[kv] + rec * 16 + 4 * (j >> 2)) = half2_bits(s_h, z_h);
+      overflow |= !(half_finite(s_h) && half_finite(z_h));
+      const float sf = __half2float(s_h), zf = __half2float(z_h);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ref[e] = __fadd_rn(zf, __fmul_rn(static_cast<float>(c[e]), sf));
+    }
+  }
+  float refref = 0.f;
+  bool have_refref = false;
+
+  // ---- residual loops
+  for (int l = 0; l < P.L - 1; ++l) {
+    float x[8];
+    load8_bf16(X + static_cast<int64_t>(l) * P.s_l + src0, x);
+    bad |= !in_range8(x);
+    float a = 0.f;
+    const int mode = P.alpha_mode[l];
+    if (mode == RQ_ALPHA_LS) {
+      if (!have_refref) {
+        refref = tree_dot(ref, ref);
+        have_refref = true;
+      }
+      const float num = tree_dot(x, ref);
+      a = (refref == 0.f) ? 0.f : __fdiv_rn(num, refref);
+    } else if (mode == RQ_ALPHA_ONE) {
+      a = 1.f;
+    }
+    const __half a_h = __float2half_rn(a);
+    overflow |= !half_finite(a_h);
+    if (j == 0)
+      *reinterpret_cast<__half*>(P.alpha[l] + rec * 4 + 2 * kv) = a_h;
+    const float af = __half2float(a_h);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], __fmul_rn(af, ref[e]));
+    if (P.rotate[l]) fwht128(x, j);
+    const int bits = P.bits[l], g = P.group[l];
+    uint32_t c[8];
+    __half s_h, z_h;
+    quantize8(x, bits, g >> 3, c, s_h, z_h);
+    overflow |= !(half_finite(s_h) && half_finite(z_h));
+    if (bits == 2) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w |= c[e] << (2 * e);
+      *reinterpret_cast<uint16_t*>(P.codes[l][kv] + rec * 32 + 2 * j) = static_cast<uint16_t>(w);
+    } else {
+      uint32_t w = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w |= c[e] << (4 * e);
+      *reinterpret_cast<uint32_t*>(P.codes[l][kv] + rec * 64 + 4 * j) = w;
+    }
+    const int lpg = g >> 3;
+    if ((j % lpg) == 0)
+      *reinterpret_cast<uint32_t*>(P.meta[l][kv] + rec * (4 * (kD / g)) + 4 * (j / lpg)) =
+          half2_bits(s_h, z_h);
+  }
+  const unsigned any_bad = __ballot_sync(kFull, bad);
+  const unsigned any_ovf = __ballot_sync(kFull, overflow);
+  if (lane == 0) {
+    if (any_bad) set_flag(P.status, RQ_FLAG_BAD_INPUT);
+    if (any_ovf) set_flag(P.status, RQ_FLAG_META_OVERFLOW);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Reconstruction (test support): fp32 alpha*ref + H^T deq(codes)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fwht128_fast(float (&x)[8], int j) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if ((e & h) == 0) {
+        const float a = x[e], b = x[e + h];
+        x[e] = a + b;
+        x[e + h] = a - b;
+      }
+#pragma unroll
+  for (int m = 1; m < 16; m <<= 1) {
+    const bool upper = (j & m) != 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float o = __shfl_xor_sync(kFull, x[e], m);
+      x[e] = upper ? (o - x[e]) : (x[e] + o);
+    }
+  }
+  const float c = inv_sqrt_d();
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] *= c;
+}
+
+__device__ __forceinline__ void dequant8(const uint8_t* codes, const uint8_t* meta, int bits,
+                                         int g, int64_t rec, int j, float (&y)[8]) {
+  const int lpg = g >> 3;
+  const float2 sz = half2_bits_to_f2(
+      *reinterpret_cast<const uint32_t*>(meta + rec * (4 * (kD / g)) + 4 * (j / lpg)));
+  if (bits == 2) {
+    const uint32_t w = *reinterpret_cast<const uint16_t*>(codes + rec * 32 + 2 * j);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = fmaf(static_cast<float>((w >> (2 * e)) & 3u), sz.x, sz.y);
+  } else {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(codes + rec * 64 + 4 * j);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = fmaf(static_cast<float>((w >> (4 * e)) & 15u), sz.x, sz.y);
+  }
+}
+
+__global__ void __launch_bounds__(256) reconstruct_kernel(const ReconstructParams P) {
+  const int warp = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int total = P.B * P.Hkv * P.n;
+  if (warp >= total) return;
+  const int lane = threadIdx.x & 31;
+  const int kv = lane >> 4, j = lane & 15;
+  const int i = warp % P.n;
+  const int bh = warp / P.n;
+  const int64_t rec = static_cast<int64_t>(bh) * P.cap_pad + P.t0 + i;
+  float ref[8];
+  if (P.ref_bits == 16) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(P.ref_plane[kv] + rec * 256 + 16 * j);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = bf16x2_to_f2(w[e]);
+      ref[2 * e] = f.x;
+      ref[2 * e + 1] = f.y;
+    }
+  } else {
+    dequant8(P.ref_plane[kv], P.ref_meta[kv], 4, 32, rec, j, ref);
+  }
+  float out[8];
+  if (P.is_ref) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = ref[e];
+  } else {
+    dequant8(P.codes[kv], P.meta[kv], P.bits, P.group, rec, j, out);
+    if (P.rotate) fwht128_fast(out, j);
+    const float a = __half2float(*reinterpret_cast<const __half*>(P.alpha + rec * 4 + 2 * kv));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = fmaf(a, ref[e], out[e]);
+  }
+  float* dst = P.out[kv] + (static_cast<int64_t>(bh) * P.n + i) * kD + 8 * j;
+  reinterpret_cast<float4*>(dst)[0] = make_float4(out[0], out[1], out[2], out[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(out[4], out[5], out[6], out[7]);
+}
+
+}  // namespace
+
+cudaError_t launch_encode(const EncodeParams& p, cudaStream_t s) {
+  const int64_t warps = static_cast<int64_t>(p.B) * p.Hkv * p.n_tokens;
+  if (warps == 0) return cudaSuccess;
+  const int64_t blocks = (warps + 7) / 8;
+  encode_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reconstruct(const ReconstructParams& p, cudaStream_t s) {
+  const int64_t warps = static_cast<int64_t>(p.B) * p.Hkv * p.n;
+  if (warps == 0) return cudaSuccess;
+  const int64_t blocks = (warps + 7) / 8;
+  reconstruct_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace rq

@@ -1,0 +1,91 @@
+// rq_internal.h -- kernel parameter blocks and launcher entry points shared by
+// the host library (rq_api.cpp) and the CUDA translation units.  Not part of
+// the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/rq_api.h"
+
+namespace rq {
+
+enum RefKind : int { kRefNone = 0, kRefBf16 = 1, kRefInt4 = 2 };
+
+struct EncodeParams {
+  int L, B, Hkv;
+  int64_t cap_pad;
+  int capacity;
+  int n_tokens;
+  int start_pos;
+  const int32_t* positions;  // device [B] or null
+  const uint16_t* k;         // bf16 bits
+  const uint16_t* v;
+  int64_t s_l, s_b, s_h, s_t;  // element strides
+  int ref_bits;                // 16 | 4
+  uint8_t* ref_plane[2];
+  uint8_t* ref_meta[2];
+  uint8_t* codes[RQ_MAX_LOOPS][2];
+  uint8_t* meta[RQ_MAX_LOOPS][2];
+  uint8_t* alpha[RQ_MAX_LOOPS];
+  int bits[RQ_MAX_LOOPS], group[RQ_MAX_LOOPS], rotate[RQ_MAX_LOOPS], alpha_mode[RQ_MAX_LOOPS];
+  int32_t* status;
+};
+
+struct ReconstructParams {
+  int B, Hkv;
+  int64_t cap_pad;
+  int t0, n;
+  int ref_bits;
+  const uint8_t* ref_plane[2];
+  const uint8_t* ref_meta[2];
+  int is_ref;  // reconstruct the reference loop itself
+  const uint8_t* codes[2];
+  const uint8_t* meta[2];
+  const uint8_t* alpha;
+  int bits, group, rotate;
+  float* out[2];
+};
+
+// One decode call: either a residual loop of a cache, its reference loop, or a
+// plain bf16 cache.  Planes are indexed by record = (b*Hkv + h)*plane_tokens + t.
+struct DecodeParams {
+  int B, Hkv, G;
+  int capacity;          // valid positions per sequence (ctx_len is clamped to it)
+  int64_t plane_tokens;  // record stride between (b, h) slabs for byte planes
+  // reference (bf16 via tensor maps; INT4 via byte planes)
+  const uint8_t* ref_codes[2];
+  const uint8_t* ref_meta[2];
+  // residual
+  const uint8_t* res_codes[2];
+  const uint8_t* res_meta[2];
+  const uint8_t* alpha;  // (alpha_K, alpha_V) fp16 pairs, or null (alpha = 1)
+  int rotate;
+  // query / lengths / tail / output
+  const uint16_t* q;     // bf16 [B][Hq][128]
+  const int32_t* ctx_len;
+  const uint16_t* k_tail;  // bf16 [B][Hkv][n_tail][128]
+  const uint16_t* v_tail;
+  int n_tail;
+  float scale_log2;      // softmax_scale * log2(e)
+  float* out;            // fp32 [B][Hq][128]
+  float* partials;       // workspace
+  int num_ctas;          // persistent grid size P of the split kernel
+  int32_t* status;
+};
+
+// Split-K partial record per (slot, head): m, l, pad, pad, acc_ref[128], acc_res[128]
+constexpr int kPartialFloats = 4 + 2 * RQ_HEAD_DIM;
+
+int64_t decode_workspace_bytes(int B, int Hkv, int G, int num_ctas);
+int decode_grid_ctas(int device);  // persistent grid size for this device
+
+cudaError_t launch_encode(const EncodeParams& p, cudaStream_t s);
+cudaError_t launch_reconstruct(const ReconstructParams& p, cudaStream_t s);
+// ref_kind: RefKind; res_bits: 0 | 2 | 4; res_group: 16 | 32
+cudaError_t launch_decode(const DecodeParams& p, int ref_kind, int res_bits, int res_group,
+                          const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
+bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G);
+
+}  // namespace rq

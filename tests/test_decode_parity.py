@@ -1,0 +1,127 @@
+"""GPU decode attention vs the float64 oracle: max over (b, q-head) of
+||o - o_ref||_inf / ||o_ref||_inf <= 2e-3, on shapes that span several pages,
+several CTAs and ragged tails, for every reference/residual format."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.rq_oracle as O
+from looped_transformer_decode_rq_b200 import synth
+from tests.helpers import ATTN_TOL, oracle_encode, rel_err_rows, to_np32
+
+pytestmark = pytest.mark.gpu
+
+
+def run_case(rq, wl, loops=None, n_tail=None, lengths=None, scale=None):
+    if n_tail is not None:
+        wl = wl.with_(n_tail=n_tail)
+    if lengths is not None:
+        wl = wl.with_(lengths=tuple(lengths))
+    inp = synth.make_inputs(wl, "cpu")
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    enc = oracle_encode(inp, cfgd)
+    ctx = inp["ctx_len"]
+    worst = 0.0
+    for loop in (loops if loops is not None else range(wl.num_loops)):
+        kt = inp["k_tail"][loop].cuda() if wl.n_tail else None
+        vt = inp["v_tail"][loop].cuda() if wl.n_tail else None
+        out = cache.decode_attention(loop, inp["q"][loop].cuda(), ctx.cuda(), kt, vt, softmax_scale=scale)
+        torch.cuda.synchronize()
+        want = O.decode_attention_f64(enc, loop, to_np32(inp["q"][loop]), ctx.numpy(),
+                                      to_np32(inp["k_tail"][loop]) if wl.n_tail else None,
+                                      to_np32(inp["v_tail"][loop]) if wl.n_tail else None,
+                                      scale if scale is not None else 1 / np.sqrt(128))
+        got = out.cpu().numpy()
+        empty = (ctx.numpy() == 0) & (wl.n_tail == 0)
+        if empty.any():
+            assert np.all(got[empty] == 0)
+        keep = ~empty
+        if keep.any():
+            err = rel_err_rows(got[keep], want[keep])
+            worst = max(worst, float(err.max()))
+            assert err.max() <= ATTN_TOL, (wl.name, loop, float(err.max()))
+    assert cache.get_error() == 0
+    return worst
+
+
+def test_tiny_all_loops(librq):
+    run_case(librq, synth.tiny())
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_ragged_batch_gqa(librq, G):
+    wl = synth.Workload(name=f"ragged_G{G}", batch=4, kv_heads=2, q_heads=2 * G, context=257,
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.02, seed=20 + G)
+    run_case(librq, wl, lengths=[1, 31, 257, 33])
+
+
+@pytest.mark.parametrize("bits,group,ref_bits", [
+    ((2, 2, 2), 16, 16), ((4, 4, 4), 32, 16), ((4, 4, 4), 16, 16),
+    ((2, 2, 4), 32, 4), ((2, 2, 2), 16, 4),
+])
+def test_formats(librq, bits, group, ref_bits):
+    wl = synth.Workload(name=f"fmt_{bits}_{group}_{ref_bits}", batch=3, kv_heads=2, q_heads=4, context=130,
+                        bits=tuple(bits) + (ref_bits,), group=(group,) * 3 + (32,),
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.02, seed=31)
+    run_case(librq, wl, lengths=[64, 65, 130], n_tail=2)
+
+
+def test_direct_and_unrotated_modes(librq):
+    wl = synth.Workload(name="modes", batch=2, kv_heads=2, q_heads=2, context=100,
+                        rotate=(0, 1, 0, 0), alpha_mode=(2, 1, 0, 0), sigma=(0.3, 0.2, 0.1), seed=32)
+    run_case(librq, wl, lengths=[100, 37])
+
+
+def test_empty_contexts_and_tail_only(librq):
+    wl = synth.Workload(name="empty", batch=3, kv_heads=2, q_heads=4, context=70, seed=33)
+    run_case(librq, wl, lengths=[0, 70, 0], n_tail=1)
+    run_case(librq, wl, lengths=[0, 0, 0], n_tail=0)
+    run_case(librq, wl, lengths=[0, 0, 0], n_tail=3)
+
+
+def test_many_pages_many_ctas(librq):
+    """Enough pages that every CTA of the persistent grid spans segment borders."""
+    wl = synth.Workload(name="long", batch=2, kv_heads=4, q_heads=8, context=3001, sigma=(0.3, 0.2, 0.1),
+                        outlier_p=0.01, seed=34)
+    run_case(librq, wl, lengths=[3001, 1777], loops=[0, 3])
+
+
+def test_softmax_scale_parameter(librq):
+    wl = synth.Workload(name="scale", batch=1, kv_heads=2, q_heads=2, context=90, seed=35)
+    run_case(librq, wl, scale=0.3, loops=[0, 3])
+
+
+def test_ctx_len_beyond_capacity_is_clamped_and_flagged(librq):
+    rq = librq
+    wl = synth.Workload(name="clamp", batch=2, kv_heads=1, q_heads=1, context=64, n_tail=0, seed=36)
+    inp = synth.make_inputs(wl, "cpu")
+    cfgd = synth.cache_config_dict(wl)  # capacity 64
+    cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    ctx = torch.tensor([64, 1000], dtype=torch.int32, device="cuda")
+    out = cache.decode_attention(0, inp["q"][0].cuda(), ctx)
+    assert cache.get_error() & rq.FLAG_CTX_LEN
+    enc = oracle_encode(inp, cfgd)
+    want = O.decode_attention_f64(enc, 0, to_np32(inp["q"][0]), np.array([64, 64]))
+    assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
+
+
+@pytest.mark.parametrize("G,lens", [(1, [200, 1, 64]), (4, [129, 0, 300])])
+def test_bf16_cache_baseline(librq, G, lens):
+    rq = librq
+    wl = synth.Workload(name="bf16", batch=3, kv_heads=2, q_heads=2 * G, context=300, seed=37, n_tail=1)
+    inp = synth.make_inputs(wl, "cpu")
+    ctx = torch.tensor(lens, dtype=torch.int32)
+    for loop in (0, 3):
+        # strided view: the cache tensor has extra capacity and a head-major layout
+        big = torch.zeros((wl.batch, wl.kv_heads, 320, 128), dtype=torch.bfloat16)
+        big[:, :, :300] = inp["k"][loop]
+        bigv = torch.zeros_like(big)
+        bigv[:, :, :300] = inp["v"][loop]
+        out = rq.bf16_decode_attention(big.cuda(), bigv.cuda(), inp["q"][loop].cuda(), ctx.cuda(),
+                                       inp["k_tail"][loop].cuda(), inp["v_tail"][loop].cuda())
+        want = O.attention_f64(to_np32(inp["q"][loop]), to_np32(inp["k"][loop]), to_np32(inp["v"][loop]),
+                               ctx.numpy(), to_np32(inp["k_tail"][loop]), to_np32(inp["v_tail"][loop]))
+        assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL

@@ -1,0 +1,129 @@
+"""GPU encode vs the oracle: packed codes, fp16 scales/offsets and alphas must
+match bit for bit (codes may differ only where the oracle flags a rounding
+near-tie); reconstruction within 1e-3 relative to the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.rq_oracle as O
+from looped_transformer_decode_rq_b200 import synth
+from tests.helpers import (RECON_TOL, compare_encoded, oracle_encode, read_planes, rel_err_rows,
+                           to_np32)
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    synth.tiny(),
+    synth.Workload(name="mixed_modes", batch=2, kv_heads=3, q_heads=3, context=33,
+                   bits=(2, 4, 2, 16), group=(16, 32, 32, 32), rotate=(1, 1, 0, 0),
+                   alpha_mode=(0, 1, 2, 0), sigma=(0.3, 0.2, 0.1), outlier_p=0.05, seed=5),
+    synth.Workload(name="int4_anchor", batch=2, kv_heads=2, q_heads=2, context=65,
+                   bits=(2, 2, 4, 4), group=(32, 16, 32, 32), rotate=(1, 1, 1, 0),
+                   sigma=(0.3, 0.2, 0.1), outlier_p=0.02, seed=6),
+    synth.Workload(name="two_loops", num_loops=2, batch=1, kv_heads=1, q_heads=1, context=1,
+                   bits=(4, 16), group=(32, 32), rotate=(1, 0), alpha_mode=(0, 0), sigma=(0.2,), seed=7),
+    synth.Workload(name="eight_loops", num_loops=8, batch=1, kv_heads=2, q_heads=2, context=17,
+                   bits=(2, 2, 2, 2, 2, 2, 2, 4), group=(16,) * 7 + (32,), rotate=(1,) * 7 + (0,),
+                   alpha_mode=(0,) * 8, sigma=(0.3, 0.25, 0.2, 0.15, 0.1, 0.1, 0.05), seed=8),
+]
+
+
+def _cache(wl, rq):
+    return rq.Cache(rq.config_from_dict(synth.cache_config_dict(wl)), device="cuda")
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
+def test_encode_bit_exact(librq, wl):
+    rq = librq
+    inp = synth.make_inputs(wl, "cpu")
+    cache = _cache(wl, rq)
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    assert cache.get_error() == 0
+    planes = read_planes(cache, wl.context)
+    enc = oracle_encode(inp, synth.cache_config_dict(wl))
+    assert not enc.error
+    stats = compare_encoded(planes, enc)
+    assert stats["near_tie_diff"] <= stats["near_tie"]
+
+
+@pytest.mark.parametrize("wl", CASES, ids=lambda w: w.name)
+def test_reconstruct_within_tolerance(librq, wl):
+    rq = librq
+    inp = synth.make_inputs(wl, "cpu")
+    cache = _cache(wl, rq)
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    enc = oracle_encode(inp, synth.cache_config_dict(wl))
+    for loop in range(wl.num_loops):
+        kg, vg = cache.reconstruct(loop, 0, wl.context)
+        ko, vo = O.reconstruct_f64(enc, loop)
+        for got, want in ((kg, ko), (vg, vo)):
+            err = rel_err_rows(got.cpu().numpy(), want)
+            assert err.max() <= RECON_TOL, (loop, float(err.max()))
+
+
+def test_append_with_device_positions_matches_prefill(librq):
+    rq = librq
+    wl = synth.Workload(name="append", batch=3, kv_heads=2, q_heads=2, context=70, bits=(2, 2, 4, 4),
+                        sigma=(0.3, 0.2, 0.1), seed=9)
+    inp = synth.make_inputs(wl, "cpu")
+    k, v = inp["k"].cuda(), inp["v"].cuda()
+    cache = _cache(wl, rq)
+    T = wl.context
+    cache.encode(k[:, :, :, :T - 5].contiguous(), v[:, :, :, :T - 5].contiguous(), start_pos=0)
+    cache.encode(k[:, :, :, T - 5:T - 3], v[:, :, :, T - 5:T - 3], start_pos=T - 5)  # strided views
+    for i in range(T - 3, T):
+        pos = torch.full((wl.batch,), i, dtype=torch.int32, device="cuda")
+        cache.encode(k[:, :, :, i:i + 1], v[:, :, :, i:i + 1], positions=pos)
+    assert cache.get_error() == 0
+    compare_encoded(read_planes(cache, T), oracle_encode(inp, synth.cache_config_dict(wl)))
+
+
+def test_ragged_append_positions(librq):
+    """Each sequence appends at its own position."""
+    rq = librq
+    wl = synth.Workload(name="ragged_append", batch=3, kv_heads=1, q_heads=1, context=40, seed=10)
+    inp = synth.make_inputs(wl, "cpu")
+    k, v = inp["k"].cuda(), inp["v"].cuda()
+    cache = _cache(wl, rq)
+    cache.encode(k, v)
+    before = read_planes(cache, wl.context)
+    # overwrite position p_b of sequence b with token j=5's data
+    pos = torch.tensor([3, 17, 39], dtype=torch.int32, device="cuda")
+    cache.encode(k[:, :, :, 5:6], v[:, :, :, 5:6], positions=pos)
+    after = read_planes(cache, wl.context)
+    for b, p in enumerate([3, 17, 39]):
+        for l in range(wl.num_loops - 1):
+            codes_after = after["loops"][l]["k"][0][b, 0, p]
+            codes_src = before["loops"][l]["k"][0][b, 0, 5]
+            assert np.array_equal(codes_after, codes_src)
+        untouched = [t for t in range(wl.context) if t != p]
+        assert np.array_equal(after["loops"][0]["k"][0][b, 0, untouched], before["loops"][0]["k"][0][b, 0, untouched])
+
+
+def test_capacity_errors(librq):
+    rq = librq
+    wl = synth.Workload(name="cap", batch=1, kv_heads=1, q_heads=1, context=8, n_tail=0, seed=11)
+    inp = synth.make_inputs(wl, "cpu")
+    cache = _cache(wl, rq)  # capacity 8
+    k, v = inp["k"].cuda(), inp["v"].cuda()
+    with pytest.raises(rq.RQError) as e:
+        cache.encode(k, v, start_pos=1)
+    assert e.value.status == rq.ERR_CAPACITY
+    pos = torch.tensor([5], dtype=torch.int32, device="cuda")
+    cache.encode(k, v, positions=pos)  # tokens 3..7 would land past capacity: dropped, flagged
+    assert cache.get_error() & rq.FLAG_POSITION
+    assert cache.get_error() == 0  # reading clears
+
+
+def test_non_finite_input_sets_device_flag(librq):
+    rq = librq
+    wl = synth.Workload(name="nan", batch=1, kv_heads=1, q_heads=1, context=4, seed=12)
+    inp = synth.make_inputs(wl, "cpu")
+    k = inp["k"].clone()
+    k[1, 0, 0, 2, 7] = float("nan")
+    cache = _cache(wl, rq)
+    cache.encode(k.cuda(), inp["v"].cuda())
+    assert cache.get_error() & rq.FLAG_BAD_INPUT
+    k[1, 0, 0, 2, 7] = 1e5  # beyond the fp16 range of the metadata
+    cache.encode(k.cuda(), inp["v"].cuda())
+    assert cache.get_error() & rq.FLAG_BAD_INPUT
