@@ -17,13 +17,17 @@
 //     cut into num_ctas contiguous ranges of equal length, so ragged batches
 //     balance to within one page; a CTA emits one partial (m, l, acc) per
 //     (b, kv-head) segment it touches;
-//   * warp 8 is a producer: one lane streams pages into a ring of shared
-//     memory stages with the Tensor Memory Accelerator -- tiled tensor copies
-//     with the 128-byte swizzle for bf16 reference tiles, bulk copies for
-//     code, metadata and alpha records -- completing on mbarriers;
-//   * warps 0-7 consume each page in three phases: scores (4G threads per
-//     token, warp-shuffle reduction), softmax weights (one thread per
-//     (token, head)), value accumulation (16 threads per token row);
+//   * warp 8 is the producer: one lane streams pages into a ring of shared
+//     memory stages through the Tensor Memory Accelerator -- tiled tensor
+//     copies with the 128-byte swizzle for bf16 reference tiles, bulk copies
+//     for code, metadata and alpha records -- completing on mbarriers;
+//   * warps 0-7 form two groups of four that take alternate pages ("ping-
+//     pong"), each with its own online softmax and group-local barriers, so
+//     one group's barrier and reduction latency overlaps the other's math.
+//     Within a group a page is processed in two phases: scores (4G lanes per
+//     token, shuffle reduction) and values (16 lanes per token row, 8 dims per
+//     lane, softmax weights recomputed per lane).  The groups merge once per
+//     segment;
 //   * packed codes become floats with one LOP3 each (1 + c*2^(p-23)), the
 //     2^(p-23) factor being folded into the query once per segment and into
 //     the accumulators once per flush; fp32 pairs use FFMA2.
@@ -36,25 +40,49 @@
 namespace rq {
 namespace {
 
-constexpr int kTT = kPage;   // tokens per page / tile
-constexpr int kNCW = 8;      // consumer warps
+constexpr int kTT = kPage;     // tokens per page / stage
+constexpr int kNCW = 8;        // consumer warps
+constexpr int kGW = 4;         // warps per consumer group
+constexpr int kGT = kGW * 32;  // threads per consumer group
 constexpr int kNCT = kNCW * 32;
-constexpr int kNT = kNCT + 32;
-constexpr int kConsumerBar = 1;
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kNT = kNCT + 32; // + producer warp
+constexpr int kConsumerBar = 1;  // all consumers (256 threads)
+constexpr int kGroupBar0 = 2;    // group g uses kGroupBar0 + g (128 threads)
+constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
+// 2^x on the special-function unit (inputs are <= 0 here: softmax weights and
+// their rescale factors)
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// max over the warp with one integer reduction on an order-preserving key
+__device__ __forceinline__ float warp_max(float v) {
+  int i = __float_as_int(v);
+  i ^= (i >> 31) & 0x7fffffff;
+  i = __reduce_max_sync(kFull, i);
+  i ^= (i >> 31) & 0x7fffffff;
+  return __int_as_float(i);
+}
+
 template <int REF, int RB, int RG, int G>
 struct Cfg {
-  static constexpr int TPT = 4 * G;       // phase-1 threads per token
-  static constexpr int D1 = 32 / G;       // phase-1 dims per thread
-  static constexpr int TOK_PASS = kNCT / TPT;
+  // phase 1 (scores): 4G lanes per token, D1 = 32/G dims per lane
+  static constexpr int TPT = 4 * G;
+  static constexpr int D1 = 32 / G;
+  static constexpr int EB = D1 >= 8 ? 8 : D1;   // elements per accumulation block
+  static constexpr int NB = D1 / EB;
+  static constexpr int TOK_PASS = kGT / TPT;    // tokens per pass of a group
   static constexpr int PASSES = kTT / TOK_PASS;
-  static constexpr int D2 = (G >= 8) ? 4 : 8;  // phase-2 dims per thread
-  static constexpr int TPR2 = kD / D2;          // phase-2 threads per token row
-  static constexpr int SLICES = kNCT / TPR2;
-  static constexpr int TOK2 = kTT / SLICES;     // tokens per phase-2 thread per tile
+  // phase 2 (values)
+  static constexpr int D2 = (G >= 8) ? 4 : 8;   // dims per lane
+  static constexpr int TPR2 = kD / D2;          // lanes per token row
+  static constexpr int SLICES = kGT / TPR2;
+  static constexpr int TOK2 = kTT / SLICES;     // tokens per lane per page
   // per-record bytes
   static constexpr int REF_REC = REF == kRefBf16 ? 256 : (REF == kRefInt4 ? 64 : 0);
   static constexpr int REFM_REC = REF == kRefInt4 ? 16 : 0;
@@ -76,26 +104,26 @@ struct Cfg {
   static constexpr int STAGE_BYTES = O_AL + al(kTT * AL_REC);
   static constexpr int TX_BYTES = kTT * (2 * REF_REC + 2 * REFM_REC + 2 * CB + 2 * MB + AL_REC);
   // non-stage shared memory
-  static constexpr int O_S = 0;                      // scores   [G][kTT]
-  static constexpr int O_P = O_S + 4 * G * kTT;      // weights  [G][kTT]  (p)
-  static constexpr int O_PA = O_P + 4 * G * kTT;     // weights  [G][kTT]  (p * alpha_V)
-  static constexpr int O_WM = O_PA + 4 * G * kTT;    // warp max [G][kNCW]
-  static constexpr int O_ACC = O_WM + 4 * G * kNCW;  // [G][256]
-  static constexpr int O_L = O_ACC + 4 * G * 2 * kD; // [G]
-  static constexpr int O_QS = O_L + 4 * 8;           // [G][128]
-  static constexpr int O_QT = O_QS + 4 * G * kD;     // [G][128]
-  static constexpr int O_PRE = O_QT + 4 * G * kD;    // [RQ_MAX_BATCH + 1]
+  static constexpr int O_S = 0;                           // scores [2 groups][2 parity][G][kTT]
+  static constexpr int O_WM = O_S + 4 * 4 * G * kTT;      // warp maxima [2][2][G][kGW]
+  static constexpr int O_ACC = O_WM + 4 * 4 * G * kGW;    // [G][256]
+  static constexpr int O_L = O_ACC + 4 * G * 2 * kD;      // [G] (padded to 8)
+  static constexpr int O_MG = O_L + 4 * 8;                // [2][G] (padded to 16)
+  static constexpr int O_QS = O_MG + 4 * 16;              // [G][128]
+  static constexpr int O_QT = O_QS + 4 * G * kD;          // [G][128]
+  static constexpr int O_PRE = O_QT + 4 * G * kD;         // [RQ_MAX_BATCH + 1]
   static constexpr int O_NT = O_PRE + 4 * (RQ_MAX_BATCH + 1);
   static constexpr int O_MISC = O_NT + 4 * RQ_MAX_BATCH;  // abort flag
   static constexpr int O_BAR = (O_MISC + 16 + 7) & ~7;
   static constexpr int MISC_BYTES = O_BAR + 16 * 8;
   static constexpr int kSmemLimit = 227 * 1024;
   static constexpr int STAGES_MAX = (kSmemLimit - 1024 - MISC_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_MAX >= 4 ? 4 : STAGES_MAX;
+  // an even number of stages keeps each stage with one group
+  static constexpr int STAGES = STAGES_MAX >= 4 ? 4 : 2;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
-  static_assert(STAGES >= 2, "stage ring does not fit in shared memory");
-  static_assert(PASSES * TOK_PASS == kTT, "phase-1 mapping");
-  static_assert(TOK2 * SLICES == kTT, "phase-2 mapping");
+  static_assert(STAGES_MAX >= 2, "stage ring does not fit in shared memory");
+  static_assert(PASSES * TOK_PASS == kTT && TOK2 * SLICES == kTT, "lane mapping");
+  static_assert((O_ACC % 16) == 0 && (O_QS % 16) == 0 && (O_WM % 16) == 0, "alignment");
 };
 
 // ---------------------------------------------------------------------------
@@ -164,22 +192,49 @@ __device__ __forceinline__ float2 f2sub1(float2 f) { return __fadd2_rn(f, make_f
 // split kernel
 // ---------------------------------------------------------------------------
 template <int REF, int RB, int RG, int G>
+__device__ __forceinline__ void issue_page(const DecodeParams& P, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                           uint8_t* st, uint32_t full, const PageIter& it, int Hkv) {
+  using C = Cfg<REF, RB, RG, G>;
+  mbar_arrive_expect_tx(full, C::TX_BYTES);
+  const int t0 = it.page * kTT;
+  const int64_t rec0 = static_cast<int64_t>(it.b * Hkv + it.h) * P.plane_tokens + t0;
+  if constexpr (REF == kRefBf16) {
+    tma_load_4d(smem_u32(st + C::O_REFK), tmK, 0, t0, it.h, it.b, full);
+    tma_load_4d(smem_u32(st + C::O_REFK + kTT * 128), tmK, 64, t0, it.h, it.b, full);
+    tma_load_4d(smem_u32(st + C::O_REFV), tmV, 0, t0, it.h, it.b, full);
+    tma_load_4d(smem_u32(st + C::O_REFV + kTT * 128), tmV, 64, t0, it.h, it.b, full);
+  } else if constexpr (REF == kRefInt4) {
+    bulk_g2s(smem_u32(st + C::O_REFK), P.ref_codes[0] + rec0 * 64, kTT * 64, full);
+    bulk_g2s(smem_u32(st + C::O_REFV), P.ref_codes[1] + rec0 * 64, kTT * 64, full);
+    bulk_g2s(smem_u32(st + C::O_REFMK), P.ref_meta[0] + rec0 * 16, kTT * 16, full);
+    bulk_g2s(smem_u32(st + C::O_REFMV), P.ref_meta[1] + rec0 * 16, kTT * 16, full);
+  }
+  if constexpr (RB != 0) {
+    bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0] + rec0 * C::CB, kTT * C::CB, full);
+    bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[1] + rec0 * C::CB, kTT * C::CB, full);
+    bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0] + rec0 * C::MB, kTT * C::MB, full);
+    bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[1] + rec0 * C::MB, kTT * C::MB, full);
+  }
+  if constexpr (C::HAS_ALPHA) bulk_g2s(smem_u32(st + C::O_AL), P.alpha + rec0 * 4, kTT * 4, full);
+}
+
+template <int REF, int RB, int RG, int G>
 __global__ void __launch_bounds__(kNT, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams P,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV) {
   using C = Cfg<REF, RB, RG, G>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  // align by offsetting the shared array itself so that every access below
+  // stays a shared-memory access
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = base;
   uint8_t* misc = base + C::STAGES * C::STAGE_BYTES;
   float* sS = reinterpret_cast<float*>(misc + C::O_S);
-  float* sP = reinterpret_cast<float*>(misc + C::O_P);
-  float* sPA = reinterpret_cast<float*>(misc + C::O_PA);
   float* sWM = reinterpret_cast<float*>(misc + C::O_WM);
   float* sACC = reinterpret_cast<float*>(misc + C::O_ACC);
   float* sL = reinterpret_cast<float*>(misc + C::O_L);
+  float* sMG = reinterpret_cast<float*>(misc + C::O_MG);
   float* sQS = reinterpret_cast<float*>(misc + C::O_QS);
   float* sQT = reinterpret_cast<float*>(misc + C::O_QT);
   int* sPre = reinterpret_cast<int*>(misc + C::O_PRE);
@@ -192,7 +247,7 @@ __global__ void __launch_bounds__(kNT, 1)
   const int warp = tid >> 5;
   const int B = P.B, Hkv = P.Hkv;
 
-  // ---- page counts and prefix over sequences
+  // ---- page counts and their prefix over sequences
   for (int b = tid; b < B; b += kNT) {
     int len = P.ctx_len[b];
     if (len < 0 || len > P.capacity) {
@@ -213,18 +268,18 @@ __global__ void __launch_bounds__(kNT, 1)
       int x = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        const int y = __shfl_up_sync(kFull, x, o);
         if (lane >= o) x += y;
       }
       if (b < B) sPre[b] = carry + x - v;
-      carry += __shfl_sync(0xffffffffu, x, 31);
+      carry += __shfl_sync(kFull, x, 31);
     }
     if (lane == 0) sPre[B] = carry;
   }
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&bars[s]), 1);                // full
-      mbar_init(smem_u32(&bars[C::STAGES + s]), kNCW);  // empty
+      mbar_init(smem_u32(&bars[s]), 1);               // full: the producer's expect_tx
+      mbar_init(smem_u32(&bars[C::STAGES + s]), kGW);  // empty: the 4 warps of the page's group
     }
     fence_barrier_init();
   }
@@ -249,38 +304,13 @@ __global__ void __launch_bounds__(kNT, 1)
       int k = 0;
       for (; k < n_pages; ++k) {
         const int s = k % C::STAGES;
-        const uint32_t full = smem_u32(&bars[s]);
-        const uint32_t empty = smem_u32(&bars[C::STAGES + s]);
-        if (!mbar_wait_bounded(empty, ((k / C::STAGES) & 1) ^ 1)) {
+        if (!mbar_wait_bounded(smem_u32(&bars[C::STAGES + s]), ((k / C::STAGES) & 1) ^ 1)) {
           set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
           *sAbort = 1;
           break;
         }
         if (*sAbort) break;
-        mbar_arrive_expect_tx(full, C::TX_BYTES);
-        uint8_t* st = stages + s * C::STAGE_BYTES;
-        const int t0 = it.page * kTT;
-        const int64_t rec0 = static_cast<int64_t>(it.b * Hkv + it.h) * P.plane_tokens + t0;
-        if constexpr (REF == kRefBf16) {
-          tma_load_4d(smem_u32(st + C::O_REFK), &tmK, 0, t0, it.h, it.b, full);
-          tma_load_4d(smem_u32(st + C::O_REFK + kTT * 128), &tmK, 64, t0, it.h, it.b, full);
-          tma_load_4d(smem_u32(st + C::O_REFV), &tmV, 0, t0, it.h, it.b, full);
-          tma_load_4d(smem_u32(st + C::O_REFV + kTT * 128), &tmV, 64, t0, it.h, it.b, full);
-        } else if constexpr (REF == kRefInt4) {
-          bulk_g2s(smem_u32(st + C::O_REFK), P.ref_codes[0] + rec0 * 64, kTT * 64, full);
-          bulk_g2s(smem_u32(st + C::O_REFV), P.ref_codes[1] + rec0 * 64, kTT * 64, full);
-          bulk_g2s(smem_u32(st + C::O_REFMK), P.ref_meta[0] + rec0 * 16, kTT * 16, full);
-          bulk_g2s(smem_u32(st + C::O_REFMV), P.ref_meta[1] + rec0 * 16, kTT * 16, full);
-        }
-        if constexpr (RB != 0) {
-          bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0] + rec0 * C::CB, kTT * C::CB, full);
-          bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[1] + rec0 * C::CB, kTT * C::CB, full);
-          bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0] + rec0 * C::MB, kTT * C::MB, full);
-          bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[1] + rec0 * C::MB, kTT * C::MB, full);
-        }
-        if constexpr (C::HAS_ALPHA) {
-          bulk_g2s(smem_u32(st + C::O_AL), P.alpha + rec0 * 4, kTT * 4, full);
-        }
+        issue_page<REF, RB, RG, G>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it, Hkv);
         it.next(sNt, B, Hkv);
       }
       // Drain: no copy this CTA issued may still be landing when it exits.
@@ -294,37 +324,42 @@ __global__ void __launch_bounds__(kNT, 1)
     return;
   }
 
-  // ========================= consumer warps =========================
-  // phase-1 mapping: token (within pass) and dim-slice index j
+  // ========================= consumer groups =========================
+  const int grp = warp / kGW;        // pages k with k % 2 == grp
+  const int gw = warp % kGW;         // warp within the group
+  const int gtid = tid % kGT;        // thread within the group
+  // phase-1 mapping: token within a pass and dim slice.  For G <= 2 the lanes
+  // of one shared-memory phase read rows whose swizzle phases differ, so the
+  // 16-byte loads of the bf16 reference never share a bank.
   int tok1, j1;
   if constexpr (G <= 2) {
     const int jj = lane & (2 * G - 1);
     const int tsub = (lane >> (G == 1 ? 1 : 2)) & ((4 / G) - 1);
     const int box = (lane >> 3) & 1;
     const int thi = lane >> 4;
-    tok1 = warp * (8 / G) + thi * (4 / G) + tsub;
+    tok1 = gw * (8 / G) + thi * (4 / G) + tsub;
     j1 = box * (2 * G) + jj;
   } else {
-    tok1 = warp * (8 / G) + lane / C::TPT;
+    tok1 = gw * (8 / G) + lane / C::TPT;
     j1 = lane % C::TPT;
   }
   const int d1 = C::D1 * j1;
-  // phase-2 mapping
-  const int slice = tid / C::TPR2;
-  const int j2 = tid % C::TPR2;
+  const int slice = gtid / C::TPR2;  // phase-2 mapping
+  const int j2 = gtid % C::TPR2;
   const int d2 = C::D2 * j2;
+  float* gS = sS + grp * 2 * G * kTT;
+  float* gWM = sWM + grp * 2 * G * kGW;
 
   PageIter it;
   it.seek(x0, sPre, sNt, B, Hkv);
   int k = 0;
-  bool aborted = false;
   while (k < n_pages) {
     const int b = it.b, h = it.h;
     const int seg_pages = min(sNt[b] - it.page, n_pages - k);
     int len_b = P.ctx_len[b];
     len_b = len_b < 0 ? 0 : (len_b > P.capacity ? P.capacity : len_b);
 
-    // ---- segment set-up: query (and its rotation) for the G heads of (b, h)
+    // ---- segment set-up: the G queries of (b, h) and their rotation
     if (warp < G) {
       const int qh = h * G + warp;
       const uint2 raw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hkv * G + qh) * kD + 4 * lane);
@@ -332,14 +367,14 @@ __global__ void __launch_bounds__(kNT, 1)
       float x[4] = {a01.x, a01.y, a23.x, a23.y};
       *reinterpret_cast<float4*>(&sQS[warp * kD + 4 * lane]) = make_float4(x[0], x[1], x[2], x[3]);
       if (RB != 0 && P.rotate) {
-        float t0 = x[0] + x[1], t1 = x[0] - x[1], t2 = x[2] + x[3], t3 = x[2] - x[3];
+        const float t0 = x[0] + x[1], t1 = x[0] - x[1], t2 = x[2] + x[3], t3 = x[2] - x[3];
         x[0] = t0 + t2; x[2] = t0 - t2; x[1] = t1 + t3; x[3] = t1 - t3;
 #pragma unroll
         for (int m = 1; m < 32; m <<= 1) {
           const bool up = (lane & m) != 0;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float o = __shfl_xor_sync(0xffffffffu, x[e], m);
+            const float o = __shfl_xor_sync(kFull, x[e], m);
             x[e] = up ? (o - x[e]) : (x[e] + o);
           }
         }
@@ -351,7 +386,8 @@ __global__ void __launch_bounds__(kNT, 1)
     }
     named_bar_sync(kConsumerBar, kNCT);
 
-    // phase-1 registers: reference-side and residual-side query slices
+    // phase-1 registers: reference- and residual-side query slices; the
+    // residual side (and an INT4 reference) pre-multiplied by 2^(23 - p_e)
     float2 qref[G][C::D1 / 2];
     float2 qres[G][C::D1 / 2];
     constexpr int NG1 = RB ? ((C::D1 >= RG) ? C::D1 / RG : 1) : 1;
@@ -372,18 +408,18 @@ __global__ void __launch_bounds__(kNT, 1)
         }
         qref[gi][e / 2] = make_float2(r0, r1);
         if constexpr (RB != 0) {
-          float t0 = sQT[gi * kD + d1 + e], t1 = sQT[gi * kD + d1 + e + 1];
+          const float t0 = sQT[gi * kD + d1 + e], t1 = sQT[gi * kD + d1 + e + 1];
           qsum_res[gi][(C::D1 >= RG) ? e / RG : 0] += t0 + t1;
-          qres[gi][e / 2] = make_float2(t0 * pow2i(23 - code_pos<RB>(e)),
-                                        t1 * pow2i(23 - code_pos<RB>(e + 1)));
+          qres[gi][e / 2] = make_float2(t0 * pow2i(23 - code_pos<RB>(e)), t1 * pow2i(23 - code_pos<RB>(e + 1)));
+        } else {
+          qres[gi][e / 2] = make_float2(0.f, 0.f);
         }
       }
     }
 
-    // running softmax state and accumulators
+    // group-local running softmax state and per-lane accumulators
     float m_run[G], l_thr[G];
-    float2 acc_ref[G][C::D2 / 2];
-    float2 acc_res[G][C::D2 / 2];
+    float2 acc_ref[G][C::D2 / 2], acc_res[G][C::D2 / 2];
     float z_ref[G], z_res[G];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
@@ -392,26 +428,28 @@ __global__ void __launch_bounds__(kNT, 1)
       z_ref[gi] = 0.f;
       z_res[gi] = 0.f;
 #pragma unroll
-      for (int e = 0; e < C::D2 / 2; ++e) {
-        acc_ref[gi][e] = make_float2(0.f, 0.f);
-        acc_res[gi][e] = make_float2(0.f, 0.f);
-      }
+      for (int e = 0; e < C::D2 / 2; ++e) acc_ref[gi][e] = acc_res[gi][e] = make_float2(0.f, 0.f);
     }
 
     for (int sp = 0; sp < seg_pages; ++sp, ++k) {
+      if ((k & 1) != grp) {  // the other group's page
+        it.next(sNt, B, Hkv);
+        continue;
+      }
       const int s = k % C::STAGES;
       const uint8_t* st = stages + s * C::STAGE_BYTES;
       if (!*sAbort) {
         if (!mbar_wait_bounded(smem_u32(&bars[s]), (k / C::STAGES) & 1)) {
           set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
           *sAbort = 1;
-          aborted = true;
         }
       }
-      const int t0 = it.page * kTT;
-      const int n_valid = min(kTT, len_b - t0);
+      const int n_valid = min(kTT, len_b - it.page * kTT);
+      const int par = (k >> 1) & 1;
+      float* pS = gS + par * G * kTT;
+      float* pWM = gWM + par * G * kGW;
 
-      // ---------------- phase 1: scores
+      // ---------------- phase 1: scores of the page's 64 tokens
       float wmax[G];
 #pragma unroll
       for (int gi = 0; gi < G; ++gi) wmax[gi] = -INFINITY;
@@ -421,16 +459,16 @@ __global__ void __launch_bounds__(kNT, 1)
         float part[G];
 #pragma unroll
         for (int gi = 0; gi < G; ++gi) part[gi] = 0.f;
-        // reference side
-        float refdot[G];
         if constexpr (REF == kRefBf16) {
-          float2 acc2[G];
+          float2 acc2[G][C::NB];
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi) acc2[gi] = make_float2(0.f, 0.f);
+          for (int gi = 0; gi < G; ++gi)
+#pragma unroll
+            for (int c = 0; c < C::NB; ++c) acc2[gi][c] = make_float2(0.f, 0.f);
           const uint8_t* rowK = st + C::O_REFK + (d1 >> 6) * (kTT * 128) + t * 128;
           if constexpr (C::D1 >= 8) {
 #pragma unroll
-            for (int c = 0; c < C::D1 / 8; ++c) {
+            for (int c = 0; c < C::NB; ++c) {
               const int chunk = ((d1 & 63) >> 3) + c;
               const uint4 v = *reinterpret_cast<const uint4*>(rowK + ((chunk ^ (t & 7)) << 4));
               const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
@@ -438,132 +476,117 @@ __global__ void __launch_bounds__(kNT, 1)
               for (int u = 0; u < 4; ++u) {
                 const float2 kv2 = bf16x2_to_f2(w4[u]);
 #pragma unroll
-                for (int gi = 0; gi < G; ++gi) acc2[gi] = __ffma2_rn(qref[gi][c * 4 + u], kv2, acc2[gi]);
+                for (int gi = 0; gi < G; ++gi) acc2[gi][c] = __ffma2_rn(qref[gi][c * 4 + u], kv2, acc2[gi][c]);
               }
             }
           } else {
             const int chunk = (d1 & 63) >> 3;
             const uint2 v = *reinterpret_cast<const uint2*>(rowK + ((chunk ^ (t & 7)) << 4) + ((d1 & 7) << 1));
-            const uint32_t w2[2] = {v.x, v.y};
+            const float2 k01 = bf16x2_to_f2(v.x), k23 = bf16x2_to_f2(v.y);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const float2 kv2 = bf16x2_to_f2(w2[u]);
-#pragma unroll
-              for (int gi = 0; gi < G; ++gi) acc2[gi] = __ffma2_rn(qref[gi][u], kv2, acc2[gi]);
+            for (int gi = 0; gi < G; ++gi) {
+              acc2[gi][0] = __ffma2_rn(qref[gi][0], k01, acc2[gi][0]);
+              acc2[gi][0] = __ffma2_rn(qref[gi][1], k23, acc2[gi][0]);
             }
           }
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi) refdot[gi] = acc2[gi].x + acc2[gi].y;
+          for (int gi = 0; gi < G; ++gi) {
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < C::NB; ++c) sum += acc2[gi][c].x + acc2[gi][c].y;
+            part[gi] = sum;
+          }
         } else if constexpr (REF == kRefInt4) {
           uint32_t cw[(C::D1 / 2 + 3) / 4];
           load_codes<C::D1 / 2>(st + C::O_REFK + t * 64 + (d1 >> 1), cw);
           const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMK + t * 16 + 4 * (d1 >> 5)));
-          float2 acc2[G];
+          float2 acc2[G][C::NB];
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi) acc2[gi] = make_float2(0.f, 0.f);
+          for (int gi = 0; gi < G; ++gi)
+#pragma unroll
+            for (int c = 0; c < C::NB; ++c) acc2[gi][c] = make_float2(0.f, 0.f);
 #pragma unroll
           for (int e = 0; e < C::D1; e += 2) {
             const float2 f = f2sub1(make_float2(code_f<4>(cw, e), code_f<4>(cw, e + 1)));
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) acc2[gi] = __ffma2_rn(qref[gi][e / 2], f, acc2[gi]);
+            for (int gi = 0; gi < G; ++gi) acc2[gi][e / C::EB] = __ffma2_rn(qref[gi][e / 2], f, acc2[gi][e / C::EB]);
           }
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi)
-            refdot[gi] = fmaf(sz.x, acc2[gi].x + acc2[gi].y, sz.y * qsum_ref[gi]);
-        }
-        if constexpr (REF != kRefNone) {
-          float aK = 1.f;
-          if constexpr (C::HAS_ALPHA) aK = __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4));
+          for (int gi = 0; gi < G; ++gi) {
+            float sum = 0.f;
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi) part[gi] = aK * refdot[gi];
+            for (int c = 0; c < C::NB; ++c) sum += acc2[gi][c].x + acc2[gi][c].y;
+            part[gi] = fmaf(sz.x, sum, sz.y * qsum_ref[gi]);
+          }
         }
-        // residual side
+        if constexpr (C::HAS_ALPHA) {
+          const float aK = __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4));
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi) part[gi] *= aK;
+        }
         if constexpr (RB != 0) {
           constexpr int NBYTES = C::D1 * RB / 8;
           uint32_t cw[(NBYTES + 3) / 4];
           load_codes<NBYTES>(st + C::O_RESK + t * C::CB + (d1 * RB >> 3), cw);
+          float2 acc2[G][C::NB];
+#pragma unroll
+          for (int gi = 0; gi < G; ++gi)
+#pragma unroll
+            for (int c = 0; c < C::NB; ++c) acc2[gi][c] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int e = 0; e < C::D1; e += 2) {
+            const float2 f = f2sub1(make_float2(code_f<RB>(cw, e), code_f<RB>(cw, e + 1)));
+#pragma unroll
+            for (int gi = 0; gi < G; ++gi) acc2[gi][e / C::EB] = __ffma2_rn(qres[gi][e / 2], f, acc2[gi][e / C::EB]);
+          }
+          constexpr int BPG = (C::D1 >= RG) ? RG / C::EB : C::NB;  // accumulation blocks per group
 #pragma unroll
           for (int n = 0; n < NG1; ++n) {
-            constexpr int EPG = (C::D1 >= RG) ? RG : C::D1;  // elements of this thread per group
             const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(
                 st + C::O_RESMK + t * C::MB + 4 * (d1 / RG + n)));
-            float2 acc2[G];
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) acc2[gi] = make_float2(0.f, 0.f);
+            for (int gi = 0; gi < G; ++gi) {
+              float sum = 0.f;
 #pragma unroll
-            for (int e = n * EPG; e < (n + 1) * EPG; e += 2) {
-              const float2 f = f2sub1(make_float2(code_f<RB>(cw, e), code_f<RB>(cw, e + 1)));
-#pragma unroll
-              for (int gi = 0; gi < G; ++gi) acc2[gi] = __ffma2_rn(qres[gi][e / 2], f, acc2[gi]);
+              for (int c = n * BPG; c < (n + 1) * BPG; ++c) sum += acc2[gi][c].x + acc2[gi][c].y;
+              part[gi] += fmaf(sz.x, sum, sz.y * qsum_res[gi][n]);
             }
-#pragma unroll
-            for (int gi = 0; gi < G; ++gi)
-              part[gi] += fmaf(sz.x, acc2[gi].x + acc2[gi].y, sz.y * qsum_res[gi][n]);
           }
         }
-        // reduce over the TPT threads of this token
+        // reduce over the TPT lanes of this token
 #pragma unroll
         for (int gi = 0; gi < G; ++gi) {
           float v = part[gi];
           if constexpr (G <= 2) {
 #pragma unroll
-            for (int o = 1; o < 2 * G; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            for (int o = 1; o < 2 * G; o <<= 1) v += __shfl_xor_sync(kFull, v, o);
+            v += __shfl_xor_sync(kFull, v, 8);
           } else {
 #pragma unroll
-            for (int o = 1; o < C::TPT; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            for (int o = 1; o < C::TPT; o <<= 1) v += __shfl_xor_sync(kFull, v, o);
           }
           const float sc = (t < n_valid) ? v * P.scale_log2 : -INFINITY;
           wmax[gi] = fmaxf(wmax[gi], sc);
-          if (j1 == 0) sS[gi * kTT + t] = sc;
+          if (j1 == 0) pS[gi * kTT + t] = sc;
         }
       }
 #pragma unroll
       for (int gi = 0; gi < G; ++gi) {
-        float v = wmax[gi];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-        if (lane == 0) sWM[gi * kNCW + warp] = v;
+        const float v = warp_max(wmax[gi]);
+        if (lane == 0) pWM[gi * kGW + gw] = v;
       }
-      named_bar_sync(kConsumerBar, kNCT);
+      named_bar_sync(kGroupBar0 + grp, kGT);
 
-      // ---------------- phase 1.5: softmax weights
+      // ---------------- softmax bookkeeping (group-uniform values)
       float corr[G];
 #pragma unroll
       for (int gi = 0; gi < G; ++gi) {
-        const float4 a = *reinterpret_cast<const float4*>(&sWM[gi * kNCW]);
-        const float4 c = *reinterpret_cast<const float4*>(&sWM[gi * kNCW + 4]);
-        const float mt = fmaxf(fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)), fmaxf(fmaxf(c.x, c.y), fmaxf(c.z, c.w)));
+        const float4 a = *reinterpret_cast<const float4*>(&pWM[gi * kGW]);
+        const float mt = fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w));
         const float mn = fmaxf(m_run[gi], mt);
-        corr[gi] = exp2f(m_run[gi] - mn);
+        corr[gi] = fast_exp2(m_run[gi] - mn);
         m_run[gi] = mn;
         l_thr[gi] *= corr[gi];
-      }
-#pragma unroll
-      for (int r = 0; r < (G * kTT + kNCT - 1) / kNCT; ++r) {
-        const int idx = tid + r * kNCT;
-        if (idx < G * kTT) {
-          const int t = idx % kTT, gi = idx / kTT;
-          float mg = m_run[0];
-#pragma unroll
-          for (int g2 = 1; g2 < G; ++g2) if (gi == g2) mg = m_run[g2];
-          float p = 0.f, pa = 0.f;
-          if (t < n_valid) {
-            p = exp2f(sS[gi * kTT + t] - mg);
-            pa = p;
-            if constexpr (C::HAS_ALPHA) pa = p * __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4 + 2));
-          }
-          sP[gi * kTT + t] = p;
-          sPA[gi * kTT + t] = pa;
-#pragma unroll
-          for (int g2 = 0; g2 < G; ++g2) if (gi == g2) l_thr[g2] += p;
-        }
-      }
-      named_bar_sync(kConsumerBar, kNCT);
-
-      // ---------------- phase 2: value accumulation
-#pragma unroll
-      for (int gi = 0; gi < G; ++gi) {
         const float2 c2 = make_float2(corr[gi], corr[gi]);
 #pragma unroll
         for (int e = 0; e < C::D2 / 2; ++e) {
@@ -573,15 +596,17 @@ __global__ void __launch_bounds__(kNT, 1)
         z_ref[gi] *= corr[gi];
         z_res[gi] *= corr[gi];
       }
-#pragma unroll
-      for (int i = 0; i < C::TOK2; ++i) {
-        const int t = slice + i * C::SLICES;
-        if (t >= n_valid) break;
+
+      // ---------------- phase 2: values (weights recomputed per lane)
+      auto value_token = [&](int t) {
         float pp[G], pa[G];
+        float aV = 1.f;
+        if constexpr (C::HAS_ALPHA) aV = __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4 + 2));
 #pragma unroll
         for (int gi = 0; gi < G; ++gi) {
-          pp[gi] = sP[gi * kTT + t];
-          pa[gi] = sPA[gi * kTT + t];
+          pp[gi] = fast_exp2(pS[gi * kTT + t] - m_run[gi]);
+          pa[gi] = pp[gi] * aV;
+          if (j2 == 0) l_thr[gi] += pp[gi];
         }
         if constexpr (REF == kRefBf16) {
           const uint8_t* rowV = st + C::O_REFV + (d2 >> 6) * (kTT * 128) + t * 128;
@@ -593,18 +618,15 @@ __global__ void __launch_bounds__(kNT, 1)
             for (int u = 0; u < 4; ++u) {
               const float2 vv = bf16x2_to_f2(w4[u]);
 #pragma unroll
-              for (int gi = 0; gi < G; ++gi)
-                acc_ref[gi][u] = __ffma2_rn(make_float2(pa[gi], pa[gi]), vv, acc_ref[gi][u]);
+              for (int gi = 0; gi < G; ++gi) acc_ref[gi][u] = __ffma2_rn(make_float2(pa[gi], pa[gi]), vv, acc_ref[gi][u]);
             }
           } else {
             const uint2 v = *reinterpret_cast<const uint2*>(rowV + ((chunk ^ (t & 7)) << 4) + ((d2 & 7) << 1));
-            const uint32_t w2[2] = {v.x, v.y};
+            const float2 v01 = bf16x2_to_f2(v.x), v23 = bf16x2_to_f2(v.y);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const float2 vv = bf16x2_to_f2(w2[u]);
-#pragma unroll
-              for (int gi = 0; gi < G; ++gi)
-                acc_ref[gi][u] = __ffma2_rn(make_float2(pa[gi], pa[gi]), vv, acc_ref[gi][u]);
+            for (int gi = 0; gi < G; ++gi) {
+              acc_ref[gi][0] = __ffma2_rn(make_float2(pa[gi], pa[gi]), v01, acc_ref[gi][0]);
+              acc_ref[gi][1] = __ffma2_rn(make_float2(pa[gi], pa[gi]), v23, acc_ref[gi][1]);
             }
           }
         } else if constexpr (REF == kRefInt4) {
@@ -639,28 +661,44 @@ __global__ void __launch_bounds__(kNT, 1)
 #pragma unroll
           for (int gi = 0; gi < G; ++gi) z_res[gi] = fmaf(pp[gi], sz.y, z_res[gi]);
         }
+      };
+      if (n_valid == kTT) {
+#pragma unroll 4
+        for (int i = 0; i < C::TOK2; ++i) value_token(slice + i * C::SLICES);
+      } else {
+        for (int i = 0; i < C::TOK2; ++i) {
+          const int t = slice + i * C::SLICES;
+          if (t < n_valid) value_token(t);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars[C::STAGES + s]));
       it.next(sNt, B, Hkv);
     }
 
-    // ---- flush this (b, h) segment: reduce over slices, write the partial
+    // ---- flush this (b, h) segment: merge the two groups, write one partial
+    if (gtid == 0) {
+#pragma unroll
+      for (int gi = 0; gi < G; ++gi) sMG[grp * G + gi] = m_run[gi];
+    }
+    named_bar_sync(kConsumerBar, kNCT);
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
+      const float M = fmaxf(sMG[gi], sMG[G + gi]);
+      const float f = (m_run[gi] == -INFINITY) ? 0.f : fast_exp2(m_run[gi] - M);
 #pragma unroll
       for (int e = 0; e < C::D2; ++e) {
-        const float2 ar = acc_ref[gi][e / 2];
+        const float2 ar = acc_ref[gi][e >> 1];
         float vr = (e & 1) ? ar.y : ar.x;
         if constexpr (REF == kRefInt4) vr = fmaf(vr, pow2i(23 - code_pos<4>(e)), z_ref[gi]);
-        atomicAdd(&sACC[gi * 2 * kD + d2 + e], vr);
+        if constexpr (REF != kRefNone) atomicAdd(&sACC[gi * 2 * kD + d2 + e], vr * f);
         if constexpr (RB != 0) {
-          const float2 as = acc_res[gi][e / 2];
+          const float2 as = acc_res[gi][e >> 1];
           const float vs = fmaf((e & 1) ? as.y : as.x, pow2i(23 - code_pos<RB>(e)), z_res[gi]);
-          atomicAdd(&sACC[gi * 2 * kD + kD + d2 + e], vs);
+          atomicAdd(&sACC[gi * 2 * kD + kD + d2 + e], vs * f);
         }
       }
-      if (l_thr[gi] != 0.f) atomicAdd(&sL[gi], l_thr[gi]);
+      if (l_thr[gi] != 0.f) atomicAdd(&sL[gi], l_thr[gi] * f);
     }
     named_bar_sync(kConsumerBar, kNCT);
     {
@@ -673,15 +711,12 @@ __global__ void __launch_bounds__(kNT, 1)
         *src = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       if (tid < G) {
-        float mg = m_run[0];
-#pragma unroll
-        for (int g2 = 1; g2 < G; ++g2) if (tid == g2) mg = m_run[g2];
-        reinterpret_cast<float4*>(rec + tid * kPartialFloats)[0] = make_float4(mg, sL[tid], 0.f, 0.f);
+        const float M = fmaxf(sMG[tid], sMG[G + tid]);
+        reinterpret_cast<float4*>(rec + tid * kPartialFloats)[0] = make_float4(M, sL[tid], 0.f, 0.f);
         sL[tid] = 0.f;
       }
     }
   }
-  (void)aborted;
 }
 
 // ---------------------------------------------------------------------------
