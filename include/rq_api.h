@@ -193,6 +193,36 @@ RQ_API rq_status rq_decode_attention(const rq_cache* cache, int32_t loop, const 
                               int32_t n_tail, float softmax_scale, float* out, void* workspace,
                               int64_t workspace_bytes, rq_stream_t stream);
 
+/* Size of the library's static split-K scratch used by
+ * rq_decode_attention_static_scratch (4 MiB). */
+#define RQ_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)
+
+/* rq_decode_attention for callers that cannot allocate device memory.  The
+ * paper has no counterpart of this entry point: it exists for callers that have
+ * no way to provide the decode workspace, such as code hosted in a framework
+ * that owns every device allocation and forbids raw cudaMalloc, or serving
+ * loops that must not allocate while running (cudaMalloc and cudaFree can
+ * synchronise the device).  It computes exactly what rq_decode_attention
+ * computes, with the split-K partials kept in a fixed RQ_STATIC_SCRATCH_BYTES
+ * array in the library's own device memory instead of a caller workspace.
+ *  - It allocates nothing and calls no allocating routine.
+ *  - Limit: rq_decode_workspace_size(cache) must not exceed
+ *    RQ_STATIC_SCRATCH_BYTES (roughly (batch*kv_heads + SMs) * G * 1040 bytes);
+ *    otherwise it returns RQ_ERR_WORKSPACE before enqueuing anything.
+ *  - Set-up: the first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.  Every GPU that loads the library keeps the
+ *    array until the process exits.
+ *  - Sharing: all calls on a device use the same array, which keeps the last
+ *    call's contents (nothing in it needs to start at zero).  Calls whose
+ *    kernels overlap on the GPU -- on different streams, or from different
+ *    host threads -- race on it; serialise them on one stream.
+ * Arguments and errors are those of rq_decode_attention, minus the workspace. */
+RQ_API rq_status rq_decode_attention_static_scratch(const rq_cache* cache, int32_t loop, const void* q,
+                                                    const int32_t* ctx_len, const void* k_tail,
+                                                    const void* v_tail, int32_t n_tail, float softmax_scale,
+                                                    float* out, rq_stream_t stream);
+
 /* Workspace bytes for rq_bf16_decode_attention with these sizes. */
 RQ_API rq_status rq_bf16_decode_workspace_size(int32_t batch, int32_t kv_heads, int32_t q_heads,
                                         int64_t* bytes_out);

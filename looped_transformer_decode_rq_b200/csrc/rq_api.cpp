@@ -118,6 +118,18 @@ int ref_kind_for(const rq_config& c, int loop) {
 
 }  // namespace
 
+namespace rq {
+rq_status set_last_error(rq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_msg = buf;
+  return s;
+}
+}  // namespace rq
+
 extern "C" {
 
 const char* rq_status_string(rq_status s) {

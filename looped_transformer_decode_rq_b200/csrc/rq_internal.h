@@ -88,4 +88,7 @@ cudaError_t launch_decode(const DecodeParams& p, int ref_kind, int res_bits, int
                           const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
 bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G);
 
+// Records the calling thread's rq_last_error_message() text and returns `s`.
+rq_status set_last_error(rq_status s, const char* fmt, ...);
+
 }  // namespace rq

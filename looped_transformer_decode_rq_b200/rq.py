@@ -35,7 +35,8 @@ ALPHA_LS, ALPHA_ONE, ALPHA_ZERO = 0, 1, 2
 EXPORTED = ("rq_cache_layout", "rq_cache_create", "rq_cache_destroy", "rq_cache_info", "rq_encode",
             "rq_decode_workspace_size", "rq_decode_attention", "rq_bf16_decode_workspace_size",
             "rq_bf16_decode_attention", "rq_reconstruct", "rq_get_error", "rq_status_string",
-            "rq_last_error_message")
+            "rq_last_error_message", "rq_decode_attention_static_scratch")
+STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 
 class Config(C.Structure):
@@ -63,6 +64,7 @@ _sig = {
     "rq_encode": (C.c_int, [_vp, _vp, _vp, C.POINTER(_i64), _i32, _vp, _i32, _vp]),
     "rq_decode_workspace_size": (C.c_int, [_vp, C.POINTER(_i64)]),
     "rq_decode_attention": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp]),
+    "rq_decode_attention_static_scratch": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp]),
     "rq_bf16_decode_workspace_size": (C.c_int, [_i32, _i32, _i32, C.POINTER(_i64)]),
     "rq_bf16_decode_attention": (C.c_int, [_i32, _i32, _i32, _vp, _vp, C.POINTER(_i64), _i32, _vp, _vp, _vp,
                                            _vp, _i32, _f32, _vp, _vp, _i64, _vp, _vp]),
@@ -191,6 +193,24 @@ class Cache:
         _check(_lib.rq_decode_attention(self._h, loop, q.data_ptr(), ctx_len.data_ptr(), _ptr(k_tail),
                                         _ptr(v_tail), n_tail, scale, out.data_ptr(), self.workspace.data_ptr(),
                                         self.workspace.numel(), _stream(stream)), "rq_decode_attention")
+        return out
+
+    def decode_attention_static_scratch(self, loop: int, q: torch.Tensor, ctx_len: torch.Tensor,
+                                        k_tail: Optional[torch.Tensor] = None, v_tail: Optional[torch.Tensor] = None,
+                                        softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                                        stream=None) -> torch.Tensor:
+        """decode_attention without a caller workspace: the library keeps the
+        split-K partials in its own fixed 4 MiB device array (for callers that
+        cannot allocate).  Calls that overlap on the GPU race on that array."""
+        cfg = self.cfg
+        assert q.dtype == torch.bfloat16 and q.is_contiguous() and ctx_len.dtype == torch.int32
+        if out is None:
+            out = torch.empty((cfg.batch, cfg.q_heads, HEAD_DIM), dtype=torch.float32, device=q.device)
+        n_tail = 0 if k_tail is None else k_tail.shape[2]
+        scale = softmax_scale if softmax_scale is not None else HEAD_DIM ** -0.5
+        _check(_lib.rq_decode_attention_static_scratch(self._h, loop, q.data_ptr(), ctx_len.data_ptr(),
+                                                       _ptr(k_tail), _ptr(v_tail), n_tail, scale, out.data_ptr(),
+                                                       _stream(stream)), "rq_decode_attention_static_scratch")
         return out
 
     def reconstruct(self, loop: int, t0: int, n: int, stream=None):
