@@ -91,12 +91,19 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank time over all ranks (the job is as slow as its slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(batch_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job decode throughput: every rank decodes its own batch each step."""
+    return batch_per_rank * world / (ms_per_step * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -344,7 +351,7 @@ def run_rq(args, world, rank):
                                for f in ("rq_decode.cu", "rq_common.cuh")])
     achieved = res_bytes / (call_ms * 1e-3) / 1e9
     traffic = read_profile_traffic(kernel_hash)
-    value = B * world / (ms * 1e-3)
+    value = job_tokens_per_s(B, world, ms)
 
     # ---- e2e through the public API with host buffers
     e2e = None
@@ -376,7 +383,7 @@ def run_rq(args, world, rank):
         torch.cuda.synchronize()
         barrier(world)
         ems = max_over_ranks(a.elapsed_time(b2) / args.steps, world)
-        e2e = {"value": round(B * world / (ems * 1e-3), 1), "unit": "tokens/s",
+        e2e = {"value": round(job_tokens_per_s(B, world, ems), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
                "d2h_bytes_per_step": int(hout.numel() * 4)}
 
@@ -403,7 +410,7 @@ def run_rq(args, world, rank):
         torch.cuda.synchronize()
         bms = max_over_ranks(a.elapsed_time(b2) / args.steps, world)
         bf_bytes = L * (tokens_total * Hkv * 512 + B * Hq * 128 * 6 + B * Hkv * n_tail * 512)
-        bf16 = {"tokens_per_s": round(B * world / (bms * 1e-3), 1), "ms_per_step": round(bms, 4),
+        bf16 = {"tokens_per_s": round(job_tokens_per_s(B, world, bms), 1), "ms_per_step": round(bms, 4),
                 "hbm_gbs": round(bf_bytes / (bms * 1e-3) / 1e9, 1),
                 "bytes_per_step": bf_bytes, "rq_speedup": round(bms / ms, 3)}
 

@@ -1,0 +1,75 @@
+"""Parity at the benchmark's full sizes, in the launch configuration bench.py
+times (persistent split over all pages of the whole batch).  The whole batch is
+encoded and decoded on the GPU; sampled (sequence, kv-head) slabs are encoded
+by the oracle and compared bit for bit, and their q-heads' attention outputs
+compared with the float64 oracle over the full context."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.rq_oracle as O
+from looped_transformer_decode_rq_b200 import synth
+from tests.helpers import ATTN_TOL, compare_encoded, rel_err_rows, unpack_alpha, unpack_codes, unpack_meta
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    (synth.ouro_8k(), [(0, 0), (7, 9), (15, 15)]),
+    (synth.mixed_int4_anchor(batch=8), [(0, 3), (7, 15)]),
+    (synth.gqa_long(batch=8), [(0, 0), (5, 7)]),
+]
+
+
+def _slab_planes(cache, b, h, n):
+    """The cache planes of one (b, h) slab, unpacked like tests.helpers.read_planes."""
+    cfg, lay = cache.cfg, cache.layout
+    L = cfg.num_loops
+
+    def grab(off, rec):
+        return cache.plane(off, rec)[b:b + 1, h:h + 1, :n].cpu().numpy()
+
+    out = {"ref": {}, "loops": []}
+    for kv, name in enumerate("kv"):
+        if cfg.bits[L - 1] == 16:
+            out["ref"][name] = grab(lay.ref_offset[kv], 256).view("<u2")
+        else:
+            s, z = unpack_meta(grab(lay.ref_meta_offset[kv], 16))
+            out["ref"][name] = (unpack_codes(grab(lay.ref_offset[kv], 64), 4), s, z)
+    for l in range(L - 1):
+        d = {}
+        for kv, name in enumerate("kv"):
+            s, z = unpack_meta(grab(lay.meta_offset[l][kv], lay.meta_record_bytes[l]))
+            d[name] = (unpack_codes(grab(lay.codes_offset[l][kv], lay.codes_record_bytes[l]), cfg.bits[l]), s, z)
+        d["alpha"] = unpack_alpha(grab(lay.alpha_offset[l], 4))
+        out["loops"].append(d)
+    return out
+
+
+@pytest.mark.parametrize("wl,samples", CASES, ids=lambda x: getattr(x, "name", "samples"))
+def test_full_size_sampled_parity(librq, wl, samples):
+    rq = librq
+    dev = torch.device("cuda")
+    inp = synth.make_inputs(wl, dev)
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
+    cache.encode(inp["k"], inp["v"])
+    ctx = inp["ctx_len"]
+    outs = [cache.decode_attention(l, inp["q"][l], ctx, inp["k_tail"][l], inp["v_tail"][l])
+            for l in range(wl.num_loops)]
+    torch.cuda.synchronize()
+    assert cache.get_error() == 0
+    G = wl.gqa
+    ocfg = O.CacheConfig.from_dict(cfgd)
+    for b, h in samples:
+        n = int(ctx[b])
+        sl = lambda t: t[:, b:b + 1, h:h + 1].float().cpu().numpy()  # noqa: E731
+        K, V = sl(inp["k"])[:, :, :, :n], sl(inp["v"])[:, :, :, :n]
+        enc = O.encode_fp32emu(K, V, ocfg)
+        compare_encoded(_slab_planes(cache, b, h, n), enc)
+        q = inp["q"][:, b:b + 1, h * G:(h + 1) * G].float().cpu().numpy()
+        kt, vt = sl(inp["k_tail"]), sl(inp["v_tail"])
+        for l in range(wl.num_loops):
+            want = O.decode_attention_f64(enc, l, q[l], np.array([n]), kt[l], vt[l])
+            got = outs[l][b:b + 1, h * G:(h + 1) * G].cpu().numpy()
+            err = rel_err_rows(got, want).max()
+            assert err <= ATTN_TOL, (wl.name, b, h, l, float(err))
