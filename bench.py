@@ -46,12 +46,13 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["rq", "reference"], default="rq")
-    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "tiny"], default="ouro8k")
+    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "tiny", "capacity"], default="ouro8k")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the mixed INT4-anchor and GQA side lines")
     return ap.parse_args()
 
 
@@ -273,6 +274,153 @@ def time_oracle(sample, wl, seconds, min_reps=1):
 # the GPU arm
 # ---------------------------------------------------------------------------
 
+def time_steps(step, steps, warmup, world, stream):
+    """Mean device time of one step over `steps` timed steps (after `warmup`),
+    max over ranks."""
+    for _ in range(warmup):
+        step()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(a.elapsed_time(b) / steps, world)
+
+
+def measure_workload(wl, steps, warmup, world, rank):
+    """RQ decode step and bf16-cache step of one workload (side lines of the
+    main result): tokens/s, residual-loop GB/s and the speed-up over bf16."""
+    from looped_transformer_decode_rq_b200 import rq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = wl.with_(seed=wl.seed + 1000 * rank)
+    inp = synth.make_inputs(wl, dev)
+    L, B, Hkv, Hq, T = wl.num_loops, wl.batch, wl.kv_heads, wl.q_heads, wl.context
+    cfgd = synth.cache_config_dict(wl, capacity=T + 1)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
+    cache.encode(inp["k"], inp["v"])
+    ctx = inp["ctx_len"]
+    tokens_total = int(ctx.sum().item())
+    k_new = inp["k_tail"][:, :, :, :1].contiguous()
+    v_new = inp["v_tail"][:, :, :, :1].contiguous()
+    q = inp["q"]
+    outs = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def rq_step():
+        for l in range(L):
+            cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
+        cache.encode(k_new, v_new, positions=ctx)
+
+    ms = time_steps(rq_step, steps, warmup, world, stream)
+    ev = []
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    call_ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    res_bytes = call_bytes(cache.layout, cfgd, 0, tokens_total, B, Hq, Hkv, 1)
+    ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+
+    def bf16_step():
+        for l in range(L):
+            rq.bf16_decode_attention(inp["k"][l], inp["v"][l], q[l], ctx, k_new[l], v_new[l], workspace=ws, out=outs[l])
+
+    bms = time_steps(bf16_step, steps, warmup, world, stream)
+    flags = cache.get_error()
+    out = {"workload": wl.name, "tokens_per_s": round(job_tokens_per_s(B, world, ms), 1),
+           "ms_per_step": round(ms, 4), "residual_loop_gbs": round(res_bytes / (call_ms * 1e-3) / 1e9, 1),
+           "residual_loop_bytes": res_bytes, "bf16_tokens_per_s": round(job_tokens_per_s(B, world, bms), 1),
+           "rq_speedup_vs_bf16": round(bms / ms, 3), "device_flags": flags}
+    del cache, inp, outs, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_capacity(args, world, rank):
+    """24-layer, 4-loop model at 8192 context: the largest batch whose caches
+    fit in HBM for a bf16 cache and for ResidualQuant caches (bf16 anchor and
+    INT4 anchor), and decode tokens/s of the full 24-layer attention step at
+    that batch.  One synthetic sequence is encoded into every (layer, sequence)
+    slot, each with its own cache memory: the timing does not depend on the
+    values."""
+    from looped_transformer_decode_rq_b200 import rq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layers, T = 24, 8192
+    base = synth.capacity_24layer(batch=1, context=T)
+    L, Hkv, Hq = base.num_loops, base.kv_heads, base.q_heads
+    steps, warmup = max(2, min(args.steps, 5)), 3
+    stream = torch.cuda.current_stream()
+    one = synth.make_inputs(base.with_(batch=1, n_tail=1), dev)  # [L, 1, Hkv, T, 128]
+    free, _ = torch.cuda.mem_get_info()
+    budget = int(free * 0.9) - (2 << 30)
+    results = {}
+    for fmt, bits in (("bf16", None), ("rq_bf16_anchor", (2, 2, 2, 16)), ("rq_int4_anchor", (2, 2, 2, 4))):
+        torch.cuda.empty_cache()
+        if fmt == "bf16":
+            per_seq = layers * L * 2 * Hkv * (T + 1) * 128 * 2
+        else:
+            lay = rq.cache_layout(rq.config_from_dict(synth.cache_config_dict(base.with_(bits=bits), capacity=T + 1)))
+            per_seq = layers * lay.total_bytes
+        B = int(max(1, min(1024, budget // per_seq)))
+        wl = base.with_(batch=B) if bits is None else base.with_(batch=B, bits=bits)
+        q = one["q"].expand(-1, B, -1, -1).contiguous()
+        ctx = torch.full((B,), T, dtype=torch.int32, device=dev)
+        k_new = one["k_tail"].expand(-1, B, -1, -1, -1).contiguous()
+        v_new = one["v_tail"].expand(-1, B, -1, -1, -1).contiguous()
+        outs = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
+        if fmt == "bf16":
+            caches = []
+            for _ in range(layers):
+                planes = []
+                for l in range(L):
+                    kv = torch.empty((2, B, Hkv, T + 1, 128), dtype=torch.bfloat16, device=dev)
+                    kv[0, :, :, :T].copy_(one["k"][l].expand(B, -1, -1, -1))
+                    kv[1, :, :, :T].copy_(one["v"][l].expand(B, -1, -1, -1))
+                    planes.append(kv)
+                caches.append(planes)
+            ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+
+            def step():
+                for planes in caches:
+                    for l in range(L):
+                        kv = planes[l]
+                        kv[0, :, :, T:T + 1].copy_(k_new[l])   # append the new token
+                        kv[1, :, :, T:T + 1].copy_(v_new[l])
+                        rq.bf16_decode_attention(kv[0], kv[1], q[l], ctx, k_new[l], v_new[l], workspace=ws,
+                                                 out=outs[l])
+        else:
+            cfgd = synth.cache_config_dict(wl, capacity=T + 1)
+            caches = [rq.Cache(rq.config_from_dict(cfgd), device=dev) for _ in range(layers)]
+            kb = one["k"].expand(-1, B, -1, -1, -1)  # batch stride 0: the same values for every sequence
+            vb = one["v"].expand(-1, B, -1, -1, -1)
+            for c in caches:
+                c.encode(kb, vb)
+
+            def step():
+                for c in caches:
+                    for l in range(L):
+                        c.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
+                    c.encode(k_new, v_new, positions=ctx)
+        ms = time_steps(step, steps, warmup, world, stream)
+        flags = 0 if fmt == "bf16" else max(c.get_error() for c in caches)
+        results[fmt] = {"max_batch": B, "bytes_per_sequence": int(per_seq),
+                        "tokens_per_s": round(job_tokens_per_s(B, world, ms), 1), "ms_per_step": round(ms, 3),
+                        "device_flags": int(flags)}
+        del caches, q, ctx, k_new, v_new, outs
+        torch.cuda.empty_cache()
+    if rank == 0:
+        print(json.dumps({"workload": "capacity_24layer_L4_H16_T8192", "metric": "decode tokens/s at the largest "
+                          "batch whose 24-layer caches fit (attention only)", "results": results,
+                          "hbm_budget_bytes": budget, "data": "synthetic", "n_gpus": world}))
+
+
 def run_rq(args, world, rank):
     from looped_transformer_decode_rq_b200 import rq
 
@@ -423,6 +571,13 @@ def run_rq(args, world, rank):
                           f"({wl.gqa} q-head(s), {int(ctx[0])} cached tokens + 1 tail) plus the encode "
                           f"of its new token, {reps} reps of {per:.3f} s; scaled by B*Hkv={B * Hkv}")}
 
+    extra = None
+    if not args.no_extra and args.workload == "ouro8k":
+        del cache, inp, outs
+        torch.cuda.empty_cache()
+        extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 10, 3, world, rank),
+                 measure_workload(synth.gqa_long(batch=8), 10, 3, world, rank)]
+
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
@@ -440,7 +595,7 @@ def run_rq(args, world, rank):
                      "algorithmic_bytes_per_launch": res_bytes, "launch_ms": round(call_ms, 4),
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                      "frac_of_8tbs": round(achieved / 8000.0, 4)},
-        "cpu_baseline": cpu, "e2e": e2e, "bf16_cache": bf16, "parity": parity,
+        "cpu_baseline": cpu, "e2e": e2e, "bf16_cache": bf16, "parity": parity, "other_workloads": extra,
         "gpu_launches": args.steps * (2 * L + 1), "clocks": clk, "device_flags": flags,
     }
     if rank == 0:
@@ -481,6 +636,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.workload == "capacity":
+            run_capacity(args, world, rank)
         else:
             run_rq(args, world, rank)
     finally:
