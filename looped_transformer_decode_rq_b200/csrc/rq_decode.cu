@@ -188,6 +188,49 @@ __device__ __forceinline__ int code_pos(int e) { return (e * BITS) & 15; }
 
 __device__ __forceinline__ float2 f2sub1(float2 f) { return __fadd2_rn(f, make_float2(-1.f, -1.f)); }
 
+// Integer-dot-product operands for a lane's D query values against BITS-bit
+// packed codes.  The values are quantised to int16 with one scale per lane
+// (|q| <= 32767 * scale) and split into a signed high byte and an unsigned low
+// byte, so that  sum_e q_e c_e = scale * (256 * dp4a(c, hi) + dp4a(c, lo))
+// exactly in 32-bit integers.  Byte b of operand [w][k] pairs with the code
+// that the unpacking of word w puts into byte b at step k:
+//   BITS = 2: (w >> 2k) & 0x03030303 holds elements 16w + 4b + k   (k < 4)
+//   BITS = 4: (w >> 4k) & 0x0F0F0F0F holds elements  8w + 2b + k   (k < 2)
+template <int BITS, int D>
+struct DotOperands {
+  static constexpr int NW = (D * BITS + 31) / 32;
+  static constexpr int KPW = BITS == 2 ? 4 : 2;
+  uint32_t hi[NW][KPW];
+  uint32_t lo[NW][KPW];
+  float scale;
+
+  __device__ __forceinline__ void build(const float* v) {
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < D; ++e) m = fmaxf(m, fabsf(v[e]));
+    scale = m * (1.f / 32767.f);
+    const float inv = m > 0.f ? 32767.f / m : 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+#pragma unroll
+      for (int k = 0; k < KPW; ++k) hi[w][k] = lo[w][k] = 0u;
+#pragma unroll
+    for (int e = 0; e < D; ++e) {
+      int qi = __float2int_rn(v[e] * inv);
+      qi = max(-32767, min(32767, qi));
+      const int per = 32 / BITS, w = e / per, in = e % per;
+      const int b = BITS == 2 ? in / 4 : in / 2, k = BITS == 2 ? in % 4 : in % 2;
+      hi[w][k] |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * b);
+      lo[w][k] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * b);
+    }
+  }
+};
+
+template <int BITS>
+__device__ __forceinline__ uint32_t unpack_bytes(uint32_t w, int k) {
+  return BITS == 2 ? ((w >> (2 * k)) & 0x03030303u) : ((w >> (4 * k)) & 0x0F0F0F0Fu);
+}
+
 // ---------------------------------------------------------------------------
 // split kernel
 // ---------------------------------------------------------------------------
@@ -386,35 +429,35 @@ __global__ void __launch_bounds__(kNT, 1)
     }
     named_bar_sync(kConsumerBar, kNCT);
 
-    // phase-1 registers: reference- and residual-side query slices; the
-    // residual side (and an INT4 reference) pre-multiplied by 2^(23 - p_e)
-    float2 qref[G][C::D1 / 2];
-    float2 qres[G][C::D1 / 2];
+    // phase-1 registers: the bf16 reference side keeps the query slice in
+    // fp32; code planes (INT4 anchor, residual) get int16 dp4a operands
     constexpr int NG1 = RB ? ((C::D1 >= RG) ? C::D1 / RG : 1) : 1;
+    float2 qref[G][REF == kRefBf16 ? C::D1 / 2 : 1];
+    DotOperands<4, REF == kRefInt4 ? C::D1 : 1> oref[G];
+    DotOperands<RB ? RB : 2, RB ? C::D1 : 1> ores[G];
     float qsum_res[G][NG1];
     float qsum_ref[G];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
+      float vr[C::D1], vt[C::D1];
       qsum_ref[gi] = 0.f;
 #pragma unroll
       for (int n = 0; n < NG1; ++n) qsum_res[gi][n] = 0.f;
 #pragma unroll
-      for (int e = 0; e < C::D1; e += 2) {
-        float r0 = sQS[gi * kD + d1 + e], r1 = sQS[gi * kD + d1 + e + 1];
-        qsum_ref[gi] += r0 + r1;
-        if constexpr (REF == kRefInt4) {
-          r0 *= pow2i(23 - code_pos<4>(e));
-          r1 *= pow2i(23 - code_pos<4>(e + 1));
-        }
-        qref[gi][e / 2] = make_float2(r0, r1);
-        if constexpr (RB != 0) {
-          const float t0 = sQT[gi * kD + d1 + e], t1 = sQT[gi * kD + d1 + e + 1];
-          qsum_res[gi][(C::D1 >= RG) ? e / RG : 0] += t0 + t1;
-          qres[gi][e / 2] = make_float2(t0 * pow2i(23 - code_pos<RB>(e)), t1 * pow2i(23 - code_pos<RB>(e + 1)));
-        } else {
-          qres[gi][e / 2] = make_float2(0.f, 0.f);
-        }
+      for (int e = 0; e < C::D1; ++e) {
+        vr[e] = sQS[gi * kD + d1 + e];
+        vt[e] = RB ? sQT[gi * kD + d1 + e] : 0.f;
+        qsum_ref[gi] += vr[e];
+        qsum_res[gi][(C::D1 >= RG) ? e / RG : 0] += vt[e];
       }
+      if constexpr (REF == kRefBf16) {
+#pragma unroll
+        for (int e = 0; e < C::D1; e += 2) qref[gi][e / 2] = make_float2(vr[e], vr[e + 1]);
+      } else {
+        qref[gi][0] = make_float2(0.f, 0.f);
+      }
+      if constexpr (REF == kRefInt4) oref[gi].build(vr);
+      if constexpr (RB != 0) ores[gi].build(vt);
     }
 
     // group-local running softmax state and per-lane accumulators
@@ -497,26 +540,29 @@ __global__ void __launch_bounds__(kNT, 1)
             part[gi] = sum;
           }
         } else if constexpr (REF == kRefInt4) {
-          uint32_t cw[(C::D1 / 2 + 3) / 4];
+          using Ops = DotOperands<4, C::D1>;
+          uint32_t cw[Ops::NW];
           load_codes<C::D1 / 2>(st + C::O_REFK + t * 64 + (d1 >> 1), cw);
           const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMK + t * 16 + 4 * (d1 >> 5)));
-          float2 acc2[G][C::NB];
+          int dhi[G];
+          unsigned dlo[G];
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi)
+          for (int gi = 0; gi < G; ++gi) { dhi[gi] = 0; dlo[gi] = 0u; }
 #pragma unroll
-            for (int c = 0; c < C::NB; ++c) acc2[gi][c] = make_float2(0.f, 0.f);
+          for (int w = 0; w < Ops::NW; ++w)
 #pragma unroll
-          for (int e = 0; e < C::D1; e += 2) {
-            const float2 f = f2sub1(make_float2(code_f<4>(cw, e), code_f<4>(cw, e + 1)));
+            for (int kk = 0; kk < Ops::KPW; ++kk) {
+              const uint32_t x = unpack_bytes<4>(cw[w], kk);
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) acc2[gi][e / C::EB] = __ffma2_rn(qref[gi][e / 2], f, acc2[gi][e / C::EB]);
-          }
+              for (int gi = 0; gi < G; ++gi) {
+                dhi[gi] = __dp4a(static_cast<int>(x), static_cast<int>(oref[gi].hi[w][kk]), dhi[gi]);
+                dlo[gi] = __dp4a(x, oref[gi].lo[w][kk], dlo[gi]);
+              }
+            }
 #pragma unroll
           for (int gi = 0; gi < G; ++gi) {
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < C::NB; ++c) sum += acc2[gi][c].x + acc2[gi][c].y;
-            part[gi] = fmaf(sz.x, sum, sz.y * qsum_ref[gi]);
+            const float dot = static_cast<float>(dhi[gi] * 256 + static_cast<int>(dlo[gi])) * oref[gi].scale;
+            part[gi] = fmaf(sz.x, dot, sz.y * qsum_ref[gi]);
           }
         }
         if constexpr (C::HAS_ALPHA) {
@@ -525,31 +571,38 @@ __global__ void __launch_bounds__(kNT, 1)
           for (int gi = 0; gi < G; ++gi) part[gi] *= aK;
         }
         if constexpr (RB != 0) {
+          using Ops = DotOperands<RB, C::D1>;
           constexpr int NBYTES = C::D1 * RB / 8;
-          uint32_t cw[(NBYTES + 3) / 4];
+          constexpr int WPG = (RG * RB) / 32;  // 32-bit code words per group
+          uint32_t cw[Ops::NW];
           load_codes<NBYTES>(st + C::O_RESK + t * C::CB + (d1 * RB >> 3), cw);
-          float2 acc2[G][C::NB];
+          int dhi[G][NG1];
+          unsigned dlo[G][NG1];
 #pragma unroll
           for (int gi = 0; gi < G; ++gi)
 #pragma unroll
-            for (int c = 0; c < C::NB; ++c) acc2[gi][c] = make_float2(0.f, 0.f);
+            for (int n = 0; n < NG1; ++n) { dhi[gi][n] = 0; dlo[gi][n] = 0u; }
 #pragma unroll
-          for (int e = 0; e < C::D1; e += 2) {
-            const float2 f = f2sub1(make_float2(code_f<RB>(cw, e), code_f<RB>(cw, e + 1)));
+          for (int w = 0; w < Ops::NW; ++w) {
+            const int n = (NG1 > 1) ? w / WPG : 0;
 #pragma unroll
-            for (int gi = 0; gi < G; ++gi) acc2[gi][e / C::EB] = __ffma2_rn(qres[gi][e / 2], f, acc2[gi][e / C::EB]);
+            for (int kk = 0; kk < Ops::KPW; ++kk) {
+              const uint32_t x = unpack_bytes<RB>(cw[w], kk);
+#pragma unroll
+              for (int gi = 0; gi < G; ++gi) {
+                dhi[gi][n] = __dp4a(static_cast<int>(x), static_cast<int>(ores[gi].hi[w][kk]), dhi[gi][n]);
+                dlo[gi][n] = __dp4a(x, ores[gi].lo[w][kk], dlo[gi][n]);
+              }
+            }
           }
-          constexpr int BPG = (C::D1 >= RG) ? RG / C::EB : C::NB;  // accumulation blocks per group
 #pragma unroll
           for (int n = 0; n < NG1; ++n) {
             const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(
                 st + C::O_RESMK + t * C::MB + 4 * (d1 / RG + n)));
 #pragma unroll
             for (int gi = 0; gi < G; ++gi) {
-              float sum = 0.f;
-#pragma unroll
-              for (int c = n * BPG; c < (n + 1) * BPG; ++c) sum += acc2[gi][c].x + acc2[gi][c].y;
-              part[gi] += fmaf(sz.x, sum, sz.y * qsum_res[gi][n]);
+              const float dot = static_cast<float>(dhi[gi][n] * 256 + static_cast<int>(dlo[gi][n])) * ores[gi].scale;
+              part[gi] += fmaf(sz.x, dot, sz.y * qsum_res[gi][n]);
             }
           }
         }
