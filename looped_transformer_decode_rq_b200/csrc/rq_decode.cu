@@ -79,7 +79,7 @@ struct Cfg {
   static constexpr int TOK_PASS = kGT / TPT;    // tokens per pass of a group
   static constexpr int PASSES = kTT / TOK_PASS;
   // phase 2 (values)
-  static constexpr int D2 = (G >= 8) ? 4 : 8;   // dims per lane
+  static constexpr int D2 = (G >= 4) ? 4 : 8;   // dims per lane
   static constexpr int TPR2 = kD / D2;          // lanes per token row
   static constexpr int SLICES = kGT / TPR2;
   static constexpr int TOK2 = kTT / SLICES;     // tokens per lane per page
