@@ -167,9 +167,10 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 def record_bytes(lay, cfgd, loop):
-    L = cfgd["num_loops"]
-    ref = 2 * lay.ref_record_bytes + 2 * lay.ref_meta_record_bytes
-    if loop == L - 1:
+    """Bytes one decode call of `loop` reads per (b, kv-head, token)."""
+    a = lay.anchor_of[loop]
+    ref = 2 * lay.codes_record_bytes[a] + 2 * lay.meta_record_bytes[a]
+    if loop == a:
         return ref
     res = 2 * lay.codes_record_bytes[loop] + 2 * lay.meta_record_bytes[loop]
     if cfgd["alpha_mode"][loop] == 2:

@@ -9,7 +9,8 @@
  *      K_l  ~  alpha_l * K_ref  +  H^T deq(codes_l)        (likewise V)
  * ([RQ] abstract; Figure 1 steps 2-5; Figure 2 caption).  Decode attention
  * scores each cached token as  alpha (q . K_ref) + (H q) . deq(codes)  and
- * never materialises a bf16 copy of loop l.
+ * never materialises a bf16 copy of loop l.  K_ref is the loop's anchor: the
+ * final loop by default (see rq_anchor_policy).
  *
  * Conventions shared by every entry point:
  *  - Memory: the caller owns all device memory and streams.  The library
@@ -23,7 +24,7 @@
  *    capacity, a pipeline wait that timed out) set bits of the cache's device
  *    status word, read by rq_get_error.  rq_last_error_message() returns a
  *    human-readable reason for the calling thread's last non-OK status.
- *  - Loop index is 0-based; loop num_loops-1 is the reference loop.
+ *  - Loop index is 0-based; by default loop num_loops-1 is every loop's reference.
  *  - head_dim is 128 everywhere (the rotation is the order-128 Hadamard).
  *  - All tensors are row-major and contiguous unless strides are passed.
  */
@@ -73,61 +74,80 @@ typedef enum rq_status {
 #define RQ_FLAG_PIPE_TIMEOUT 8u   /* a decode pipeline wait exceeded its limit (output invalid) */
 #define RQ_FLAG_META_OVERFLOW 16u /* an alpha, scale or offset overflowed fp16 */
 
-/* Least-squares scale: [RQ] Figure 1 step 3 ("LS"); Figure 3 caption ("alpha = 1"
- * ablation); Figure 1 step 1 (direct quantisation = alpha 0, no rotation). */
-typedef enum rq_alpha_mode { RQ_ALPHA_LS = 0, RQ_ALPHA_ONE = 1, RQ_ALPHA_ZERO = 2 } rq_alpha_mode;
+/* Scaling coefficient of the reference: [RQ] Figure 1 step 3 (least squares,
+ * "LS"); Figure 3 caption ("alpha = 1" ablation); Figure 1 step 1 (direct
+ * quantisation = alpha 0, no rotation); Table 9 ("Norm-ratio": ||x||/||ref||). */
+typedef enum rq_alpha_mode {
+  RQ_ALPHA_LS = 0,
+  RQ_ALPHA_ONE = 1,
+  RQ_ALPHA_ZERO = 2,
+  RQ_ALPHA_NORM_RATIO = 3
+} rq_alpha_mode;
+
+/* Which loop is each loop's reference ("anchor"): [RQ] Table 1 ("First-loop",
+ * "Last-loop" reference choice) and Table 8 (anchor intervals N x [2^n, 4]:
+ * groups of loops each ending in its own INT4 anchor). */
+typedef enum rq_anchor_policy {
+  RQ_ANCHOR_LAST = 0,     /* the final loop is every loop's reference (the pages' choice) */
+  RQ_ANCHOR_FIRST = 1,    /* loop 0 is every loop's reference */
+  RQ_ANCHOR_INTERVAL = 2  /* blocks of anchor_interval loops; each block's last loop
+                             (the final loop for a short last block) anchors the block */
+} rq_anchor_policy;
 
 /* Cache configuration ([RQ] Table 5 caption: loop-wise precision, INT2 with
  * g = 16 or 32, INT4 with g = 32; Figure 1 step 5: mixed precision such as
- * [2,2,2,4]).  Per-loop arrays use entries [0, num_loops). */
+ * [2,2,2,4]).  Per-loop arrays use entries [0, num_loops).  A zero-filled
+ * anchor_policy is the pages' Last-loop reference. */
 typedef struct rq_config {
-  int32_t num_loops;  /* L in [2, 16]; loop L-1 is the reference */
+  int32_t num_loops;  /* L in [2, 16] */
   int32_t batch;      /* B >= 1 sequences */
   int32_t kv_heads;   /* Hkv >= 1 */
   int32_t q_heads;    /* Hq = G * Hkv with G in {1, 2, 4, 8} */
   int32_t head_dim;   /* must be RQ_HEAD_DIM */
   int32_t capacity;   /* maximum cached tokens per sequence, >= 1 */
-  int32_t bits[RQ_MAX_LOOPS];  /* residual loops: 2 or 4; reference loop: 16 (bf16) or 4 (INT4) */
-  int32_t group[RQ_MAX_LOOPS]; /* residual loops: 16 or 32; reference loop: 32 (ignored for bf16) */
-  int32_t rotate[RQ_MAX_LOOPS];      /* residual loops: 1 = Hadamard-128 rotation, 0 = none; ref: 0 */
-  int32_t alpha_mode[RQ_MAX_LOOPS];  /* residual loops: rq_alpha_mode; ref: ignored */
+  int32_t bits[RQ_MAX_LOOPS];  /* residual loops: 2 or 4; anchor loops: 16 (bf16) or 4 (INT4) */
+  int32_t group[RQ_MAX_LOOPS]; /* residual loops: 16 or 32; anchor loops: 32 (ignored for bf16) */
+  int32_t rotate[RQ_MAX_LOOPS];      /* residual loops: 1 = Hadamard-128 rotation, 0 = none; anchors: 0 */
+  int32_t alpha_mode[RQ_MAX_LOOPS];  /* residual loops: rq_alpha_mode; anchors: ignored */
+  int32_t anchor_policy;    /* rq_anchor_policy */
+  int32_t anchor_interval;  /* RQ_ANCHOR_INTERVAL: loops per block, in [2, num_loops] */
 } rq_config;
 
 /* Where each plane lives inside the caller's cache buffer.  Every plane is
  * indexed [b][h][t] with t < capacity_padded, one fixed-size record per
  * (b, h, t), and starts on a 1024-byte boundary.  Offsets are bytes from the
  * start of the buffer; -1 marks a plane the configuration does not have.
+ * Every loop l has planes codes[l][k|v]; the rest depends on its role:
  *
- *  reference, bf16:  ref[k|v]   128 bf16 per record (256 B)
- *  reference, INT4:  ref[k|v]   128 4-bit codes (64 B; element d in bits 4*(d%8)
- *                               of little-endian 32-bit word d/8), ref_meta[k|v]
- *                               4 groups x (fp16 scale, fp16 offset) = 16 B
- *  residual loop l:  codes[l][k|v]  128 b-bit codes, rotated domain (INT2: element
- *                               d in bits 2*(d%16) of word d/16, 32 B; INT4 as above)
- *                    meta[l][k|v]   (128/g) x (fp16 scale, fp16 offset)
- *                    alpha[l]       (fp16 alpha_K, fp16 alpha_V) = 4 B
- *  status:           one 32-bit device status word (256 B reserved)
+ *  anchor, bf16:  codes = 128 bf16 per record (256 B); no meta, no alpha
+ *  anchor, INT4:  codes = 128 4-bit codes (64 B; element d in bits 4*(d%8) of
+ *                 little-endian 32-bit word d/8); meta = 4 groups x (fp16 scale,
+ *                 fp16 offset) = 16 B; no alpha
+ *  residual:      codes = 128 b-bit codes in the rotated domain (INT2: element d
+ *                 in bits 2*(d%16) of word d/16, 32 B; INT4 as above);
+ *                 meta = (128/g) x (fp16 scale, fp16 offset);
+ *                 alpha = (fp16 alpha_K, fp16 alpha_V) = 4 B
+ *  status:        one 32-bit device status word (256 B reserved)
+ *  anchor_of[l] is the loop whose anchor planes loop l is decoded against
+ *  (anchor_of[l] == l for an anchor loop).
  */
 typedef struct rq_layout {
   int64_t capacity_padded;
   int64_t total_bytes;
   int64_t status_offset;
-  int64_t ref_offset[2];
-  int64_t ref_meta_offset[2];
-  int64_t ref_record_bytes;
-  int64_t ref_meta_record_bytes;
   int64_t codes_offset[RQ_MAX_LOOPS][2];
   int64_t meta_offset[RQ_MAX_LOOPS][2];
   int64_t alpha_offset[RQ_MAX_LOOPS];
   int64_t codes_record_bytes[RQ_MAX_LOOPS];
   int64_t meta_record_bytes[RQ_MAX_LOOPS];
+  int32_t anchor_of[RQ_MAX_LOOPS];
 } rq_layout;
 
 typedef struct rq_cache rq_cache;
 
 /* Validates cfg and fills *out.  Host only, pure.  RQ_ERR_INVALID_ARG for a
  * null pointer or an out-of-range field; RQ_ERR_UNSUPPORTED for head_dim != 128
- * or a bits/group/G combination this build does not implement. */
+ * or a bits/group/G/anchor combination this build does not implement. */
 RQ_API rq_status rq_cache_layout(const rq_config* cfg, rq_layout* out);
 
 /* Binds a cache handle to the caller's device buffer (>= layout.total_bytes,
@@ -145,11 +165,12 @@ RQ_API rq_status rq_cache_info(const rq_cache* cache, rq_config* cfg_out, rq_lay
 
 /* Encode ([RQ] abstract; Figure 1 steps 2-5): for every loop, sequence b,
  * kv-head h and the n_tokens tokens at positions [pos_b, pos_b + n_tokens):
- * store the reference loop (bf16 copy or direct INT4 g=32), then for each
- * other loop the fp16 LS scale alpha = <x, ref>/<ref, ref> (per 128-vector,
- * K and V separately; 0 if <ref, ref> = 0), the residual x - alpha*ref, its
- * Hadamard-128 rotation and asymmetric min-max group quantisation.  The INT4
- * anchor's dequantised value is the reference the residuals are taken against.
+ * store each anchor loop (bf16 copy or direct INT4 g=32), then for every other
+ * loop the fp16 scale alpha against its anchor (LS: <x, ref>/<ref, ref>; norm
+ * ratio: ||x||/||ref||; per 128-vector, K and V separately; 0 if ref is 0), the
+ * residual x - alpha*ref, its Hadamard-128 rotation and asymmetric min-max group
+ * quantisation.  An INT4 anchor's dequantised value is the reference the
+ * residuals are taken against.
  *
  *  k, v        device bf16, element [l][b][h][i][d] at
  *              l*strides[0] + b*strides[1] + h*strides[2] + i*strides[3] + d
@@ -177,8 +198,8 @@ RQ_API rq_status rq_decode_workspace_size(const rq_cache* cache, int64_t* bytes_
  * and the output is
  *     ( sum_t p_t alpha_V,t ref_v,t  +  H^T sum_t p_t deq(codes_V,t)
  *       + sum_tail p_j v_tail,j ) / sum p
- * with one inverse rotation per (b, q-head).  The reference loop is plain
- * attention over its bf16 or INT4 reference.  n_tail current tokens (bf16,
+ * with one inverse rotation per (b, q-head), ref being the loop's anchor.  An
+ * anchor loop is plain attention over its bf16 or INT4 planes.  n_tail current tokens (bf16,
  * not yet encoded) join the softmax.  Split-K over 64-token pages with an
  * online softmax, merged by a second kernel.
  *
@@ -245,7 +266,7 @@ RQ_API rq_status rq_bf16_decode_attention(int32_t batch, int32_t kv_heads, int32
 /* Reconstruction (test support): fp32 K_hat, V_hat of loop `loop` for tokens
  * [t0, t0 + n) of every (b, h), written to k_out/v_out [B][Hkv][n][128]:
  * alpha * ref + H^T deq(codes) for a residual loop, the (dequantised)
- * reference for the reference loop. */
+ * anchor for an anchor loop. */
 RQ_API rq_status rq_reconstruct(const rq_cache* cache, int32_t loop, int32_t t0, int32_t n, float* k_out,
                          float* v_out, rq_stream_t stream);
 

@@ -21,8 +21,8 @@ struct rq_cache {
   uint8_t* base;
   int device;
   int num_ctas;
-  bool tmaps_ready;
-  CUtensorMap tm_ref[2];
+  bool tmaps_ready[RQ_MAX_LOOPS];        // per bf16 anchor loop
+  CUtensorMap tm_anchor[RQ_MAX_LOOPS][2];
 };
 
 namespace {
@@ -79,6 +79,18 @@ rq_status make_plane_map(CUtensorMap* map, const void* base, int B, int H, int64
   return RQ_OK;
 }
 
+// The loop whose anchor planes loop l is stored against (l itself for an anchor).
+int anchor_of(const rq_config& c, int l) {
+  const int L = c.num_loops;
+  if (c.anchor_policy == RQ_ANCHOR_FIRST) return 0;
+  if (c.anchor_policy == RQ_ANCHOR_INTERVAL && c.anchor_interval >= 2) {
+    const int n = c.anchor_interval;
+    const int a = (l / n) * n + n - 1;
+    return a < L - 1 ? a : L - 1;
+  }
+  return L - 1;
+}
+
 rq_status validate_config(const rq_config* c) {
   if (c == nullptr) return fail(RQ_ERR_INVALID_ARG, "config is null");
   if (c->num_loops < 2 || c->num_loops > RQ_MAX_LOOPS)
@@ -92,28 +104,35 @@ rq_status validate_config(const rq_config* c) {
     return fail(RQ_ERR_UNSUPPORTED, "q_heads / kv_heads = %d (supported: 1, 2, 4, 8)", G);
   if (c->head_dim != RQ_HEAD_DIM) return fail(RQ_ERR_UNSUPPORTED, "head_dim %d != 128", c->head_dim);
   if (c->capacity < 1) return fail(RQ_ERR_INVALID_ARG, "capacity %d < 1", c->capacity);
-  const int ref = c->num_loops - 1;
-  if (c->bits[ref] != 16 && c->bits[ref] != 4)
-    return fail(RQ_ERR_UNSUPPORTED, "reference loop bits %d (supported: 16, 4)", c->bits[ref]);
-  if (c->bits[ref] == 4 && c->group[ref] != 32)
-    return fail(RQ_ERR_UNSUPPORTED, "INT4 reference group %d (supported: 32)", c->group[ref]);
-  for (int l = 0; l < ref; ++l) {
+  if (c->anchor_policy < RQ_ANCHOR_LAST || c->anchor_policy > RQ_ANCHOR_INTERVAL)
+    return fail(RQ_ERR_INVALID_ARG, "anchor_policy %d", c->anchor_policy);
+  if (c->anchor_policy == RQ_ANCHOR_INTERVAL && (c->anchor_interval < 2 || c->anchor_interval > c->num_loops))
+    return fail(RQ_ERR_INVALID_ARG, "anchor_interval %d outside [2, num_loops]", c->anchor_interval);
+  for (int l = 0; l < c->num_loops; ++l) {
+    if (anchor_of(*c, l) != l) continue;
+    if (c->bits[l] != 16 && c->bits[l] != 4)
+      return fail(RQ_ERR_UNSUPPORTED, "anchor loop %d bits %d (supported: 16, 4)", l, c->bits[l]);
+    if (c->bits[l] == 4 && c->group[l] != 32)
+      return fail(RQ_ERR_UNSUPPORTED, "INT4 anchor loop %d group %d (supported: 32)", l, c->group[l]);
+  }
+  for (int l = 0; l < c->num_loops; ++l) {
+    if (anchor_of(*c, l) == l) continue;
     if (c->bits[l] != 2 && c->bits[l] != 4)
       return fail(RQ_ERR_UNSUPPORTED, "loop %d bits %d (supported: 2, 4)", l, c->bits[l]);
     if (c->group[l] != 16 && c->group[l] != 32)
       return fail(RQ_ERR_UNSUPPORTED, "loop %d group %d (supported: 16, 32)", l, c->group[l]);
     if (c->rotate[l] != 0 && c->rotate[l] != 1)
       return fail(RQ_ERR_INVALID_ARG, "loop %d rotate %d", l, c->rotate[l]);
-    if (c->alpha_mode[l] < RQ_ALPHA_LS || c->alpha_mode[l] > RQ_ALPHA_ZERO)
+    if (c->alpha_mode[l] < RQ_ALPHA_LS || c->alpha_mode[l] > RQ_ALPHA_NORM_RATIO)
       return fail(RQ_ERR_INVALID_ARG, "loop %d alpha_mode %d", l, c->alpha_mode[l]);
   }
   return RQ_OK;
 }
 
 int ref_kind_for(const rq_config& c, int loop) {
-  const int ref = c.num_loops - 1;
-  if (loop != ref && c.alpha_mode[loop] == RQ_ALPHA_ZERO) return rq::kRefNone;
-  return c.bits[ref] == 16 ? rq::kRefBf16 : rq::kRefInt4;
+  const int a = anchor_of(c, loop);
+  if (loop != a && c.alpha_mode[loop] == RQ_ALPHA_ZERO) return rq::kRefNone;
+  return c.bits[a] == 16 ? rq::kRefBf16 : rq::kRefInt4;
 }
 
 }  // namespace
@@ -153,7 +172,6 @@ rq_status rq_cache_layout(const rq_config* cfg, rq_layout* out) {
   if (st != RQ_OK) return st;
   rq_layout L;
   std::memset(&L, 0, sizeof(L));
-  const int ref = cfg->num_loops - 1;
   const int64_t cap_pad = align_up(cfg->capacity, RQ_PAGE_TOKENS);
   const int64_t recs = static_cast<int64_t>(cfg->batch) * cfg->kv_heads * cap_pad;
   int64_t off = 0;
@@ -164,22 +182,26 @@ rq_status rq_cache_layout(const rq_config* cfg, rq_layout* out) {
   };
   L.capacity_padded = cap_pad;
   L.status_offset = place(256);
-  L.ref_record_bytes = cfg->bits[ref] == 16 ? 256 : 64;
-  L.ref_meta_record_bytes = cfg->bits[ref] == 16 ? 0 : 16;
-  for (int kv = 0; kv < 2; ++kv) L.ref_offset[kv] = place(recs * L.ref_record_bytes);
-  for (int kv = 0; kv < 2; ++kv)
-    L.ref_meta_offset[kv] = L.ref_meta_record_bytes ? place(recs * L.ref_meta_record_bytes) : -1;
   for (int l = 0; l < RQ_MAX_LOOPS; ++l) {
     L.codes_offset[l][0] = L.codes_offset[l][1] = -1;
     L.meta_offset[l][0] = L.meta_offset[l][1] = -1;
     L.alpha_offset[l] = -1;
+    L.anchor_of[l] = -1;
   }
-  for (int l = 0; l < ref; ++l) {
-    L.codes_record_bytes[l] = cfg->bits[l] * RQ_HEAD_DIM / 8;
-    L.meta_record_bytes[l] = 4 * (RQ_HEAD_DIM / cfg->group[l]);
+  for (int l = 0; l < cfg->num_loops; ++l) {
+    const int a = anchor_of(*cfg, l);
+    L.anchor_of[l] = a;
+    if (a == l) {
+      L.codes_record_bytes[l] = cfg->bits[l] == 16 ? 256 : 64;
+      L.meta_record_bytes[l] = cfg->bits[l] == 16 ? 0 : 16;
+    } else {
+      L.codes_record_bytes[l] = cfg->bits[l] * RQ_HEAD_DIM / 8;
+      L.meta_record_bytes[l] = 4 * (RQ_HEAD_DIM / cfg->group[l]);
+    }
     for (int kv = 0; kv < 2; ++kv) L.codes_offset[l][kv] = place(recs * L.codes_record_bytes[l]);
-    for (int kv = 0; kv < 2; ++kv) L.meta_offset[l][kv] = place(recs * L.meta_record_bytes[l]);
-    L.alpha_offset[l] = place(recs * 4);
+    if (L.meta_record_bytes[l])
+      for (int kv = 0; kv < 2; ++kv) L.meta_offset[l][kv] = place(recs * L.meta_record_bytes[l]);
+    if (a != l) L.alpha_offset[l] = place(recs * 4);
   }
   L.total_bytes = off;
   *out = L;
@@ -210,7 +232,7 @@ rq_status rq_cache_create(const rq_config* cfg, void* device_buffer, int64_t buf
   c->base = static_cast<uint8_t*>(device_buffer);
   c->device = dev;
   c->num_ctas = rq::decode_grid_ctas(dev);
-  c->tmaps_ready = false;
+  for (int l = 0; l < RQ_MAX_LOOPS; ++l) c->tmaps_ready[l] = false;
   *out = c;
   return RQ_OK;
 }
@@ -260,22 +282,18 @@ rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const int64_t
   p.s_b = strides[1];
   p.s_h = strides[2];
   p.s_t = strides[3];
-  const int ref = c.num_loops - 1;
-  p.ref_bits = c.bits[ref];
-  for (int kv = 0; kv < 2; ++kv) {
-    p.ref_plane[kv] = cache->base + cache->lay.ref_offset[kv];
-    p.ref_meta[kv] = cache->lay.ref_meta_offset[kv] >= 0 ? cache->base + cache->lay.ref_meta_offset[kv] : nullptr;
-  }
-  for (int l = 0; l < ref; ++l) {
+  const rq_layout& lay = cache->lay;
+  for (int l = 0; l < c.num_loops; ++l) {
     for (int kv = 0; kv < 2; ++kv) {
-      p.codes[l][kv] = cache->base + cache->lay.codes_offset[l][kv];
-      p.meta[l][kv] = cache->base + cache->lay.meta_offset[l][kv];
+      p.codes[l][kv] = cache->base + lay.codes_offset[l][kv];
+      p.meta[l][kv] = lay.meta_offset[l][kv] >= 0 ? cache->base + lay.meta_offset[l][kv] : nullptr;
     }
-    p.alpha[l] = cache->base + cache->lay.alpha_offset[l];
+    p.alpha[l] = lay.alpha_offset[l] >= 0 ? cache->base + lay.alpha_offset[l] : nullptr;
     p.bits[l] = c.bits[l];
     p.group[l] = c.group[l];
     p.rotate[l] = c.rotate[l];
     p.alpha_mode[l] = c.alpha_mode[l];
+    p.anchor[l] = lay.anchor_of[l];
   }
   p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
   cudaError_t e = rq::launch_encode(p, static_cast<cudaStream_t>(stream));
@@ -338,20 +356,21 @@ rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void*
   rq_status st = check_decode_common(c.batch, c.kv_heads, c.q_heads, q, ctx_len, k_tail, v_tail, n_tail,
                                      softmax_scale, out, workspace, workspace_bytes, need);
   if (st != RQ_OK) return st;
-  const int ref = c.num_loops - 1;
+  const rq_layout& lay = cache->lay;
+  const int a = lay.anchor_of[loop];
   const int ref_kind = ref_kind_for(c, loop);
-  const int res_bits = loop == ref ? 0 : c.bits[loop];
-  const int res_group = loop == ref ? 32 : c.group[loop];
+  const int res_bits = loop == a ? 0 : c.bits[loop];
+  const int res_group = loop == a ? 32 : c.group[loop];
   if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G))
     return fail(RQ_ERR_UNSUPPORTED, "no decode kernel for this loop format");
-  if (ref_kind == rq::kRefBf16 && !cache->tmaps_ready) {
-    const int64_t cp = cache->lay.capacity_padded;
+  if (ref_kind == rq::kRefBf16 && !cache->tmaps_ready[a]) {
+    const int64_t cp = lay.capacity_padded;
     for (int kv = 0; kv < 2; ++kv) {
-      st = make_plane_map(&cache->tm_ref[kv], cache->base + cache->lay.ref_offset[kv], c.batch, c.kv_heads, cp,
+      st = make_plane_map(&cache->tm_anchor[a][kv], cache->base + lay.codes_offset[a][kv], c.batch, c.kv_heads, cp,
                           static_cast<int64_t>(c.kv_heads) * cp * RQ_HEAD_DIM, cp * RQ_HEAD_DIM, RQ_HEAD_DIM);
       if (st != RQ_OK) return st;
     }
-    cache->tmaps_ready = true;
+    cache->tmaps_ready[a] = true;
   }
   rq::DecodeParams p;
   std::memset(&p, 0, sizeof(p));
@@ -359,19 +378,19 @@ rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void*
   p.Hkv = c.kv_heads;
   p.G = G;
   p.capacity = c.capacity;
-  p.plane_tokens = cache->lay.capacity_padded;
+  p.plane_tokens = lay.capacity_padded;
   if (ref_kind == rq::kRefInt4) {
     for (int kv = 0; kv < 2; ++kv) {
-      p.ref_codes[kv] = cache->base + cache->lay.ref_offset[kv];
-      p.ref_meta[kv] = cache->base + cache->lay.ref_meta_offset[kv];
+      p.ref_codes[kv] = cache->base + lay.codes_offset[a][kv];
+      p.ref_meta[kv] = cache->base + lay.meta_offset[a][kv];
     }
   }
   if (res_bits) {
     for (int kv = 0; kv < 2; ++kv) {
-      p.res_codes[kv] = cache->base + cache->lay.codes_offset[loop][kv];
-      p.res_meta[kv] = cache->base + cache->lay.meta_offset[loop][kv];
+      p.res_codes[kv] = cache->base + lay.codes_offset[loop][kv];
+      p.res_meta[kv] = cache->base + lay.meta_offset[loop][kv];
     }
-    p.alpha = cache->base + cache->lay.alpha_offset[loop];
+    p.alpha = cache->base + lay.alpha_offset[loop];
     p.rotate = c.rotate[loop];
   }
   p.q = static_cast<const uint16_t*>(q);
@@ -384,8 +403,8 @@ rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void*
   p.partials = static_cast<float*>(workspace);
   p.num_ctas = cache->num_ctas;
   p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
-  cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, &cache->tm_ref[0], &cache->tm_ref[1],
-                                    static_cast<cudaStream_t>(stream));
+  cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, &cache->tm_anchor[a][0],
+                                    &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return RQ_OK;
 }
@@ -452,20 +471,21 @@ rq_status rq_reconstruct(const rq_cache* cache, int32_t loop, int32_t t0, int32_
   if (n == 0) return RQ_OK;
   if (k_out == nullptr || v_out == nullptr || !aligned(k_out, 16) || !aligned(v_out, 16))
     return fail(RQ_ERR_INVALID_ARG, "outputs null or not 16-byte aligned");
-  const int ref = c.num_loops - 1;
+  const rq_layout& lay = cache->lay;
+  const int a = lay.anchor_of[loop];
   rq::ReconstructParams p;
   std::memset(&p, 0, sizeof(p));
   p.B = c.batch;
   p.Hkv = c.kv_heads;
-  p.cap_pad = cache->lay.capacity_padded;
+  p.cap_pad = lay.capacity_padded;
   p.t0 = t0;
   p.n = n;
-  p.ref_bits = c.bits[ref];
+  p.ref_bits = c.bits[a];
   for (int kv = 0; kv < 2; ++kv) {
-    p.ref_plane[kv] = cache->base + cache->lay.ref_offset[kv];
-    p.ref_meta[kv] = cache->lay.ref_meta_offset[kv] >= 0 ? cache->base + cache->lay.ref_meta_offset[kv] : nullptr;
+    p.ref_plane[kv] = cache->base + lay.codes_offset[a][kv];
+    p.ref_meta[kv] = lay.meta_offset[a][kv] >= 0 ? cache->base + lay.meta_offset[a][kv] : nullptr;
   }
-  p.is_ref = loop == ref;
+  p.is_ref = loop == a;
   if (!p.is_ref) {
     for (int kv = 0; kv < 2; ++kv) {
       p.codes[kv] = cache->base + cache->lay.codes_offset[loop][kv];

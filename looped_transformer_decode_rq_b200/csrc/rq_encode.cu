@@ -2,9 +2,11 @@
 // sm_100a.
 //
 // Encode follows "ResidualQuant: KV Cache Quantization for Looped Transformers
-// with 2-Bit Residuals" (abstract; Figure 1 steps 2-5; Figure 2 caption): the
-// final loop is the reference, every other loop is stored as the LS-scaled
-// residual, rotated by the order-128 Hadamard, quantised per group to INT2 or
+// with 2-Bit Residuals" (abstract; Figure 1 steps 2-5; Figure 2 caption): an
+// anchor loop (the final loop by default; Table 1 and Table 8 for the First-
+// loop and anchor-interval variants) is the reference, every other loop is
+// stored as the scaled residual against its anchor (LS, or Table 9's norm
+// ratio), rotated by the order-128 Hadamard, quantised per group to INT2 or
 // INT4 with an fp16 scale and offset.
 //
 // One warp handles one (b, h, token) for all loops: lanes 0-15 the key,
@@ -140,79 +142,86 @@ __global__ void __launch_bounds__(256) encode_kernel(const EncodeParams P) {
   const int64_t rec = static_cast<int64_t>(b * P.Hkv + h) * P.cap_pad + pos;
   bool bad = false, overflow = false;
 
-  // ---- reference loop
-  float ref[8];
-  {
-    const uint16_t* src = X + static_cast<int64_t>(P.L - 1) * P.s_l + src0;
-    load8_bf16(src, ref);
-    bad |= !in_range8(ref);
-    if (P.ref_bits == 16) {
-      *reinterpret_cast<uint4*>(P.ref_plane[kv] + rec * 256 + 16 * j) =
-          __ldg(reinterpret_cast<const uint4*>(src));
-    } else {
+  for (int a = 0; a < P.L; ++a) {  // every anchor, then the loops it anchors
+    if (P.anchor[a] != a) continue;
+    float ref[8];
+    {
+      const uint16_t* src = X + static_cast<int64_t>(a) * P.s_l + src0;
+      load8_bf16(src, ref);
+      bad |= !in_range8(ref);
+      if (P.bits[a] == 16) {
+        *reinterpret_cast<uint4*>(P.codes[a][kv] + rec * 256 + 16 * j) =
+            __ldg(reinterpret_cast<const uint4*>(src));
+      } else {
+        uint32_t c[8];
+        __half s_h, z_h;
+        quantize8(ref, 4, 4, c, s_h, z_h);
+        uint32_t w = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w |= c[e] << (4 * e);
+        *reinterpret_cast<uint32_t*>(P.codes[a][kv] + rec * 64 + 4 * j) = w;
+        if ((j & 3) == 0)
+          *reinterpret_cast<uint32_t*>(P.meta[a][kv] + rec * 16 + 4 * (j >> 2)) = half2_bits(s_h, z_h);
+        overflow |= !(half_finite(s_h) && half_finite(z_h));
+        const float sf = __half2float(s_h), zf = __half2float(z_h);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ref[e] = __fadd_rn(zf, __fmul_rn(static_cast<float>(c[e]), sf));
+      }
+    }
+    float refref = 0.f;
+    bool have_refref = false;
+
+    for (int l = 0; l < P.L; ++l) {
+      if (l == a || P.anchor[l] != a) continue;
+      float x[8];
+      load8_bf16(X + static_cast<int64_t>(l) * P.s_l + src0, x);
+      bad |= !in_range8(x);
+      float al = 0.f;
+      const int mode = P.alpha_mode[l];
+      if (mode == RQ_ALPHA_LS || mode == RQ_ALPHA_NORM_RATIO) {
+        if (!have_refref) {
+          refref = tree_dot(ref, ref);
+          have_refref = true;
+        }
+        if (mode == RQ_ALPHA_LS) {
+          const float num = tree_dot(x, ref);
+          al = (refref == 0.f) ? 0.f : __fdiv_rn(num, refref);
+        } else {
+          const float xx = tree_dot(x, x);
+          al = (refref == 0.f) ? 0.f : __fdiv_rn(__fsqrt_rn(xx), __fsqrt_rn(refref));
+        }
+      } else if (mode == RQ_ALPHA_ONE) {
+        al = 1.f;
+      }
+      const __half a_h = __float2half_rn(al);
+      overflow |= !half_finite(a_h);
+      if (j == 0)
+        *reinterpret_cast<__half*>(P.alpha[l] + rec * 4 + 2 * kv) = a_h;
+      const float af = __half2float(a_h);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], __fmul_rn(af, ref[e]));
+      if (P.rotate[l]) fwht128(x, j);
+      const int bits = P.bits[l], g = P.group[l];
       uint32_t c[8];
       __half s_h, z_h;
-      quantize8(ref, 4, 4, c, s_h, z_h);
-      uint32_t w = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w |= c[e] << (4 * e);
-      *reinterpret_cast<uint32_t*>(P.ref_plane[kv] + rec * 64 + 4 * j) = w;
-      if ((j & 3) == 0)
-        *reinterpret_cast<uint32_t*>(P.ref_meta[kv] + rec * 16 + 4 * (j >> 2)) = half2_bits(s_h, z_h);
+      quantize8(x, bits, g >> 3, c, s_h, z_h);
       overflow |= !(half_finite(s_h) && half_finite(z_h));
-      const float sf = __half2float(s_h), zf = __half2float(z_h);
+      if (bits == 2) {
+        uint32_t w = 0;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ref[e] = __fadd_rn(zf, __fmul_rn(static_cast<float>(c[e]), sf));
-    }
-  }
-  float refref = 0.f;
-  bool have_refref = false;
-
-  // ---- residual loops
-  for (int l = 0; l < P.L - 1; ++l) {
-    float x[8];
-    load8_bf16(X + static_cast<int64_t>(l) * P.s_l + src0, x);
-    bad |= !in_range8(x);
-    float a = 0.f;
-    const int mode = P.alpha_mode[l];
-    if (mode == RQ_ALPHA_LS) {
-      if (!have_refref) {
-        refref = tree_dot(ref, ref);
-        have_refref = true;
+        for (int e = 0; e < 8; ++e) w |= c[e] << (2 * e);
+        *reinterpret_cast<uint16_t*>(P.codes[l][kv] + rec * 32 + 2 * j) = static_cast<uint16_t>(w);
+      } else {
+        uint32_t w = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w |= c[e] << (4 * e);
+        *reinterpret_cast<uint32_t*>(P.codes[l][kv] + rec * 64 + 4 * j) = w;
       }
-      const float num = tree_dot(x, ref);
-      a = (refref == 0.f) ? 0.f : __fdiv_rn(num, refref);
-    } else if (mode == RQ_ALPHA_ONE) {
-      a = 1.f;
+      const int lpg = g >> 3;
+      if ((j % lpg) == 0)
+        *reinterpret_cast<uint32_t*>(P.meta[l][kv] + rec * (4 * (kD / g)) + 4 * (j / lpg)) =
+            half2_bits(s_h, z_h);
     }
-    const __half a_h = __float2half_rn(a);
-    overflow |= !half_finite(a_h);
-    if (j == 0)
-      *reinterpret_cast<__half*>(P.alpha[l] + rec * 4 + 2 * kv) = a_h;
-    const float af = __half2float(a_h);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], __fmul_rn(af, ref[e]));
-    if (P.rotate[l]) fwht128(x, j);
-    const int bits = P.bits[l], g = P.group[l];
-    uint32_t c[8];
-    __half s_h, z_h;
-    quantize8(x, bits, g >> 3, c, s_h, z_h);
-    overflow |= !(half_finite(s_h) && half_finite(z_h));
-    if (bits == 2) {
-      uint32_t w = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w |= c[e] << (2 * e);
-      *reinterpret_cast<uint16_t*>(P.codes[l][kv] + rec * 32 + 2 * j) = static_cast<uint16_t>(w);
-    } else {
-      uint32_t w = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w |= c[e] << (4 * e);
-      *reinterpret_cast<uint32_t*>(P.codes[l][kv] + rec * 64 + 4 * j) = w;
-    }
-    const int lpg = g >> 3;
-    if ((j % lpg) == 0)
-      *reinterpret_cast<uint32_t*>(P.meta[l][kv] + rec * (4 * (kD / g)) + 4 * (j / lpg)) =
-          half2_bits(s_h, z_h);
   }
   const unsigned any_bad = __ballot_sync(kFull, bad);
   const unsigned any_ovf = __ballot_sync(kFull, overflow);

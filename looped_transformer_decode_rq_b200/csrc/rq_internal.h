@@ -23,13 +23,13 @@ struct EncodeParams {
   const uint16_t* k;         // bf16 bits
   const uint16_t* v;
   int64_t s_l, s_b, s_h, s_t;  // element strides
-  int ref_bits;                // 16 | 4
-  uint8_t* ref_plane[2];
-  uint8_t* ref_meta[2];
+  // per loop: anchors (anchor[l] == l) store bf16 values or INT4 codes + meta
+  // in codes/meta; the others store residual codes, meta and alpha
   uint8_t* codes[RQ_MAX_LOOPS][2];
   uint8_t* meta[RQ_MAX_LOOPS][2];
   uint8_t* alpha[RQ_MAX_LOOPS];
   int bits[RQ_MAX_LOOPS], group[RQ_MAX_LOOPS], rotate[RQ_MAX_LOOPS], alpha_mode[RQ_MAX_LOOPS];
+  int anchor[RQ_MAX_LOOPS];
   int32_t* status;
 };
 
@@ -40,7 +40,7 @@ struct ReconstructParams {
   int ref_bits;
   const uint8_t* ref_plane[2];
   const uint8_t* ref_meta[2];
-  int is_ref;  // reconstruct the reference loop itself
+  int is_ref;  // reconstruct the anchor loop itself
   const uint8_t* codes[2];
   const uint8_t* meta[2];
   const uint8_t* alpha;
@@ -48,7 +48,7 @@ struct ReconstructParams {
   float* out[2];
 };
 
-// One decode call: either a residual loop of a cache, its reference loop, or a
+// One decode call: either a residual loop of a cache, an anchor loop, or a
 // plain bf16 cache.  Planes are indexed by record = (b*Hkv + h)*plane_tokens + t.
 struct DecodeParams {
   int B, Hkv, G;

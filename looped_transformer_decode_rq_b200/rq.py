@@ -29,7 +29,8 @@ MAX_BATCH = 1024
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_FLAG = range(7)
 FLAG_BAD_INPUT, FLAG_POSITION, FLAG_CTX_LEN, FLAG_PIPE_TIMEOUT, FLAG_META_OVERFLOW = 1, 2, 4, 8, 16
-ALPHA_LS, ALPHA_ONE, ALPHA_ZERO = 0, 1, 2
+ALPHA_LS, ALPHA_ONE, ALPHA_ZERO, ALPHA_NORM_RATIO = 0, 1, 2, 3
+ANCHOR_LAST, ANCHOR_FIRST, ANCHOR_INTERVAL = 0, 1, 2
 
 # every symbol the header declares (checked by the ABI tests)
 EXPORTED = ("rq_cache_layout", "rq_cache_create", "rq_cache_destroy", "rq_cache_info", "rq_encode",
@@ -43,16 +44,15 @@ class Config(C.Structure):
     _fields_ = [("num_loops", C.c_int32), ("batch", C.c_int32), ("kv_heads", C.c_int32),
                 ("q_heads", C.c_int32), ("head_dim", C.c_int32), ("capacity", C.c_int32),
                 ("bits", C.c_int32 * MAX_LOOPS), ("group", C.c_int32 * MAX_LOOPS),
-                ("rotate", C.c_int32 * MAX_LOOPS), ("alpha_mode", C.c_int32 * MAX_LOOPS)]
+                ("rotate", C.c_int32 * MAX_LOOPS), ("alpha_mode", C.c_int32 * MAX_LOOPS),
+                ("anchor_policy", C.c_int32), ("anchor_interval", C.c_int32)]
 
 
 class Layout(C.Structure):
     _fields_ = [("capacity_padded", C.c_int64), ("total_bytes", C.c_int64), ("status_offset", C.c_int64),
-                ("ref_offset", C.c_int64 * 2), ("ref_meta_offset", C.c_int64 * 2),
-                ("ref_record_bytes", C.c_int64), ("ref_meta_record_bytes", C.c_int64),
                 ("codes_offset", (C.c_int64 * 2) * MAX_LOOPS), ("meta_offset", (C.c_int64 * 2) * MAX_LOOPS),
                 ("alpha_offset", C.c_int64 * MAX_LOOPS), ("codes_record_bytes", C.c_int64 * MAX_LOOPS),
-                ("meta_record_bytes", C.c_int64 * MAX_LOOPS)]
+                ("meta_record_bytes", C.c_int64 * MAX_LOOPS), ("anchor_of", C.c_int32 * MAX_LOOPS)]
 
 
 _vp, _i32, _i64, _f32 = C.c_void_p, C.c_int32, C.c_int64, C.c_float
@@ -103,10 +103,12 @@ def _stream(stream=None) -> Optional[int]:
 
 def make_config(num_loops: int, batch: int, kv_heads: int, q_heads: int, capacity: int,
                 bits: Sequence[int], group: Sequence[int], rotate: Sequence[int],
-                alpha_mode: Sequence[int], head_dim: int = HEAD_DIM) -> Config:
+                alpha_mode: Sequence[int], head_dim: int = HEAD_DIM, anchor_policy: int = ANCHOR_LAST,
+                anchor_interval: int = 0) -> Config:
     c = Config()
     c.num_loops, c.batch, c.kv_heads, c.q_heads, c.head_dim, c.capacity = (
         num_loops, batch, kv_heads, q_heads, head_dim, capacity)
+    c.anchor_policy, c.anchor_interval = anchor_policy, anchor_interval
     for i in range(min(num_loops, MAX_LOOPS, len(bits))):
         c.bits[i], c.group[i], c.rotate[i], c.alpha_mode[i] = bits[i], group[i], rotate[i], alpha_mode[i]
     return c
@@ -114,7 +116,8 @@ def make_config(num_loops: int, batch: int, kv_heads: int, q_heads: int, capacit
 
 def config_from_dict(d: dict) -> Config:
     return make_config(d["num_loops"], d["batch"], d["kv_heads"], d["q_heads"], d["capacity"], d["bits"],
-                       d["group"], d["rotate"], d["alpha_mode"], d.get("head_dim", HEAD_DIM))
+                       d["group"], d["rotate"], d["alpha_mode"], d.get("head_dim", HEAD_DIM),
+                       d.get("anchor_policy", ANCHOR_LAST), d.get("anchor_interval", 0))
 
 
 def cache_layout(cfg: Config) -> Layout:

@@ -59,6 +59,8 @@ class Workload:
     n_tail: int = 1
     seed: int = 0
     layers: int = 1
+    anchor_policy: int = 0      # 0: final loop is the reference; 1: loop 0; 2: blocks of anchor_interval
+    anchor_interval: int = 0
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -190,4 +192,5 @@ def cache_config_dict(wl: Workload, capacity: Optional[int] = None) -> dict:
                 q_heads=wl.q_heads, head_dim=wl.head_dim,
                 capacity=capacity if capacity is not None else wl.context + wl.n_tail,
                 bits=list(wl.bits), group=list(wl.group), rotate=list(wl.rotate),
-                alpha_mode=list(wl.alpha_mode))
+                alpha_mode=list(wl.alpha_mode), anchor_policy=wl.anchor_policy,
+                anchor_interval=wl.anchor_interval)

@@ -65,7 +65,8 @@ F16 = np.float16
 INV_SQRT_D_F32 = np.float32(1.0 / np.sqrt(128.0))
 FP16_MAX = 65504.0
 
-ALPHA_LS, ALPHA_ONE, ALPHA_ZERO = 0, 1, 2
+ALPHA_LS, ALPHA_ONE, ALPHA_ZERO, ALPHA_NORM = 0, 1, 2, 3
+ANCHOR_LAST, ANCHOR_FIRST, ANCHOR_INTERVAL = 0, 1, 2
 
 
 # ---------------------------------------------------------------------------
@@ -124,13 +125,22 @@ def lane_tree_dot_fp32(a: np.ndarray, b: np.ndarray) -> np.ndarray:
 def ls_alpha_fp32(x: np.ndarray, ref: np.ndarray, mode: int = ALPHA_LS) -> np.ndarray:
     """Stored (fp16) scale alpha_hat per vector; x, ref float32 [..., 128].
 
-    LS mode: alpha = <x, ref> / <ref, ref>, the minimiser of ||x - a ref||^2.
+    LS mode: alpha = <x, ref> / <ref, ref>, the minimiser of ||x - a ref||^2
+    ([RQ] Figure 1 step 3).  Norm-ratio mode ([RQ] Table 9, "Norm-ratio"):
+    alpha = ||x|| / ||ref||, each norm the correctly rounded square root of
+    the same fixed-order dot product.
     """
     lead = np.asarray(x).shape[:-1]
     if mode == ALPHA_ONE:
         return np.ones(lead, dtype=F16)
     if mode == ALPHA_ZERO:
         return np.zeros(lead, dtype=F16)
+    if mode == ALPHA_NORM:
+        nx = np.sqrt(lane_tree_dot_fp32(x, x)).astype(F32)
+        nr = np.sqrt(lane_tree_dot_fp32(ref, ref)).astype(F32)
+        with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
+            alpha = np.where(nr == 0, F32(0), nx / np.where(nr == 0, F32(1), nr)).astype(F32)
+            return alpha.astype(F16)
     num = lane_tree_dot_fp32(x, ref)
     den = lane_tree_dot_fp32(ref, ref)
     with np.errstate(divide="ignore", invalid="ignore", over="ignore"):
@@ -201,20 +211,45 @@ def dequant_f64(codes: np.ndarray, scale: np.ndarray, zero: np.ndarray, g: int) 
 
 @dataclass
 class CacheConfig:
+    """Per-loop formats and which loop each loop takes as its reference.
+
+    Anchor policies ([RQ] Table 1 "First-loop" / "Last-loop"; Table 8 anchor
+    intervals "N x [2^n, 4]", each group ending in its own anchor):
+      ANCHOR_LAST: the final loop is every loop's reference;
+      ANCHOR_FIRST: loop 0 is every loop's reference;
+      ANCHOR_INTERVAL: blocks of `anchor_interval` consecutive loops, the last
+        loop of each block (or the final loop, for a short last block) being
+        the reference of the others in its block.
+    Anchor loops use bits 16 (bf16) or 4 (INT4, g = 32); the others 2 or 4.
+    """
     num_loops: int
-    bits: Sequence[int]        # per loop; last = reference: 16 (bf16) or 4 (INT4 g=32)
+    bits: Sequence[int]
     group: Sequence[int]
     rotate: Sequence[int]
     alpha_mode: Sequence[int]
+    anchor_policy: int = ANCHOR_LAST
+    anchor_interval: int = 0
 
     @staticmethod
     def from_dict(d: dict) -> "CacheConfig":
         return CacheConfig(d["num_loops"], list(d["bits"]), list(d["group"]),
-                           list(d["rotate"]), list(d["alpha_mode"]))
+                           list(d["rotate"]), list(d["alpha_mode"]),
+                           d.get("anchor_policy", ANCHOR_LAST), d.get("anchor_interval", 0))
 
-    @property
-    def ref(self) -> int:
-        return self.num_loops - 1
+    def anchor_of(self, loop: int) -> int:
+        L = self.num_loops
+        if self.anchor_policy == ANCHOR_LAST:
+            return L - 1
+        if self.anchor_policy == ANCHOR_FIRST:
+            return 0
+        n = self.anchor_interval
+        return min((loop // n) * n + n - 1, L - 1)
+
+    def is_anchor(self, loop: int) -> bool:
+        return self.anchor_of(loop) == loop
+
+    def anchors(self) -> List[int]:
+        return sorted({self.anchor_of(l) for l in range(self.num_loops)})
 
 
 @dataclass
@@ -233,10 +268,11 @@ class EncodedPlane:
 @dataclass
 class Encoded:
     cfg: CacheConfig
-    ref_bf16: Dict[str, np.ndarray] = field(default_factory=dict)      # 'k','v' float32 values
-    ref_q: Dict[str, EncodedPlane] = field(default_factory=dict)       # INT4 anchor
-    ref_hat32: Dict[str, np.ndarray] = field(default_factory=dict)     # encoder's fp32 view of ref
-    loops: List[Dict[str, EncodedPlane]] = field(default_factory=list)
+    # per anchor loop a: 'k'/'v' float32 bf16 values, or the INT4 EncodedPlane
+    anchor_bf16: Dict[int, Dict[str, np.ndarray]] = field(default_factory=dict)
+    anchor_q: Dict[int, Dict[str, EncodedPlane]] = field(default_factory=dict)
+    anchor_hat32: Dict[int, Dict[str, np.ndarray]] = field(default_factory=dict)  # encoder's fp32 view
+    loops: List[Optional[Dict[str, EncodedPlane]]] = field(default_factory=list)  # None for anchors
     error: bool = False
 
 
@@ -254,23 +290,28 @@ def encode_fp32emu(K: np.ndarray, V: np.ndarray, cfg: CacheConfig) -> Encoded:
     assert K.shape[0] == L and V.shape == K.shape
     enc = Encoded(cfg=cfg)
     enc.error = not (_check_range(K) and _check_range(V))
-    rb = cfg.bits[cfg.ref]
-    for name, X in (("k", K), ("v", V)):
-        ref = np.asarray(X[cfg.ref], dtype=F32)
-        if rb == 16:
-            enc.ref_bf16[name] = ref
-            enc.ref_hat32[name] = ref
-        elif rb == 4:
-            qg = quantize_groups_fp32(ref, 4, 32)
-            enc.ref_q[name] = EncodedPlane(qg.codes, qg.scale, qg.zero, None, qg.near_tie, 4, 32, 0)
-            enc.ref_hat32[name] = dequant_fp32(qg, 32)
-        else:
-            raise ValueError("reference bits must be 16 or 4")
-    for l in range(L - 1):
+    for a in cfg.anchors():
+        rb = cfg.bits[a]
+        enc.anchor_bf16[a], enc.anchor_q[a], enc.anchor_hat32[a] = {}, {}, {}
+        for name, X in (("k", K), ("v", V)):
+            ref = np.asarray(X[a], dtype=F32)
+            if rb == 16:
+                enc.anchor_bf16[a][name] = ref
+                enc.anchor_hat32[a][name] = ref
+            elif rb == 4:
+                qg = quantize_groups_fp32(ref, 4, 32)
+                enc.anchor_q[a][name] = EncodedPlane(qg.codes, qg.scale, qg.zero, None, qg.near_tie, 4, 32, 0)
+                enc.anchor_hat32[a][name] = dequant_fp32(qg, 32)
+            else:
+                raise ValueError("anchor bits must be 16 or 4")
+    for l in range(L):
+        if cfg.is_anchor(l):
+            enc.loops.append(None)
+            continue
         planes = {}
         for name, X in (("k", K), ("v", V)):
             x = np.asarray(X[l], dtype=F32)
-            ref = enc.ref_hat32[name]
+            ref = enc.anchor_hat32[cfg.anchor_of(l)][name]
             a_hat = ls_alpha_fp32(x, ref, cfg.alpha_mode[l])
             if not np.all(np.isfinite(a_hat.astype(np.float64))):
                 enc.error = True
@@ -291,11 +332,13 @@ def encode_fp32emu(K: np.ndarray, V: np.ndarray, cfg: CacheConfig) -> Encoded:
 # Reconstruction (float64)
 # ---------------------------------------------------------------------------
 
-def reference_f64(enc: Encoded, name: str) -> np.ndarray:
-    """The decoder's reference: exact bf16 values, or the INT4 anchor dequantised in float64."""
-    if enc.cfg.bits[enc.cfg.ref] == 16:
-        return enc.ref_bf16[name].astype(np.float64)
-    p = enc.ref_q[name]
+def reference_f64(enc: Encoded, name: str, anchor: Optional[int] = None) -> np.ndarray:
+    """The decoder's view of an anchor loop (default: the final loop): exact
+    bf16 values, or the INT4 anchor dequantised in float64."""
+    a = enc.cfg.num_loops - 1 if anchor is None else anchor
+    if enc.cfg.bits[a] == 16:
+        return enc.anchor_bf16[a][name].astype(np.float64)
+    p = enc.anchor_q[a][name]
     return dequant_f64(p.codes, p.scale, p.zero, 32)
 
 
@@ -309,12 +352,13 @@ def residual_f64(p: EncodedPlane) -> np.ndarray:
 
 def reconstruct_f64(enc: Encoded, loop: int):
     """(K_hat, V_hat) float64 of one loop: alpha_hat * ref + H^T deq(codes)."""
-    if loop == enc.cfg.ref:
-        return reference_f64(enc, "k"), reference_f64(enc, "v")
+    a = enc.cfg.anchor_of(loop)
+    if loop == a:
+        return reference_f64(enc, "k", a), reference_f64(enc, "v", a)
     out = []
     for name in ("k", "v"):
         p = enc.loops[loop][name]
-        ref = reference_f64(enc, name)
+        ref = reference_f64(enc, name, a)
         out.append(p.alpha.astype(np.float64)[..., None] * ref + residual_f64(p))
     return out[0], out[1]
 
@@ -348,13 +392,14 @@ def decode_attention_f64(enc: Encoded, loop: int, q: np.ndarray, ctx_len: np.nda
     cfg = enc.cfg
     q = np.asarray(q, dtype=np.float64)
     B, Hq, _ = q.shape
-    refk = reference_f64(enc, "k")
-    refv = reference_f64(enc, "v")
+    a = cfg.anchor_of(loop)
+    refk = reference_f64(enc, "k", a)
+    refv = reference_f64(enc, "v", a)
     Hkv = refk.shape[1]
     G = Hq // Hkv
     Hn = hadamard_orthonormal(D)
     out = np.zeros((B, Hq, D))
-    is_ref = loop == cfg.ref
+    is_ref = loop == a
     if not is_ref:
         pk, pv = enc.loops[loop]["k"], enc.loops[loop]["v"]
         yk = dequant_f64(pk.codes, pk.scale, pk.zero, pk.group)

@@ -51,16 +51,21 @@ def read_planes(cache, n_tokens: int):
     def grab(off, rec):
         return cache.plane(off, rec)[:, :, :n_tokens].cpu().numpy()
 
-    ref_bits = cfg.bits[L - 1]
-    for kv, name in enumerate("kv"):
-        if ref_bits == 16:
-            raw = grab(lay.ref_offset[kv], 256)
-            out["ref"][name] = raw.view("<u2")
-        else:
-            codes = unpack_codes(grab(lay.ref_offset[kv], 64), 4)
-            s, z = unpack_meta(grab(lay.ref_meta_offset[kv], 16))
-            out["ref"][name] = (codes, s, z)
-    for l in range(L - 1):
+    for l in range(L):
+        if lay.alpha_offset[l] >= 0:
+            continue
+        out["ref"][l] = {}
+        for kv, name in enumerate("kv"):
+            if cfg.bits[l] == 16:
+                out["ref"][l][name] = grab(lay.codes_offset[l][kv], 256).view("<u2")
+            else:
+                codes = unpack_codes(grab(lay.codes_offset[l][kv], 64), 4)
+                s, z = unpack_meta(grab(lay.meta_offset[l][kv], 16))
+                out["ref"][l][name] = (codes, s, z)
+    for l in range(L):
+        if lay.alpha_offset[l] < 0:
+            out["loops"].append(None)
+            continue
         d = {}
         for kv, name in enumerate("kv"):
             codes = unpack_codes(grab(lay.codes_offset[l][kv], lay.codes_record_bytes[l]), cfg.bits[l])
@@ -83,19 +88,23 @@ def compare_encoded(planes: dict, enc: O.Encoded) -> dict:
     rounding near-tie.  Returns counts; raises AssertionError on mismatch."""
     stats = {"codes": 0, "near_tie": 0, "near_tie_diff": 0}
     cfg = enc.cfg
-    if cfg.bits[cfg.ref] == 16:
+    assert sorted(planes["ref"]) == cfg.anchors()
+    for a in cfg.anchors():
         for name in "kv":
-            want = enc.ref_bf16[name].view(np.uint32) >> 16
-            assert np.array_equal(planes["ref"][name].astype(np.uint32), want), f"ref {name} copy differs"
-    else:
-        for name in "kv":
-            codes, s, z = planes["ref"][name]
-            p = enc.ref_q[name]
-            assert np.array_equal(s.view(np.uint16), p.scale.view(np.uint16)), f"ref {name} scale differs"
-            assert np.array_equal(z.view(np.uint16), p.zero.view(np.uint16)), f"ref {name} zero differs"
-            diff = codes != p.codes
-            assert not np.any(diff & ~p.near_tie), f"ref {name} codes differ at {np.argwhere(diff & ~p.near_tie)[:5]}"
+            if cfg.bits[a] == 16:
+                want = enc.anchor_bf16[a][name].view(np.uint32) >> 16
+                assert np.array_equal(planes["ref"][a][name].astype(np.uint32), want), f"anchor {a} {name} differs"
+            else:
+                codes, s, z = planes["ref"][a][name]
+                p = enc.anchor_q[a][name]
+                assert np.array_equal(s.view(np.uint16), p.scale.view(np.uint16)), f"anchor {a} {name} scale differs"
+                assert np.array_equal(z.view(np.uint16), p.zero.view(np.uint16)), f"anchor {a} {name} zero differs"
+                diff = codes != p.codes
+                assert not np.any(diff & ~p.near_tie), f"anchor {a} {name} codes differ"
     for l, d in enumerate(planes["loops"]):
+        if d is None:
+            assert cfg.is_anchor(l)
+            continue
         ak, av = d["alpha"]
         assert np.array_equal(ak.view(np.uint16), enc.loops[l]["k"].alpha.view(np.uint16)), f"loop {l} alpha_K differs"
         assert np.array_equal(av.view(np.uint16), enc.loops[l]["v"].alpha.view(np.uint16)), f"loop {l} alpha_V differs"

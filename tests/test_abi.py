@@ -48,21 +48,22 @@ def _cfg(librq, **kw):
 def test_layout_bytes_per_token_head(librq):
     lay = librq.cache_layout(_cfg(librq))
     assert lay.capacity_padded == 8192
-    assert lay.ref_record_bytes == 256 and lay.ref_meta_offset[0] == -1
+    assert lay.codes_record_bytes[3] == 256 and lay.meta_offset[3][0] == -1 and lay.alpha_offset[3] == -1
+    assert list(lay.anchor_of)[:4] == [3, 3, 3, 3]
     per = 2 * 256 + sum(2 * lay.codes_record_bytes[l] + 2 * lay.meta_record_bytes[l] + 4 for l in range(3))
     assert per == 2 * 256 + 3 * (2 * 32 + 2 * 16 + 4)   # 812 B per (b, h, token) over all loops
     recs = 16 * 16 * 8192
     assert lay.total_bytes >= per * recs
     assert lay.total_bytes - per * recs <= 1024 * 16
-    offs = [lay.ref_offset[0], lay.ref_offset[1]] + [lay.codes_offset[l][kv] for l in range(3) for kv in range(2)]
+    offs = [lay.codes_offset[l][kv] for l in range(4) for kv in range(2)]
     assert all(o % 1024 == 0 for o in offs)
-    assert lay.codes_offset[3][0] == -1
+    assert lay.codes_offset[4][0] == -1
 
 
 def test_layout_int4_anchor_and_padding(librq):
     lay = librq.cache_layout(_cfg(librq, capacity=100, bits=[2, 2, 4, 4]))
     assert lay.capacity_padded == 128
-    assert lay.ref_record_bytes == 64 and lay.ref_meta_record_bytes == 16
+    assert lay.codes_record_bytes[3] == 64 and lay.meta_record_bytes[3] == 16
     assert lay.codes_record_bytes[2] == 64 and lay.meta_record_bytes[2] == 16
     lay16 = librq.cache_layout(_cfg(librq, group=[16, 16, 16, 32]))
     assert lay16.meta_record_bytes[0] == 32
@@ -72,7 +73,7 @@ def test_layout_int4_anchor_and_padding(librq):
     ("num_loops", 1, 1), ("num_loops", 17, 1), ("batch", 0, 1), ("kv_heads", 0, 1),
     ("q_heads", 24, 1), ("q_heads", 48, 2), ("head_dim", 64, 2), ("capacity", 0, 1),
     ("bits", [3, 2, 2, 16], 2), ("bits", [2, 2, 2, 8], 2), ("group", [64, 32, 32, 32], 2),
-    ("group", [32, 32, 32, 16], 1), ("rotate", [2, 1, 1, 0], 1), ("alpha_mode", [3, 0, 0, 0], 1),
+    ("group", [32, 32, 32, 16], 1), ("rotate", [2, 1, 1, 0], 1), ("alpha_mode", [4, 0, 0, 0], 1),
 ])
 def test_layout_rejects_bad_config(librq, field, value, status):
     cfg = _cfg(librq, **({field: value} if field not in ("head_dim",) else {}))
@@ -124,3 +125,24 @@ def test_bf16_decode_rejects_bad_arguments(librq):
     assert call(k=4097) == 1
     assert call(strides=(C.c_int64 * 3)(16 * 128 * 64, 128 * 64, 100)) == 1
     assert call(cap=0) == 1
+
+
+def test_layout_anchor_policies(librq):
+    rq = librq
+    first = rq.cache_layout(_cfg(librq, bits=[16, 2, 2, 2], group=[32] * 4, rotate=[0, 1, 1, 1],
+                                 anchor_policy=rq.ANCHOR_FIRST))
+    assert list(first.anchor_of)[:4] == [0, 0, 0, 0]
+    assert first.alpha_offset[0] == -1 and all(first.alpha_offset[l] >= 0 for l in (1, 2, 3))
+    cfg = rq.config_from_dict(dict(num_loops=8, batch=2, kv_heads=2, q_heads=2, capacity=64,
+                                   bits=[2, 2, 2, 4, 2, 2, 2, 4], group=[32] * 8, rotate=[1, 1, 1, 0] * 2,
+                                   alpha_mode=[0] * 8, anchor_policy=rq.ANCHOR_INTERVAL, anchor_interval=4))
+    lay = rq.cache_layout(cfg)
+    assert list(lay.anchor_of)[:8] == [3, 3, 3, 3, 7, 7, 7, 7]
+    assert lay.codes_record_bytes[3] == 64 and lay.meta_record_bytes[3] == 16
+    # an anchor must be bf16 or INT4, a residual loop INT2 or INT4
+    bad = rq.config_from_dict(dict(num_loops=8, batch=2, kv_heads=2, q_heads=2, capacity=64,
+                                   bits=[2] * 8, group=[32] * 8, rotate=[1] * 8, alpha_mode=[0] * 8,
+                                   anchor_policy=rq.ANCHOR_INTERVAL, anchor_interval=4))
+    assert rq.lib().rq_cache_layout(C.byref(bad), C.byref(rq.Layout())) == rq.ERR_UNSUPPORTED
+    bad.anchor_interval = 1
+    assert rq.lib().rq_cache_layout(C.byref(bad), C.byref(rq.Layout())) == rq.ERR_INVALID_ARG

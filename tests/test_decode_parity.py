@@ -125,3 +125,17 @@ def test_bf16_cache_baseline(librq, G, lens):
         want = O.attention_f64(to_np32(inp["q"][loop]), to_np32(inp["k"][loop]), to_np32(inp["v"][loop]),
                                ctx.numpy(), to_np32(inp["k_tail"][loop]), to_np32(inp["v_tail"][loop]))
         assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
+
+
+@pytest.mark.parametrize("policy,interval,L,bits,alpha", [
+    (1, 0, 4, (16, 2, 2, 4), (0, 0, 3, 0)),                        # First-loop, norm ratio on loop 2
+    (2, 4, 8, (2, 2, 2, 4, 2, 2, 4, 16), (0,) * 8),                # 2 x [2,2,2,4]-style blocks
+    (2, 3, 7, (2, 2, 4, 2, 2, 4, 4), (0, 3, 0, 0, 1, 0, 0)),       # short last block [2, 4]
+])
+def test_anchor_policies(librq, policy, interval, L, bits, alpha):
+    rot = tuple(0 if b in (16,) else 1 for b in bits)
+    wl = synth.Workload(name=f"anchors_{policy}_{interval}", num_loops=L, batch=2, kv_heads=2, q_heads=4,
+                        context=150, bits=bits, group=(32,) * L, rotate=rot, alpha_mode=alpha,
+                        sigma=tuple(0.1 + 0.03 * i for i in range(L - 1)), anchor_policy=policy,
+                        anchor_interval=interval, outlier_p=0.01, seed=40 + policy + interval)
+    run_case(librq, wl, lengths=[150, 70])

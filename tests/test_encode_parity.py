@@ -25,6 +25,15 @@ CASES = [
     synth.Workload(name="eight_loops", num_loops=8, batch=1, kv_heads=2, q_heads=2, context=17,
                    bits=(2, 2, 2, 2, 2, 2, 2, 4), group=(16,) * 7 + (32,), rotate=(1,) * 7 + (0,),
                    alpha_mode=(0,) * 8, sigma=(0.3, 0.25, 0.2, 0.15, 0.1, 0.1, 0.05), seed=8),
+    # First-loop reference ([RQ] Table 1) with norm-ratio and LS scales ([RQ] Table 9)
+    synth.Workload(name="first_loop_norm_ratio", batch=2, kv_heads=2, q_heads=2, context=45,
+                   bits=(16, 2, 2, 4), group=(32, 32, 16, 32), rotate=(0, 1, 1, 1), alpha_mode=(0, 3, 0, 3),
+                   sigma=(0.3, 0.2, 0.1), anchor_policy=1, seed=13),
+    # anchor intervals 2 x [2^3, 4] ([RQ] Table 8), INT4 and bf16 anchors
+    synth.Workload(name="anchor_interval_2x4", num_loops=8, batch=2, kv_heads=2, q_heads=2, context=33,
+                   bits=(2, 2, 2, 4, 2, 2, 2, 16), group=(16, 32, 32, 32, 32, 16, 32, 32),
+                   rotate=(1, 1, 1, 0, 1, 1, 0, 0), alpha_mode=(0, 0, 3, 0, 0, 1, 0, 0),
+                   sigma=(0.3, 0.25, 0.2, 0.15, 0.1, 0.1, 0.05), anchor_policy=2, anchor_interval=4, seed=14),
 ]
 
 

@@ -29,13 +29,20 @@ def _slab_planes(cache, b, h, n):
         return cache.plane(off, rec)[b:b + 1, h:h + 1, :n].cpu().numpy()
 
     out = {"ref": {}, "loops": []}
-    for kv, name in enumerate("kv"):
-        if cfg.bits[L - 1] == 16:
-            out["ref"][name] = grab(lay.ref_offset[kv], 256).view("<u2")
-        else:
-            s, z = unpack_meta(grab(lay.ref_meta_offset[kv], 16))
-            out["ref"][name] = (unpack_codes(grab(lay.ref_offset[kv], 64), 4), s, z)
-    for l in range(L - 1):
+    for l in range(L):
+        if lay.anchor_of[l] != l:
+            continue
+        out["ref"][l] = {}
+        for kv, name in enumerate("kv"):
+            if cfg.bits[l] == 16:
+                out["ref"][l][name] = grab(lay.codes_offset[l][kv], 256).view("<u2")
+            else:
+                s, z = unpack_meta(grab(lay.meta_offset[l][kv], 16))
+                out["ref"][l][name] = (unpack_codes(grab(lay.codes_offset[l][kv], 64), 4), s, z)
+    for l in range(L):
+        if lay.anchor_of[l] == l:
+            out["loops"].append(None)
+            continue
         d = {}
         for kv, name in enumerate("kv"):
             s, z = unpack_meta(grab(lay.meta_offset[l][kv], lay.meta_record_bytes[l]))

@@ -29,9 +29,10 @@ def _alpha_swapped(x, ref, mode=O.ALPHA_LS):
 
 
 def _reconstruct_no_alpha(enc, loop):
-    if loop == enc.cfg.ref:
+    if enc.cfg.is_anchor(loop):
         return ORIG["reconstruct_f64"](enc, loop)
-    return tuple(O.reference_f64(enc, n) + O.residual_f64(enc.loops[loop][n]) for n in ("k", "v"))
+    a = enc.cfg.anchor_of(loop)
+    return tuple(O.reference_f64(enc, n, a) + O.residual_f64(enc.loops[loop][n]) for n in ("k", "v"))
 
 
 def _residual_unnormalised(p):
@@ -60,7 +61,7 @@ def _dequant_strided_groups(codes, scale, zero, g):
 
 
 def _decode_drop_value_alpha(enc, loop, q, ctx_len, k_tail=None, v_tail=None, scale=1 / np.sqrt(128)):
-    if loop == enc.cfg.ref:
+    if enc.cfg.is_anchor(loop):
         return ORIG["decode_attention_f64"](enc, loop, q, ctx_len, k_tail, v_tail, scale)
     saved = enc.loops[loop]["v"].alpha
     enc.loops[loop]["v"].alpha = np.ones_like(saved)

@@ -318,3 +318,91 @@ def test_p9_storage_reduction_matches_abstract():
     for printed, blocks, g, hd in _rows("storage_reduction_pages.txt"):
         b = O.effective_bitwidth(_parse_blocks(blocks), int(g), head_dim=int(hd))
         assert _round_printed(100 * (1 - b / 16), printed) == Decimal(printed)
+
+
+# ------------------------------------------- norm-ratio alpha ([RQ] Table 9)
+
+def test_norm_ratio_alpha_matches_norms():
+    rng = np.random.default_rng(91)
+    ref = bf16_values(rng, (200, 128), scale=1.3)
+    x = bf16_values(rng, (200, 128), scale=0.7)
+    a = O.ls_alpha_fp32(x, ref, O.ALPHA_NORM).astype(np.float64)
+    want = np.linalg.norm(x.astype(np.float64), axis=1) / np.linalg.norm(ref.astype(np.float64), axis=1)
+    assert np.all(np.abs(a - want) <= 0.5 * np.spacing(want.astype(np.float16)).astype(np.float64) + 1e-6 * want)
+    # a scaled copy: the ratio is |c| whatever the sign (it is not the LS scale)
+    for c in (2.0, -0.5):
+        assert np.all(O.ls_alpha_fp32(np.float32(c) * ref, ref, O.ALPHA_NORM).astype(np.float64) == abs(c))
+    assert np.all(O.ls_alpha_fp32(x, np.zeros_like(ref), O.ALPHA_NORM) == 0)
+
+
+# --------------------- anchor policies ([RQ] Table 1 First/Last-loop; Table 8)
+
+def _loops_from(ref, scales, rng):
+    return np.stack([np.float32(c) * ref for c in scales]).astype(np.float32)
+
+
+def test_anchor_of_each_policy():
+    cfg = O.CacheConfig(8, [2] * 8, [32] * 8, [1] * 8, [0] * 8, O.ANCHOR_INTERVAL, 4)
+    assert [cfg.anchor_of(l) for l in range(8)] == [3, 3, 3, 3, 7, 7, 7, 7]
+    assert cfg.anchors() == [3, 7]
+    cfg6 = O.CacheConfig(6, [2] * 6, [32] * 6, [1] * 6, [0] * 6, O.ANCHOR_INTERVAL, 4)
+    assert [cfg6.anchor_of(l) for l in range(6)] == [3, 3, 3, 3, 5, 5]
+    first = O.CacheConfig(4, [16, 2, 2, 2], [32] * 4, [0, 1, 1, 1], [0] * 4, O.ANCHOR_FIRST)
+    assert [first.anchor_of(l) for l in range(4)] == [0, 0, 0, 0]
+    last = O.CacheConfig(4, [2, 2, 2, 16], [32] * 4, [1, 1, 1, 0], [0] * 4)
+    assert [last.anchor_of(l) for l in range(4)] == [3, 3, 3, 3]
+
+
+def test_interval_of_all_loops_equals_last_loop_policy():
+    rng = np.random.default_rng(92)
+    ref = bf16_values(rng, (1, 2, 11, 128))
+    K = np.stack([bf16_values(rng, (1, 2, 11, 128)) for _ in range(3)] + [ref])
+    V = np.stack([bf16_values(rng, (1, 2, 11, 128)) for _ in range(3)] + [ref])
+    a = O.encode_fp32emu(K, V, O.CacheConfig(4, [2, 2, 4, 4], [32] * 4, [1, 1, 1, 0], [0] * 4))
+    b = O.encode_fp32emu(K, V, O.CacheConfig(4, [2, 2, 4, 4], [32] * 4, [1, 1, 1, 0], [0] * 4, O.ANCHOR_INTERVAL, 4))
+    for l in range(3):
+        for n in "kv":
+            assert np.array_equal(a.loops[l][n].codes, b.loops[l][n].codes)
+            assert np.array_equal(a.loops[l][n].alpha, b.loops[l][n].alpha)
+
+
+@pytest.mark.parametrize("policy,interval", [(O.ANCHOR_FIRST, 0), (O.ANCHOR_INTERVAL, 3)])
+def test_scaled_copies_of_their_anchor_have_zero_residual(policy, interval):
+    rng = np.random.default_rng(93)
+    L = 6
+    cfg = O.CacheConfig(L, [2] * L, [32] * L, [1] * L, [0] * L, policy, interval)
+    bits = list(cfg.bits)
+    for l in range(L):
+        if cfg.is_anchor(l):
+            bits[l] = 16
+            cfg.rotate[l] = 0
+    cfg.bits = bits
+    base = {a: bf16_values(rng, (1, 1, 7, 128)) for a in cfg.anchors()}
+    scales = [1.0, -2.0, 0.5, 2.0, -1.0, 0.5]
+    K = np.stack([np.float32(scales[l]) * base[cfg.anchor_of(l)] if not cfg.is_anchor(l) else base[l]
+                  for l in range(L)]).astype(np.float32)
+    enc = O.encode_fp32emu(K, K.copy(), cfg)
+    for l in range(L):
+        kh, _ = O.reconstruct_f64(enc, l)
+        assert np.array_equal(kh, K[l].astype(np.float64))
+        if not cfg.is_anchor(l):
+            assert np.all(enc.loops[l]["k"].codes == 0)
+            assert np.all(enc.loops[l]["k"].alpha.astype(np.float64) == scales[l])
+
+
+def test_anchor_interval_decode_equals_brute_force():
+    rng = np.random.default_rng(94)
+    L, B, H, T = 8, 2, 2, 19
+    cfg = O.CacheConfig(L, [2, 2, 2, 4, 2, 4, 2, 16], [32, 16, 32, 32, 32, 32, 16, 32],
+                        [1, 1, 0, 0, 1, 0, 1, 0], [0, 3, 0, 0, 1, 0, 0, 0], O.ANCHOR_INTERVAL, 4)
+    K = np.stack([bf16_values(rng, (B, H, T, 128)) for _ in range(L)])
+    V = np.stack([bf16_values(rng, (B, H, T, 128)) for _ in range(L)])
+    enc = O.encode_fp32emu(K, V, cfg)
+    q = bf16_values(rng, (B, 2 * H, 128))
+    kt, vt = bf16_values(rng, (B, H, 1, 128)), bf16_values(rng, (B, H, 1, 128))
+    ctx = np.array([19, 4])
+    for loop in range(L):
+        got = O.decode_attention_f64(enc, loop, q, ctx, kt, vt)
+        Kh, Vh = O.reconstruct_f64(enc, loop)
+        want = O.attention_f64(q, Kh, Vh, ctx, kt, vt)
+        assert np.abs(got - want).max() <= 1e-12 * max(1.0, np.abs(want).max())
