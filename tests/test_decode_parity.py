@@ -139,3 +139,12 @@ def test_anchor_policies(librq, policy, interval, L, bits, alpha):
                         sigma=tuple(0.1 + 0.03 * i for i in range(L - 1)), anchor_policy=policy,
                         anchor_interval=interval, outlier_p=0.01, seed=40 + policy + interval)
     run_case(librq, wl, lengths=[150, 70])
+
+
+@pytest.mark.parametrize("n_tail", [64, 127])
+def test_recent_window_bf16_tail(librq, n_tail):
+    """A window of the most recent 64-127 tokens kept in bf16 next to the compact
+    cache ([RQ] Table 10: "Recent 64" / "Recent 64-127" bf16 KV tokens)."""
+    wl = synth.Workload(name=f"tail{n_tail}", batch=2, kv_heads=2, q_heads=4, context=200, bits=(2, 2, 4, 4),
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, seed=50 + n_tail)
+    run_case(librq, wl, lengths=[200, 0], n_tail=n_tail)
