@@ -203,10 +203,12 @@ def read_profile_traffic(kernel_hash):
             vals[k.strip()] = v.strip()
     if vals.get("kernel_source_sha256_16") != kernel_hash:
         return None
-    try:
-        return int(vals["dram_bytes_per_launch_scaled"])
-    except (KeyError, ValueError):
-        return None
+    for key in ("dram_bytes_per_launch", "dram_bytes_per_launch_scaled"):
+        try:
+            return int(vals[key])
+        except (KeyError, ValueError):
+            continue
+    return None
 
 
 def load_peaks():
