@@ -187,6 +187,29 @@ RQ_API rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const 
                     int32_t start_pos, const int32_t* positions, int32_t n_tokens,
                     rq_stream_t stream);
 
+/* Decode kernel selection (not a numerical choice: both kernels compute the
+ * same attention within the decode tolerance).
+ *  RQ_DECODE_KERNEL_SIMT    split kernel on the CUDA cores, 64-token pages,
+ *                           integer dot products for scores and paired fp32
+ *                           FMAs for values; every G.
+ *  RQ_DECODE_KERNEL_TENSOR  split kernel on the tensor cores (tcgen05), 128-token
+ *                           pages: bf16 and int8 MMAs for the scores of all G
+ *                           query heads of a kv-head at once and for the
+ *                           probability-weighted value sums; G in {2, 4, 8}.
+ *  RQ_DECODE_KERNEL_AUTO    the tensor-core kernel for G >= 4 where it has a
+ *                           variant, else the CUDA-core kernel (the default). */
+typedef enum {
+  RQ_DECODE_KERNEL_AUTO = 0,
+  RQ_DECODE_KERNEL_SIMT = 1,
+  RQ_DECODE_KERNEL_TENSOR = 2
+} rq_decode_kernel;
+
+/* Sets the decode kernel of later rq_decode_attention calls on this handle.
+ * RQ_DECODE_KERNEL_TENSOR for a loop format or G it has no variant for makes
+ * those calls return RQ_ERR_UNSUPPORTED.  Not thread-safe against concurrent
+ * decode calls on the same handle. */
+RQ_API rq_status rq_cache_set_decode_kernel(rq_cache* cache, int32_t kernel);
+
 /* Bytes of workspace rq_decode_attention needs for this cache on the current
  * device (split-K partials; independent of context length). */
 RQ_API rq_status rq_decode_workspace_size(const rq_cache* cache, int64_t* bytes_out);
@@ -200,8 +223,9 @@ RQ_API rq_status rq_decode_workspace_size(const rq_cache* cache, int64_t* bytes_
  *       + sum_tail p_j v_tail,j ) / sum p
  * with one inverse rotation per (b, q-head), ref being the loop's anchor.  An
  * anchor loop is plain attention over its bf16 or INT4 planes.  n_tail current tokens (bf16,
- * not yet encoded) join the softmax.  Split-K over 64-token pages with an
- * online softmax, merged by a second kernel.
+ * not yet encoded) join the softmax.  Split-K over pages (64 tokens on the
+ * CUDA-core kernel, 128 on the tensor-core kernel) with an online softmax,
+ * merged by a second kernel.
  *
  *  q          device bf16 [B][Hq][128]
  *  ctx_len    device int32 [B], each in [0, capacity] (clamped, RQ_FLAG_CTX_LEN)

@@ -21,6 +21,7 @@ struct rq_cache {
   uint8_t* base;
   int device;
   int num_ctas;
+  int decode_kernel;                     // rq_decode_kernel
   bool tmaps_ready[RQ_MAX_LOOPS];        // per bf16 anchor loop
   CUtensorMap tm_anchor[RQ_MAX_LOOPS][2];
 };
@@ -232,12 +233,21 @@ rq_status rq_cache_create(const rq_config* cfg, void* device_buffer, int64_t buf
   c->base = static_cast<uint8_t*>(device_buffer);
   c->device = dev;
   c->num_ctas = rq::decode_grid_ctas(dev);
+  c->decode_kernel = RQ_DECODE_KERNEL_AUTO;
   for (int l = 0; l < RQ_MAX_LOOPS; ++l) c->tmaps_ready[l] = false;
   *out = c;
   return RQ_OK;
 }
 
 void rq_cache_destroy(rq_cache* cache) { delete cache; }
+
+rq_status rq_cache_set_decode_kernel(rq_cache* cache, int32_t kernel) {
+  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  if (kernel != RQ_DECODE_KERNEL_AUTO && kernel != RQ_DECODE_KERNEL_SIMT && kernel != RQ_DECODE_KERNEL_TENSOR)
+    return fail(RQ_ERR_INVALID_ARG, "decode kernel %d", kernel);
+  cache->decode_kernel = kernel;
+  return RQ_OK;
+}
 
 rq_status rq_cache_info(const rq_cache* cache, rq_config* cfg_out, rq_layout* layout_out) {
   if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
@@ -361,8 +371,9 @@ rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void*
   const int ref_kind = ref_kind_for(c, loop);
   const int res_bits = loop == a ? 0 : c.bits[loop];
   const int res_group = loop == a ? 32 : c.group[loop];
-  if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G))
-    return fail(RQ_ERR_UNSUPPORTED, "no decode kernel for this loop format");
+  if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G, cache->decode_kernel))
+    return fail(RQ_ERR_UNSUPPORTED, "no %s decode kernel for this loop format and G = %d",
+                cache->decode_kernel == RQ_DECODE_KERNEL_TENSOR ? "tensor-core" : "", G);
   if (ref_kind == rq::kRefBf16 && !cache->tmaps_ready[a]) {
     const int64_t cp = lay.capacity_padded;
     for (int kv = 0; kv < 2; ++kv) {
@@ -403,7 +414,8 @@ rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void*
   p.partials = static_cast<float*>(workspace);
   p.num_ctas = cache->num_ctas;
   p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
-  cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, &cache->tm_anchor[a][0],
+  p.tma_tokens = lay.capacity_padded;
+  cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, cache->decode_kernel, &cache->tm_anchor[a][0],
                                     &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return RQ_OK;
@@ -456,7 +468,9 @@ rq_status rq_bf16_decode_attention(int32_t batch, int32_t kv_heads, int32_t q_he
   p.partials = static_cast<float*>(workspace);
   p.num_ctas = rq::decode_grid_ctas(dev);
   p.status = status_word;
-  cudaError_t e = rq::launch_decode(p, rq::kRefBf16, 0, 32, &tk, &tv, static_cast<cudaStream_t>(stream));
+  p.tma_tokens = capacity;
+  cudaError_t e = rq::launch_decode(p, rq::kRefBf16, 0, 32, rq::kKernelAuto, &tk, &tv,
+                                    static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return RQ_OK;
 }

@@ -153,4 +153,30 @@ __device__ __forceinline__ float2 half2_bits_to_f2(uint32_t w) {
   return __half22float2(h);
 }
 
+// ---------------------------------------------------------------------------
+// page walk over the flattened (b, h, page) sequence (pages of any fixed size;
+// nt[b] = pages of sequence b, pre[b] = pages of the sequences before b)
+// ---------------------------------------------------------------------------
+struct PageIter {
+  int b, h, page;
+  __device__ __forceinline__ void seek(int64_t x, const int* pre, const int* nt, int B, int Hkv) {
+    int lo = 0, hi = B - 1;  // largest b with pre[b]*Hkv <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (static_cast<int64_t>(pre[mid]) * Hkv <= x) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    const int64_t r = x - static_cast<int64_t>(pre[b]) * Hkv;
+    h = static_cast<int>(r / nt[b]);
+    page = static_cast<int>(r % nt[b]);
+  }
+  __device__ __forceinline__ void next(const int* nt, int B, int Hkv) {
+    if (++page < nt[b]) return;
+    page = 0;
+    if (++h < Hkv) return;
+    h = 0;
+    do { ++b; } while (b < B && nt[b] == 0);
+  }
+};
+
 }  // namespace rq

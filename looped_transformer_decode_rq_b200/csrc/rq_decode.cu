@@ -127,31 +127,6 @@ struct Cfg {
 };
 
 // ---------------------------------------------------------------------------
-// page walk over the flattened (b, h, page) sequence
-// ---------------------------------------------------------------------------
-struct PageIter {
-  int b, h, page;
-  __device__ __forceinline__ void seek(int64_t x, const int* pre, const int* nt, int B, int Hkv) {
-    int lo = 0, hi = B - 1;  // largest b with pre[b]*Hkv <= x
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (static_cast<int64_t>(pre[mid]) * Hkv <= x) lo = mid; else hi = mid - 1;
-    }
-    b = lo;
-    const int64_t r = x - static_cast<int64_t>(pre[b]) * Hkv;
-    h = static_cast<int>(r / nt[b]);
-    page = static_cast<int>(r % nt[b]);
-  }
-  __device__ __forceinline__ void next(const int* nt, int B, int Hkv) {
-    if (++page < nt[b]) return;
-    page = 0;
-    if (++h < Hkv) return;
-    h = 0;
-    do { ++b; } while (b < B && nt[b] == 0);
-  }
-};
-
-// ---------------------------------------------------------------------------
 // code unpacking helpers
 // ---------------------------------------------------------------------------
 // Load `NB` bytes (1, 2, 4, 8 or 16) of packed codes into 32-bit words.
@@ -782,10 +757,11 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   if (wid >= P.B * Hq) return;
   const int b = wid / Hq, qh = wid % Hq, h = qh / G, gi = qh % G;
   auto clamp_len = [&](int len) { return len < 0 ? 0 : (len > P.capacity ? P.capacity : len); };
-  // page offsets (same arithmetic as the split kernel)
+  // page offsets (same arithmetic as the split kernel that wrote the partials)
+  const int pt = P.page_tokens;
   int64_t pre = 0, tot = 0;
   for (int b2 = lane; b2 < P.B; b2 += 32) {
-    const int nt = (clamp_len(P.ctx_len[b2]) + kTT - 1) / kTT;
+    const int nt = (clamp_len(P.ctx_len[b2]) + pt - 1) / pt;
     tot += nt;
     if (b2 < b) pre += nt;
   }
@@ -794,7 +770,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     tot += __shfl_xor_sync(0xffffffffu, tot, o);
     pre += __shfl_xor_sync(0xffffffffu, pre, o);
   }
-  const int nt_b = (clamp_len(P.ctx_len[b]) + kTT - 1) / kTT;
+  const int nt_b = (clamp_len(P.ctx_len[b]) + pt - 1) / pt;
   const int64_t total = tot * P.Hkv;
   const int64_t P_eff = total < P.num_ctas ? total : P.num_ctas;
 
@@ -911,9 +887,18 @@ SplitFn pick(int ref_kind, int res_bits, int res_group, int G) {
 
 }  // namespace
 
-bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G) {
+int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel) {
+  if (kernel == kKernelAuto)
+    return (G >= 4 && tc_variant_supported(ref_kind, res_bits, res_group, G)) ? kKernelTensor : kKernelSimt;
+  return kernel;
+}
+
+bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, int kernel) {
   if (res_bits != 0 && res_group != 16 && res_group != 32) return false;
-  return pick(ref_kind, res_bits, res_group, G) != nullptr;
+  kernel = decode_kernel_choice(ref_kind, res_bits, res_group, G, kernel);
+  if (kernel == kKernelTensor) return tc_variant_supported(ref_kind, res_bits, res_group, G);
+  if (kernel == kKernelSimt) return pick(ref_kind, res_bits, res_group, G) != nullptr;
+  return false;
 }
 
 int decode_grid_ctas(int device) {
@@ -927,11 +912,19 @@ int64_t decode_workspace_bytes(int B, int Hkv, int G, int num_ctas) {
   return slots * G * kPartialFloats * static_cast<int64_t>(sizeof(float));
 }
 
-cudaError_t launch_decode(const DecodeParams& p, int ref_kind, int res_bits, int res_group,
+cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_group, int kernel,
                           const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s) {
-  SplitFn fn = pick(ref_kind, res_bits, res_group, p.G);
-  if (fn == nullptr) return cudaErrorInvalidValue;
-  cudaError_t e = fn(p, tmap_k, tmap_v, s);
+  kernel = decode_kernel_choice(ref_kind, res_bits, res_group, p.G, kernel);
+  cudaError_t e;
+  if (kernel == kKernelTensor) {
+    p.page_tokens = kTcPage;
+    e = launch_split_tc(p, ref_kind, res_bits, res_group, tmap_k, tmap_v, s);
+  } else {
+    SplitFn fn = pick(ref_kind, res_bits, res_group, p.G);
+    if (fn == nullptr) return cudaErrorInvalidValue;
+    p.page_tokens = kTT;
+    e = fn(p, tmap_k, tmap_v, s);
+  }
   if (e != cudaSuccess) return e;
   const int warps = p.B * p.Hkv * p.G;
   if (warps == 0) return cudaSuccess;

@@ -1,0 +1,1047 @@
+// rq_decode_tc.cu -- split-K decode attention on the fifth-generation tensor
+// cores (tcgen05) of sm_100a, for kv-heads shared by G in {2, 4, 8} query heads.
+//
+// It computes what the CUDA-core split kernel in rq_decode.cu computes and
+// writes the same partial records (so the same combine kernel finishes the
+// call): "ResidualQuant: KV Cache Quantization for Looped Transformers with
+// 2-Bit Residuals" keeps loop l's keys and values as alpha * anchor + H^T deq(R_l)
+// (abstract, Figure 1, Figure 2 caption), and every cached token is scored and
+// summed straight from that compact form:
+//     q . K_l,t = alpha_K,t (q . K_anchor,t) + (H q) . deq(R^K_l,t)
+//     o ~ sum_t p_t alpha_V,t V_anchor,t + H^T sum_t p_t deq(R^V_l,t).
+// With G query heads per kv-head the score and value sums are small matrix
+// products, and this kernel runs them on the tensor cores:
+//
+//  * a page is 128 tokens of one (sequence, kv-head).  A producer warp streams
+//    pages into a ring of shared-memory stages: bf16 anchor tiles by tiled
+//    tensor copies with the 128-byte swizzle, code / metadata / alpha records by
+//    bulk copies, completing on mbarriers;
+//  * two consumer warpgroups expand the packed 2/4-bit codes into int8 tiles
+//    (one token per thread, rows of 128 bytes in the 128-byte swizzle); the
+//    bytes of a 32-dim chunk are kept in the order the shift-and-mask expansion
+//    produces them, and every operand that meets them uses the same order;
+//  * one thread issues the score MMAs into tensor memory (M = 128 tokens):
+//      bf16 anchor:  K_anchor (bf16) x q (bf16, one column per query head)
+//      INT4 anchor:  codes (int8) x q (int16 as signed hi/lo bytes), per group
+//      residual:     codes (int8) x H q (int16 as signed hi/lo bytes), per group
+//    so that per group  (H q)_g . c_g = s_q (256 D_hi + D_lo)  exactly in int32;
+//  * thread t reads token t's row, applies the per-token scale, offset and
+//    alpha, and each warpgroup -- one per half of the query heads -- takes the
+//    page maximum.  The page's softmax weights become the B operands of the
+//    value MMAs (M = 128 dims): a bf16 hi + lo pair per weight against the bf16
+//    anchor values, and per group an int16 (hi/lo bytes) weight relative to the
+//    page's largest scale against the code tiles; the per-group offsets are
+//    accumulated per thread;
+//  * thread d then reads dim d's row of the page's value sums and merges it
+//    into fp32 accumulators with the online-softmax rescale.
+#include "rq_common.cuh"
+#include "rq_internal.h"
+#include "rq_tcgen05.cuh"
+
+namespace rq {
+namespace {
+
+constexpr int kTP = kTcPage;   // tokens per page
+constexpr int kNCW = 8;        // consumer warps (two warpgroups)
+constexpr int kNCT = kNCW * 32;
+constexpr int kNT = kNCT + 32; // + producer warp
+constexpr int kBarAll = 1;     // the 256 consumer threads
+constexpr int kBarWG = 2;      // warpgroup w uses kBarWG + w
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kQ3 = 8323072.f;  // 24-bit range whose top byte stays in [-127, 127]
+constexpr int kSmemLimit = 227 * 1024;
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+  int i = __float_as_int(v);
+  i ^= (i >> 31) & 0x7fffffff;
+  i = __reduce_max_sync(kFull, i);
+  i ^= (i >> 31) & 0x7fffffff;
+  return __int_as_float(i);
+}
+
+// max of non-negative floats (their bit patterns order as integers)
+__device__ __forceinline__ float warp_max_nonneg(float v) {
+  return __int_as_float(__reduce_max_sync(kFull, __float_as_int(v)));
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// code expansion order.  Within a 32-dim chunk, byte j of the expanded row
+// holds dim e(j):
+//   2-bit codes: j = 8k + 4w + b  <->  e = 16w + 4b + k   ((word_w >> 2k) & 0x03030303)
+//   4-bit codes: j = 16k + 4w + b <->  e = 8w + 2b + k    ((word_w >> 4k) & 0x0F0F0F0F)
+// ---------------------------------------------------------------------------
+template <int BITS>
+__device__ __forceinline__ int pos_dim(int j) {  // position in chunk -> dim in chunk
+  return BITS == 2 ? 16 * ((j >> 2) & 1) + 4 * (j & 3) + (j >> 3) : 8 * ((j >> 2) & 3) + 2 * (j & 3) + (j >> 4);
+}
+template <int BITS>
+__device__ __forceinline__ int dim_pos(int e) {  // dim in chunk -> position in chunk
+  return BITS == 2 ? 8 * (e & 3) + 4 * (e >> 4) + ((e >> 2) & 3) : 16 * (e & 1) + 4 * (e >> 3) + ((e >> 1) & 3);
+}
+
+// Expand one token's packed codes (BITS * 16 bytes) into row r of a 128 x 128
+// int8 tile with the 128-byte swizzle (16-byte chunk q of row r stored at
+// chunk q ^ (r & 7)).
+template <int BITS>
+__device__ __forceinline__ void expand_row(const uint8_t* src, uint8_t* tile, int r) {
+  uint8_t* row = tile + r * 128;
+  const int sw = r & 7;
+  constexpr int NW = BITS * 4;  // packed 32-bit words per token
+  uint32_t w[NW];
+#pragma unroll
+  for (int i = 0; i < NW / 4; ++i) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+  constexpr int WPC = BITS == 2 ? 2 : 4;  // words per 32-dim chunk
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t o[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int k = u / WPC, ww = u % WPC;
+      o[u] = BITS == 2 ? ((w[WPC * c + ww] >> (2 * k)) & 0x03030303u) : ((w[WPC * c + ww] >> (4 * k)) & 0x0F0F0F0Fu);
+    }
+    *reinterpret_cast<uint4*>(row + (((2 * c) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(row + (((2 * c + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// byte (n, j) of an N x 128 int8 K-major operand with the 128-byte swizzle
+__device__ __forceinline__ int kmaj_byte(int n, int j) {
+  return (n >> 3) * 1024 + (n & 7) * 128 + (((j >> 4) ^ (n & 7)) << 4) + (j & 15);
+}
+
+// signed bytes of a 24-bit-range integer: v = 65536 b2 + 256 b1 + b0
+__device__ __forceinline__ void split24(int v, int& b2, int& b1, int& b0) {
+  const int t = (v + 128) >> 8;
+  b0 = v - (t << 8);
+  b2 = (t + 128) >> 8;
+  b1 = t - (b2 << 8);
+}
+
+constexpr int round16(int x) { return (x + 15) & ~15; }
+
+template <int REF, int RB, int RG, int G>
+struct TcCfg {
+  static constexpr int GH = G / 2;                       // query heads per warpgroup
+  static constexpr int NGR = RB ? kD / RG : 0;            // residual groups
+  static constexpr int NPAR = RG == 16 ? 2 : 1;           // residual groups per 32-dim chunk
+  static constexpr int NGA = REF == kRefInt4 ? 4 : 0;     // INT4 anchor groups
+  static constexpr bool HAS_ALPHA = (REF != kRefNone) && (RB != 0);
+  // per-token record bytes
+  static constexpr int REF_REC = REF == kRefBf16 ? 256 : (REF == kRefInt4 ? 64 : 0);
+  static constexpr int REFM_REC = REF == kRefInt4 ? 16 : 0;
+  static constexpr int CB = RB * 16;
+  static constexpr int MB = RB ? 4 * NGR : 0;
+  static constexpr int AL_REC = HAS_ALPHA ? 4 : 0;
+  // MMA widths (N).  Query and weight operands carry 24-bit integers as three
+  // signed bytes (j = 0: top, 1: middle, 2: bottom), one B row per byte.
+  //   score rows per 32-dim chunk: (parity, head, byte)  n = p * 3G + 3 h + j
+  //   value rows: (byte, group, head)                    n = j * NG * G + g * G + h
+  static constexpr int N_SA = round16(3 * G);                          // INT4 anchor score columns per chunk
+  static constexpr int N_SR = round16(3 * G * NPAR);                   // residual score columns per chunk
+  static constexpr int N_VA = round16(3 * 4 * G);                      // INT4 anchor value columns
+  static constexpr int N_VR = round16(3 * NGR * G);                    // residual value columns
+  // tensor-memory columns: the value sums reuse the score columns (the scores
+  // are read before the value MMAs are issued)
+  static constexpr int S_REF = 0;
+  static constexpr int S_REF_COLS = REF == kRefBf16 ? 16 : (REF == kRefInt4 ? 4 * N_SA : 0);
+  static constexpr int S_RES = S_REF + S_REF_COLS;
+  static constexpr int S_COLS = S_RES + (RB ? 4 * N_SR : 0);
+  static constexpr int O_REF = 0;
+  static constexpr int O_REF_COLS = REF == kRefBf16 ? 16 : (REF == kRefInt4 ? N_VA : 0);
+  static constexpr int O_RES = O_REF + O_REF_COLS;
+  static constexpr int O_COLS = O_RES + (RB ? N_VR : 0);
+  static constexpr int COLS = S_COLS > O_COLS ? S_COLS : O_COLS;
+  static constexpr int TMEM_COLS = COLS <= 32 ? 32 : COLS <= 64 ? 64 : COLS <= 128 ? 128 : COLS <= 256 ? 256 : 512;
+  // stage layout (pieces 1024-byte aligned)
+  static constexpr int al(int x) { return (x + 1023) & ~1023; }
+  static constexpr int O_REFK = 0;
+  static constexpr int O_REFV = O_REFK + al(kTP * REF_REC);
+  static constexpr int O_REFMK = O_REFV + al(kTP * REF_REC);
+  static constexpr int O_REFMV = O_REFMK + al(kTP * REFM_REC);
+  static constexpr int O_RESK = O_REFMV + al(kTP * REFM_REC);
+  static constexpr int O_RESV = O_RESK + al(kTP * CB);
+  static constexpr int O_RESMK = O_RESV + al(kTP * CB);
+  static constexpr int O_RESMV = O_RESMK + al(kTP * MB);
+  static constexpr int O_AL = O_RESMV + al(kTP * MB);
+  static constexpr int STAGE_BYTES = O_AL + al(kTP * AL_REC);
+  // operand tiles (after the stages)
+  static constexpr int F_UK = 0;                                   // residual K codes, int8 [128 tok][128]
+  static constexpr int F_UV = F_UK + (RB ? 16384 : 0);             // residual V codes
+  static constexpr int F_URK = F_UV + (RB ? 16384 : 0);            // INT4 anchor K codes
+  static constexpr int F_URV = F_URK + (REF == kRefInt4 ? 16384 : 0);
+  static constexpr int F_QB = F_URV + (REF == kRefInt4 ? 16384 : 0);  // bf16 q [16][128], K-major sw128
+  static constexpr int F_QA = F_QB + (REF == kRefBf16 ? 4096 : 0);    // int8 q bytes [N_SA][128]
+  static constexpr int F_HQ = F_QA + (REF == kRefInt4 ? al(N_SA * 128) : 0);  // int8 H q bytes [N_SR][128]
+  static constexpr int F_WB = F_HQ + (RB ? al(N_SR * 128) : 0);       // bf16 weights, MN-major [16 x 128 tok]
+  static constexpr int F_WA = F_WB + (REF == kRefBf16 ? 4096 : 0);    // int8 weights [N_VA x 128 tok]
+  static constexpr int F_WR = F_WA + (REF == kRefInt4 ? al(N_VA * 128) : 0);
+  static constexpr int F_END = F_WR + (RB ? al(N_VR * 128) : 0);
+  // small state (after the tiles; 4-byte words)
+  static constexpr int NRED = 1 + 8 + 4;                 // l, residual offsets, anchor offsets
+  static constexpr int W_CS = 0;                         // [G] residual q scale * scale_log2
+  static constexpr int W_QS = W_CS + 8;                  // [G][8] residual group sums of H q
+  static constexpr int W_CA = W_QS + 64;                 // [G] anchor q scale * scale_log2
+  static constexpr int W_QA = W_CA + 8;                  // [G][4] anchor group sums of q
+  static constexpr int W_WM = W_QA + 32;                 // [2][4 warps][4] warp maxima of scores
+  static constexpr int W_SIG = W_WM + 32;                // [2][4 warps][12] warp maxima of scales
+  static constexpr int W_RED = W_SIG + 96;               // [G][NRED] flush sums
+  static constexpr int W_PRE = W_RED + 8 * NRED;         // [RQ_MAX_BATCH + 1] page prefix
+  static constexpr int W_MISC = W_PRE + RQ_MAX_BATCH + 1;  // abort flag, tensor-memory base
+  static constexpr int W_BAR = (W_MISC + 2 + 1) & ~1;    // 8-byte aligned mbarriers
+  static constexpr int NBARS = 2 * 4 + 2;
+  static constexpr int SMALL_BYTES = 4 * W_BAR + 8 * NBARS;
+  static constexpr int FIXED = 1024 + F_END + SMALL_BYTES;
+  static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT >= 4 ? 4 : (STAGES_FIT >= 2 ? STAGES_FIT : 2);
+  static constexpr bool FITS = STAGES_FIT >= 2;
+  static constexpr int SMEM_BYTES = FIXED + STAGES * STAGE_BYTES;
+  // instruction descriptors
+  static constexpr uint32_t ID_SB = tc::instr_desc(tc::kAccF32, tc::kFmtBf16, tc::kFmtBf16, 0, 0, 128, 16);
+  static constexpr uint32_t ID_SA = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 0, 0, 128, N_SA);
+  static constexpr uint32_t ID_SR = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 0, 0, 128, N_SR);
+  static constexpr uint32_t ID_VB = tc::instr_desc(tc::kAccF32, tc::kFmtBf16, tc::kFmtBf16, 1, 1, 128, 16);
+  static constexpr uint32_t ID_VA = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 1, 1, 128, N_VA);
+  static constexpr uint32_t ID_VR = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 1, 1, 128, N_VR);
+  static_assert(G == 2 || G == 4 || G == 8, "query heads per kv-head");
+  static_assert(N_VA <= 256 && N_VR <= 256 && N_SR <= 256, "MMA width");
+  static_assert(COLS <= 512, "tensor memory");
+};
+
+// ---------------------------------------------------------------------------
+// producer: one page into stage `st`
+// ---------------------------------------------------------------------------
+template <int REF, int RB, int RG, int G>
+__device__ __forceinline__ void tc_issue_page(const DecodeParams& P, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                              uint8_t* st, uint32_t full, const PageIter& it, int Hkv) {
+  using C = TcCfg<REF, RB, RG, G>;
+  const int t0 = it.page * kTP;
+  // byte planes hold plane_tokens (a multiple of 64) records per (b, h)
+  const int nrec = (P.plane_tokens > 0 && t0 + kTP > P.plane_tokens) ? static_cast<int>(P.plane_tokens - t0) : kTP;
+  const int halves = (REF == kRefBf16) ? ((t0 + 64 < P.tma_tokens) ? 2 : 1) : 0;
+  const uint32_t bytes = halves * 4 * 8192 +
+                         nrec * (2 * (REF == kRefInt4 ? 64 + 16 : 0) + 2 * C::CB + 2 * C::MB + C::AL_REC);
+  mbar_arrive_expect_tx(full, bytes);
+  const int64_t rec0 = static_cast<int64_t>(it.b * Hkv + it.h) * P.plane_tokens + t0;
+  if constexpr (REF == kRefBf16) {
+    for (int th = 0; th < halves; ++th) {
+#pragma unroll
+      for (int dh = 0; dh < 2; ++dh) {
+        tma_load_4d(smem_u32(st + C::O_REFK + dh * 16384 + th * 8192), tmK, 64 * dh, t0 + 64 * th, it.h, it.b, full);
+        tma_load_4d(smem_u32(st + C::O_REFV + dh * 16384 + th * 8192), tmV, 64 * dh, t0 + 64 * th, it.h, it.b, full);
+      }
+    }
+  } else if constexpr (REF == kRefInt4) {
+    bulk_g2s(smem_u32(st + C::O_REFK), P.ref_codes[0] + rec0 * 64, nrec * 64, full);
+    bulk_g2s(smem_u32(st + C::O_REFV), P.ref_codes[1] + rec0 * 64, nrec * 64, full);
+    bulk_g2s(smem_u32(st + C::O_REFMK), P.ref_meta[0] + rec0 * 16, nrec * 16, full);
+    bulk_g2s(smem_u32(st + C::O_REFMV), P.ref_meta[1] + rec0 * 16, nrec * 16, full);
+  }
+  if constexpr (RB != 0) {
+    bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0] + rec0 * C::CB, nrec * C::CB, full);
+    bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[1] + rec0 * C::CB, nrec * C::CB, full);
+    bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0] + rec0 * C::MB, nrec * C::MB, full);
+    bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[1] + rec0 * C::MB, nrec * C::MB, full);
+  }
+  if constexpr (C::HAS_ALPHA) bulk_g2s(smem_u32(st + C::O_AL), P.alpha + rec0 * 4, nrec * 4, full);
+}
+
+// ---------------------------------------------------------------------------
+// segment set-up (warp w < G: query head w of kv-head h): the B operands that
+// carry the queries.  Rows of the int8 operands are (sub-group, head, hi/lo).
+// ---------------------------------------------------------------------------
+// x: dims 4 lane .. 4 lane + 3 of query head hq, quantised to 24-bit integers
+// with one scale per head and written as three signed bytes into rows
+// p * 3 GG + 3 hq + j.  With 16-dim groups p is the group's parity within its
+// 32-dim chunk and the rows of the other parity are zero there; with 32-dim
+// groups p = 0.
+template <int BITS, int RGRP, int GG>
+__device__ __forceinline__ void put_q_s24(uint8_t* tile, const float (&x)[4], int hq, int lane, float* scale_out,
+                                          float* gsum_out, float scale_log2) {
+  float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+  m = warp_max_nonneg(m);
+  const float inv = m > 0.f ? kQ3 / m : 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int d = 4 * lane + e;
+    int qi = __float2int_rn(x[e] * inv);
+    qi = max(-8323072, min(8323072, qi));
+    int b[3];
+    split24(qi, b[0], b[1], b[2]);
+    const int j = 32 * (d >> 5) + dim_pos<BITS>(d & 31);
+    const int par = RGRP == 16 ? ((d >> 4) & 1) : 0;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      tile[kmaj_byte(par * 3 * GG + 3 * hq + k, j)] = static_cast<uint8_t>(b[k]);
+      if constexpr (RGRP == 16) tile[kmaj_byte((1 - par) * 3 * GG + 3 * hq + k, j)] = 0;
+    }
+  }
+  float s = x[0] + x[1] + x[2] + x[3];
+  constexpr int LPG = RGRP / 4;  // lanes per group
+#pragma unroll
+  for (int o = 1; o < LPG; o <<= 1) s += __shfl_xor_sync(kFull, s, o);
+  if ((lane % LPG) == 0) gsum_out[lane / LPG] = s * scale_log2;
+  if (lane == 0) *scale_out = m * (1.f / kQ3) * scale_log2;
+}
+
+// 65536 b2 + 256 b1 + b0 of three int32 byte-products (as fp32)
+__device__ __forceinline__ float comb24(uint32_t b2, uint32_t b1, uint32_t b0) {
+  return fmaf(65536.f, static_cast<float>(static_cast<int>(b2)),
+              fmaf(256.f, static_cast<float>(static_cast<int>(b1)), static_cast<float>(static_cast<int>(b0))));
+}
+
+// ---------------------------------------------------------------------------
+// split kernel
+// ---------------------------------------------------------------------------
+template <int REF, int RB, int RG, int G>
+__global__ void __launch_bounds__(kNT, 1)
+    decode_tc_kernel(const __grid_constant__ DecodeParams P, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV) {
+  using C = TcCfg<REF, RB, RG, G>;
+  constexpr int GH = C::GH;
+  constexpr int NGR = C::NGR;
+  constexpr int NGA = C::NGA;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = base;
+  uint8_t* fx = base + C::STAGES * C::STAGE_BYTES;
+  float* sw = reinterpret_cast<float*>(fx + C::F_END);
+  float* sCS = sw + C::W_CS;
+  float* sQS = sw + C::W_QS;
+  float* sCA = sw + C::W_CA;
+  float* sQA = sw + C::W_QA;
+  float* sWM = sw + C::W_WM;
+  float* sSig = sw + C::W_SIG;
+  float* sRed = sw + C::W_RED;
+  int* sPre = reinterpret_cast<int*>(sw + C::W_PRE);
+  volatile int* sAbort = reinterpret_cast<volatile int*>(sw + C::W_MISC);
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(sw + C::W_MISC + 1);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sw + C::W_BAR);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + 4;
+  uint64_t* sbar = bars + 8;
+  uint64_t* obar = bars + 9;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int B = P.B, Hkv = P.Hkv;
+
+  // ---- pages per sequence and their prefix (pre[b+1] - pre[b] = pages of b)
+  if (warp == 0) {
+    int carry = 0;
+    for (int b0 = 0; b0 < B; b0 += 32) {
+      const int b = b0 + lane;
+      int v = 0;
+      if (b < B) {
+        int len = P.ctx_len[b];
+        if (len < 0 || len > P.capacity) {
+          if (blockIdx.x == 0) set_flag(P.status, RQ_FLAG_CTX_LEN);
+          len = len < 0 ? 0 : P.capacity;
+        }
+        v = (len + kTP - 1) / kTP;
+      }
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+      }
+      if (b < B) sPre[b] = carry + x - v;
+      carry += __shfl_sync(kFull, x, 31);
+    }
+    if (lane == 0) sPre[B] = carry;
+  }
+  for (int i = tid; i < 8 * C::NRED; i += kNT) sRed[i] = 0.f;
+  if (tid == 0) {
+    *sAbort = 0;
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);   // the producer's expect_tx
+      mbar_init(smem_u32(&empty[s]), 1);  // the commit after the page's value MMAs
+    }
+    mbar_init(smem_u32(sbar), 1);
+    mbar_init(smem_u32(obar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  const int64_t total = static_cast<int64_t>(sPre[B]) * Hkv;
+  const int64_t P_eff = total < P.num_ctas ? total : P.num_ctas;
+  if (static_cast<int64_t>(blockIdx.x) >= P_eff) return;
+  const int64_t x0 = static_cast<int64_t>(blockIdx.x) * total / P_eff;
+  const int64_t x1 = static_cast<int64_t>(blockIdx.x + 1) * total / P_eff;
+  const int n_pages = static_cast<int>(x1 - x0);
+
+  // page counts as a view of the prefix
+  auto nt_of = [&](int b) { return sPre[b + 1] - sPre[b]; };
+  auto seek = [&](PageIter& it, int64_t x) {
+    int lo = 0, hi = B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (static_cast<int64_t>(sPre[mid]) * Hkv <= x) lo = mid; else hi = mid - 1;
+    }
+    it.b = lo;
+    const int64_t r = x - static_cast<int64_t>(sPre[lo]) * Hkv;
+    const int nt = nt_of(lo);
+    it.h = static_cast<int>(r / nt);
+    it.page = static_cast<int>(r % nt);
+  };
+  auto advance = [&](PageIter& it) {
+    if (++it.page < nt_of(it.b)) return;
+    it.page = 0;
+    if (++it.h < Hkv) return;
+    it.h = 0;
+    do { ++it.b; } while (it.b < B && nt_of(it.b) == 0);
+  };
+
+  // ---- tensor memory for the page's score and value sums
+  if (warp == 0) {
+    tc::tmem_alloc(smem_u32(sTmem), C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = *sTmem;
+
+  // ========================= producer warp =========================
+  if (warp == kNCW) {
+    if (lane == 0) {
+      if constexpr (REF == kRefBf16) {
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+      }
+      PageIter it;
+      seek(it, x0);
+      int k = 0;
+      for (; k < n_pages; ++k) {
+        const int s = k % C::STAGES;
+        if (!mbar_wait_bounded(smem_u32(&empty[s]), ((k / C::STAGES) & 1) ^ 1)) {
+          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+          break;
+        }
+        tc_issue_page<REF, RB, RG, G>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&full[s]), it, Hkv);
+        advance(it);
+      }
+      // no copy this CTA issued may still be landing when it exits
+      for (int kk = (k > C::STAGES ? k - C::STAGES : 0); kk < k; ++kk) {
+        if (!mbar_wait_bounded(smem_u32(&full[kk % C::STAGES]), (kk / C::STAGES) & 1)) {
+          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+          break;
+        }
+      }
+    }
+    return;
+  }
+
+  // ========================= consumer warpgroups =========================
+  const int wg = warp >> 2;                  // query heads [wg * GH, wg * GH + GH)
+  const int r = tid & 127;                   // tensor-memory lane: token, then dim position
+  const uint32_t tl = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+  const int chunk = warp & 3;                // 32-dim chunk of this thread's position
+  uint8_t* UK = fx + C::F_UK;
+  uint8_t* UV = fx + C::F_UV;
+  uint8_t* URK = fx + C::F_URK;
+  uint8_t* URV = fx + C::F_URV;
+  uint8_t* QB = fx + C::F_QB;
+  uint8_t* QA = fx + C::F_QA;
+  uint8_t* HQ = fx + C::F_HQ;
+  uint8_t* WB = fx + C::F_WB;
+  uint8_t* WA = fx + C::F_WA;
+  uint8_t* WR = fx + C::F_WR;
+  // residual group of this thread's dim position (and its parity for 16-groups)
+  const int par_r = RB == 2 ? ((r >> 2) & 1) : ((r >> 3) & 1);
+  const int g_res = RG == 16 ? 2 * chunk + par_r : chunk;
+
+  PageIter it;
+  seek(it, x0);
+  int k = 0;
+  uint32_t sph = 0, oph = 0;
+  bool aborted = false;
+  while (k < n_pages && !aborted) {
+    const int b = it.b, h = it.h;
+    const int seg_pages = min(nt_of(b) - it.page, n_pages - k);
+    int len_b = P.ctx_len[b];
+    len_b = len_b < 0 ? 0 : (len_b > P.capacity ? P.capacity : len_b);
+
+    // ---- segment set-up: query operands of the G heads of (b, h)
+    if (warp < G) {
+      const int hq = warp;
+      const int qh = h * G + hq;
+      const uint2 raw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hkv * G + qh) * kD + 4 * lane);
+      const int d = 4 * lane;
+      if constexpr (REF == kRefBf16) {
+        *reinterpret_cast<uint2*>(QB + (d >> 6) * 2048 + (hq >> 3) * 1024 + (hq & 7) * 128 +
+                                  ((((d & 63) >> 3) ^ (hq & 7)) << 4) + (d & 7) * 2) = raw;
+      }
+      const float2 a01 = bf16x2_to_f2(raw.x), a23 = bf16x2_to_f2(raw.y);
+      float x[4] = {a01.x, a01.y, a23.x, a23.y};
+      if constexpr (REF == kRefInt4) put_q_s24<4, 32, G>(QA, x, hq, lane, &sCA[hq], &sQA[hq * 4], P.scale_log2);
+      if constexpr (RB != 0) {
+        if (P.rotate) {
+          const float t0 = x[0] + x[1], t1 = x[0] - x[1], t2 = x[2] + x[3], t3 = x[2] - x[3];
+          x[0] = t0 + t2; x[2] = t0 - t2; x[1] = t1 + t3; x[3] = t1 - t3;
+#pragma unroll
+          for (int m = 1; m < 32; m <<= 1) {
+            const bool up = (lane & m) != 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float o = __shfl_xor_sync(kFull, x[e], m);
+              x[e] = up ? (o - x[e]) : (x[e] + o);
+            }
+          }
+          const float c = 0.08838834764831845f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[e] *= c;
+        }
+        put_q_s24<RB, RG, G>(HQ, x, hq, lane, &sCS[hq], &sQS[hq * 8], P.scale_log2);
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(kBarAll, kNCT);
+
+    // per-warpgroup running state (query heads wg*GH + i)
+    float m_run[GH], l_thr[GH], acc_ref[GH], acc_res[GH];
+    float zr[GH][NGR > 0 ? NGR : 1], za[GH][NGA > 0 ? NGA : 1];
+#pragma unroll
+    for (int i = 0; i < GH; ++i) {
+      m_run[i] = -INFINITY;
+      l_thr[i] = acc_ref[i] = acc_res[i] = 0.f;
+#pragma unroll
+      for (int g = 0; g < (NGR > 0 ? NGR : 1); ++g) zr[i][g] = 0.f;
+#pragma unroll
+      for (int g = 0; g < (NGA > 0 ? NGA : 1); ++g) za[i][g] = 0.f;
+    }
+
+    for (int sp = 0; sp < seg_pages; ++sp, ++k) {
+      const int s = k % C::STAGES;
+      uint8_t* st = stages + s * C::STAGE_BYTES;
+      const int n_valid = min(kTP, len_b - it.page * kTP);
+      if (!mbar_wait_bounded(smem_u32(&full[s]), (k / C::STAGES) & 1)) {
+        set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+        *sAbort = 1;
+      }
+      // ---- expand the packed codes (warpgroup 0: keys, 1: values)
+      if constexpr (RB != 0) expand_row<RB>(st + (wg ? C::O_RESV : C::O_RESK) + r * C::CB, wg ? UV : UK, r);
+      if constexpr (REF == kRefInt4) expand_row<4>(st + (wg ? C::O_REFV : C::O_REFK) + r * 64, wg ? URV : URK, r);
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      named_bar_sync(kBarAll, kNCT);
+      if (*sAbort) {  // written only before the barrier above: uniform
+        aborted = true;
+        break;
+      }
+
+      // ---- score MMAs: D[t][n] over the page's 128 tokens
+      if (tid == 0) {
+        tc::fence_after_sync();
+        if constexpr (REF == kRefBf16) {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            tc::mma_bf16(tbase + C::S_REF, tc::desc_k_sw128(smem_u32(st + C::O_REFK + (ks >> 2) * 16384 + (ks & 3) * 32)),
+                         tc::desc_k_sw128(smem_u32(QB + (ks >> 2) * 2048 + (ks & 3) * 32)), C::ID_SB, ks > 0);
+        } else if constexpr (REF == kRefInt4) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tc::mma_s8(tbase + C::S_REF + C::N_SA * c, tc::desc_k_sw128(smem_u32(URK + 32 * c)),
+                       tc::desc_k_sw128(smem_u32(QA + 32 * c)), C::ID_SA, 0);
+        }
+        if constexpr (RB != 0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tc::mma_s8(tbase + C::S_RES + C::N_SR * c, tc::desc_k_sw128(smem_u32(UK + 32 * c)),
+                       tc::desc_k_sw128(smem_u32(HQ + 32 * c)), C::ID_SR, 0);
+        }
+        tc::commit(smem_u32(sbar));
+      }
+
+      // ---- per-token metadata (thread = token r), zero past the context
+      const bool valid = r < n_valid;
+      float aK = 1.f, aV = 1.f;
+      if constexpr (C::HAS_ALPHA) {
+        const float2 a = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_AL + r * 4));
+        aK = a.x;
+        aV = a.y;
+      }
+      if (!valid) aK = aV = 0.f;
+      float sK[NGR > 0 ? NGR : 1], zK[NGR > 0 ? NGR : 1], sV[NGR > 0 ? NGR : 1], zV[NGR > 0 ? NGR : 1];
+      if constexpr (RB != 0) {
+#pragma unroll
+        for (int g = 0; g < NGR; g += 4) {
+          const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_RESMK + r * C::MB + 4 * g);
+          const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_RESMV + r * C::MB + 4 * g);
+          const uint32_t wk[4] = {mk.x, mk.y, mk.z, mk.w}, wv[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 a = half2_bits_to_f2(wk[u]), c2 = half2_bits_to_f2(wv[u]);
+            sK[g + u] = valid ? a.x : 0.f;
+            zK[g + u] = valid ? a.y : 0.f;
+            sV[g + u] = valid ? c2.x : 0.f;
+            zV[g + u] = valid ? c2.y : 0.f;
+          }
+        }
+      }
+      float sAk[4], zAk[4], sAv[4], zAv[4];
+      if constexpr (REF == kRefInt4) {
+        const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_REFMK + r * 16);
+        const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_REFMV + r * 16);
+        const uint32_t wk[4] = {mk.x, mk.y, mk.z, mk.w}, wv[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 a = half2_bits_to_f2(wk[u]), c2 = half2_bits_to_f2(wv[u]);
+          sAk[u] = valid ? a.x : 0.f;
+          zAk[u] = valid ? a.y : 0.f;
+          sAv[u] = valid ? c2.x : 0.f;
+          zAv[u] = valid ? c2.y : 0.f;
+        }
+      }
+
+      if (!mbar_wait_bounded(smem_u32(sbar), sph)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+      sph ^= 1u;
+      tc::fence_after_sync();
+
+      // ---- scores of token r for this warpgroup's heads
+      float S[GH];
+#pragma unroll
+      for (int i = 0; i < GH; ++i) S[i] = 0.f;
+      if constexpr (REF == kRefBf16) {
+        uint32_t v[GH > 1 ? GH : 2];
+        if constexpr (GH == 1) {
+          uint32_t v2[2];
+          tc::tmem_ld<2>(tl + C::S_REF, v2);  // columns 0, 1 (column wg is this head)
+          tc::tmem_wait_ld();
+          tc::reg_fence(v2);
+          v[0] = wg ? v2[1] : v2[0];
+        } else {
+          uint32_t vv[GH];
+          tc::tmem_ld<GH>(tl + C::S_REF + wg * GH, vv);
+          tc::tmem_wait_ld();
+          tc::reg_fence(vv);
+#pragma unroll
+          for (int i = 0; i < GH; ++i) v[i] = vv[i];
+        }
+        const float ak = aK * P.scale_log2;
+#pragma unroll
+        for (int i = 0; i < GH; ++i) S[i] = __uint_as_float(v[i]) * ak;
+      }
+      if constexpr (REF == kRefInt4 || RB != 0) {
+        float dotA[GH], offA[GH], dotR[GH], offR[GH];
+#pragma unroll
+        for (int i = 0; i < GH; ++i) dotA[i] = offA[i] = dotR[i] = offR[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t va[3 * GH], vr[C::NPAR][3 * GH];
+          if constexpr (REF == kRefInt4) tc::tmem_ld_n<3 * GH>(tl + C::S_REF + C::N_SA * c + 3 * wg * GH, va);
+          if constexpr (RB != 0) {
+#pragma unroll
+            for (int p = 0; p < C::NPAR; ++p)
+              tc::tmem_ld_n<3 * GH>(tl + C::S_RES + C::N_SR * c + p * 3 * G + 3 * wg * GH, vr[p]);
+          }
+          tc::tmem_wait_ld();
+          if constexpr (REF == kRefInt4) tc::reg_fence(va);
+          if constexpr (RB != 0) {
+#pragma unroll
+            for (int p = 0; p < C::NPAR; ++p) tc::reg_fence(vr[p]);
+          }
+#pragma unroll
+          for (int i = 0; i < GH; ++i) {
+            const int hq = wg * GH + i;
+            if constexpr (REF == kRefInt4) {
+              dotA[i] = fmaf(sAk[c], comb24(va[3 * i], va[3 * i + 1], va[3 * i + 2]), dotA[i]);
+              offA[i] = fmaf(zAk[c], sQA[hq * 4 + c], offA[i]);
+            }
+            if constexpr (RB != 0) {
+#pragma unroll
+              for (int p = 0; p < C::NPAR; ++p) {
+                const int g = c * C::NPAR + p;
+                dotR[i] = fmaf(sK[g], comb24(vr[p][3 * i], vr[p][3 * i + 1], vr[p][3 * i + 2]), dotR[i]);
+                offR[i] = fmaf(zK[g], sQS[hq * 8 + g], offR[i]);
+              }
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < GH; ++i) {
+          const int hq = wg * GH + i;
+          if constexpr (REF == kRefInt4) S[i] = aK * fmaf(dotA[i], sCA[hq], offA[i]);
+          if constexpr (RB != 0) S[i] += fmaf(dotR[i], sCS[hq], offR[i]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < GH; ++i) S[i] = valid ? S[i] : -INFINITY;
+
+      // ---- page maxima of the scores (per head) and of the value scales (per group)
+#pragma unroll
+      for (int i = 0; i < GH; ++i) {
+        const float v = warp_max(S[i]);
+        if (lane == 0) sWM[(wg * 4 + (warp & 3)) * 4 + i] = v;
+      }
+      if constexpr (RB != 0) {
+#pragma unroll
+        for (int g = 0; g < NGR; ++g) {
+          const float v = warp_max_nonneg(sV[g]);
+          if (lane == 0) sSig[(wg * 4 + (warp & 3)) * 12 + g] = v;
+        }
+      }
+      if constexpr (REF == kRefInt4) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float v = warp_max_nonneg(fabsf(aV * sAv[g]));
+          if (lane == 0) sSig[(wg * 4 + (warp & 3)) * 12 + 8 + g] = v;
+        }
+      }
+      named_bar_sync(kBarWG + wg, 128);
+      float pm[GH], crun[GH], prel[GH];
+#pragma unroll
+      for (int i = 0; i < GH; ++i) {
+        const float* wm = sWM + wg * 16 + i;
+        const float mp = fmaxf(fmaxf(wm[0], wm[4]), fmaxf(wm[8], wm[12]));
+        const float mn = fmaxf(m_run[i], mp);
+        crun[i] = fast_exp2(m_run[i] - mn);
+        pm[i] = fast_exp2(mp - mn);
+        m_run[i] = mn;
+        prel[i] = fast_exp2(S[i] - mp);
+      }
+      float sig[NGR > 0 ? NGR : 1], siga[4];
+      if constexpr (RB != 0) {
+#pragma unroll
+        for (int g = 0; g < NGR; ++g) {
+          const float* sg = sSig + wg * 48 + g;
+          sig[g] = fmaxf(fmaxf(sg[0], sg[12]), fmaxf(sg[24], sg[36]));
+        }
+      }
+      if constexpr (REF == kRefInt4) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float* sg = sSig + wg * 48 + 8 + g;
+          siga[g] = fmaxf(fmaxf(sg[0], sg[12]), fmaxf(sg[24], sg[36]));
+        }
+      }
+
+      // ---- B operands of the value MMAs: column t = token r, rows (group, head, hi/lo)
+      const int wrow = (r >> 3) * 128 + (r & 7) * 16;  // MN-major core-matrix row of token r
+      if constexpr (REF == kRefBf16) {
+        uint32_t pk[GH];
+#pragma unroll
+        for (int i = 0; i < GH; ++i) {
+          const float w = prel[i] * aV;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(w - __bfloat162float(hi));
+          pk[i] = static_cast<uint32_t>(__bfloat16_as_ushort(hi)) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(lo)) << 16);
+        }
+        const int n0 = wg * G;  // rows n = 2 * head + (0: hi, 1: lo)
+        uint8_t* dst = WB + (n0 >> 3) * 2048 + wrow + (n0 & 7) * 2;
+        if constexpr (GH == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        else if constexpr (GH == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+        else *reinterpret_cast<uint32_t*>(dst) = pk[0];
+      }
+      auto put_w8 = [&](uint8_t* tile, int ng, int g, const float (&w)[GH]) {
+        // three signed bytes per weight; this warpgroup's GH heads are contiguous rows
+        uint32_t bj[3] = {0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < GH; ++i) {
+          int qi = __float2int_rn(w[i] * kQ3);
+          qi = max(-8323072, min(8323072, qi));
+          int b2, b1, b0;
+          split24(qi, b2, b1, b0);
+          bj[0] |= (static_cast<uint32_t>(b2) & 0xFFu) << (8 * i);
+          bj[1] |= (static_cast<uint32_t>(b1) & 0xFFu) << (8 * i);
+          bj[2] |= (static_cast<uint32_t>(b0) & 0xFFu) << (8 * i);
+        }
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const int n0 = j * ng * G + g * G + wg * GH;
+          uint8_t* dst = tile + (n0 >> 4) * 2048 + wrow + (n0 & 15);
+          if constexpr (GH == 4) *reinterpret_cast<uint32_t*>(dst) = bj[j];
+          else if constexpr (GH == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(bj[j]);
+          else *dst = static_cast<uint8_t>(bj[j]);
+        }
+      };
+      if constexpr (REF == kRefInt4) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float inv = siga[g] > 0.f ? 1.f / siga[g] : 0.f;
+          float w[GH];
+#pragma unroll
+          for (int i = 0; i < GH; ++i) w[i] = prel[i] * aV * sAv[g] * inv;
+          put_w8(WA, 4, g, w);
+        }
+      }
+      if constexpr (RB != 0) {
+#pragma unroll
+        for (int g = 0; g < NGR; ++g) {
+          const float inv = sig[g] > 0.f ? 1.f / sig[g] : 0.f;
+          float w[GH];
+#pragma unroll
+          for (int i = 0; i < GH; ++i) w[i] = prel[i] * sV[g] * inv;
+          put_w8(WR, NGR, g, w);
+        }
+      }
+      // bf16 anchor rows past the context may hold anything: clear them so that
+      // their zero weights give exact zeros
+      if constexpr (REF == kRefBf16) {
+        if (!valid) {
+          uint4* row = reinterpret_cast<uint4*>(st + C::O_REFV + wg * 16384 + r * 128);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) row[q] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      tc::fence_before_sync();
+      named_bar_sync(kBarAll, kNCT);
+
+      // ---- value MMAs: D[d][n] over the page's 128 tokens
+      if (tid == 0) {
+        tc::fence_after_sync();
+        if constexpr (REF == kRefBf16) {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            tc::mma_bf16(tbase + C::O_REF, tc::desc_mn_sw128(smem_u32(st + C::O_REFV + ks * 2048), 16384),
+                         tc::desc_mn_plain(smem_u32(WB + ks * 256), 128, 2048), C::ID_VB, ks > 0);
+        } else if constexpr (REF == kRefInt4) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_s8(tbase + C::O_REF, tc::desc_mn_sw128(smem_u32(URV + ks * 4096), 16384),
+                       tc::desc_mn_plain(smem_u32(WA + ks * 512), 128, 2048), C::ID_VA, ks > 0);
+        }
+        if constexpr (RB != 0) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_s8(tbase + C::O_RES, tc::desc_mn_sw128(smem_u32(UV + ks * 4096), 16384),
+                       tc::desc_mn_plain(smem_u32(WR + ks * 512), 128, 2048), C::ID_VR, ks > 0);
+        }
+        tc::commit(smem_u32(obar));
+        tc::commit(smem_u32(&empty[s]));
+      }
+
+      // ---- running denominators and offset sums (thread = token r)
+#pragma unroll
+      for (int i = 0; i < GH; ++i) {
+        const float pr = prel[i] * pm[i];
+        l_thr[i] = fmaf(l_thr[i], crun[i], pr);
+        if constexpr (RB != 0) {
+#pragma unroll
+          for (int g = 0; g < NGR; ++g) zr[i][g] = fmaf(zr[i][g], crun[i], pr * zV[g]);
+        }
+        if constexpr (REF == kRefInt4) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) za[i][g] = fmaf(za[i][g], crun[i], pr * aV * zAv[g]);
+        }
+      }
+
+      if (!mbar_wait_bounded(smem_u32(obar), oph)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+      oph ^= 1u;
+      tc::fence_after_sync();
+
+      // ---- merge the page's value sums (thread = dim position r)
+      if constexpr (REF == kRefBf16) {
+        uint32_t v[G];
+        tc::tmem_ld<G>(tl + C::O_REF + wg * G, v);
+        tc::tmem_wait_ld();
+        tc::reg_fence(v);
+#pragma unroll
+        for (int i = 0; i < GH; ++i)
+          acc_ref[i] = fmaf(acc_ref[i], crun[i], pm[i] * (__uint_as_float(v[2 * i]) + __uint_as_float(v[2 * i + 1])));
+      } else if constexpr (REF == kRefInt4) {
+        uint32_t v[3][GH];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) tc::tmem_ld<GH>(tl + C::O_REF + j * 4 * G + chunk * G + wg * GH, v[j]);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 3; ++j) tc::reg_fence(v[j]);
+        float sg = siga[0];
+#pragma unroll
+        for (int g = 1; g < 4; ++g) sg = (chunk == g) ? siga[g] : sg;
+        const float f = sg * (1.f / kQ3);
+#pragma unroll
+        for (int i = 0; i < GH; ++i) {
+          const float x = fmaf(65536.f, static_cast<float>(static_cast<int>(v[0][i])),
+                               fmaf(256.f, static_cast<float>(static_cast<int>(v[1][i])),
+                                    static_cast<float>(static_cast<int>(v[2][i]))));
+          acc_ref[i] = fmaf(acc_ref[i], crun[i], pm[i] * f * x);
+        }
+      }
+      if constexpr (RB != 0) {
+        uint32_t v[C::NPAR][3][GH];
+#pragma unroll
+        for (int p = 0; p < C::NPAR; ++p)
+#pragma unroll
+          for (int j = 0; j < 3; ++j)
+            tc::tmem_ld<GH>(tl + C::O_RES + j * NGR * G + (chunk * C::NPAR + p) * G + wg * GH, v[p][j]);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int p = 0; p < C::NPAR; ++p)
+#pragma unroll
+          for (int j = 0; j < 3; ++j) tc::reg_fence(v[p][j]);
+        float sg = sig[0];
+#pragma unroll
+        for (int g = 1; g < NGR; ++g) sg = (g_res == g) ? sig[g] : sg;
+        const float f = sg * (1.f / kQ3);
+#pragma unroll
+        for (int i = 0; i < GH; ++i) {
+          int b2 = static_cast<int>(v[0][0][i]), b1 = static_cast<int>(v[0][1][i]), b0 = static_cast<int>(v[0][2][i]);
+          if constexpr (C::NPAR == 2) {
+            b2 = par_r ? static_cast<int>(v[1][0][i]) : b2;
+            b1 = par_r ? static_cast<int>(v[1][1][i]) : b1;
+            b0 = par_r ? static_cast<int>(v[1][2][i]) : b0;
+          }
+          const float x = fmaf(65536.f, static_cast<float>(b2), fmaf(256.f, static_cast<float>(b1), static_cast<float>(b0)));
+          acc_res[i] = fmaf(acc_res[i], crun[i], pm[i] * f * x);
+        }
+      }
+      tc::fence_before_sync();
+      advance(it);
+    }
+    if (aborted) break;
+
+    // ---- flush this (b, h) segment: one partial record per query head
+#pragma unroll
+    for (int i = 0; i < GH; ++i) {
+      const int hq = wg * GH + i;
+      const float lsum = warp_sum(l_thr[i]);
+      if (lane == 0) atomicAdd(&sRed[hq * C::NRED], lsum);
+      if constexpr (RB != 0) {
+#pragma unroll
+        for (int g = 0; g < NGR; ++g) {
+          const float z = warp_sum(zr[i][g]);
+          if (lane == 0) atomicAdd(&sRed[hq * C::NRED + 1 + g], z);
+        }
+      }
+      if constexpr (REF == kRefInt4) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const float z = warp_sum(za[i][g]);
+          if (lane == 0) atomicAdd(&sRed[hq * C::NRED + 9 + g], z);
+        }
+      }
+    }
+    named_bar_sync(kBarWG + wg, 128);
+    {
+      const int pair = b * Hkv + h;
+      const int d_ref = REF == kRefInt4 ? 32 * chunk + pos_dim<4>(r & 31) : r;
+      const int d_res = RB ? 32 * chunk + pos_dim<RB ? RB : 2>(r & 31) : r;
+#pragma unroll
+      for (int i = 0; i < GH; ++i) {
+        const int hq = wg * GH + i;
+        float* rec = P.partials + (static_cast<int64_t>(pair + blockIdx.x) * G + hq) * kPartialFloats;
+        float vref = 0.f, vres = 0.f;
+        if constexpr (REF != kRefNone) vref = acc_ref[i];
+        if constexpr (REF == kRefInt4) {
+          float z = sRed[hq * C::NRED + 9];
+#pragma unroll
+          for (int g = 1; g < 4; ++g) z = (chunk == g) ? sRed[hq * C::NRED + 9 + g] : z;
+          vref += z;
+        }
+        if constexpr (RB != 0) {
+          float z = sRed[hq * C::NRED + 1];
+#pragma unroll
+          for (int g = 1; g < NGR; ++g) z = (g_res == g) ? sRed[hq * C::NRED + 1 + g] : z;
+          vres = acc_res[i] + z;
+        }
+        rec[4 + d_ref] = vref;
+        rec[4 + kD + d_res] = vres;
+        if (r == 0) {
+          rec[0] = m_run[i];
+          rec[1] = sRed[hq * C::NRED];
+        }
+      }
+    }
+    named_bar_sync(kBarWG + wg, 128);
+    if (r < GH * C::NRED) sRed[wg * GH * C::NRED + r] = 0.f;
+  }
+
+  // ---- release the tensor memory once every consumer is done with it
+  tc::fence_before_sync();
+  named_bar_sync(kBarAll, kNCT);
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dispatch
+// ---------------------------------------------------------------------------
+template <int REF, int RB, int RG, int G>
+cudaError_t launch_tc(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv, cudaStream_t s) {
+  using C = TcCfg<REF, RB, RG, G>;
+  if constexpr (!C::FITS) {
+    return cudaErrorInvalidValue;
+  } else {
+    auto kern = decode_tc_kernel<REF, RB, RG, G>;
+    static bool attr_done = false;  // per instantiation; set once per process
+    if (!attr_done) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      attr_done = true;
+    }
+    kern<<<p.num_ctas, kNT, C::SMEM_BYTES, s>>>(p, *tk, *tv);
+    return cudaGetLastError();
+  }
+}
+
+using TcFn = cudaError_t (*)(const DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);
+
+template <int REF, int RB, int RG, int G>
+TcFn tc_if_fits() {
+  if constexpr (TcCfg<REF, RB, RG, G>::FITS) return launch_tc<REF, RB, RG, G>;
+  else return nullptr;
+}
+
+template <int REF, int RB, int RG>
+TcFn tc_pick_g(int G) {
+  switch (G) {
+    case 2: return tc_if_fits<REF, RB, RG, 2>();
+    case 4: return tc_if_fits<REF, RB, RG, 4>();
+    case 8: return tc_if_fits<REF, RB, RG, 8>();
+    default: return nullptr;
+  }
+}
+
+TcFn tc_pick(int ref_kind, int res_bits, int res_group, int G) {
+  if (res_bits != 0 && res_group != 16 && res_group != 32) return nullptr;
+  const bool g16 = res_group == 16;
+  if (ref_kind == kRefBf16) {
+    if (res_bits == 0) return tc_pick_g<kRefBf16, 0, 32>(G);
+    if (res_bits == 2) return g16 ? tc_pick_g<kRefBf16, 2, 16>(G) : tc_pick_g<kRefBf16, 2, 32>(G);
+    if (res_bits == 4) return g16 ? tc_pick_g<kRefBf16, 4, 16>(G) : tc_pick_g<kRefBf16, 4, 32>(G);
+  } else if (ref_kind == kRefInt4) {
+    if (res_bits == 0) return tc_pick_g<kRefInt4, 0, 32>(G);
+    if (res_bits == 2) return g16 ? tc_pick_g<kRefInt4, 2, 16>(G) : tc_pick_g<kRefInt4, 2, 32>(G);
+    if (res_bits == 4) return g16 ? tc_pick_g<kRefInt4, 4, 16>(G) : tc_pick_g<kRefInt4, 4, 32>(G);
+  } else if (ref_kind == kRefNone) {
+    if (res_bits == 2) return g16 ? tc_pick_g<kRefNone, 2, 16>(G) : tc_pick_g<kRefNone, 2, 32>(G);
+    if (res_bits == 4) return g16 ? tc_pick_g<kRefNone, 4, 16>(G) : tc_pick_g<kRefNone, 4, 32>(G);
+  }
+  return nullptr;
+}
+
+}  // namespace
+
+bool tc_variant_supported(int ref_kind, int res_bits, int res_group, int G) {
+  return tc_pick(ref_kind, res_bits, res_group, G) != nullptr;
+}
+
+cudaError_t launch_split_tc(const DecodeParams& p, int ref_kind, int res_bits, int res_group,
+                            const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s) {
+  TcFn fn = tc_pick(ref_kind, res_bits, res_group, p.G);
+  if (fn == nullptr) return cudaErrorInvalidValue;
+  return fn(p, tmap_k, tmap_v, s);
+}
+
+}  // namespace rq

@@ -73,6 +73,8 @@ struct DecodeParams {
   float* partials;       // workspace
   int num_ctas;          // persistent grid size P of the split kernel
   int32_t* status;
+  int64_t tma_tokens;    // token extent of the bf16 tensor maps
+  int page_tokens;       // split granularity (set by launch_decode for the chosen kernel)
 };
 
 // Split-K partial record per (slot, head): m, l, pad, pad, acc_ref[128], acc_res[128]
@@ -83,10 +85,23 @@ int decode_grid_ctas(int device);  // persistent grid size for this device
 
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconstructParams& p, cudaStream_t s);
+// Decode kernels: the CUDA-core split kernel (64-token pages, any G) and the
+// tensor-core split kernel (128-token pages, G in {2, 4, 8}).
+enum DecodeKernel : int { kKernelAuto = RQ_DECODE_KERNEL_AUTO, kKernelSimt = RQ_DECODE_KERNEL_SIMT,
+                          kKernelTensor = RQ_DECODE_KERNEL_TENSOR };
+
 // ref_kind: RefKind; res_bits: 0 | 2 | 4; res_group: 16 | 32
-cudaError_t launch_decode(const DecodeParams& p, int ref_kind, int res_bits, int res_group,
+cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_group, int kernel,
                           const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
-bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G);
+bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, int kernel);
+// the kernel an automatic choice resolves to
+int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel);
+
+// tensor-core split kernel (rq_decode_tc.cu)
+bool tc_variant_supported(int ref_kind, int res_bits, int res_group, int G);
+cudaError_t launch_split_tc(const DecodeParams& p, int ref_kind, int res_bits, int res_group,
+                            const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
+constexpr int kTcPage = 128;
 
 // Records the calling thread's rq_last_error_message() text and returns `s`.
 rq_status set_last_error(rq_status s, const char* fmt, ...);

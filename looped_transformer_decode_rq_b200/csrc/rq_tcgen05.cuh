@@ -1,0 +1,168 @@
+// rq_tcgen05.cuh -- fifth-generation tensor-core (tcgen05) building blocks for
+// sm_100a, as inline PTX: tensor-memory allocation, shared-memory matrix
+// descriptors, instruction descriptors, single-thread MMA issue with mbarrier
+// commit, and 32-lane tensor-memory loads.
+//
+// Shared-memory matrix descriptor (64 bits): start address >> 4 in [0, 14),
+// leading-dimension byte offset >> 4 in [16, 30), stride-dimension byte offset
+// >> 4 in [32, 46), descriptor version 1 in [46, 48), base offset 0, layout
+// type in [61, 64) (0: no swizzle, 2: 128-byte swizzle).  The meaning of the
+// two offsets depends on the operand's major-ness and swizzle:
+//   K-major,  128B swizzle: rows of 128 bytes, 8-row groups `sbo` apart (lbo unused)
+//   MN-major, 128B swizzle: 8 K-rows of 128 MN-bytes form an atom; atoms along
+//                           K are `sbo` apart, 128-byte MN blocks `lbo` apart
+//   MN-major, no swizzle:   core matrices of 8 K-rows x 16 MN-bytes (128 bytes
+//                           contiguous); along K `lbo` apart, along MN `sbo` apart
+// Within a 128-byte swizzled K-major row the K offset of an MMA step is added
+// to the start address (the swizzle is applied to the final address bits).
+#pragma once
+
+#include <stdint.h>
+
+namespace rq {
+namespace tc {
+
+constexpr uint32_t kLayoutNone = 0;
+constexpr uint32_t kLayoutSw128 = 2;
+
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) |
+         (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
+         (static_cast<uint64_t>(layout) << 61);
+}
+
+// K-major operand, 128-byte swizzle, 8-row groups 1024 bytes apart
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) { return smem_desc(saddr, 16, 1024, kLayoutSw128); }
+
+// MN-major operand, 128-byte swizzle, K atoms 1024 bytes apart, MN blocks `mn_stride` apart
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t mn_stride) {
+  return smem_desc(saddr, mn_stride, 1024, kLayoutSw128);
+}
+
+// MN-major operand without swizzle: K groups of 8 rows `k_stride` apart,
+// 16-byte MN units `mn_stride` apart
+__device__ __forceinline__ uint64_t desc_mn_plain(uint32_t saddr, uint32_t k_stride, uint32_t mn_stride) {
+  return smem_desc(saddr, k_stride, mn_stride, kLayoutNone);
+}
+
+// Instruction descriptor of kind::f16 / kind::i8 (dense):
+//   [4,6) accumulator format (1: f32, 2: s32); [7,10) A format and [10,13) B
+//   format (kind::f16: 1 = bf16; kind::i8: 1 = signed); bit 15 / 16: A / B
+//   MN-major; [17,23) N >> 3; [24,29) M >> 4.
+constexpr uint32_t kAccF32 = 1, kAccS32 = 2;
+constexpr uint32_t kFmtBf16 = 1, kFmtS8 = 1;
+__host__ __device__ constexpr uint32_t instr_desc(uint32_t acc, uint32_t afmt, uint32_t bfmt, uint32_t a_mn, uint32_t b_mn, int M,
+                              int N) {
+  return (acc << 4) | (afmt << 7) | (bfmt << 10) | (a_mn << 15) | (b_mn << 16) |
+         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// ---- tensor memory allocation (executed by one whole warp)
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// ordering of tcgen05 operations around thread synchronisation
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// ---- MMA issue (one thread); D (+)= A * B^T with A: M x K, B: N x K
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_s8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The mbarrier at `bar` receives one arrival once every MMA this thread issued
+// before has completed.
+__device__ __forceinline__ void commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// ---- tensor memory -> registers.  Warp w may address lanes [32 (w % 4), +32);
+// thread i of the warp receives N consecutive 32-bit columns of lane base + i.
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]);
+
+template <>
+__device__ __forceinline__ void tmem_ld<1>(uint32_t taddr, uint32_t (&r)[1]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<2>(uint32_t taddr, uint32_t (&r)[2]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<4>(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+}
+template <>
+__device__ __forceinline__ void tmem_ld<8>(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+// N columns for N in {1, 2, 3, 4, 6, 8, 12}: one or two loads in one asm block,
+// straight into the destination registers
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 1 || N == 2 || N == 4 || N == 8) {
+    tmem_ld<N>(taddr, r);
+  } else if constexpr (N == 3) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%3];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%2}, [%4];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2])
+        : "r"(taddr), "r"(taddr + 2));
+  } else if constexpr (N == 6) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%6];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x2.b32 {%4, %5}, [%7];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5])
+        : "r"(taddr), "r"(taddr + 4));
+  } else {
+    static_assert(N == 12, "tensor-memory load width");
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%12];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8, %9, %10, %11}, [%13];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11])
+        : "r"(taddr), "r"(taddr + 8));
+  }
+}
+
+// Wait for this thread's tensor-memory loads; the registers passed through
+// afterwards cannot be read earlier by reordered code.
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+}  // namespace tc
+}  // namespace rq

@@ -31,12 +31,13 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_WORKSPACE, ERR_CUDA, ERR
 FLAG_BAD_INPUT, FLAG_POSITION, FLAG_CTX_LEN, FLAG_PIPE_TIMEOUT, FLAG_META_OVERFLOW = 1, 2, 4, 8, 16
 ALPHA_LS, ALPHA_ONE, ALPHA_ZERO, ALPHA_NORM_RATIO = 0, 1, 2, 3
 ANCHOR_LAST, ANCHOR_FIRST, ANCHOR_INTERVAL = 0, 1, 2
+DECODE_KERNEL_AUTO, DECODE_KERNEL_SIMT, DECODE_KERNEL_TENSOR = 0, 1, 2
 
 # every symbol the header declares (checked by the ABI tests)
 EXPORTED = ("rq_cache_layout", "rq_cache_create", "rq_cache_destroy", "rq_cache_info", "rq_encode",
             "rq_decode_workspace_size", "rq_decode_attention", "rq_bf16_decode_workspace_size",
             "rq_bf16_decode_attention", "rq_reconstruct", "rq_get_error", "rq_status_string",
-            "rq_last_error_message", "rq_decode_attention_static_scratch")
+            "rq_last_error_message", "rq_decode_attention_static_scratch", "rq_cache_set_decode_kernel")
 STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 
@@ -62,6 +63,7 @@ _sig = {
     "rq_cache_destroy": (None, [_vp]),
     "rq_cache_info": (C.c_int, [_vp, C.POINTER(Config), C.POINTER(Layout)]),
     "rq_encode": (C.c_int, [_vp, _vp, _vp, C.POINTER(_i64), _i32, _vp, _i32, _vp]),
+    "rq_cache_set_decode_kernel": (C.c_int, [_vp, _i32]),
     "rq_decode_workspace_size": (C.c_int, [_vp, C.POINTER(_i64)]),
     "rq_decode_attention": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp]),
     "rq_decode_attention_static_scratch": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp]),
@@ -149,6 +151,10 @@ class Cache:
     @property
     def handle(self):
         return self._h
+
+    def set_decode_kernel(self, kernel: int) -> None:
+        """DECODE_KERNEL_AUTO (default), DECODE_KERNEL_SIMT or DECODE_KERNEL_TENSOR."""
+        _check(_lib.rq_cache_set_decode_kernel(self._h, kernel), "rq_cache_set_decode_kernel")
 
     @property
     def G(self) -> int:

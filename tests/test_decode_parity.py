@@ -12,7 +12,7 @@ from tests.helpers import ATTN_TOL, oracle_encode, rel_err_rows, to_np32
 pytestmark = pytest.mark.gpu
 
 
-def run_case(rq, wl, loops=None, n_tail=None, lengths=None, scale=None):
+def run_case(rq, wl, loops=None, n_tail=None, lengths=None, scale=None, kernel=None):
     if n_tail is not None:
         wl = wl.with_(n_tail=n_tail)
     if lengths is not None:
@@ -20,6 +20,8 @@ def run_case(rq, wl, loops=None, n_tail=None, lengths=None, scale=None):
     inp = synth.make_inputs(wl, "cpu")
     cfgd = synth.cache_config_dict(wl)
     cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    if kernel is not None:
+        cache.set_decode_kernel(kernel)
     cache.encode(inp["k"].cuda(), inp["v"].cuda())
     enc = oracle_encode(inp, cfgd)
     ctx = inp["ctx_len"]
@@ -148,3 +150,53 @@ def test_recent_window_bf16_tail(librq, n_tail):
     wl = synth.Workload(name=f"tail{n_tail}", batch=2, kv_heads=2, q_heads=4, context=200, bits=(2, 2, 4, 4),
                         sigma=(0.3, 0.2, 0.1), outlier_p=0.01, seed=50 + n_tail)
     run_case(librq, wl, lengths=[200, 0], n_tail=n_tail)
+
+
+# ---------------------------------------------------------------------------
+# both decode kernels on the same cases: the CUDA-core kernel (64-token pages)
+# and the tensor-core kernel (128-token pages, G in {2, 4, 8})
+# ---------------------------------------------------------------------------
+TC_FORMATS = {
+    # name: (bits, group, rotate, alpha_mode, G values)
+    "bf16ref_int2g32_int4g32": ((2, 4, 2, 16), (32, 32, 32, 32), (1, 1, 1, 0), (0, 0, 3, 0), (2, 4)),
+    "bf16ref_int2g32": ((2, 2, 2, 16), (32, 32, 32, 32), (1, 1, 1, 0), (0, 3, 1, 0), (8,)),
+    "bf16ref_int2g16": ((2, 2, 2, 16), (16, 16, 16, 32), (1, 1, 0, 0), (0, 1, 0, 0), (2, 4)),
+    "int4anchor_int2g32_int4g16": ((2, 4, 2, 4), (32, 16, 16, 32), (1, 1, 1, 0), (0, 0, 3, 0), (2, 4, 8)),
+    "no_anchor_term": ((2, 4, 2, 16), (32, 32, 16, 32), (1, 0, 1, 0), (2, 2, 2, 0), (2, 4, 8)),
+}
+
+
+@pytest.mark.parametrize("kernel", ["simt", "tensor"])
+@pytest.mark.parametrize("fmt", sorted(TC_FORMATS))
+def test_both_kernels_formats_and_pages(librq, fmt, kernel):
+    """Every loop of the format (residual loops and the anchor loop) at each G the
+    tensor-core kernel implements, over 0, 1, 127, 128, 129 and 300 cached tokens
+    (several 128-token pages, partial pages and a partial last record block)."""
+    rq = librq
+    bits, group, rotate, alpha, Gs = TC_FORMATS[fmt]
+    for G in Gs:
+        wl = synth.Workload(name=f"{fmt}_G{G}", batch=6, kv_heads=2, q_heads=2 * G, context=300, bits=bits,
+                            group=group, rotate=rotate, alpha_mode=alpha, sigma=(0.3, 0.2, 0.1), outlier_p=0.02,
+                            seed=60 + G)
+        k = rq.DECODE_KERNEL_SIMT if kernel == "simt" else rq.DECODE_KERNEL_TENSOR
+        run_case(rq, wl, lengths=[300, 0, 128, 1, 129, 127], n_tail=2, kernel=k)
+
+
+@pytest.mark.parametrize("G", [4, 8])
+def test_tensor_kernel_many_pages(librq, G):
+    """Enough 128-token pages that every CTA of the persistent grid spans
+    segment borders, with ragged lengths."""
+    wl = synth.Workload(name=f"tc_long_G{G}", batch=3, kv_heads=4, q_heads=4 * G, context=5000,
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, seed=70 + G)
+    run_case(librq, wl, lengths=[5000, 2222, 129], loops=[0, 3], kernel=librq.DECODE_KERNEL_TENSOR)
+
+
+def test_tensor_kernel_rejects_unimplemented(librq):
+    rq = librq
+    wl = synth.Workload(name="tc_g1", batch=1, kv_heads=2, q_heads=2, context=64, seed=80)
+    cache = rq.Cache(rq.config_from_dict(synth.cache_config_dict(wl)), device="cuda")
+    cache.set_decode_kernel(rq.DECODE_KERNEL_TENSOR)
+    inp = synth.make_inputs(wl, "cpu")
+    with pytest.raises(rq.RQError) as e:
+        cache.decode_attention(0, inp["q"][0].cuda(), inp["ctx_len"].cuda())
+    assert e.value.status == rq.ERR_UNSUPPORTED
