@@ -329,6 +329,28 @@ def measure_workload(wl, steps, warmup, world, rank):
     torch.cuda.synchronize()
     call_ms = statistics.median(a.elapsed_time(b) for a, b in ev)
     res_bytes = call_bytes(cache.layout, cfgd, 0, tokens_total, B, Hq, Hkv, 1)
+
+    def call_gbs(kernel):
+        cache.set_decode_kernel(kernel)
+        for _ in range(3):
+            cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
+        evs = []
+        for _ in range(7):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        cache.set_decode_kernel(rq.DECODE_KERNEL_AUTO)
+        return round(res_bytes / (statistics.median(a.elapsed_time(b) for a, b in evs) * 1e-3) / 1e9, 1)
+
+    per_kernel = {"simt": call_gbs(rq.DECODE_KERNEL_SIMT)}
+    if wl.gqa in (2, 4, 8):
+        try:
+            per_kernel["tensor"] = call_gbs(rq.DECODE_KERNEL_TENSOR)
+        except rq.RQError:
+            per_kernel["tensor"] = None
     ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
 
     def bf16_step():
@@ -339,7 +361,8 @@ def measure_workload(wl, steps, warmup, world, rank):
     flags = cache.get_error()
     out = {"workload": wl.name, "tokens_per_s": round(job_tokens_per_s(B, world, ms), 1),
            "ms_per_step": round(ms, 4), "residual_loop_gbs": round(res_bytes / (call_ms * 1e-3) / 1e9, 1),
-           "residual_loop_bytes": res_bytes, "bf16_tokens_per_s": round(job_tokens_per_s(B, world, bms), 1),
+           "residual_loop_bytes": res_bytes, "residual_loop_gbs_by_kernel": per_kernel,
+           "bf16_tokens_per_s": round(job_tokens_per_s(B, world, bms), 1),
            "rq_speedup_vs_bf16": round(bms / ms, 3), "device_flags": flags}
     del cache, inp, outs, ws
     torch.cuda.empty_cache()
@@ -579,7 +602,8 @@ def run_rq(args, world, rank):
         del cache, inp, outs
         torch.cuda.empty_cache()
         extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 10, 3, world, rank),
-                 measure_workload(synth.gqa_long(batch=8), 10, 3, world, rank)]
+                 measure_workload(synth.gqa_long(batch=8), 10, 3, world, rank),
+                 measure_workload(synth.gqa_long(batch=8, q_heads=64), 10, 3, world, rank)]
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

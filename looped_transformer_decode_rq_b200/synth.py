@@ -106,11 +106,11 @@ def capacity_24layer(batch: int = 1, context: int = 8192) -> Workload:
                     seed=3, layers=24)
 
 
-def gqa_long(batch: int = 8, context: int = 32768) -> Workload:
-    """4 loops, 32 query heads / 8 KV heads, batch 8, ragged lengths
-    U{context/2 .. context}, INT2 loops 1-3 g=32, bf16 reference."""
-    return Workload(name=f"gqa_L4_Hq32_Hkv8_B{batch}_T{context}_ragged", batch=batch,
-                    kv_heads=8, q_heads=32, context=context,
+def gqa_long(batch: int = 8, context: int = 32768, q_heads: int = 32) -> Workload:
+    """4 loops, 32 (or `q_heads`) query heads / 8 KV heads, batch 8, ragged
+    lengths U{context/2 .. context}, INT2 loops 1-3 g=32, bf16 reference."""
+    return Workload(name=f"gqa_L4_Hq{q_heads}_Hkv8_B{batch}_T{context}_ragged", batch=batch,
+                    kv_heads=8, q_heads=q_heads, context=context,
                     length_range=(context // 2, context), sigma=(0.3, 0.2, 0.1),
                     outlier_p=0.01, seed=4)
 
