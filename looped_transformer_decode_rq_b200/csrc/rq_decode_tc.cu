@@ -44,7 +44,9 @@ namespace {
 constexpr int kTP = kTcPage;   // tokens per page
 constexpr int kNCW = 8;        // consumer warps (two warpgroups)
 constexpr int kNCT = kNCW * 32;
-constexpr int kNT = kNCT + 32; // + producer warp
+constexpr int kProducerWarp = kNCW;
+constexpr int kMmaWarp = kNCW + 1;
+constexpr int kNT = kNCT + 64; // + producer warp + MMA-issuing warp
 constexpr int kBarAll = 1;     // the 256 consumer threads
 constexpr int kBarWG = 2;      // warpgroup w uses kBarWG + w
 constexpr unsigned kFull = 0xffffffffu;
@@ -203,7 +205,7 @@ struct TcCfg {
   static constexpr int W_PRE = W_RED + 8 * NRED;         // [RQ_MAX_BATCH + 1] page prefix
   static constexpr int W_MISC = W_PRE + RQ_MAX_BATCH + 1;  // abort flag, tensor-memory base
   static constexpr int W_BAR = (W_MISC + 2 + 1) & ~1;    // 8-byte aligned mbarriers
-  static constexpr int NBARS = 2 * 4 + 2;
+  static constexpr int NBARS = 2 * 4 + 8;
   static constexpr int SMALL_BYTES = 4 * W_BAR + 8 * NBARS;
   static constexpr int FIXED = 1024 + F_END + SMALL_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
@@ -331,10 +333,15 @@ __global__ void __launch_bounds__(kNT, 1)
   volatile int* sAbort = reinterpret_cast<volatile int*>(sw + C::W_MISC);
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(sw + C::W_MISC + 1);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sw + C::W_BAR);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + 4;
-  uint64_t* sbar = bars + 8;
-  uint64_t* obar = bars + 9;
+  uint64_t* full = bars;       // [stage] the page's copies landed
+  uint64_t* empty = bars + 4;  // [stage] the page's value MMAs completed
+  uint64_t* sbar = bars + 8;   // score MMAs completed
+  uint64_t* obar = bars + 9;   // value MMAs completed
+  uint64_t* pstart = bars + 10;  // consumers are done with the previous page's tensor memory and tiles
+  uint64_t* kready = bars + 11;  // key code tiles written
+  uint64_t* v1ready = bars + 12; // anchor value weights (and cleared anchor rows) written
+  uint64_t* v2ready = bars + 13; // residual value weights (and value code tiles) written
+  uint64_t* done = bars + 14;    // every MMA of the CTA completed
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -375,6 +382,11 @@ __global__ void __launch_bounds__(kNT, 1)
     }
     mbar_init(smem_u32(sbar), 1);
     mbar_init(smem_u32(obar), 1);
+    mbar_init(smem_u32(pstart), kNCW);
+    mbar_init(smem_u32(kready), 4);
+    mbar_init(smem_u32(v1ready), kNCW);
+    mbar_init(smem_u32(v2ready), kNCW);
+    mbar_init(smem_u32(done), 1);
     fence_barrier_init();
   }
   __syncthreads();
@@ -408,6 +420,19 @@ __global__ void __launch_bounds__(kNT, 1)
     do { ++it.b; } while (it.b < B && nt_of(it.b) == 0);
   };
 
+  // A wait that timed out marks the CTA aborted; later waits then return at once
+  // so that every thread still walks the same barrier sequence to the end.
+  auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) -> bool {
+    if (*sAbort) return false;
+    if (mbar_wait_bounded(smem_u32(bar), parity)) return true;
+    set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+    *sAbort = 1;
+    return false;
+  };
+  constexpr bool NEED_KREADY = (RB != 0) || (REF == kRefInt4);
+  constexpr bool HAS_V1 = REF != kRefNone;
+  constexpr bool HAS_V2 = RB != 0;
+
   // ---- tensor memory for the page's score and value sums
   if (warp == 0) {
     tc::tmem_alloc(smem_u32(sTmem), C::TMEM_COLS);
@@ -419,7 +444,7 @@ __global__ void __launch_bounds__(kNT, 1)
   const uint32_t tbase = *sTmem;
 
   // ========================= producer warp =========================
-  if (warp == kNCW) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       if constexpr (REF == kRefBf16) {
         prefetch_tensormap(&tmK);
@@ -448,6 +473,84 @@ __global__ void __launch_bounds__(kNT, 1)
     return;
   }
 
+  // ========================= MMA-issuing warp =========================
+  // One thread issues every tcgen05 MMA of the CTA, page by page, as soon as
+  // its operands are ready: the bf16 anchor score MMAs when the page lands,
+  // the integer score MMAs when the key code tiles are written, and the value
+  // MMAs in two groups as their weight operands are written.
+  if (warp == kMmaWarp) {
+    if (lane == 0) {
+      uint8_t* UKm = fx + C::F_UK;
+      uint8_t* UVm = fx + C::F_UV;
+      uint8_t* URKm = fx + C::F_URK;
+      uint8_t* URVm = fx + C::F_URV;
+      uint8_t* QBm = fx + C::F_QB;
+      uint8_t* QAm = fx + C::F_QA;
+      uint8_t* HQm = fx + C::F_HQ;
+      uint8_t* WBm = fx + C::F_WB;
+      uint8_t* WAm = fx + C::F_WA;
+      uint8_t* WRm = fx + C::F_WR;
+      for (int k = 0; k < n_pages; ++k) {
+        const int s = k % C::STAGES;
+        uint8_t* st = stages + s * C::STAGE_BYTES;
+        const uint32_t ph = k & 1;
+        wait_or_abort(pstart, ph);
+        wait_or_abort(&full[s], (k / C::STAGES) & 1);
+        tc::fence_after_sync();
+        if constexpr (REF == kRefBf16) {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            tc::mma_bf16(tbase + C::S_REF, tc::desc_k_sw128(smem_u32(st + C::O_REFK + (ks >> 2) * 16384 + (ks & 3) * 32)),
+                         tc::desc_k_sw128(smem_u32(QBm + (ks >> 2) * 2048 + (ks & 3) * 32)), C::ID_SB, ks > 0);
+        }
+        if constexpr (NEED_KREADY) {
+          wait_or_abort(kready, ph);
+          tc::fence_after_sync();
+          if constexpr (REF == kRefInt4) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tc::mma_s8(tbase + C::S_REF + C::N_SA * c, tc::desc_k_sw128(smem_u32(URKm + 32 * c)),
+                         tc::desc_k_sw128(smem_u32(QAm + 32 * c)), C::ID_SA, 0);
+          }
+          if constexpr (RB != 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tc::mma_s8(tbase + C::S_RES + C::N_SR * c, tc::desc_k_sw128(smem_u32(UKm + 32 * c)),
+                         tc::desc_k_sw128(smem_u32(HQm + 32 * c)), C::ID_SR, 0);
+          }
+        }
+        tc::commit(smem_u32(sbar));
+        if constexpr (HAS_V1) {
+          wait_or_abort(v1ready, ph);
+          tc::fence_after_sync();
+          if constexpr (REF == kRefBf16) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              tc::mma_bf16(tbase + C::O_REF, tc::desc_mn_sw128(smem_u32(st + C::O_REFV + ks * 2048), 16384),
+                           tc::desc_mn_plain(smem_u32(WBm + ks * 256), 128, 2048), C::ID_VB, ks > 0);
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              tc::mma_s8(tbase + C::O_REF, tc::desc_mn_sw128(smem_u32(URVm + ks * 4096), 16384),
+                         tc::desc_mn_plain(smem_u32(WAm + ks * 512), 128, 2048), C::ID_VA, ks > 0);
+          }
+        }
+        if constexpr (HAS_V2) {
+          wait_or_abort(v2ready, ph);
+          tc::fence_after_sync();
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_s8(tbase + C::O_RES, tc::desc_mn_sw128(smem_u32(UVm + ks * 4096), 16384),
+                       tc::desc_mn_plain(smem_u32(WRm + ks * 512), 128, 2048), C::ID_VR, ks > 0);
+        }
+        tc::commit(smem_u32(obar));
+        tc::commit(smem_u32(&empty[s]));
+      }
+      tc::commit(smem_u32(done));
+    }
+    return;
+  }
+
   // ========================= consumer warpgroups =========================
   const int wg = warp >> 2;                  // query heads [wg * GH, wg * GH + GH)
   const int r = tid & 127;                   // tensor-memory lane: token, then dim position
@@ -470,9 +573,7 @@ __global__ void __launch_bounds__(kNT, 1)
   PageIter it;
   seek(it, x0);
   int k = 0;
-  uint32_t sph = 0, oph = 0;
-  bool aborted = false;
-  while (k < n_pages && !aborted) {
+  while (k < n_pages) {
     const int b = it.b, h = it.h;
     const int seg_pages = min(nt_of(b) - it.page, n_pages - k);
     int len_b = P.ctx_len[b];
@@ -531,42 +632,19 @@ __global__ void __launch_bounds__(kNT, 1)
       const int s = k % C::STAGES;
       uint8_t* st = stages + s * C::STAGE_BYTES;
       const int n_valid = min(kTP, len_b - it.page * kTP);
-      if (!mbar_wait_bounded(smem_u32(&full[s]), (k / C::STAGES) & 1)) {
-        set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-        *sAbort = 1;
-      }
+      const uint32_t ph = k & 1;
+      // the previous page's tensor memory and operand tiles are free
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(pstart));
+      wait_or_abort(&full[s], (k / C::STAGES) & 1);
       // ---- expand the packed codes (warpgroup 0: keys, 1: values)
       if constexpr (RB != 0) expand_row<RB>(st + (wg ? C::O_RESV : C::O_RESK) + r * C::CB, wg ? UV : UK, r);
       if constexpr (REF == kRefInt4) expand_row<4>(st + (wg ? C::O_REFV : C::O_REFK) + r * 64, wg ? URV : URK, r);
       fence_proxy_async_smem();
-      tc::fence_before_sync();
-      named_bar_sync(kBarAll, kNCT);
-      if (*sAbort) {  // written only before the barrier above: uniform
-        aborted = true;
-        break;
-      }
-
-      // ---- score MMAs: D[t][n] over the page's 128 tokens
-      if (tid == 0) {
-        tc::fence_after_sync();
-        if constexpr (REF == kRefBf16) {
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            tc::mma_bf16(tbase + C::S_REF, tc::desc_k_sw128(smem_u32(st + C::O_REFK + (ks >> 2) * 16384 + (ks & 3) * 32)),
-                         tc::desc_k_sw128(smem_u32(QB + (ks >> 2) * 2048 + (ks & 3) * 32)), C::ID_SB, ks > 0);
-        } else if constexpr (REF == kRefInt4) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tc::mma_s8(tbase + C::S_REF + C::N_SA * c, tc::desc_k_sw128(smem_u32(URK + 32 * c)),
-                       tc::desc_k_sw128(smem_u32(QA + 32 * c)), C::ID_SA, 0);
-        }
-        if constexpr (RB != 0) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tc::mma_s8(tbase + C::S_RES + C::N_SR * c, tc::desc_k_sw128(smem_u32(UK + 32 * c)),
-                       tc::desc_k_sw128(smem_u32(HQ + 32 * c)), C::ID_SR, 0);
-        }
-        tc::commit(smem_u32(sbar));
+      if constexpr (NEED_KREADY) {
+        __syncwarp();
+        if (wg == 0 && lane == 0) mbar_arrive(smem_u32(kready));
       }
 
       // ---- per-token metadata (thread = token r), zero past the context
@@ -610,8 +688,7 @@ __global__ void __launch_bounds__(kNT, 1)
         }
       }
 
-      if (!mbar_wait_bounded(smem_u32(sbar), sph)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-      sph ^= 1u;
+      wait_or_abort(sbar, ph);
       tc::fence_after_sync();
 
       // ---- scores of token r for this warpgroup's heads
@@ -749,6 +826,13 @@ __global__ void __launch_bounds__(kNT, 1)
         if constexpr (GH == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         else if constexpr (GH == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
         else *reinterpret_cast<uint32_t*>(dst) = pk[0];
+        // bf16 anchor rows past the context may hold anything: clear them so
+        // that their zero weights give exact zeros
+        if (!valid) {
+          uint4* row = reinterpret_cast<uint4*>(st + C::O_REFV + wg * 16384 + r * 128);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) row[q] = make_uint4(0u, 0u, 0u, 0u);
+        }
       }
       auto put_w8 = [&](uint8_t* tile, int ng, int g, const float (&w)[GH]) {
         // three signed bytes per weight; this warpgroup's GH heads are contiguous rows
@@ -782,6 +866,13 @@ __global__ void __launch_bounds__(kNT, 1)
           put_w8(WA, 4, g, w);
         }
       }
+      // the scores are in registers: the value sums may now overwrite their columns
+      tc::fence_before_sync();
+      if constexpr (HAS_V1) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(v1ready));
+      }
       if constexpr (RB != 0) {
 #pragma unroll
         for (int g = 0; g < NGR; ++g) {
@@ -792,41 +883,10 @@ __global__ void __launch_bounds__(kNT, 1)
           put_w8(WR, NGR, g, w);
         }
       }
-      // bf16 anchor rows past the context may hold anything: clear them so that
-      // their zero weights give exact zeros
-      if constexpr (REF == kRefBf16) {
-        if (!valid) {
-          uint4* row = reinterpret_cast<uint4*>(st + C::O_REFV + wg * 16384 + r * 128);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) row[q] = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-      fence_proxy_async_smem();
-      tc::fence_before_sync();
-      named_bar_sync(kBarAll, kNCT);
-
-      // ---- value MMAs: D[d][n] over the page's 128 tokens
-      if (tid == 0) {
-        tc::fence_after_sync();
-        if constexpr (REF == kRefBf16) {
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            tc::mma_bf16(tbase + C::O_REF, tc::desc_mn_sw128(smem_u32(st + C::O_REFV + ks * 2048), 16384),
-                         tc::desc_mn_plain(smem_u32(WB + ks * 256), 128, 2048), C::ID_VB, ks > 0);
-        } else if constexpr (REF == kRefInt4) {
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            tc::mma_s8(tbase + C::O_REF, tc::desc_mn_sw128(smem_u32(URV + ks * 4096), 16384),
-                       tc::desc_mn_plain(smem_u32(WA + ks * 512), 128, 2048), C::ID_VA, ks > 0);
-        }
-        if constexpr (RB != 0) {
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            tc::mma_s8(tbase + C::O_RES, tc::desc_mn_sw128(smem_u32(UV + ks * 4096), 16384),
-                       tc::desc_mn_plain(smem_u32(WR + ks * 512), 128, 2048), C::ID_VR, ks > 0);
-        }
-        tc::commit(smem_u32(obar));
-        tc::commit(smem_u32(&empty[s]));
+      if constexpr (HAS_V2) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(v2ready));
       }
 
       // ---- running denominators and offset sums (thread = token r)
@@ -844,8 +904,7 @@ __global__ void __launch_bounds__(kNT, 1)
         }
       }
 
-      if (!mbar_wait_bounded(smem_u32(obar), oph)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-      oph ^= 1u;
+      wait_or_abort(obar, ph);
       tc::fence_after_sync();
 
       // ---- merge the page's value sums (thread = dim position r)
@@ -904,10 +963,8 @@ __global__ void __launch_bounds__(kNT, 1)
           acc_res[i] = fmaf(acc_res[i], crun[i], pm[i] * f * x);
         }
       }
-      tc::fence_before_sync();
       advance(it);
     }
-    if (aborted) break;
 
     // ---- flush this (b, h) segment: one partial record per query head
 #pragma unroll
@@ -965,10 +1022,11 @@ __global__ void __launch_bounds__(kNT, 1)
     if (r < GH * C::NRED) sRed[wg * GH * C::NRED + r] = 0.f;
   }
 
-  // ---- release the tensor memory once every consumer is done with it
+  // ---- release the tensor memory once every MMA and every consumer is done with it
   tc::fence_before_sync();
   named_bar_sync(kBarAll, kNCT);
   if (warp == 0) {
+    if (!mbar_wait_bounded(smem_u32(done), 0)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
     tc::fence_after_sync();
     tc::tmem_dealloc(tbase, C::TMEM_COLS);
   }
