@@ -346,7 +346,7 @@ def measure_workload(wl, steps, warmup, world, rank):
         return round(res_bytes / (statistics.median(a.elapsed_time(b) for a, b in evs) * 1e-3) / 1e9, 1)
 
     per_kernel = {"simt": call_gbs(rq.DECODE_KERNEL_SIMT)}
-    if wl.gqa in (2, 4, 8):
+    if wl.gqa in (1, 2, 4, 8):
         try:
             per_kernel["tensor"] = call_gbs(rq.DECODE_KERNEL_TENSOR)
         except rq.RQError:

@@ -50,12 +50,19 @@ constexpr int kNT = kNCT + 64; // + producer warp + MMA-issuing warp
 constexpr int kBarAll = 1;     // the 256 consumer threads
 constexpr int kBarWG = 2;      // warpgroup w uses kBarWG + w
 constexpr unsigned kFull = 0xffffffffu;
-constexpr float kQ3 = 8323072.f;  // 24-bit range whose top byte stays in [-127, 127]
+constexpr float kQ3 = 8323072.f;  // signed 24-bit range whose top byte stays in [-127, 127]
+constexpr float kU3 = 16777215.f; // unsigned 24-bit range
 constexpr int kSmemLimit = 227 * 1024;
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -138,7 +145,7 @@ constexpr int round16(int x) { return (x + 15) & ~15; }
 
 template <int REF, int RB, int RG, int G>
 struct TcCfg {
-  static constexpr int GH = G / 2;                       // query heads per warpgroup
+  static constexpr int GH = G == 1 ? 1 : G / 2;          // query heads per warpgroup
   static constexpr int NGR = RB ? kD / RG : 0;            // residual groups
   static constexpr int NPAR = RG == 16 ? 2 : 1;           // residual groups per 32-dim chunk
   static constexpr int NGA = REF == kRefInt4 ? 4 : 0;     // INT4 anchor groups
@@ -150,24 +157,26 @@ struct TcCfg {
   static constexpr int MB = RB ? 4 * NGR : 0;
   static constexpr int AL_REC = HAS_ALPHA ? 4 : 0;
   // MMA widths (N).  Query and weight operands carry 24-bit integers as three
-  // signed bytes (j = 0: top, 1: middle, 2: bottom), one B row per byte.
-  //   score rows per 32-dim chunk: (parity, head, byte)  n = p * 3G + 3 h + j
-  //   value rows: (byte, group, head)                    n = j * NG * G + g * G + h
+  // bytes (j = 0: top, 1: middle, 2: bottom), one B row per byte; signed except
+  // the residual value weights, which are non-negative.
+  //   score rows per 32-dim chunk: (parity, head, byte)   n = p * 3G + 3 h + j
+  //   value rows: (byte, warpgroup, group, head in it)    n = j * NG * G + wg * NG * GH + g * GH + i
+  // so that a thread writes each byte plane of its warpgroup as one vector
   static constexpr int N_SA = round16(3 * G);                          // INT4 anchor score columns per chunk
   static constexpr int N_SR = round16(3 * G * NPAR);                   // residual score columns per chunk
   static constexpr int N_VA = round16(3 * 4 * G);                      // INT4 anchor value columns
   static constexpr int N_VR = round16(3 * NGR * G);                    // residual value columns
-  // tensor-memory columns: the value sums reuse the score columns (the scores
-  // are read before the value MMAs are issued)
+  // tensor-memory columns: scores, then value sums (separate, so that the next
+  // page's scores can be computed while this page's value sums are read)
   static constexpr int S_REF = 0;
   static constexpr int S_REF_COLS = REF == kRefBf16 ? 16 : (REF == kRefInt4 ? 4 * N_SA : 0);
   static constexpr int S_RES = S_REF + S_REF_COLS;
   static constexpr int S_COLS = S_RES + (RB ? 4 * N_SR : 0);
-  static constexpr int O_REF = 0;
+  static constexpr int O_REF = S_COLS;
   static constexpr int O_REF_COLS = REF == kRefBf16 ? 16 : (REF == kRefInt4 ? N_VA : 0);
   static constexpr int O_RES = O_REF + O_REF_COLS;
   static constexpr int O_COLS = O_RES + (RB ? N_VR : 0);
-  static constexpr int COLS = S_COLS > O_COLS ? S_COLS : O_COLS;
+  static constexpr int COLS = O_COLS;
   static constexpr int TMEM_COLS = COLS <= 32 ? 32 : COLS <= 64 ? 64 : COLS <= 128 ? 128 : COLS <= 256 ? 256 : 512;
   // stage layout (pieces 1024-byte aligned)
   static constexpr int al(int x) { return (x + 1023) & ~1023; }
@@ -210,7 +219,7 @@ struct TcCfg {
   static constexpr int FIXED = 1024 + F_END + SMALL_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT >= 4 ? 4 : (STAGES_FIT >= 2 ? STAGES_FIT : 2);
-  static constexpr bool FITS = STAGES_FIT >= 2;
+  static constexpr bool FITS = STAGES_FIT >= 2 && COLS <= 512;
   static constexpr int SMEM_BYTES = FIXED + STAGES * STAGE_BYTES;
   // instruction descriptors
   static constexpr uint32_t ID_SB = tc::instr_desc(tc::kAccF32, tc::kFmtBf16, tc::kFmtBf16, 0, 0, 128, 16);
@@ -218,10 +227,9 @@ struct TcCfg {
   static constexpr uint32_t ID_SR = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 0, 0, 128, N_SR);
   static constexpr uint32_t ID_VB = tc::instr_desc(tc::kAccF32, tc::kFmtBf16, tc::kFmtBf16, 1, 1, 128, 16);
   static constexpr uint32_t ID_VA = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 1, 1, 128, N_VA);
-  static constexpr uint32_t ID_VR = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 1, 1, 128, N_VR);
-  static_assert(G == 2 || G == 4 || G == 8, "query heads per kv-head");
+  static constexpr uint32_t ID_VR = tc::instr_desc(tc::kAccS32, 0, 0, 1, 1, 128, N_VR);  // unsigned bytes
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "query heads per kv-head");
   static_assert(N_VA <= 256 && N_VR <= 256 && N_SR <= 256, "MMA width");
-  static_assert(COLS <= 512, "tensor memory");
 };
 
 // ---------------------------------------------------------------------------
@@ -300,6 +308,40 @@ __device__ __forceinline__ void put_q_s24(uint8_t* tile, const float (&x)[4], in
   if (lane == 0) *scale_out = m * (1.f / kQ3) * scale_log2;
 }
 
+// Byte planes of NB 24-bit values v[] (byte 2 = top): out[j] holds byte 2 - j
+// of every value, value m at byte m of the plane.
+template <int NB>
+__device__ __forceinline__ void byte_planes(const uint32_t (&v)[NB], uint32_t (&out)[3][NB / 4]) {
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    const uint32_t sel = (2 - j) | ((6 - j) << 4);
+#pragma unroll
+    for (int w = 0; w < NB / 4; ++w) {
+      const uint32_t lo = __byte_perm(v[4 * w], v[4 * w + 1], sel);
+      const uint32_t hi = __byte_perm(v[4 * w + 2], v[4 * w + 3], sel);
+      out[j][w] = __byte_perm(lo, hi, 0x5410);
+    }
+  }
+}
+
+// store NB bytes (4, 8, 16 or 32) of a byte plane at rows n0.. of an MN-major
+// (no swizzle) int8 operand, token row offset `wrow`
+template <int NB>
+__device__ __forceinline__ void put_plane(uint8_t* tile, int n0, int wrow, const uint32_t (&w)[NB / 4]) {
+  uint8_t* dst = tile + (n0 >> 4) * 2048 + wrow + (n0 & 15);
+  if constexpr (NB == 4) {
+    *reinterpret_cast<uint32_t*>(dst) = w[0];
+  } else if constexpr (NB == 8) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+  } else if constexpr (NB == 16) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    static_assert(NB == 32, "byte plane width");
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(dst + 2048) = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
 // 65536 b2 + 256 b1 + b0 of three int32 byte-products (as fp32)
 __device__ __forceinline__ float comb24(uint32_t b2, uint32_t b1, uint32_t b0) {
   return fmaf(65536.f, static_cast<float>(static_cast<int>(b2)),
@@ -337,7 +379,7 @@ __global__ void __launch_bounds__(kNT, 1)
   uint64_t* empty = bars + 4;  // [stage] the page's value MMAs completed
   uint64_t* sbar = bars + 8;   // score MMAs completed
   uint64_t* obar = bars + 9;   // value MMAs completed
-  uint64_t* pstart = bars + 10;  // consumers are done with the previous page's tensor memory and tiles
+  uint64_t* sfree = bars + 10;   // the page's query operands are written, the previous scores read
   uint64_t* kready = bars + 11;  // key code tiles written
   uint64_t* v1ready = bars + 12; // anchor value weights (and cleared anchor rows) written
   uint64_t* v2ready = bars + 13; // residual value weights (and value code tiles) written
@@ -382,7 +424,7 @@ __global__ void __launch_bounds__(kNT, 1)
     }
     mbar_init(smem_u32(sbar), 1);
     mbar_init(smem_u32(obar), 1);
-    mbar_init(smem_u32(pstart), kNCW);
+    mbar_init(smem_u32(sfree), kNCW);
     mbar_init(smem_u32(kready), 4);
     mbar_init(smem_u32(v1ready), kNCW);
     mbar_init(smem_u32(v2ready), kNCW);
@@ -494,7 +536,7 @@ __global__ void __launch_bounds__(kNT, 1)
         const int s = k % C::STAGES;
         uint8_t* st = stages + s * C::STAGE_BYTES;
         const uint32_t ph = k & 1;
-        wait_or_abort(pstart, ph);
+        wait_or_abort(sfree, ph);
         wait_or_abort(&full[s], (k / C::STAGES) & 1);
         tc::fence_after_sync();
         if constexpr (REF == kRefBf16) {
@@ -552,10 +594,20 @@ __global__ void __launch_bounds__(kNT, 1)
   }
 
   // ========================= consumer warpgroups =========================
-  const int wg = warp >> 2;                  // query heads [wg * GH, wg * GH + GH)
+  // G >= 2: warpgroup wg scores and sums query heads [wg GH, wg GH + GH).
+  // G == 1: both warpgroups score the one head; warpgroup 0 owns the anchor
+  // value sums and the denominator, warpgroup 1 the residual value sums.
+  // Pages are software-pipelined by one: while page k's value MMAs run, the
+  // next page's key codes are expanded and its score MMAs issued.
+  constexpr bool SPLIT = (G == 1);
+  const int wg = warp >> 2;
   const int r = tid & 127;                   // tensor-memory lane: token, then dim position
   const uint32_t tl = tbase + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
   const int chunk = warp & 3;                // 32-dim chunk of this thread's position
+  const int hb = SPLIT ? 0 : wg * GH;        // first query head of this warpgroup
+  const int wgo = SPLIT ? 0 : wg;            // warpgroup slot in operand rows / columns
+  const bool own_ref = !SPLIT || wg == 0;    // anchor value sums, maximum and denominator
+  const bool own_res = !SPLIT || wg == 1;    // residual value sums
   uint8_t* UK = fx + C::F_UK;
   uint8_t* UV = fx + C::F_UV;
   uint8_t* URK = fx + C::F_URK;
@@ -570,16 +622,13 @@ __global__ void __launch_bounds__(kNT, 1)
   const int par_r = RB == 2 ? ((r >> 2) & 1) : ((r >> 3) & 1);
   const int g_res = RG == 16 ? 2 * chunk + par_r : chunk;
 
-  PageIter it;
-  seek(it, x0);
-  int k = 0;
-  while (k < n_pages) {
-    const int b = it.b, h = it.h;
-    const int seg_pages = min(nt_of(b) - it.page, n_pages - k);
-    int len_b = P.ctx_len[b];
-    len_b = len_b < 0 ? 0 : (len_b > P.capacity ? P.capacity : len_b);
+  auto seq_len = [&](int b) {
+    const int len = P.ctx_len[b];
+    return len < 0 ? 0 : (len > P.capacity ? P.capacity : len);
+  };
 
-    // ---- segment set-up: query operands of the G heads of (b, h)
+  // query operands of the G heads of (b, h), for the score MMAs
+  auto setup = [&](int b, int h) {
     if (warp < G) {
       const int hq = warp;
       const int qh = h * G + hq;
@@ -614,10 +663,35 @@ __global__ void __launch_bounds__(kNT, 1)
     }
     fence_proxy_async_smem();
     named_bar_sync(kBarAll, kNCT);
+  };
+  // "page k may be scored": its query operands are written and the previous
+  // page's scores have been read out of tensor memory
+  auto release_scores = [&]() {
+    tc::fence_before_sync();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(sfree));
+  };
+  // warpgroup 0: key-side code tiles of the page in stage `st`
+  auto expand_keys = [&](const uint8_t* st) {
+    if constexpr (RB != 0) expand_row<RB>(st + C::O_RESK + r * C::CB, UK, r);
+    if constexpr (REF == kRefInt4) expand_row<4>(st + C::O_REFK + r * 64, URK, r);
+    fence_proxy_async_smem();
+    if constexpr (NEED_KREADY) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(kready));
+    }
+  };
+  // warpgroup 1: value-side code tiles (published by its later weight arrivals)
+  auto expand_values = [&](const uint8_t* st) {
+    if constexpr (RB != 0) expand_row<RB>(st + C::O_RESV + r * C::CB, UV, r);
+    if constexpr (REF == kRefInt4) expand_row<4>(st + C::O_REFV + r * 64, URV, r);
+    fence_proxy_async_smem();
+  };
 
-    // per-warpgroup running state (query heads wg*GH + i)
-    float m_run[GH], l_thr[GH], acc_ref[GH], acc_res[GH];
-    float zr[GH][NGR > 0 ? NGR : 1], za[GH][NGA > 0 ? NGA : 1];
+  // per-segment running state (query heads hb + i)
+  float m_run[GH], l_thr[GH], acc_ref[GH], acc_res[GH];
+  float zr[GH][NGR > 0 ? NGR : 1], za[GH][NGA > 0 ? NGA : 1];
+  auto reset_state = [&]() {
 #pragma unroll
     for (int i = 0; i < GH; ++i) {
       m_run[i] = -INFINITY;
@@ -627,191 +701,185 @@ __global__ void __launch_bounds__(kNT, 1)
 #pragma unroll
       for (int g = 0; g < (NGA > 0 ? NGA : 1); ++g) za[i][g] = 0.f;
     }
+  };
 
-    for (int sp = 0; sp < seg_pages; ++sp, ++k) {
-      const int s = k % C::STAGES;
-      uint8_t* st = stages + s * C::STAGE_BYTES;
-      const int n_valid = min(kTP, len_b - it.page * kTP);
-      const uint32_t ph = k & 1;
-      // the previous page's tensor memory and operand tiles are free
-      tc::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(pstart));
-      wait_or_abort(&full[s], (k / C::STAGES) & 1);
-      // ---- expand the packed codes (warpgroup 0: keys, 1: values)
-      if constexpr (RB != 0) expand_row<RB>(st + (wg ? C::O_RESV : C::O_RESK) + r * C::CB, wg ? UV : UK, r);
-      if constexpr (REF == kRefInt4) expand_row<4>(st + (wg ? C::O_REFV : C::O_REFK) + r * 64, wg ? URV : URK, r);
-      fence_proxy_async_smem();
-      if constexpr (NEED_KREADY) {
-        __syncwarp();
-        if (wg == 0 && lane == 0) mbar_arrive(smem_u32(kready));
-      }
+  // ---- prologue: operands of page 0
+  PageIter cur;
+  seek(cur, x0);
+  reset_state();
+  setup(cur.b, cur.h);
+  release_scores();
+  wait_or_abort(&full[0], 0);
+  if (wg == 0) expand_keys(stages);
+  else expand_values(stages);
 
-      // ---- per-token metadata (thread = token r), zero past the context
-      const bool valid = r < n_valid;
-      float aK = 1.f, aV = 1.f;
-      if constexpr (C::HAS_ALPHA) {
-        const float2 a = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_AL + r * 4));
-        aK = a.x;
-        aV = a.y;
-      }
-      if (!valid) aK = aV = 0.f;
-      float sK[NGR > 0 ? NGR : 1], zK[NGR > 0 ? NGR : 1], sV[NGR > 0 ? NGR : 1], zV[NGR > 0 ? NGR : 1];
-      if constexpr (RB != 0) {
+  for (int k = 0; k < n_pages; ++k) {
+    const int s = k % C::STAGES;
+    uint8_t* st = stages + s * C::STAGE_BYTES;
+    const uint32_t ph = k & 1;
+    const int n_valid = min(kTP, seq_len(cur.b) - cur.page * kTP);
+    const bool last = k + 1 == n_pages;
+    PageIter nxt = cur;
+    if (!last) advance(nxt);
+    const bool seg_end = last || nxt.b != cur.b || nxt.h != cur.h;
+    const int s1 = (k + 1) % C::STAGES;
+    uint8_t* st1 = stages + s1 * C::STAGE_BYTES;
+
+    // ---- per-token metadata (thread = token r), zero past the context
+    const bool valid = r < n_valid;
+    float aK = 1.f, aV = 1.f;
+    if constexpr (C::HAS_ALPHA) {
+      const float2 a = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_AL + r * 4));
+      aK = a.x;
+      aV = a.y;
+    }
+    if (!valid) aK = aV = 0.f;
+    float sK[NGR > 0 ? NGR : 1], zK[NGR > 0 ? NGR : 1], sV[NGR > 0 ? NGR : 1], zV[NGR > 0 ? NGR : 1];
+    if constexpr (RB != 0) {
 #pragma unroll
-        for (int g = 0; g < NGR; g += 4) {
-          const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_RESMK + r * C::MB + 4 * g);
-          const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_RESMV + r * C::MB + 4 * g);
-          const uint32_t wk[4] = {mk.x, mk.y, mk.z, mk.w}, wv[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 a = half2_bits_to_f2(wk[u]), c2 = half2_bits_to_f2(wv[u]);
-            sK[g + u] = valid ? a.x : 0.f;
-            zK[g + u] = valid ? a.y : 0.f;
-            sV[g + u] = valid ? c2.x : 0.f;
-            zV[g + u] = valid ? c2.y : 0.f;
-          }
-        }
-      }
-      float sAk[4], zAk[4], sAv[4], zAv[4];
-      if constexpr (REF == kRefInt4) {
-        const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_REFMK + r * 16);
-        const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_REFMV + r * 16);
+      for (int g = 0; g < NGR; g += 4) {
+        const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_RESMK + r * C::MB + 4 * g);
+        const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_RESMV + r * C::MB + 4 * g);
         const uint32_t wk[4] = {mk.x, mk.y, mk.z, mk.w}, wv[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float2 a = half2_bits_to_f2(wk[u]), c2 = half2_bits_to_f2(wv[u]);
-          sAk[u] = valid ? a.x : 0.f;
-          zAk[u] = valid ? a.y : 0.f;
-          sAv[u] = valid ? c2.x : 0.f;
-          zAv[u] = valid ? c2.y : 0.f;
+          sK[g + u] = valid ? a.x : 0.f;
+          zK[g + u] = valid ? a.y : 0.f;
+          sV[g + u] = valid ? c2.x : 0.f;
+          zV[g + u] = valid ? c2.y : 0.f;
         }
       }
-
-      wait_or_abort(sbar, ph);
-      tc::fence_after_sync();
-
-      // ---- scores of token r for this warpgroup's heads
-      float S[GH];
+    }
+    float sAk[4], zAk[4], sAv[4], zAv[4];
+    if constexpr (REF == kRefInt4) {
+      const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_REFMK + r * 16);
+      const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_REFMV + r * 16);
+      const uint32_t wk[4] = {mk.x, mk.y, mk.z, mk.w}, wv[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
-      for (int i = 0; i < GH; ++i) S[i] = 0.f;
-      if constexpr (REF == kRefBf16) {
-        uint32_t v[GH > 1 ? GH : 2];
-        if constexpr (GH == 1) {
-          uint32_t v2[2];
-          tc::tmem_ld<2>(tl + C::S_REF, v2);  // columns 0, 1 (column wg is this head)
-          tc::tmem_wait_ld();
-          tc::reg_fence(v2);
-          v[0] = wg ? v2[1] : v2[0];
-        } else {
-          uint32_t vv[GH];
-          tc::tmem_ld<GH>(tl + C::S_REF + wg * GH, vv);
-          tc::tmem_wait_ld();
-          tc::reg_fence(vv);
-#pragma unroll
-          for (int i = 0; i < GH; ++i) v[i] = vv[i];
-        }
-        const float ak = aK * P.scale_log2;
-#pragma unroll
-        for (int i = 0; i < GH; ++i) S[i] = __uint_as_float(v[i]) * ak;
+      for (int u = 0; u < 4; ++u) {
+        const float2 a = half2_bits_to_f2(wk[u]), c2 = half2_bits_to_f2(wv[u]);
+        sAk[u] = valid ? a.x : 0.f;
+        zAk[u] = valid ? a.y : 0.f;
+        sAv[u] = valid ? c2.x : 0.f;
+        zAv[u] = valid ? c2.y : 0.f;
       }
-      if constexpr (REF == kRefInt4 || RB != 0) {
-        float dotA[GH], offA[GH], dotR[GH], offR[GH];
+    }
+
+    wait_or_abort(sbar, ph);
+    tc::fence_after_sync();
+
+    // ---- scores of token r for this warpgroup's heads
+    float S[GH];
 #pragma unroll
-        for (int i = 0; i < GH; ++i) dotA[i] = offA[i] = dotR[i] = offR[i] = 0.f;
+    for (int i = 0; i < GH; ++i) S[i] = 0.f;
+    if constexpr (REF == kRefBf16) {
+      uint32_t v[GH];
+      tc::tmem_ld_n<GH>(tl + C::S_REF + hb, v);
+      tc::tmem_wait_ld();
+      tc::reg_fence(v);
+      const float ak = aK * P.scale_log2;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t va[3 * GH], vr[C::NPAR][3 * GH];
-          if constexpr (REF == kRefInt4) tc::tmem_ld_n<3 * GH>(tl + C::S_REF + C::N_SA * c + 3 * wg * GH, va);
-          if constexpr (RB != 0) {
+      for (int i = 0; i < GH; ++i) S[i] = __uint_as_float(v[i]) * ak;
+    }
+    if constexpr (REF == kRefInt4 || RB != 0) {
+      float dotA[GH], offA[GH], dotR[GH], offR[GH];
 #pragma unroll
-            for (int p = 0; p < C::NPAR; ++p)
-              tc::tmem_ld_n<3 * GH>(tl + C::S_RES + C::N_SR * c + p * 3 * G + 3 * wg * GH, vr[p]);
-          }
-          tc::tmem_wait_ld();
-          if constexpr (REF == kRefInt4) tc::reg_fence(va);
-          if constexpr (RB != 0) {
+      for (int i = 0; i < GH; ++i) dotA[i] = offA[i] = dotR[i] = offR[i] = 0.f;
 #pragma unroll
-            for (int p = 0; p < C::NPAR; ++p) tc::reg_fence(vr[p]);
-          }
+      for (int c = 0; c < 4; ++c) {
+        uint32_t va[3 * GH], vr[C::NPAR][3 * GH];
+        if constexpr (REF == kRefInt4) tc::tmem_ld_n<3 * GH>(tl + C::S_REF + C::N_SA * c + 3 * hb, va);
+        if constexpr (RB != 0) {
 #pragma unroll
-          for (int i = 0; i < GH; ++i) {
-            const int hq = wg * GH + i;
-            if constexpr (REF == kRefInt4) {
-              dotA[i] = fmaf(sAk[c], comb24(va[3 * i], va[3 * i + 1], va[3 * i + 2]), dotA[i]);
-              offA[i] = fmaf(zAk[c], sQA[hq * 4 + c], offA[i]);
-            }
-            if constexpr (RB != 0) {
+          for (int p = 0; p < C::NPAR; ++p)
+            tc::tmem_ld_n<3 * GH>(tl + C::S_RES + C::N_SR * c + p * 3 * G + 3 * hb, vr[p]);
+        }
+        tc::tmem_wait_ld();
+        if constexpr (REF == kRefInt4) tc::reg_fence(va);
+        if constexpr (RB != 0) {
 #pragma unroll
-              for (int p = 0; p < C::NPAR; ++p) {
-                const int g = c * C::NPAR + p;
-                dotR[i] = fmaf(sK[g], comb24(vr[p][3 * i], vr[p][3 * i + 1], vr[p][3 * i + 2]), dotR[i]);
-                offR[i] = fmaf(zK[g], sQS[hq * 8 + g], offR[i]);
-              }
-            }
-          }
+          for (int p = 0; p < C::NPAR; ++p) tc::reg_fence(vr[p]);
         }
 #pragma unroll
         for (int i = 0; i < GH; ++i) {
-          const int hq = wg * GH + i;
-          if constexpr (REF == kRefInt4) S[i] = aK * fmaf(dotA[i], sCA[hq], offA[i]);
-          if constexpr (RB != 0) S[i] += fmaf(dotR[i], sCS[hq], offR[i]);
+          const int hq = hb + i;
+          if constexpr (REF == kRefInt4) {
+            dotA[i] = fmaf(sAk[c], comb24(va[3 * i], va[3 * i + 1], va[3 * i + 2]), dotA[i]);
+            offA[i] = fmaf(zAk[c], sQA[hq * 4 + c], offA[i]);
+          }
+          if constexpr (RB != 0) {
+#pragma unroll
+            for (int p = 0; p < C::NPAR; ++p) {
+              const int g = c * C::NPAR + p;
+              dotR[i] = fmaf(sK[g], comb24(vr[p][3 * i], vr[p][3 * i + 1], vr[p][3 * i + 2]), dotR[i]);
+              offR[i] = fmaf(zK[g], sQS[hq * 8 + g], offR[i]);
+            }
+          }
         }
       }
-#pragma unroll
-      for (int i = 0; i < GH; ++i) S[i] = valid ? S[i] : -INFINITY;
-
-      // ---- page maxima of the scores (per head) and of the value scales (per group)
 #pragma unroll
       for (int i = 0; i < GH; ++i) {
-        const float v = warp_max(S[i]);
-        if (lane == 0) sWM[(wg * 4 + (warp & 3)) * 4 + i] = v;
+        const int hq = hb + i;
+        if constexpr (REF == kRefInt4) S[i] = aK * fmaf(dotA[i], sCA[hq], offA[i]);
+        if constexpr (RB != 0) S[i] += fmaf(dotR[i], sCS[hq], offR[i]);
       }
-      if constexpr (RB != 0) {
+    }
 #pragma unroll
-        for (int g = 0; g < NGR; ++g) {
-          const float v = warp_max_nonneg(sV[g]);
-          if (lane == 0) sSig[(wg * 4 + (warp & 3)) * 12 + g] = v;
-        }
-      }
-      if constexpr (REF == kRefInt4) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float v = warp_max_nonneg(fabsf(aV * sAv[g]));
-          if (lane == 0) sSig[(wg * 4 + (warp & 3)) * 12 + 8 + g] = v;
-        }
-      }
-      named_bar_sync(kBarWG + wg, 128);
-      float pm[GH], crun[GH], prel[GH];
-#pragma unroll
-      for (int i = 0; i < GH; ++i) {
-        const float* wm = sWM + wg * 16 + i;
-        const float mp = fmaxf(fmaxf(wm[0], wm[4]), fmaxf(wm[8], wm[12]));
-        const float mn = fmaxf(m_run[i], mp);
-        crun[i] = fast_exp2(m_run[i] - mn);
-        pm[i] = fast_exp2(mp - mn);
-        m_run[i] = mn;
-        prel[i] = fast_exp2(S[i] - mp);
-      }
-      float sig[NGR > 0 ? NGR : 1], siga[4];
-      if constexpr (RB != 0) {
-#pragma unroll
-        for (int g = 0; g < NGR; ++g) {
-          const float* sg = sSig + wg * 48 + g;
-          sig[g] = fmaxf(fmaxf(sg[0], sg[12]), fmaxf(sg[24], sg[36]));
-        }
-      }
-      if constexpr (REF == kRefInt4) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float* sg = sSig + wg * 48 + 8 + g;
-          siga[g] = fmaxf(fmaxf(sg[0], sg[12]), fmaxf(sg[24], sg[36]));
-        }
-      }
+    for (int i = 0; i < GH; ++i) S[i] = valid ? S[i] : -INFINITY;
 
-      // ---- B operands of the value MMAs: column t = token r, rows (group, head, hi/lo)
-      const int wrow = (r >> 3) * 128 + (r & 7) * 16;  // MN-major core-matrix row of token r
-      if constexpr (REF == kRefBf16) {
+    // ---- page maxima of the scores (per head) and of the value scales (per group)
+#pragma unroll
+    for (int i = 0; i < GH; ++i) {
+      const float v = warp_max(S[i]);
+      if (lane == 0) sWM[(wg * 4 + (warp & 3)) * 4 + i] = v;
+    }
+    if constexpr (RB != 0) {
+#pragma unroll
+      for (int g = 0; g < NGR; ++g) {
+        const float v = warp_max_nonneg(sV[g]);
+        if (lane == 0) sSig[(wg * 4 + (warp & 3)) * 12 + g] = v;
+      }
+    }
+    if constexpr (REF == kRefInt4) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float v = warp_max_nonneg(fabsf(aV * sAv[g]));
+        if (lane == 0) sSig[(wg * 4 + (warp & 3)) * 12 + 8 + g] = v;
+      }
+    }
+    named_bar_sync(kBarWG + wg, 128);
+    float pm[GH], crun[GH], prel[GH];
+#pragma unroll
+    for (int i = 0; i < GH; ++i) {
+      const float* wm = sWM + wg * 16 + i;
+      const float mp = fmaxf(fmaxf(wm[0], wm[4]), fmaxf(wm[8], wm[12]));
+      const float mn = fmaxf(m_run[i], mp);
+      crun[i] = fast_exp2(m_run[i] - mn);
+      pm[i] = fast_exp2(mp - mn);
+      m_run[i] = mn;
+      prel[i] = fast_exp2(S[i] - mp);
+    }
+    float sig[NGR > 0 ? NGR : 1], siga[4];
+    if constexpr (RB != 0) {
+#pragma unroll
+      for (int g = 0; g < NGR; ++g) {
+        const float* sg = sSig + wg * 48 + g;
+        sig[g] = fmaxf(fmaxf(sg[0], sg[12]), fmaxf(sg[24], sg[36]));
+      }
+    }
+    if constexpr (REF == kRefInt4) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float* sg = sSig + wg * 48 + 8 + g;
+        siga[g] = fmaxf(fmaxf(sg[0], sg[12]), fmaxf(sg[24], sg[36]));
+      }
+    }
+
+    // ---- B operands of the value MMAs: column t = token r
+    const int wrow = (r >> 3) * 128 + (r & 7) * 16;  // MN-major core-matrix row of token r
+    if constexpr (REF == kRefBf16) {
+      if (own_ref) {
         uint32_t pk[GH];
 #pragma unroll
         for (int i = 0; i < GH; ++i) {
@@ -821,105 +889,126 @@ __global__ void __launch_bounds__(kNT, 1)
           pk[i] = static_cast<uint32_t>(__bfloat16_as_ushort(hi)) |
                   (static_cast<uint32_t>(__bfloat16_as_ushort(lo)) << 16);
         }
-        const int n0 = wg * G;  // rows n = 2 * head + (0: hi, 1: lo)
+        const int n0 = wgo * G;  // rows n = 2 * head + (0: hi, 1: lo)
         uint8_t* dst = WB + (n0 >> 3) * 2048 + wrow + (n0 & 7) * 2;
         if constexpr (GH == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         else if constexpr (GH == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
         else *reinterpret_cast<uint32_t*>(dst) = pk[0];
-        // bf16 anchor rows past the context may hold anything: clear them so
-        // that their zero weights give exact zeros
-        if (!valid) {
-          uint4* row = reinterpret_cast<uint4*>(st + C::O_REFV + wg * 16384 + r * 128);
+      }
+      // bf16 anchor rows past the context may hold anything: clear them so
+      // that their zero weights give exact zeros
+      if (!valid && (!SPLIT || wg == 0)) {
+#pragma unroll
+        for (int half = 0; half < (SPLIT ? 2 : 1); ++half) {
+          uint4* row = reinterpret_cast<uint4*>(st + C::O_REFV + (SPLIT ? half : wg) * 16384 + r * 128);
 #pragma unroll
           for (int q = 0; q < 8; ++q) row[q] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      auto put_w8 = [&](uint8_t* tile, int ng, int g, const float (&w)[GH]) {
-        // three signed bytes per weight; this warpgroup's GH heads are contiguous rows
-        uint32_t bj[3] = {0u, 0u, 0u};
-#pragma unroll
-        for (int i = 0; i < GH; ++i) {
-          int qi = __float2int_rn(w[i] * kQ3);
-          qi = max(-8323072, min(8323072, qi));
-          int b2, b1, b0;
-          split24(qi, b2, b1, b0);
-          bj[0] |= (static_cast<uint32_t>(b2) & 0xFFu) << (8 * i);
-          bj[1] |= (static_cast<uint32_t>(b1) & 0xFFu) << (8 * i);
-          bj[2] |= (static_cast<uint32_t>(b0) & 0xFFu) << (8 * i);
-        }
-#pragma unroll
-        for (int j = 0; j < 3; ++j) {
-          const int n0 = j * ng * G + g * G + wg * GH;
-          uint8_t* dst = tile + (n0 >> 4) * 2048 + wrow + (n0 & 15);
-          if constexpr (GH == 4) *reinterpret_cast<uint32_t*>(dst) = bj[j];
-          else if constexpr (GH == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(bj[j]);
-          else *dst = static_cast<uint8_t>(bj[j]);
-        }
-      };
-      if constexpr (REF == kRefInt4) {
+    }
+    if constexpr (REF == kRefInt4) {
+      if (own_ref) {
+        // signed weights (alpha may be negative): three signed bytes each
+        constexpr int NB = 4 * GH;
+        uint32_t v[NB];
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
-          const float inv = siga[g] > 0.f ? 1.f / siga[g] : 0.f;
-          float w[GH];
+          const float t = siga[g] > 0.f ? aV * sAv[g] * rcp_approx(siga[g]) * kQ3 : 0.f;
 #pragma unroll
-          for (int i = 0; i < GH; ++i) w[i] = prel[i] * aV * sAv[g] * inv;
-          put_w8(WA, 4, g, w);
+          for (int i = 0; i < GH; ++i) {
+            int qi = __float2int_rn(prel[i] * t);
+            qi = max(-8323072, min(8323072, qi));
+            int b2, b1, b0;
+            split24(qi, b2, b1, b0);
+            v[g * GH + i] = (static_cast<uint32_t>(b0) & 0xFFu) | ((static_cast<uint32_t>(b1) & 0xFFu) << 8) |
+                            ((static_cast<uint32_t>(b2) & 0xFFu) << 16);
+          }
         }
+        uint32_t planes[3][NB / 4];
+        byte_planes<NB>(v, planes);
+#pragma unroll
+        for (int j = 0; j < 3; ++j) put_plane<NB>(WA, j * 4 * G + wgo * NB, wrow, planes[j]);
       }
-      // the scores are in registers: the value sums may now overwrite their columns
-      tc::fence_before_sync();
-      if constexpr (HAS_V1) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(v1ready));
-      }
-      if constexpr (RB != 0) {
+    }
+    // the scores are in registers: the value sums may now be written
+    tc::fence_before_sync();
+    if constexpr (HAS_V1) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(v1ready));
+    }
+    if constexpr (RB != 0) {
+      if (own_res) {
+        // non-negative weights p * s_g / max_page(s_g) as unsigned 24-bit integers
+        constexpr int NB = NGR * GH;
+        uint32_t v[NB];
 #pragma unroll
         for (int g = 0; g < NGR; ++g) {
-          const float inv = sig[g] > 0.f ? 1.f / sig[g] : 0.f;
-          float w[GH];
+          const float t = sig[g] > 0.f ? sV[g] * rcp_approx(sig[g]) * kU3 : 0.f;
 #pragma unroll
-          for (int i = 0; i < GH; ++i) w[i] = prel[i] * sV[g] * inv;
-          put_w8(WR, NGR, g, w);
+          for (int i = 0; i < GH; ++i) v[g * GH + i] = min(__float2uint_rn(prel[i] * t), 16777215u);
         }
-      }
-      if constexpr (HAS_V2) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(v2ready));
-      }
-
-      // ---- running denominators and offset sums (thread = token r)
+        uint32_t planes[3][NB / 4];
+        byte_planes<NB>(v, planes);
 #pragma unroll
-      for (int i = 0; i < GH; ++i) {
-        const float pr = prel[i] * pm[i];
-        l_thr[i] = fmaf(l_thr[i], crun[i], pr);
-        if constexpr (RB != 0) {
+        for (int j = 0; j < 3; ++j) put_plane<NB>(WR, j * NGR * G + wgo * NB, wrow, planes[j]);
+      }
+    }
+    if constexpr (HAS_V2) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(v2ready));
+    }
+
+    // ---- running denominators and offset sums (thread = token r)
+#pragma unroll
+    for (int i = 0; i < GH; ++i) {
+      const float pr = prel[i] * pm[i];
+      if (own_ref) l_thr[i] = fmaf(l_thr[i], crun[i], pr);
+      if constexpr (RB != 0) {
+        if (own_res) {
 #pragma unroll
           for (int g = 0; g < NGR; ++g) zr[i][g] = fmaf(zr[i][g], crun[i], pr * zV[g]);
         }
-        if constexpr (REF == kRefInt4) {
+      }
+      if constexpr (REF == kRefInt4) {
+        if (own_ref) {
 #pragma unroll
           for (int g = 0; g < 4; ++g) za[i][g] = fmaf(za[i][g], crun[i], pr * aV * zAv[g]);
         }
       }
+    }
 
-      wait_or_abort(obar, ph);
-      tc::fence_after_sync();
+    // ---- run ahead: operands of page k + 1 (query operands of a new
+    // segment, then its key code tiles) while page k's value MMAs run
+    if (!last) {
+      if (seg_end) setup(nxt.b, nxt.h);
+      release_scores();
+      if (wg == 0) {
+        wait_or_abort(&full[s1], ((k + 1) / C::STAGES) & 1);
+        expand_keys(st1);
+      }
+    }
 
-      // ---- merge the page's value sums (thread = dim position r)
-      if constexpr (REF == kRefBf16) {
-        uint32_t v[G];
-        tc::tmem_ld<G>(tl + C::O_REF + wg * G, v);
+    wait_or_abort(obar, ph);
+    tc::fence_after_sync();
+
+    // ---- merge the page's value sums (thread = dim position r)
+    if constexpr (REF == kRefBf16) {
+      if (own_ref) {
+        uint32_t v[2 * GH];
+        tc::tmem_ld_n<2 * GH>(tl + C::O_REF + wgo * G, v);
         tc::tmem_wait_ld();
         tc::reg_fence(v);
 #pragma unroll
         for (int i = 0; i < GH; ++i)
           acc_ref[i] = fmaf(acc_ref[i], crun[i], pm[i] * (__uint_as_float(v[2 * i]) + __uint_as_float(v[2 * i + 1])));
-      } else if constexpr (REF == kRefInt4) {
+      }
+    } else if constexpr (REF == kRefInt4) {
+      if (own_ref) {
         uint32_t v[3][GH];
 #pragma unroll
-        for (int j = 0; j < 3; ++j) tc::tmem_ld<GH>(tl + C::O_REF + j * 4 * G + chunk * G + wg * GH, v[j]);
+        for (int j = 0; j < 3; ++j) tc::tmem_ld_n<GH>(tl + C::O_REF + j * 4 * G + wgo * 4 * GH + chunk * GH, v[j]);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 3; ++j) tc::reg_fence(v[j]);
@@ -928,20 +1017,17 @@ __global__ void __launch_bounds__(kNT, 1)
         for (int g = 1; g < 4; ++g) sg = (chunk == g) ? siga[g] : sg;
         const float f = sg * (1.f / kQ3);
 #pragma unroll
-        for (int i = 0; i < GH; ++i) {
-          const float x = fmaf(65536.f, static_cast<float>(static_cast<int>(v[0][i])),
-                               fmaf(256.f, static_cast<float>(static_cast<int>(v[1][i])),
-                                    static_cast<float>(static_cast<int>(v[2][i]))));
-          acc_ref[i] = fmaf(acc_ref[i], crun[i], pm[i] * f * x);
-        }
+        for (int i = 0; i < GH; ++i) acc_ref[i] = fmaf(acc_ref[i], crun[i], pm[i] * f * comb24(v[0][i], v[1][i], v[2][i]));
       }
-      if constexpr (RB != 0) {
+    }
+    if constexpr (RB != 0) {
+      if (own_res) {
         uint32_t v[C::NPAR][3][GH];
 #pragma unroll
         for (int p = 0; p < C::NPAR; ++p)
 #pragma unroll
           for (int j = 0; j < 3; ++j)
-            tc::tmem_ld<GH>(tl + C::O_RES + j * NGR * G + (chunk * C::NPAR + p) * G + wg * GH, v[p][j]);
+            tc::tmem_ld_n<GH>(tl + C::O_RES + j * NGR * G + wgo * NGR * GH + (chunk * C::NPAR + p) * GH, v[p][j]);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int p = 0; p < C::NPAR; ++p)
@@ -950,76 +1036,93 @@ __global__ void __launch_bounds__(kNT, 1)
         float sg = sig[0];
 #pragma unroll
         for (int g = 1; g < NGR; ++g) sg = (g_res == g) ? sig[g] : sg;
-        const float f = sg * (1.f / kQ3);
+        const float f = sg * (1.f / kU3);
 #pragma unroll
         for (int i = 0; i < GH; ++i) {
-          int b2 = static_cast<int>(v[0][0][i]), b1 = static_cast<int>(v[0][1][i]), b0 = static_cast<int>(v[0][2][i]);
+          uint32_t b2 = v[0][0][i], b1 = v[0][1][i], b0 = v[0][2][i];
           if constexpr (C::NPAR == 2) {
-            b2 = par_r ? static_cast<int>(v[1][0][i]) : b2;
-            b1 = par_r ? static_cast<int>(v[1][1][i]) : b1;
-            b0 = par_r ? static_cast<int>(v[1][2][i]) : b0;
+            b2 = par_r ? v[1][0][i] : b2;
+            b1 = par_r ? v[1][1][i] : b1;
+            b0 = par_r ? v[1][2][i] : b0;
           }
-          const float x = fmaf(65536.f, static_cast<float>(b2), fmaf(256.f, static_cast<float>(b1), static_cast<float>(b0)));
-          acc_res[i] = fmaf(acc_res[i], crun[i], pm[i] * f * x);
+          acc_res[i] = fmaf(acc_res[i], crun[i], pm[i] * f * comb24(b2, b1, b0));
         }
       }
-      advance(it);
     }
 
-    // ---- flush this (b, h) segment: one partial record per query head
+    // ---- flush a finished (b, h) segment: one partial record per query head
+    if (seg_end) {
 #pragma unroll
-    for (int i = 0; i < GH; ++i) {
-      const int hq = wg * GH + i;
-      const float lsum = warp_sum(l_thr[i]);
-      if (lane == 0) atomicAdd(&sRed[hq * C::NRED], lsum);
-      if constexpr (RB != 0) {
+      for (int i = 0; i < GH; ++i) {
+        const int hq = hb + i;
+        if (own_ref) {
+          const float lsum = warp_sum(l_thr[i]);
+          if (lane == 0) atomicAdd(&sRed[hq * C::NRED], lsum);
+        }
+        if constexpr (RB != 0) {
+          if (own_res) {
 #pragma unroll
-        for (int g = 0; g < NGR; ++g) {
-          const float z = warp_sum(zr[i][g]);
-          if (lane == 0) atomicAdd(&sRed[hq * C::NRED + 1 + g], z);
+            for (int g = 0; g < NGR; ++g) {
+              const float z = warp_sum(zr[i][g]);
+              if (lane == 0) atomicAdd(&sRed[hq * C::NRED + 1 + g], z);
+            }
+          }
+        }
+        if constexpr (REF == kRefInt4) {
+          if (own_ref) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const float z = warp_sum(za[i][g]);
+              if (lane == 0) atomicAdd(&sRed[hq * C::NRED + 9 + g], z);
+            }
+          }
         }
       }
-      if constexpr (REF == kRefInt4) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float z = warp_sum(za[i][g]);
-          if (lane == 0) atomicAdd(&sRed[hq * C::NRED + 9 + g], z);
-        }
-      }
-    }
-    named_bar_sync(kBarWG + wg, 128);
-    {
-      const int pair = b * Hkv + h;
+      named_bar_sync(kBarAll, kNCT);  // both warpgroups' sums (G == 1 splits them)
+      const int pair = cur.b * Hkv + cur.h;
       const int d_ref = REF == kRefInt4 ? 32 * chunk + pos_dim<4>(r & 31) : r;
       const int d_res = RB ? 32 * chunk + pos_dim<RB ? RB : 2>(r & 31) : r;
 #pragma unroll
       for (int i = 0; i < GH; ++i) {
-        const int hq = wg * GH + i;
+        const int hq = hb + i;
         float* rec = P.partials + (static_cast<int64_t>(pair + blockIdx.x) * G + hq) * kPartialFloats;
-        float vref = 0.f, vres = 0.f;
-        if constexpr (REF != kRefNone) vref = acc_ref[i];
-        if constexpr (REF == kRefInt4) {
-          float z = sRed[hq * C::NRED + 9];
+        if (own_ref) {
+          float vref = 0.f;
+          if constexpr (REF != kRefNone) vref = acc_ref[i];
+          if constexpr (REF == kRefInt4) {
+            float z = sRed[hq * C::NRED + 9];
 #pragma unroll
-          for (int g = 1; g < 4; ++g) z = (chunk == g) ? sRed[hq * C::NRED + 9 + g] : z;
-          vref += z;
+            for (int g = 1; g < 4; ++g) z = (chunk == g) ? sRed[hq * C::NRED + 9 + g] : z;
+            vref += z;
+          }
+          rec[4 + d_ref] = vref;
+          if (r == 0) {
+            rec[0] = m_run[i];
+            rec[1] = sRed[hq * C::NRED];
+          }
         }
-        if constexpr (RB != 0) {
-          float z = sRed[hq * C::NRED + 1];
+        if (own_res) {
+          float vres = 0.f;
+          if constexpr (RB != 0) {
+            float z = sRed[hq * C::NRED + 1];
 #pragma unroll
-          for (int g = 1; g < NGR; ++g) z = (g_res == g) ? sRed[hq * C::NRED + 1 + g] : z;
-          vres = acc_res[i] + z;
-        }
-        rec[4 + d_ref] = vref;
-        rec[4 + kD + d_res] = vres;
-        if (r == 0) {
-          rec[0] = m_run[i];
-          rec[1] = sRed[hq * C::NRED];
+            for (int g = 1; g < NGR; ++g) z = (g_res == g) ? sRed[hq * C::NRED + 1 + g] : z;
+            vres = acc_res[i] + z;
+          }
+          rec[4 + kD + d_res] = vres;
         }
       }
+      named_bar_sync(kBarAll, kNCT);
+      if (tid < G * C::NRED) sRed[tid] = 0.f;
+      reset_state();
     }
-    named_bar_sync(kBarWG + wg, 128);
-    if (r < GH * C::NRED) sRed[wg * GH * C::NRED + r] = 0.f;
+
+    // ---- run ahead: value code tiles of page k + 1 (page k's value MMAs are done)
+    if (!last && wg == 1) {
+      wait_or_abort(&full[s1], ((k + 1) / C::STAGES) & 1);
+      expand_values(st1);
+    }
+    cur = nxt;
   }
 
   // ---- release the tensor memory once every MMA and every consumer is done with it
@@ -1064,6 +1167,7 @@ TcFn tc_if_fits() {
 template <int REF, int RB, int RG>
 TcFn tc_pick_g(int G) {
   switch (G) {
+    case 1: return tc_if_fits<REF, RB, RG, 1>();
     case 2: return tc_if_fits<REF, RB, RG, 2>();
     case 4: return tc_if_fits<REF, RB, RG, 4>();
     case 8: return tc_if_fits<REF, RB, RG, 8>();

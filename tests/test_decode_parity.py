@@ -158,11 +158,12 @@ def test_recent_window_bf16_tail(librq, n_tail):
 # ---------------------------------------------------------------------------
 TC_FORMATS = {
     # name: (bits, group, rotate, alpha_mode, G values)
-    "bf16ref_int2g32_int4g32": ((2, 4, 2, 16), (32, 32, 32, 32), (1, 1, 1, 0), (0, 0, 3, 0), (2, 4)),
+    "bf16ref_int2g32_int4g32": ((2, 4, 2, 16), (32, 32, 32, 32), (1, 1, 1, 0), (0, 0, 3, 0), (1, 2, 4)),
     "bf16ref_int2g32": ((2, 2, 2, 16), (32, 32, 32, 32), (1, 1, 1, 0), (0, 3, 1, 0), (8,)),
-    "bf16ref_int2g16": ((2, 2, 2, 16), (16, 16, 16, 32), (1, 1, 0, 0), (0, 1, 0, 0), (2, 4)),
-    "int4anchor_int2g32_int4g16": ((2, 4, 2, 4), (32, 16, 16, 32), (1, 1, 1, 0), (0, 0, 3, 0), (2, 4, 8)),
-    "no_anchor_term": ((2, 4, 2, 16), (32, 32, 16, 32), (1, 0, 1, 0), (2, 2, 2, 0), (2, 4, 8)),
+    "bf16ref_int2g16": ((2, 2, 2, 16), (16, 16, 16, 32), (1, 1, 0, 0), (0, 1, 0, 0), (1, 2, 4)),
+    "int4anchor_int2g32_int4g16": ((2, 4, 2, 4), (32, 16, 16, 32), (1, 1, 1, 0), (0, 0, 3, 0), (1, 2, 4)),
+    "int4anchor_2244_g32": ((2, 2, 4, 4), (32, 32, 32, 32), (1, 1, 1, 0), (0, 3, 0, 0), (1, 8)),
+    "no_anchor_term": ((2, 4, 2, 16), (32, 32, 16, 32), (1, 0, 1, 0), (2, 2, 2, 0), (1, 2, 4, 8)),
 }
 
 
@@ -192,11 +193,22 @@ def test_tensor_kernel_many_pages(librq, G):
 
 
 def test_tensor_kernel_rejects_unimplemented(librq):
+    """INT4 anchor with 16-dim residual groups at G = 8 needs more tensor memory
+    than the tensor-core kernel has: that kernel reports it, the default picks
+    the CUDA-core kernel."""
     rq = librq
-    wl = synth.Workload(name="tc_g1", batch=1, kv_heads=2, q_heads=2, context=64, seed=80)
+    wl = synth.Workload(name="tc_unsupported", batch=1, kv_heads=2, q_heads=16, context=64, bits=(2, 2, 4, 4),
+                        group=(16, 32, 32, 32), seed=80)
     cache = rq.Cache(rq.config_from_dict(synth.cache_config_dict(wl)), device="cuda")
-    cache.set_decode_kernel(rq.DECODE_KERNEL_TENSOR)
     inp = synth.make_inputs(wl, "cpu")
+    cache.set_decode_kernel(rq.DECODE_KERNEL_TENSOR)
     with pytest.raises(rq.RQError) as e:
         cache.decode_attention(0, inp["q"][0].cuda(), inp["ctx_len"].cuda())
     assert e.value.status == rq.ERR_UNSUPPORTED
+    cache.set_decode_kernel(rq.DECODE_KERNEL_AUTO)
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    out = cache.decode_attention(0, inp["q"][0].cuda(), inp["ctx_len"].cuda())
+    torch.cuda.synchronize()
+    enc = oracle_encode(inp, synth.cache_config_dict(wl))
+    want = O.decode_attention_f64(enc, 0, to_np32(inp["q"][0]), inp["ctx_len"].numpy())
+    assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
