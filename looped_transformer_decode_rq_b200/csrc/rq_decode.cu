@@ -40,7 +40,6 @@
 namespace rq {
 namespace {
 
-constexpr int kTT = kPage;     // tokens per page / stage
 constexpr int kNCW = 8;        // consumer warps
 constexpr int kGW = 4;         // warps per consumer group
 constexpr int kGT = kGW * 32;  // threads per consumer group
@@ -69,20 +68,21 @@ __device__ __forceinline__ float warp_max(float v) {
   return __int_as_float(i);
 }
 
-template <int REF, int RB, int RG, int G>
+template <int REF, int RB, int RG, int G, int TT>
 struct Cfg {
+  static constexpr int PAGE = TT;  // tokens per page / stage
   // phase 1 (scores): 4G lanes per token, D1 = 32/G dims per lane
   static constexpr int TPT = 4 * G;
   static constexpr int D1 = 32 / G;
   static constexpr int EB = D1 >= 8 ? 8 : D1;   // elements per accumulation block
   static constexpr int NB = D1 / EB;
   static constexpr int TOK_PASS = kGT / TPT;    // tokens per pass of a group
-  static constexpr int PASSES = kTT / TOK_PASS;
+  static constexpr int PASSES = TT / TOK_PASS;
   // phase 2 (values)
   static constexpr int D2 = (G >= 4) ? 4 : 8;   // dims per lane
   static constexpr int TPR2 = kD / D2;          // lanes per token row
   static constexpr int SLICES = kGT / TPR2;
-  static constexpr int TOK2 = kTT / SLICES;     // tokens per lane per page
+  static constexpr int TOK2 = TT / SLICES;     // tokens per lane per page
   // per-record bytes
   static constexpr int REF_REC = REF == kRefBf16 ? 256 : (REF == kRefInt4 ? 64 : 0);
   static constexpr int REFM_REC = REF == kRefInt4 ? 16 : 0;
@@ -93,19 +93,19 @@ struct Cfg {
   // stage layout (each piece 1024-byte aligned)
   static constexpr int al(int x) { return (x + 1023) & ~1023; }
   static constexpr int O_REFK = 0;
-  static constexpr int O_REFV = O_REFK + al(kTT * REF_REC);
-  static constexpr int O_REFMK = O_REFV + al(kTT * REF_REC);
-  static constexpr int O_REFMV = O_REFMK + al(kTT * REFM_REC);
-  static constexpr int O_RESK = O_REFMV + al(kTT * REFM_REC);
-  static constexpr int O_RESV = O_RESK + al(kTT * CB);
-  static constexpr int O_RESMK = O_RESV + al(kTT * CB);
-  static constexpr int O_RESMV = O_RESMK + al(kTT * MB);
-  static constexpr int O_AL = O_RESMV + al(kTT * MB);
-  static constexpr int STAGE_BYTES = O_AL + al(kTT * AL_REC);
-  static constexpr int TX_BYTES = kTT * (2 * REF_REC + 2 * REFM_REC + 2 * CB + 2 * MB + AL_REC);
+  static constexpr int O_REFV = O_REFK + al(TT * REF_REC);
+  static constexpr int O_REFMK = O_REFV + al(TT * REF_REC);
+  static constexpr int O_REFMV = O_REFMK + al(TT * REFM_REC);
+  static constexpr int O_RESK = O_REFMV + al(TT * REFM_REC);
+  static constexpr int O_RESV = O_RESK + al(TT * CB);
+  static constexpr int O_RESMK = O_RESV + al(TT * CB);
+  static constexpr int O_RESMV = O_RESMK + al(TT * MB);
+  static constexpr int O_AL = O_RESMV + al(TT * MB);
+  static constexpr int STAGE_BYTES = O_AL + al(TT * AL_REC);
+  static constexpr int TX_BYTES = TT * (2 * REF_REC + 2 * REFM_REC + 2 * CB + 2 * MB + AL_REC);
   // non-stage shared memory
-  static constexpr int O_S = 0;                           // scores [2 groups][2 parity][G][kTT]
-  static constexpr int O_WM = O_S + 4 * 4 * G * kTT;      // warp maxima [2][2][G][kGW]
+  static constexpr int O_S = 0;                           // scores [2 groups][2 parity][G][TT]
+  static constexpr int O_WM = O_S + 4 * 4 * G * TT;      // warp maxima [2][2][G][kGW]
   static constexpr int O_ACC = O_WM + 4 * 4 * G * kGW;    // [G][256]
   static constexpr int O_L = O_ACC + 4 * G * 2 * kD;      // [G] (padded to 8)
   static constexpr int O_MG = O_L + 4 * 8;                // [2][G] (padded to 16)
@@ -122,7 +122,7 @@ struct Cfg {
   static constexpr int STAGES = STAGES_MAX >= 4 ? 4 : 2;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
   static_assert(STAGES_MAX >= 2, "stage ring does not fit in shared memory");
-  static_assert(PASSES * TOK_PASS == kTT && TOK2 * SLICES == kTT, "lane mapping");
+  static_assert(PASSES * TOK_PASS == TT && TOK2 * SLICES == TT, "lane mapping");
   static_assert((O_ACC % 16) == 0 && (O_QS % 16) == 0 && (O_WM % 16) == 0, "alignment");
 };
 
@@ -209,39 +209,44 @@ __device__ __forceinline__ uint32_t unpack_bytes(uint32_t w, int k) {
 // ---------------------------------------------------------------------------
 // split kernel
 // ---------------------------------------------------------------------------
-template <int REF, int RB, int RG, int G>
+template <int REF, int RB, int RG, int G, int TT>
 __device__ __forceinline__ void issue_page(const DecodeParams& P, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                            uint8_t* st, uint32_t full, const PageIter& it, int Hkv) {
-  using C = Cfg<REF, RB, RG, G>;
-  mbar_arrive_expect_tx(full, C::TX_BYTES);
-  const int t0 = it.page * kTT;
+  using C = Cfg<REF, RB, RG, G, TT>;
+  const int t0 = it.page * TT;
+  // byte planes hold plane_tokens (a multiple of 64) records per (b, h): a
+  // 128-token page may find only 64 of them at the plane's end
+  const int nrec = (TT > kPage && P.plane_tokens > 0 && t0 + TT > P.plane_tokens)
+                       ? static_cast<int>(P.plane_tokens - t0) : TT;
+  mbar_arrive_expect_tx(full, REF == kRefBf16 ? C::TX_BYTES : static_cast<uint32_t>(nrec) * (C::TX_BYTES / TT));
   const int64_t rec0 = static_cast<int64_t>(it.b * Hkv + it.h) * P.plane_tokens + t0;
   if constexpr (REF == kRefBf16) {
+    static_assert(TT == kPage, "bf16 anchor pages are one 64-token tile");
     tma_load_4d(smem_u32(st + C::O_REFK), tmK, 0, t0, it.h, it.b, full);
-    tma_load_4d(smem_u32(st + C::O_REFK + kTT * 128), tmK, 64, t0, it.h, it.b, full);
+    tma_load_4d(smem_u32(st + C::O_REFK + TT * 128), tmK, 64, t0, it.h, it.b, full);
     tma_load_4d(smem_u32(st + C::O_REFV), tmV, 0, t0, it.h, it.b, full);
-    tma_load_4d(smem_u32(st + C::O_REFV + kTT * 128), tmV, 64, t0, it.h, it.b, full);
+    tma_load_4d(smem_u32(st + C::O_REFV + TT * 128), tmV, 64, t0, it.h, it.b, full);
   } else if constexpr (REF == kRefInt4) {
-    bulk_g2s(smem_u32(st + C::O_REFK), P.ref_codes[0] + rec0 * 64, kTT * 64, full);
-    bulk_g2s(smem_u32(st + C::O_REFV), P.ref_codes[1] + rec0 * 64, kTT * 64, full);
-    bulk_g2s(smem_u32(st + C::O_REFMK), P.ref_meta[0] + rec0 * 16, kTT * 16, full);
-    bulk_g2s(smem_u32(st + C::O_REFMV), P.ref_meta[1] + rec0 * 16, kTT * 16, full);
+    bulk_g2s(smem_u32(st + C::O_REFK), P.ref_codes[0] + rec0 * 64, nrec * 64, full);
+    bulk_g2s(smem_u32(st + C::O_REFV), P.ref_codes[1] + rec0 * 64, nrec * 64, full);
+    bulk_g2s(smem_u32(st + C::O_REFMK), P.ref_meta[0] + rec0 * 16, nrec * 16, full);
+    bulk_g2s(smem_u32(st + C::O_REFMV), P.ref_meta[1] + rec0 * 16, nrec * 16, full);
   }
   if constexpr (RB != 0) {
-    bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0] + rec0 * C::CB, kTT * C::CB, full);
-    bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[1] + rec0 * C::CB, kTT * C::CB, full);
-    bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0] + rec0 * C::MB, kTT * C::MB, full);
-    bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[1] + rec0 * C::MB, kTT * C::MB, full);
+    bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0] + rec0 * C::CB, nrec * C::CB, full);
+    bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[1] + rec0 * C::CB, nrec * C::CB, full);
+    bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0] + rec0 * C::MB, nrec * C::MB, full);
+    bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[1] + rec0 * C::MB, nrec * C::MB, full);
   }
-  if constexpr (C::HAS_ALPHA) bulk_g2s(smem_u32(st + C::O_AL), P.alpha + rec0 * 4, kTT * 4, full);
+  if constexpr (C::HAS_ALPHA) bulk_g2s(smem_u32(st + C::O_AL), P.alpha + rec0 * 4, nrec * 4, full);
 }
 
-template <int REF, int RB, int RG, int G>
+template <int REF, int RB, int RG, int G, int TT>
 __global__ void __launch_bounds__(kNT, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams P,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV) {
-  using C = Cfg<REF, RB, RG, G>;
+  using C = Cfg<REF, RB, RG, G, TT>;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // align by offsetting the shared array itself so that every access below
   // stays a shared-memory access
@@ -272,7 +277,7 @@ __global__ void __launch_bounds__(kNT, 1)
       if (blockIdx.x == 0) set_flag(P.status, RQ_FLAG_CTX_LEN);
       len = len < 0 ? 0 : P.capacity;
     }
-    sNt[b] = (len + kTT - 1) / kTT;
+    sNt[b] = (len + TT - 1) / TT;
   }
   for (int i = tid; i < G * 2 * kD; i += kNT) sACC[i] = 0.f;
   if (tid < 8) sL[tid] = 0.f;
@@ -328,7 +333,7 @@ __global__ void __launch_bounds__(kNT, 1)
           break;
         }
         if (*sAbort) break;
-        issue_page<REF, RB, RG, G>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it, Hkv);
+        issue_page<REF, RB, RG, G, TT>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it, Hkv);
         it.next(sNt, B, Hkv);
       }
       // Drain: no copy this CTA issued may still be landing when it exits.
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(kNT, 1)
   const int slice = gtid / C::TPR2;  // phase-2 mapping
   const int j2 = gtid % C::TPR2;
   const int d2 = C::D2 * j2;
-  float* gS = sS + grp * 2 * G * kTT;
+  float* gS = sS + grp * 2 * G * TT;
   float* gWM = sWM + grp * 2 * G * kGW;
 
   PageIter it;
@@ -462,9 +467,9 @@ __global__ void __launch_bounds__(kNT, 1)
           *sAbort = 1;
         }
       }
-      const int n_valid = min(kTT, len_b - it.page * kTT);
+      const int n_valid = min(TT, len_b - it.page * TT);
       const int par = (k >> 1) & 1;
-      float* pS = gS + par * G * kTT;
+      float* pS = gS + par * G * TT;
       float* pWM = gWM + par * G * kGW;
 
       // ---------------- phase 1: scores of the page's 64 tokens
@@ -483,7 +488,7 @@ __global__ void __launch_bounds__(kNT, 1)
           for (int gi = 0; gi < G; ++gi)
 #pragma unroll
             for (int c = 0; c < C::NB; ++c) acc2[gi][c] = make_float2(0.f, 0.f);
-          const uint8_t* rowK = st + C::O_REFK + (d1 >> 6) * (kTT * 128) + t * 128;
+          const uint8_t* rowK = st + C::O_REFK + (d1 >> 6) * (TT * 128) + t * 128;
           if constexpr (C::D1 >= 8) {
 #pragma unroll
             for (int c = 0; c < C::NB; ++c) {
@@ -595,7 +600,7 @@ __global__ void __launch_bounds__(kNT, 1)
           }
           const float sc = (t < n_valid) ? v * P.scale_log2 : -INFINITY;
           wmax[gi] = fmaxf(wmax[gi], sc);
-          if (j1 == 0) pS[gi * kTT + t] = sc;
+          if (j1 == 0) pS[gi * TT + t] = sc;
         }
       }
 #pragma unroll
@@ -632,12 +637,12 @@ __global__ void __launch_bounds__(kNT, 1)
         if constexpr (C::HAS_ALPHA) aV = __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4 + 2));
 #pragma unroll
         for (int gi = 0; gi < G; ++gi) {
-          pp[gi] = fast_exp2(pS[gi * kTT + t] - m_run[gi]);
+          pp[gi] = fast_exp2(pS[gi * TT + t] - m_run[gi]);
           pa[gi] = pp[gi] * aV;
           if (j2 == 0) l_thr[gi] += pp[gi];
         }
         if constexpr (REF == kRefBf16) {
-          const uint8_t* rowV = st + C::O_REFV + (d2 >> 6) * (kTT * 128) + t * 128;
+          const uint8_t* rowV = st + C::O_REFV + (d2 >> 6) * (TT * 128) + t * 128;
           const int chunk = (d2 & 63) >> 3;
           if constexpr (C::D2 == 8) {
             const uint4 v = *reinterpret_cast<const uint4*>(rowV + ((chunk ^ (t & 7)) << 4));
@@ -690,7 +695,7 @@ __global__ void __launch_bounds__(kNT, 1)
           for (int gi = 0; gi < G; ++gi) z_res[gi] = fmaf(pp[gi], sz.y, z_res[gi]);
         }
       };
-      if (n_valid == kTT) {
+      if (n_valid == TT) {
 #pragma unroll 4
         for (int i = 0; i < C::TOK2; ++i) value_token(slice + i * C::SLICES);
       } else {
@@ -841,11 +846,21 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
 // ---------------------------------------------------------------------------
 // dispatch
 // ---------------------------------------------------------------------------
+// Pages of 64 tokens for a bf16 anchor (one tensor-copy tile); 128 for the
+// byte-plane formats, whose 64-token pages are too small to amortise the
+// per-page synchronisation, when four stages still fit.
 template <int REF, int RB, int RG, int G>
-cudaError_t launch_split(const DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv,
-                         cudaStream_t s) {
-  using C = Cfg<REF, RB, RG, G>;
-  auto kern = decode_split_kernel<REF, RB, RG, G>;
+constexpr int page_tokens_of() {
+  if constexpr (REF == kRefBf16) return kPage;
+  else return Cfg<REF, RB, RG, G, 2 * kPage>::STAGES_MAX >= 4 ? 2 * kPage : kPage;
+}
+
+template <int REF, int RB, int RG, int G>
+cudaError_t launch_split(DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv, cudaStream_t s) {
+  constexpr int TT = page_tokens_of<REF, RB, RG, G>();
+  using C = Cfg<REF, RB, RG, G, TT>;
+  auto kern = decode_split_kernel<REF, RB, RG, G, TT>;
+  p.page_tokens = TT;
   static bool attr_done = false;  // per instantiation; set once per process
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -856,7 +871,7 @@ cudaError_t launch_split(const DecodeParams& p, const CUtensorMap* tk, const CUt
   return cudaGetLastError();
 }
 
-using SplitFn = cudaError_t (*)(const DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);
+using SplitFn = cudaError_t (*)(DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);
 
 template <int REF, int RB, int RG>
 SplitFn pick_g(int G) {
@@ -922,8 +937,7 @@ cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_gr
   } else {
     SplitFn fn = pick(ref_kind, res_bits, res_group, p.G);
     if (fn == nullptr) return cudaErrorInvalidValue;
-    p.page_tokens = kTT;
-    e = fn(p, tmap_k, tmap_v, s);
+    e = fn(p, tmap_k, tmap_v, s);  // sets p.page_tokens
   }
   if (e != cudaSuccess) return e;
   const int warps = p.B * p.Hkv * p.G;

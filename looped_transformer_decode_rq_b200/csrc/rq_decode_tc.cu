@@ -706,6 +706,7 @@ __global__ void __launch_bounds__(kNT, 1)
   // ---- prologue: operands of page 0
   PageIter cur;
   seek(cur, x0);
+  int len_cur = seq_len(cur.b);  // cached per segment: no global load on a page's path
   reset_state();
   setup(cur.b, cur.h);
   release_scores();
@@ -717,7 +718,7 @@ __global__ void __launch_bounds__(kNT, 1)
     const int s = k % C::STAGES;
     uint8_t* st = stages + s * C::STAGE_BYTES;
     const uint32_t ph = k & 1;
-    const int n_valid = min(kTP, seq_len(cur.b) - cur.page * kTP);
+    const int n_valid = min(kTP, len_cur - cur.page * kTP);
     const bool last = k + 1 == n_pages;
     PageIter nxt = cur;
     if (!last) advance(nxt);
@@ -981,8 +982,12 @@ __global__ void __launch_bounds__(kNT, 1)
 
     // ---- run ahead: operands of page k + 1 (query operands of a new
     // segment, then its key code tiles) while page k's value MMAs run
+    int len_nxt = len_cur;
     if (!last) {
-      if (seg_end) setup(nxt.b, nxt.h);
+      if (seg_end) {
+        len_nxt = seq_len(nxt.b);
+        setup(nxt.b, nxt.h);
+      }
       release_scores();
       if (wg == 0) {
         wait_or_abort(&full[s1], ((k + 1) / C::STAGES) & 1);
@@ -1123,6 +1128,7 @@ __global__ void __launch_bounds__(kNT, 1)
       expand_values(st1);
     }
     cur = nxt;
+    len_cur = len_nxt;
   }
 
   // ---- release the tensor memory once every MMA and every consumer is done with it
