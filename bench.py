@@ -11,6 +11,8 @@ encode of the new token into every loop's cache.  ``value`` is decode tokens/s
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rq|reference]
                     [--workload ouro8k|mixed|gqa|tiny] [--batch B]
+    python bench.py --workload capacity       # 24-layer capacity sweep (own JSON line)
+    python bench.py --workload mixed_sweep    # [2,2,4,4] INT4-anchor batch 1/8/32/64 vs bf16
 
 Multi-GPU (torchrun) runs independent replicas, one per rank (the path has no
 exchange step); timing is the max over ranks.  ``--impl reference`` times the
@@ -46,7 +48,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["rq", "reference"], default="rq")
-    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "tiny", "capacity"], default="ouro8k")
+    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "tiny", "capacity", "mixed_sweep"],
+                    default="ouro8k")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -447,6 +450,90 @@ def run_capacity(args, world, rank):
                           "hbm_budget_bytes": budget, "data": "synthetic", "n_gpus": world}))
 
 
+def run_mixed_sweep(args, world, rank):
+    """Mixed-precision format [2,2,4,4] with an INT4 anchor at 8k context,
+    batch 1 / 8 / 32 / 64: the decode step (4 loop decodes + append-encode of the
+    new token) against the bf16-cache step on the same values, and the
+    append-encode alone.  A step that reads less than twice the L2 is timed
+    alone after writing a 256 MB buffer (L2 flushed between timed steps)."""
+    from looped_transformer_decode_rq_b200 import rq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    steps, warmup = max(3, min(args.steps, 20)), max(3, args.warmup)
+
+    def timed(step, flush):
+        for _ in range(warmup):
+            step()
+        barrier(world)
+        torch.cuda.synchronize()
+        if not flush:
+            return time_steps(step, steps, 0, world, stream)
+        total = 0.0
+        for _ in range(steps):
+            flush_buf.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b.record(stream)
+            b.synchronize()
+            total += a.elapsed_time(b)
+        barrier(world)
+        return max_over_ranks(total / steps, world)
+
+    results = []
+    for B in (1, 8, 32, 64):
+        wl = synth.mixed_int4_anchor(batch=B).with_(seed=2 + 1000 * rank)
+        inp = synth.make_inputs(wl, dev)
+        L, Hkv, Hq, T = wl.num_loops, wl.kv_heads, wl.q_heads, wl.context
+        cfgd = synth.cache_config_dict(wl, capacity=T + 1)
+        cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
+        cache.encode(inp["k"], inp["v"])
+        ctx = inp["ctx_len"]
+        k_new = inp["k_tail"][:, :, :, :1].contiguous()
+        v_new = inp["v_tail"][:, :, :, :1].contiguous()
+        q = inp["q"]
+        outs = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
+        lay = cache.layout
+        step_bytes = sum(B * Hkv * T * (2 * (lay.codes_record_bytes[lay.anchor_of[l]] + lay.meta_record_bytes[lay.anchor_of[l]])
+                                        + (2 * (lay.codes_record_bytes[l] + lay.meta_record_bytes[l]) + 4
+                                           if lay.anchor_of[l] != l else 0)) for l in range(L))
+        flush = step_bytes < 2 * (126 << 20)
+
+        def rq_step():
+            for l in range(L):
+                cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
+            cache.encode(k_new, v_new, positions=ctx)
+
+        def append():
+            cache.encode(k_new, v_new, positions=ctx)
+
+        ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+
+        def bf16_step():
+            for l in range(L):
+                rq.bf16_decode_attention(inp["k"][l], inp["v"][l], q[l], ctx, k_new[l], v_new[l], workspace=ws,
+                                         out=outs[l])
+
+        ms = timed(rq_step, flush)
+        enc_ms = timed(append, flush)
+        bms = timed(bf16_step, flush)
+        flags = cache.get_error()
+        results.append({"batch": B, "tokens_per_s": round(job_tokens_per_s(B, world, ms), 1),
+                        "ms_per_step": round(ms, 4), "hbm_gbs": round(step_bytes / (ms * 1e-3) / 1e9, 1),
+                        "step_bytes": step_bytes, "append_encode_us": round(enc_ms * 1e3, 1),
+                        "bf16_tokens_per_s": round(job_tokens_per_s(B, world, bms), 1),
+                        "bf16_ms_per_step": round(bms, 4), "rq_speedup_vs_bf16": round(bms / ms, 3),
+                        "l2_flushed": flush, "device_flags": int(flags)})
+        del cache, inp, outs, ws
+        torch.cuda.empty_cache()
+    if rank == 0:
+        print(json.dumps({"workload": "mixed_2244_H16_T8192_int4ref_batch_sweep",
+                          "metric": "decode step tokens/s (4 loops + append-encode) vs BF16 cache",
+                          "results": results, "steps": steps, "warmup": warmup, "data": "synthetic",
+                          "n_gpus": world}))
+
+
 def run_rq(args, world, rank):
     from looped_transformer_decode_rq_b200 import rq
 
@@ -665,6 +752,8 @@ def main():
             run_reference(args, world, rank)
         elif args.workload == "capacity":
             run_capacity(args, world, rank)
+        elif args.workload == "mixed_sweep":
+            run_mixed_sweep(args, world, rank)
         else:
             run_rq(args, world, rank)
     finally:
