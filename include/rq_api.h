@@ -210,6 +210,15 @@ typedef enum {
  * decode calls on the same handle. */
 RQ_API rq_status rq_cache_set_decode_kernel(rq_cache* cache, int32_t kernel);
 
+/* Test hook for the failure path (the paper has no counterpart).  With page
+ * >= 0, the producer warp of every CTA of later rq_decode_attention calls on
+ * this handle waits, before issuing its page-th page, on a barrier that nothing
+ * arrives at.  That wait, like every wait in the decode kernels, gives up after
+ * its limit (about 2 s); the call then completes with RQ_FLAG_PIPE_TIMEOUT set
+ * in the status word (its output is unspecified) and the context stays usable.
+ * -1 (the default) turns the hook off; other values are RQ_ERR_INVALID_ARG. */
+RQ_API rq_status rq_cache_set_debug_stall(rq_cache* cache, int32_t page);
+
 /* Bytes of workspace rq_decode_attention needs for this cache on the current
  * device (split-K partials; independent of context length). */
 RQ_API rq_status rq_decode_workspace_size(const rq_cache* cache, int64_t* bytes_out);

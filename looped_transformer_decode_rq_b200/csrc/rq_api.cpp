@@ -22,6 +22,7 @@ struct rq_cache {
   int device;
   int num_ctas;
   int decode_kernel;                     // rq_decode_kernel
+  int stall_page;                        // test hook (rq_cache_set_debug_stall)
   bool tmaps_ready[RQ_MAX_LOOPS];        // per bf16 anchor loop
   CUtensorMap tm_anchor[RQ_MAX_LOOPS][2];
 };
@@ -234,6 +235,7 @@ rq_status rq_cache_create(const rq_config* cfg, void* device_buffer, int64_t buf
   c->device = dev;
   c->num_ctas = rq::decode_grid_ctas(dev);
   c->decode_kernel = RQ_DECODE_KERNEL_AUTO;
+  c->stall_page = -1;
   for (int l = 0; l < RQ_MAX_LOOPS; ++l) c->tmaps_ready[l] = false;
   *out = c;
   return RQ_OK;
@@ -246,6 +248,13 @@ rq_status rq_cache_set_decode_kernel(rq_cache* cache, int32_t kernel) {
   if (kernel != RQ_DECODE_KERNEL_AUTO && kernel != RQ_DECODE_KERNEL_SIMT && kernel != RQ_DECODE_KERNEL_TENSOR)
     return fail(RQ_ERR_INVALID_ARG, "decode kernel %d", kernel);
   cache->decode_kernel = kernel;
+  return RQ_OK;
+}
+
+rq_status rq_cache_set_debug_stall(rq_cache* cache, int32_t page) {
+  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  if (page < -1) return fail(RQ_ERR_INVALID_ARG, "stall page %d < -1", page);
+  cache->stall_page = page;
   return RQ_OK;
 }
 
@@ -415,6 +424,7 @@ rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void*
   p.num_ctas = cache->num_ctas;
   p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
   p.tma_tokens = lay.capacity_padded;
+  p.stall_page = cache->stall_page;
   cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, cache->decode_kernel, &cache->tm_anchor[a][0],
                                     &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
@@ -469,6 +479,7 @@ rq_status rq_bf16_decode_attention(int32_t batch, int32_t kv_heads, int32_t q_he
   p.num_ctas = rq::decode_grid_ctas(dev);
   p.status = status_word;
   p.tma_tokens = capacity;
+  p.stall_page = -1;
   cudaError_t e = rq::launch_decode(p, rq::kRefBf16, 0, 32, rq::kKernelAuto, &tk, &tv,
                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");

@@ -304,6 +304,7 @@ __global__ void __launch_bounds__(kNT, 1)
       mbar_init(smem_u32(&bars[s]), 1);               // full: the producer's expect_tx
       mbar_init(smem_u32(&bars[C::STAGES + s]), kGW);  // empty: the 4 warps of the page's group
     }
+    mbar_init(smem_u32(&bars[15]), 1);  // never arrived at: the wait of the stall test hook
     fence_barrier_init();
   }
   __syncthreads();
@@ -332,6 +333,7 @@ __global__ void __launch_bounds__(kNT, 1)
           *sAbort = 1;
           break;
         }
+        if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[15]), 0)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
         if (*sAbort) break;
         issue_page<REF, RB, RG, G, TT>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it, Hkv);
         it.next(sNt, B, Hkv);

@@ -384,6 +384,7 @@ __global__ void __launch_bounds__(kNT, 1)
   uint64_t* v1ready = bars + 12; // anchor value weights (and cleared anchor rows) written
   uint64_t* v2ready = bars + 13; // residual value weights (and value code tiles) written
   uint64_t* done = bars + 14;    // every MMA of the CTA completed
+  uint64_t* never = bars + 15;   // never arrived at: the wait of the stall test hook
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -429,6 +430,7 @@ __global__ void __launch_bounds__(kNT, 1)
     mbar_init(smem_u32(v1ready), kNCW);
     mbar_init(smem_u32(v2ready), kNCW);
     mbar_init(smem_u32(done), 1);
+    mbar_init(smem_u32(never), 1);
     fence_barrier_init();
   }
   __syncthreads();
@@ -501,6 +503,7 @@ __global__ void __launch_bounds__(kNT, 1)
           set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
           break;
         }
+        if (k == P.stall_page && !mbar_wait_bounded(smem_u32(never), 0)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
         tc_issue_page<REF, RB, RG, G>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&full[s]), it, Hkv);
         advance(it);
       }

@@ -75,6 +75,7 @@ struct DecodeParams {
   int32_t* status;
   int64_t tma_tokens;    // token extent of the bf16 tensor maps
   int page_tokens;       // split granularity (set by launch_decode for the chosen kernel)
+  int stall_page;        // test hook: CTA-local page before which the producer waits out its limit (-1: none)
 };
 
 // Split-K partial record per (slot, head): m, l, pad, pad, acc_ref[128], acc_res[128]

@@ -37,7 +37,8 @@ DECODE_KERNEL_AUTO, DECODE_KERNEL_SIMT, DECODE_KERNEL_TENSOR = 0, 1, 2
 EXPORTED = ("rq_cache_layout", "rq_cache_create", "rq_cache_destroy", "rq_cache_info", "rq_encode",
             "rq_decode_workspace_size", "rq_decode_attention", "rq_bf16_decode_workspace_size",
             "rq_bf16_decode_attention", "rq_reconstruct", "rq_get_error", "rq_status_string",
-            "rq_last_error_message", "rq_decode_attention_static_scratch", "rq_cache_set_decode_kernel")
+            "rq_last_error_message", "rq_decode_attention_static_scratch", "rq_cache_set_decode_kernel",
+            "rq_cache_set_debug_stall")
 STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 
@@ -64,6 +65,7 @@ _sig = {
     "rq_cache_info": (C.c_int, [_vp, C.POINTER(Config), C.POINTER(Layout)]),
     "rq_encode": (C.c_int, [_vp, _vp, _vp, C.POINTER(_i64), _i32, _vp, _i32, _vp]),
     "rq_cache_set_decode_kernel": (C.c_int, [_vp, _i32]),
+    "rq_cache_set_debug_stall": (C.c_int, [_vp, _i32]),
     "rq_decode_workspace_size": (C.c_int, [_vp, C.POINTER(_i64)]),
     "rq_decode_attention": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp]),
     "rq_decode_attention_static_scratch": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp]),
@@ -151,6 +153,11 @@ class Cache:
     @property
     def handle(self):
         return self._h
+
+    def set_debug_stall(self, page: int) -> None:
+        """Failure-path test hook: the decode producers wait out their limit before
+        CTA-local page `page` (-1: off); the call then sets FLAG_PIPE_TIMEOUT."""
+        _check(_lib.rq_cache_set_debug_stall(self._h, page), "rq_cache_set_debug_stall")
 
     def set_decode_kernel(self, kernel: int) -> None:
         """DECODE_KERNEL_AUTO (default), DECODE_KERNEL_SIMT or DECODE_KERNEL_TENSOR."""

@@ -212,3 +212,38 @@ def test_tensor_kernel_rejects_unimplemented(librq):
     enc = oracle_encode(inp, synth.cache_config_dict(wl))
     want = O.decode_attention_f64(enc, 0, to_np32(inp["q"][0]), inp["ctx_len"].numpy())
     assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
+
+
+@pytest.mark.parametrize("kernel", ["simt", "tensor"])
+def test_wait_limit_sets_flag_and_context_recovers(librq, kernel):
+    """Failure path without a fault: the producers wait on a barrier nothing
+    arrives at (test hook); every wait gives up after its limit, the call sets
+    FLAG_PIPE_TIMEOUT and returns, and the next call on the same context is
+    correct."""
+    import time
+    rq = librq
+    wl = synth.Workload(name="stall", batch=2, kv_heads=2, q_heads=8, context=300, seed=90)
+    inp = synth.make_inputs(wl, "cpu")
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    cache.set_decode_kernel(rq.DECODE_KERNEL_SIMT if kernel == "simt" else rq.DECODE_KERNEL_TENSOR)
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    assert cache.get_error() == 0
+    q, ctx = inp["q"][0].cuda(), inp["ctx_len"].cuda()
+    kt, vt = inp["k_tail"][0].cuda(), inp["v_tail"][0].cuda()
+    with pytest.raises(rq.RQError):
+        cache.set_debug_stall(-2)
+    cache.set_debug_stall(0)
+    t0 = time.time()
+    cache.decode_attention(0, q, ctx, kt, vt)
+    flags = cache.get_error()
+    assert flags & rq.FLAG_PIPE_TIMEOUT
+    assert time.time() - t0 < 60
+    cache.set_debug_stall(-1)
+    out = cache.decode_attention(0, q, ctx, kt, vt)
+    torch.cuda.synchronize()
+    assert cache.get_error() == 0
+    enc = oracle_encode(inp, cfgd)
+    want = O.decode_attention_f64(enc, 0, to_np32(inp["q"][0]), inp["ctx_len"].numpy(),
+                                  to_np32(inp["k_tail"][0]), to_np32(inp["v_tail"][0]))
+    assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
