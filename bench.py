@@ -4,8 +4,9 @@
 One step = one decode step of a 4-loop looped model's attention layer over a
 synthetic Ouro-1.4B-shaped cache (16 KV heads, head_dim 128, batch 16, 8192
 cached tokens): decode attention of every loop (three INT2 residual loops and
-the bf16 reference loop, each with the current token as a bf16 tail), then the
-encode of the new token into every loop's cache.  ``value`` is decode tokens/s
+the bf16 reference loop, each with the current token as a bf16 tail), and the
+encode of the new token into every loop's cache, fused into the final loop's
+decode call (rq_decode_attention_append).  ``value`` is decode tokens/s
 (sequences x steps / s) over all ranks; the same step over a plain bf16 cache
 (same library, same kernels without the residual) is reported beside it.
 
@@ -317,9 +318,10 @@ def measure_workload(wl, steps, warmup, world, rank):
     stream = torch.cuda.current_stream()
 
     def rq_step():
-        for l in range(L):
+        for l in range(L - 1):
             cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
-        cache.encode(k_new, v_new, positions=ctx)
+        cache.decode_attention_append(L - 1, q[L - 1], ctx, k_new[L - 1], v_new[L - 1], k_new, v_new, ctx,
+                                      out=outs[L - 1])
 
     ms = time_steps(rq_step, steps, warmup, world, stream)
     ev = []
@@ -434,9 +436,10 @@ def run_capacity(args, world, rank):
 
             def step():
                 for c in caches:
-                    for l in range(L):
+                    for l in range(L - 1):
                         c.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
-                    c.encode(k_new, v_new, positions=ctx)
+                    c.decode_attention_append(L - 1, q[L - 1], ctx, k_new[L - 1], v_new[L - 1], k_new, v_new, ctx,
+                                              out=outs[L - 1])
         ms = time_steps(step, steps, warmup, world, stream)
         flags = 0 if fmt == "bf16" else max(c.get_error() for c in caches)
         results[fmt] = {"max_batch": B, "bytes_per_sequence": int(per_seq),
@@ -501,9 +504,10 @@ def run_mixed_sweep(args, world, rank):
         flush = step_bytes < 2 * (126 << 20)
 
         def rq_step():
-            for l in range(L):
+            for l in range(L - 1):
                 cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
-            cache.encode(k_new, v_new, positions=ctx)
+            cache.decode_attention_append(L - 1, q[L - 1], ctx, k_new[L - 1], v_new[L - 1], k_new, v_new, ctx,
+                                          out=outs[L - 1])
 
         def append():
             cache.encode(k_new, v_new, positions=ctx)
@@ -558,15 +562,18 @@ def run_rq(args, world, rank):
     ev_pairs = []
 
     def step(record=False):
-        for l in range(L):
-            if record and l < L - 1:
+        # loops 0 .. L-2, then the final loop's decode with the new token's
+        # append-encode (every loop) fused into its combine launch
+        for l in range(L - 1):
+            if record:
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
             cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
-            if record and l < L - 1:
+            if record:
                 e1.record(stream)
                 ev_pairs.append((e0, e1))
-        cache.encode(k_new, v_new, positions=pos)
+        cache.decode_attention_append(L - 1, q[L - 1], ctx, k_new[L - 1], v_new[L - 1], k_new, v_new, pos,
+                                      out=outs[L - 1])
 
     for _ in range(args.warmup):
         step()
@@ -627,9 +634,9 @@ def run_rq(args, world, rank):
             dq.copy_(hq, non_blocking=True)
             dk.copy_(hk, non_blocking=True)
             dv.copy_(hv, non_blocking=True)
-            for l in range(L):
+            for l in range(L - 1):
                 cache.decode_attention(l, dq[l], ctx, dk[l], dv[l], out=outs[l])
-            cache.encode(dk, dv, positions=pos)
+            cache.decode_attention_append(L - 1, dq[L - 1], ctx, dk[L - 1], dv[L - 1], dk, dv, pos, out=outs[L - 1])
             hout.copy_(outs, non_blocking=True)
 
         for _ in range(2):
@@ -710,7 +717,7 @@ def run_rq(args, world, rank):
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                      "frac_of_8tbs": round(achieved / 8000.0, 4)},
         "cpu_baseline": cpu, "e2e": e2e, "bf16_cache": bf16, "parity": parity, "other_workloads": extra,
-        "gpu_launches": args.steps * (2 * L + 1), "clocks": clk, "device_flags": flags,
+        "gpu_launches": args.steps * (2 * L), "clocks": clk, "device_flags": flags,
     }
     if rank == 0:
         print(json.dumps(out))

@@ -247,6 +247,27 @@ RQ_API rq_status rq_decode_attention(const rq_cache* cache, int32_t loop, const 
                               int32_t n_tail, float softmax_scale, float* out, void* workspace,
                               int64_t workspace_bytes, rq_stream_t stream);
 
+/* rq_decode_attention of `loop`, plus the encode of n_new new tokens of every
+ * loop into the cache in the same call: the per-step append of a decoding
+ * model ([RQ] abstract; Figure 1 steps 2-5), which can run once the final
+ * loop has produced its keys and values, so it is typically fused into the
+ * final loop's decode.  The encode runs in the launch of the combine kernel,
+ * by extra warps, saving one launch per layer and step.
+ *  k_new/v_new, strides   as rq_encode (all loops; n_new tokens)
+ *  positions              device int32 [B], required: sequence b's new tokens go
+ *                         to positions[b] .. positions[b] + n_new - 1; positions
+ *                         past capacity are skipped with RQ_FLAG_POSITION
+ * The decode reads positions < ctx_len[b] only: to append the current token,
+ * pass positions = ctx_len (its values join this decode through the tail).
+ * Arithmetic and results are those of rq_decode_attention followed by
+ * rq_encode with device positions. */
+RQ_API rq_status rq_decode_attention_append(rq_cache* cache, int32_t loop, const void* q,
+                                            const int32_t* ctx_len, const void* k_tail, const void* v_tail,
+                                            int32_t n_tail, float softmax_scale, float* out, void* workspace,
+                                            int64_t workspace_bytes, const void* k_new, const void* v_new,
+                                            const int64_t* strides, const int32_t* positions, int32_t n_new,
+                                            rq_stream_t stream);
+
 /* Size of the library's static split-K scratch used by
  * rq_decode_attention_static_scratch (4 MiB). */
 #define RQ_STATIC_SCRATCH_BYTES (4u * 1024u * 1024u)

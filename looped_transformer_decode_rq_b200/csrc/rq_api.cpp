@@ -265,12 +265,11 @@ rq_status rq_cache_info(const rq_cache* cache, rq_config* cfg_out, rq_layout* la
   return RQ_OK;
 }
 
-rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const int64_t* strides,
-                    int32_t start_pos, const int32_t* positions, int32_t n_tokens,
-                    rq_stream_t stream) {
-  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
-  if (n_tokens < 0) return fail(RQ_ERR_INVALID_ARG, "n_tokens %d < 0", n_tokens);
-  if (n_tokens == 0) return RQ_OK;
+namespace {
+
+// Validates an encode request and fills its kernel parameters (n_tokens > 0).
+rq_status build_encode(rq_cache* cache, const void* k, const void* v, const int64_t* strides, int32_t start_pos,
+                       const int32_t* positions, int32_t n_tokens, rq::EncodeParams* out) {
   if (k == nullptr || v == nullptr || strides == nullptr) return fail(RQ_ERR_INVALID_ARG, "k, v or strides is null");
   if (!aligned(k, 16) || !aligned(v, 16)) return fail(RQ_ERR_INVALID_ARG, "k/v not 16-byte aligned");
   for (int i = 0; i < 4; ++i)
@@ -285,7 +284,7 @@ rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const int64_t
   }
   if (static_cast<int64_t>(c.batch) * c.kv_heads * n_tokens > (int64_t(1) << 31) - 8)
     return fail(RQ_ERR_UNSUPPORTED, "too many vectors in one encode call");
-  rq::EncodeParams p;
+  rq::EncodeParams& p = *out;
   std::memset(&p, 0, sizeof(p));
   p.L = c.num_loops;
   p.B = c.batch;
@@ -315,6 +314,20 @@ rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const int64_t
     p.anchor[l] = lay.anchor_of[l];
   }
   p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
+  return RQ_OK;
+}
+
+}  // namespace
+
+rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const int64_t* strides,
+                    int32_t start_pos, const int32_t* positions, int32_t n_tokens,
+                    rq_stream_t stream) {
+  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  if (n_tokens < 0) return fail(RQ_ERR_INVALID_ARG, "n_tokens %d < 0", n_tokens);
+  if (n_tokens == 0) return RQ_OK;
+  rq::EncodeParams p;
+  const rq_status st = build_encode(cache, k, v, strides, start_pos, positions, n_tokens, &p);
+  if (st != RQ_OK) return st;
   cudaError_t e = rq::launch_encode(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "encode launch");
   return RQ_OK;
@@ -361,10 +374,12 @@ rq_status check_decode_common(int B, int Hkv, int Hq, const void* q, const int32
 
 }  // namespace
 
-rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void* q,
-                              const int32_t* ctx_len, const void* k_tail, const void* v_tail,
-                              int32_t n_tail, float softmax_scale, float* out, void* workspace,
-                              int64_t workspace_bytes, rq_stream_t stream) {
+namespace {
+
+rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, const int32_t* ctx_len,
+                      const void* k_tail, const void* v_tail, int32_t n_tail, float softmax_scale, float* out,
+                      void* workspace, int64_t workspace_bytes, rq_stream_t stream,
+                      const rq::EncodeParams* append) {
   if (cache_c == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
   rq_cache* cache = const_cast<rq_cache*>(cache_c);
   const rq_config& c = cache->cfg;
@@ -426,9 +441,35 @@ rq_status rq_decode_attention(const rq_cache* cache_c, int32_t loop, const void*
   p.tma_tokens = lay.capacity_padded;
   p.stall_page = cache->stall_page;
   cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, cache->decode_kernel, &cache->tm_anchor[a][0],
-                                    &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream));
+                                    &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream), append);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return RQ_OK;
+}
+
+}  // namespace
+
+rq_status rq_decode_attention(const rq_cache* cache, int32_t loop, const void* q, const int32_t* ctx_len,
+                              const void* k_tail, const void* v_tail, int32_t n_tail, float softmax_scale,
+                              float* out, void* workspace, int64_t workspace_bytes, rq_stream_t stream) {
+  return decode_impl(cache, loop, q, ctx_len, k_tail, v_tail, n_tail, softmax_scale, out, workspace,
+                     workspace_bytes, stream, nullptr);
+}
+
+rq_status rq_decode_attention_append(rq_cache* cache, int32_t loop, const void* q, const int32_t* ctx_len,
+                                     const void* k_tail, const void* v_tail, int32_t n_tail, float softmax_scale,
+                                     float* out, void* workspace, int64_t workspace_bytes, const void* k_new,
+                                     const void* v_new, const int64_t* strides, const int32_t* positions,
+                                     int32_t n_new, rq_stream_t stream) {
+  if (cache == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
+  if (positions == nullptr) return fail(RQ_ERR_INVALID_ARG, "positions is null (device int32 [batch] required)");
+  if (n_new < 0) return fail(RQ_ERR_INVALID_ARG, "n_new %d < 0", n_new);
+  rq::EncodeParams ep;
+  if (n_new > 0) {
+    const rq_status st = build_encode(cache, k_new, v_new, strides, 0, positions, n_new, &ep);
+    if (st != RQ_OK) return st;
+  }
+  return decode_impl(cache, loop, q, ctx_len, k_tail, v_tail, n_tail, softmax_scale, out, workspace,
+                     workspace_bytes, stream, n_new > 0 ? &ep : nullptr);
 }
 
 rq_status rq_bf16_decode_attention(int32_t batch, int32_t kv_heads, int32_t q_heads,

@@ -34,7 +34,10 @@
 // Combine kernel: one warp per (b, q-head) merges the CTA partials with the
 // max-rescale rule, adds the bf16 tail tokens, applies the inverse rotation and
 // normalises.
+#include <cstring>
+
 #include "rq_common.cuh"
+#include "rq_encode_dev.cuh"
 #include "rq_internal.h"
 
 namespace rq {
@@ -717,6 +720,11 @@ __global__ void __launch_bounds__(kNT, 1)
       for (int gi = 0; gi < G; ++gi) sMG[grp * G + gi] = m_run[gi];
     }
     named_bar_sync(kConsumerBar, kNCT);
+    // Sum the slices' contributions in a fixed order (warp by warp, and within a
+    // warp its two slices by one shuffle), so that a decode is reproducible bit
+    // for bit from run to run.
+    constexpr int SPW = 32 / C::TPR2;  // token slices per warp (1 or 2)
+    float cref[G][C::D2], cres[G][C::D2], cl[G];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
       const float M = fmaxf(sMG[gi], sMG[G + gi]);
@@ -726,16 +734,35 @@ __global__ void __launch_bounds__(kNT, 1)
         const float2 ar = acc_ref[gi][e >> 1];
         float vr = (e & 1) ? ar.y : ar.x;
         if constexpr (REF == kRefInt4) vr = fmaf(vr, pow2i(23 - code_pos<4>(e)), z_ref[gi]);
-        if constexpr (REF != kRefNone) atomicAdd(&sACC[gi * 2 * kD + d2 + e], vr * f);
+        cref[gi][e] = __fmul_rn(vr, f);
+        float vs = 0.f;
         if constexpr (RB != 0) {
           const float2 as = acc_res[gi][e >> 1];
-          const float vs = fmaf((e & 1) ? as.y : as.x, pow2i(23 - code_pos<RB>(e)), z_res[gi]);
-          atomicAdd(&sACC[gi * 2 * kD + kD + d2 + e], vs * f);
+          vs = fmaf((e & 1) ? as.y : as.x, pow2i(23 - code_pos<RB>(e)), z_res[gi]);
+        }
+        cres[gi][e] = __fmul_rn(vs, f);
+        if constexpr (SPW == 2) {
+          cref[gi][e] = __fadd_rn(cref[gi][e], __shfl_xor_sync(kFull, cref[gi][e], 16));
+          cres[gi][e] = __fadd_rn(cres[gi][e], __shfl_xor_sync(kFull, cres[gi][e], 16));
         }
       }
-      if (l_thr[gi] != 0.f) atomicAdd(&sL[gi], l_thr[gi] * f);
+      cl[gi] = __fmul_rn(l_thr[gi], f);
+      if constexpr (SPW == 2) cl[gi] = __fadd_rn(cl[gi], __shfl_xor_sync(kFull, cl[gi], 16));
     }
-    named_bar_sync(kConsumerBar, kNCT);
+    for (int w = 0; w < kNCW; ++w) {
+      if (warp == w && lane < 32 / SPW) {
+#pragma unroll
+        for (int gi = 0; gi < G; ++gi) {
+#pragma unroll
+          for (int e = 0; e < C::D2; ++e) {
+            if constexpr (REF != kRefNone) sACC[gi * 2 * kD + d2 + e] = __fadd_rn(sACC[gi * 2 * kD + d2 + e], cref[gi][e]);
+            if constexpr (RB != 0) sACC[gi * 2 * kD + kD + d2 + e] = __fadd_rn(sACC[gi * 2 * kD + kD + d2 + e], cres[gi][e]);
+          }
+          if (j2 == 0) sL[gi] = __fadd_rn(sL[gi], cl[gi]);
+        }
+      }
+      named_bar_sync(kConsumerBar, kNCT);
+    }
     {
       const int pair = b * Hkv + h;
       float* rec = P.partials + static_cast<int64_t>(pair + blockIdx.x) * G * kPartialFloats;
@@ -757,11 +784,23 @@ __global__ void __launch_bounds__(kNT, 1)
 // ---------------------------------------------------------------------------
 // combine kernel: one warp per (b, q-head)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams P, int G, int rotate_res) {
+// x * a + y * b with a fixed rounding order (the result must not depend on how
+// the compiler contracts this kernel's instances)
+__device__ __forceinline__ float mix(float x, float a, float y, float b) { return __fmaf_rn(x, a, __fmul_rn(y, b)); }
+
+// With APPEND, the warps past the B * Hq combine warps encode the new tokens of
+// `E` into every loop's planes instead (positions past every context the split
+// kernel read, so the two never touch the same records).
+template <bool APPEND>
+__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams P, int G, int rotate_res,
+                                                             const __grid_constant__ EncodeParams E) {
   const int lane = threadIdx.x & 31;
   const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int Hq = P.Hkv * G;
-  if (wid >= P.B * Hq) return;
+  if (wid >= P.B * Hq) {
+    if constexpr (APPEND) enc::encode_warp(E, wid - P.B * Hq, lane);
+    return;
+  }
   const int b = wid / Hq, qh = wid % Hq, h = qh / G, gi = qh % G;
   auto clamp_len = [&](int len) { return len < 0 ? 0 : (len > P.capacity ? P.capacity : len); };
   // page offsets (same arithmetic as the split kernel that wrote the partials)
@@ -796,9 +835,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
       const float4 s = reinterpret_cast<const float4*>(rec + 4 + kD)[lane];
       const float mn = fmaxf(m, ml.x);
       const float a = exp2f(m - mn), bb = exp2f(ml.x - mn);
-      l = l * a + ml.y * bb;
-      ar = make_float4(ar.x * a + r.x * bb, ar.y * a + r.y * bb, ar.z * a + r.z * bb, ar.w * a + r.w * bb);
-      as = make_float4(as.x * a + s.x * bb, as.y * a + s.y * bb, as.z * a + s.z * bb, as.w * a + s.w * bb);
+      l = mix(l, a, ml.y, bb);
+      ar = make_float4(mix(ar.x, a, r.x, bb), mix(ar.y, a, r.y, bb), mix(ar.z, a, r.z, bb), mix(ar.w, a, r.w, bb));
+      as = make_float4(mix(as.x, a, s.x, bb), mix(as.y, a, s.y, bb), mix(as.z, a, s.z, bb), mix(as.w, a, s.w, bb));
       m = mn;
     }
   }
@@ -811,16 +850,16 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
       const uint2 kr = *reinterpret_cast<const uint2*>(P.k_tail + off);
       const uint2 vr = *reinterpret_cast<const uint2*>(P.v_tail + off);
       const float2 k01 = bf16x2_to_f2(kr.x), k23 = bf16x2_to_f2(kr.y);
-      float d = q01.x * k01.x + q01.y * k01.y + q23.x * k23.x + q23.y * k23.y;
+      float d = __fmaf_rn(q23.y, k23.y, __fmaf_rn(q23.x, k23.x, __fmaf_rn(q01.y, k01.y, __fmul_rn(q01.x, k01.x))));
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
       const float sc = d * P.scale_log2;
       const float mn = fmaxf(m, sc);
       const float a = exp2f(m - mn), p = exp2f(sc - mn);
       const float2 v01 = bf16x2_to_f2(vr.x), v23 = bf16x2_to_f2(vr.y);
-      l = l * a + p;
-      ar = make_float4(ar.x * a + p * v01.x, ar.y * a + p * v01.y, ar.z * a + p * v23.x, ar.w * a + p * v23.y);
-      as = make_float4(as.x * a, as.y * a, as.z * a, as.w * a);
+      l = __fmaf_rn(l, a, p);
+      ar = make_float4(mix(ar.x, a, p, v01.x), mix(ar.y, a, p, v01.y), mix(ar.z, a, p, v23.x), mix(ar.w, a, p, v23.y));
+      as = make_float4(__fmul_rn(as.x, a), __fmul_rn(as.y, a), __fmul_rn(as.z, a), __fmul_rn(as.w, a));
       m = mn;
     }
   }
@@ -841,7 +880,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     as = make_float4(x[0] * c, x[1] * c, x[2] * c, x[3] * c);
   }
   const float inv = l > 0.f ? 1.f / l : 0.f;
-  float4 o = make_float4((ar.x + as.x) * inv, (ar.y + as.y) * inv, (ar.z + as.z) * inv, (ar.w + as.w) * inv);
+  float4 o = make_float4(__fmul_rn(__fadd_rn(ar.x, as.x), inv), __fmul_rn(__fadd_rn(ar.y, as.y), inv),
+                         __fmul_rn(__fadd_rn(ar.z, as.z), inv), __fmul_rn(__fadd_rn(ar.w, as.w), inv));
   reinterpret_cast<float4*>(P.out + (static_cast<int64_t>(b) * Hq + qh) * kD)[lane] = o;
 }
 
@@ -930,7 +970,8 @@ int64_t decode_workspace_bytes(int B, int Hkv, int G, int num_ctas) {
 }
 
 cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_group, int kernel,
-                          const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s) {
+                          const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s,
+                          const EncodeParams* append) {
   kernel = decode_kernel_choice(ref_kind, res_bits, res_group, p.G, kernel);
   cudaError_t e;
   if (kernel == kKernelTensor) {
@@ -942,9 +983,16 @@ cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_gr
     e = fn(p, tmap_k, tmap_v, s);  // sets p.page_tokens
   }
   if (e != cudaSuccess) return e;
-  const int warps = p.B * p.Hkv * p.G;
-  if (warps == 0) return cudaSuccess;
-  decode_combine_kernel<<<(warps + 3) / 4, 128, 0, s>>>(p, p.G, (res_bits != 0 && p.rotate) ? 1 : 0);
+  const int64_t warps = static_cast<int64_t>(p.B) * p.Hkv * p.G;
+  const int64_t enc_warps = append ? static_cast<int64_t>(append->B) * append->Hkv * append->n_tokens : 0;
+  const int rot = (res_bits != 0 && p.rotate) ? 1 : 0;
+  if (enc_warps > 0) {
+    decode_combine_kernel<true><<<static_cast<unsigned>((warps + enc_warps + 3) / 4), 128, 0, s>>>(p, p.G, rot, *append);
+  } else {
+    EncodeParams none;
+    memset(&none, 0, sizeof(none));
+    decode_combine_kernel<false><<<static_cast<unsigned>((warps + 3) / 4), 128, 0, s>>>(p, p.G, rot, none);
+  }
   return cudaGetLastError();
 }
 

@@ -210,8 +210,8 @@ struct TcCfg {
   static constexpr int W_QA = W_CA + 8;                  // [G][4] anchor group sums of q
   static constexpr int W_WM = W_QA + 32;                 // [2][4 warps][4] warp maxima of scores
   static constexpr int W_SIG = W_WM + 32;                // [2][4 warps][12] warp maxima of scales
-  static constexpr int W_RED = W_SIG + 96;               // [G][NRED] flush sums
-  static constexpr int W_PRE = W_RED + 8 * NRED;         // [RQ_MAX_BATCH + 1] page prefix
+  static constexpr int W_RED = W_SIG + 96;               // [4 warps][8 heads][NRED] flush sums
+  static constexpr int W_PRE = W_RED + 4 * 8 * NRED;     // [RQ_MAX_BATCH + 1] page prefix
   static constexpr int W_MISC = W_PRE + RQ_MAX_BATCH + 1;  // abort flag, tensor-memory base
   static constexpr int W_BAR = (W_MISC + 2 + 1) & ~1;    // 8-byte aligned mbarriers
   static constexpr int NBARS = 2 * 4 + 8;
@@ -416,7 +416,6 @@ __global__ void __launch_bounds__(kNT, 1)
     }
     if (lane == 0) sPre[B] = carry;
   }
-  for (int i = tid; i < 8 * C::NRED; i += kNT) sRed[i] = 0.f;
   if (tid == 0) {
     *sAbort = 0;
     for (int s = 0; s < C::STAGES; ++s) {
@@ -1060,19 +1059,22 @@ __global__ void __launch_bounds__(kNT, 1)
 
     // ---- flush a finished (b, h) segment: one partial record per query head
     if (seg_end) {
+      // per-warp sums into their own slots, added in a fixed order below, so
+      // that a decode is reproducible bit for bit from run to run
+      float* myred = sRed + (warp & 3) * 8 * C::NRED;
 #pragma unroll
       for (int i = 0; i < GH; ++i) {
         const int hq = hb + i;
         if (own_ref) {
           const float lsum = warp_sum(l_thr[i]);
-          if (lane == 0) atomicAdd(&sRed[hq * C::NRED], lsum);
+          if (lane == 0) myred[hq * C::NRED] = lsum;
         }
         if constexpr (RB != 0) {
           if (own_res) {
 #pragma unroll
             for (int g = 0; g < NGR; ++g) {
               const float z = warp_sum(zr[i][g]);
-              if (lane == 0) atomicAdd(&sRed[hq * C::NRED + 1 + g], z);
+              if (lane == 0) myred[hq * C::NRED + 1 + g] = z;
             }
           }
         }
@@ -1081,12 +1083,16 @@ __global__ void __launch_bounds__(kNT, 1)
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const float z = warp_sum(za[i][g]);
-              if (lane == 0) atomicAdd(&sRed[hq * C::NRED + 9 + g], z);
+              if (lane == 0) myred[hq * C::NRED + 9 + g] = z;
             }
           }
         }
       }
       named_bar_sync(kBarAll, kNCT);  // both warpgroups' sums (G == 1 splits them)
+      auto red = [&](int hq, int slot) {
+        const float* p = sRed + hq * C::NRED + slot;
+        return __fadd_rn(__fadd_rn(p[0], p[8 * C::NRED]), __fadd_rn(p[16 * C::NRED], p[24 * C::NRED]));
+      };
       const int pair = cur.b * Hkv + cur.h;
       const int d_ref = REF == kRefInt4 ? 32 * chunk + pos_dim<4>(r & 31) : r;
       const int d_res = RB ? 32 * chunk + pos_dim<RB ? RB : 2>(r & 31) : r;
@@ -1097,31 +1103,20 @@ __global__ void __launch_bounds__(kNT, 1)
         if (own_ref) {
           float vref = 0.f;
           if constexpr (REF != kRefNone) vref = acc_ref[i];
-          if constexpr (REF == kRefInt4) {
-            float z = sRed[hq * C::NRED + 9];
-#pragma unroll
-            for (int g = 1; g < 4; ++g) z = (chunk == g) ? sRed[hq * C::NRED + 9 + g] : z;
-            vref += z;
-          }
+          if constexpr (REF == kRefInt4) vref += red(hq, 9 + chunk);
           rec[4 + d_ref] = vref;
           if (r == 0) {
             rec[0] = m_run[i];
-            rec[1] = sRed[hq * C::NRED];
+            rec[1] = red(hq, 0);
           }
         }
         if (own_res) {
           float vres = 0.f;
-          if constexpr (RB != 0) {
-            float z = sRed[hq * C::NRED + 1];
-#pragma unroll
-            for (int g = 1; g < NGR; ++g) z = (g_res == g) ? sRed[hq * C::NRED + 1 + g] : z;
-            vres = acc_res[i] + z;
-          }
+          if constexpr (RB != 0) vres = acc_res[i] + red(hq, 1 + g_res);
           rec[4 + kD + d_res] = vres;
         }
       }
       named_bar_sync(kBarAll, kNCT);
-      if (tid < G * C::NRED) sRed[tid] = 0.f;
       reset_state();
     }
 

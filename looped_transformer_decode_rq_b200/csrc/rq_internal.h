@@ -92,8 +92,11 @@ enum DecodeKernel : int { kKernelAuto = RQ_DECODE_KERNEL_AUTO, kKernelSimt = RQ_
                           kKernelTensor = RQ_DECODE_KERNEL_TENSOR };
 
 // ref_kind: RefKind; res_bits: 0 | 2 | 4; res_group: 16 | 32
+// `append` (or null): tokens to encode into the cache in the same launch as
+// the combine kernel (positions past every context of this decode).
 cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_group, int kernel,
-                          const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
+                          const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s,
+                          const EncodeParams* append = nullptr);
 bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, int kernel);
 // the kernel an automatic choice resolves to
 int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel);

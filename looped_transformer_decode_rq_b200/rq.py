@@ -38,7 +38,7 @@ EXPORTED = ("rq_cache_layout", "rq_cache_create", "rq_cache_destroy", "rq_cache_
             "rq_decode_workspace_size", "rq_decode_attention", "rq_bf16_decode_workspace_size",
             "rq_bf16_decode_attention", "rq_reconstruct", "rq_get_error", "rq_status_string",
             "rq_last_error_message", "rq_decode_attention_static_scratch", "rq_cache_set_decode_kernel",
-            "rq_cache_set_debug_stall")
+            "rq_cache_set_debug_stall", "rq_decode_attention_append")
 STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 
@@ -69,6 +69,8 @@ _sig = {
     "rq_decode_workspace_size": (C.c_int, [_vp, C.POINTER(_i64)]),
     "rq_decode_attention": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp]),
     "rq_decode_attention_static_scratch": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp]),
+    "rq_decode_attention_append": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp, _vp,
+                                             C.POINTER(_i64), _vp, _i32, _vp]),
     "rq_bf16_decode_workspace_size": (C.c_int, [_i32, _i32, _i32, C.POINTER(_i64)]),
     "rq_bf16_decode_attention": (C.c_int, [_i32, _i32, _i32, _vp, _vp, C.POINTER(_i64), _i32, _vp, _vp, _vp,
                                            _vp, _i32, _f32, _vp, _vp, _i64, _vp, _vp]),
@@ -209,6 +211,31 @@ class Cache:
         _check(_lib.rq_decode_attention(self._h, loop, q.data_ptr(), ctx_len.data_ptr(), _ptr(k_tail),
                                         _ptr(v_tail), n_tail, scale, out.data_ptr(), self.workspace.data_ptr(),
                                         self.workspace.numel(), _stream(stream)), "rq_decode_attention")
+        return out
+
+    def decode_attention_append(self, loop: int, q: torch.Tensor, ctx_len: torch.Tensor,
+                                k_tail: Optional[torch.Tensor], v_tail: Optional[torch.Tensor],
+                                k_new: torch.Tensor, v_new: torch.Tensor, positions: torch.Tensor,
+                                softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+        """decode_attention(loop, ...) and the encode of k_new/v_new (bf16 [L, B, Hkv, n, 128])
+        at device positions (int32 [B]) in one call."""
+        cfg = self.cfg
+        assert q.dtype == torch.bfloat16 and q.is_contiguous() and ctx_len.dtype == torch.int32
+        assert k_new.dtype == torch.bfloat16 and v_new.dtype == torch.bfloat16 and k_new.shape == v_new.shape
+        assert k_new.stride() == v_new.stride() and k_new.stride(-1) == 1 and positions.dtype == torch.int32
+        if out is None:
+            out = torch.empty((cfg.batch, cfg.q_heads, HEAD_DIM), dtype=torch.float32, device=q.device)
+        n_tail = 0 if k_tail is None else k_tail.shape[2]
+        if n_tail:
+            assert k_tail.is_contiguous() and v_tail.is_contiguous()
+        scale = softmax_scale if softmax_scale is not None else HEAD_DIM ** -0.5
+        strides = (_i64 * 4)(*k_new.stride()[:4])
+        _check(_lib.rq_decode_attention_append(self._h, loop, q.data_ptr(), ctx_len.data_ptr(), _ptr(k_tail),
+                                               _ptr(v_tail), n_tail, scale, out.data_ptr(), self.workspace.data_ptr(),
+                                               self.workspace.numel(), k_new.data_ptr(), v_new.data_ptr(), strides,
+                                               positions.data_ptr(), k_new.shape[3], _stream(stream)),
+               "rq_decode_attention_append")
         return out
 
     def decode_attention_static_scratch(self, loop: int, q: torch.Tensor, ctx_len: torch.Tensor,

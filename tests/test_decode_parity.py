@@ -247,3 +247,53 @@ def test_wait_limit_sets_flag_and_context_recovers(librq, kernel):
     want = O.decode_attention_f64(enc, 0, to_np32(inp["q"][0]), inp["ctx_len"].numpy(),
                                   to_np32(inp["k_tail"][0]), to_np32(inp["v_tail"][0]))
     assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
+
+
+def _same_planes(a, b):
+    if isinstance(a, dict):
+        assert a.keys() == b.keys()
+        for key in a:
+            _same_planes(a[key], b[key])
+    elif isinstance(a, (list, tuple)):
+        assert len(a) == len(b)
+        for x, y in zip(a, b):
+            _same_planes(x, y)
+    elif a is None:
+        assert b is None
+    else:
+        assert np.array_equal(np.ascontiguousarray(a).view(np.uint8), np.ascontiguousarray(b).view(np.uint8))
+
+
+@pytest.mark.parametrize("kernel", ["simt", "tensor"])
+@pytest.mark.parametrize("bits", [(2, 2, 2, 16), (2, 2, 4, 4)])
+def test_decode_with_fused_append_matches_separate_calls(librq, kernel, bits):
+    """rq_decode_attention_append (the final loop's decode plus the per-step
+    append of every loop's new token, one combine launch) gives the same output
+    and the same cache bytes as a decode followed by an encode at device positions."""
+    from tests.helpers import read_planes
+    rq = librq
+    wl = synth.Workload(name="fused_append", batch=3, kv_heads=2, q_heads=8, context=200, bits=bits,
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, seed=95)
+    inp = synth.make_inputs(wl, "cpu")
+    cfgd = synth.cache_config_dict(wl)
+    k, v = inp["k"].cuda(), inp["v"].cuda()
+    caches = []
+    lay = rq.cache_layout(rq.config_from_dict(cfgd))
+    for _ in range(2):
+        # zeroed buffers: positions neither call writes compare equal too
+        c = rq.Cache(rq.config_from_dict(cfgd), buffer=torch.zeros(lay.total_bytes + 1024, dtype=torch.uint8,
+                                                                    device="cuda"))
+        c.set_decode_kernel(rq.DECODE_KERNEL_SIMT if kernel == "simt" else rq.DECODE_KERNEL_TENSOR)
+        c.encode(k, v)
+        caches.append(c)
+    ctx = torch.tensor([200, 137, 5], dtype=torch.int32, device="cuda")
+    last = wl.num_loops - 1
+    q, kt, vt = inp["q"][last].cuda(), inp["k_tail"][last].cuda(), inp["v_tail"][last].cuda()
+    k_new, v_new = inp["k_tail"].cuda(), inp["v_tail"].cuda()  # [L, B, Hkv, 1, 128]
+    out_a = caches[0].decode_attention(last, q, ctx, kt, vt)
+    caches[0].encode(k_new, v_new, positions=ctx)
+    out_b = caches[1].decode_attention_append(last, q, ctx, kt, vt, k_new, v_new, ctx)
+    torch.cuda.synchronize()
+    assert caches[0].get_error() == 0 and caches[1].get_error() == 0
+    assert torch.equal(out_a, out_b)
+    _same_planes(read_planes(caches[0], wl.context + 1), read_planes(caches[1], wl.context + 1))
