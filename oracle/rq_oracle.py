@@ -41,6 +41,14 @@ with round-to-nearest-even, each operation rounded separately):
   INT4 anchor: the reference loop is group-quantised directly (4 bits, g = 32,
       no alpha, no rotation); the other loops take their alpha and residual
       against its dequantised value  ref_hat = z_hat + (code * s_hat)  (fp32).
+  Chained references ([RQ] Table 9 and Figure 3 caption: the "Previous-loop"
+      and "Next-loop" reference families): loop l's reference is loop l-1
+      (Previous) or l+1 (Next), and the chain ends at loop 0 or L-1, the anchor.
+      A loop that is the reference of another is seen by the encoder as its
+      binary32 reconstruction  x_hat = (alpha_hat * ref_hat) + u  with
+      u = the rotation of deq (the rotation is its own inverse), deq = z_hat +
+      (code * s_hat); alpha and the residual of the next loop are taken against
+      that x_hat, since it is all a decoder has.
 
 Reconstruction and decode attention are computed in float64 from the stored
 codes and metadata.  The rotation there is an explicit 128x128 matrix built
@@ -66,7 +74,7 @@ INV_SQRT_D_F32 = np.float32(1.0 / np.sqrt(128.0))
 FP16_MAX = 65504.0
 
 ALPHA_LS, ALPHA_ONE, ALPHA_ZERO, ALPHA_NORM = 0, 1, 2, 3
-ANCHOR_LAST, ANCHOR_FIRST, ANCHOR_INTERVAL = 0, 1, 2
+ANCHOR_LAST, ANCHOR_FIRST, ANCHOR_INTERVAL, ANCHOR_PREVIOUS, ANCHOR_NEXT = 0, 1, 2, 3, 4
 
 
 # ---------------------------------------------------------------------------
@@ -214,12 +222,15 @@ class CacheConfig:
     """Per-loop formats and which loop each loop takes as its reference.
 
     Anchor policies ([RQ] Table 1 "First-loop" / "Last-loop"; Table 8 anchor
-    intervals "N x [2^n, 4]", each group ending in its own anchor):
+    intervals "N x [2^n, 4]", each group ending in its own anchor; Table 9
+    "Previous-loop" / "Next-loop"):
       ANCHOR_LAST: the final loop is every loop's reference;
       ANCHOR_FIRST: loop 0 is every loop's reference;
       ANCHOR_INTERVAL: blocks of `anchor_interval` consecutive loops, the last
         loop of each block (or the final loop, for a short last block) being
-        the reference of the others in its block.
+        the reference of the others in its block;
+      ANCHOR_PREVIOUS: loop l's reference is loop l-1; loop 0 is the anchor;
+      ANCHOR_NEXT: loop l's reference is loop l+1; the final loop is the anchor.
     Anchor loops use bits 16 (bf16) or 4 (INT4, g = 32); the others 2 or 4.
     """
     num_loops: int
@@ -236,14 +247,34 @@ class CacheConfig:
                            list(d["rotate"]), list(d["alpha_mode"]),
                            d.get("anchor_policy", ANCHOR_LAST), d.get("anchor_interval", 0))
 
-    def anchor_of(self, loop: int) -> int:
+    def ref_of(self, loop: int) -> int:
+        """The loop whose (reconstructed) values loop `loop` is stored against;
+        `loop` itself for an anchor."""
         L = self.num_loops
         if self.anchor_policy == ANCHOR_LAST:
             return L - 1
         if self.anchor_policy == ANCHOR_FIRST:
             return 0
+        if self.anchor_policy == ANCHOR_PREVIOUS:
+            return max(loop - 1, 0)
+        if self.anchor_policy == ANCHOR_NEXT:
+            return min(loop + 1, L - 1)
         n = self.anchor_interval
         return min((loop // n) * n + n - 1, L - 1)
+
+    def chain(self, loop: int) -> List[int]:
+        """The residual loops from `loop` toward its anchor (the anchor itself
+        excluded): [loop, ref_of(loop), ...]; empty for an anchor."""
+        out = []
+        while self.ref_of(loop) != loop:
+            out.append(loop)
+            loop = self.ref_of(loop)
+        return out
+
+    def anchor_of(self, loop: int) -> int:
+        while self.ref_of(loop) != loop:
+            loop = self.ref_of(loop)
+        return loop
 
     def is_anchor(self, loop: int) -> bool:
         return self.anchor_of(loop) == loop
@@ -271,7 +302,7 @@ class Encoded:
     # per anchor loop a: 'k'/'v' float32 bf16 values, or the INT4 EncodedPlane
     anchor_bf16: Dict[int, Dict[str, np.ndarray]] = field(default_factory=dict)
     anchor_q: Dict[int, Dict[str, EncodedPlane]] = field(default_factory=dict)
-    anchor_hat32: Dict[int, Dict[str, np.ndarray]] = field(default_factory=dict)  # encoder's fp32 view
+    hat32: Dict[int, Dict[str, np.ndarray]] = field(default_factory=dict)  # encoder's fp32 view of references
     loops: List[Optional[Dict[str, EncodedPlane]]] = field(default_factory=list)  # None for anchors
     error: bool = False
 
@@ -280,11 +311,25 @@ def _check_range(x: np.ndarray) -> bool:
     return bool(np.all(np.isfinite(x)) and np.all(np.abs(x) <= FP16_MAX))
 
 
+def reconstruct_fp32(qg: QuantGroups, g: int, rotate: int, alpha_hat: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """The encoder's binary32 view of a stored residual loop, used as the next
+    loop's reference under a chained policy:  (alpha_hat * ref) + u,  with u the
+    rotation of z_hat + (code * s_hat) (the orthonormal Hadamard is symmetric,
+    so the same transform undoes it)."""
+    u = dequant_fp32(qg, g)
+    if rotate:
+        u = fwht_fp32(u)
+    a32 = np.asarray(alpha_hat).astype(F32)[..., None]
+    return ((a32 * np.asarray(ref, F32)).astype(F32) + u).astype(F32)
+
+
 def encode_fp32emu(K: np.ndarray, V: np.ndarray, cfg: CacheConfig) -> Encoded:
     """Encode every loop of the cached tokens.
 
     K, V: float32 [L, ..., 128] holding bf16 values (any leading shape after
-    the loop axis, e.g. [B, H, T]).  The last loop is the reference.
+    the loop axis, e.g. [B, H, T]).  Anchors are stored first; every other loop
+    is encoded against its reference after that reference (nearest the anchor
+    first, so a chain is walked outward from its anchor).
     """
     L = cfg.num_loops
     assert K.shape[0] == L and V.shape == K.shape
@@ -292,26 +337,27 @@ def encode_fp32emu(K: np.ndarray, V: np.ndarray, cfg: CacheConfig) -> Encoded:
     enc.error = not (_check_range(K) and _check_range(V))
     for a in cfg.anchors():
         rb = cfg.bits[a]
-        enc.anchor_bf16[a], enc.anchor_q[a], enc.anchor_hat32[a] = {}, {}, {}
+        enc.anchor_bf16[a], enc.anchor_q[a], enc.hat32[a] = {}, {}, {}
         for name, X in (("k", K), ("v", V)):
             ref = np.asarray(X[a], dtype=F32)
             if rb == 16:
                 enc.anchor_bf16[a][name] = ref
-                enc.anchor_hat32[a][name] = ref
+                enc.hat32[a][name] = ref
             elif rb == 4:
                 qg = quantize_groups_fp32(ref, 4, 32)
                 enc.anchor_q[a][name] = EncodedPlane(qg.codes, qg.scale, qg.zero, None, qg.near_tie, 4, 32, 0)
-                enc.anchor_hat32[a][name] = dequant_fp32(qg, 32)
+                enc.hat32[a][name] = dequant_fp32(qg, 32)
             else:
                 raise ValueError("anchor bits must be 16 or 4")
-    for l in range(L):
-        if cfg.is_anchor(l):
-            enc.loops.append(None)
-            continue
+    enc.loops = [None] * L
+    is_ref = {cfg.ref_of(l) for l in range(L) if not cfg.is_anchor(l)}
+    for l in sorted((l for l in range(L) if not cfg.is_anchor(l)), key=lambda l: len(cfg.chain(l))):
         planes = {}
+        if l in is_ref:
+            enc.hat32[l] = {}
         for name, X in (("k", K), ("v", V)):
             x = np.asarray(X[l], dtype=F32)
-            ref = enc.anchor_hat32[cfg.anchor_of(l)][name]
+            ref = enc.hat32[cfg.ref_of(l)][name]
             a_hat = ls_alpha_fp32(x, ref, cfg.alpha_mode[l])
             if not np.all(np.isfinite(a_hat.astype(np.float64))):
                 enc.error = True
@@ -324,7 +370,9 @@ def encode_fp32emu(K: np.ndarray, V: np.ndarray, cfg: CacheConfig) -> Encoded:
                 enc.error = True
             planes[name] = EncodedPlane(qg.codes, qg.scale, qg.zero, a_hat, qg.near_tie,
                                         cfg.bits[l], cfg.group[l], cfg.rotate[l])
-        enc.loops.append(planes)
+            if l in is_ref:
+                enc.hat32[l][name] = reconstruct_fp32(qg, cfg.group[l], cfg.rotate[l], a_hat, ref)
+        enc.loops[l] = planes
     return enc
 
 
@@ -351,14 +399,16 @@ def residual_f64(p: EncodedPlane) -> np.ndarray:
 
 
 def reconstruct_f64(enc: Encoded, loop: int):
-    """(K_hat, V_hat) float64 of one loop: alpha_hat * ref + H^T deq(codes)."""
-    a = enc.cfg.anchor_of(loop)
-    if loop == a:
-        return reference_f64(enc, "k", a), reference_f64(enc, "v", a)
+    """(K_hat, V_hat) float64 of one loop: alpha_hat * ref_hat + H^T deq(codes),
+    where ref_hat is the anchor's values or, under a chained policy, the
+    reconstruction of the loop's reference (computed the same way)."""
+    cfg = enc.cfg
+    if cfg.is_anchor(loop):
+        return reference_f64(enc, "k", loop), reference_f64(enc, "v", loop)
+    refs = reconstruct_f64(enc, cfg.ref_of(loop))
     out = []
-    for name in ("k", "v"):
+    for name, ref in zip(("k", "v"), refs):
         p = enc.loops[loop][name]
-        ref = reference_f64(enc, name, a)
         out.append(p.alpha.astype(np.float64)[..., None] * ref + residual_f64(p))
     return out[0], out[1]
 
@@ -387,6 +437,12 @@ def decode_attention_f64(enc: Encoded, loop: int, q: np.ndarray, ctx_len: np.nda
         scale * (alpha_K (q . ref_k) + (H q) . deq(codes_K))
     and the output is
         (sum_t p_t alpha_V,t ref_v,t + H^T sum_t p_t deq(codes_V,t) + sum_tail p v) / sum p.
+    Under a chained policy the loop's chain l = c_0 -> c_1 -> ... -> c_{n-1} ->
+    anchor unrolls the recursion  x_hat_c = alpha_c x_hat_{ref(c)} + H^T deq_c:
+        x_hat_l = beta_n ref + sum_i beta_i H^T deq(codes_{c_i}),
+        beta_0 = 1, beta_{i+1} = beta_i * alpha_{c_i}   (per token, K and V apart),
+    so the score takes beta_n (q . ref_k) + sum_i beta_i (H q) . deq_i and the
+    value sums weigh each term by p_t times its beta.
     Returns float64 [B, Hq, 128].
     """
     cfg = enc.cfg
@@ -399,37 +455,36 @@ def decode_attention_f64(enc: Encoded, loop: int, q: np.ndarray, ctx_len: np.nda
     G = Hq // Hkv
     Hn = hadamard_orthonormal(D)
     out = np.zeros((B, Hq, D))
-    is_ref = loop == a
-    if not is_ref:
-        pk, pv = enc.loops[loop]["k"], enc.loops[loop]["v"]
-        yk = dequant_f64(pk.codes, pk.scale, pk.zero, pk.group)
-        yv = dequant_f64(pv.codes, pv.scale, pv.zero, pv.group)
+    members = cfg.chain(loop)
+    terms = []  # per chain member: (deq K, deq V, rotate, beta K, beta V), betas [B, Hkv, T]
+    bk = np.ones(refk.shape[:-1])
+    bv = np.ones(refv.shape[:-1])
+    for c in members:
+        pk, pv = enc.loops[c]["k"], enc.loops[c]["v"]
+        terms.append((dequant_f64(pk.codes, pk.scale, pk.zero, pk.group),
+                      dequant_f64(pv.codes, pv.scale, pv.zero, pv.group), pk.rotate, bk, bv))
+        bk = bk * pk.alpha.astype(np.float64)
+        bv = bv * pv.alpha.astype(np.float64)
     for b in range(B):
         n = int(ctx_len[b])
         for qh in range(Hq):
             h = qh // G
             qv = q[b, qh]
-            scores = []
-            if is_ref:
-                scores.append(scale * (refk[b, h, :n] @ qv))
-            else:
-                qr = Hn @ qv if pk.rotate else qv
-                ak = pk.alpha[b, h, :n].astype(np.float64)
-                scores.append(scale * (ak * (refk[b, h, :n] @ qv) + yk[b, h, :n] @ qr))
+            s_c = bk[b, h, :n] * (refk[b, h, :n] @ qv)
+            for yk, _, rot, tk, _ in terms:
+                qr = Hn @ qv if rot else qv
+                s_c = s_c + tk[b, h, :n] * (yk[b, h, :n] @ qr)
+            scores = [scale * s_c]
             if k_tail is not None and k_tail.shape[2] > 0:
                 scores.append(scale * (np.asarray(k_tail[b, h], np.float64) @ qv))
             p, lsum = _softmax_combine(scores)
             if p is None:
                 continue
             pc, pt = p[:n], p[n:]
-            if is_ref:
-                o = pc @ refv[b, h, :n]
-            else:
-                av = pv.alpha[b, h, :n].astype(np.float64)
-                acc_res = pc @ yv[b, h, :n]
-                if pv.rotate:
-                    acc_res = Hn @ acc_res
-                o = (pc * av) @ refv[b, h, :n] + acc_res
+            o = (pc * bv[b, h, :n]) @ refv[b, h, :n]
+            for _, yv, rot, _, tv in terms:
+                acc_res = (pc * tv[b, h, :n]) @ yv[b, h, :n]
+                o = o + (Hn @ acc_res if rot else acc_res)
             if pt.size:
                 o = o + pt @ np.asarray(v_tail[b, h], np.float64)
             out[b, qh] = o / lsum

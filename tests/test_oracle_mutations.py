@@ -71,6 +71,31 @@ def _decode_drop_value_alpha(enc, loop, q, ctx_len, k_tail=None, v_tail=None, sc
         enc.loops[loop]["v"].alpha = saved
 
 
+def _reconstruct_chain_via_anchor(enc, loop):
+    cfg = enc.cfg
+    if cfg.is_anchor(loop):
+        return ORIG["reconstruct_f64"](enc, loop)
+    a = cfg.anchor_of(loop)
+    return tuple(enc.loops[loop][n].alpha.astype(np.float64)[..., None] * O.reference_f64(enc, n, a)
+                 + O.residual_f64(enc.loops[loop][n]) for n in ("k", "v"))
+
+
+def _chain_view_without_residual(qg, g, rotate, alpha_hat, ref):
+    return (np.asarray(alpha_hat).astype(np.float32)[..., None] * np.asarray(ref, np.float32)).astype(np.float32)
+
+
+def _decode_chain_drops_link_alpha(enc, loop, q, ctx_len, k_tail=None, v_tail=None, scale=1 / np.sqrt(128)):
+    deeper = enc.cfg.chain(loop)[1:]
+    saved = {c: enc.loops[c]["k"].alpha for c in deeper}
+    for c in deeper:
+        enc.loops[c]["k"].alpha = np.ones_like(saved[c])
+    try:
+        return ORIG["decode_attention_f64"](enc, loop, q, ctx_len, k_tail, v_tail, scale)
+    finally:
+        for c in deeper:
+            enc.loops[c]["k"].alpha = saved[c]
+
+
 def _tree_dot_drops_last_lane(a, b):
     prod = (np.asarray(a, np.float32) * np.asarray(b, np.float32)).astype(np.float32)
     return prod[..., :120].sum(-1, dtype=np.float32)
@@ -78,7 +103,7 @@ def _tree_dot_drops_last_lane(a, b):
 
 ORIG = {n: getattr(O, n) for n in ("fwht_fp32", "ls_alpha_fp32", "reconstruct_f64", "residual_f64",
                                    "quantize_groups_fp32", "dequant_f64", "decode_attention_f64",
-                                   "lane_tree_dot_fp32")}
+                                   "lane_tree_dot_fp32", "reconstruct_fp32")}
 
 PINS = [
     P.test_p1_alpha_minimises_squared_error,
@@ -94,6 +119,9 @@ PINS = [
     P.test_p6_two_token_softmax_by_hand,
     P.test_p7_ls_scaling_never_worse_than_unit_scale,
     lambda: [P.test_p8_full_precision_residual_reconstructs(r) for r in (0, 1)],
+    lambda: [P.test_chained_scaled_copies_reconstruct_exactly(p, 1) for p in (O.ANCHOR_PREVIOUS, O.ANCHOR_NEXT)],
+    lambda: P.test_chained_reconstruction_error_is_the_quantiser_error(O.ANCHOR_NEXT, 16),
+    lambda: P.test_chained_decode_equals_brute_force(O.ANCHOR_NEXT, 4),
 ]
 
 
@@ -115,6 +143,9 @@ def _any_pin_fails():
     ("dequant_f64", _dequant_strided_groups),
     ("decode_attention_f64", _decode_drop_value_alpha),
     ("lane_tree_dot_fp32", _tree_dot_drops_last_lane),
+    ("reconstruct_f64", _reconstruct_chain_via_anchor),
+    ("reconstruct_fp32", _chain_view_without_residual),
+    ("decode_attention_f64", _decode_chain_drops_link_alpha),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, mutant):
     monkeypatch.setattr(O, name, mutant)

@@ -406,3 +406,155 @@ def test_anchor_interval_decode_equals_brute_force():
         Kh, Vh = O.reconstruct_f64(enc, loop)
         want = O.attention_f64(q, Kh, Vh, ctx, kt, vt)
         assert np.abs(got - want).max() <= 1e-12 * max(1.0, np.abs(want).max())
+
+
+# ------------------------------------------- chained references (Previous-/Next-loop)
+# [RQ] Table 9 ("Previous-loop", "Next-loop" rows) and Figure 3 caption (the
+# Previous-/Next-loop reference family): each loop is stored against its
+# neighbour, so a loop is reconstructed through the chain down to the anchor.
+
+def test_ref_of_chain_policies():
+    prev = O.CacheConfig(4, [4, 2, 2, 2], [32] * 4, [0, 1, 1, 1], [0] * 4, O.ANCHOR_PREVIOUS)
+    assert [prev.ref_of(l) for l in range(4)] == [0, 0, 1, 2]
+    assert [prev.anchor_of(l) for l in range(4)] == [0, 0, 0, 0]
+    assert [prev.chain(l) for l in range(4)] == [[], [1], [2, 1], [3, 2, 1]]
+    nxt = O.CacheConfig(4, [2, 2, 2, 4], [32] * 4, [1, 1, 1, 0], [0] * 4, O.ANCHOR_NEXT)
+    assert [nxt.ref_of(l) for l in range(4)] == [1, 2, 3, 3]
+    assert [nxt.anchor_of(l) for l in range(4)] == [3, 3, 3, 3]
+    assert [nxt.chain(l) for l in range(4)] == [[0, 1, 2], [1, 2], [2], []]
+    assert nxt.anchors() == [3] and prev.anchors() == [0]
+
+
+@pytest.mark.parametrize("policy", [O.ANCHOR_PREVIOUS, O.ANCHOR_NEXT])
+@pytest.mark.parametrize("rotate", [0, 1])
+def test_chained_scaled_copies_reconstruct_exactly(policy, rotate):
+    """Each loop an exact power-of-two multiple of its neighbour: every alpha is
+    that factor, every residual and code is zero, and the reconstruction through
+    the chain gives back the loops exactly (products of powers of two are exact)."""
+    rng = np.random.default_rng(95)
+    L = 4
+    anchor = 0 if policy == O.ANCHOR_PREVIOUS else L - 1
+    bits = [2] * L
+    bits[anchor] = 16
+    rot = [rotate] * L
+    rot[anchor] = 0
+    cfg = O.CacheConfig(L, bits, [32] * L, rot, [0] * L, policy)
+    factor = {0: 2.0, 1: -0.5, 2: -2.0, 3: 0.5}
+    X = [None] * L
+    X[anchor] = bf16_values(rng, (1, 2, 9, 128))
+    for l in sorted(range(L), key=lambda l: len(cfg.chain(l))):
+        if l != anchor:
+            X[l] = (np.float32(factor[l]) * X[cfg.ref_of(l)]).astype(np.float32)
+    K = np.stack(X)
+    enc = O.encode_fp32emu(K, -K, cfg)
+    for l in range(L):
+        kh, vh = O.reconstruct_f64(enc, l)
+        assert np.array_equal(kh, K[l].astype(np.float64))
+        assert np.array_equal(vh, -K[l].astype(np.float64))
+        if l != anchor:
+            assert np.all(enc.loops[l]["k"].codes == 0)
+            assert np.all(enc.loops[l]["k"].alpha.astype(np.float64) == factor[l])
+
+
+def _neighbour_chain_loops(rng, cfg, shape, noise=0.25):
+    """Loops that each resemble their reference: x_l = a_l x_ref(l) + noise."""
+    L = cfg.num_loops
+    X = [None] * L
+    for l in sorted(range(L), key=lambda l: len(cfg.chain(l))):
+        if cfg.is_anchor(l):
+            X[l] = bf16_values(rng, shape)
+        else:
+            x = (np.float32(rng.uniform(0.8, 1.2)) * X[cfg.ref_of(l)]
+                 + np.float32(noise) * rng.standard_normal(shape).astype(np.float32))
+            u = x.astype(np.float32).view(np.uint32)  # round to bf16, nearest even
+            X[l] = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32).view(np.float32)
+    return np.stack(X)
+
+
+@pytest.mark.parametrize("policy,anchor_bits", [(O.ANCHOR_NEXT, 16), (O.ANCHOR_NEXT, 4), (O.ANCHOR_PREVIOUS, 4)])
+def test_chained_reconstruction_error_is_the_quantiser_error(policy, anchor_bits):
+    """In the rotated domain the chained reconstruction differs from the input
+    loop only by the quantiser: H (x_hat_l - x_l) = deq - H (x_l - alpha x_hat_ref)
+    with x_hat_ref the reconstruction of the reference, so every coordinate obeys
+    the min-max quantiser's bound.  A residual taken against anything but the
+    reconstructed reference breaks the bound at depth >= 2."""
+    rng = np.random.default_rng(96)
+    L = 4
+    anchor = 0 if policy == O.ANCHOR_PREVIOUS else L - 1
+    bits, group = [2] * L, [32] * L
+    bits[anchor] = anchor_bits
+    group[1] = 16
+    rot = [1] * L
+    rot[anchor] = 0
+    cfg = O.CacheConfig(L, bits, group, rot, [0] * L, policy)
+    K = _neighbour_chain_loops(rng, cfg, (2, 2, 40, 128))
+    V = _neighbour_chain_loops(rng, cfg, (2, 2, 40, 128))
+    enc = O.encode_fp32emu(K, V, cfg)
+    Hn = scipy.linalg.hadamard(128) / np.sqrt(128.0)
+    for l in range(L):
+        if cfg.is_anchor(l):
+            continue
+        refs = O.reconstruct_f64(enc, cfg.ref_of(l))
+        hats = O.reconstruct_f64(enc, l)
+        for name, X, ref, hat in (("k", K, refs[0], hats[0]), ("v", V, refs[1], hats[1])):
+            p = enc.loops[l][name]
+            x = X[l].astype(np.float64)
+            y = (x - p.alpha.astype(np.float64)[..., None] * ref)
+            if p.rotate:
+                y = y @ Hn
+            g, qmax = p.group, (1 << p.bits) - 1
+            ys = y.reshape(y.shape[:-1] + (128 // g, g))
+            mn = ys.min(-1)
+            s = (ys.max(-1) - mn) / qmax
+            sh, zh = p.scale.astype(np.float64), p.zero.astype(np.float64)
+            bound = 0.5 * sh + qmax * np.abs(sh - s) + np.abs(zh - mn) + 1e-5 * np.abs(x).max(-1)[..., None]
+            err = hat - x
+            if p.rotate:
+                err = err @ Hn
+            err = np.abs(err.reshape(ys.shape)).max(-1)
+            assert np.all(err <= bound), (l, name)
+
+
+@pytest.mark.parametrize("policy", [O.ANCHOR_PREVIOUS, O.ANCHOR_NEXT])
+@pytest.mark.parametrize("anchor_bits", [16, 4])
+def test_chained_decode_equals_brute_force(policy, anchor_bits):
+    rng = np.random.default_rng(97)
+    L, B, H, T = 5, 2, 2, 17
+    anchor = 0 if policy == O.ANCHOR_PREVIOUS else L - 1
+    bits, group = [2, 4, 2, 2, 4], [32, 32, 16, 32, 16]
+    rot, modes = [1, 0, 1, 1, 1], [0, 3, 1, 0, 0]
+    bits[anchor], group[anchor], rot[anchor] = anchor_bits, 32, 0
+    cfg = O.CacheConfig(L, bits, group, rot, modes, policy)
+    K = _neighbour_chain_loops(rng, cfg, (B, H, T, 128))
+    V = _neighbour_chain_loops(rng, cfg, (B, H, T, 128))
+    enc = O.encode_fp32emu(K, V, cfg)
+    q = bf16_values(rng, (B, 2 * H, 128))
+    kt, vt = bf16_values(rng, (B, H, 2, 128)), bf16_values(rng, (B, H, 2, 128))
+    ctx = np.array([17, 5])
+    for loop in range(L):
+        got = O.decode_attention_f64(enc, loop, q, ctx, kt, vt)
+        Kh, Vh = O.reconstruct_f64(enc, loop)
+        want = O.attention_f64(q, Kh, Vh, ctx, kt, vt)
+        assert np.abs(got - want).max() <= 1e-12 * max(1.0, np.abs(want).max())
+
+
+def test_chain_of_one_link_equals_star_policies():
+    """With two loops the Next-loop chain is the Last-loop policy and the
+    Previous-loop chain the First-loop policy; with four loops the loop next to
+    the anchor is stored identically under both families."""
+    rng = np.random.default_rng(98)
+    K = np.stack([bf16_values(rng, (1, 2, 13, 128)) for _ in range(4)])
+    V = np.stack([bf16_values(rng, (1, 2, 13, 128)) for _ in range(4)])
+    for star, chain, L, loop in ((O.ANCHOR_LAST, O.ANCHOR_NEXT, 2, 0), (O.ANCHOR_FIRST, O.ANCHOR_PREVIOUS, 2, 1),
+                                 (O.ANCHOR_LAST, O.ANCHOR_NEXT, 4, 2), (O.ANCHOR_FIRST, O.ANCHOR_PREVIOUS, 4, 1)):
+        anchor = L - 1 if star == O.ANCHOR_LAST else 0
+        bits = [2] * L
+        bits[anchor] = 16
+        rot = [1] * L
+        rot[anchor] = 0
+        a = O.encode_fp32emu(K[:L], V[:L], O.CacheConfig(L, bits, [32] * L, rot, [0] * L, star))
+        b = O.encode_fp32emu(K[:L], V[:L], O.CacheConfig(L, bits, [32] * L, rot, [0] * L, chain))
+        for n in "kv":
+            assert np.array_equal(a.loops[loop][n].codes, b.loops[loop][n].codes)
+            assert np.array_equal(a.loops[loop][n].alpha, b.loops[loop][n].alpha)
+            assert np.array_equal(a.loops[loop][n].scale, b.loops[loop][n].scale)
