@@ -171,15 +171,20 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 
 def record_bytes(lay, cfgd, loop):
-    """Bytes one decode call of `loop` reads per (b, kv-head, token)."""
+    """Bytes one decode call of `loop` reads per (b, kv-head, token): its
+    anchor's record and, for every residual link between the loop and the
+    anchor (one, or up to three under a chained policy), codes, meta and alpha."""
     a = lay.anchor_of[loop]
     ref = 2 * lay.codes_record_bytes[a] + 2 * lay.meta_record_bytes[a]
     if loop == a:
         return ref
-    res = 2 * lay.codes_record_bytes[loop] + 2 * lay.meta_record_bytes[loop]
     if cfgd["alpha_mode"][loop] == 2:
-        return res
-    return ref + res + 4
+        return 2 * lay.codes_record_bytes[loop] + 2 * lay.meta_record_bytes[loop]
+    total, link = ref, loop
+    while link != a:
+        total += 2 * lay.codes_record_bytes[link] + 2 * lay.meta_record_bytes[link] + 4
+        link = lay.ref_of[link]
+    return total
 
 
 def call_bytes(lay, cfgd, loop, tokens_total, B, Hq, Hkv, n_tail):
@@ -298,7 +303,7 @@ def time_steps(step, steps, warmup, world, stream):
     return max_over_ranks(a.elapsed_time(b) / steps, world)
 
 
-def measure_workload(wl, steps, warmup, world, rank):
+def measure_workload(wl, steps, warmup, world, rank, per_loop=False):
     """RQ decode step and bf16-cache step of one workload (side lines of the
     main result): tokens/s, residual-loop GB/s and the speed-up over bf16."""
     from looped_transformer_decode_rq_b200 import rq
@@ -337,17 +342,19 @@ def measure_workload(wl, steps, warmup, world, rank):
 
     def call_gbs(kernel):
         cache.set_decode_kernel(kernel)
-        for _ in range(3):
-            cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
-        evs = []
-        for _ in range(7):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
-            b.record(stream)
-            evs.append((a, b))
-        torch.cuda.synchronize()
-        cache.set_decode_kernel(rq.DECODE_KERNEL_AUTO)
+        try:
+            for _ in range(3):
+                cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
+            evs = []
+            for _ in range(7):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
+                b.record(stream)
+                evs.append((a, b))
+            torch.cuda.synchronize()
+        finally:
+            cache.set_decode_kernel(rq.DECODE_KERNEL_AUTO)
         return round(res_bytes / (statistics.median(a.elapsed_time(b) for a, b in evs) * 1e-3) / 1e9, 1)
 
     per_kernel = {"simt": call_gbs(rq.DECODE_KERNEL_SIMT)}
@@ -363,12 +370,30 @@ def measure_workload(wl, steps, warmup, world, rank):
             rq.bf16_decode_attention(inp["k"][l], inp["v"][l], q[l], ctx, k_new[l], v_new[l], workspace=ws, out=outs[l])
 
     bms = time_steps(bf16_step, steps, warmup, world, stream)
+    loop_gbs = None
+    if per_loop:  # every loop's decode call alone (a chained policy reads more links for farther loops)
+        loop_gbs = {}
+        for l in range(L):
+            evs = []
+            for i in range(8):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
+                b.record(stream)
+                if i >= 3:
+                    evs.append((a, b))
+            torch.cuda.synchronize()
+            lb = call_bytes(cache.layout, cfgd, l, tokens_total, B, Hq, Hkv, 1)
+            loop_gbs[str(l)] = {"bytes": lb, "gbs": round(lb / (statistics.median(a.elapsed_time(b) for a, b in evs)
+                                                                 * 1e-3) / 1e9, 1)}
     flags = cache.get_error()
     out = {"workload": wl.name, "tokens_per_s": round(job_tokens_per_s(B, world, ms), 1),
            "ms_per_step": round(ms, 4), "residual_loop_gbs": round(res_bytes / (call_ms * 1e-3) / 1e9, 1),
            "residual_loop_bytes": res_bytes, "residual_loop_gbs_by_kernel": per_kernel,
            "bf16_tokens_per_s": round(job_tokens_per_s(B, world, bms), 1),
            "rq_speedup_vs_bf16": round(bms / ms, 3), "device_flags": flags}
+    if loop_gbs is not None:
+        out["loop_gbs"] = loop_gbs
     del cache, inp, outs, ws
     torch.cuda.empty_cache()
     return out
@@ -616,7 +641,7 @@ def run_rq(args, world, rank):
     step_bytes += L * B * Hkv * 512 + B * Hkv * (sum(record_bytes(lay, cfgd, l) for l in range(L)))
     peak, peak_kind = load_peaks()
     kernel_hash = source_hash([os.path.join(ROOT, "looped_transformer_decode_rq_b200", "csrc", f)
-                               for f in ("rq_decode.cu", "rq_common.cuh")])
+                               for f in ("rq_decode.cu", "rq_decode_split.cuh", "rq_common.cuh")])
     achieved = res_bytes / (call_ms * 1e-3) / 1e9
     traffic = read_profile_traffic(kernel_hash)
     value = job_tokens_per_s(B, world, ms)
@@ -697,7 +722,8 @@ def run_rq(args, world, rank):
         torch.cuda.empty_cache()
         extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 10, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8), 10, 3, world, rank),
-                 measure_workload(synth.gqa_long(batch=8, q_heads=64), 10, 3, world, rank)]
+                 measure_workload(synth.gqa_long(batch=8, q_heads=64), 10, 3, world, rank),
+                 measure_workload(synth.ouro_8k_next_loop(), 10, 3, world, rank, per_loop=True)]
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

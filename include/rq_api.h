@@ -84,15 +84,29 @@ typedef enum rq_alpha_mode {
   RQ_ALPHA_NORM_RATIO = 3
 } rq_alpha_mode;
 
-/* Which loop is each loop's reference ("anchor"): [RQ] Table 1 ("First-loop",
- * "Last-loop" reference choice) and Table 8 (anchor intervals N x [2^n, 4]:
- * groups of loops each ending in its own INT4 anchor). */
+/* Which loop is each loop's reference: [RQ] Table 1 ("First-loop",
+ * "Last-loop" reference choice), Table 8 (anchor intervals N x [2^n, 4]:
+ * groups of loops each ending in its own INT4 anchor) and Table 9 / Figure 3
+ * caption (the "Previous-loop" and "Next-loop" reference family).
+ * Under the two chained policies loop l is stored against the reconstruction
+ *     x_hat_ref = alpha_ref * x_hat_ref(ref) + H^T deq(codes_ref)
+ * of its neighbour (binary32, in that order: the product, the rotation of the
+ * dequantised codes, then their sum), so that decoding loop l reads the codes
+ * of every loop between it and the anchor.  Chained policies need every
+ * residual loop in one format (same bits, group and rotate; alpha_mode not
+ * RQ_ALPHA_ZERO) and num_loops <= 4 (at most RQ_MAX_CHAIN residual loops on a
+ * chain); other configurations are RQ_ERR_UNSUPPORTED. */
 typedef enum rq_anchor_policy {
   RQ_ANCHOR_LAST = 0,     /* the final loop is every loop's reference (the pages' choice) */
   RQ_ANCHOR_FIRST = 1,    /* loop 0 is every loop's reference */
-  RQ_ANCHOR_INTERVAL = 2  /* blocks of anchor_interval loops; each block's last loop
+  RQ_ANCHOR_INTERVAL = 2, /* blocks of anchor_interval loops; each block's last loop
                              (the final loop for a short last block) anchors the block */
+  RQ_ANCHOR_PREVIOUS = 3, /* loop l's reference is loop l-1; loop 0 is the anchor */
+  RQ_ANCHOR_NEXT = 4      /* loop l's reference is loop l+1; the final loop is the anchor */
 } rq_anchor_policy;
+
+/* Longest chain of residual loops a decode call reads (chained policies). */
+#define RQ_MAX_CHAIN 3
 
 /* Cache configuration ([RQ] Table 5 caption: loop-wise precision, INT2 with
  * g = 16 or 32, INT4 with g = 32; Figure 1 step 5: mixed precision such as
@@ -129,7 +143,9 @@ typedef struct rq_config {
  *                 alpha = (fp16 alpha_K, fp16 alpha_V) = 4 B
  *  status:        one 32-bit device status word (256 B reserved)
  *  anchor_of[l] is the loop whose anchor planes loop l is decoded against
- *  (anchor_of[l] == l for an anchor loop).
+ *  (anchor_of[l] == l for an anchor loop); ref_of[l] is the loop whose
+ *  (reconstructed) values loop l is stored against: anchor_of[l] except under
+ *  the chained policies, where it is the neighbouring loop.
  */
 typedef struct rq_layout {
   int64_t capacity_padded;
@@ -141,6 +157,7 @@ typedef struct rq_layout {
   int64_t codes_record_bytes[RQ_MAX_LOOPS];
   int64_t meta_record_bytes[RQ_MAX_LOOPS];
   int32_t anchor_of[RQ_MAX_LOOPS];
+  int32_t ref_of[RQ_MAX_LOOPS];
 } rq_layout;
 
 typedef struct rq_cache rq_cache;
@@ -189,13 +206,15 @@ RQ_API rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const 
 
 /* Decode kernel selection (not a numerical choice: both kernels compute the
  * same attention within the decode tolerance).
- *  RQ_DECODE_KERNEL_SIMT    split kernel on the CUDA cores, 64-token pages,
+ *  RQ_DECODE_KERNEL_SIMT    split kernel on the CUDA cores, 64-token pages
+ *                           (128 for the INT4-anchor and anchor-free formats),
  *                           integer dot products for scores and paired fp32
- *                           FMAs for values; every G.
+ *                           FMAs for values; every G and every format.
  *  RQ_DECODE_KERNEL_TENSOR  split kernel on the tensor cores (tcgen05), 128-token
  *                           pages: bf16 and int8 MMAs for the scores of all G
  *                           query heads of a kv-head at once and for the
- *                           probability-weighted value sums; G in {2, 4, 8}.
+ *                           probability-weighted value sums; G in {1, 2, 4, 8},
+ *                           not for the residual loops of chained policies.
  *  RQ_DECODE_KERNEL_AUTO    the tensor-core kernel for G >= 4 where it has a
  *                           variant, else the CUDA-core kernel (the default). */
 typedef enum {
@@ -230,7 +249,11 @@ RQ_API rq_status rq_decode_workspace_size(const rq_cache* cache, int64_t* bytes_
  * and the output is
  *     ( sum_t p_t alpha_V,t ref_v,t  +  H^T sum_t p_t deq(codes_V,t)
  *       + sum_tail p_j v_tail,j ) / sum p
- * with one inverse rotation per (b, q-head), ref being the loop's anchor.  An
+ * with one inverse rotation per (b, q-head), ref being the loop's anchor.  Under
+ * a chained policy the loop's chain l = c_0 -> c_1 -> ... -> anchor unrolls to
+ *     s_t = softmax_scale * ( beta_n (q . ref_k) + sum_i beta_i (H q) . deq(codes_K of c_i) )
+ * with beta_0 = 1 and beta_(i+1) = beta_i * alpha_K of c_i per token (alpha_V
+ * likewise for the value sums); it runs on the CUDA-core kernel only.  An
  * anchor loop is plain attention over its bf16 or INT4 planes.  n_tail current tokens (bf16,
  * not yet encoded) join the softmax.  Split-K over pages (64 tokens on the
  * CUDA-core kernel, 128 on the tensor-core kernel) with an online softmax,
@@ -320,7 +343,9 @@ RQ_API rq_status rq_bf16_decode_attention(int32_t batch, int32_t kv_heads, int32
 /* Reconstruction (test support): fp32 K_hat, V_hat of loop `loop` for tokens
  * [t0, t0 + n) of every (b, h), written to k_out/v_out [B][Hkv][n][128]:
  * alpha * ref + H^T deq(codes) for a residual loop, the (dequantised)
- * anchor for an anchor loop. */
+ * anchor for an anchor loop.  Under a chained policy ref is the reconstruction
+ * of the loop's reference, computed in the same buffers from the anchor
+ * outward (one launch per loop of the chain). */
 RQ_API rq_status rq_reconstruct(const rq_cache* cache, int32_t loop, int32_t t0, int32_t n, float* k_out,
                          float* v_out, rq_stream_t stream);
 

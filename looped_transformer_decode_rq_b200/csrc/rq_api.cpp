@@ -81,16 +81,29 @@ rq_status make_plane_map(CUtensorMap* map, const void* base, int B, int H, int64
   return RQ_OK;
 }
 
-// The loop whose anchor planes loop l is stored against (l itself for an anchor).
-int anchor_of(const rq_config& c, int l) {
+bool chained(const rq_config& c) {
+  return c.anchor_policy == RQ_ANCHOR_PREVIOUS || c.anchor_policy == RQ_ANCHOR_NEXT;
+}
+
+// The loop whose (reconstructed) values loop l is stored against (l itself
+// for an anchor).
+int ref_of(const rq_config& c, int l) {
   const int L = c.num_loops;
   if (c.anchor_policy == RQ_ANCHOR_FIRST) return 0;
+  if (c.anchor_policy == RQ_ANCHOR_PREVIOUS) return l > 0 ? l - 1 : 0;
+  if (c.anchor_policy == RQ_ANCHOR_NEXT) return l < L - 1 ? l + 1 : L - 1;
   if (c.anchor_policy == RQ_ANCHOR_INTERVAL && c.anchor_interval >= 2) {
     const int n = c.anchor_interval;
     const int a = (l / n) * n + n - 1;
     return a < L - 1 ? a : L - 1;
   }
   return L - 1;
+}
+
+// The anchor at the end of loop l's reference chain (l itself for an anchor).
+int anchor_of(const rq_config& c, int l) {
+  for (int i = 0; i < RQ_MAX_LOOPS && ref_of(c, l) != l; ++i) l = ref_of(c, l);
+  return l;
 }
 
 rq_status validate_config(const rq_config* c) {
@@ -106,7 +119,7 @@ rq_status validate_config(const rq_config* c) {
     return fail(RQ_ERR_UNSUPPORTED, "q_heads / kv_heads = %d (supported: 1, 2, 4, 8)", G);
   if (c->head_dim != RQ_HEAD_DIM) return fail(RQ_ERR_UNSUPPORTED, "head_dim %d != 128", c->head_dim);
   if (c->capacity < 1) return fail(RQ_ERR_INVALID_ARG, "capacity %d < 1", c->capacity);
-  if (c->anchor_policy < RQ_ANCHOR_LAST || c->anchor_policy > RQ_ANCHOR_INTERVAL)
+  if (c->anchor_policy < RQ_ANCHOR_LAST || c->anchor_policy > RQ_ANCHOR_NEXT)
     return fail(RQ_ERR_INVALID_ARG, "anchor_policy %d", c->anchor_policy);
   if (c->anchor_policy == RQ_ANCHOR_INTERVAL && (c->anchor_interval < 2 || c->anchor_interval > c->num_loops))
     return fail(RQ_ERR_INVALID_ARG, "anchor_interval %d outside [2, num_loops]", c->anchor_interval);
@@ -127,6 +140,25 @@ rq_status validate_config(const rq_config* c) {
       return fail(RQ_ERR_INVALID_ARG, "loop %d rotate %d", l, c->rotate[l]);
     if (c->alpha_mode[l] < RQ_ALPHA_LS || c->alpha_mode[l] > RQ_ALPHA_NORM_RATIO)
       return fail(RQ_ERR_INVALID_ARG, "loop %d alpha_mode %d", l, c->alpha_mode[l]);
+  }
+  if (chained(*c)) {
+    // the decode sums every link's rotated residual in one accumulator, so
+    // the links share one format; the chain is at most RQ_MAX_CHAIN long
+    if (c->num_loops > RQ_MAX_CHAIN + 1)
+      return fail(RQ_ERR_UNSUPPORTED, "chained references with %d loops (at most %d)", c->num_loops,
+                  RQ_MAX_CHAIN + 1);
+    int first = -1;
+    for (int l = 0; l < c->num_loops; ++l) {
+      if (anchor_of(*c, l) == l) continue;
+      if (c->alpha_mode[l] == RQ_ALPHA_ZERO)
+        return fail(RQ_ERR_UNSUPPORTED, "chained references with alpha_mode ZERO (loop %d)", l);
+      if (first < 0) {
+        first = l;
+      } else if (c->bits[l] != c->bits[first] || c->group[l] != c->group[first] || c->rotate[l] != c->rotate[first]) {
+        return fail(RQ_ERR_UNSUPPORTED, "chained references need one residual format (loops %d and %d differ)",
+                    first, l);
+      }
+    }
   }
   return RQ_OK;
 }
@@ -189,10 +221,12 @@ rq_status rq_cache_layout(const rq_config* cfg, rq_layout* out) {
     L.meta_offset[l][0] = L.meta_offset[l][1] = -1;
     L.alpha_offset[l] = -1;
     L.anchor_of[l] = -1;
+    L.ref_of[l] = -1;
   }
   for (int l = 0; l < cfg->num_loops; ++l) {
     const int a = anchor_of(*cfg, l);
     L.anchor_of[l] = a;
+    L.ref_of[l] = ref_of(*cfg, l);
     if (a == l) {
       L.codes_record_bytes[l] = cfg->bits[l] == 16 ? 256 : 64;
       L.meta_record_bytes[l] = cfg->bits[l] == 16 ? 0 : 16;
@@ -312,7 +346,9 @@ rq_status build_encode(rq_cache* cache, const void* k, const void* v, const int6
     p.rotate[l] = c.rotate[l];
     p.alpha_mode[l] = c.alpha_mode[l];
     p.anchor[l] = lay.anchor_of[l];
+    p.ref[l] = lay.ref_of[l];
   }
+  p.chained = chained(c) ? 1 : 0;
   p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
   return RQ_OK;
 }
@@ -395,9 +431,16 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, cons
   const int ref_kind = ref_kind_for(c, loop);
   const int res_bits = loop == a ? 0 : c.bits[loop];
   const int res_group = loop == a ? 32 : c.group[loop];
-  if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G, cache->decode_kernel))
-    return fail(RQ_ERR_UNSUPPORTED, "no %s decode kernel for this loop format and G = %d",
-                cache->decode_kernel == RQ_DECODE_KERNEL_TENSOR ? "tensor-core" : "", G);
+  // the loop's chain of residual links toward its anchor (one link unless chained)
+  int chain[RQ_MAX_CHAIN];
+  int n_chain = 0;
+  for (int l = loop; l != a; l = lay.ref_of[l]) {
+    if (n_chain == RQ_MAX_CHAIN) return fail(RQ_ERR_UNSUPPORTED, "reference chain longer than %d", RQ_MAX_CHAIN);
+    chain[n_chain++] = l;
+  }
+  if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G, cache->decode_kernel, n_chain > 1 ? n_chain : 1))
+    return fail(RQ_ERR_UNSUPPORTED, "no %s decode kernel for this loop format, G = %d and a chain of %d",
+                cache->decode_kernel == RQ_DECODE_KERNEL_TENSOR ? "tensor-core" : "", G, n_chain);
   if (ref_kind == rq::kRefBf16 && !cache->tmaps_ready[a]) {
     const int64_t cp = lay.capacity_padded;
     for (int kv = 0; kv < 2; ++kv) {
@@ -420,12 +463,16 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, cons
       p.ref_meta[kv] = cache->base + lay.meta_offset[a][kv];
     }
   }
+  p.n_chain = 1;
   if (res_bits) {
-    for (int kv = 0; kv < 2; ++kv) {
-      p.res_codes[kv] = cache->base + lay.codes_offset[loop][kv];
-      p.res_meta[kv] = cache->base + lay.meta_offset[loop][kv];
+    p.n_chain = n_chain;
+    for (int i = 0; i < n_chain; ++i) {
+      for (int kv = 0; kv < 2; ++kv) {
+        p.res_codes[i][kv] = cache->base + lay.codes_offset[chain[i]][kv];
+        p.res_meta[i][kv] = cache->base + lay.meta_offset[chain[i]][kv];
+      }
+      p.alpha[i] = cache->base + lay.alpha_offset[chain[i]];
     }
-    p.alpha = cache->base + lay.alpha_offset[loop];
     p.rotate = c.rotate[loop];
   }
   p.q = static_cast<const uint16_t*>(q);
@@ -539,33 +586,42 @@ rq_status rq_reconstruct(const rq_cache* cache, int32_t loop, int32_t t0, int32_
     return fail(RQ_ERR_INVALID_ARG, "outputs null or not 16-byte aligned");
   const rq_layout& lay = cache->lay;
   const int a = lay.anchor_of[loop];
-  rq::ReconstructParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.B = c.batch;
-  p.Hkv = c.kv_heads;
-  p.cap_pad = lay.capacity_padded;
-  p.t0 = t0;
-  p.n = n;
-  p.ref_bits = c.bits[a];
-  for (int kv = 0; kv < 2; ++kv) {
-    p.ref_plane[kv] = cache->base + lay.codes_offset[a][kv];
-    p.ref_meta[kv] = lay.meta_offset[a][kv] >= 0 ? cache->base + lay.meta_offset[a][kv] : nullptr;
-  }
-  p.is_ref = loop == a;
-  if (!p.is_ref) {
+  // links from the anchor outward: the first reads the anchor planes, every
+  // later one the previous link's reconstruction, in place in k_out / v_out
+  int links[RQ_MAX_LOOPS];
+  int n_links = 0;
+  for (int l = loop; l != a && n_links < RQ_MAX_LOOPS; l = lay.ref_of[l]) links[n_links++] = l;
+  for (int i = n_links - 1; i >= (n_links > 0 ? 0 : -1); --i) {
+    const int l = i >= 0 ? links[i] : loop;
+    rq::ReconstructParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = c.batch;
+    p.Hkv = c.kv_heads;
+    p.cap_pad = lay.capacity_padded;
+    p.t0 = t0;
+    p.n = n;
+    p.ref_bits = c.bits[a];
     for (int kv = 0; kv < 2; ++kv) {
-      p.codes[kv] = cache->base + cache->lay.codes_offset[loop][kv];
-      p.meta[kv] = cache->base + cache->lay.meta_offset[loop][kv];
+      p.ref_plane[kv] = cache->base + lay.codes_offset[a][kv];
+      p.ref_meta[kv] = lay.meta_offset[a][kv] >= 0 ? cache->base + lay.meta_offset[a][kv] : nullptr;
     }
-    p.alpha = cache->base + cache->lay.alpha_offset[loop];
-    p.bits = c.bits[loop];
-    p.group = c.group[loop];
-    p.rotate = c.rotate[loop];
+    p.is_ref = l == a;
+    p.ref_from_out = i >= 0 && i < n_links - 1;
+    if (!p.is_ref) {
+      for (int kv = 0; kv < 2; ++kv) {
+        p.codes[kv] = cache->base + lay.codes_offset[l][kv];
+        p.meta[kv] = cache->base + lay.meta_offset[l][kv];
+      }
+      p.alpha = cache->base + lay.alpha_offset[l];
+      p.bits = c.bits[l];
+      p.group = c.group[l];
+      p.rotate = c.rotate[l];
+    }
+    p.out[0] = k_out;
+    p.out[1] = v_out;
+    cudaError_t e = rq::launch_reconstruct(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "reconstruct launch");
   }
-  p.out[0] = k_out;
-  p.out[1] = v_out;
-  cudaError_t e = rq::launch_reconstruct(p, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "reconstruct launch");
   return RQ_OK;
 }
 

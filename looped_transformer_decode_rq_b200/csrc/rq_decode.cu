@@ -37,749 +37,12 @@
 #include <cstring>
 
 #include "rq_common.cuh"
+#include "rq_decode_split.cuh"
 #include "rq_encode_dev.cuh"
 #include "rq_internal.h"
 
 namespace rq {
 namespace {
-
-constexpr int kNCW = 8;        // consumer warps
-constexpr int kGW = 4;         // warps per consumer group
-constexpr int kGT = kGW * 32;  // threads per consumer group
-constexpr int kNCT = kNCW * 32;
-constexpr int kNT = kNCT + 32; // + producer warp
-constexpr int kConsumerBar = 1;  // all consumers (256 threads)
-constexpr int kGroupBar0 = 2;    // group g uses kGroupBar0 + g (128 threads)
-constexpr unsigned kFull = 0xffffffffu;
-
-__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
-
-// 2^x on the special-function unit (inputs are <= 0 here: softmax weights and
-// their rescale factors)
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// max over the warp with one integer reduction on an order-preserving key
-__device__ __forceinline__ float warp_max(float v) {
-  int i = __float_as_int(v);
-  i ^= (i >> 31) & 0x7fffffff;
-  i = __reduce_max_sync(kFull, i);
-  i ^= (i >> 31) & 0x7fffffff;
-  return __int_as_float(i);
-}
-
-template <int REF, int RB, int RG, int G, int TT>
-struct Cfg {
-  static constexpr int PAGE = TT;  // tokens per page / stage
-  // phase 1 (scores): 4G lanes per token, D1 = 32/G dims per lane
-  static constexpr int TPT = 4 * G;
-  static constexpr int D1 = 32 / G;
-  static constexpr int EB = D1 >= 8 ? 8 : D1;   // elements per accumulation block
-  static constexpr int NB = D1 / EB;
-  static constexpr int TOK_PASS = kGT / TPT;    // tokens per pass of a group
-  static constexpr int PASSES = TT / TOK_PASS;
-  // phase 2 (values)
-  static constexpr int D2 = (G >= 4) ? 4 : 8;   // dims per lane
-  static constexpr int TPR2 = kD / D2;          // lanes per token row
-  static constexpr int SLICES = kGT / TPR2;
-  static constexpr int TOK2 = TT / SLICES;     // tokens per lane per page
-  // per-record bytes
-  static constexpr int REF_REC = REF == kRefBf16 ? 256 : (REF == kRefInt4 ? 64 : 0);
-  static constexpr int REFM_REC = REF == kRefInt4 ? 16 : 0;
-  static constexpr int CB = RB * 16;
-  static constexpr int MB = RB ? 4 * (kD / RG) : 0;
-  static constexpr bool HAS_ALPHA = (REF != kRefNone) && (RB != 0);
-  static constexpr int AL_REC = HAS_ALPHA ? 4 : 0;
-  // stage layout (each piece 1024-byte aligned)
-  static constexpr int al(int x) { return (x + 1023) & ~1023; }
-  static constexpr int O_REFK = 0;
-  static constexpr int O_REFV = O_REFK + al(TT * REF_REC);
-  static constexpr int O_REFMK = O_REFV + al(TT * REF_REC);
-  static constexpr int O_REFMV = O_REFMK + al(TT * REFM_REC);
-  static constexpr int O_RESK = O_REFMV + al(TT * REFM_REC);
-  static constexpr int O_RESV = O_RESK + al(TT * CB);
-  static constexpr int O_RESMK = O_RESV + al(TT * CB);
-  static constexpr int O_RESMV = O_RESMK + al(TT * MB);
-  static constexpr int O_AL = O_RESMV + al(TT * MB);
-  static constexpr int STAGE_BYTES = O_AL + al(TT * AL_REC);
-  static constexpr int TX_BYTES = TT * (2 * REF_REC + 2 * REFM_REC + 2 * CB + 2 * MB + AL_REC);
-  // non-stage shared memory
-  static constexpr int O_S = 0;                           // scores [2 groups][2 parity][G][TT]
-  static constexpr int O_WM = O_S + 4 * 4 * G * TT;      // warp maxima [2][2][G][kGW]
-  static constexpr int O_ACC = O_WM + 4 * 4 * G * kGW;    // [G][256]
-  static constexpr int O_L = O_ACC + 4 * G * 2 * kD;      // [G] (padded to 8)
-  static constexpr int O_MG = O_L + 4 * 8;                // [2][G] (padded to 16)
-  static constexpr int O_QS = O_MG + 4 * 16;              // [G][128]
-  static constexpr int O_QT = O_QS + 4 * G * kD;          // [G][128]
-  static constexpr int O_PRE = O_QT + 4 * G * kD;         // [RQ_MAX_BATCH + 1]
-  static constexpr int O_NT = O_PRE + 4 * (RQ_MAX_BATCH + 1);
-  static constexpr int O_MISC = O_NT + 4 * RQ_MAX_BATCH;  // abort flag
-  static constexpr int O_BAR = (O_MISC + 16 + 7) & ~7;
-  static constexpr int MISC_BYTES = O_BAR + 16 * 8;
-  static constexpr int kSmemLimit = 227 * 1024;
-  static constexpr int STAGES_MAX = (kSmemLimit - 1024 - MISC_BYTES) / STAGE_BYTES;
-  // an even number of stages keeps each stage with one group
-  static constexpr int STAGES = STAGES_MAX >= 4 ? 4 : 2;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
-  static_assert(STAGES_MAX >= 2, "stage ring does not fit in shared memory");
-  static_assert(PASSES * TOK_PASS == TT && TOK2 * SLICES == TT, "lane mapping");
-  static_assert((O_ACC % 16) == 0 && (O_QS % 16) == 0 && (O_WM % 16) == 0, "alignment");
-};
-
-// ---------------------------------------------------------------------------
-// code unpacking helpers
-// ---------------------------------------------------------------------------
-// Load `NB` bytes (1, 2, 4, 8 or 16) of packed codes into 32-bit words.
-template <int NB>
-__device__ __forceinline__ void load_codes(const uint8_t* p, uint32_t (&w)[(NB + 3) / 4]) {
-  if constexpr (NB == 16) {
-    const uint4 v = *reinterpret_cast<const uint4*>(p);
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-  } else if constexpr (NB == 8) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);
-    w[0] = v.x; w[1] = v.y;
-  } else if constexpr (NB == 4) {
-    w[0] = *reinterpret_cast<const uint32_t*>(p);
-  } else if constexpr (NB == 2) {
-    w[0] = *reinterpret_cast<const uint16_t*>(p);
-  } else {
-    w[0] = *p;
-  }
-}
-
-// code e of a thread's unit (bits per code BITS) as 1 + c*2^(p_e - 23)
-template <int BITS>
-__device__ __forceinline__ float code_f(const uint32_t* w, int e) {
-  const int bit = e * BITS;
-  const uint32_t word = w[bit >> 5];
-  const int b32 = bit & 31;
-  const uint32_t src = (b32 >= 16) ? (word >> 16) : word;
-  const int p = b32 & 15;
-  return code_float(src, ((1u << BITS) - 1u) << p);
-}
-
-template <int BITS>
-__device__ __forceinline__ int code_pos(int e) { return (e * BITS) & 15; }
-
-__device__ __forceinline__ float2 f2sub1(float2 f) { return __fadd2_rn(f, make_float2(-1.f, -1.f)); }
-
-// Integer-dot-product operands for a lane's D query values against BITS-bit
-// packed codes.  The values are quantised to int16 with one scale per lane
-// (|q| <= 32767 * scale) and split into a signed high byte and an unsigned low
-// byte, so that  sum_e q_e c_e = scale * (256 * dp4a(c, hi) + dp4a(c, lo))
-// exactly in 32-bit integers.  Byte b of operand [w][k] pairs with the code
-// that the unpacking of word w puts into byte b at step k:
-//   BITS = 2: (w >> 2k) & 0x03030303 holds elements 16w + 4b + k   (k < 4)
-//   BITS = 4: (w >> 4k) & 0x0F0F0F0F holds elements  8w + 2b + k   (k < 2)
-template <int BITS, int D>
-struct DotOperands {
-  static constexpr int NW = (D * BITS + 31) / 32;
-  static constexpr int KPW = BITS == 2 ? 4 : 2;
-  uint32_t hi[NW][KPW];
-  uint32_t lo[NW][KPW];
-  float scale;
-
-  __device__ __forceinline__ void build(const float* v) {
-    float m = 0.f;
-#pragma unroll
-    for (int e = 0; e < D; ++e) m = fmaxf(m, fabsf(v[e]));
-    scale = m * (1.f / 32767.f);
-    const float inv = m > 0.f ? 32767.f / m : 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w)
-#pragma unroll
-      for (int k = 0; k < KPW; ++k) hi[w][k] = lo[w][k] = 0u;
-#pragma unroll
-    for (int e = 0; e < D; ++e) {
-      int qi = __float2int_rn(v[e] * inv);
-      qi = max(-32767, min(32767, qi));
-      const int per = 32 / BITS, w = e / per, in = e % per;
-      const int b = BITS == 2 ? in / 4 : in / 2, k = BITS == 2 ? in % 4 : in % 2;
-      hi[w][k] |= (static_cast<uint32_t>(qi >> 8) & 0xFFu) << (8 * b);
-      lo[w][k] |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * b);
-    }
-  }
-};
-
-template <int BITS>
-__device__ __forceinline__ uint32_t unpack_bytes(uint32_t w, int k) {
-  return BITS == 2 ? ((w >> (2 * k)) & 0x03030303u) : ((w >> (4 * k)) & 0x0F0F0F0Fu);
-}
-
-// ---------------------------------------------------------------------------
-// split kernel
-// ---------------------------------------------------------------------------
-template <int REF, int RB, int RG, int G, int TT>
-__device__ __forceinline__ void issue_page(const DecodeParams& P, const CUtensorMap* tmK, const CUtensorMap* tmV,
-                                           uint8_t* st, uint32_t full, const PageIter& it, int Hkv) {
-  using C = Cfg<REF, RB, RG, G, TT>;
-  const int t0 = it.page * TT;
-  // byte planes hold plane_tokens (a multiple of 64) records per (b, h): a
-  // 128-token page may find only 64 of them at the plane's end
-  const int nrec = (TT > kPage && P.plane_tokens > 0 && t0 + TT > P.plane_tokens)
-                       ? static_cast<int>(P.plane_tokens - t0) : TT;
-  mbar_arrive_expect_tx(full, REF == kRefBf16 ? C::TX_BYTES : static_cast<uint32_t>(nrec) * (C::TX_BYTES / TT));
-  const int64_t rec0 = static_cast<int64_t>(it.b * Hkv + it.h) * P.plane_tokens + t0;
-  if constexpr (REF == kRefBf16) {
-    static_assert(TT == kPage, "bf16 anchor pages are one 64-token tile");
-    tma_load_4d(smem_u32(st + C::O_REFK), tmK, 0, t0, it.h, it.b, full);
-    tma_load_4d(smem_u32(st + C::O_REFK + TT * 128), tmK, 64, t0, it.h, it.b, full);
-    tma_load_4d(smem_u32(st + C::O_REFV), tmV, 0, t0, it.h, it.b, full);
-    tma_load_4d(smem_u32(st + C::O_REFV + TT * 128), tmV, 64, t0, it.h, it.b, full);
-  } else if constexpr (REF == kRefInt4) {
-    bulk_g2s(smem_u32(st + C::O_REFK), P.ref_codes[0] + rec0 * 64, nrec * 64, full);
-    bulk_g2s(smem_u32(st + C::O_REFV), P.ref_codes[1] + rec0 * 64, nrec * 64, full);
-    bulk_g2s(smem_u32(st + C::O_REFMK), P.ref_meta[0] + rec0 * 16, nrec * 16, full);
-    bulk_g2s(smem_u32(st + C::O_REFMV), P.ref_meta[1] + rec0 * 16, nrec * 16, full);
-  }
-  if constexpr (RB != 0) {
-    bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0] + rec0 * C::CB, nrec * C::CB, full);
-    bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[1] + rec0 * C::CB, nrec * C::CB, full);
-    bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0] + rec0 * C::MB, nrec * C::MB, full);
-    bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[1] + rec0 * C::MB, nrec * C::MB, full);
-  }
-  if constexpr (C::HAS_ALPHA) bulk_g2s(smem_u32(st + C::O_AL), P.alpha + rec0 * 4, nrec * 4, full);
-}
-
-template <int REF, int RB, int RG, int G, int TT>
-__global__ void __launch_bounds__(kNT, 1)
-    decode_split_kernel(const __grid_constant__ DecodeParams P,
-                        const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV) {
-  using C = Cfg<REF, RB, RG, G, TT>;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  // align by offsetting the shared array itself so that every access below
-  // stays a shared-memory access
-  uint8_t* base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* stages = base;
-  uint8_t* misc = base + C::STAGES * C::STAGE_BYTES;
-  float* sS = reinterpret_cast<float*>(misc + C::O_S);
-  float* sWM = reinterpret_cast<float*>(misc + C::O_WM);
-  float* sACC = reinterpret_cast<float*>(misc + C::O_ACC);
-  float* sL = reinterpret_cast<float*>(misc + C::O_L);
-  float* sMG = reinterpret_cast<float*>(misc + C::O_MG);
-  float* sQS = reinterpret_cast<float*>(misc + C::O_QS);
-  float* sQT = reinterpret_cast<float*>(misc + C::O_QT);
-  int* sPre = reinterpret_cast<int*>(misc + C::O_PRE);
-  int* sNt = reinterpret_cast<int*>(misc + C::O_NT);
-  volatile int* sAbort = reinterpret_cast<volatile int*>(misc + C::O_MISC);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + C::O_BAR);
-
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int B = P.B, Hkv = P.Hkv;
-
-  // ---- page counts and their prefix over sequences
-  for (int b = tid; b < B; b += kNT) {
-    int len = P.ctx_len[b];
-    if (len < 0 || len > P.capacity) {
-      if (blockIdx.x == 0) set_flag(P.status, RQ_FLAG_CTX_LEN);
-      len = len < 0 ? 0 : P.capacity;
-    }
-    sNt[b] = (len + TT - 1) / TT;
-  }
-  for (int i = tid; i < G * 2 * kD; i += kNT) sACC[i] = 0.f;
-  if (tid < 8) sL[tid] = 0.f;
-  if (tid == 0) *sAbort = 0;
-  __syncthreads();
-  if (warp == 0) {
-    int carry = 0;
-    for (int b0 = 0; b0 < B; b0 += 32) {
-      const int b = b0 + lane;
-      const int v = b < B ? sNt[b] : 0;
-      int x = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, x, o);
-        if (lane >= o) x += y;
-      }
-      if (b < B) sPre[b] = carry + x - v;
-      carry += __shfl_sync(kFull, x, 31);
-    }
-    if (lane == 0) sPre[B] = carry;
-  }
-  if (tid == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(smem_u32(&bars[s]), 1);               // full: the producer's expect_tx
-      mbar_init(smem_u32(&bars[C::STAGES + s]), kGW);  // empty: the 4 warps of the page's group
-    }
-    mbar_init(smem_u32(&bars[15]), 1);  // never arrived at: the wait of the stall test hook
-    fence_barrier_init();
-  }
-  __syncthreads();
-
-  const int64_t total = static_cast<int64_t>(sPre[B]) * Hkv;
-  const int64_t P_eff = total < P.num_ctas ? total : P.num_ctas;
-  if (static_cast<int64_t>(blockIdx.x) >= P_eff) return;
-  const int64_t x0 = static_cast<int64_t>(blockIdx.x) * total / P_eff;
-  const int64_t x1 = static_cast<int64_t>(blockIdx.x + 1) * total / P_eff;
-  const int n_pages = static_cast<int>(x1 - x0);
-
-  // ========================= producer warp =========================
-  if (warp == kNCW) {
-    if (lane == 0) {
-      if constexpr (REF == kRefBf16) {
-        prefetch_tensormap(&tmK);
-        prefetch_tensormap(&tmV);
-      }
-      PageIter it;
-      it.seek(x0, sPre, sNt, B, Hkv);
-      int k = 0;
-      for (; k < n_pages; ++k) {
-        const int s = k % C::STAGES;
-        if (!mbar_wait_bounded(smem_u32(&bars[C::STAGES + s]), ((k / C::STAGES) & 1) ^ 1)) {
-          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-          *sAbort = 1;
-          break;
-        }
-        if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[15]), 0)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-        if (*sAbort) break;
-        issue_page<REF, RB, RG, G, TT>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it, Hkv);
-        it.next(sNt, B, Hkv);
-      }
-      // Drain: no copy this CTA issued may still be landing when it exits.
-      for (int kk = (k > C::STAGES ? k - C::STAGES : 0); kk < k; ++kk) {
-        if (!mbar_wait_bounded(smem_u32(&bars[kk % C::STAGES]), (kk / C::STAGES) & 1)) {
-          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-          break;
-        }
-      }
-    }
-    return;
-  }
-
-  // ========================= consumer groups =========================
-  const int grp = warp / kGW;        // pages k with k % 2 == grp
-  const int gw = warp % kGW;         // warp within the group
-  const int gtid = tid % kGT;        // thread within the group
-  // phase-1 mapping: token within a pass and dim slice.  For G <= 2 the lanes
-  // of one shared-memory phase read rows whose swizzle phases differ, so the
-  // 16-byte loads of the bf16 reference never share a bank.
-  int tok1, j1;
-  if constexpr (G <= 2) {
-    const int jj = lane & (2 * G - 1);
-    const int tsub = (lane >> (G == 1 ? 1 : 2)) & ((4 / G) - 1);
-    const int box = (lane >> 3) & 1;
-    const int thi = lane >> 4;
-    tok1 = gw * (8 / G) + thi * (4 / G) + tsub;
-    j1 = box * (2 * G) + jj;
-  } else {
-    tok1 = gw * (8 / G) + lane / C::TPT;
-    j1 = lane % C::TPT;
-  }
-  const int d1 = C::D1 * j1;
-  const int slice = gtid / C::TPR2;  // phase-2 mapping
-  const int j2 = gtid % C::TPR2;
-  const int d2 = C::D2 * j2;
-  float* gS = sS + grp * 2 * G * TT;
-  float* gWM = sWM + grp * 2 * G * kGW;
-
-  PageIter it;
-  it.seek(x0, sPre, sNt, B, Hkv);
-  int k = 0;
-  while (k < n_pages) {
-    const int b = it.b, h = it.h;
-    const int seg_pages = min(sNt[b] - it.page, n_pages - k);
-    int len_b = P.ctx_len[b];
-    len_b = len_b < 0 ? 0 : (len_b > P.capacity ? P.capacity : len_b);
-
-    // ---- segment set-up: the G queries of (b, h) and their rotation
-    if (warp < G) {
-      const int qh = h * G + warp;
-      const uint2 raw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hkv * G + qh) * kD + 4 * lane);
-      const float2 a01 = bf16x2_to_f2(raw.x), a23 = bf16x2_to_f2(raw.y);
-      float x[4] = {a01.x, a01.y, a23.x, a23.y};
-      *reinterpret_cast<float4*>(&sQS[warp * kD + 4 * lane]) = make_float4(x[0], x[1], x[2], x[3]);
-      if (RB != 0 && P.rotate) {
-        const float t0 = x[0] + x[1], t1 = x[0] - x[1], t2 = x[2] + x[3], t3 = x[2] - x[3];
-        x[0] = t0 + t2; x[2] = t0 - t2; x[1] = t1 + t3; x[3] = t1 - t3;
-#pragma unroll
-        for (int m = 1; m < 32; m <<= 1) {
-          const bool up = (lane & m) != 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float o = __shfl_xor_sync(kFull, x[e], m);
-            x[e] = up ? (o - x[e]) : (x[e] + o);
-          }
-        }
-        const float c = 0.08838834764831845f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] *= c;
-      }
-      *reinterpret_cast<float4*>(&sQT[warp * kD + 4 * lane]) = make_float4(x[0], x[1], x[2], x[3]);
-    }
-    named_bar_sync(kConsumerBar, kNCT);
-
-    // phase-1 registers: the bf16 reference side keeps the query slice in
-    // fp32; code planes (INT4 anchor, residual) get int16 dp4a operands
-    constexpr int NG1 = RB ? ((C::D1 >= RG) ? C::D1 / RG : 1) : 1;
-    float2 qref[G][REF == kRefBf16 ? C::D1 / 2 : 1];
-    DotOperands<4, REF == kRefInt4 ? C::D1 : 1> oref[G];
-    DotOperands<RB ? RB : 2, RB ? C::D1 : 1> ores[G];
-    float qsum_res[G][NG1];
-    float qsum_ref[G];
-#pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
-      float vr[C::D1], vt[C::D1];
-      qsum_ref[gi] = 0.f;
-#pragma unroll
-      for (int n = 0; n < NG1; ++n) qsum_res[gi][n] = 0.f;
-#pragma unroll
-      for (int e = 0; e < C::D1; ++e) {
-        vr[e] = sQS[gi * kD + d1 + e];
-        vt[e] = RB ? sQT[gi * kD + d1 + e] : 0.f;
-        qsum_ref[gi] += vr[e];
-        qsum_res[gi][(C::D1 >= RG) ? e / RG : 0] += vt[e];
-      }
-      if constexpr (REF == kRefBf16) {
-#pragma unroll
-        for (int e = 0; e < C::D1; e += 2) qref[gi][e / 2] = make_float2(vr[e], vr[e + 1]);
-      } else {
-        qref[gi][0] = make_float2(0.f, 0.f);
-      }
-      if constexpr (REF == kRefInt4) oref[gi].build(vr);
-      if constexpr (RB != 0) ores[gi].build(vt);
-    }
-
-    // group-local running softmax state and per-lane accumulators
-    float m_run[G], l_thr[G];
-    float2 acc_ref[G][C::D2 / 2], acc_res[G][C::D2 / 2];
-    float z_ref[G], z_res[G];
-#pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
-      m_run[gi] = -INFINITY;
-      l_thr[gi] = 0.f;
-      z_ref[gi] = 0.f;
-      z_res[gi] = 0.f;
-#pragma unroll
-      for (int e = 0; e < C::D2 / 2; ++e) acc_ref[gi][e] = acc_res[gi][e] = make_float2(0.f, 0.f);
-    }
-
-    for (int sp = 0; sp < seg_pages; ++sp, ++k) {
-      if ((k & 1) != grp) {  // the other group's page
-        it.next(sNt, B, Hkv);
-        continue;
-      }
-      const int s = k % C::STAGES;
-      const uint8_t* st = stages + s * C::STAGE_BYTES;
-      if (!*sAbort) {
-        if (!mbar_wait_bounded(smem_u32(&bars[s]), (k / C::STAGES) & 1)) {
-          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-          *sAbort = 1;
-        }
-      }
-      const int n_valid = min(TT, len_b - it.page * TT);
-      const int par = (k >> 1) & 1;
-      float* pS = gS + par * G * TT;
-      float* pWM = gWM + par * G * kGW;
-
-      // ---------------- phase 1: scores of the page's 64 tokens
-      float wmax[G];
-#pragma unroll
-      for (int gi = 0; gi < G; ++gi) wmax[gi] = -INFINITY;
-#pragma unroll
-      for (int ps = 0; ps < C::PASSES; ++ps) {
-        const int t = ps * C::TOK_PASS + tok1;
-        float part[G];
-#pragma unroll
-        for (int gi = 0; gi < G; ++gi) part[gi] = 0.f;
-        if constexpr (REF == kRefBf16) {
-          float2 acc2[G][C::NB];
-#pragma unroll
-          for (int gi = 0; gi < G; ++gi)
-#pragma unroll
-            for (int c = 0; c < C::NB; ++c) acc2[gi][c] = make_float2(0.f, 0.f);
-          const uint8_t* rowK = st + C::O_REFK + (d1 >> 6) * (TT * 128) + t * 128;
-          if constexpr (C::D1 >= 8) {
-#pragma unroll
-            for (int c = 0; c < C::NB; ++c) {
-              const int chunk = ((d1 & 63) >> 3) + c;
-              const uint4 v = *reinterpret_cast<const uint4*>(rowK + ((chunk ^ (t & 7)) << 4));
-              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const float2 kv2 = bf16x2_to_f2(w4[u]);
-#pragma unroll
-                for (int gi = 0; gi < G; ++gi) acc2[gi][c] = __ffma2_rn(qref[gi][c * 4 + u], kv2, acc2[gi][c]);
-              }
-            }
-          } else {
-            const int chunk = (d1 & 63) >> 3;
-            const uint2 v = *reinterpret_cast<const uint2*>(rowK + ((chunk ^ (t & 7)) << 4) + ((d1 & 7) << 1));
-            const float2 k01 = bf16x2_to_f2(v.x), k23 = bf16x2_to_f2(v.y);
-#pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-              acc2[gi][0] = __ffma2_rn(qref[gi][0], k01, acc2[gi][0]);
-              acc2[gi][0] = __ffma2_rn(qref[gi][1], k23, acc2[gi][0]);
-            }
-          }
-#pragma unroll
-          for (int gi = 0; gi < G; ++gi) {
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < C::NB; ++c) sum += acc2[gi][c].x + acc2[gi][c].y;
-            part[gi] = sum;
-          }
-        } else if constexpr (REF == kRefInt4) {
-          using Ops = DotOperands<4, C::D1>;
-          uint32_t cw[Ops::NW];
-          load_codes<C::D1 / 2>(st + C::O_REFK + t * 64 + (d1 >> 1), cw);
-          const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMK + t * 16 + 4 * (d1 >> 5)));
-          int dhi[G];
-          unsigned dlo[G];
-#pragma unroll
-          for (int gi = 0; gi < G; ++gi) { dhi[gi] = 0; dlo[gi] = 0u; }
-#pragma unroll
-          for (int w = 0; w < Ops::NW; ++w)
-#pragma unroll
-            for (int kk = 0; kk < Ops::KPW; ++kk) {
-              const uint32_t x = unpack_bytes<4>(cw[w], kk);
-#pragma unroll
-              for (int gi = 0; gi < G; ++gi) {
-                dhi[gi] = __dp4a(static_cast<int>(x), static_cast<int>(oref[gi].hi[w][kk]), dhi[gi]);
-                dlo[gi] = __dp4a(x, oref[gi].lo[w][kk], dlo[gi]);
-              }
-            }
-#pragma unroll
-          for (int gi = 0; gi < G; ++gi) {
-            const float dot = static_cast<float>(dhi[gi] * 256 + static_cast<int>(dlo[gi])) * oref[gi].scale;
-            part[gi] = fmaf(sz.x, dot, sz.y * qsum_ref[gi]);
-          }
-        }
-        if constexpr (C::HAS_ALPHA) {
-          const float aK = __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4));
-#pragma unroll
-          for (int gi = 0; gi < G; ++gi) part[gi] *= aK;
-        }
-        if constexpr (RB != 0) {
-          using Ops = DotOperands<RB, C::D1>;
-          constexpr int NBYTES = C::D1 * RB / 8;
-          constexpr int WPG = (RG * RB) / 32;  // 32-bit code words per group
-          uint32_t cw[Ops::NW];
-          load_codes<NBYTES>(st + C::O_RESK + t * C::CB + (d1 * RB >> 3), cw);
-          int dhi[G][NG1];
-          unsigned dlo[G][NG1];
-#pragma unroll
-          for (int gi = 0; gi < G; ++gi)
-#pragma unroll
-            for (int n = 0; n < NG1; ++n) { dhi[gi][n] = 0; dlo[gi][n] = 0u; }
-#pragma unroll
-          for (int w = 0; w < Ops::NW; ++w) {
-            const int n = (NG1 > 1) ? w / WPG : 0;
-#pragma unroll
-            for (int kk = 0; kk < Ops::KPW; ++kk) {
-              const uint32_t x = unpack_bytes<RB>(cw[w], kk);
-#pragma unroll
-              for (int gi = 0; gi < G; ++gi) {
-                dhi[gi][n] = __dp4a(static_cast<int>(x), static_cast<int>(ores[gi].hi[w][kk]), dhi[gi][n]);
-                dlo[gi][n] = __dp4a(x, ores[gi].lo[w][kk], dlo[gi][n]);
-              }
-            }
-          }
-#pragma unroll
-          for (int n = 0; n < NG1; ++n) {
-            const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(
-                st + C::O_RESMK + t * C::MB + 4 * (d1 / RG + n)));
-#pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-              const float dot = static_cast<float>(dhi[gi][n] * 256 + static_cast<int>(dlo[gi][n])) * ores[gi].scale;
-              part[gi] += fmaf(sz.x, dot, sz.y * qsum_res[gi][n]);
-            }
-          }
-        }
-        // reduce over the TPT lanes of this token
-#pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
-          float v = part[gi];
-          if constexpr (G <= 2) {
-#pragma unroll
-            for (int o = 1; o < 2 * G; o <<= 1) v += __shfl_xor_sync(kFull, v, o);
-            v += __shfl_xor_sync(kFull, v, 8);
-          } else {
-#pragma unroll
-            for (int o = 1; o < C::TPT; o <<= 1) v += __shfl_xor_sync(kFull, v, o);
-          }
-          const float sc = (t < n_valid) ? v * P.scale_log2 : -INFINITY;
-          wmax[gi] = fmaxf(wmax[gi], sc);
-          if (j1 == 0) pS[gi * TT + t] = sc;
-        }
-      }
-#pragma unroll
-      for (int gi = 0; gi < G; ++gi) {
-        const float v = warp_max(wmax[gi]);
-        if (lane == 0) pWM[gi * kGW + gw] = v;
-      }
-      named_bar_sync(kGroupBar0 + grp, kGT);
-
-      // ---------------- softmax bookkeeping (group-uniform values)
-      float corr[G];
-#pragma unroll
-      for (int gi = 0; gi < G; ++gi) {
-        const float4 a = *reinterpret_cast<const float4*>(&pWM[gi * kGW]);
-        const float mt = fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w));
-        const float mn = fmaxf(m_run[gi], mt);
-        corr[gi] = fast_exp2(m_run[gi] - mn);
-        m_run[gi] = mn;
-        l_thr[gi] *= corr[gi];
-        const float2 c2 = make_float2(corr[gi], corr[gi]);
-#pragma unroll
-        for (int e = 0; e < C::D2 / 2; ++e) {
-          acc_ref[gi][e] = __fmul2_rn(acc_ref[gi][e], c2);
-          acc_res[gi][e] = __fmul2_rn(acc_res[gi][e], c2);
-        }
-        z_ref[gi] *= corr[gi];
-        z_res[gi] *= corr[gi];
-      }
-
-      // ---------------- phase 2: values (weights recomputed per lane)
-      auto value_token = [&](int t) {
-        float pp[G], pa[G];
-        float aV = 1.f;
-        if constexpr (C::HAS_ALPHA) aV = __half2float(*reinterpret_cast<const __half*>(st + C::O_AL + t * 4 + 2));
-#pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
-          pp[gi] = fast_exp2(pS[gi * TT + t] - m_run[gi]);
-          pa[gi] = pp[gi] * aV;
-          if (j2 == 0) l_thr[gi] += pp[gi];
-        }
-        if constexpr (REF == kRefBf16) {
-          const uint8_t* rowV = st + C::O_REFV + (d2 >> 6) * (TT * 128) + t * 128;
-          const int chunk = (d2 & 63) >> 3;
-          if constexpr (C::D2 == 8) {
-            const uint4 v = *reinterpret_cast<const uint4*>(rowV + ((chunk ^ (t & 7)) << 4));
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 vv = bf16x2_to_f2(w4[u]);
-#pragma unroll
-              for (int gi = 0; gi < G; ++gi) acc_ref[gi][u] = __ffma2_rn(make_float2(pa[gi], pa[gi]), vv, acc_ref[gi][u]);
-            }
-          } else {
-            const uint2 v = *reinterpret_cast<const uint2*>(rowV + ((chunk ^ (t & 7)) << 4) + ((d2 & 7) << 1));
-            const float2 v01 = bf16x2_to_f2(v.x), v23 = bf16x2_to_f2(v.y);
-#pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-              acc_ref[gi][0] = __ffma2_rn(make_float2(pa[gi], pa[gi]), v01, acc_ref[gi][0]);
-              acc_ref[gi][1] = __ffma2_rn(make_float2(pa[gi], pa[gi]), v23, acc_ref[gi][1]);
-            }
-          }
-        } else if constexpr (REF == kRefInt4) {
-          uint32_t cw[1];
-          load_codes<C::D2 / 2>(st + C::O_REFV + t * 64 + (d2 >> 1), cw);
-          const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMV + t * 16 + 4 * (d2 >> 5)));
-#pragma unroll
-          for (int e = 0; e < C::D2; e += 2) {
-            const float2 f = f2sub1(make_float2(code_f<4>(cw, e), code_f<4>(cw, e + 1)));
-#pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-              const float w = pa[gi] * sz.x;
-              acc_ref[gi][e / 2] = __ffma2_rn(make_float2(w, w), f, acc_ref[gi][e / 2]);
-            }
-          }
-#pragma unroll
-          for (int gi = 0; gi < G; ++gi) z_ref[gi] = fmaf(pa[gi], sz.y, z_ref[gi]);
-        }
-        if constexpr (RB != 0) {
-          uint32_t cw[1];
-          load_codes<C::D2 * RB / 8>(st + C::O_RESV + t * C::CB + (d2 * RB >> 3), cw);
-          const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_RESMV + t * C::MB + 4 * (d2 / RG)));
-#pragma unroll
-          for (int e = 0; e < C::D2; e += 2) {
-            const float2 f = f2sub1(make_float2(code_f<RB>(cw, e), code_f<RB>(cw, e + 1)));
-#pragma unroll
-            for (int gi = 0; gi < G; ++gi) {
-              const float w = pp[gi] * sz.x;
-              acc_res[gi][e / 2] = __ffma2_rn(make_float2(w, w), f, acc_res[gi][e / 2]);
-            }
-          }
-#pragma unroll
-          for (int gi = 0; gi < G; ++gi) z_res[gi] = fmaf(pp[gi], sz.y, z_res[gi]);
-        }
-      };
-      if (n_valid == TT) {
-#pragma unroll 4
-        for (int i = 0; i < C::TOK2; ++i) value_token(slice + i * C::SLICES);
-      } else {
-        for (int i = 0; i < C::TOK2; ++i) {
-          const int t = slice + i * C::SLICES;
-          if (t < n_valid) value_token(t);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars[C::STAGES + s]));
-      it.next(sNt, B, Hkv);
-    }
-
-    // ---- flush this (b, h) segment: merge the two groups, write one partial
-    if (gtid == 0) {
-#pragma unroll
-      for (int gi = 0; gi < G; ++gi) sMG[grp * G + gi] = m_run[gi];
-    }
-    named_bar_sync(kConsumerBar, kNCT);
-    // Sum the slices' contributions in a fixed order (warp by warp, and within a
-    // warp its two slices by one shuffle), so that a decode is reproducible bit
-    // for bit from run to run.
-    constexpr int SPW = 32 / C::TPR2;  // token slices per warp (1 or 2)
-    float cref[G][C::D2], cres[G][C::D2], cl[G];
-#pragma unroll
-    for (int gi = 0; gi < G; ++gi) {
-      const float M = fmaxf(sMG[gi], sMG[G + gi]);
-      const float f = (m_run[gi] == -INFINITY) ? 0.f : fast_exp2(m_run[gi] - M);
-#pragma unroll
-      for (int e = 0; e < C::D2; ++e) {
-        const float2 ar = acc_ref[gi][e >> 1];
-        float vr = (e & 1) ? ar.y : ar.x;
-        if constexpr (REF == kRefInt4) vr = fmaf(vr, pow2i(23 - code_pos<4>(e)), z_ref[gi]);
-        cref[gi][e] = __fmul_rn(vr, f);
-        float vs = 0.f;
-        if constexpr (RB != 0) {
-          const float2 as = acc_res[gi][e >> 1];
-          vs = fmaf((e & 1) ? as.y : as.x, pow2i(23 - code_pos<RB>(e)), z_res[gi]);
-        }
-        cres[gi][e] = __fmul_rn(vs, f);
-        if constexpr (SPW == 2) {
-          cref[gi][e] = __fadd_rn(cref[gi][e], __shfl_xor_sync(kFull, cref[gi][e], 16));
-          cres[gi][e] = __fadd_rn(cres[gi][e], __shfl_xor_sync(kFull, cres[gi][e], 16));
-        }
-      }
-      cl[gi] = __fmul_rn(l_thr[gi], f);
-      if constexpr (SPW == 2) cl[gi] = __fadd_rn(cl[gi], __shfl_xor_sync(kFull, cl[gi], 16));
-    }
-    for (int w = 0; w < kNCW; ++w) {
-      if (warp == w && lane < 32 / SPW) {
-#pragma unroll
-        for (int gi = 0; gi < G; ++gi) {
-#pragma unroll
-          for (int e = 0; e < C::D2; ++e) {
-            if constexpr (REF != kRefNone) sACC[gi * 2 * kD + d2 + e] = __fadd_rn(sACC[gi * 2 * kD + d2 + e], cref[gi][e]);
-            if constexpr (RB != 0) sACC[gi * 2 * kD + kD + d2 + e] = __fadd_rn(sACC[gi * 2 * kD + kD + d2 + e], cres[gi][e]);
-          }
-          if (j2 == 0) sL[gi] = __fadd_rn(sL[gi], cl[gi]);
-        }
-      }
-      named_bar_sync(kConsumerBar, kNCT);
-    }
-    {
-      const int pair = b * Hkv + h;
-      float* rec = P.partials + static_cast<int64_t>(pair + blockIdx.x) * G * kPartialFloats;
-      for (int i = tid; i < G * (2 * kD / 4); i += kNCT) {
-        const int gi = i / (2 * kD / 4), f4 = i % (2 * kD / 4);
-        float4* src = reinterpret_cast<float4*>(&sACC[gi * 2 * kD]) + f4;
-        reinterpret_cast<float4*>(rec + gi * kPartialFloats + 4)[f4] = *src;
-        *src = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-      if (tid < G) {
-        const float M = fmaxf(sMG[tid], sMG[G + tid]);
-        reinterpret_cast<float4*>(rec + tid * kPartialFloats)[0] = make_float4(M, sL[tid], 0.f, 0.f);
-        sL[tid] = 0.f;
-      }
-    }
-  }
-}
 
 // ---------------------------------------------------------------------------
 // combine kernel: one warp per (b, q-head)
@@ -885,76 +148,38 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   reinterpret_cast<float4*>(P.out + (static_cast<int64_t>(b) * Hq + qh) * kD)[lane] = o;
 }
 
-// ---------------------------------------------------------------------------
-// dispatch
-// ---------------------------------------------------------------------------
-// Pages of 64 tokens for a bf16 anchor (one tensor-copy tile); 128 for the
-// byte-plane formats, whose 64-token pages are too small to amortise the
-// per-page synchronisation, when four stages still fit.
-template <int REF, int RB, int RG, int G>
-constexpr int page_tokens_of() {
-  if constexpr (REF == kRefBf16) return kPage;
-  else return Cfg<REF, RB, RG, G, 2 * kPage>::STAGES_MAX >= 4 ? 2 * kPage : kPage;
-}
 
-template <int REF, int RB, int RG, int G>
-cudaError_t launch_split(DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv, cudaStream_t s) {
-  constexpr int TT = page_tokens_of<REF, RB, RG, G>();
-  using C = Cfg<REF, RB, RG, G, TT>;
-  auto kern = decode_split_kernel<REF, RB, RG, G, TT>;
-  p.page_tokens = TT;
-  static bool attr_done = false;  // per instantiation; set once per process
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_done = true;
-  }
-  kern<<<p.num_ctas, kNT, C::SMEM_BYTES, s>>>(p, *tk, *tv);
-  return cudaGetLastError();
-}
-
-using SplitFn = cudaError_t (*)(DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);
-
-template <int REF, int RB, int RG>
-SplitFn pick_g(int G) {
-  switch (G) {
-    case 1: return launch_split<REF, RB, RG, 1>;
-    case 2: return launch_split<REF, RB, RG, 2>;
-    case 4: return launch_split<REF, RB, RG, 4>;
-    case 8: return launch_split<REF, RB, RG, 8>;
-    default: return nullptr;
-  }
-}
-
-SplitFn pick(int ref_kind, int res_bits, int res_group, int G) {
+SplitFn pick(int ref_kind, int res_bits, int res_group, int G, int n_chain) {
+  if (n_chain > 1) return pick_chain(ref_kind, res_bits, res_group, G, n_chain);
   if (ref_kind == kRefBf16) {
-    if (res_bits == 0) return pick_g<kRefBf16, 0, 32>(G);
-    if (res_bits == 2) return res_group == 16 ? pick_g<kRefBf16, 2, 16>(G) : pick_g<kRefBf16, 2, 32>(G);
-    if (res_bits == 4) return res_group == 16 ? pick_g<kRefBf16, 4, 16>(G) : pick_g<kRefBf16, 4, 32>(G);
+    if (res_bits == 0) return pick_g<kRefBf16, 0, 32, 1>(G);
+    if (res_bits == 2) return res_group == 16 ? pick_g<kRefBf16, 2, 16, 1>(G) : pick_g<kRefBf16, 2, 32, 1>(G);
+    if (res_bits == 4) return res_group == 16 ? pick_g<kRefBf16, 4, 16, 1>(G) : pick_g<kRefBf16, 4, 32, 1>(G);
   } else if (ref_kind == kRefInt4) {
-    if (res_bits == 0) return pick_g<kRefInt4, 0, 32>(G);
-    if (res_bits == 2) return res_group == 16 ? pick_g<kRefInt4, 2, 16>(G) : pick_g<kRefInt4, 2, 32>(G);
-    if (res_bits == 4) return res_group == 16 ? pick_g<kRefInt4, 4, 16>(G) : pick_g<kRefInt4, 4, 32>(G);
+    if (res_bits == 0) return pick_g<kRefInt4, 0, 32, 1>(G);
+    if (res_bits == 2) return res_group == 16 ? pick_g<kRefInt4, 2, 16, 1>(G) : pick_g<kRefInt4, 2, 32, 1>(G);
+    if (res_bits == 4) return res_group == 16 ? pick_g<kRefInt4, 4, 16, 1>(G) : pick_g<kRefInt4, 4, 32, 1>(G);
   } else if (ref_kind == kRefNone) {
-    if (res_bits == 2) return res_group == 16 ? pick_g<kRefNone, 2, 16>(G) : pick_g<kRefNone, 2, 32>(G);
-    if (res_bits == 4) return res_group == 16 ? pick_g<kRefNone, 4, 16>(G) : pick_g<kRefNone, 4, 32>(G);
+    if (res_bits == 2) return res_group == 16 ? pick_g<kRefNone, 2, 16, 1>(G) : pick_g<kRefNone, 2, 32, 1>(G);
+    if (res_bits == 4) return res_group == 16 ? pick_g<kRefNone, 4, 16, 1>(G) : pick_g<kRefNone, 4, 32, 1>(G);
   }
   return nullptr;
 }
 
 }  // namespace
 
-int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel) {
+int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel, int n_chain) {
   if (kernel == kKernelAuto)
-    return (G >= 4 && tc_variant_supported(ref_kind, res_bits, res_group, G)) ? kKernelTensor : kKernelSimt;
+    return (G >= 4 && n_chain <= 1 && tc_variant_supported(ref_kind, res_bits, res_group, G)) ? kKernelTensor
+                                                                                              : kKernelSimt;
   return kernel;
 }
 
-bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, int kernel) {
+bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, int kernel, int n_chain) {
   if (res_bits != 0 && res_group != 16 && res_group != 32) return false;
-  kernel = decode_kernel_choice(ref_kind, res_bits, res_group, G, kernel);
-  if (kernel == kKernelTensor) return tc_variant_supported(ref_kind, res_bits, res_group, G);
-  if (kernel == kKernelSimt) return pick(ref_kind, res_bits, res_group, G) != nullptr;
+  kernel = decode_kernel_choice(ref_kind, res_bits, res_group, G, kernel, n_chain);
+  if (kernel == kKernelTensor) return n_chain <= 1 && tc_variant_supported(ref_kind, res_bits, res_group, G);
+  if (kernel == kKernelSimt) return pick(ref_kind, res_bits, res_group, G, n_chain) != nullptr;
   return false;
 }
 
@@ -972,13 +197,15 @@ int64_t decode_workspace_bytes(int B, int Hkv, int G, int num_ctas) {
 cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_group, int kernel,
                           const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s,
                           const EncodeParams* append) {
-  kernel = decode_kernel_choice(ref_kind, res_bits, res_group, p.G, kernel);
+  const int n_chain = (res_bits != 0 && p.n_chain > 1) ? p.n_chain : 1;
+  kernel = decode_kernel_choice(ref_kind, res_bits, res_group, p.G, kernel, n_chain);
   cudaError_t e;
   if (kernel == kKernelTensor) {
+    if (n_chain > 1) return cudaErrorInvalidValue;
     p.page_tokens = kTcPage;
     e = launch_split_tc(p, ref_kind, res_bits, res_group, tmap_k, tmap_v, s);
   } else {
-    SplitFn fn = pick(ref_kind, res_bits, res_group, p.G);
+    SplitFn fn = pick(ref_kind, res_bits, res_group, p.G, n_chain);
     if (fn == nullptr) return cudaErrorInvalidValue;
     e = fn(p, tmap_k, tmap_v, s);  // sets p.page_tokens
   }

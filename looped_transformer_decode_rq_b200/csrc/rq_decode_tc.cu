@@ -262,12 +262,12 @@ __device__ __forceinline__ void tc_issue_page(const DecodeParams& P, const CUten
     bulk_g2s(smem_u32(st + C::O_REFMV), P.ref_meta[1] + rec0 * 16, nrec * 16, full);
   }
   if constexpr (RB != 0) {
-    bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0] + rec0 * C::CB, nrec * C::CB, full);
-    bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[1] + rec0 * C::CB, nrec * C::CB, full);
-    bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0] + rec0 * C::MB, nrec * C::MB, full);
-    bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[1] + rec0 * C::MB, nrec * C::MB, full);
+    bulk_g2s(smem_u32(st + C::O_RESK), P.res_codes[0][0] + rec0 * C::CB, nrec * C::CB, full);
+    bulk_g2s(smem_u32(st + C::O_RESV), P.res_codes[0][1] + rec0 * C::CB, nrec * C::CB, full);
+    bulk_g2s(smem_u32(st + C::O_RESMK), P.res_meta[0][0] + rec0 * C::MB, nrec * C::MB, full);
+    bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[0][1] + rec0 * C::MB, nrec * C::MB, full);
   }
-  if constexpr (C::HAS_ALPHA) bulk_g2s(smem_u32(st + C::O_AL), P.alpha + rec0 * 4, nrec * 4, full);
+  if constexpr (C::HAS_ALPHA) bulk_g2s(smem_u32(st + C::O_AL), P.alpha[0] + rec0 * 4, nrec * 4, full);
 }
 
 // ---------------------------------------------------------------------------

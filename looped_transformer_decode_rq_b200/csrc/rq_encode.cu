@@ -37,7 +37,8 @@ __global__ void __launch_bounds__(256) encode_kernel(const EncodeParams P) {
 }
 
 // ---------------------------------------------------------------------------
-// Reconstruction (test support): fp32 alpha*ref + H^T deq(codes)
+// Reconstruction (test support): fp32 alpha*ref + H^T deq(codes); under a
+// chained policy ref is the previous link's reconstruction, already in out[]
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void fwht128_fast(float (&x)[8], int j) {
 #pragma unroll
@@ -88,8 +89,13 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(const ReconstructParam
   const int i = warp % P.n;
   const int bh = warp / P.n;
   const int64_t rec = static_cast<int64_t>(bh) * P.cap_pad + P.t0 + i;
+  float* dst = P.out[kv] + (static_cast<int64_t>(bh) * P.n + i) * kD + 8 * j;
   float ref[8];
-  if (P.ref_bits == 16) {
+  if (P.ref_from_out) {  // the previous link of a chain, reconstructed in place
+    const float4 a = reinterpret_cast<const float4*>(dst)[0], b = reinterpret_cast<const float4*>(dst)[1];
+    ref[0] = a.x; ref[1] = a.y; ref[2] = a.z; ref[3] = a.w;
+    ref[4] = b.x; ref[5] = b.y; ref[6] = b.z; ref[7] = b.w;
+  } else if (P.ref_bits == 16) {
     const uint4 raw = *reinterpret_cast<const uint4*>(P.ref_plane[kv] + rec * 256 + 16 * j);
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
@@ -112,7 +118,6 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(const ReconstructParam
 #pragma unroll
     for (int e = 0; e < 8; ++e) out[e] = fmaf(a, ref[e], out[e]);
   }
-  float* dst = P.out[kv] + (static_cast<int64_t>(bh) * P.n + i) * kD + 8 * j;
   reinterpret_cast<float4*>(dst)[0] = make_float4(out[0], out[1], out[2], out[3]);
   reinterpret_cast<float4*>(dst)[1] = make_float4(out[4], out[5], out[6], out[7]);
 }

@@ -155,56 +155,77 @@ static __device__ __forceinline__ void encode_warp(const EncodeParams& P, int wa
     float refref = 0.f;
     bool have_refref = false;
 
-    for (int l = 0; l < P.L; ++l) {
-      if (l == a || P.anchor[l] != a) continue;
-      float x[8];
-      load8_bf16(X + static_cast<int64_t>(l) * P.s_l + src0, x);
-      bad |= !in_range8(x);
-      float al = 0.f;
-      const int mode = P.alpha_mode[l];
-      if (mode == RQ_ALPHA_LS || mode == RQ_ALPHA_NORM_RATIO) {
-        if (!have_refref) {
-          refref = tree_dot(ref, ref);
-          have_refref = true;
+    // Loops stored against `cur` (the anchor first).  Under a chained policy
+    // exactly one loop takes `cur` as its reference; its binary32
+    // reconstruction then becomes `ref` and the walk moves one link outward.
+    int cur = a;
+    for (int link = 0; link < P.L; ++link) {
+      int next = -1;
+      for (int l = 0; l < P.L; ++l) {
+        if (l == cur || P.ref[l] != cur) continue;
+        float x[8];
+        load8_bf16(X + static_cast<int64_t>(l) * P.s_l + src0, x);
+        bad |= !in_range8(x);
+        float al = 0.f;
+        const int mode = P.alpha_mode[l];
+        if (mode == RQ_ALPHA_LS || mode == RQ_ALPHA_NORM_RATIO) {
+          if (!have_refref) {
+            refref = tree_dot(ref, ref);
+            have_refref = true;
+          }
+          if (mode == RQ_ALPHA_LS) {
+            const float num = tree_dot(x, ref);
+            al = (refref == 0.f) ? 0.f : __fdiv_rn(num, refref);
+          } else {
+            const float xx = tree_dot(x, x);
+            al = (refref == 0.f) ? 0.f : __fdiv_rn(__fsqrt_rn(xx), __fsqrt_rn(refref));
+          }
+        } else if (mode == RQ_ALPHA_ONE) {
+          al = 1.f;
         }
-        if (mode == RQ_ALPHA_LS) {
-          const float num = tree_dot(x, ref);
-          al = (refref == 0.f) ? 0.f : __fdiv_rn(num, refref);
+        const __half a_h = __float2half_rn(al);
+        overflow |= !half_finite(a_h);
+        if (j == 0)
+          *reinterpret_cast<__half*>(P.alpha[l] + rec * 4 + 2 * kv) = a_h;
+        const float af = __half2float(a_h);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], __fmul_rn(af, ref[e]));
+        if (P.rotate[l]) fwht128(x, j);
+        const int bits = P.bits[l], g = P.group[l];
+        uint32_t c[8];
+        __half s_h, z_h;
+        quantize8(x, bits, g >> 3, c, s_h, z_h);
+        overflow |= !(half_finite(s_h) && half_finite(z_h));
+        if (bits == 2) {
+          uint32_t w = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w |= c[e] << (2 * e);
+          *reinterpret_cast<uint16_t*>(P.codes[l][kv] + rec * 32 + 2 * j) = static_cast<uint16_t>(w);
         } else {
-          const float xx = tree_dot(x, x);
-          al = (refref == 0.f) ? 0.f : __fdiv_rn(__fsqrt_rn(xx), __fsqrt_rn(refref));
+          uint32_t w = 0;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w |= c[e] << (4 * e);
+          *reinterpret_cast<uint32_t*>(P.codes[l][kv] + rec * 64 + 4 * j) = w;
         }
-      } else if (mode == RQ_ALPHA_ONE) {
-        al = 1.f;
+        const int lpg = g >> 3;
+        if ((j % lpg) == 0)
+          *reinterpret_cast<uint32_t*>(P.meta[l][kv] + rec * (4 * (kD / g)) + 4 * (j / lpg)) =
+              half2_bits(s_h, z_h);
+        if (P.chained) {  // x_hat = (alpha_hat * ref) + H deq, deq = z_hat + (code * s_hat)
+          const float sf = __half2float(s_h), zf = __half2float(z_h);
+          float u[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) u[e] = __fadd_rn(zf, __fmul_rn(static_cast<float>(c[e]), sf));
+          if (P.rotate[l]) fwht128(u, j);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ref[e] = __fadd_rn(__fmul_rn(af, ref[e]), u[e]);
+          have_refref = false;
+          next = l;
+          break;
+        }
       }
-      const __half a_h = __float2half_rn(al);
-      overflow |= !half_finite(a_h);
-      if (j == 0)
-        *reinterpret_cast<__half*>(P.alpha[l] + rec * 4 + 2 * kv) = a_h;
-      const float af = __half2float(a_h);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], __fmul_rn(af, ref[e]));
-      if (P.rotate[l]) fwht128(x, j);
-      const int bits = P.bits[l], g = P.group[l];
-      uint32_t c[8];
-      __half s_h, z_h;
-      quantize8(x, bits, g >> 3, c, s_h, z_h);
-      overflow |= !(half_finite(s_h) && half_finite(z_h));
-      if (bits == 2) {
-        uint32_t w = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w |= c[e] << (2 * e);
-        *reinterpret_cast<uint16_t*>(P.codes[l][kv] + rec * 32 + 2 * j) = static_cast<uint16_t>(w);
-      } else {
-        uint32_t w = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w |= c[e] << (4 * e);
-        *reinterpret_cast<uint32_t*>(P.codes[l][kv] + rec * 64 + 4 * j) = w;
-      }
-      const int lpg = g >> 3;
-      if ((j % lpg) == 0)
-        *reinterpret_cast<uint32_t*>(P.meta[l][kv] + rec * (4 * (kD / g)) + 4 * (j / lpg)) =
-            half2_bits(s_h, z_h);
+      if (next < 0) break;
+      cur = next;
     }
   }
   const unsigned any_bad = __ballot_sync(kFull, bad);

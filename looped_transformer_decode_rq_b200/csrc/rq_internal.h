@@ -30,6 +30,8 @@ struct EncodeParams {
   uint8_t* alpha[RQ_MAX_LOOPS];
   int bits[RQ_MAX_LOOPS], group[RQ_MAX_LOOPS], rotate[RQ_MAX_LOOPS], alpha_mode[RQ_MAX_LOOPS];
   int anchor[RQ_MAX_LOOPS];
+  int ref[RQ_MAX_LOOPS];  // the loop each loop is stored against (== anchor unless chained)
+  int chained;            // 1: references are reconstructed neighbours (Previous-/Next-loop)
   int32_t* status;
 };
 
@@ -41,6 +43,7 @@ struct ReconstructParams {
   const uint8_t* ref_plane[2];
   const uint8_t* ref_meta[2];
   int is_ref;  // reconstruct the anchor loop itself
+  int ref_from_out;  // take the reference from out[] (a chain's previous link), not the anchor
   const uint8_t* codes[2];
   const uint8_t* meta[2];
   const uint8_t* alpha;
@@ -57,10 +60,12 @@ struct DecodeParams {
   // reference (bf16 via tensor maps; INT4 via byte planes)
   const uint8_t* ref_codes[2];
   const uint8_t* ref_meta[2];
-  // residual
-  const uint8_t* res_codes[2];
-  const uint8_t* res_meta[2];
-  const uint8_t* alpha;  // (alpha_K, alpha_V) fp16 pairs, or null (alpha = 1)
+  // residual: the loop's chain c_0 = loop, c_1 = its reference, ... (n_chain
+  // links, 1 unless the policy is chained), all in one format
+  const uint8_t* res_codes[RQ_MAX_CHAIN][2];
+  const uint8_t* res_meta[RQ_MAX_CHAIN][2];
+  const uint8_t* alpha[RQ_MAX_CHAIN];  // (alpha_K, alpha_V) fp16 pairs, or null (alpha = 1)
+  int n_chain;
   int rotate;
   // query / lengths / tail / output
   const uint16_t* q;     // bf16 [B][Hq][128]
@@ -94,12 +99,18 @@ enum DecodeKernel : int { kKernelAuto = RQ_DECODE_KERNEL_AUTO, kKernelSimt = RQ_
 // ref_kind: RefKind; res_bits: 0 | 2 | 4; res_group: 16 | 32
 // `append` (or null): tokens to encode into the cache in the same launch as
 // the combine kernel (positions past every context of this decode).
+// p.n_chain > 1 (a chained loop) is CUDA-core only.
 cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_group, int kernel,
                           const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s,
                           const EncodeParams* append = nullptr);
-bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, int kernel);
+bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, int kernel, int n_chain = 1);
 // the kernel an automatic choice resolves to
-int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel);
+int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel, int n_chain = 1);
+
+// CUDA-core split kernel for the loops of chained policies (rq_decode_chain.cu):
+// the launcher for a chain of n_chain (2 or 3) links, or null
+using SplitLaunchFn = cudaError_t (*)(DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);
+SplitLaunchFn pick_chain(int ref_kind, int res_bits, int res_group, int G, int n_chain);
 
 // tensor-core split kernel (rq_decode_tc.cu)
 bool tc_variant_supported(int ref_kind, int res_bits, int res_group, int G);

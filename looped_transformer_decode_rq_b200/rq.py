@@ -30,7 +30,8 @@ MAX_BATCH = 1024
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_FLAG = range(7)
 FLAG_BAD_INPUT, FLAG_POSITION, FLAG_CTX_LEN, FLAG_PIPE_TIMEOUT, FLAG_META_OVERFLOW = 1, 2, 4, 8, 16
 ALPHA_LS, ALPHA_ONE, ALPHA_ZERO, ALPHA_NORM_RATIO = 0, 1, 2, 3
-ANCHOR_LAST, ANCHOR_FIRST, ANCHOR_INTERVAL = 0, 1, 2
+ANCHOR_LAST, ANCHOR_FIRST, ANCHOR_INTERVAL, ANCHOR_PREVIOUS, ANCHOR_NEXT = 0, 1, 2, 3, 4
+MAX_CHAIN = 3
 DECODE_KERNEL_AUTO, DECODE_KERNEL_SIMT, DECODE_KERNEL_TENSOR = 0, 1, 2
 
 # every symbol the header declares (checked by the ABI tests)
@@ -54,7 +55,8 @@ class Layout(C.Structure):
     _fields_ = [("capacity_padded", C.c_int64), ("total_bytes", C.c_int64), ("status_offset", C.c_int64),
                 ("codes_offset", (C.c_int64 * 2) * MAX_LOOPS), ("meta_offset", (C.c_int64 * 2) * MAX_LOOPS),
                 ("alpha_offset", C.c_int64 * MAX_LOOPS), ("codes_record_bytes", C.c_int64 * MAX_LOOPS),
-                ("meta_record_bytes", C.c_int64 * MAX_LOOPS), ("anchor_of", C.c_int32 * MAX_LOOPS)]
+                ("meta_record_bytes", C.c_int64 * MAX_LOOPS), ("anchor_of", C.c_int32 * MAX_LOOPS),
+                ("ref_of", C.c_int32 * MAX_LOOPS)]
 
 
 _vp, _i32, _i64, _f32 = C.c_void_p, C.c_int32, C.c_int64, C.c_float

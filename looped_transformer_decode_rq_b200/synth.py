@@ -59,7 +59,8 @@ class Workload:
     n_tail: int = 1
     seed: int = 0
     layers: int = 1
-    anchor_policy: int = 0      # 0: final loop is the reference; 1: loop 0; 2: blocks of anchor_interval
+    anchor_policy: int = 0      # 0: final loop is the reference; 1: loop 0; 2: blocks of anchor_interval;
+                                # 3 / 4: chained, loop l against loop l-1 / l+1
     anchor_interval: int = 0
 
     def with_(self, **kw) -> "Workload":
@@ -89,6 +90,14 @@ def ouro_8k(batch: int = 16, context: int = 8192) -> Workload:
     return Workload(name=f"ouro_L4_H16_B{batch}_T{context}_int2g32_bf16ref", batch=batch,
                     kv_heads=16, q_heads=16, context=context, sigma=(0.3, 0.2, 0.1),
                     outlier_p=0.01, seed=1)
+
+
+def ouro_8k_next_loop(batch: int = 16, context: int = 8192) -> Workload:
+    """The Ouro-shaped 8k layer stored with the Next-loop chained reference
+    (loop l against loop l+1, the final loop the bf16 anchor): decoding loop 1
+    reads the codes of loops 1-3 and the anchor."""
+    return ouro_8k(batch, context).with_(name=f"ouro_L4_H16_B{batch}_T{context}_int2g32_bf16ref_next_loop",
+                                         anchor_policy=4)
 
 
 def mixed_int4_anchor(batch: int = 8, context: int = 8192) -> Workload:

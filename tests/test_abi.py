@@ -146,3 +146,42 @@ def test_layout_anchor_policies(librq):
     assert rq.lib().rq_cache_layout(C.byref(bad), C.byref(rq.Layout())) == rq.ERR_UNSUPPORTED
     bad.anchor_interval = 1
     assert rq.lib().rq_cache_layout(C.byref(bad), C.byref(rq.Layout())) == rq.ERR_INVALID_ARG
+
+
+def test_layout_chained_policies(librq):
+    """Previous-/Next-loop references: ref_of is the neighbour, anchor_of the
+    chain's end; a chain must share one residual format, keep alpha and stay
+    within RQ_MAX_CHAIN links."""
+    rq = librq
+    nxt = rq.cache_layout(_cfg(librq, bits=[2, 2, 2, 4], group=[32] * 4, rotate=[1, 1, 1, 0],
+                               anchor_policy=rq.ANCHOR_NEXT))
+    assert list(nxt.ref_of)[:4] == [1, 2, 3, 3]
+    assert list(nxt.anchor_of)[:4] == [3, 3, 3, 3]
+    assert nxt.alpha_offset[3] == -1 and all(nxt.alpha_offset[l] >= 0 for l in (0, 1, 2))
+    prev = rq.cache_layout(_cfg(librq, bits=[4, 2, 2, 2], group=[32] * 4, rotate=[0, 1, 1, 1],
+                                anchor_policy=rq.ANCHOR_PREVIOUS))
+    assert list(prev.ref_of)[:4] == [0, 0, 1, 2]
+    assert list(prev.anchor_of)[:4] == [0, 0, 0, 0]
+    last = rq.cache_layout(_cfg(librq, bits=[2, 2, 2, 16], group=[32] * 4, rotate=[1, 1, 1, 0]))
+    assert list(last.ref_of)[:4] == [3, 3, 3, 3]
+
+    def status(**kw):
+        c = _cfg(librq, **kw)
+        return rq.lib().rq_cache_layout(C.byref(c), C.byref(rq.Layout()))
+    # mixed residual formats on one chain
+    assert status(bits=[2, 2, 4, 16], group=[32] * 4, rotate=[1, 1, 1, 0], anchor_policy=rq.ANCHOR_NEXT) == rq.ERR_UNSUPPORTED
+    assert status(bits=[2, 2, 2, 16], group=[16, 32, 32, 32], rotate=[1, 1, 1, 0],
+                  anchor_policy=rq.ANCHOR_NEXT) == rq.ERR_UNSUPPORTED
+    assert status(bits=[2, 2, 2, 16], group=[32] * 4, rotate=[0, 1, 1, 0], anchor_policy=rq.ANCHOR_NEXT) == rq.ERR_UNSUPPORTED
+    # direct quantisation (alpha 0) has no reference to chain through
+    assert status(bits=[2, 2, 2, 16], group=[32] * 4, rotate=[1, 1, 1, 0], alpha_mode=[2, 0, 0, 0],
+                  anchor_policy=rq.ANCHOR_NEXT) == rq.ERR_UNSUPPORTED
+    # at most three links
+    c5 = rq.config_from_dict(dict(num_loops=5, batch=1, kv_heads=1, q_heads=1, capacity=64, bits=[2, 2, 2, 2, 16],
+                                  group=[32] * 5, rotate=[1, 1, 1, 1, 0], alpha_mode=[0] * 5,
+                                  anchor_policy=rq.ANCHOR_NEXT))
+    assert rq.lib().rq_cache_layout(C.byref(c5), C.byref(rq.Layout())) == rq.ERR_UNSUPPORTED
+    c5.anchor_policy = rq.ANCHOR_LAST
+    assert rq.lib().rq_cache_layout(C.byref(c5), C.byref(rq.Layout())) == rq.OK
+    c5.anchor_policy = 5
+    assert rq.lib().rq_cache_layout(C.byref(c5), C.byref(rq.Layout())) == rq.ERR_INVALID_ARG

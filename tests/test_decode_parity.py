@@ -143,6 +143,40 @@ def test_anchor_policies(librq, policy, interval, L, bits, alpha):
     run_case(librq, wl, lengths=[150, 70])
 
 
+@pytest.mark.parametrize("policy,bits,group,G", [
+    (4, (2, 2, 2, 16), (32,) * 4, 1),          # Next-loop, bf16 anchor, INT2 g=32
+    (4, (2, 2, 2, 4), (32,) * 4, 4),           # Next-loop, INT4 anchor ([RQ] Table 9's [2,2,2,4])
+    (3, (4, 2, 2, 2), (32, 16, 16, 16), 2),    # Previous-loop, INT4 anchor ([4,2,2,2]), INT2 g=16
+    (3, (16, 4, 4, 4), (32,) * 4, 8),          # Previous-loop, bf16 anchor, INT4 links
+])
+def test_chained_policies(librq, policy, bits, group, G):
+    """Previous-/Next-loop references ([RQ] Table 9): a loop one, two or three
+    links from its anchor is decoded from every link's codes."""
+    anchor = 0 if policy == 3 else 3
+    rot = tuple(0 if l == anchor else 1 for l in range(4))
+    wl = synth.Workload(name=f"chain_{policy}_{G}", batch=3, kv_heads=2, q_heads=2 * G, context=300, bits=bits,
+                        group=group, rotate=rot, sigma=(0.3, 0.2, 0.1), outlier_p=0.01, anchor_policy=policy,
+                        seed=60 + policy + G)
+    run_case(librq, wl, lengths=[300, 129, 1])
+
+
+def test_chained_loops_run_on_the_cuda_core_kernel(librq):
+    """The tensor-core kernel decodes the anchor and the loop next to it (one
+    link) but reports a longer chain as unsupported; the default then picks the
+    CUDA-core kernel."""
+    rq = librq
+    wl = synth.Workload(name="chain_tc", batch=2, kv_heads=2, q_heads=8, context=260, sigma=(0.3, 0.2, 0.1),
+                        anchor_policy=4, seed=66)
+    run_case(rq, wl, loops=[2, 3], kernel=rq.DECODE_KERNEL_TENSOR)
+    cache = rq.Cache(rq.config_from_dict(synth.cache_config_dict(wl)), device="cuda")
+    inp = synth.make_inputs(wl, "cpu")
+    cache.set_decode_kernel(rq.DECODE_KERNEL_TENSOR)
+    with pytest.raises(rq.RQError) as e:
+        cache.decode_attention(0, inp["q"][0].cuda(), inp["ctx_len"].cuda())
+    assert e.value.status == rq.ERR_UNSUPPORTED
+    run_case(rq, wl, loops=[0, 1])
+
+
 @pytest.mark.parametrize("n_tail", [64, 127])
 def test_recent_window_bf16_tail(librq, n_tail):
     """A window of the most recent 64-127 tokens kept in bf16 next to the compact
@@ -265,15 +299,15 @@ def _same_planes(a, b):
 
 
 @pytest.mark.parametrize("kernel", ["simt", "tensor"])
-@pytest.mark.parametrize("bits", [(2, 2, 2, 16), (2, 2, 4, 4)])
-def test_decode_with_fused_append_matches_separate_calls(librq, kernel, bits):
+@pytest.mark.parametrize("bits,policy", [((2, 2, 2, 16), 0), ((2, 2, 4, 4), 0), ((2, 2, 2, 16), 4)])
+def test_decode_with_fused_append_matches_separate_calls(librq, kernel, bits, policy):
     """rq_decode_attention_append (the final loop's decode plus the per-step
     append of every loop's new token, one combine launch) gives the same output
     and the same cache bytes as a decode followed by an encode at device positions."""
     from tests.helpers import read_planes
     rq = librq
     wl = synth.Workload(name="fused_append", batch=3, kv_heads=2, q_heads=8, context=200, bits=bits,
-                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, seed=95)
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, anchor_policy=policy, seed=95)
     inp = synth.make_inputs(wl, "cpu")
     cfgd = synth.cache_config_dict(wl)
     k, v = inp["k"].cuda(), inp["v"].cuda()

@@ -34,6 +34,17 @@ CASES = [
                    bits=(2, 2, 2, 4, 2, 2, 2, 16), group=(16, 32, 32, 32, 32, 16, 32, 32),
                    rotate=(1, 1, 1, 0, 1, 1, 0, 0), alpha_mode=(0, 0, 3, 0, 0, 1, 0, 0),
                    sigma=(0.3, 0.25, 0.2, 0.15, 0.1, 0.1, 0.05), anchor_policy=2, anchor_interval=4, seed=14),
+    # chained references ([RQ] Table 9: Next-loop with [2,2,2,4]-style formats, Previous-loop with [4,2,2,2]):
+    # each loop is stored against its neighbour's binary32 reconstruction
+    synth.Workload(name="next_loop_chain", batch=2, kv_heads=3, q_heads=3, context=45,
+                   bits=(2, 2, 2, 16), group=(32,) * 4, rotate=(1, 1, 1, 0), alpha_mode=(0, 3, 1, 0),
+                   sigma=(0.3, 0.2, 0.1), outlier_p=0.02, anchor_policy=4, seed=15),
+    synth.Workload(name="previous_loop_chain_int4", batch=2, kv_heads=2, q_heads=2, context=70,
+                   bits=(4, 2, 2, 2), group=(32, 16, 16, 16), rotate=(0, 1, 1, 1),
+                   sigma=(0.3, 0.2, 0.1), outlier_p=0.02, anchor_policy=3, seed=16),
+    synth.Workload(name="next_loop_chain_int4_unrotated", batch=1, kv_heads=2, q_heads=2, context=33,
+                   bits=(4, 4, 4, 4), group=(32,) * 4, rotate=(0, 0, 0, 0), sigma=(0.3, 0.2, 0.1),
+                   anchor_policy=4, seed=17),
 ]
 
 
