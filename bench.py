@@ -363,7 +363,7 @@ def measure_workload(wl, steps, warmup, world, rank, per_loop=False):
             per_kernel["tensor"] = call_gbs(rq.DECODE_KERNEL_TENSOR)
         except rq.RQError:
             per_kernel["tensor"] = None
-    ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+    ws = torch.zeros(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
 
     def bf16_step():
         for l in range(L):
@@ -441,7 +441,7 @@ def run_capacity(args, world, rank):
                     kv[1, :, :, :T].copy_(one["v"][l].expand(B, -1, -1, -1))
                     planes.append(kv)
                 caches.append(planes)
-            ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+            ws = torch.zeros(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
 
             def step():
                 for planes in caches:
@@ -537,7 +537,7 @@ def run_mixed_sweep(args, world, rank):
         def append():
             cache.encode(k_new, v_new, positions=ctx)
 
-        ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
 
         def bf16_step():
             for l in range(L):
@@ -685,7 +685,7 @@ def run_rq(args, world, rank):
     if not args.no_bf16:
         kc = [inp["k"][l] for l in range(L)]
         vc = [inp["v"][l] for l in range(L)]
-        ws = torch.empty(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
+        ws = torch.zeros(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
 
         def bf16_step():
             for l in range(L):
@@ -743,6 +743,7 @@ def run_rq(args, world, rank):
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                      "frac_of_8tbs": round(achieved / 8000.0, 4)},
         "cpu_baseline": cpu, "e2e": e2e, "bf16_cache": bf16, "parity": parity, "other_workloads": extra,
+        # per step: a split and a combine kernel per loop (the final loop's combine also appends)
         "gpu_launches": args.steps * (2 * L), "clocks": clk, "device_flags": flags,
     }
     if rank == 0:

@@ -34,6 +34,17 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
+// Programmatic dependent launch (sm_90 and later).  A split kernel lets the
+// combine kernel that follows it on the stream (launched with programmatic
+// stream serialization) be scheduled at once; the combine kernel does its
+// input-only set-up, then waits in pdl_wait() until the split grid has
+// completed and its writes are visible.  This takes the combine kernel's launch
+// and set-up off the critical path.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }

@@ -61,7 +61,10 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int Hq = P.Hkv * G;
   if (wid >= P.B * Hq) {
-    if constexpr (APPEND) enc::encode_warp(E, wid - P.B * Hq, lane);
+    if constexpr (APPEND) {
+      pdl_wait();  // the split kernel reads the pages these positions are written into
+      enc::encode_warp(E, wid - P.B * Hq, lane);
+    }
     return;
   }
   const int b = wid / Hq, qh = wid % Hq, h = qh / G, gi = qh % G;
@@ -82,6 +85,15 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   const int nt_b = (clamp_len(P.ctx_len[b]) + pt - 1) / pt;
   const int64_t total = tot * P.Hkv;
   const int64_t P_eff = total < P.num_ctas ? total : P.num_ctas;
+  // inputs the split kernel does not write: the query and the first tail token
+  const uint2 qraw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hq + qh) * kD + 4 * lane);
+  uint2 kr0 = make_uint2(0u, 0u), vr0 = kr0;
+  if (P.n_tail > 0) {
+    const int64_t off = (static_cast<int64_t>(b) * P.Hkv + h) * P.n_tail * kD + 4 * lane;
+    kr0 = *reinterpret_cast<const uint2*>(P.k_tail + off);
+    vr0 = *reinterpret_cast<const uint2*>(P.v_tail + off);
+  }
+  pdl_wait();  // the split kernel's partials are complete and visible from here on
 
   float m = -INFINITY, l = 0.f;
   float4 ar = make_float4(0.f, 0.f, 0.f, 0.f), as = ar;
@@ -106,12 +118,11 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   }
   // current (tail) tokens in bf16
   if (P.n_tail > 0) {
-    const uint2 qraw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hq + qh) * kD + 4 * lane);
     const float2 q01 = bf16x2_to_f2(qraw.x), q23 = bf16x2_to_f2(qraw.y);
     for (int j = 0; j < P.n_tail; ++j) {
       const int64_t off = ((static_cast<int64_t>(b) * P.Hkv + h) * P.n_tail + j) * kD + 4 * lane;
-      const uint2 kr = *reinterpret_cast<const uint2*>(P.k_tail + off);
-      const uint2 vr = *reinterpret_cast<const uint2*>(P.v_tail + off);
+      const uint2 kr = j == 0 ? kr0 : *reinterpret_cast<const uint2*>(P.k_tail + off);
+      const uint2 vr = j == 0 ? vr0 : *reinterpret_cast<const uint2*>(P.v_tail + off);
       const float2 k01 = bf16x2_to_f2(kr.x), k23 = bf16x2_to_f2(kr.y);
       float d = __fmaf_rn(q23.y, k23.y, __fmaf_rn(q23.x, k23.x, __fmaf_rn(q01.y, k01.y, __fmul_rn(q01.x, k01.x))));
 #pragma unroll
@@ -213,13 +224,28 @@ cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_gr
   const int64_t warps = static_cast<int64_t>(p.B) * p.Hkv * p.G;
   const int64_t enc_warps = append ? static_cast<int64_t>(append->B) * append->Hkv * append->n_tokens : 0;
   const int rot = (res_bits != 0 && p.rotate) ? 1 : 0;
+  // programmatic dependent launch: scheduled while the split kernel runs, the
+  // combine kernel waits for it in pdl_wait()
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (enc_warps > 0) {
-    decode_combine_kernel<true><<<static_cast<unsigned>((warps + enc_warps + 3) / 4), 128, 0, s>>>(p, p.G, rot, *append);
+    cfg.gridDim = dim3(static_cast<unsigned>((warps + enc_warps + 3) / 4), 1, 1);
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<true>, p, p.G, rot, *append);
   } else {
     EncodeParams none;
     memset(&none, 0, sizeof(none));
-    decode_combine_kernel<false><<<static_cast<unsigned>((warps + 3) / 4), 128, 0, s>>>(p, p.G, rot, none);
+    cfg.gridDim = dim3(static_cast<unsigned>((warps + 3) / 4), 1, 1);
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<false>, p, p.G, rot, none);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

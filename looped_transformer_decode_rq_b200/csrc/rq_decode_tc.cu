@@ -433,6 +433,7 @@ __global__ void __launch_bounds__(kNT, 1)
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_launch_dependents();  // the combine kernel may be scheduled (it waits for this grid's completion)
 
   const int64_t total = static_cast<int64_t>(sPre[B]) * Hkv;
   const int64_t P_eff = total < P.num_ctas ? total : P.num_ctas;

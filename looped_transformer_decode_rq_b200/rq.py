@@ -152,7 +152,7 @@ class Cache:
         self._h = h
         ws = _i64()
         _check(_lib.rq_decode_workspace_size(self._h, C.byref(ws)), "rq_decode_workspace_size")
-        self.workspace = torch.empty(ws.value, dtype=torch.uint8, device=self.base.device)
+        self.workspace = torch.zeros(ws.value, dtype=torch.uint8, device=self.base.device)
 
     @property
     def handle(self):
@@ -291,7 +291,7 @@ def bf16_decode_attention(k_cache: torch.Tensor, v_cache: torch.Tensor, q: torch
     Hq = q.shape[1]
     assert D == HEAD_DIM and k_cache.stride() == v_cache.stride() and k_cache.stride(-1) == 1
     if workspace is None:
-        workspace = torch.empty(bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=q.device)
+        workspace = torch.zeros(bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=q.device)
     if out is None:
         out = torch.empty((B, Hq, HEAD_DIM), dtype=torch.float32, device=q.device)
     n_tail = 0 if k_tail is None else k_tail.shape[2]

@@ -331,3 +331,60 @@ def test_decode_with_fused_append_matches_separate_calls(librq, kernel, bits, po
     assert caches[0].get_error() == 0 and caches[1].get_error() == 0
     assert torch.equal(out_a, out_b)
     _same_planes(read_planes(caches[0], wl.context + 1), read_planes(caches[1], wl.context + 1))
+
+
+@pytest.mark.parametrize("kernel", ["simt", "tensor"])
+def test_any_workspace_contents_repeated_calls_and_graph_replay(librq, kernel):
+    """The workspace needs no initial contents; repeated calls and replays of a
+    captured CUDA graph (split kernel, then the combine kernel as a programmatic
+    dependent launch) give the same, correct output, with ragged and empty
+    sequences."""
+    rq = librq
+    wl = synth.Workload(name="segment_combine", batch=5, kv_heads=3, q_heads=12, context=700,
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, seed=97)
+    wl = wl.with_(lengths=(700, 0, 1, 333, 64))
+    inp = synth.make_inputs(wl, "cpu")
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    cache.set_decode_kernel(rq.DECODE_KERNEL_SIMT if kernel == "simt" else rq.DECODE_KERNEL_TENSOR)
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    q, ctx = inp["q"][0].cuda(), inp["ctx_len"].cuda()
+    kt, vt = inp["k_tail"][0].cuda(), inp["v_tail"][0].cuda()
+    enc = oracle_encode(inp, cfgd)
+    want = O.decode_attention_f64(enc, 0, to_np32(inp["q"][0]), inp["ctx_len"].numpy(),
+                                  to_np32(inp["k_tail"][0]), to_np32(inp["v_tail"][0]))
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    first = None
+    for fill in ("ones", "random", "zeros"):
+        if fill == "ones":
+            cache.workspace.fill_(0xFF)
+        elif fill == "random":
+            cache.workspace.copy_(torch.randint(0, 256, cache.workspace.shape, generator=gen, device="cuda",
+                                                dtype=torch.int32).to(torch.uint8))
+        else:
+            cache.workspace.zero_()
+        for _ in range(3):
+            out = cache.decode_attention(0, q, ctx, kt, vt)
+            torch.cuda.synchronize()
+            assert cache.get_error() == 0
+            assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL, fill
+            if first is None:
+                first = out.clone()
+            assert torch.equal(out, first), fill
+    static_out = torch.zeros_like(first)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        cache.decode_attention(0, q, ctx, kt, vt, out=static_out)  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cache.decode_attention(0, q, ctx, kt, vt, out=static_out)
+    for _ in range(3):
+        static_out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(static_out, first)
+    del graph
+    assert cache.get_error() == 0
