@@ -491,6 +491,22 @@ def decode_attention_f64(enc: Encoded, loop: int, q: np.ndarray, ctx_len: np.nda
     return out
 
 
+def decode_attention_multi_f64(enc: Encoded, loop: int, q: np.ndarray, ctx_len: np.ndarray,
+                               k_tail: np.ndarray, v_tail: np.ndarray,
+                               scale: float = 1.0 / np.sqrt(128.0)) -> np.ndarray:
+    """Several query tokens per sequence (speculative verification of n_q draft
+    tokens): q [B, n_q, Hq, 128]; the last n_q tail tokens are the draft tokens'
+    keys and values.  Draft token i is an ordinary decode whose tail stops at
+    itself: tail tokens 0 .. n_tail - n_q + i.  Returns float64 [B, n_q, Hq, 128]."""
+    q = np.asarray(q)
+    n_q, n_tail = q.shape[1], k_tail.shape[2]
+    out = np.zeros(q.shape, dtype=np.float64)
+    for i in range(n_q):
+        n_vis = n_tail - n_q + i + 1
+        out[:, i] = decode_attention_f64(enc, loop, q[:, i], ctx_len, k_tail[:, :, :n_vis], v_tail[:, :, :n_vis], scale)
+    return out
+
+
 def attention_f64(q: np.ndarray, Kc: np.ndarray, Vc: np.ndarray, ctx_len: np.ndarray,
                   k_tail: Optional[np.ndarray] = None, v_tail: Optional[np.ndarray] = None,
                   scale: float = 1.0 / np.sqrt(128.0)) -> np.ndarray:

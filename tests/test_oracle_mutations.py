@@ -96,6 +96,15 @@ def _decode_chain_drops_link_alpha(enc, loop, q, ctx_len, k_tail=None, v_tail=No
             enc.loops[c]["k"].alpha = saved[c]
 
 
+def _multi_query_tail_excludes_self(enc, loop, q, ctx_len, k_tail, v_tail, scale=1 / np.sqrt(128)):
+    n_q, n_tail = q.shape[1], k_tail.shape[2]
+    out = np.zeros(q.shape)
+    for i in range(n_q):
+        n_vis = n_tail - n_q + i
+        out[:, i] = O.decode_attention_f64(enc, loop, q[:, i], ctx_len, k_tail[:, :, :n_vis], v_tail[:, :, :n_vis], scale)
+    return out
+
+
 def _tree_dot_drops_last_lane(a, b):
     prod = (np.asarray(a, np.float32) * np.asarray(b, np.float32)).astype(np.float32)
     return prod[..., :120].sum(-1, dtype=np.float32)
@@ -103,7 +112,7 @@ def _tree_dot_drops_last_lane(a, b):
 
 ORIG = {n: getattr(O, n) for n in ("fwht_fp32", "ls_alpha_fp32", "reconstruct_f64", "residual_f64",
                                    "quantize_groups_fp32", "dequant_f64", "decode_attention_f64",
-                                   "lane_tree_dot_fp32", "reconstruct_fp32")}
+                                   "lane_tree_dot_fp32", "reconstruct_fp32", "decode_attention_multi_f64")}
 
 PINS = [
     P.test_p1_alpha_minimises_squared_error,
@@ -122,6 +131,7 @@ PINS = [
     lambda: [P.test_chained_scaled_copies_reconstruct_exactly(p, 1) for p in (O.ANCHOR_PREVIOUS, O.ANCHOR_NEXT)],
     lambda: P.test_chained_reconstruction_error_is_the_quantiser_error(O.ANCHOR_NEXT, 16),
     lambda: P.test_chained_decode_equals_brute_force(O.ANCHOR_NEXT, 4),
+    P.test_multi_query_decode_equals_masked_brute_force,
 ]
 
 
@@ -146,6 +156,7 @@ def _any_pin_fails():
     ("reconstruct_f64", _reconstruct_chain_via_anchor),
     ("reconstruct_fp32", _chain_view_without_residual),
     ("decode_attention_f64", _decode_chain_drops_link_alpha),
+    ("decode_attention_multi_f64", _multi_query_tail_excludes_self),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, mutant):
     monkeypatch.setattr(O, name, mutant)

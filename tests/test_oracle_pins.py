@@ -558,3 +558,37 @@ def test_chain_of_one_link_equals_star_policies():
             assert np.array_equal(a.loops[loop][n].codes, b.loops[loop][n].codes)
             assert np.array_equal(a.loops[loop][n].alpha, b.loops[loop][n].alpha)
             assert np.array_equal(a.loops[loop][n].scale, b.loops[loop][n].scale)
+
+
+# ----------------------------------------------- multi-query (draft token) decode
+
+def test_multi_query_decode_equals_masked_brute_force():
+    """Each draft token's row equals softmax attention over the reconstructed
+    cache and the whole tail under an explicit causal mask (tail token j is
+    visible to draft token i iff j <= n_tail - n_q + i), built here as one score
+    matrix instead of the oracle's truncated tails."""
+    rng = np.random.default_rng(99)
+    B, H, G, T, n_q, n_tail = 2, 2, 2, 21, 3, 5
+    cfg = O.CacheConfig(4, [2, 2, 4, 16], [32, 16, 32, 32], [1, 1, 0, 0], [0, 3, 0, 0])
+    K = np.stack([bf16_values(rng, (B, H, T, 128)) for _ in range(4)])
+    V = np.stack([bf16_values(rng, (B, H, T, 128)) for _ in range(4)])
+    enc = O.encode_fp32emu(K, V, cfg)
+    q = bf16_values(rng, (B, n_q, G * H, 128))
+    kt, vt = bf16_values(rng, (B, H, n_tail, 128)), bf16_values(rng, (B, H, n_tail, 128))
+    ctx = np.array([21, 6])
+    scale = 1 / np.sqrt(128)
+    for loop in (0, 3):
+        got = O.decode_attention_multi_f64(enc, loop, q, ctx, kt, vt)
+        Kh, Vh = O.reconstruct_f64(enc, loop)
+        for b in range(B):
+            n = int(ctx[b])
+            for qh in range(G * H):
+                h = qh // G
+                Kall = np.concatenate([Kh[b, h, :n], kt[b, h].astype(np.float64)])
+                Vall = np.concatenate([Vh[b, h, :n], vt[b, h].astype(np.float64)])
+                S = scale * (q[b, :, qh].astype(np.float64) @ Kall.T)          # [n_q, n + n_tail]
+                visible = np.arange(n + n_tail)[None, :] <= (n + n_tail - n_q + np.arange(n_q))[:, None]
+                S = np.where(visible, S, -np.inf)
+                P_ = np.exp(S - S.max(1, keepdims=True))
+                want = (P_ @ Vall) / P_.sum(1, keepdims=True)
+                assert np.abs(got[b, :, qh] - want).max() <= 1e-12 * max(1.0, np.abs(want).max())
