@@ -399,6 +399,62 @@ def measure_workload(wl, steps, warmup, world, rank, per_loop=False):
     return out
 
 
+def measure_multi_query(wl, n_q, steps, warmup, world, rank):
+    """Side line: one step of n_q draft tokens per sequence (speculative
+    verification) through rq_decode_attention_multi on every loop, against the
+    single-query step of the same cache; the cache is read once per call."""
+    from looped_transformer_decode_rq_b200 import rq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = wl.with_(seed=wl.seed + 1000 * rank, n_tail=n_q)
+    inp = synth.make_inputs(wl, dev)
+    qm = synth.draft_queries(wl, n_q, dev)
+    L, B, Hkv, Hq, T = wl.num_loops, wl.batch, wl.kv_heads, wl.q_heads, wl.context
+    cfgd = synth.cache_config_dict(wl, capacity=T + n_q)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
+    cache.encode(inp["k"], inp["v"])
+    ctx = inp["ctx_len"]
+    tokens_total = int(ctx.sum().item())
+    kt, vt = inp["k_tail"], inp["v_tail"]
+    outs = torch.empty((L, B, n_q, Hq, 128), dtype=torch.float32, device=dev)
+    out1 = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def multi_step():
+        for l in range(L):
+            cache.decode_attention_multi(l, qm[l], ctx, kt[l], vt[l], out=outs[l])
+
+    kt1 = [kt[l][:, :, :1].contiguous() for l in range(L)]
+    vt1 = [vt[l][:, :, :1].contiguous() for l in range(L)]
+
+    def single_step():
+        for l in range(L):
+            cache.decode_attention(l, inp["q"][l], ctx, kt1[l], vt1[l], out=out1[l])
+
+    ms = time_steps(multi_step, steps, warmup, world, stream)
+    ms1 = time_steps(single_step, steps, warmup, world, stream)
+    ev = []
+    for _ in range(8):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        cache.decode_attention_multi(0, qm[0], ctx, kt[0], vt[0], out=outs[0])
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    call_ms = statistics.median(a.elapsed_time(b) for a, b in ev[3:])
+    res_bytes = (tokens_total * Hkv * record_bytes(cache.layout, cfgd, 0) + B * n_q * Hq * 128 * (2 + 4) +
+                 B * Hkv * n_q * 512)
+    flags = cache.get_error()
+    out = {"workload": f"{wl.name}_verify{n_q}", "n_q": n_q,
+           "query_tokens_per_s": round(job_tokens_per_s(B * n_q, world, ms), 1), "ms_per_step": round(ms, 4),
+           "single_query_tokens_per_s": round(job_tokens_per_s(B, world, ms1), 1),
+           "single_query_ms_per_step": round(ms1, 4),
+           "residual_loop_gbs": round(res_bytes / (call_ms * 1e-3) / 1e9, 1), "residual_loop_bytes": res_bytes,
+           "device_flags": flags}
+    del cache, inp, outs, out1, qm
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_capacity(args, world, rank):
     """24-layer, 4-loop model at 8192 context: the largest batch whose caches
     fit in HBM for a bf16 cache and for ResidualQuant caches (bf16 anchor and
@@ -723,7 +779,8 @@ def run_rq(args, world, rank):
         extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 10, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8), 10, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8, q_heads=64), 10, 3, world, rank),
-                 measure_workload(synth.ouro_8k_next_loop(), 10, 3, world, rank, per_loop=True)]
+                 measure_workload(synth.ouro_8k_next_loop(), 10, 3, world, rank, per_loop=True),
+                 measure_multi_query(synth.ouro_8k(), 4, 10, 3, world, rank)]
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,

@@ -412,7 +412,9 @@ rq_status check_decode_common(int B, int Hkv, int Hq, const void* q, const int32
 
 namespace {
 
-rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, const int32_t* ctx_len,
+// n_q > 1: a multi-query call (q and out [B][n_q][Hq][128]; the last n_q tail
+// tokens are the draft tokens, each seen by itself and the later ones)
+rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int32_t n_q, const int32_t* ctx_len,
                       const void* k_tail, const void* v_tail, int32_t n_tail, float softmax_scale, float* out,
                       void* workspace, int64_t workspace_bytes, rq_stream_t stream,
                       const rq::EncodeParams* append) {
@@ -420,9 +422,14 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, cons
   rq_cache* cache = const_cast<rq_cache*>(cache_c);
   const rq_config& c = cache->cfg;
   if (loop < 0 || loop >= c.num_loops) return fail(RQ_ERR_INVALID_ARG, "loop %d outside [0, %d)", loop, c.num_loops);
-  const int G = c.q_heads / c.kv_heads;
-  int64_t need = 0;
-  rq_decode_workspace_size(cache, &need);
+  const int gq = c.q_heads / c.kv_heads;
+  if (n_q < 1) return fail(RQ_ERR_INVALID_ARG, "n_q %d < 1", n_q);
+  const int G = n_q * gq;  // query rows per kv-head
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(RQ_ERR_UNSUPPORTED, "n_q * q_heads / kv_heads = %d (supported: 1, 2, 4, 8)", G);
+  if (n_q > 1 && n_tail < n_q)
+    return fail(RQ_ERR_INVALID_ARG, "n_tail %d < n_q %d (the draft tokens are the last n_q tail tokens)", n_tail, n_q);
+  const int64_t need = rq::decode_workspace_bytes(c.batch, c.kv_heads, G, cache->num_ctas);
   rq_status st = check_decode_common(c.batch, c.kv_heads, c.q_heads, q, ctx_len, k_tail, v_tail, n_tail,
                                      softmax_scale, out, workspace, workspace_bytes, need);
   if (st != RQ_OK) return st;
@@ -455,6 +462,10 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, cons
   p.B = c.batch;
   p.Hkv = c.kv_heads;
   p.G = G;
+  p.gq = gq;
+  p.n_q = n_q;
+  p.q_stride_i = static_cast<int64_t>(c.q_heads) * RQ_HEAD_DIM;
+  p.q_stride_b = n_q * p.q_stride_i;
   p.capacity = c.capacity;
   p.plane_tokens = lay.capacity_padded;
   if (ref_kind == rq::kRefInt4) {
@@ -498,7 +509,23 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, cons
 rq_status rq_decode_attention(const rq_cache* cache, int32_t loop, const void* q, const int32_t* ctx_len,
                               const void* k_tail, const void* v_tail, int32_t n_tail, float softmax_scale,
                               float* out, void* workspace, int64_t workspace_bytes, rq_stream_t stream) {
-  return decode_impl(cache, loop, q, ctx_len, k_tail, v_tail, n_tail, softmax_scale, out, workspace,
+  return decode_impl(cache, loop, q, 1, ctx_len, k_tail, v_tail, n_tail, softmax_scale, out, workspace,
+                     workspace_bytes, stream, nullptr);
+}
+
+rq_status rq_decode_multi_workspace_size(const rq_cache* cache, int32_t n_q, int64_t* bytes_out) {
+  if (cache == nullptr || bytes_out == nullptr) return fail(RQ_ERR_INVALID_ARG, "null argument");
+  if (n_q < 1 || n_q > 8) return fail(RQ_ERR_INVALID_ARG, "n_q %d outside [1, 8]", n_q);
+  const int G = n_q * (cache->cfg.q_heads / cache->cfg.kv_heads);
+  *bytes_out = rq::decode_workspace_bytes(cache->cfg.batch, cache->cfg.kv_heads, G, cache->num_ctas);
+  return RQ_OK;
+}
+
+rq_status rq_decode_attention_multi(const rq_cache* cache, int32_t loop, const void* q, int32_t n_q,
+                                    const int32_t* ctx_len, const void* k_tail, const void* v_tail, int32_t n_tail,
+                                    float softmax_scale, float* out, void* workspace, int64_t workspace_bytes,
+                                    rq_stream_t stream) {
+  return decode_impl(cache, loop, q, n_q, ctx_len, k_tail, v_tail, n_tail, softmax_scale, out, workspace,
                      workspace_bytes, stream, nullptr);
 }
 
@@ -515,7 +542,7 @@ rq_status rq_decode_attention_append(rq_cache* cache, int32_t loop, const void* 
     const rq_status st = build_encode(cache, k_new, v_new, strides, 0, positions, n_new, &ep);
     if (st != RQ_OK) return st;
   }
-  return decode_impl(cache, loop, q, ctx_len, k_tail, v_tail, n_tail, softmax_scale, out, workspace,
+  return decode_impl(cache, loop, q, 1, ctx_len, k_tail, v_tail, n_tail, softmax_scale, out, workspace,
                      workspace_bytes, stream, n_new > 0 ? &ep : nullptr);
 }
 
@@ -554,6 +581,10 @@ rq_status rq_bf16_decode_attention(int32_t batch, int32_t kv_heads, int32_t q_he
   p.B = batch;
   p.Hkv = kv_heads;
   p.G = G;
+  p.gq = G;
+  p.n_q = 1;
+  p.q_stride_i = static_cast<int64_t>(q_heads) * RQ_HEAD_DIM;
+  p.q_stride_b = p.q_stride_i;
   p.capacity = capacity;
   p.plane_tokens = 0;
   p.q = static_cast<const uint16_t*>(q);

@@ -86,9 +86,12 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   const int64_t total = tot * P.Hkv;
   const int64_t P_eff = total < P.num_ctas ? total : P.num_ctas;
   // inputs the split kernel does not write: the query and the first tail token
-  const uint2 qraw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hq + qh) * kD + 4 * lane);
+  const int64_t row = q_row_offset(P, b, h, gi);
+  const uint2 qraw = *reinterpret_cast<const uint2*>(P.q + row + 4 * lane);
+  // draft token i of a multi-query call sees the tail up to itself
+  const int n_vis = P.n_tail - P.n_q + gi / P.gq + 1;
   uint2 kr0 = make_uint2(0u, 0u), vr0 = kr0;
-  if (P.n_tail > 0) {
+  if (n_vis > 0) {
     const int64_t off = (static_cast<int64_t>(b) * P.Hkv + h) * P.n_tail * kD + 4 * lane;
     kr0 = *reinterpret_cast<const uint2*>(P.k_tail + off);
     vr0 = *reinterpret_cast<const uint2*>(P.v_tail + off);
@@ -117,9 +120,9 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     }
   }
   // current (tail) tokens in bf16
-  if (P.n_tail > 0) {
+  if (n_vis > 0) {
     const float2 q01 = bf16x2_to_f2(qraw.x), q23 = bf16x2_to_f2(qraw.y);
-    for (int j = 0; j < P.n_tail; ++j) {
+    for (int j = 0; j < n_vis; ++j) {
       const int64_t off = ((static_cast<int64_t>(b) * P.Hkv + h) * P.n_tail + j) * kD + 4 * lane;
       const uint2 kr = j == 0 ? kr0 : *reinterpret_cast<const uint2*>(P.k_tail + off);
       const uint2 vr = j == 0 ? vr0 : *reinterpret_cast<const uint2*>(P.v_tail + off);
@@ -156,7 +159,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   const float inv = l > 0.f ? 1.f / l : 0.f;
   float4 o = make_float4(__fmul_rn(__fadd_rn(ar.x, as.x), inv), __fmul_rn(__fadd_rn(ar.y, as.y), inv),
                          __fmul_rn(__fadd_rn(ar.z, as.z), inv), __fmul_rn(__fadd_rn(ar.w, as.w), inv));
-  reinterpret_cast<float4*>(P.out + (static_cast<int64_t>(b) * Hq + qh) * kD)[lane] = o;
+  reinterpret_cast<float4*>(P.out + row)[lane] = o;
 }
 
 

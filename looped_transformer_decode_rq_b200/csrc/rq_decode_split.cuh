@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(kNT, 1)
     // ---- segment set-up: the G queries of (b, h) and their rotation
     if (warp < G) {
       const int qh = h * G + warp;
-      const uint2 raw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hkv * G + qh) * kD + 4 * lane);
+      const uint2 raw = *reinterpret_cast<const uint2*>(P.q + q_row_offset(P, b, h, warp) + 4 * lane);
       const float2 a01 = bf16x2_to_f2(raw.x), a23 = bf16x2_to_f2(raw.y);
       float x[4] = {a01.x, a01.y, a23.x, a23.y};
       *reinterpret_cast<float4*>(&sQS[warp * kD + 4 * lane]) = make_float4(x[0], x[1], x[2], x[3]);

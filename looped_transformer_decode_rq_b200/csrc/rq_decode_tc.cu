@@ -634,8 +634,7 @@ __global__ void __launch_bounds__(kNT, 1)
   auto setup = [&](int b, int h) {
     if (warp < G) {
       const int hq = warp;
-      const int qh = h * G + hq;
-      const uint2 raw = *reinterpret_cast<const uint2*>(P.q + (static_cast<int64_t>(b) * Hkv * G + qh) * kD + 4 * lane);
+      const uint2 raw = *reinterpret_cast<const uint2*>(P.q + q_row_offset(P, b, h, hq) + 4 * lane);
       const int d = 4 * lane;
       if constexpr (REF == kRefBf16) {
         *reinterpret_cast<uint2*>(QB + (d >> 6) * 2048 + (hq >> 3) * 1024 + (hq & 7) * 128 +

@@ -54,7 +54,7 @@ struct ReconstructParams {
 // One decode call: either a residual loop of a cache, an anchor loop, or a
 // plain bf16 cache.  Planes are indexed by record = (b*Hkv + h)*plane_tokens + t.
 struct DecodeParams {
-  int B, Hkv, G;
+  int B, Hkv, G;         // G: query rows per kv-head (n_q * gq)
   int capacity;          // valid positions per sequence (ctx_len is clamped to it)
   int64_t plane_tokens;  // record stride between (b, h) slabs for byte planes
   // reference (bf16 via tensor maps; INT4 via byte planes)
@@ -67,8 +67,12 @@ struct DecodeParams {
   const uint8_t* alpha[RQ_MAX_CHAIN];  // (alpha_K, alpha_V) fp16 pairs, or null (alpha = 1)
   int n_chain;
   int rotate;
-  // query / lengths / tail / output
-  const uint16_t* q;     // bf16 [B][Hq][128]
+  // query / lengths / tail / output.  Row gi of kv-head h is draft token
+  // i = gi / gq, head h * gq + gi % gq (see q_row_offset); q and out are
+  // [B][n_q][Hkv * gq][128], so one decode query per sequence is n_q = 1
+  int gq, n_q;
+  int64_t q_stride_b, q_stride_i;  // elements between sequences / draft tokens
+  const uint16_t* q;     // bf16
   const int32_t* ctx_len;
   const uint16_t* k_tail;  // bf16 [B][Hkv][n_tail][128]
   const uint16_t* v_tail;
@@ -82,6 +86,13 @@ struct DecodeParams {
   int page_tokens;       // split granularity (set by launch_decode for the chosen kernel)
   int stall_page;        // test hook: CTA-local page before which the producer waits out its limit (-1: none)
 };
+
+// Element offset of query row gi of kv-head h of sequence b in q and out.
+__host__ __device__ inline int64_t q_row_offset(const DecodeParams& P, int b, int h, int gi) {
+  const int i = gi / P.gq, g = gi - i * P.gq;
+  return static_cast<int64_t>(b) * P.q_stride_b + static_cast<int64_t>(i) * P.q_stride_i +
+         static_cast<int64_t>(h * P.gq + g) * RQ_HEAD_DIM;
+}
 
 // Split-K partial record per (slot, head): m, l, pad, pad, acc_ref[128], acc_res[128]
 constexpr int kPartialFloats = 4 + 2 * RQ_HEAD_DIM;

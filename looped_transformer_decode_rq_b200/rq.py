@@ -39,7 +39,8 @@ EXPORTED = ("rq_cache_layout", "rq_cache_create", "rq_cache_destroy", "rq_cache_
             "rq_decode_workspace_size", "rq_decode_attention", "rq_bf16_decode_workspace_size",
             "rq_bf16_decode_attention", "rq_reconstruct", "rq_get_error", "rq_status_string",
             "rq_last_error_message", "rq_decode_attention_static_scratch", "rq_cache_set_decode_kernel",
-            "rq_cache_set_debug_stall", "rq_decode_attention_append")
+            "rq_cache_set_debug_stall", "rq_decode_attention_append", "rq_decode_multi_workspace_size",
+            "rq_decode_attention_multi")
 STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 
@@ -69,6 +70,8 @@ _sig = {
     "rq_cache_set_decode_kernel": (C.c_int, [_vp, _i32]),
     "rq_cache_set_debug_stall": (C.c_int, [_vp, _i32]),
     "rq_decode_workspace_size": (C.c_int, [_vp, C.POINTER(_i64)]),
+    "rq_decode_multi_workspace_size": (C.c_int, [_vp, _i32, C.POINTER(_i64)]),
+    "rq_decode_attention_multi": (C.c_int, [_vp, _i32, _vp, _i32, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp]),
     "rq_decode_attention": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp]),
     "rq_decode_attention_static_scratch": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp]),
     "rq_decode_attention_append": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp, _vp,
@@ -153,6 +156,7 @@ class Cache:
         ws = _i64()
         _check(_lib.rq_decode_workspace_size(self._h, C.byref(ws)), "rq_decode_workspace_size")
         self.workspace = torch.zeros(ws.value, dtype=torch.uint8, device=self.base.device)
+        self._multi_ws = {}
 
     @property
     def handle(self):
@@ -213,6 +217,29 @@ class Cache:
         _check(_lib.rq_decode_attention(self._h, loop, q.data_ptr(), ctx_len.data_ptr(), _ptr(k_tail),
                                         _ptr(v_tail), n_tail, scale, out.data_ptr(), self.workspace.data_ptr(),
                                         self.workspace.numel(), _stream(stream)), "rq_decode_attention")
+        return out
+
+    def decode_attention_multi(self, loop: int, q: torch.Tensor, ctx_len: torch.Tensor,
+                               k_tail: torch.Tensor, v_tail: torch.Tensor, softmax_scale: Optional[float] = None,
+                               out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """n_q query tokens per sequence: q bf16 [B, n_q, Hq, 128]; the last n_q of the
+        tail tokens (bf16 [B, Hkv, n_tail, 128]) are the draft tokens.  Returns fp32
+        [B, n_q, Hq, 128]."""
+        cfg = self.cfg
+        assert q.dtype == torch.bfloat16 and q.is_contiguous() and q.dim() == 4 and ctx_len.dtype == torch.int32
+        n_q = q.shape[1]
+        assert k_tail.is_contiguous() and v_tail.is_contiguous()
+        if out is None:
+            out = torch.empty((cfg.batch, n_q, cfg.q_heads, HEAD_DIM), dtype=torch.float32, device=q.device)
+        ws = self._multi_ws.get(n_q)
+        if ws is None:
+            need = C.c_int64()
+            _check(_lib.rq_decode_multi_workspace_size(self._h, n_q, C.byref(need)), "rq_decode_multi_workspace_size")
+            ws = self._multi_ws[n_q] = torch.zeros(need.value, dtype=torch.uint8, device=self.base.device)
+        scale = softmax_scale if softmax_scale is not None else HEAD_DIM ** -0.5
+        _check(_lib.rq_decode_attention_multi(self._h, loop, q.data_ptr(), n_q, ctx_len.data_ptr(), _ptr(k_tail),
+                                              _ptr(v_tail), k_tail.shape[2], scale, out.data_ptr(), ws.data_ptr(),
+                                              ws.numel(), _stream(stream)), "rq_decode_attention_multi")
         return out
 
     def decode_attention_append(self, loop: int, q: torch.Tensor, ctx_len: torch.Tensor,

@@ -195,6 +195,16 @@ def make_inputs(wl: Workload, device="cpu", layer: int = 0) -> dict:
     return out
 
 
+def draft_queries(wl: Workload, n_q: int, device="cpu") -> torch.Tensor:
+    """Queries of n_q draft tokens per sequence and loop, bf16 [L, B, n_q, Hq, D],
+    drawn like the single decode queries (N(0, 1), rounded to bf16) from a
+    generator of their own."""
+    dev = torch.device(device)
+    g = torch.Generator(device=dev).manual_seed(wl.seed * 1000003 + 7919 * n_q + 17)
+    x = torch.randn(wl.num_loops, wl.batch, n_q, wl.q_heads, wl.head_dim, generator=g, device=dev)
+    return _bf16(x)
+
+
 def cache_config_dict(wl: Workload, capacity: Optional[int] = None) -> dict:
     """The cache configuration (fields of the C ABI's ``rq_config``)."""
     return dict(num_loops=wl.num_loops, batch=wl.batch, kv_heads=wl.kv_heads,

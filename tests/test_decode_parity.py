@@ -388,3 +388,59 @@ def test_any_workspace_contents_repeated_calls_and_graph_replay(librq, kernel):
         assert torch.equal(static_out, first)
     del graph
     assert cache.get_error() == 0
+
+
+@pytest.mark.parametrize("gq,n_q,bits,kernel", [
+    (1, 2, (2, 2, 2, 16), None),          # two draft tokens on the Ouro-shaped rows: CUDA cores
+    (1, 4, (2, 2, 2, 16), None),          # four rows per kv-head: tensor cores by default
+    (1, 4, (2, 2, 2, 16), "simt"),
+    (2, 4, (2, 2, 4, 4), None),           # GQA pairs x 4 drafts = 8 rows, INT4 anchor
+    (1, 8, (2, 2, 2, 16), "simt"),
+])
+def test_multi_query_decode(librq, gq, n_q, bits, kernel):
+    """n_q draft tokens per sequence in one call: every draft token sees the
+    cache, the earlier tail tokens and the draft tokens up to itself."""
+    rq = librq
+    wl = synth.Workload(name=f"multi_{gq}_{n_q}", batch=3, kv_heads=2, q_heads=2 * gq, context=300, bits=bits,
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, n_tail=n_q + 1, seed=110 + n_q + gq)
+    wl = wl.with_(lengths=(300, 0, 129))
+    inp = synth.make_inputs(wl, "cpu")
+    qm = synth.draft_queries(wl, n_q, "cpu")
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    if kernel == "simt":
+        cache.set_decode_kernel(rq.DECODE_KERNEL_SIMT)
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    enc = oracle_encode(inp, cfgd)
+    ctx = inp["ctx_len"]
+    for loop in (0, wl.num_loops - 1):
+        kt, vt = inp["k_tail"][loop], inp["v_tail"][loop]
+        out = cache.decode_attention_multi(loop, qm[loop].cuda(), ctx.cuda(), kt.cuda(), vt.cuda())
+        torch.cuda.synchronize()
+        want = O.decode_attention_multi_f64(enc, loop, to_np32(qm[loop]), ctx.numpy(), to_np32(kt), to_np32(vt))
+        err = rel_err_rows(out.cpu().numpy(), want)
+        assert err.max() <= ATTN_TOL, (loop, float(err.max()))
+    assert cache.get_error() == 0
+
+
+def test_multi_query_of_one_token_is_the_single_decode(librq):
+    rq = librq
+    wl = synth.Workload(name="multi_one", batch=2, kv_heads=2, q_heads=4, context=200, sigma=(0.3, 0.2, 0.1),
+                        seed=120)
+    inp = synth.make_inputs(wl, "cpu")
+    cache = rq.Cache(rq.config_from_dict(synth.cache_config_dict(wl)), device="cuda")
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    q, ctx, kt, vt = inp["q"][0].cuda(), inp["ctx_len"].cuda(), inp["k_tail"][0].cuda(), inp["v_tail"][0].cuda()
+    one = cache.decode_attention(0, q, ctx, kt, vt)
+    multi = cache.decode_attention_multi(0, q.unsqueeze(1).contiguous(), ctx, kt, vt)
+    torch.cuda.synchronize()
+    assert torch.equal(one, multi[:, 0])
+    # too many rows per kv-head, or fewer tail tokens than draft tokens
+    q8 = torch.zeros((2, 8, 4, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rq.RQError) as e:
+        cache.decode_attention_multi(0, q8, ctx, kt, vt)
+    assert e.value.status in (rq.ERR_UNSUPPORTED, rq.ERR_INVALID_ARG)
+    q2 = torch.zeros((2, 2, 4, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rq.RQError) as e:
+        cache.decode_attention_multi(0, q2, ctx, kt, vt)
+    assert e.value.status == rq.ERR_INVALID_ARG
