@@ -697,7 +697,7 @@ def run_rq(args, world, rank):
     step_bytes += L * B * Hkv * 512 + B * Hkv * (sum(record_bytes(lay, cfgd, l) for l in range(L)))
     peak, peak_kind = load_peaks()
     kernel_hash = source_hash([os.path.join(ROOT, "looped_transformer_decode_rq_b200", "csrc", f)
-                               for f in ("rq_decode.cu", "rq_decode_split.cuh", "rq_common.cuh")])
+                               for f in ("rq_decode_split.cuh", "rq_common.cuh", "rq_internal.h")])
     achieved = res_bytes / (call_ms * 1e-3) / 1e9
     traffic = read_profile_traffic(kernel_hash)
     value = job_tokens_per_s(B, world, ms)

@@ -270,8 +270,11 @@ RQ_API rq_status rq_decode_attention(const rq_cache* cache, int32_t loop, const 
                               int32_t n_tail, float softmax_scale, float* out, void* workspace,
                               int64_t workspace_bytes, rq_stream_t stream);
 
+/* Largest number of draft tokens of one rq_decode_attention_multi call. */
+#define RQ_MAX_DRAFT 16
+
 /* Bytes of workspace rq_decode_attention_multi needs for n_q draft tokens
- * (n_q in [1, 8]). */
+ * (n_q in [1, RQ_MAX_DRAFT]). */
 RQ_API rq_status rq_decode_multi_workspace_size(const rq_cache* cache, int32_t n_q, int64_t* bytes_out);
 
 /* Multi-query decode: rq_decode_attention for n_q query tokens per sequence at
@@ -281,13 +284,14 @@ RQ_API rq_status rq_decode_multi_workspace_size(const rq_cache* cache, int32_t n
  * sequence b attends to the ctx_len[b] cached tokens and to tail tokens
  * 0 .. n_tail - n_q + i: the last n_q tail tokens are the draft tokens' own
  * keys and values (bf16, not yet encoded), each visible to itself and to the
- * later ones, and any earlier tail tokens to all.  The n_q * G query rows of a
- * kv-head share every read of its cached pages, so the cache is read once per
- * call whatever n_q is; with 4 or more rows the automatic kernel choice is the
- * tensor-core kernel.
+ * later ones, and any earlier tail tokens to all.  Up to 8 query rows per
+ * kv-head (n_q * G) share every read of its cached pages; more rows run in
+ * blocks of 8, one pass over the cache each.  With 4 or more rows in a block
+ * the automatic kernel choice is the tensor-core kernel.
  *  q        device bf16 [B][n_q][Hq][128]
  *  out      device fp32 [B][n_q][Hq][128]
- *  n_q      >= 1 with n_q * (Hq / Hkv) in {1, 2, 4, 8}, else RQ_ERR_UNSUPPORTED
+ *  n_q      in [1, RQ_MAX_DRAFT] (else RQ_ERR_INVALID_ARG) with n_q * (Hq / Hkv)
+ *           in {1, 2, 4} or a multiple of 8 (else RQ_ERR_UNSUPPORTED)
  *  n_tail   >= n_q when n_q > 1 (RQ_ERR_INVALID_ARG otherwise)
  *  workspace  >= rq_decode_multi_workspace_size(cache, n_q) bytes
  * Other arguments, layouts and errors as rq_decode_attention (which is n_q = 1). */

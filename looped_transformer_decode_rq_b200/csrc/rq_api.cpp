@@ -163,6 +163,9 @@ rq_status validate_config(const rq_config* c) {
   return RQ_OK;
 }
 
+// query rows per kv-head a decode call takes: 1, 2, 4, or blocks of 8
+bool rows_supported(int rows) { return rows == 1 || rows == 2 || rows == 4 || (rows >= 8 && rows % 8 == 0); }
+
 int ref_kind_for(const rq_config& c, int loop) {
   const int a = anchor_of(c, loop);
   if (loop != a && c.alpha_mode[loop] == RQ_ALPHA_ZERO) return rq::kRefNone;
@@ -423,10 +426,11 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int3
   const rq_config& c = cache->cfg;
   if (loop < 0 || loop >= c.num_loops) return fail(RQ_ERR_INVALID_ARG, "loop %d outside [0, %d)", loop, c.num_loops);
   const int gq = c.q_heads / c.kv_heads;
-  if (n_q < 1) return fail(RQ_ERR_INVALID_ARG, "n_q %d < 1", n_q);
-  const int G = n_q * gq;  // query rows per kv-head
-  if (G != 1 && G != 2 && G != 4 && G != 8)
-    return fail(RQ_ERR_UNSUPPORTED, "n_q * q_heads / kv_heads = %d (supported: 1, 2, 4, 8)", G);
+  if (n_q < 1 || n_q > RQ_MAX_DRAFT) return fail(RQ_ERR_INVALID_ARG, "n_q %d outside [1, %d]", n_q, RQ_MAX_DRAFT);
+  const int rows = n_q * gq;  // query rows per kv-head, decoded in blocks of up to 8
+  if (!rows_supported(rows))
+    return fail(RQ_ERR_UNSUPPORTED, "n_q * q_heads / kv_heads = %d (supported: 1, 2, 4, or a multiple of 8)", rows);
+  int G = rows < 8 ? rows : 8;
   if (n_q > 1 && n_tail < n_q)
     return fail(RQ_ERR_INVALID_ARG, "n_tail %d < n_q %d (the draft tokens are the last n_q tail tokens)", n_tail, n_q);
   const int64_t need = rq::decode_workspace_bytes(c.batch, c.kv_heads, G, cache->num_ctas);
@@ -445,6 +449,13 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int3
     if (n_chain == RQ_MAX_CHAIN) return fail(RQ_ERR_UNSUPPORTED, "reference chain longer than %d", RQ_MAX_CHAIN);
     chain[n_chain++] = l;
   }
+  // The CUDA-core kernel's 8-row variants spill registers (about a tenth of the
+  // 4-row rate): by default, 8 rows that would land there run as two passes of
+  // 4 rows instead (each reads the cache once more).
+  if (G == 8 && cache->decode_kernel == RQ_DECODE_KERNEL_AUTO &&
+      rq::decode_kernel_choice(ref_kind, res_bits, res_group, 8, RQ_DECODE_KERNEL_AUTO, n_chain > 1 ? n_chain : 1) ==
+          rq::kKernelSimt)
+    G = 4;
   if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G, cache->decode_kernel, n_chain > 1 ? n_chain : 1))
     return fail(RQ_ERR_UNSUPPORTED, "no %s decode kernel for this loop format, G = %d and a chain of %d",
                 cache->decode_kernel == RQ_DECODE_KERNEL_TENSOR ? "tensor-core" : "", G, n_chain);
@@ -464,6 +475,7 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int3
   p.G = G;
   p.gq = gq;
   p.n_q = n_q;
+  p.row0 = 0;
   p.q_stride_i = static_cast<int64_t>(c.q_heads) * RQ_HEAD_DIM;
   p.q_stride_b = n_q * p.q_stride_i;
   p.capacity = c.capacity;
@@ -498,9 +510,14 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int3
   p.status = reinterpret_cast<int32_t*>(cache->base + cache->lay.status_offset);
   p.tma_tokens = lay.capacity_padded;
   p.stall_page = cache->stall_page;
-  cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, cache->decode_kernel, &cache->tm_anchor[a][0],
-                                    &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream), append);
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  // one pass over the cache per block of 8 rows (stream-ordered, so the blocks
+  // reuse one workspace)
+  for (int row0 = 0; row0 < rows; row0 += G) {
+    p.row0 = row0;
+    cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, cache->decode_kernel, &cache->tm_anchor[a][0],
+                                      &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream), append);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  }
   return RQ_OK;
 }
 
@@ -515,8 +532,9 @@ rq_status rq_decode_attention(const rq_cache* cache, int32_t loop, const void* q
 
 rq_status rq_decode_multi_workspace_size(const rq_cache* cache, int32_t n_q, int64_t* bytes_out) {
   if (cache == nullptr || bytes_out == nullptr) return fail(RQ_ERR_INVALID_ARG, "null argument");
-  if (n_q < 1 || n_q > 8) return fail(RQ_ERR_INVALID_ARG, "n_q %d outside [1, 8]", n_q);
-  const int G = n_q * (cache->cfg.q_heads / cache->cfg.kv_heads);
+  if (n_q < 1 || n_q > RQ_MAX_DRAFT) return fail(RQ_ERR_INVALID_ARG, "n_q %d outside [1, %d]", n_q, RQ_MAX_DRAFT);
+  const int rows = n_q * (cache->cfg.q_heads / cache->cfg.kv_heads);
+  const int G = rows < 8 ? rows : 8;
   *bytes_out = rq::decode_workspace_bytes(cache->cfg.batch, cache->cfg.kv_heads, G, cache->num_ctas);
   return RQ_OK;
 }

@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   const int64_t row = q_row_offset(P, b, h, gi);
   const uint2 qraw = *reinterpret_cast<const uint2*>(P.q + row + 4 * lane);
   // draft token i of a multi-query call sees the tail up to itself
-  const int n_vis = P.n_tail - P.n_q + gi / P.gq + 1;
+  const int n_vis = P.n_tail - P.n_q + (P.row0 + gi) / P.gq + 1;
   uint2 kr0 = make_uint2(0u, 0u), vr0 = kr0;
   if (n_vis > 0) {
     const int64_t off = (static_cast<int64_t>(b) * P.Hkv + h) * P.n_tail * kD + 4 * lane;

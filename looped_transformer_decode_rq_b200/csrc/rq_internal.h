@@ -71,6 +71,7 @@ struct DecodeParams {
   // i = gi / gq, head h * gq + gi % gq (see q_row_offset); q and out are
   // [B][n_q][Hkv * gq][128], so one decode query per sequence is n_q = 1
   int gq, n_q;
+  int row0;              // rows [row0, row0 + G) of the n_q * gq rows of a kv-head (blocks of 8 beyond 8 rows)
   int64_t q_stride_b, q_stride_i;  // elements between sequences / draft tokens
   const uint16_t* q;     // bf16
   const int32_t* ctx_len;
@@ -89,7 +90,8 @@ struct DecodeParams {
 
 // Element offset of query row gi of kv-head h of sequence b in q and out.
 __host__ __device__ inline int64_t q_row_offset(const DecodeParams& P, int b, int h, int gi) {
-  const int i = gi / P.gq, g = gi - i * P.gq;
+  const int r = P.row0 + gi;
+  const int i = r / P.gq, g = r - i * P.gq;
   return static_cast<int64_t>(b) * P.q_stride_b + static_cast<int64_t>(i) * P.q_stride_i +
          static_cast<int64_t>(h * P.gq + g) * RQ_HEAD_DIM;
 }

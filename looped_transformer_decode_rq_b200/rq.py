@@ -32,6 +32,7 @@ FLAG_BAD_INPUT, FLAG_POSITION, FLAG_CTX_LEN, FLAG_PIPE_TIMEOUT, FLAG_META_OVERFL
 ALPHA_LS, ALPHA_ONE, ALPHA_ZERO, ALPHA_NORM_RATIO = 0, 1, 2, 3
 ANCHOR_LAST, ANCHOR_FIRST, ANCHOR_INTERVAL, ANCHOR_PREVIOUS, ANCHOR_NEXT = 0, 1, 2, 3, 4
 MAX_CHAIN = 3
+MAX_DRAFT = 16
 DECODE_KERNEL_AUTO, DECODE_KERNEL_SIMT, DECODE_KERNEL_TENSOR = 0, 1, 2
 
 # every symbol the header declares (checked by the ABI tests)

@@ -396,6 +396,8 @@ def test_any_workspace_contents_repeated_calls_and_graph_replay(librq, kernel):
     (1, 4, (2, 2, 2, 16), "simt"),
     (2, 4, (2, 2, 4, 4), None),           # GQA pairs x 4 drafts = 8 rows, INT4 anchor
     (1, 8, (2, 2, 2, 16), "simt"),
+    (4, 4, (2, 2, 2, 16), None),          # 16 rows: two blocks of 8, one cache pass each
+    (1, 16, (2, 2, 4, 4), None),
 ])
 def test_multi_query_decode(librq, gq, n_q, bits, kernel):
     """n_q draft tokens per sequence in one call: every draft token sees the
@@ -435,11 +437,11 @@ def test_multi_query_of_one_token_is_the_single_decode(librq):
     multi = cache.decode_attention_multi(0, q.unsqueeze(1).contiguous(), ctx, kt, vt)
     torch.cuda.synchronize()
     assert torch.equal(one, multi[:, 0])
-    # too many rows per kv-head, or fewer tail tokens than draft tokens
-    q8 = torch.zeros((2, 8, 4, 128), dtype=torch.bfloat16, device="cuda")
+    # rows per kv-head neither 1, 2, 4 nor a multiple of 8; fewer tail tokens than drafts
+    q6 = torch.zeros((2, 3, 4, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(rq.RQError) as e:
-        cache.decode_attention_multi(0, q8, ctx, kt, vt)
-    assert e.value.status in (rq.ERR_UNSUPPORTED, rq.ERR_INVALID_ARG)
+        cache.decode_attention_multi(0, q6, ctx, kt, vt)
+    assert e.value.status == rq.ERR_UNSUPPORTED
     q2 = torch.zeros((2, 2, 4, 128), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(rq.RQError) as e:
         cache.decode_attention_multi(0, q2, ctx, kt, vt)
