@@ -17,6 +17,8 @@ CASES = [
     (synth.ouro_8k(), [(0, 0), (7, 9), (15, 15)]),
     (synth.mixed_int4_anchor(batch=8), [(0, 3), (7, 15)]),
     (synth.gqa_long(batch=8), [(0, 0), (5, 7)]),
+    (synth.gqa_long(batch=8, q_heads=64), [(3, 4)]),
+    (synth.ouro_8k_next_loop(), [(0, 0), (15, 15)]),
 ]
 
 
@@ -80,3 +82,33 @@ def test_full_size_sampled_parity(librq, wl, samples):
             got = outs[l][b:b + 1, h * G:(h + 1) * G].cpu().numpy()
             err = rel_err_rows(got, want).max()
             assert err <= ATTN_TOL, (wl.name, b, h, l, float(err))
+
+
+def test_full_size_multi_query(librq):
+    """Four draft tokens per sequence on the full Ouro-shaped cache, in the
+    configuration bench.py times (the tensor-core kernel, 4 rows per kv-head)."""
+    rq = librq
+    n_q = 4
+    wl = synth.ouro_8k().with_(n_tail=n_q)
+    dev = torch.device("cuda")
+    inp = synth.make_inputs(wl, dev)
+    qm = synth.draft_queries(wl, n_q, dev)
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
+    cache.encode(inp["k"], inp["v"])
+    ctx = inp["ctx_len"]
+    outs = [cache.decode_attention_multi(l, qm[l], ctx, inp["k_tail"][l], inp["v_tail"][l]) for l in (0, 3)]
+    torch.cuda.synchronize()
+    assert cache.get_error() == 0
+    ocfg = O.CacheConfig.from_dict(cfgd)
+    for b, h in [(2, 5), (14, 0)]:
+        n = int(ctx[b])
+        sl = lambda t: t[:, b:b + 1, h:h + 1].float().cpu().numpy()  # noqa: E731
+        enc = O.encode_fp32emu(sl(inp["k"])[:, :, :, :n], sl(inp["v"])[:, :, :, :n], ocfg)
+        kt, vt = sl(inp["k_tail"]), sl(inp["v_tail"])
+        for i, l in enumerate((0, 3)):
+            q = qm[l][b:b + 1, :, h:h + 1].float().cpu().numpy()
+            want = O.decode_attention_multi_f64(enc, l, q, np.array([n]), kt[l], vt[l])
+            got = outs[i][b:b + 1, :, h:h + 1].cpu().numpy()
+            err = rel_err_rows(got, want).max()
+            assert err <= ATTN_TOL, (b, h, l, float(err))
