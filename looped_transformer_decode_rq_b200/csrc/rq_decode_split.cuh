@@ -14,12 +14,11 @@
 namespace rq {
 namespace {
 
-constexpr int kNCW = 8;        // consumer warps
+// Consumer warps come in groups of four; a CTA has NG = 2 or 3 groups (8 or 12
+// consumer warps) plus the producer warp.
 constexpr int kGW = 4;         // warps per consumer group
 constexpr int kGT = kGW * 32;  // threads per consumer group
-constexpr int kNCT = kNCW * 32;
-constexpr int kNT = kNCT + 32; // + producer warp
-constexpr int kConsumerBar = 1;  // all consumers (256 threads)
+constexpr int kConsumerBar = 1;  // all consumers
 constexpr int kGroupBar0 = 2;    // group g uses kGroupBar0 + g (128 threads)
 constexpr unsigned kFull = 0xffffffffu;
 
@@ -43,10 +42,16 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // NCH: residual links per token (1; 2-3 for the loops of a chained policy,
-// whose links share one format)
-template <int REF, int RB, int RG, int G, int TT, int NCH = 1>
+// whose links share one format).  NG: consumer groups (pages k with k % NG == g
+// go to group g).
+template <int REF, int RB, int RG, int G, int TT, int NCH = 1, int NG = 2>
 struct Cfg {
   static_assert(NCH >= 1 && NCH <= RQ_MAX_CHAIN && (NCH == 1 || (RB != 0 && REF != kRefNone)), "chain");
+  static_assert(NG == 2 || NG == 3, "consumer groups");
+  static constexpr int NCW = kGW * NG;   // consumer warps
+  static constexpr int NCT = NCW * 32;   // consumer threads
+  static constexpr int NT = NCT + 32;    // + producer warp
+  static_assert(G <= NCW, "one warp per query head in the segment set-up");
   static constexpr int PAGE = TT;  // tokens per page / stage
   // phase 1 (scores): 4G lanes per token, D1 = 32/G dims per lane
   static constexpr int TPT = 4 * G;
@@ -84,12 +89,12 @@ struct Cfg {
   static constexpr int STAGE_BYTES = O_RES + NCH * RES_BLK;
   static constexpr int TX_BYTES = TT * (2 * REF_REC + 2 * REFM_REC + NCH * (2 * CB + 2 * MB + AL_REC));
   // non-stage shared memory
-  static constexpr int O_S = 0;                           // scores [2 groups][2 parity][G][TT]
-  static constexpr int O_WM = O_S + 4 * 4 * G * TT;      // warp maxima [2][2][G][kGW]
-  static constexpr int O_ACC = O_WM + 4 * 4 * G * kGW;    // [G][256]
+  static constexpr int O_S = 0;                           // scores [NG groups][2 parity][G][TT]
+  static constexpr int O_WM = O_S + 4 * NG * 2 * G * TT;  // warp maxima [NG][2][G][kGW]
+  static constexpr int O_ACC = O_WM + 4 * NG * 2 * G * kGW;  // [G][256]
   static constexpr int O_L = O_ACC + 4 * G * 2 * kD;      // [G] (padded to 8)
-  static constexpr int O_MG = O_L + 4 * 8;                // [2][G] (padded to 16)
-  static constexpr int O_QS = O_MG + 4 * 16;              // [G][128]
+  static constexpr int O_MG = O_L + 4 * 8;                // [NG][G] (padded to 32)
+  static constexpr int O_QS = O_MG + 4 * 32;              // [G][128]
   static constexpr int O_QT = O_QS + 4 * G * kD;          // [G][128]
   static constexpr int O_PRE = O_QT + 4 * G * kD;         // [RQ_MAX_BATCH + 1]
   static constexpr int O_NT = O_PRE + 4 * (RQ_MAX_BATCH + 1);
@@ -98,8 +103,10 @@ struct Cfg {
   static constexpr int MISC_BYTES = O_BAR + 16 * 8;
   static constexpr int kSmemLimit = 227 * 1024;
   static constexpr int STAGES_MAX = (kSmemLimit - 1024 - MISC_BYTES) / STAGE_BYTES;
-  // an even number of stages keeps each stage with one group
-  static constexpr int STAGES = STAGES_MAX >= 4 ? 4 : 2;
+  // A multiple of NG stages keeps each stage with one group, so that a group
+  // waiting on a stage's parity never sees a phase of another group's page.
+  static constexpr int STAGES = STAGES_MAX >= 2 * NG ? 2 * NG : NG;
+  static_assert(2 * STAGES < 15, "full and empty barriers below the stall barrier");
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + MISC_BYTES;
   static_assert(PASSES * TOK_PASS == TT && TOK2 * SLICES == TT, "lane mapping");
   static_assert((O_ACC % 16) == 0 && (O_QS % 16) == 0 && (O_WM % 16) == 0, "alignment");
@@ -188,10 +195,10 @@ __device__ __forceinline__ uint32_t unpack_bytes(uint32_t w, int k) {
 // ---------------------------------------------------------------------------
 // split kernel
 // ---------------------------------------------------------------------------
-template <int REF, int RB, int RG, int G, int TT, int NCH>
+template <int REF, int RB, int RG, int G, int TT, int NCH, int NG>
 __device__ __forceinline__ void issue_page(const DecodeParams& P, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                            uint8_t* st, uint32_t full, const PageIter& it, int Hkv) {
-  using C = Cfg<REF, RB, RG, G, TT, NCH>;
+  using C = Cfg<REF, RB, RG, G, TT, NCH, NG>;
   const int t0 = it.page * TT;
   // byte planes hold plane_tokens (a multiple of 64) records per (b, h): a
   // 128-token page may find only 64 of them at the plane's end
@@ -223,12 +230,13 @@ __device__ __forceinline__ void issue_page(const DecodeParams& P, const CUtensor
   }
 }
 
-template <int REF, int RB, int RG, int G, int TT, int NCH>
-__global__ void __launch_bounds__(kNT, 1)
+template <int REF, int RB, int RG, int G, int TT, int NCH, int NG>
+__global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
     decode_split_kernel(const __grid_constant__ DecodeParams P,
                         const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV) {
-  using C = Cfg<REF, RB, RG, G, TT, NCH>;
+  using C = Cfg<REF, RB, RG, G, TT, NCH, NG>;
+  constexpr int kNCW = C::NCW, kNCT = C::NCT, kNT = C::NT;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // align by offsetting the shared array itself so that every access below
   // stays a shared-memory access
@@ -318,7 +326,7 @@ __global__ void __launch_bounds__(kNT, 1)
         }
         if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[15]), 0)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
         if (*sAbort) break;
-        issue_page<REF, RB, RG, G, TT, NCH>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it, Hkv);
+        issue_page<REF, RB, RG, G, TT, NCH, NG>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it, Hkv);
         it.next(sNt, B, Hkv);
       }
       // Drain: no copy this CTA issued may still be landing when it exits.
@@ -333,7 +341,7 @@ __global__ void __launch_bounds__(kNT, 1)
   }
 
   // ========================= consumer groups =========================
-  const int grp = warp / kGW;        // pages k with k % 2 == grp
+  const int grp = warp / kGW;        // pages k with k % NG == grp
   const int gw = warp % kGW;         // warp within the group
   const int gtid = tid % kGT;        // thread within the group
   // phase-1 mapping: token within a pass and dim slice.  For G <= 2 the lanes
@@ -355,7 +363,7 @@ __global__ void __launch_bounds__(kNT, 1)
   const int slice = gtid / C::TPR2;  // phase-2 mapping
   const int j2 = gtid % C::TPR2;
   const int d2 = C::D2 * j2;
-  float* gS = sS + grp * 2 * G * TT;
+  float* gS = sS + grp * 2 * G * TT;    // [2 parity][G][TT] of this group
   float* gWM = sWM + grp * 2 * G * kGW;
 
   PageIter it;
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(kNT, 1)
     }
 
     for (int sp = 0; sp < seg_pages; ++sp, ++k) {
-      if ((k & 1) != grp) {  // the other group's page
+      if ((k % NG) != grp) {  // another group's page
         it.next(sNt, B, Hkv);
         continue;
       }
@@ -453,7 +461,7 @@ __global__ void __launch_bounds__(kNT, 1)
         }
       }
       const int n_valid = min(TT, len_b - it.page * TT);
-      const int par = (k >> 1) & 1;
+      const int par = (k / NG) & 1;
       float* pS = gS + par * G * TT;
       float* pWM = gWM + par * G * kGW;
 
@@ -725,7 +733,8 @@ __global__ void __launch_bounds__(kNT, 1)
     float cref[G][C::D2], cres[G][C::D2], cl[G];
 #pragma unroll
     for (int gi = 0; gi < G; ++gi) {
-      const float M = fmaxf(sMG[gi], sMG[G + gi]);
+      float M = fmaxf(sMG[gi], sMG[G + gi]);
+      if constexpr (NG == 3) M = fmaxf(M, sMG[2 * G + gi]);
       const float f = (m_run[gi] == -INFINITY) ? 0.f : fast_exp2(m_run[gi] - M);
 #pragma unroll
       for (int e = 0; e < C::D2; ++e) {
@@ -771,7 +780,8 @@ __global__ void __launch_bounds__(kNT, 1)
         *src = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       if (tid < G) {
-        const float M = fmaxf(sMG[tid], sMG[G + tid]);
+        float M = fmaxf(sMG[tid], sMG[G + tid]);
+        if constexpr (NG == 3) M = fmaxf(M, sMG[2 * G + tid]);
         reinterpret_cast<float4*>(rec + tid * kPartialFloats)[0] = make_float4(M, sL[tid], 0.f, 0.f);
         sL[tid] = 0.f;
       }
@@ -785,18 +795,28 @@ __global__ void __launch_bounds__(kNT, 1)
 // Pages of 64 tokens for a bf16 anchor (one tensor-copy tile); 128 for the
 // byte-plane formats, whose 64-token pages are too small to amortise the
 // per-page synchronisation, when four stages still fit.
+// Three consumer groups (12 warps) for the byte-plane formats at G <= 2, which
+// are bound by instruction latency with two; two elsewhere (the bf16-anchor
+// formats are bound by HBM, and larger G or chains need the registers).
+template <int REF, int RB, int RG, int G, int NCH>
+constexpr int groups_of() {
+  return (REF != kRefBf16 && G <= 2 && NCH == 1) ? 3 : 2;
+}
+
 template <int REF, int RB, int RG, int G, int NCH>
 constexpr int page_tokens_of() {
+  constexpr int NG = groups_of<REF, RB, RG, G, NCH>();
   if constexpr (REF == kRefBf16) return kPage;
-  else return Cfg<REF, RB, RG, G, 2 * kPage, NCH>::STAGES_MAX >= 4 ? 2 * kPage : kPage;
+  else return Cfg<REF, RB, RG, G, 2 * kPage, NCH, NG>::STAGES_MAX >= (NG == 3 ? 3 : 4) ? 2 * kPage : kPage;
 }
 
 template <int REF, int RB, int RG, int G, int NCH>
 cudaError_t launch_split(DecodeParams& p, const CUtensorMap* tk, const CUtensorMap* tv, cudaStream_t s) {
   constexpr int TT = page_tokens_of<REF, RB, RG, G, NCH>();
-  using C = Cfg<REF, RB, RG, G, TT, NCH>;
-  static_assert(C::STAGES_MAX >= 2, "stage ring does not fit in shared memory");
-  auto kern = decode_split_kernel<REF, RB, RG, G, TT, NCH>;
+  constexpr int NG = groups_of<REF, RB, RG, G, NCH>();
+  using C = Cfg<REF, RB, RG, G, TT, NCH, NG>;
+  static_assert(C::STAGES_MAX >= NG, "stage ring does not fit in shared memory");
+  auto kern = decode_split_kernel<REF, RB, RG, G, TT, NCH, NG>;
   p.page_tokens = TT;
   static bool attr_done = false;  // per instantiation; set once per process
   if (!attr_done) {
@@ -804,7 +824,7 @@ cudaError_t launch_split(DecodeParams& p, const CUtensorMap* tk, const CUtensorM
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  kern<<<p.num_ctas, kNT, C::SMEM_BYTES, s>>>(p, *tk, *tv);
+  kern<<<p.num_ctas, C::NT, C::SMEM_BYTES, s>>>(p, *tk, *tv);
   return cudaGetLastError();
 }
 
