@@ -46,8 +46,10 @@ PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "rq_decode_split_ouro8k_traffic
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    # 100 steps of about 0.8 ms: a timed window long enough that run-to-run clock
+    # drift averages out
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["rq", "reference"], default="rq")
     ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "tiny", "capacity", "mixed_sweep"],
                     default="ouro8k")
@@ -705,36 +707,62 @@ def run_rq(args, world, rank):
     # ---- e2e through the public API with host buffers
     e2e = None
     if not args.no_e2e:
+        # Every step copies its inputs from pinned host memory and its outputs
+        # back.  As in a serving loop, the copies run on their own streams and
+        # overlap the neighbouring steps' decode (inputs and outputs double-
+        # buffered, ordered by events); the timed region spans the first
+        # input copy to the last output copy.
         hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q.cpu())
         hk = torch.empty(k_new.shape, dtype=k_new.dtype, pin_memory=True).copy_(k_new.cpu())
         hv = torch.empty(v_new.shape, dtype=v_new.dtype, pin_memory=True).copy_(v_new.cpu())
-        hout = torch.empty(outs.shape, dtype=outs.dtype, pin_memory=True)
-        dq, dk, dv = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+        hout = [torch.empty(outs.shape, dtype=outs.dtype, pin_memory=True) for _ in range(2)]
+        dbuf = [(torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(outs))
+                for _ in range(2)]
+        h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("h2d", "comp", "d2h")}
 
-        def e2e_step():
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-            for l in range(L - 1):
-                cache.decode_attention(l, dq[l], ctx, dk[l], dv[l], out=outs[l])
-            cache.decode_attention_append(L - 1, dq[L - 1], ctx, dk[L - 1], dv[L - 1], dk, dv, pos, out=outs[L - 1])
-            hout.copy_(outs, non_blocking=True)
+        def e2e_run(nsteps, start_ev=None):
+            if start_ev is not None:
+                h2d_s.wait_event(start_ev)
+            for i in range(nsteps):
+                j = i % 2
+                dq, dk, dv, do = dbuf[j]
+                if i >= 2:
+                    h2d_s.wait_event(ev["comp"][j])  # step i-2 no longer reads these inputs
+                with torch.cuda.stream(h2d_s):
+                    dq.copy_(hq, non_blocking=True)
+                    dk.copy_(hk, non_blocking=True)
+                    dv.copy_(hv, non_blocking=True)
+                ev["h2d"][j].record(h2d_s)
+                stream.wait_event(ev["h2d"][j])
+                if i >= 2:
+                    stream.wait_event(ev["d2h"][j])  # step i-2's output has left the device
+                for l in range(L - 1):
+                    cache.decode_attention(l, dq[l], ctx, dk[l], dv[l], out=do[l])
+                cache.decode_attention_append(L - 1, dq[L - 1], ctx, dk[L - 1], dv[L - 1], dk, dv, pos, out=do[L - 1])
+                ev["comp"][j].record(stream)
+                d2h_s.wait_event(ev["comp"][j])
+                with torch.cuda.stream(d2h_s):
+                    hout[j].copy_(do, non_blocking=True)
+                ev["d2h"][j].record(d2h_s)
+            stream.wait_stream(d2h_s)
+            stream.wait_stream(h2d_s)
 
-        for _ in range(2):
-            e2e_step()
+        e2e_run(3)
+        torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
         a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        e2e_run(args.steps, start_ev=a)
         b2.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         ems = max_over_ranks(a.elapsed_time(b2) / args.steps, world)
         e2e = {"value": round(job_tokens_per_s(B, world, ems), 1), "unit": "tokens/s",
                "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
-               "d2h_bytes_per_step": int(hout.numel() * 4)}
+               "d2h_bytes_per_step": int(hout[0].numel() * 4),
+               "copies": "own streams, overlapping the neighbouring steps (double-buffered)"}
 
     # ---- the same step over a bf16 cache (same library)
     bf16 = None
@@ -776,11 +804,11 @@ def run_rq(args, world, rank):
     if not args.no_extra and args.workload == "ouro8k":
         del cache, inp, outs
         torch.cuda.empty_cache()
-        extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 10, 3, world, rank),
-                 measure_workload(synth.gqa_long(batch=8), 10, 3, world, rank),
-                 measure_workload(synth.gqa_long(batch=8, q_heads=64), 10, 3, world, rank),
-                 measure_workload(synth.ouro_8k_next_loop(), 10, 3, world, rank, per_loop=True),
-                 measure_multi_query(synth.ouro_8k(), 4, 10, 3, world, rank)]
+        extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 30, 3, world, rank),
+                 measure_workload(synth.gqa_long(batch=8), 30, 3, world, rank),
+                 measure_workload(synth.gqa_long(batch=8, q_heads=64), 30, 3, world, rank),
+                 measure_workload(synth.ouro_8k_next_loop(), 30, 3, world, rank, per_loop=True),
+                 measure_multi_query(synth.ouro_8k(), 4, 30, 3, world, rank)]
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
