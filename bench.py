@@ -202,9 +202,9 @@ def source_hash(paths):
     return h.hexdigest()[:16]
 
 
-def read_profile_traffic(kernel_hash):
+def read_profile_traffic(kernel_hash, workload):
     """Per-launch DRAM bytes of the split kernel from the committed ncu summary,
-    if it was taken on the current kernel source."""
+    if it was taken on the current kernel source and on this workload."""
     if not os.path.exists(PROFILE_TRAFFIC):
         return None
     vals = {}
@@ -212,7 +212,7 @@ def read_profile_traffic(kernel_hash):
         if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("kernel_source_sha256_16") != kernel_hash:
+    if vals.get("kernel_source_sha256_16") != kernel_hash or vals.get("workload") != workload:
         return None
     for key in ("dram_bytes_per_launch", "dram_bytes_per_launch_scaled"):
         try:
@@ -701,7 +701,7 @@ def run_rq(args, world, rank):
     kernel_hash = source_hash([os.path.join(ROOT, "looped_transformer_decode_rq_b200", "csrc", f)
                                for f in ("rq_decode_split.cuh", "rq_common.cuh", "rq_internal.h")])
     achieved = res_bytes / (call_ms * 1e-3) / 1e9
-    traffic = read_profile_traffic(kernel_hash)
+    traffic = read_profile_traffic(kernel_hash, wl.name)
     value = job_tokens_per_s(B, world, ms)
 
     # ---- e2e through the public API with host buffers
