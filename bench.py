@@ -808,6 +808,7 @@ def run_rq(args, world, rank):
                  measure_workload(synth.gqa_long(batch=8), 30, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8, q_heads=64), 30, 3, world, rank),
                  measure_workload(synth.ouro_8k_next_loop(), 30, 3, world, rank, per_loop=True),
+                 measure_workload(synth.ouro_8k_next_loop_int4(), 30, 3, world, rank, per_loop=True),
                  measure_multi_query(synth.ouro_8k(), 4, 30, 3, world, rank)]
 
     out = {

@@ -800,7 +800,7 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
 // formats are bound by HBM, and larger G or chains need the registers).
 template <int REF, int RB, int RG, int G, int NCH>
 constexpr int groups_of() {
-  return (REF != kRefBf16 && G <= 2 && NCH == 1) ? 3 : 2;
+  return (REF != kRefBf16 && (G == 1 || (G == 2 && NCH == 1))) ? 3 : 2;
 }
 
 template <int REF, int RB, int RG, int G, int NCH>

@@ -100,6 +100,13 @@ def ouro_8k_next_loop(batch: int = 16, context: int = 8192) -> Workload:
                                          anchor_policy=4)
 
 
+def ouro_8k_next_loop_int4(batch: int = 16, context: int = 8192) -> Workload:
+    """Next-loop chain with an INT4 anchor, loops 1-3 INT2 g=32 ([2,2,2,4], the
+    mixed Next-loop setting of the pages' Table 9)."""
+    return ouro_8k(batch, context).with_(name=f"ouro_L4_H16_B{batch}_T{context}_2224_int4ref_next_loop",
+                                         bits=(2, 2, 2, 4), anchor_policy=4)
+
+
 def mixed_int4_anchor(batch: int = 8, context: int = 8192) -> Workload:
     """Same shape, loops 1-2 INT2, loop 3 INT4, reference loop INT4 g=32."""
     return Workload(name=f"mixed_2244_H16_B{batch}_T{context}_int4ref", batch=batch,

@@ -148,6 +148,8 @@ def test_anchor_policies(librq, policy, interval, L, bits, alpha):
     (4, (2, 2, 2, 4), (32,) * 4, 4),           # Next-loop, INT4 anchor ([RQ] Table 9's [2,2,2,4])
     (3, (4, 2, 2, 2), (32, 16, 16, 16), 2),    # Previous-loop, INT4 anchor ([4,2,2,2]), INT2 g=16
     (3, (16, 4, 4, 4), (32,) * 4, 8),          # Previous-loop, bf16 anchor, INT4 links
+    (4, (2, 2, 2, 4), (32,) * 4, 1),           # INT4-anchor chains at G = 1 run three consumer groups
+    (3, (4, 2, 2, 2), (32, 16, 16, 16), 1),
 ])
 def test_chained_policies(librq, policy, bits, group, G):
     """Previous-/Next-loop references ([RQ] Table 9): a loop one, two or three
