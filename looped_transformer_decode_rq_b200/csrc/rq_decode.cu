@@ -12,28 +12,14 @@
 // brought back with a single inverse Hadamard per (sequence, q-head) in the
 // combine kernel.  No bf16 copy of loop l is ever formed.
 //
-// Split kernel (persistent, one CTA per SM):
-//   * the flattened sequence of 64-token pages over all (b, kv-head) pairs is
-//     cut into num_ctas contiguous ranges of equal length, so ragged batches
-//     balance to within one page; a CTA emits one partial (m, l, acc) per
-//     (b, kv-head) segment it touches;
-//   * warp 8 is the producer: one lane streams pages into a ring of shared
-//     memory stages through the Tensor Memory Accelerator -- tiled tensor
-//     copies with the 128-byte swizzle for bf16 reference tiles, bulk copies
-//     for code, metadata and alpha records -- completing on mbarriers;
-//   * warps 0-7 form two groups of four that take alternate pages ("ping-
-//     pong"), each with its own online softmax and group-local barriers, so
-//     one group's barrier and reduction latency overlaps the other's math.
-//     Within a group a page is processed in two phases: scores (4G lanes per
-//     token, shuffle reduction) and values (16 lanes per token row, 8 dims per
-//     lane, softmax weights recomputed per lane).  The groups merge once per
-//     segment;
-//   * packed codes become floats with one LOP3 each (1 + c*2^(p-23)), the
-//     2^(p-23) factor being folded into the query once per segment and into
-//     the accumulators once per flush; fp32 pairs use FFMA2.
-// Combine kernel: one warp per (b, q-head) merges the CTA partials with the
-// max-rescale rule, adds the bf16 tail tokens, applies the inverse rotation and
-// normalises.
+// This file holds the combine kernel and the dispatch; the CUDA-core split
+// kernel is in rq_decode_split.cuh, the tensor-core one in rq_decode_tc.cu.
+// Combine kernel: one warp per (b, query row) merges the CTA partials with the
+// max-rescale rule, adds the bf16 tail tokens (a draft token of a multi-query
+// call sees the tail up to itself), applies the inverse rotation and
+// normalises.  It is a programmatic dependent launch: scheduled while the split
+// kernel runs, it reads its inputs, then waits for the split grid's completion.
+// With an append it also encodes the step's new tokens into every loop.
 #include <cstring>
 
 #include "rq_common.cuh"

@@ -1,10 +1,32 @@
 // rq_decode_split.cuh -- the CUDA-core split kernel of the fused decode
-// attention (see rq_decode.cu for the method and the launch structure), as
-// templates over the loop format: anchor kind, residual bits and group, query
-// heads per kv-head G, page size and the number of residual links NCH (1, or
-// 2-3 for the loops of a chained Previous-/Next-loop policy).  Included by
+// attention (see rq_decode.cu for the method), as templates over the loop
+// format: anchor kind, residual bits and group, query rows per kv-head G, page
+// size, the number of residual links NCH (1, or 2-3 for the loops of a chained
+// Previous-/Next-loop policy) and the number of consumer groups NG.  Included by
 // rq_decode.cu (NCH = 1) and rq_decode_chain.cu (NCH = 2, 3), so that the two
 // sets of instantiations compile in parallel.
+//
+// Persistent, one CTA per SM:
+//   * the flattened sequence of pages (64 tokens with a bf16 anchor, 128 for
+//     the byte-plane formats) over all (b, kv-head) pairs is cut into num_ctas
+//     contiguous ranges of equal length, so ragged batches balance to within
+//     one page; a CTA emits one partial (m, l, acc) per (b, kv-head) segment
+//     it touches;
+//   * the last warp is the producer: one lane streams pages into a ring of
+//     shared-memory stages through the Tensor Memory Accelerator -- tiled
+//     tensor copies with the 128-byte swizzle for bf16 anchor tiles, bulk
+//     copies for code, metadata and alpha records -- completing on mbarriers;
+//   * the consumer warps form NG groups of four (2, or 3 for the byte-plane
+//     formats at G <= 2) that take pages in turn, each with its own online
+//     softmax and group-local barriers, so that one group's barrier and
+//     reduction latency overlaps the others' math.  Within a group a page is
+//     processed in two phases: scores (4G lanes per token, dp4a on the packed
+//     codes, shuffle reduction) and values (16 lanes per token row, 8 dims per
+//     lane, softmax weights recomputed per lane).  The groups merge once per
+//     segment, in a fixed order;
+//   * packed codes become floats with one LOP3 each (1 + c*2^(p-23)), the
+//     2^(p-23) factor being folded into the accumulators once per flush; fp32
+//     pairs use FFMA2.
 #pragma once
 
 #include "rq_common.cuh"
