@@ -400,13 +400,16 @@ def test_any_workspace_contents_repeated_calls_and_graph_replay(librq, kernel):
     (1, 8, (2, 2, 2, 16), "simt"),
     (4, 4, (2, 2, 2, 16), None),          # 16 rows: two blocks of 8, one cache pass each
     (1, 16, (2, 2, 4, 4), None),
+    (1, 4, (2, 2, 2, 16), "next_loop"),   # draft tokens on a Next-loop chained cache (CUDA cores)
+    (2, 4, (2, 2, 2, 4), "next_loop"),    # 8 rows of a chain: two passes of 4 by default
 ])
 def test_multi_query_decode(librq, gq, n_q, bits, kernel):
     """n_q draft tokens per sequence in one call: every draft token sees the
     cache, the earlier tail tokens and the draft tokens up to itself."""
     rq = librq
     wl = synth.Workload(name=f"multi_{gq}_{n_q}", batch=3, kv_heads=2, q_heads=2 * gq, context=300, bits=bits,
-                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, n_tail=n_q + 1, seed=110 + n_q + gq)
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, n_tail=n_q + 1, seed=110 + n_q + gq,
+                        anchor_policy=4 if kernel == "next_loop" else 0)
     wl = wl.with_(lengths=(300, 0, 129))
     inp = synth.make_inputs(wl, "cpu")
     qm = synth.draft_queries(wl, n_q, "cpu")
