@@ -82,28 +82,44 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     kr0 = *reinterpret_cast<const uint2*>(P.k_tail + off);
     vr0 = *reinterpret_cast<const uint2*>(P.v_tail + off);
   }
+  // CTA range [c0, c1] of the split kernel that covered this segment
+  const int64_t ts = pre * P.Hkv + static_cast<int64_t>(h) * nt_b;
+  const int64_t c0 = nt_b > 0 ? ((ts + 1) * P_eff - 1) / total : 0;
+  const int64_t c1 = nt_b > 0 ? ((ts + nt_b) * P_eff - 1) / total : -1;
+  const float* rec0 = P.partials + ((static_cast<int64_t>(b) * P.Hkv + h + c0) * G + gi) * kPartialFloats;
   pdl_wait();  // the split kernel's partials are complete and visible from here on
 
+  // the first kPre partials are loaded together (one memory round trip), then
+  // merged in CTA order like the rest
+  constexpr int kPre = 4;
+  const int64_t npart = c1 - c0 + 1;
+  float4 pml[kPre], pr[kPre], ps[kPre];
+#pragma unroll
+  for (int u = 0; u < kPre; ++u) {
+    if (u < npart) {
+      const float* rec = rec0 + static_cast<int64_t>(u) * G * kPartialFloats;
+      pml[u] = reinterpret_cast<const float4*>(rec)[0];
+      pr[u] = reinterpret_cast<const float4*>(rec + 4)[lane];
+      ps[u] = reinterpret_cast<const float4*>(rec + 4 + kD)[lane];
+    }
+  }
   float m = -INFINITY, l = 0.f;
   float4 ar = make_float4(0.f, 0.f, 0.f, 0.f), as = ar;
-  if (nt_b > 0) {
-    const int64_t ts = pre * P.Hkv + static_cast<int64_t>(h) * nt_b;
-    const int64_t te = ts + nt_b;
-    const int64_t c0 = ((ts + 1) * P_eff - 1) / total;
-    const int64_t c1 = (te * P_eff - 1) / total;
-    const int pair = b * P.Hkv + h;
-    for (int64_t c = c0; c <= c1; ++c) {
-      const float* rec = P.partials + ((pair + c) * G + gi) * kPartialFloats;
-      const float4 ml = reinterpret_cast<const float4*>(rec)[0];
-      const float4 r = reinterpret_cast<const float4*>(rec + 4)[lane];
-      const float4 s = reinterpret_cast<const float4*>(rec + 4 + kD)[lane];
-      const float mn = fmaxf(m, ml.x);
-      const float a = exp2f(m - mn), bb = exp2f(ml.x - mn);
-      l = mix(l, a, ml.y, bb);
-      ar = make_float4(mix(ar.x, a, r.x, bb), mix(ar.y, a, r.y, bb), mix(ar.z, a, r.z, bb), mix(ar.w, a, r.w, bb));
-      as = make_float4(mix(as.x, a, s.x, bb), mix(as.y, a, s.y, bb), mix(as.z, a, s.z, bb), mix(as.w, a, s.w, bb));
-      m = mn;
-    }
+  auto merge = [&](const float4& ml, const float4& r, const float4& s) {
+    const float mn = fmaxf(m, ml.x);
+    const float a = exp2f(m - mn), bb = exp2f(ml.x - mn);
+    l = mix(l, a, ml.y, bb);
+    ar = make_float4(mix(ar.x, a, r.x, bb), mix(ar.y, a, r.y, bb), mix(ar.z, a, r.z, bb), mix(ar.w, a, r.w, bb));
+    as = make_float4(mix(as.x, a, s.x, bb), mix(as.y, a, s.y, bb), mix(as.z, a, s.z, bb), mix(as.w, a, s.w, bb));
+    m = mn;
+  };
+#pragma unroll
+  for (int u = 0; u < kPre; ++u)
+    if (u < npart) merge(pml[u], pr[u], ps[u]);
+  for (int64_t u = kPre; u < npart; ++u) {
+    const float* rec = rec0 + u * G * kPartialFloats;
+    merge(reinterpret_cast<const float4*>(rec)[0], reinterpret_cast<const float4*>(rec + 4)[lane],
+          reinterpret_cast<const float4*>(rec + 4 + kD)[lane]);
   }
   // current (tail) tokens in bf16
   if (n_vis > 0) {
