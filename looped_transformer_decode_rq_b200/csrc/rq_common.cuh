@@ -34,16 +34,36 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
-// Programmatic dependent launch (sm_90 and later).  A split kernel lets the
-// combine kernel that follows it on the stream (launched with programmatic
-// stream serialization) be scheduled at once; the combine kernel does its
-// input-only set-up, then waits in pdl_wait() until the split grid has
-// completed and its writes are visible.  This takes the combine kernel's launch
-// and set-up off the critical path.
+// Programmatic dependent launch (sm_90 and later).  Each decode kernel lets the
+// kernel that follows it on the stream (launched with programmatic stream
+// serialization) be scheduled early; the follower does its input-only set-up,
+// then waits in pdl_wait() until its predecessor has completed and its writes
+// are visible.  This takes launches and set-up off the critical path.
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launches `kern` as a programmatic dependent of the previous kernel on
+// stream `s`: it may be scheduled once that kernel has called
+// pdl_launch_dependents() (or exited), and must call pdl_wait() before it
+// touches memory the previous kernel writes or reads.
+template <typename... Params, typename... Args>
+inline cudaError_t launch_dependent(void (*kern)(Params...), unsigned grid, unsigned block, size_t smem,
+                                    cudaStream_t s, Args&&... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");

@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
   const int lane = threadIdx.x & 31;
   const int wid = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int Hq = P.Hkv * G;
+  pdl_launch_dependents();  // the next call's split kernel may be scheduled (it waits for this grid)
   if (wid >= P.B * Hq) {
     if constexpr (APPEND) {
       pdl_wait();  // the split kernel reads the pages these positions are written into
@@ -231,24 +232,14 @@ cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_gr
   const int rot = (res_bits != 0 && p.rotate) ? 1 : 0;
   // programmatic dependent launch: scheduled while the split kernel runs, the
   // combine kernel waits for it in pdl_wait()
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   if (enc_warps > 0) {
-    cfg.gridDim = dim3(static_cast<unsigned>((warps + enc_warps + 3) / 4), 1, 1);
-    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<true>, p, p.G, rot, *append);
+    e = launch_dependent(decode_combine_kernel<true>, static_cast<unsigned>((warps + enc_warps + 3) / 4), 128, 0, s,
+                         p, p.G, rot, *append);
   } else {
     EncodeParams none;
     memset(&none, 0, sizeof(none));
-    cfg.gridDim = dim3(static_cast<unsigned>((warps + 3) / 4), 1, 1);
-    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<false>, p, p.G, rot, none);
+    e = launch_dependent(decode_combine_kernel<false>, static_cast<unsigned>((warps + 3) / 4), 128, 0, s, p, p.G,
+                         rot, none);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

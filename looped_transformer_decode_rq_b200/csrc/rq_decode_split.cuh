@@ -281,6 +281,11 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int B = P.B, Hkv = P.Hkv;
+  // Launched as a programmatic dependent of the previous kernel on the stream
+  // (typically the previous call's combine kernel, which reads the partials
+  // this grid writes): everything above overlaps its tail; nothing global is
+  // touched before it has completed.
+  pdl_wait();
 
   // ---- page counts and their prefix over sequences
   for (int b = tid; b < B; b += kNT) {
@@ -846,8 +851,7 @@ cudaError_t launch_split(DecodeParams& p, const CUtensorMap* tk, const CUtensorM
     if (e != cudaSuccess) return e;
     attr_done = true;
   }
-  kern<<<p.num_ctas, C::NT, C::SMEM_BYTES, s>>>(p, *tk, *tv);
-  return cudaGetLastError();
+  return launch_dependent(kern, p.num_ctas, C::NT, C::SMEM_BYTES, s, p, *tk, *tv);
 }
 
 using SplitFn = cudaError_t (*)(DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);

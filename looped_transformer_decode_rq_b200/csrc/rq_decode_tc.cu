@@ -390,6 +390,7 @@ __global__ void __launch_bounds__(kNT, 1)
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int B = P.B, Hkv = P.Hkv;
+  pdl_wait();  // programmatic dependent of the previous kernel: no global access before it completed
 
   // ---- pages per sequence and their prefix (pre[b+1] - pre[b] = pages of b)
   if (warp == 0) {
@@ -1155,8 +1156,7 @@ cudaError_t launch_tc(const DecodeParams& p, const CUtensorMap* tk, const CUtens
       if (e != cudaSuccess) return e;
       attr_done = true;
     }
-    kern<<<p.num_ctas, kNT, C::SMEM_BYTES, s>>>(p, *tk, *tv);
-    return cudaGetLastError();
+    return launch_dependent(kern, p.num_ctas, kNT, C::SMEM_BYTES, s, p, *tk, *tv);
   }
 }
 
