@@ -51,7 +51,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["rq", "reference"], default="rq")
-    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "tiny", "capacity", "mixed_sweep"],
+    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "next_loop", "next_loop_int4", "tiny", "capacity",
+                                           "mixed_sweep"],
                     default="ouro8k")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -69,6 +70,10 @@ def make_workload(args) -> synth.Workload:
         return synth.mixed_int4_anchor(batch=args.batch or 8)
     if args.workload == "gqa":
         return synth.gqa_long(batch=args.batch or 8)
+    if args.workload == "next_loop":
+        return synth.ouro_8k_next_loop(batch=args.batch or 16)
+    if args.workload == "next_loop_int4":
+        return synth.ouro_8k_next_loop_int4(batch=args.batch or 16)
     return synth.tiny()
 
 
