@@ -451,3 +451,43 @@ def test_multi_query_of_one_token_is_the_single_decode(librq):
     with pytest.raises(rq.RQError) as e:
         cache.decode_attention_multi(0, q2, ctx, kt, vt)
     assert e.value.status == rq.ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("G,kernel", [(1, "simt"), (4, "tensor")])
+def test_maximum_batch(librq, G, kernel):
+    """RQ_MAX_BATCH sequences of ragged, partly empty lengths (the per-sequence
+    page prefix lives in shared memory); sampled sequences against the oracle."""
+    rq = librq
+    B = rq.MAX_BATCH
+    wl = synth.Workload(name=f"max_batch_G{G}", batch=B, kv_heads=1, q_heads=G, context=70,
+                        length_range=(0, 70), sigma=(0.3, 0.2, 0.1), seed=130 + G)
+    inp = synth.make_inputs(wl, "cpu")
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    cache.set_decode_kernel(rq.DECODE_KERNEL_SIMT if kernel == "simt" else rq.DECODE_KERNEL_TENSOR)
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    ctx = inp["ctx_len"]
+    idx = np.array([0, 1, 2, 511, 777, B - 2, B - 1])
+    sub = O.CacheConfig.from_dict(cfgd)
+    enc = O.encode_fp32emu(to_np32(inp["k"])[:, idx], to_np32(inp["v"])[:, idx], sub)
+    for loop in (0, 3):
+        out = cache.decode_attention(loop, inp["q"][loop].cuda(), ctx.cuda(), inp["k_tail"][loop].cuda(),
+                                     inp["v_tail"][loop].cuda())
+        torch.cuda.synchronize()
+        want = O.decode_attention_f64(enc, loop, to_np32(inp["q"][loop])[idx], ctx.numpy()[idx],
+                                      to_np32(inp["k_tail"][loop])[idx], to_np32(inp["v_tail"][loop])[idx])
+        err = rel_err_rows(out.cpu().numpy()[idx], want)
+        assert err.max() <= ATTN_TOL, (loop, float(err.max()))
+    assert cache.get_error() == 0
+
+
+def test_batch_beyond_maximum_is_refused(librq):
+    rq = librq
+    wl = synth.Workload(name="over_max_batch", batch=rq.MAX_BATCH + 1, kv_heads=1, q_heads=1, context=3, seed=140)
+    inp = synth.make_inputs(wl, "cpu")
+    cache = rq.Cache(rq.config_from_dict(synth.cache_config_dict(wl)), device="cuda")
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    with pytest.raises(rq.RQError) as e:
+        cache.decode_attention(0, inp["q"][0].cuda(), inp["ctx_len"].cuda())
+    assert e.value.status == rq.ERR_UNSUPPORTED
+    assert cache.get_error() == 0

@@ -147,3 +147,38 @@ def test_non_finite_input_sets_device_flag(librq):
     k[1, 0, 0, 2, 7] = 1e5  # beyond the fp16 range of the metadata
     cache.encode(k.cuda(), inp["v"].cuda())
     assert cache.get_error() & rq.FLAG_BAD_INPUT
+
+
+@pytest.mark.parametrize("policy", [0, 4])
+def test_degenerate_vectors_bit_exact(librq, policy):
+    """Zero anchor vectors (alpha = 0), exact multiples of the reference (zero
+    residual, zero scale, codes 0), constant vectors (min = max) and signed
+    zeros, under the Last-loop and the Next-loop policies: the GPU matches the
+    oracle bit for bit and decodes within tolerance."""
+    rq = librq
+    wl = synth.Workload(name=f"degenerate_{policy}", batch=2, kv_heads=2, q_heads=2, context=9,
+                        sigma=(0.3, 0.2, 0.1), anchor_policy=policy, seed=18)
+    inp = synth.make_inputs(wl, "cpu")
+    k, v = inp["k"].clone(), inp["v"].clone()
+    k[3, 0, 0, 0] = 0.0                       # zero anchor vector
+    k[:3, 0, 0, 0] = 0.5                      # constant loops against it
+    k[2, 0, 1, 1] = k[3, 0, 1, 1] * 2         # exact multiple of the anchor
+    k[1, 0, 1, 1] = k[2, 0, 1, 1] * -0.5      # ... and of the neighbour (Next-loop)
+    v[:, 1, 0, 2] = -0.0                      # signed zeros everywhere
+    v[0, 1, 1, 3] = 1.25                      # one constant vector
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    cache.encode(k.cuda(), v.cuda())
+    assert cache.get_error() == 0
+    planes = read_planes(cache, wl.context)
+    enc = O.encode_fp32emu(to_np32(k), to_np32(v), O.CacheConfig.from_dict(cfgd))
+    assert not enc.error
+    compare_encoded(planes, enc)
+    ctx = inp["ctx_len"]
+    for loop in range(wl.num_loops):
+        out = cache.decode_attention(loop, inp["q"][loop].cuda(), ctx.cuda(), inp["k_tail"][loop].cuda(),
+                                     inp["v_tail"][loop].cuda())
+        torch.cuda.synchronize()
+        want = O.decode_attention_f64(enc, loop, to_np32(inp["q"][loop]), ctx.numpy(),
+                                      to_np32(inp["k_tail"][loop]), to_np32(inp["v_tail"][loop]))
+        assert rel_err_rows(out.cpu().numpy(), want).max() <= 2e-3
