@@ -16,7 +16,12 @@
  *  - Memory: the caller owns all device memory and streams.  The library
  *    allocates nothing on the device; a cache handle holds only host metadata.
  *  - Asynchrony: calls that take a cudaStream_t enqueue work on that stream and
- *    return without synchronising (rq_get_error is the one exception).
+ *    return without synchronising (rq_get_error is the one exception).  The
+ *    decode kernels are launched as programmatic dependents (CUDA's
+ *    programmatic stream serialization): a decode kernel may be scheduled
+ *    while the previous kernel on the stream finishes, but it touches no
+ *    global memory before that kernel has completed, so stream order is kept;
+ *    this also holds inside captured CUDA graphs.
  *  - Errors: argument errors are detected on the host before anything is
  *    enqueued and are returned as RQ_ERR_INVALID_ARG / RQ_ERR_UNSUPPORTED /
  *    RQ_ERR_CAPACITY / RQ_ERR_WORKSPACE; a failed launch returns RQ_ERR_CUDA.
