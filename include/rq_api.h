@@ -260,8 +260,8 @@ RQ_API rq_status rq_decode_workspace_size(const rq_cache* cache, int64_t* bytes_
  * with beta_0 = 1 and beta_(i+1) = beta_i * alpha_K of c_i per token (alpha_V
  * likewise for the value sums); it runs on the CUDA-core kernel only.  An
  * anchor loop is plain attention over its bf16 or INT4 planes.  n_tail current tokens (bf16,
- * not yet encoded) join the softmax.  Split-K over pages (64 tokens on the
- * CUDA-core kernel, 128 on the tensor-core kernel) with an online softmax,
+ * not yet encoded) join the softmax.  Split-K over pages (64 or 128 tokens on
+ * the CUDA-core kernel, 128 on the tensor-core kernel) with an online softmax,
  * merged by a second kernel.
  *
  *  q          device bf16 [B][Hq][128]
