@@ -132,6 +132,7 @@ PINS = [
     lambda: P.test_chained_reconstruction_error_is_the_quantiser_error(O.ANCHOR_NEXT, 16),
     lambda: P.test_chained_decode_equals_brute_force(O.ANCHOR_NEXT, 4),
     P.test_multi_query_decode_equals_masked_brute_force,
+    lambda: P.test_encoder_chain_view_is_the_decoders_reconstruction(O.ANCHOR_NEXT, 16, 1),
 ]
 
 

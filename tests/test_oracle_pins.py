@@ -592,3 +592,30 @@ def test_multi_query_decode_equals_masked_brute_force():
                 P_ = np.exp(S - S.max(1, keepdims=True))
                 want = (P_ @ Vall) / P_.sum(1, keepdims=True)
                 assert np.abs(got[b, :, qh] - want).max() <= 1e-12 * max(1.0, np.abs(want).max())
+
+
+@pytest.mark.parametrize("policy,anchor_bits,rotate", [(O.ANCHOR_NEXT, 16, 1), (O.ANCHOR_PREVIOUS, 4, 1),
+                                                       (O.ANCHOR_NEXT, 4, 0)])
+def test_encoder_chain_view_is_the_decoders_reconstruction(policy, anchor_bits, rotate):
+    """The binary32 view the encoder keeps of a chained reference equals the
+    float64 reconstruction a decoder forms from the stored codes, up to binary32
+    rounding: the two are written independently (fast transform in binary32
+    against an explicit matrix in float64)."""
+    rng = np.random.default_rng(100)
+    L = 4
+    anchor = 0 if policy == O.ANCHOR_PREVIOUS else L - 1
+    bits = [2] * L
+    bits[anchor] = anchor_bits
+    rot = [rotate] * L
+    rot[anchor] = 0
+    cfg = O.CacheConfig(L, bits, [32] * L, rot, [0, 3, 0, 0], policy)
+    K = _neighbour_chain_loops(rng, cfg, (2, 2, 30, 128))
+    V = _neighbour_chain_loops(rng, cfg, (2, 2, 30, 128))
+    enc = O.encode_fp32emu(K, V, cfg)
+    for l in range(L):
+        if cfg.is_anchor(l) or l not in enc.hat32:
+            continue
+        kh, vh = O.reconstruct_f64(enc, l)
+        for view, ref in ((enc.hat32[l]["k"], kh), (enc.hat32[l]["v"], vh)):
+            scale = np.abs(ref).max(-1, keepdims=True) + 1e-30
+            assert np.abs(view.astype(np.float64) - ref).max() <= 2e-6 * scale.max()
