@@ -514,8 +514,10 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int3
   // reuse one workspace)
   for (int row0 = 0; row0 < rows; row0 += G) {
     p.row0 = row0;
+    // the step's append rides with the last block's combine, after every block has read the cache
+    const rq::EncodeParams* app = row0 + G >= rows ? append : nullptr;
     cudaError_t e = rq::launch_decode(p, ref_kind, res_bits, res_group, cache->decode_kernel, &cache->tm_anchor[a][0],
-                                      &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream), append);
+                                      &cache->tm_anchor[a][1], static_cast<cudaStream_t>(stream), app);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   }
   return RQ_OK;
