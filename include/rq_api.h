@@ -29,6 +29,9 @@
  *    capacity, a pipeline wait that timed out) set bits of the cache's device
  *    status word, read by rq_get_error.  rq_last_error_message() returns a
  *    human-readable reason for the calling thread's last non-OK status.
+ *  - Devices: one process drives one device (one process per GPU).  Each decode
+ *    kernel's shared-memory attribute is set once per process, on the device
+ *    current at its first launch.
  *  - Loop index is 0-based; by default loop num_loops-1 is every loop's reference.
  *  - head_dim is 128 everywhere (the rotation is the order-128 Hadamard).
  *  - All tensors are row-major and contiguous unless strides are passed.
