@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the mixed INT4-anchor and GQA side lines")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="skip the mixed-format batch sweep and the 24-layer capacity sweep")
     return ap.parse_args()
 
 
@@ -310,6 +312,29 @@ def time_steps(step, steps, warmup, world, stream):
     return max_over_ranks(a.elapsed_time(b) / steps, world)
 
 
+def workload_config(wl, world):
+    """The `config` object of a bench line (the same keys for both arms)."""
+    return {"workload": wl.name, "global_batch": wl.batch * world, "seq_len": wl.context, "loops": wl.num_loops,
+            "kv_heads": wl.kv_heads, "q_heads": wl.q_heads, "head_dim": 128, "bits": list(wl.bits),
+            "group": list(wl.group), "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (>= 1 GB read per call), no flush"}
+
+
+def residual_call_ms(call, stream, reps=50, warmup=5):
+    """Mean device time of one decode call issued `reps` times back to back
+    (one event pair around the whole run, none between the calls)."""
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps, reps
+
+
 def measure_workload(wl, steps, warmup, world, rank, per_loop=False):
     """RQ decode step and bf16-cache step of one workload (side lines of the
     main result): tokens/s, residual-loop GB/s and the speed-up over bf16."""
@@ -336,33 +361,20 @@ def measure_workload(wl, steps, warmup, world, rank, per_loop=False):
                                       out=outs[L - 1])
 
     ms = time_steps(rq_step, steps, warmup, world, stream)
-    ev = []
-    for _ in range(5):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
-        b.record(stream)
-        ev.append((a, b))
-    torch.cuda.synchronize()
-    call_ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    def loop_call(l):
+        return lambda: cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
+
+    call_ms, _ = residual_call_ms(loop_call(0), stream, reps=20)
     res_bytes = call_bytes(cache.layout, cfgd, 0, tokens_total, B, Hq, Hkv, 1)
 
     def call_gbs(kernel):
         cache.set_decode_kernel(kernel)
         try:
-            for _ in range(3):
-                cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
-            evs = []
-            for _ in range(7):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0], out=outs[0])
-                b.record(stream)
-                evs.append((a, b))
-            torch.cuda.synchronize()
+            t, _ = residual_call_ms(loop_call(0), stream, reps=10, warmup=3)
         finally:
             cache.set_decode_kernel(rq.DECODE_KERNEL_AUTO)
-        return round(res_bytes / (statistics.median(a.elapsed_time(b) for a, b in evs) * 1e-3) / 1e9, 1)
+        return round(res_bytes / (t * 1e-3) / 1e9, 1)
 
     per_kernel = {"simt": call_gbs(rq.DECODE_KERNEL_SIMT)}
     if wl.gqa in (1, 2, 4, 8):
@@ -381,18 +393,9 @@ def measure_workload(wl, steps, warmup, world, rank, per_loop=False):
     if per_loop:  # every loop's decode call alone (a chained policy reads more links for farther loops)
         loop_gbs = {}
         for l in range(L):
-            evs = []
-            for i in range(8):
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
-                b.record(stream)
-                if i >= 3:
-                    evs.append((a, b))
-            torch.cuda.synchronize()
+            t, _ = residual_call_ms(loop_call(l), stream, reps=10, warmup=3)
             lb = call_bytes(cache.layout, cfgd, l, tokens_total, B, Hq, Hkv, 1)
-            loop_gbs[str(l)] = {"bytes": lb, "gbs": round(lb / (statistics.median(a.elapsed_time(b) for a, b in evs)
-                                                                 * 1e-3) / 1e9, 1)}
+            loop_gbs[str(l)] = {"bytes": lb, "gbs": round(lb / (t * 1e-3) / 1e9, 1)}
     flags = cache.get_error()
     out = {"workload": wl.name, "tokens_per_s": round(job_tokens_per_s(B, world, ms), 1),
            "ms_per_step": round(ms, 4), "residual_loop_gbs": round(res_bytes / (call_ms * 1e-3) / 1e9, 1),
@@ -439,15 +442,8 @@ def measure_multi_query(wl, n_q, steps, warmup, world, rank):
 
     ms = time_steps(multi_step, steps, warmup, world, stream)
     ms1 = time_steps(single_step, steps, warmup, world, stream)
-    ev = []
-    for _ in range(8):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        cache.decode_attention_multi(0, qm[0], ctx, kt[0], vt[0], out=outs[0])
-        b.record(stream)
-        ev.append((a, b))
-    torch.cuda.synchronize()
-    call_ms = statistics.median(a.elapsed_time(b) for a, b in ev[3:])
+    call_ms, _ = residual_call_ms(lambda: cache.decode_attention_multi(0, qm[0], ctx, kt[0], vt[0], out=outs[0]),
+                                  stream, reps=10, warmup=3)
     res_bytes = (tokens_total * Hkv * record_bytes(cache.layout, cfgd, 0) + B * n_q * Hq * 128 * (2 + 4) +
                  B * Hkv * n_q * 512)
     flags = cache.get_error()
@@ -462,21 +458,21 @@ def measure_multi_query(wl, n_q, steps, warmup, world, rank):
     return out
 
 
-def run_capacity(args, world, rank):
-    """24-layer, 4-loop model at 8192 context: the largest batch whose caches
-    fit in HBM for a bf16 cache and for ResidualQuant caches (bf16 anchor and
-    INT4 anchor), and decode tokens/s of the full 24-layer attention step at
-    that batch.  One synthetic sequence is encoded into every (layer, sequence)
-    slot, each with its own cache memory: the timing does not depend on the
-    values."""
+def measure_capacity(steps, warmup, world, rank, fractions=(1.0,)):
+    """24-layer, 4-loop model at 8192 context: for a bf16 cache and for
+    ResidualQuant caches (bf16 anchor, INT4 anchor), the largest batch whose 24
+    layers of caches fit in HBM, and decode tokens/s of the full 24-layer
+    attention step at `fractions` of that batch (1.0: the largest).  One
+    synthetic sequence is encoded into every (layer, sequence) slot, each with
+    its own cache memory: the timing does not depend on the values."""
     from looped_transformer_decode_rq_b200 import rq
     dev = torch.device("cuda", torch.cuda.current_device())
     layers, T = 24, 8192
     base = synth.capacity_24layer(batch=1, context=T)
     L, Hkv, Hq = base.num_loops, base.kv_heads, base.q_heads
-    steps, warmup = max(2, min(args.steps, 5)), 3
     stream = torch.cuda.current_stream()
     one = synth.make_inputs(base.with_(batch=1, n_tail=1), dev)  # [L, 1, Hkv, T, 128]
+    torch.cuda.empty_cache()
     free, _ = torch.cuda.mem_get_info()
     budget = int(free * 0.9) - (2 << 30)
     results = {}
@@ -487,71 +483,90 @@ def run_capacity(args, world, rank):
         else:
             lay = rq.cache_layout(rq.config_from_dict(synth.cache_config_dict(base.with_(bits=bits), capacity=T + 1)))
             per_seq = layers * lay.total_bytes
-        B = int(max(1, min(1024, budget // per_seq)))
-        wl = base.with_(batch=B) if bits is None else base.with_(batch=B, bits=bits)
-        q = one["q"].expand(-1, B, -1, -1).contiguous()
-        ctx = torch.full((B,), T, dtype=torch.int32, device=dev)
-        k_new = one["k_tail"].expand(-1, B, -1, -1, -1).contiguous()
-        v_new = one["v_tail"].expand(-1, B, -1, -1, -1).contiguous()
-        outs = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
-        if fmt == "bf16":
-            caches = []
-            for _ in range(layers):
-                planes = []
-                for l in range(L):
-                    kv = torch.empty((2, B, Hkv, T + 1, 128), dtype=torch.bfloat16, device=dev)
-                    kv[0, :, :, :T].copy_(one["k"][l].expand(B, -1, -1, -1))
-                    kv[1, :, :, :T].copy_(one["v"][l].expand(B, -1, -1, -1))
-                    planes.append(kv)
-                caches.append(planes)
-            ws = torch.zeros(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
-
-            def step():
-                for planes in caches:
+        max_b = int(max(1, min(1024, budget // per_seq)))
+        points = sorted({max(1, int(round(f * max_b))) for f in fractions})
+        sweep = []
+        for B in points:
+            torch.cuda.empty_cache()
+            wl = base.with_(batch=B) if bits is None else base.with_(batch=B, bits=bits)
+            q = one["q"].expand(-1, B, -1, -1).contiguous()
+            ctx = torch.full((B,), T, dtype=torch.int32, device=dev)
+            k_new = one["k_tail"].expand(-1, B, -1, -1, -1).contiguous()
+            v_new = one["v_tail"].expand(-1, B, -1, -1, -1).contiguous()
+            outs = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
+            if fmt == "bf16":
+                caches = []
+                for _ in range(layers):
+                    planes = []
                     for l in range(L):
-                        kv = planes[l]
-                        kv[0, :, :, T:T + 1].copy_(k_new[l])   # append the new token
-                        kv[1, :, :, T:T + 1].copy_(v_new[l])
-                        rq.bf16_decode_attention(kv[0], kv[1], q[l], ctx, k_new[l], v_new[l], workspace=ws,
-                                                 out=outs[l])
-        else:
-            cfgd = synth.cache_config_dict(wl, capacity=T + 1)
-            caches = [rq.Cache(rq.config_from_dict(cfgd), device=dev) for _ in range(layers)]
-            kb = one["k"].expand(-1, B, -1, -1, -1)  # batch stride 0: the same values for every sequence
-            vb = one["v"].expand(-1, B, -1, -1, -1)
-            for c in caches:
-                c.encode(kb, vb)
+                        kv = torch.empty((2, B, Hkv, T + 1, 128), dtype=torch.bfloat16, device=dev)
+                        kv[0, :, :, :T].copy_(one["k"][l].expand(B, -1, -1, -1))
+                        kv[1, :, :, :T].copy_(one["v"][l].expand(B, -1, -1, -1))
+                        planes.append(kv)
+                    caches.append(planes)
+                ws = torch.zeros(rq.bf16_workspace_bytes(B, Hkv, Hq), dtype=torch.uint8, device=dev)
 
-            def step():
+                def step():
+                    for planes in caches:
+                        for l in range(L):
+                            kv = planes[l]
+                            kv[0, :, :, T:T + 1].copy_(k_new[l])   # append the new token
+                            kv[1, :, :, T:T + 1].copy_(v_new[l])
+                            rq.bf16_decode_attention(kv[0], kv[1], q[l], ctx, k_new[l], v_new[l], workspace=ws,
+                                                     out=outs[l])
+            else:
+                ws = None
+                cfgd = synth.cache_config_dict(wl, capacity=T + 1)
+                caches = [rq.Cache(rq.config_from_dict(cfgd), device=dev) for _ in range(layers)]
+                kb = one["k"].expand(-1, B, -1, -1, -1)  # batch stride 0: the same values for every sequence
+                vb = one["v"].expand(-1, B, -1, -1, -1)
                 for c in caches:
-                    for l in range(L - 1):
-                        c.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
-                    c.decode_attention_append(L - 1, q[L - 1], ctx, k_new[L - 1], v_new[L - 1], k_new, v_new, ctx,
-                                              out=outs[L - 1])
-        ms = time_steps(step, steps, warmup, world, stream)
-        flags = 0 if fmt == "bf16" else max(c.get_error() for c in caches)
-        results[fmt] = {"max_batch": B, "bytes_per_sequence": int(per_seq),
-                        "tokens_per_s": round(job_tokens_per_s(B, world, ms), 1), "ms_per_step": round(ms, 3),
-                        "device_flags": int(flags)}
-        del caches, q, ctx, k_new, v_new, outs
-        torch.cuda.empty_cache()
+                    c.encode(kb, vb)
+
+                def step():
+                    for c in caches:
+                        for l in range(L - 1):
+                            c.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
+                        c.decode_attention_append(L - 1, q[L - 1], ctx, k_new[L - 1], v_new[L - 1], k_new, v_new,
+                                                  ctx, out=outs[L - 1])
+            ms = time_steps(step, steps, warmup, world, stream)
+            flags = 0 if fmt == "bf16" else max(c.get_error() for c in caches)
+            sweep.append({"batch": B, "tokens_per_s": round(job_tokens_per_s(B, world, ms), 1),
+                          "ms_per_step": round(ms, 3), "device_flags": int(flags)})
+            del caches, q, ctx, k_new, v_new, outs, ws
+            torch.cuda.empty_cache()
+        top = sweep[-1]
+        results[fmt] = {"max_batch": max_b, "bytes_per_sequence": int(per_seq),
+                        "tokens_per_s": top["tokens_per_s"], "ms_per_step": top["ms_per_step"],
+                        "peak_tokens_per_s": max(r["tokens_per_s"] for r in sweep),
+                        "device_flags": max(r["device_flags"] for r in sweep), "sweep": sweep}
+    del one
+    torch.cuda.empty_cache()
+    return {"workload": "capacity_24layer_L4_H16_T8192", "metric": "decode tokens/s of the 24-layer attention step "
+            "against batch, up to the largest batch whose caches fit", "results": results,
+            "peak_vs_bf16": {k: round(v["peak_tokens_per_s"] / results["bf16"]["peak_tokens_per_s"], 3)
+                             for k, v in results.items()},
+            "max_batch_vs_bf16": {k: round(v["max_batch"] / results["bf16"]["max_batch"], 2)
+                                  for k, v in results.items()},
+            "hbm_budget_bytes": budget, "steps": steps, "warmup": warmup, "data": "synthetic", "n_gpus": world}
+
+
+def run_capacity(args, world, rank):
+    out = measure_capacity(max(2, min(args.steps, 5)), 3, world, rank, fractions=(0.25, 0.5, 0.75, 1.0))
     if rank == 0:
-        print(json.dumps({"workload": "capacity_24layer_L4_H16_T8192", "metric": "decode tokens/s at the largest "
-                          "batch whose 24-layer caches fit (attention only)", "results": results,
-                          "hbm_budget_bytes": budget, "data": "synthetic", "n_gpus": world}))
+        print(json.dumps(out))
 
 
-def run_mixed_sweep(args, world, rank):
-    """Mixed-precision format [2,2,4,4] with an INT4 anchor at 8k context,
-    batch 1 / 8 / 32 / 64: the decode step (4 loop decodes + append-encode of the
-    new token) against the bf16-cache step on the same values, and the
+def measure_mixed_sweep(steps, warmup, world, rank, batches=(1, 8, 32, 64)):
+    """Mixed-precision format [2,2,4,4] with an INT4 anchor at 8k context, batch
+    1 / 8 / 32 / 64: the decode step (4 loop decodes + append-encode of the new
+    token) against the bf16-cache step on the same values, and the
     append-encode alone.  A step that reads less than twice the L2 is timed
     alone after writing a 256 MB buffer (L2 flushed between timed steps)."""
     from looped_transformer_decode_rq_b200 import rq
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    steps, warmup = max(3, min(args.steps, 20)), max(3, args.warmup)
 
     def timed(step, flush):
         for _ in range(warmup):
@@ -573,7 +588,7 @@ def run_mixed_sweep(args, world, rank):
         return max_over_ranks(total / steps, world)
 
     results = []
-    for B in (1, 8, 32, 64):
+    for B in batches:
         wl = synth.mixed_int4_anchor(batch=B).with_(seed=2 + 1000 * rank)
         inp = synth.make_inputs(wl, dev)
         L, Hkv, Hq, T = wl.num_loops, wl.kv_heads, wl.q_heads, wl.context
@@ -586,9 +601,7 @@ def run_mixed_sweep(args, world, rank):
         q = inp["q"]
         outs = torch.empty((L, B, Hq, 128), dtype=torch.float32, device=dev)
         lay = cache.layout
-        step_bytes = sum(B * Hkv * T * (2 * (lay.codes_record_bytes[lay.anchor_of[l]] + lay.meta_record_bytes[lay.anchor_of[l]])
-                                        + (2 * (lay.codes_record_bytes[l] + lay.meta_record_bytes[l]) + 4
-                                           if lay.anchor_of[l] != l else 0)) for l in range(L))
+        step_bytes = sum(B * Hkv * T * record_bytes(lay, cfgd, l) for l in range(L))
         flush = step_bytes < 2 * (126 << 20)
 
         def rq_step():
@@ -619,11 +632,17 @@ def run_mixed_sweep(args, world, rank):
                         "l2_flushed": flush, "device_flags": int(flags)})
         del cache, inp, outs, ws
         torch.cuda.empty_cache()
+    del flush_buf
+    torch.cuda.empty_cache()
+    return {"workload": "mixed_2244_H16_T8192_int4ref_batch_sweep",
+            "metric": "decode step tokens/s (4 loops + append-encode) vs BF16 cache",
+            "results": results, "steps": steps, "warmup": warmup, "data": "synthetic", "n_gpus": world}
+
+
+def run_mixed_sweep(args, world, rank):
+    out = measure_mixed_sweep(max(3, min(args.steps, 20)), max(3, args.warmup), world, rank)
     if rank == 0:
-        print(json.dumps({"workload": "mixed_2244_H16_T8192_int4ref_batch_sweep",
-                          "metric": "decode step tokens/s (4 loops + append-encode) vs BF16 cache",
-                          "results": results, "steps": steps, "warmup": warmup, "data": "synthetic",
-                          "n_gpus": world}))
+        print(json.dumps(out))
 
 
 def run_rq(args, world, rank):
@@ -633,7 +652,9 @@ def run_rq(args, world, rank):
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = synth.make_inputs(wl, dev)
     L, B, Hkv, Hq, T = wl.num_loops, wl.batch, wl.kv_heads, wl.q_heads, wl.context
-    cfgd = synth.cache_config_dict(wl, capacity=T + 1)
+    # room for the end-to-end leg, whose decode run grows the cache by a token per step
+    e2e_warm = 3
+    cfgd = synth.cache_config_dict(wl, capacity=T + 1 + (0 if args.no_e2e else e2e_warm + args.steps))
     cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
     cache.encode(inp["k"], inp["v"])
     ctx = inp["ctx_len"]
@@ -647,19 +668,11 @@ def run_rq(args, world, rank):
     stream = torch.cuda.current_stream()
     n_tail = 1
 
-    ev_pairs = []
-
-    def step(record=False):
+    def step():
         # loops 0 .. L-2, then the final loop's decode with the new token's
         # append-encode (every loop) fused into its combine launch
         for l in range(L - 1):
-            if record:
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
             cache.decode_attention(l, q[l], ctx, k_new[l], v_new[l], out=outs[l])
-            if record:
-                e1.record(stream)
-                ev_pairs.append((e0, e1))
         cache.decode_attention_append(L - 1, q[L - 1], ctx, k_new[L - 1], v_new[L - 1], k_new, v_new, pos,
                                       out=outs[L - 1])
 
@@ -689,14 +702,19 @@ def run_rq(args, world, rank):
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for _ in range(args.steps):
-        step(record=True)
+        step()
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end) / args.steps
     ms = max_over_ranks(ms, world)
-    call_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_pairs)
+    # Per-launch time of the dominant call (a residual loop's split + combine),
+    # in a pass of its own so that no event sits inside the timed steps: the
+    # call is issued back to back, as in the step, where each split kernel
+    # overlaps the previous combine (programmatic dependent launches).
+    call_ms, call_reps = residual_call_ms(lambda: cache.decode_attention(0, q[0], ctx, k_new[0], v_new[0],
+                                                                         out=outs[0]), stream)
     flags |= cache.get_error()
 
     res_bytes = call_bytes(lay, cfgd, 0, tokens_total, B, Hq, Hkv, n_tail)
@@ -712,39 +730,49 @@ def run_rq(args, world, rank):
     # ---- e2e through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        # Every step copies its inputs from pinned host memory and its outputs
-        # back.  As in a serving loop, the copies run on their own streams and
-        # overlap the neighbouring steps' decode (inputs and outputs double-
-        # buffered, ordered by events); the timed region spans the first
-        # input copy to the last output copy.
+        # A decode run through the public API: every step copies its inputs
+        # (the queries, the new token of every loop and the context lengths)
+        # from pinned host memory and its outputs back, and the cache grows by
+        # one token per step (step i attends ctx_len + i cached tokens plus the
+        # new token, which it appends at position ctx_len + i).  As in a serving
+        # loop, the copies run on their own streams and overlap the neighbouring
+        # steps' decode (inputs and outputs double-buffered, ordered by events);
+        # the timed region spans the first input copy to the last output copy.
         hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q.cpu())
         hk = torch.empty(k_new.shape, dtype=k_new.dtype, pin_memory=True).copy_(k_new.cpu())
         hv = torch.empty(v_new.shape, dtype=v_new.dtype, pin_memory=True).copy_(v_new.cpu())
+        ctx0 = ctx.cpu()
+        n_total = e2e_warm + args.steps
+        hctx = torch.empty((n_total, B), dtype=torch.int32, pin_memory=True)
+        for i in range(n_total):
+            hctx[i].copy_(ctx0 + i)
         hout = [torch.empty(outs.shape, dtype=outs.dtype, pin_memory=True) for _ in range(2)]
-        dbuf = [(torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(outs))
-                for _ in range(2)]
+        dbuf = [(torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new), torch.empty_like(outs),
+                 torch.empty_like(ctx)) for _ in range(2)]
         h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
         ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("h2d", "comp", "d2h")}
 
-        def e2e_run(nsteps, start_ev=None):
+        def e2e_run(first, nsteps, start_ev=None):
             if start_ev is not None:
                 h2d_s.wait_event(start_ev)
             for i in range(nsteps):
                 j = i % 2
-                dq, dk, dv, do = dbuf[j]
+                dq, dk, dv, do, dctx = dbuf[j]
                 if i >= 2:
                     h2d_s.wait_event(ev["comp"][j])  # step i-2 no longer reads these inputs
                 with torch.cuda.stream(h2d_s):
                     dq.copy_(hq, non_blocking=True)
                     dk.copy_(hk, non_blocking=True)
                     dv.copy_(hv, non_blocking=True)
+                    dctx.copy_(hctx[first + i], non_blocking=True)
                 ev["h2d"][j].record(h2d_s)
                 stream.wait_event(ev["h2d"][j])
                 if i >= 2:
                     stream.wait_event(ev["d2h"][j])  # step i-2's output has left the device
                 for l in range(L - 1):
-                    cache.decode_attention(l, dq[l], ctx, dk[l], dv[l], out=do[l])
-                cache.decode_attention_append(L - 1, dq[L - 1], ctx, dk[L - 1], dv[L - 1], dk, dv, pos, out=do[L - 1])
+                    cache.decode_attention(l, dq[l], dctx, dk[l], dv[l], out=do[l])
+                cache.decode_attention_append(L - 1, dq[L - 1], dctx, dk[L - 1], dv[L - 1], dk, dv, dctx,
+                                              out=do[L - 1])
                 ev["comp"][j].record(stream)
                 d2h_s.wait_event(ev["comp"][j])
                 with torch.cuda.stream(d2h_s):
@@ -753,20 +781,21 @@ def run_rq(args, world, rank):
             stream.wait_stream(d2h_s)
             stream.wait_stream(h2d_s)
 
-        e2e_run(3)
+        e2e_run(0, e2e_warm)
         torch.cuda.synchronize()
         barrier(world)
         torch.cuda.synchronize()
         a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        e2e_run(args.steps, start_ev=a)
+        e2e_run(e2e_warm, args.steps, start_ev=a)
         b2.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         ems = max_over_ranks(a.elapsed_time(b2) / args.steps, world)
         e2e = {"value": round(job_tokens_per_s(B, world, ems), 1), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2),
+               "h2d_bytes_per_step": int(hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + B * 4),
                "d2h_bytes_per_step": int(hout[0].numel() * 4),
+               "context": f"decode run: ctx_len grows from {int(ctx0.min()) + e2e_warm} by one token per step",
                "copies": "own streams, overlapping the neighbouring steps (double-buffered)"}
 
     # ---- the same step over a bf16 cache (same library)
@@ -795,6 +824,7 @@ def run_rq(args, world, rank):
         bf16 = {"tokens_per_s": round(job_tokens_per_s(B, world, bms), 1), "ms_per_step": round(bms, 4),
                 "hbm_gbs": round(bf_bytes / (bms * 1e-3) / 1e9, 1),
                 "bytes_per_step": bf_bytes, "rq_speedup": round(bms / ms, 3)}
+        del kc, vc, ws
 
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
@@ -806,34 +836,42 @@ def run_rq(args, world, rank):
                           f"of its new token, {reps} reps of {per:.3f} s; scaled by B*Hkv={B * Hkv}")}
 
     extra = None
-    if not args.no_extra and args.workload == "ouro8k":
+    side = args.workload == "ouro8k" and not (args.no_extra and args.no_sweeps)
+    if side:  # free the main workload's memory for the side lines
         del cache, inp, outs
         torch.cuda.empty_cache()
+    if not args.no_extra and args.workload == "ouro8k":
         extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 30, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8), 30, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8, q_heads=64), 30, 3, world, rank),
                  measure_workload(synth.ouro_8k_next_loop(), 30, 3, world, rank, per_loop=True),
                  measure_workload(synth.ouro_8k_next_loop_int4(), 30, 3, world, rank, per_loop=True),
                  measure_multi_query(synth.ouro_8k(), 4, 30, 3, world, rank)]
+    sweeps = None
+    if not args.no_sweeps and args.workload == "ouro8k":
+        # the mixed-precision [2,2,4,4] batch sweep and the 24-layer capacity
+        # sweep, each its own workload (side results, not the headline)
+        sweeps = {"mixed_2244_batch_sweep": measure_mixed_sweep(10, 3, world, rank),
+                  "capacity_24layer_sweep": measure_capacity(3, 2, world, rank,
+                                                             fractions=(0.25, 0.5, 0.75, 1.0))}
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+int2 (fp32 math)",
         "data": "synthetic (seeded generator; Ouro-1.4B-shaped caches, random values)",
-        "config": {"workload": wl.name, "global_batch": B * world, "seq_len": T, "loops": L,
-                   "kv_heads": Hkv, "q_heads": Hq, "head_dim": 128, "bits": list(wl.bits),
-                   "group": list(wl.group), "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (>= 1 GB read per call), no flush"},
+        "config": workload_config(wl, world),
         "hbm_gbs_step": round(step_bytes / (ms * 1e-3) / 1e9, 1),
         "bytes_per_step": step_bytes,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "kernel": "rq_decode_attention on a residual loop (split + combine kernels)",
                      "algorithmic_bytes_per_launch": res_bytes, "launch_ms": round(call_ms, 4),
+                     "launch_timing": f"mean of {call_reps} back-to-back calls, one event pair, outside the timed steps",
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback",
                      "frac_of_8tbs": round(achieved / 8000.0, 4)},
         "cpu_baseline": cpu, "e2e": e2e, "bf16_cache": bf16, "parity": parity, "other_workloads": extra,
+        "sweeps": sweeps,
         # per step: a split and a combine kernel per loop (the final loop's combine also appends)
         "gpu_launches": args.steps * (2 * L), "clocks": clk, "device_flags": flags,
     }
@@ -842,6 +880,11 @@ def run_rq(args, world, rank):
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on the GPU arm's
+    workload.  Each step times one (sequence, kv-head) slab (decode of every
+    loop plus the encode of its new token); the full step is B*Hkv such slabs,
+    so the reported step time is that sample time times B*Hkv (stated in
+    `extrapolation`)."""
     if rank != 0:
         return
     wl = make_workload(args)
@@ -855,15 +898,19 @@ def run_reference(args, world, rank):
         sample.step()
         t.append(time.perf_counter() - t0)
     per = statistics.mean(t)
-    full = per * wl.batch * wl.kv_heads
+    slabs = wl.batch * wl.kv_heads
+    full = per * slabs
     value = wl.batch / full
     cpu = {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
            "sample": (f"one (sequence, kv-head) slab per step: decode of all {wl.num_loops} loops over "
-                      f"{wl.context} tokens + encode of the new token; scaled by B*Hkv={wl.batch * wl.kv_heads}")}
+                      f"{wl.context} tokens + encode of the new token; scaled by B*Hkv={slabs}")}
     out = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(full * 1e3, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-           "config": {"workload": wl.name, "global_batch": wl.batch, "seq_len": wl.context},
+           "config": workload_config(wl, 1),
+           "extrapolation": {"slabs_timed_per_step": 1, "slabs_per_step": slabs,
+                             "factor": slabs, "measured_ms_per_timed_step": round(per * 1e3, 3),
+                             "timed_wall_s": round(sum(t), 3)},
            "impl": "reference", "cpu_baseline": cpu,
            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out))

@@ -14,7 +14,10 @@
  *
  * Conventions shared by every entry point:
  *  - Memory: the caller owns all device memory and streams.  The library
- *    allocates nothing on the device; a cache handle holds only host metadata.
+ *    allocates nothing on the device at run time; a cache handle holds only
+ *    host metadata.  The one piece of device memory the library owns is a
+ *    fixed RQ_STATIC_SCRATCH_BYTES array that every GPU loading the library
+ *    holds until exit, used only by rq_decode_attention_static_scratch.
  *  - Asynchrony: calls that take a cudaStream_t enqueue work on that stream and
  *    return without synchronising (rq_get_error is the one exception).  The
  *    decode kernels are launched as programmatic dependents (CUDA's
@@ -342,9 +345,13 @@ RQ_API rq_status rq_decode_attention_append(rq_cache* cache, int32_t loop, const
  * computes, with the split-K partials kept in a fixed RQ_STATIC_SCRATCH_BYTES
  * array in the library's own device memory instead of a caller workspace.
  *  - It allocates nothing and calls no allocating routine.
- *  - Limit: rq_decode_workspace_size(cache) must not exceed
- *    RQ_STATIC_SCRATCH_BYTES (roughly (batch*kv_heads + SMs) * G * 1040 bytes);
- *    otherwise it returns RQ_ERR_WORKSPACE before enqueuing anything.
+ *  - Limit: the split-K partials of this decode must fit in
+ *    RQ_STATIC_SCRATCH_BYTES: (batch*kv_heads + SMs) * G * 1040 bytes, with G
+ *    the query rows of one pass over the cache (q_heads / kv_heads, or 4 where
+ *    the default decode runs 8 rows as two passes of 4); otherwise it returns
+ *    RQ_ERR_WORKSPACE before enqueuing anything.
+ *  - Device: the device current at the call must be the one the cache was
+ *    created on (RQ_ERR_INVALID_ARG otherwise).
  *  - Set-up: the first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.  Every GPU that loads the library keeps the

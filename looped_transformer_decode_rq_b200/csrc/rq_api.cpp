@@ -415,6 +415,69 @@ rq_status check_decode_common(int B, int Hkv, int Hq, const void* q, const int32
 
 namespace {
 
+// The loop's chain of residual links toward its anchor (one link unless the
+// policy is chained); returns the number of links, or -1 if longer than
+// RQ_MAX_CHAIN.
+int loop_chain(const rq_cache* cache, int loop, int (&chain)[RQ_MAX_CHAIN]) {
+  const rq_layout& lay = cache->lay;
+  const int a = lay.anchor_of[loop];
+  int n_chain = 0;
+  for (int l = loop; l != a; l = lay.ref_of[l]) {
+    if (n_chain == RQ_MAX_CHAIN) return -1;
+    chain[n_chain++] = l;
+  }
+  return n_chain;
+}
+
+// Query rows per pass over the cache (G of the kernels) for a decode of `loop`
+// with n_q query tokens per sequence: all rows up to 8, else blocks of 8.  The
+// CUDA-core kernel's 8-row variants spill registers (about a tenth of the
+// 4-row rate): by default, 8 rows that would land there run as two passes of
+// 4 rows instead (each reads the cache once more).
+rq_status block_rows(const rq_cache* cache, int loop, int n_q, int* G_out) {
+  const rq_config& c = cache->cfg;
+  if (loop < 0 || loop >= c.num_loops) return fail(RQ_ERR_INVALID_ARG, "loop %d outside [0, %d)", loop, c.num_loops);
+  if (n_q < 1 || n_q > RQ_MAX_DRAFT) return fail(RQ_ERR_INVALID_ARG, "n_q %d outside [1, %d]", n_q, RQ_MAX_DRAFT);
+  const int rows = n_q * (c.q_heads / c.kv_heads);
+  if (!rows_supported(rows))
+    return fail(RQ_ERR_UNSUPPORTED, "n_q * q_heads / kv_heads = %d (supported: 1, 2, 4, or a multiple of 8)", rows);
+  int G = rows < 8 ? rows : 8;
+  int chain[RQ_MAX_CHAIN];
+  const int n_chain = loop_chain(cache, loop, chain);
+  if (n_chain < 0) return fail(RQ_ERR_UNSUPPORTED, "reference chain longer than %d", RQ_MAX_CHAIN);
+  const int a = cache->lay.anchor_of[loop];
+  const int ref_kind = ref_kind_for(c, loop);
+  const int res_bits = loop == a ? 0 : c.bits[loop];
+  const int res_group = loop == a ? 32 : c.group[loop];
+  if (G == 8 && cache->decode_kernel == RQ_DECODE_KERNEL_AUTO &&
+      rq::decode_kernel_choice(ref_kind, res_bits, res_group, 8, RQ_DECODE_KERNEL_AUTO, n_chain > 1 ? n_chain : 1) ==
+          rq::kKernelSimt)
+    G = 4;
+  *G_out = G;
+  return RQ_OK;
+}
+
+}  // namespace
+
+}  // extern "C"
+
+namespace rq {
+rq_status decode_scratch_need(const rq_cache* cache, int loop, int n_q, int64_t* bytes_out) {
+  if (cache == nullptr || bytes_out == nullptr) return fail(RQ_ERR_INVALID_ARG, "null argument");
+  int G = 0;
+  const rq_status st = block_rows(cache, loop, n_q, &G);
+  if (st != RQ_OK) return st;
+  *bytes_out = decode_workspace_bytes(cache->cfg.batch, cache->cfg.kv_heads, G, cache->num_ctas);
+  return RQ_OK;
+}
+
+int cache_device(const rq_cache* cache) { return cache->device; }
+}  // namespace rq
+
+extern "C" {
+
+namespace {
+
 // n_q > 1: a multi-query call (q and out [B][n_q][Hq][128]; the last n_q tail
 // tokens are the draft tokens, each seen by itself and the later ones)
 rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int32_t n_q, const int32_t* ctx_len,
@@ -424,17 +487,15 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int3
   if (cache_c == nullptr) return fail(RQ_ERR_INVALID_ARG, "cache is null");
   rq_cache* cache = const_cast<rq_cache*>(cache_c);
   const rq_config& c = cache->cfg;
-  if (loop < 0 || loop >= c.num_loops) return fail(RQ_ERR_INVALID_ARG, "loop %d outside [0, %d)", loop, c.num_loops);
   const int gq = c.q_heads / c.kv_heads;
-  if (n_q < 1 || n_q > RQ_MAX_DRAFT) return fail(RQ_ERR_INVALID_ARG, "n_q %d outside [1, %d]", n_q, RQ_MAX_DRAFT);
-  const int rows = n_q * gq;  // query rows per kv-head, decoded in blocks of up to 8
-  if (!rows_supported(rows))
-    return fail(RQ_ERR_UNSUPPORTED, "n_q * q_heads / kv_heads = %d (supported: 1, 2, 4, or a multiple of 8)", rows);
-  int G = rows < 8 ? rows : 8;
+  int G = 0;  // rows per pass over the cache
+  rq_status st = block_rows(cache, loop, n_q, &G);
+  if (st != RQ_OK) return st;
+  const int rows = n_q * gq;  // query rows per kv-head, decoded in blocks of G
   if (n_q > 1 && n_tail < n_q)
     return fail(RQ_ERR_INVALID_ARG, "n_tail %d < n_q %d (the draft tokens are the last n_q tail tokens)", n_tail, n_q);
   const int64_t need = rq::decode_workspace_bytes(c.batch, c.kv_heads, G, cache->num_ctas);
-  rq_status st = check_decode_common(c.batch, c.kv_heads, c.q_heads, q, ctx_len, k_tail, v_tail, n_tail,
+  st = check_decode_common(c.batch, c.kv_heads, c.q_heads, q, ctx_len, k_tail, v_tail, n_tail,
                                      softmax_scale, out, workspace, workspace_bytes, need);
   if (st != RQ_OK) return st;
   const rq_layout& lay = cache->lay;
@@ -444,18 +505,7 @@ rq_status decode_impl(const rq_cache* cache_c, int32_t loop, const void* q, int3
   const int res_group = loop == a ? 32 : c.group[loop];
   // the loop's chain of residual links toward its anchor (one link unless chained)
   int chain[RQ_MAX_CHAIN];
-  int n_chain = 0;
-  for (int l = loop; l != a; l = lay.ref_of[l]) {
-    if (n_chain == RQ_MAX_CHAIN) return fail(RQ_ERR_UNSUPPORTED, "reference chain longer than %d", RQ_MAX_CHAIN);
-    chain[n_chain++] = l;
-  }
-  // The CUDA-core kernel's 8-row variants spill registers (about a tenth of the
-  // 4-row rate): by default, 8 rows that would land there run as two passes of
-  // 4 rows instead (each reads the cache once more).
-  if (G == 8 && cache->decode_kernel == RQ_DECODE_KERNEL_AUTO &&
-      rq::decode_kernel_choice(ref_kind, res_bits, res_group, 8, RQ_DECODE_KERNEL_AUTO, n_chain > 1 ? n_chain : 1) ==
-          rq::kKernelSimt)
-    G = 4;
+  const int n_chain = loop_chain(cache, loop, chain);
   if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G, cache->decode_kernel, n_chain > 1 ? n_chain : 1))
     return fail(RQ_ERR_UNSUPPORTED, "no %s decode kernel for this loop format, G = %d and a chain of %d",
                 cache->decode_kernel == RQ_DECODE_KERNEL_TENSOR ? "tensor-core" : "", G, n_chain);

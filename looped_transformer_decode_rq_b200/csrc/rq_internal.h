@@ -131,6 +131,13 @@ cudaError_t launch_split_tc(const DecodeParams& p, int ref_kind, int res_bits, i
                             const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
 constexpr int kTcPage = 128;
 
+// Split-K workspace bytes a decode of `loop` with n_q query tokens per
+// sequence needs (the rows of one pass over the cache, as the decode entry
+// points size it).
+rq_status decode_scratch_need(const rq_cache* cache, int loop, int n_q, int64_t* bytes_out);
+// The device the cache was created on (current when rq_cache_create ran).
+int cache_device(const rq_cache* cache);
+
 // Records the calling thread's rq_last_error_message() text and returns `s`.
 rq_status set_last_error(rq_status s, const char* fmt, ...);
 

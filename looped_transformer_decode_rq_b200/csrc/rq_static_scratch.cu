@@ -31,8 +31,10 @@ extern "C" RQ_API rq_status rq_decode_attention_static_scratch(
     const rq_cache* cache, int32_t loop, const void* q, const int32_t* ctx_len, const void* k_tail,
     const void* v_tail, int32_t n_tail, float softmax_scale, float* out, rq_stream_t stream) {
   if (cache == nullptr) return rq::set_last_error(RQ_ERR_INVALID_ARG, "cache is null");
+  // the split-K partials of this loop's decode: the same rows per pass over
+  // the cache as rq_decode_attention takes
   int64_t need = 0;
-  rq_status st = rq_decode_workspace_size(cache, &need);
+  rq_status st = rq::decode_scratch_need(cache, loop, 1, &need);
   if (st != RQ_OK) return st;
   if (need > static_cast<int64_t>(kStaticScratchBytes))
     return rq::set_last_error(RQ_ERR_WORKSPACE,
@@ -43,6 +45,11 @@ extern "C" RQ_API rq_status rq_decode_attention_static_scratch(
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return rq::set_last_error(RQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return rq::set_last_error(RQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  // The array used is the current device's; the cache's planes must live there too.
+  if (dev != rq::cache_device(cache))
+    return rq::set_last_error(RQ_ERR_INVALID_ARG,
+                              "current device %d is not the device %d the cache was created on", dev,
+                              rq::cache_device(cache));
   void* scratch = nullptr;
   {
     // One-time set-up per device, done with that device current: in host code

@@ -202,18 +202,37 @@ class Cache:
         _check(_lib.rq_encode(self._h, k.data_ptr(), v.data_ptr(), strides, start_pos, _ptr(positions),
                               k.shape[3], _stream(stream)), "rq_encode")
 
+    def _check_decode_args(self, q, ctx_len, k_tail, v_tail, out):
+        """Shapes, dtypes, devices and layouts of a single-query decode's tensors
+        (the kernels read and write them as these shapes, so a wrong one must
+        not reach the library)."""
+        cfg = self.cfg
+        dev = self.base.device
+        B, Hq, Hkv = cfg.batch, cfg.q_heads, cfg.kv_heads
+        if q.dtype != torch.bfloat16 or not q.is_contiguous() or tuple(q.shape) != (B, Hq, HEAD_DIM) or q.device != dev:
+            raise ValueError(f"q must be a contiguous bf16 [{B}, {Hq}, {HEAD_DIM}] tensor on {dev}")
+        if ctx_len.dtype != torch.int32 or tuple(ctx_len.shape) != (B,) or ctx_len.device != dev:
+            raise ValueError(f"ctx_len must be an int32 [{B}] tensor on {dev}")
+        n_tail = 0 if k_tail is None else k_tail.shape[2]
+        if n_tail:
+            for t in (k_tail, v_tail):
+                if (t is None or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != dev
+                        or t.dim() != 4 or tuple(t.shape) != (B, Hkv, n_tail, HEAD_DIM)):
+                    raise ValueError(f"k_tail and v_tail must be contiguous bf16 [{B}, {Hkv}, n_tail, {HEAD_DIM}] "
+                                     f"tensors on {dev}")
+        if out is None:
+            out = torch.empty((B, Hq, HEAD_DIM), dtype=torch.float32, device=dev)
+        elif (out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != (B, Hq, HEAD_DIM)
+              or out.device != dev):
+            raise ValueError(f"out must be a contiguous fp32 [{B}, {Hq}, {HEAD_DIM}] tensor on {dev}")
+        return q, ctx_len, k_tail, v_tail, out, n_tail
+
     def decode_attention(self, loop: int, q: torch.Tensor, ctx_len: torch.Tensor,
                          k_tail: Optional[torch.Tensor] = None, v_tail: Optional[torch.Tensor] = None,
                          softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                          stream=None) -> torch.Tensor:
         """q: bf16 [B, Hq, 128]; ctx_len: int32 [B]; tails bf16 [B, Hkv, n_tail, 128]."""
-        cfg = self.cfg
-        assert q.dtype == torch.bfloat16 and q.is_contiguous() and ctx_len.dtype == torch.int32
-        if out is None:
-            out = torch.empty((cfg.batch, cfg.q_heads, HEAD_DIM), dtype=torch.float32, device=q.device)
-        n_tail = 0 if k_tail is None else k_tail.shape[2]
-        if n_tail:
-            assert k_tail.is_contiguous() and v_tail.is_contiguous()
+        q, ctx_len, k_tail, v_tail, out, n_tail = self._check_decode_args(q, ctx_len, k_tail, v_tail, out)
         scale = softmax_scale if softmax_scale is not None else HEAD_DIM ** -0.5
         _check(_lib.rq_decode_attention(self._h, loop, q.data_ptr(), ctx_len.data_ptr(), _ptr(k_tail),
                                         _ptr(v_tail), n_tail, scale, out.data_ptr(), self.workspace.data_ptr(),
@@ -250,15 +269,9 @@ class Cache:
                                 stream=None) -> torch.Tensor:
         """decode_attention(loop, ...) and the encode of k_new/v_new (bf16 [L, B, Hkv, n, 128])
         at device positions (int32 [B]) in one call."""
-        cfg = self.cfg
-        assert q.dtype == torch.bfloat16 and q.is_contiguous() and ctx_len.dtype == torch.int32
+        q, ctx_len, k_tail, v_tail, out, n_tail = self._check_decode_args(q, ctx_len, k_tail, v_tail, out)
         assert k_new.dtype == torch.bfloat16 and v_new.dtype == torch.bfloat16 and k_new.shape == v_new.shape
         assert k_new.stride() == v_new.stride() and k_new.stride(-1) == 1 and positions.dtype == torch.int32
-        if out is None:
-            out = torch.empty((cfg.batch, cfg.q_heads, HEAD_DIM), dtype=torch.float32, device=q.device)
-        n_tail = 0 if k_tail is None else k_tail.shape[2]
-        if n_tail:
-            assert k_tail.is_contiguous() and v_tail.is_contiguous()
         scale = softmax_scale if softmax_scale is not None else HEAD_DIM ** -0.5
         strides = (_i64 * 4)(*k_new.stride()[:4])
         _check(_lib.rq_decode_attention_append(self._h, loop, q.data_ptr(), ctx_len.data_ptr(), _ptr(k_tail),
@@ -275,11 +288,7 @@ class Cache:
         """decode_attention without a caller workspace: the library keeps the
         split-K partials in its own fixed 4 MiB device array (for callers that
         cannot allocate).  Calls that overlap on the GPU race on that array."""
-        cfg = self.cfg
-        assert q.dtype == torch.bfloat16 and q.is_contiguous() and ctx_len.dtype == torch.int32
-        if out is None:
-            out = torch.empty((cfg.batch, cfg.q_heads, HEAD_DIM), dtype=torch.float32, device=q.device)
-        n_tail = 0 if k_tail is None else k_tail.shape[2]
+        q, ctx_len, k_tail, v_tail, out, n_tail = self._check_decode_args(q, ctx_len, k_tail, v_tail, out)
         scale = softmax_scale if softmax_scale is not None else HEAD_DIM ** -0.5
         _check(_lib.rq_decode_attention_static_scratch(self._h, loop, q.data_ptr(), ctx_len.data_ptr(),
                                                        _ptr(k_tail), _ptr(v_tail), n_tail, scale, out.data_ptr(),

@@ -18,6 +18,8 @@ Residuals", abstract and Figure 2/Figure 5 captions):
   ``a_l ~ U(0.8, 1.2)`` drawn per (loop, head); rounded to bf16;
 * values are drawn the same way with their own scales and ``a_l``;
 * queries ``q ~ N(0, 1)`` rounded to bf16, one per (loop, sequence, q-head);
+  with probability ``q_outlier_p`` a query element is an outlier, multiplied
+  by ``U(q_outlier_mult)`` (30-100x by default);
 * the current token of every loop (the "tail", attended in bf16 before it is
   encoded) follows the same recipe as the cached tokens.
 """
@@ -62,6 +64,8 @@ class Workload:
     anchor_policy: int = 0      # 0: final loop is the reference; 1: loop 0; 2: blocks of anchor_interval;
                                 # 3 / 4: chained, loop l against loop l-1 / l+1
     anchor_interval: int = 0
+    q_outlier_p: float = 0.0    # per (loop, sequence, q-head, channel): the query element is an outlier
+    q_outlier_mult: Sequence[float] = (30.0, 100.0)  # outlier query elements are multiplied by U(lo, hi)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -197,7 +201,16 @@ def make_inputs(wl: Workload, device="cpu", layer: int = 0) -> dict:
             del ref, reff
         out[name] = planes
         out[name + "_tail"] = tails
-    out["q"] = _bf16(randn(L, B, Hq, D))
+    q = randn(L, B, Hq, D)
+    if wl.q_outlier_p > 0:
+        # outlier query channels, from a generator of their own (the other
+        # inputs of the workload are unchanged by it)
+        go = torch.Generator(device=dev).manual_seed(wl.seed * 1000003 + layer + 7777)
+        mask = torch.rand(L, B, Hq, D, generator=go, device=dev) < wl.q_outlier_p
+        lo, hi = wl.q_outlier_mult
+        mult = lo + (hi - lo) * torch.rand(L, B, Hq, D, generator=go, device=dev)
+        q = torch.where(mask, q * mult, q)
+    out["q"] = _bf16(q)
     out["ctx_len"] = draw_lengths(wl, device=dev)
     return out
 

@@ -41,15 +41,22 @@ def unpack_alpha(raw: np.ndarray):
     return h[..., 0].view(np.float16), h[..., 1].view(np.float16)
 
 
-def read_planes(cache, n_tokens: int):
-    """Copy the cache's planes (first n_tokens positions) to numpy."""
+def read_planes(cache, n_tokens: int = 0, positions=None):
+    """Copy the cache's planes to numpy: the first n_tokens positions of every
+    sequence, or (``positions``: one position per sequence) the one record of
+    sequence b at positions[b], as a length-1 token axis."""
     from looped_transformer_decode_rq_b200 import rq  # noqa: F401
     cfg, lay = cache.cfg, cache.layout
     L = cfg.num_loops
     out = {"ref": {}, "loops": []}
 
     def grab(off, rec):
-        return cache.plane(off, rec)[:, :, :n_tokens].cpu().numpy()
+        pl = cache.plane(off, rec)
+        if positions is None:
+            return pl[:, :, :n_tokens].cpu().numpy()
+        pos = torch.as_tensor(positions, dtype=torch.long, device=pl.device)
+        idx = pos.view(-1, 1, 1, 1).expand(-1, pl.shape[1], 1, rec)
+        return torch.gather(pl, 2, idx).cpu().numpy()
 
     for l in range(L):
         if lay.alpha_offset[l] >= 0:

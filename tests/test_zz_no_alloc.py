@@ -4,35 +4,38 @@ every allocation, or serving loops that must not call cudaMalloc once they are
 running).  It keeps its split-K partials in the library's own fixed-size
 device array instead of a caller workspace.
 
-The test calls it through the C ABI twice in a row and checks each output
-against rq_decode_attention (same kernels, caller workspace) within the
-attention tolerance the other parity tests use.  It lives in a file of its own
-that pytest collects last and passes both alone and after the other tests."""
+The test calls it through the C ABI twice in a row on each cache and checks
+each output against rq_decode_attention (same kernels on the same grid, caller
+workspace): the two must agree bit for bit, and both must match the float64
+oracle within the attention tolerance of the other parity tests.  It lives in
+a file of its own that pytest collects last and passes both alone and after
+the other tests."""
 import ctypes as C
 
 import numpy as np
 import pytest
 import torch
 
+import oracle.rq_oracle as O
 from looped_transformer_decode_rq_b200 import synth
-from tests.helpers import ATTN_TOL, rel_err_rows
+from tests.helpers import ATTN_TOL, oracle_encode, rel_err_rows, to_np32
 
 pytestmark = pytest.mark.gpu
 
 
-def _rel(a, b):
-    return float(rel_err_rows(a.cpu().numpy(), b.cpu().numpy().astype(np.float64)).max())
-
-
-def test_static_scratch_matches_workspace_entry_point_twice(librq):
+@pytest.mark.parametrize("q_heads", [8, 32])
+def test_static_scratch_matches_workspace_entry_point_twice(librq, q_heads):
+    """q_heads / kv_heads = 2 (the CUDA-core kernel) and 8 (the largest group:
+    the tensor-core kernel's 8-row variant)."""
     rq = librq
-    wl = synth.Workload(name="static_scratch", batch=3, kv_heads=4, q_heads=8, context=700,
+    wl = synth.Workload(name="static_scratch", batch=3, kv_heads=4, q_heads=q_heads, context=700,
                         lengths=(700, 65, 333), sigma=(0.3, 0.2, 0.1), outlier_p=0.01, seed=77)
     inp = synth.make_inputs(wl, "cpu")
     cfgd = synth.cache_config_dict(wl)
     cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
     assert cache.workspace.numel() <= rq.STATIC_SCRATCH_BYTES
     cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    enc = oracle_encode(inp, cfgd)
     ctx = inp["ctx_len"].cuda()
     lib = rq.lib()
     stream = torch.cuda.current_stream().cuda_stream
@@ -48,7 +51,10 @@ def test_static_scratch_matches_workspace_entry_point_twice(librq):
         assert st == rq.OK, lib.rq_last_error_message()
         torch.cuda.synchronize()
         assert torch.isfinite(got).all()
-        assert _rel(got, want) <= ATTN_TOL
+        assert torch.equal(got, want)
+        oracle = O.decode_attention_f64(enc, loop, to_np32(inp["q"][loop]), inp["ctx_len"].numpy(),
+                                        to_np32(inp["k_tail"][loop]), to_np32(inp["v_tail"][loop]))
+        assert rel_err_rows(got.cpu().numpy(), oracle).max() <= ATTN_TOL
     assert cache.get_error() == 0
 
 
