@@ -27,7 +27,8 @@ NVCC_FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompil
 
 CU_SOURCES = ["rq_encode.cu", "rq_decode.cu", "rq_decode_chain.cu", "rq_decode_tc.cu", "rq_static_scratch.cu"]
 CPP_SOURCES = ["rq_api.cpp"]
-HEADERS = ["rq_common.cuh", "rq_internal.h", "rq_tcgen05.cuh", "rq_encode_dev.cuh", "rq_decode_split.cuh"]
+HEADERS = ["rq_common.cuh", "rq_internal.h", "rq_tcgen05.cuh", "rq_encode_dev.cuh", "rq_decode_split.cuh",
+           "rq_decode_bp.cuh"]
 
 
 def _sources():

@@ -119,13 +119,27 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // healthy pipeline.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// A try-wait that may suspend the thread for up to `hint_ns` while the phase
+// is incomplete (it returns as soon as the phase completes), so that a waiting
+// warp spends few issue slots polling.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  uint32_t it = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++it & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
   }
 }
 
@@ -171,11 +185,24 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
 
 __device__ __forceinline__ float bf16_bits_to_f(uint32_t lo16) { return __uint_as_float(lo16 << 16); }
 
+// The bits of 1.0f (0x3F800000) in a register the compiler cannot see
+// through.  An instruction carries at most one 32-bit immediate, so with both
+// the code mask and the exponent as immediates (w & mask) | exponent costs two
+// logic operations; with the exponent in this register it is one LOP3.
+__device__ __forceinline__ uint32_t opaque_one_bits() {
+  uint32_t lid;
+  asm volatile("mov.u32 %0, %%laneid;" : "=r"(lid));
+  return 0x3F800000u | (lid >> 5);  // lid < 32
+}
+
 // A b-bit code c sitting at bit p (p + b <= 23) of `w` becomes the float
-// 1 + c * 2^(p - 23) with one LOP3; subtracting 1 is then exact, and the
-// 2^(p - 23) factor is folded into the operand it multiplies.
-__device__ __forceinline__ float code_float(uint32_t w, uint32_t mask_at_p) {
-  return __uint_as_float((w & mask_at_p) | 0x3F800000u);
+// 1 + c * 2^(p - 23) with one LOP3 ((w & mask) | one, one = opaque_one_bits());
+// subtracting 1 is then exact, and the 2^(p - 23) factor is folded into the
+// operand it multiplies.
+__device__ __forceinline__ float code_float(uint32_t w, uint32_t mask_at_p, uint32_t one) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "r"(mask_at_p), "r"(one));
+  return __uint_as_float(d);
 }
 
 // fp16 (scale, offset) pair packed in a 32-bit word

@@ -23,7 +23,7 @@
 #include <cstring>
 
 #include "rq_common.cuh"
-#include "rq_decode_split.cuh"
+#include "rq_decode_bp.cuh"
 #include "rq_encode_dev.cuh"
 #include "rq_internal.h"
 

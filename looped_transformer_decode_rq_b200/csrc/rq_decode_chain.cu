@@ -9,7 +9,7 @@
 // i's value codes the weight p_t beta_i; all links share one rotated
 // accumulator, since they share one format and rotation.  Separate from
 // rq_decode.cu so that the two sets of instantiations compile in parallel.
-#include "rq_decode_split.cuh"
+#include "rq_decode_bp.cuh"
 
 namespace rq {
 namespace {

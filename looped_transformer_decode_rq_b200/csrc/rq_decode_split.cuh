@@ -156,14 +156,15 @@ __device__ __forceinline__ void load_codes(const uint8_t* p, uint32_t (&w)[(NB +
 }
 
 // code e of a thread's unit (bits per code BITS) as 1 + c*2^(p_e - 23)
+// (`one`: opaque_one_bits())
 template <int BITS>
-__device__ __forceinline__ float code_f(const uint32_t* w, int e) {
+__device__ __forceinline__ float code_f(const uint32_t* w, int e, uint32_t one) {
   const int bit = e * BITS;
   const uint32_t word = w[bit >> 5];
   const int b32 = bit & 31;
   const uint32_t src = (b32 >= 16) ? (word >> 16) : word;
   const int p = b32 & 15;
-  return code_float(src, ((1u << BITS) - 1u) << p);
+  return code_float(src, ((1u << BITS) - 1u) << p, one);
 }
 
 template <int BITS>
@@ -212,6 +213,60 @@ struct DotOperands {
 template <int BITS>
 __device__ __forceinline__ uint32_t unpack_bytes(uint32_t w, int k) {
   return BITS == 2 ? ((w >> (2 * k)) & 0x03030303u) : ((w >> (4 * k)) & 0x0F0F0F0Fu);
+}
+
+constexpr float kQ24 = 8323072.f;  // signed 24-bit range whose top byte stays in [-127, 127]
+
+// signed bytes of a 24-bit-range integer: v = 65536 b2 + 256 b1 + b0
+__device__ __forceinline__ void split24s(int v, int& b2, int& b1, int& b0) {
+  const int t = (v + 128) >> 8;
+  b0 = v - (t << 8);
+  b2 = (t + 128) >> 8;
+  b1 = t - (b2 << 8);
+}
+
+// Integer-dot-product operands for a lane's D query values against 4-bit
+// packed codes (the INT4 anchor, which is not rotated), with 24 bits of
+// precision: the values are quantised to signed 24-bit integers with one
+// scale (|q| <= kQ24 * scale) and split into three signed bytes, so that
+//     sum_e q_e c_e = scale * (65536 dp4a(c, b2) + 256 dp4a(c, b1) + dp4a(c, b0))
+// exactly.  Byte b of operand [w][k] pairs with element 8w + 2b + k, the code
+// that (word_w >> 4k) & 0x0F0F0F0F puts into byte b.  A query with a few large
+// channels keeps the precision of the others (16 bits per lane would lose it).
+template <int D>
+struct DotOperands24 {
+  static constexpr int NW = (D + 7) / 8;
+  uint32_t b2[NW][2], b1[NW][2], b0[NW][2];
+  float scale;
+
+  __device__ __forceinline__ void build(const float* v) {
+    float m = 0.f;
+#pragma unroll
+    for (int e = 0; e < D; ++e) m = fmaxf(m, fabsf(v[e]));
+    scale = m * (1.f / kQ24);
+    const float inv = m > 0.f ? kQ24 / m : 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+#pragma unroll
+      for (int k = 0; k < 2; ++k) b2[w][k] = b1[w][k] = b0[w][k] = 0u;
+#pragma unroll
+    for (int e = 0; e < D; ++e) {
+      int qi = __float2int_rn(v[e] * inv);
+      qi = max(-8323072, min(8323072, qi));
+      int x2, x1, x0;
+      split24s(qi, x2, x1, x0);
+      const int w = e / 8, b = (e % 8) / 2, k = e % 2;
+      b2[w][k] |= (static_cast<uint32_t>(x2) & 0xFFu) << (8 * b);
+      b1[w][k] |= (static_cast<uint32_t>(x1) & 0xFFu) << (8 * b);
+      b0[w][k] |= (static_cast<uint32_t>(x0) & 0xFFu) << (8 * b);
+    }
+  }
+};
+
+// 65536 x2 + 256 x1 + x0 of three byte-plane dot products, as fp32: |x1|, |x0|
+// <= 32 * 15 * 128, so 256 x1 + x0 is exact in fp32 and the sum rounds once.
+__device__ __forceinline__ float comb24s(int x2, int x1, int x0) {
+  return fmaf(65536.f, static_cast<float>(x2), static_cast<float>(x1 * 256 + x0));
 }
 
 // ---------------------------------------------------------------------------
@@ -281,6 +336,7 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int B = P.B, Hkv = P.Hkv;
+  const uint32_t one = opaque_one_bits();
   // Launched as a programmatic dependent of the previous kernel on the stream
   // (typically the previous call's combine kernel, which reads the partials
   // this grid writes): everything above overlaps its tail; nothing global is
@@ -433,7 +489,7 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
     // fp32; code planes (INT4 anchor, residual) get int16 dp4a operands
     constexpr int NG1 = RB ? ((C::D1 >= RG) ? C::D1 / RG : 1) : 1;
     float2 qref[G][REF == kRefBf16 ? C::D1 / 2 : 1];
-    DotOperands<4, REF == kRefInt4 ? C::D1 : 1> oref[G];
+    DotOperands24<REF == kRefInt4 ? C::D1 : 1> oref[G];
     DotOperands<RB ? RB : 2, RB ? C::D1 : 1> ores[G];
     float qsum_res[G][NG1];
     float qsum_ref[G];
@@ -540,28 +596,28 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
             part[gi] = sum;
           }
         } else if constexpr (REF == kRefInt4) {
-          using Ops = DotOperands<4, C::D1>;
+          using Ops = DotOperands24<C::D1>;
           uint32_t cw[Ops::NW];
           load_codes<C::D1 / 2>(st + C::O_REFK + t * 64 + (d1 >> 1), cw);
           const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMK + t * 16 + 4 * (d1 >> 5)));
-          int dhi[G];
-          unsigned dlo[G];
+          int x2[G], x1[G], x0[G];
 #pragma unroll
-          for (int gi = 0; gi < G; ++gi) { dhi[gi] = 0; dlo[gi] = 0u; }
+          for (int gi = 0; gi < G; ++gi) x2[gi] = x1[gi] = x0[gi] = 0;
 #pragma unroll
           for (int w = 0; w < Ops::NW; ++w)
 #pragma unroll
-            for (int kk = 0; kk < Ops::KPW; ++kk) {
-              const uint32_t x = unpack_bytes<4>(cw[w], kk);
+            for (int kk = 0; kk < 2; ++kk) {
+              const int x = static_cast<int>(unpack_bytes<4>(cw[w], kk));
 #pragma unroll
               for (int gi = 0; gi < G; ++gi) {
-                dhi[gi] = __dp4a(static_cast<int>(x), static_cast<int>(oref[gi].hi[w][kk]), dhi[gi]);
-                dlo[gi] = __dp4a(x, oref[gi].lo[w][kk], dlo[gi]);
+                x2[gi] = __dp4a(x, static_cast<int>(oref[gi].b2[w][kk]), x2[gi]);
+                x1[gi] = __dp4a(x, static_cast<int>(oref[gi].b1[w][kk]), x1[gi]);
+                x0[gi] = __dp4a(x, static_cast<int>(oref[gi].b0[w][kk]), x0[gi]);
               }
             }
 #pragma unroll
           for (int gi = 0; gi < G; ++gi) {
-            const float dot = static_cast<float>(dhi[gi] * 256 + static_cast<int>(dlo[gi])) * oref[gi].scale;
+            const float dot = comb24s(x2[gi], x1[gi], x0[gi]) * oref[gi].scale;
             part[gi] = fmaf(sz.x, dot, sz.y * qsum_ref[gi]);
           }
         }
@@ -702,7 +758,7 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
           const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMV + t * 16 + 4 * (d2 >> 5)));
 #pragma unroll
           for (int e = 0; e < C::D2; e += 2) {
-            const float2 f = f2sub1(make_float2(code_f<4>(cw, e), code_f<4>(cw, e + 1)));
+            const float2 f = f2sub1(make_float2(code_f<4>(cw, e, one), code_f<4>(cw, e + 1, one)));
 #pragma unroll
             for (int gi = 0; gi < G; ++gi) {
               const float w = pa[gi] * sz.x;
@@ -721,7 +777,7 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
                 half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::o_resmv(ci) + t * C::MB + 4 * (d2 / RG)));
 #pragma unroll
             for (int e = 0; e < C::D2; e += 2) {
-              const float2 f = f2sub1(make_float2(code_f<RB>(cw, e), code_f<RB>(cw, e + 1)));
+              const float2 f = f2sub1(make_float2(code_f<RB>(cw, e, one), code_f<RB>(cw, e + 1, one)));
 #pragma unroll
               for (int gi = 0; gi < G; ++gi) {
                 const float w = pw[ci][gi] * sz.x;
@@ -855,17 +911,6 @@ cudaError_t launch_split(DecodeParams& p, const CUtensorMap* tk, const CUtensorM
 }
 
 using SplitFn = cudaError_t (*)(DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);
-
-template <int REF, int RB, int RG, int NCH>
-SplitFn pick_g(int G) {
-  switch (G) {
-    case 1: return launch_split<REF, RB, RG, 1, NCH>;
-    case 2: return launch_split<REF, RB, RG, 2, NCH>;
-    case 4: return launch_split<REF, RB, RG, 4, NCH>;
-    case 8: return launch_split<REF, RB, RG, 8, NCH>;
-    default: return nullptr;
-  }
-}
 
 }  // namespace
 }  // namespace rq

@@ -7,7 +7,7 @@ import torch
 
 import oracle.rq_oracle as O
 from looped_transformer_decode_rq_b200 import synth
-from tests.helpers import ATTN_TOL, oracle_encode, rel_err_rows, to_np32
+from tests.helpers import ATTN_TOL, compare_encoded, oracle_encode, rel_err_rows, to_np32
 
 pytestmark = pytest.mark.gpu
 
@@ -179,6 +179,24 @@ def test_chained_loops_run_on_the_cuda_core_kernel(librq):
     run_case(rq, wl, loops=[0, 1])
 
 
+OUTLIER_FORMATS = {"bf16ref_int2": ((2, 2, 2, 16), (32,) * 4), "int4anchor_2244": ((2, 2, 4, 4), (32,) * 4),
+                   "int4anchor_int4g16": ((4, 4, 4, 4), (16, 16, 16, 32)),
+                   "bf16ref_int4g16": ((4, 2, 4, 16), (16, 32, 16, 32))}
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+@pytest.mark.parametrize("fmt", sorted(OUTLIER_FORMATS))
+def test_outlier_query_channels(librq, fmt, G):
+    """Queries with a few large channels (2% of elements at 30-100x) on the
+    CUDA-core kernels: the INT4 anchor's unrotated query keeps 24 bits per
+    lane, so the other channels keep their precision; the residual's rotated
+    query has no outliers left to lose it to."""
+    bits, group = OUTLIER_FORMATS[fmt]
+    wl = synth.Workload(name=f"qout_{fmt}_{G}", batch=3, kv_heads=2, q_heads=2 * G, context=300, bits=bits,
+                        group=group, sigma=(0.3, 0.2, 0.1), outlier_p=0.01, q_outlier_p=0.02, seed=170 + G)
+    run_case(librq, wl, lengths=[300, 129, 1], n_tail=1, kernel=librq.DECODE_KERNEL_SIMT)
+
+
 @pytest.mark.parametrize("n_tail", [64, 127])
 def test_recent_window_bf16_tail(librq, n_tail):
     """A window of the most recent 64-127 tokens kept in bf16 next to the compact
@@ -250,19 +268,22 @@ def test_tensor_kernel_rejects_unimplemented(librq):
     assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
 
 
-@pytest.mark.parametrize("kernel", ["simt", "tensor"])
+@pytest.mark.parametrize("kernel", ["simt", "tensor", "simt_int4_anchor_g1"])
 def test_wait_limit_sets_flag_and_context_recovers(librq, kernel):
     """Failure path without a fault: the producers wait on a barrier nothing
     arrives at (test hook); every wait gives up after its limit, the call sets
     FLAG_PIPE_TIMEOUT and returns, and the next call on the same context is
-    correct."""
+    correct.  The last case is the byte-plane kernel (INT4 anchor, one query
+    row per kv-head)."""
     import time
     rq = librq
     wl = synth.Workload(name="stall", batch=2, kv_heads=2, q_heads=8, context=300, seed=90)
+    if kernel == "simt_int4_anchor_g1":
+        wl = wl.with_(q_heads=2, bits=(2, 2, 4, 4))
     inp = synth.make_inputs(wl, "cpu")
     cfgd = synth.cache_config_dict(wl)
     cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
-    cache.set_decode_kernel(rq.DECODE_KERNEL_SIMT if kernel == "simt" else rq.DECODE_KERNEL_TENSOR)
+    cache.set_decode_kernel(rq.DECODE_KERNEL_TENSOR if kernel == "tensor" else rq.DECODE_KERNEL_SIMT)
     cache.encode(inp["k"].cuda(), inp["v"].cuda())
     assert cache.get_error() == 0
     q, ctx = inp["q"][0].cuda(), inp["ctx_len"].cuda()
@@ -333,6 +354,15 @@ def test_decode_with_fused_append_matches_separate_calls(librq, kernel, bits, po
     assert caches[0].get_error() == 0 and caches[1].get_error() == 0
     assert torch.equal(out_a, out_b)
     _same_planes(read_planes(caches[0], wl.context + 1), read_planes(caches[1], wl.context + 1))
+    # the fused call against the oracle: its attention output (the cache before
+    # the append plus the tail) and the records it appended (the oracle's encode
+    # of the new token, bit for bit)
+    enc = oracle_encode(inp, cfgd)
+    want = O.decode_attention_f64(enc, last, to_np32(inp["q"][last]), ctx.cpu().numpy(),
+                                  to_np32(inp["k_tail"][last]), to_np32(inp["v_tail"][last]))
+    assert rel_err_rows(out_b.cpu().numpy(), want).max() <= ATTN_TOL
+    enc_new = O.encode_fp32emu(to_np32(inp["k_tail"]), to_np32(inp["v_tail"]), O.CacheConfig.from_dict(cfgd))
+    compare_encoded(read_planes(caches[1], positions=ctx.cpu()), enc_new)
 
 
 @pytest.mark.parametrize("kernel", ["simt", "tensor"])
