@@ -431,9 +431,10 @@ int loop_chain(const rq_cache* cache, int loop, int (&chain)[RQ_MAX_CHAIN]) {
 
 // Query rows per pass over the cache (G of the kernels) for a decode of `loop`
 // with n_q query tokens per sequence: all rows up to 8, else blocks of 8.  The
-// CUDA-core kernel's 8-row variants spill registers (about a tenth of the
-// 4-row rate): by default, 8 rows that would land there run as two passes of
-// 4 rows instead (each reads the cache once more).
+// CUDA-core kernel has no 8-row variant (its registers would spill, at about a
+// tenth of the 4-row rate): 8 rows that land on the CUDA cores -- by the
+// automatic choice or a forced one -- run as two passes of 4 rows (each reads
+// the cache once more).
 rq_status block_rows(const rq_cache* cache, int loop, int n_q, int* G_out) {
   const rq_config& c = cache->cfg;
   if (loop < 0 || loop >= c.num_loops) return fail(RQ_ERR_INVALID_ARG, "loop %d outside [0, %d)", loop, c.num_loops);
@@ -449,9 +450,8 @@ rq_status block_rows(const rq_cache* cache, int loop, int n_q, int* G_out) {
   const int ref_kind = ref_kind_for(c, loop);
   const int res_bits = loop == a ? 0 : c.bits[loop];
   const int res_group = loop == a ? 32 : c.group[loop];
-  if (G == 8 && cache->decode_kernel == RQ_DECODE_KERNEL_AUTO &&
-      rq::decode_kernel_choice(ref_kind, res_bits, res_group, 8, RQ_DECODE_KERNEL_AUTO, n_chain > 1 ? n_chain : 1) ==
-          rq::kKernelSimt)
+  if (G == 8 && rq::decode_kernel_choice(ref_kind, res_bits, res_group, 8, cache->decode_kernel,
+                                         n_chain > 1 ? n_chain : 1) == rq::kKernelSimt)
     G = 4;
   *G_out = G;
   return RQ_OK;

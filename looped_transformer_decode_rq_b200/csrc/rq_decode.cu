@@ -185,6 +185,17 @@ SplitFn pick(int ref_kind, int res_bits, int res_group, int G, int n_chain) {
 
 }  // namespace
 
+namespace {
+// one query row of a byte-plane format on the tensor cores: the ping-pong kernel
+bool pp_case(int ref_kind, int res_bits, int res_group, int G, int n_chain) {
+  return G == 1 && n_chain <= 1 && ref_kind != kRefBf16 && pp_variant_supported(ref_kind, res_bits, res_group);
+}
+}  // namespace
+
+// The automatic choice: the tensor cores from 4 query rows per kv-head, the
+// CUDA cores below (at one row the byte-plane CUDA-core kernel measured faster
+// than the ping-pong tensor-core kernel: 4.3 against 3.3 TB/s on the INT4-anchor
+// [2,2,4,4] residual loop).
 int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel, int n_chain) {
   if (kernel == kKernelAuto)
     return (G >= 4 && n_chain <= 1 && tc_variant_supported(ref_kind, res_bits, res_group, G)) ? kKernelTensor
@@ -195,7 +206,9 @@ int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int k
 bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, int kernel, int n_chain) {
   if (res_bits != 0 && res_group != 16 && res_group != 32) return false;
   kernel = decode_kernel_choice(ref_kind, res_bits, res_group, G, kernel, n_chain);
-  if (kernel == kKernelTensor) return n_chain <= 1 && tc_variant_supported(ref_kind, res_bits, res_group, G);
+  if (kernel == kKernelTensor)
+    return n_chain <= 1 && (pp_case(ref_kind, res_bits, res_group, G, n_chain) ||
+                            tc_variant_supported(ref_kind, res_bits, res_group, G));
   if (kernel == kKernelSimt) return pick(ref_kind, res_bits, res_group, G, n_chain) != nullptr;
   return false;
 }
@@ -220,7 +233,10 @@ cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_gr
   if (kernel == kKernelTensor) {
     if (n_chain > 1) return cudaErrorInvalidValue;
     p.page_tokens = kTcPage;
-    e = launch_split_tc(p, ref_kind, res_bits, res_group, tmap_k, tmap_v, s);
+    if (pp_case(ref_kind, res_bits, res_group, p.G, n_chain))
+      e = launch_split_pp(p, ref_kind, res_bits, res_group, s);
+    else
+      e = launch_split_tc(p, ref_kind, res_bits, res_group, tmap_k, tmap_v, s);
   } else {
     SplitFn fn = pick(ref_kind, res_bits, res_group, p.G, n_chain);
     if (fn == nullptr) return cudaErrorInvalidValue;

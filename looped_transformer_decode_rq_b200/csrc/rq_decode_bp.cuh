@@ -590,8 +590,7 @@ SplitFn pick_g(int G) {
     case 1: return pick_g1<REF, RB, RG, NCH>();
     case 2: return launch_split<REF, RB, RG, 2, NCH>;
     case 4: return launch_split<REF, RB, RG, 4, NCH>;
-    case 8: return launch_split<REF, RB, RG, 8, NCH>;
-    default: return nullptr;
+    default: return nullptr;  // 8 rows run as two passes of 4 (rq_api.cpp)
   }
 }
 

@@ -130,6 +130,10 @@ bool tc_variant_supported(int ref_kind, int res_bits, int res_group, int G);
 cudaError_t launch_split_tc(const DecodeParams& p, int ref_kind, int res_bits, int res_group,
                             const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
 constexpr int kTcPage = 128;
+// tensor-core split kernel for the byte-plane formats at one query row per
+// kv-head, two warpgroups on alternate pages (rq_decode_pp.cu)
+bool pp_variant_supported(int ref_kind, int res_bits, int res_group);
+cudaError_t launch_split_pp(const DecodeParams& p, int ref_kind, int res_bits, int res_group, cudaStream_t s);
 
 // Split-K workspace bytes a decode of `loop` with n_q query tokens per
 // sequence needs (the rows of one pass over the cache, as the decode entry

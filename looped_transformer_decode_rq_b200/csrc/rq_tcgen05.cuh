@@ -1,7 +1,8 @@
 // rq_tcgen05.cuh -- fifth-generation tensor-core (tcgen05) building blocks for
 // sm_100a, as inline PTX: tensor-memory allocation, shared-memory matrix
 // descriptors, instruction descriptors, single-thread MMA issue with mbarrier
-// commit, and 32-lane tensor-memory loads.
+// commit (A from shared or tensor memory), and 32-lane tensor-memory loads and
+// stores.
 //
 // Shared-memory matrix descriptor (64 bits): start address >> 4 in [0, 14),
 // leading-dimension byte offset >> 4 in [16, 30), stride-dimension byte offset
@@ -92,6 +93,18 @@ __device__ __forceinline__ void mma_s8(uint32_t d_tmem, uint64_t a, uint64_t b, 
       : "memory");
 }
 
+// The same with A (M x K, K-major) in tensor memory at `a_tmem`: row i in lane
+// i, K elements packed along consecutive 32-bit columns (four int8 per column).
+__device__ __forceinline__ void mma_s8_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // The mbarrier at `bar` receives one arrival once every MMA this thread issued
 // before has completed.
 __device__ __forceinline__ void commit(uint32_t bar) {
@@ -101,6 +114,8 @@ __device__ __forceinline__ void commit(uint32_t bar) {
 
 // ---- tensor memory -> registers.  Warp w may address lanes [32 (w % 4), +32);
 // thread i of the warp receives N consecutive 32-bit columns of lane base + i.
+// The load is warp-collective: the address must be the same in every thread
+// of the warp (a per-thread column choice is made after the load).
 template <int N>
 __device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&r)[N]);
 
@@ -153,6 +168,21 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N]) {
         : "r"(taddr), "r"(taddr + 8));
   }
 }
+
+// ---- registers -> tensor memory: thread i of the warp writes 32 consecutive
+// 32-bit columns of lane base + i (the warp's own 32-lane quarter)
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
+      "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+      "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Wait for this thread's tensor-memory stores to complete.
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Wait for this thread's tensor-memory loads; the registers passed through
 // afterwards cannot be read earlier by reordered code.

@@ -268,22 +268,22 @@ def test_tensor_kernel_rejects_unimplemented(librq):
     assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
 
 
-@pytest.mark.parametrize("kernel", ["simt", "tensor", "simt_int4_anchor_g1"])
+@pytest.mark.parametrize("kernel", ["simt", "tensor", "simt_int4_anchor_g1", "tensor_int4_anchor_g1"])
 def test_wait_limit_sets_flag_and_context_recovers(librq, kernel):
     """Failure path without a fault: the producers wait on a barrier nothing
     arrives at (test hook); every wait gives up after its limit, the call sets
     FLAG_PIPE_TIMEOUT and returns, and the next call on the same context is
-    correct.  The last case is the byte-plane kernel (INT4 anchor, one query
-    row per kv-head)."""
+    correct.  The last two cases are the byte-plane kernels (INT4 anchor, one
+    query row per kv-head) on the CUDA cores and on the tensor cores."""
     import time
     rq = librq
     wl = synth.Workload(name="stall", batch=2, kv_heads=2, q_heads=8, context=300, seed=90)
-    if kernel == "simt_int4_anchor_g1":
+    if kernel.endswith("int4_anchor_g1"):
         wl = wl.with_(q_heads=2, bits=(2, 2, 4, 4))
     inp = synth.make_inputs(wl, "cpu")
     cfgd = synth.cache_config_dict(wl)
     cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
-    cache.set_decode_kernel(rq.DECODE_KERNEL_TENSOR if kernel == "tensor" else rq.DECODE_KERNEL_SIMT)
+    cache.set_decode_kernel(rq.DECODE_KERNEL_TENSOR if kernel.startswith("tensor") else rq.DECODE_KERNEL_SIMT)
     cache.encode(inp["k"].cuda(), inp["v"].cuda())
     assert cache.get_error() == 0
     q, ctx = inp["q"][0].cuda(), inp["ctx_len"].cuda()
