@@ -39,8 +39,8 @@ namespace {
 constexpr int kPP = kTcPage;        // tokens per page
 constexpr int kPpNCT = 256;         // two consumer warpgroups
 constexpr int kPpProducer = 8;      // producer warp
-constexpr int kPpMma = 9;           // MMA-issuing warp
-constexpr int kPpNT = kPpNCT + 64;
+constexpr int kPpMma = 9;           // MMA-issuing warps: kPpMma + w serves warpgroup w
+constexpr int kPpNT = kPpNCT + 96;
 constexpr int kPpBarAll = 1;        // the 256 consumer threads
 constexpr int kPpBarWG = 2;         // warpgroup w uses kPpBarWG + w
 constexpr int kPpSmemLimit = 227 * 1024;
@@ -57,19 +57,18 @@ struct PpCfg {
   static constexpr int CB = RB * 16;
   static constexpr int MB = RB ? 4 * NGR : 0;
   static constexpr int AL_REC = HAS_ALPHA ? 4 : 0;
-  // MMA widths (one query head): score columns per 32-dim chunk are the three
-  // byte planes of the query (x2 parities for 16-dim groups); value columns are
-  // (byte plane, group)
-  static constexpr int N_SA = 16;
-  static constexpr int N_SR = round16(3 * NPAR);
+  // MMA widths (one query head): score columns are (group, byte plane) of the
+  // query, value columns (byte plane, group) of the weights
+  static constexpr int N_SA = 16;                 // 4 groups x 3
+  static constexpr int N_SR = round16(3 * NGR1);  // 12 or 24
   static constexpr int N_VA = 16;
   static constexpr int N_VR = round16(3 * NGR1);
   // tensor-memory columns of one warpgroup
   static constexpr int T_KA = 0;                          // anchor key codes, int8 [128 tok][128]: 32 columns
   static constexpr int T_KR = T_KA + (ANCH ? 32 : 0);     // residual key codes
-  static constexpr int T_SA = T_KR + (RB ? 32 : 0);       // anchor scores: 4 chunks x N_SA
-  static constexpr int T_SR = T_SA + (ANCH ? 4 * N_SA : 0);
-  static constexpr int T_OA = T_SR + (RB ? 4 * N_SR : 0); // anchor value sums
+  static constexpr int T_SA = T_KR + (RB ? 32 : 0);       // anchor scores
+  static constexpr int T_SR = T_SA + (ANCH ? N_SA : 0);   // residual scores
+  static constexpr int T_OA = T_SR + (RB ? N_SR : 0);     // anchor value sums
   static constexpr int T_OR = T_OA + (ANCH ? N_VA : 0);   // residual value sums
   static constexpr int T_WG = T_OR + (RB ? N_VR : 0);
   static constexpr int TMEM_COLS = 2 * T_WG <= 128 ? 128 : (2 * T_WG <= 256 ? 256 : 512);
@@ -238,7 +237,7 @@ __global__ void __launch_bounds__(kPpNT, 1) decode_pp_kernel(const __grid_consta
       mbar_init(smem_u32(&vready[w]), 4);
       mbar_init(smem_u32(&obar[w]), 1);
     }
-    mbar_init(smem_u32(done), 1);
+    mbar_init(smem_u32(done), 2);  // both MMA-issuing warps
     mbar_init(smem_u32(never), 1);
     fence_barrier_init();
   }
@@ -320,76 +319,49 @@ __global__ void __launch_bounds__(kPpNT, 1) decode_pp_kernel(const __grid_consta
     return;
   }
 
-  // ========================= MMA-issuing warp =========================
-  // One thread issues the MMAs of both warpgroups.  Each warpgroup's pages are
-  // k = w, w + 2, ...; for each, its score MMAs once its key codes are in
-  // tensor memory, then its value MMAs once its weights are written.  The
-  // thread serves whichever warpgroup is ready, so the two interleave.
-  if (warp == kPpMma) {
+  // ========================= MMA-issuing warps =========================
+  // Warp kPpMma + w issues the MMAs of warpgroup w, whose pages are k = w,
+  // w + 2, ...: for each, the score MMAs once its key codes are in tensor
+  // memory, then the value MMAs once its weights are written.  The two warps
+  // wait on their own warpgroup's barriers, so each reacts at once.
+  if (warp == kPpMma || warp == kPpMma + 1) {
     if (lane == 0) {
-      int cnt[2], step[2];  // pages issued per warpgroup; 0: scores next, 1: values next
-      int todo[2];
-      for (int w = 0; w < 2; ++w) {
-        cnt[w] = step[w] = 0;
-        todo[w] = n_pages > w ? (n_pages - w + 1) / 2 : 0;
-      }
-      const uint64_t t_start = global_timer_ns();
-      uint64_t t_last = t_start;
-      while ((cnt[0] < todo[0] || cnt[1] < todo[1]) && !*sAbort) {
-        bool issued = false;
-#pragma unroll 1
-        for (int w = 0; w < 2; ++w) {
-          if (cnt[w] >= todo[w]) continue;
-          const uint32_t ph = cnt[w] & 1;
-          uint8_t* fw = fx + w * C::F_WG;
-          const uint32_t tw = tbase + w * C::T_WG;
-          if (step[w] == 0) {
-            if (!mbar_test_wait(smem_u32(&kready[w]), ph)) continue;
-            tc::fence_after_sync();
-            if constexpr (ANCH) {
+      const int w = warp - kPpMma;
+      const int todo = n_pages > w ? (n_pages - w + 1) / 2 : 0;
+      uint8_t* fw = fx + w * C::F_WG;
+      const uint32_t tw = tbase + w * C::T_WG;
+      for (int cnt = 0; cnt < todo; ++cnt) {
+        const uint32_t ph = cnt & 1;
+        if (!wait_or_abort(&kready[w], ph)) break;
+        tc::fence_after_sync();
+        if constexpr (ANCH) {
 #pragma unroll
-              for (int c = 0; c < 4; ++c)
-                tc::mma_s8_ta(tw + C::T_SA + C::N_SA * c, tw + C::T_KA + 8 * c,
-                              tc::desc_k_sw128(smem_u32(fw + C::F_QA + 32 * c)), C::ID_SA, 0);
-            }
-            if constexpr (RB != 0) {
-#pragma unroll
-              for (int c = 0; c < 4; ++c)
-                tc::mma_s8_ta(tw + C::T_SR + C::N_SR * c, tw + C::T_KR + 8 * c,
-                              tc::desc_k_sw128(smem_u32(fw + C::F_HQ + 32 * c)), C::ID_SR, 0);
-            }
-            tc::commit(smem_u32(&sbar[w]));
-            step[w] = 1;
-          } else {
-            if (!mbar_test_wait(smem_u32(&vready[w]), ph)) continue;
-            tc::fence_after_sync();
-            if constexpr (ANCH) {
-#pragma unroll
-              for (int ks = 0; ks < 4; ++ks)
-                tc::mma_s8(tw + C::T_OA, tc::desc_mn_sw128(smem_u32(fw + C::F_URV + ks * 4096), 16384),
-                           tc::desc_mn_plain(smem_u32(fw + C::F_WA + ks * 512), 128, 2048), C::ID_VA, ks > 0);
-            }
-            if constexpr (RB != 0) {
-#pragma unroll
-              for (int ks = 0; ks < 4; ++ks)
-                tc::mma_s8(tw + C::T_OR, tc::desc_mn_sw128(smem_u32(fw + C::F_UV + ks * 4096), 16384),
-                           tc::desc_mn_plain(smem_u32(fw + C::F_WR + ks * 512), 128, 2048), C::ID_VR, ks > 0);
-            }
-            tc::commit(smem_u32(&obar[w]));
-            step[w] = 0;
-            ++cnt[w];
-          }
-          issued = true;
+          for (int c = 0; c < 4; ++c)
+            tc::mma_s8_ta(tw + C::T_SA, tw + C::T_KA + 8 * c, tc::desc_k_sw128(smem_u32(fw + C::F_QA + 32 * c)),
+                          C::ID_SA, c > 0);
         }
-        const uint64_t now = global_timer_ns();
-        if (issued) {
-          t_last = now;
-        } else if (now - t_last > kWaitLimitNs) {
-          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-          *sAbort = 1;
-        } else {
-          __nanosleep(32);
+        if constexpr (RB != 0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tc::mma_s8_ta(tw + C::T_SR, tw + C::T_KR + 8 * c, tc::desc_k_sw128(smem_u32(fw + C::F_HQ + 32 * c)),
+                          C::ID_SR, c > 0);
         }
+        tc::commit(smem_u32(&sbar[w]));
+        if (!wait_or_abort(&vready[w], ph)) break;
+        tc::fence_after_sync();
+        if constexpr (ANCH) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_s8(tw + C::T_OA, tc::desc_mn_sw128(smem_u32(fw + C::F_URV + ks * 4096), 16384),
+                       tc::desc_mn_plain(smem_u32(fw + C::F_WA + ks * 512), 128, 2048), C::ID_VA, ks > 0);
+        }
+        if constexpr (RB != 0) {
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            tc::mma_s8(tw + C::T_OR, tc::desc_mn_sw128(smem_u32(fw + C::F_UV + ks * 4096), 16384),
+                       tc::desc_mn_plain(smem_u32(fw + C::F_WR + ks * 512), 128, 2048), C::ID_VR, ks > 0);
+        }
+        tc::commit(smem_u32(&obar[w]));
       }
       tc::commit(smem_u32(done));
     }
@@ -417,7 +389,7 @@ __global__ void __launch_bounds__(kPpNT, 1) decode_pp_kernel(const __grid_consta
       const uint2 raw = *reinterpret_cast<const uint2*>(P.q + q_row_offset(P, b, h, 0) + 4 * lane);
       const float2 a01 = bf16x2_to_f2(raw.x), a23 = bf16x2_to_f2(raw.y);
       float x[4] = {a01.x, a01.y, a23.x, a23.y};
-      if constexpr (ANCH) put_q_s24<4, 32, 1>(fw + C::F_QA, x, 0, lane, &q_sc[0], &q_sc[2], P.scale_log2);
+      if constexpr (ANCH) put_q_grouped<4, 32>(fw + C::F_QA, x, lane, &q_sc[0], &q_sc[2], P.scale_log2);
       if constexpr (RB != 0) {
         if (P.rotate) {
           const float t0 = x[0] + x[1], t1 = x[0] - x[1], t2 = x[2] + x[3], t3 = x[2] - x[3];
@@ -435,7 +407,7 @@ __global__ void __launch_bounds__(kPpNT, 1) decode_pp_kernel(const __grid_consta
 #pragma unroll
           for (int e = 0; e < 4; ++e) x[e] *= c;
         }
-        put_q_s24<RB, RG, 1>(fw + C::F_HQ, x, 0, lane, &q_sc[1], &q_sc[6], P.scale_log2);
+        put_q_grouped<RB, RG>(fw + C::F_HQ, x, lane, &q_sc[1], &q_sc[6], P.scale_log2);
       }
     }
     fence_proxy_async_smem();
@@ -454,10 +426,53 @@ __global__ void __launch_bounds__(kPpNT, 1) decode_pp_kernel(const __grid_consta
     for (int g = 0; g < NGR1; ++g) zr[g] = 0.f;
   };
 
+  // A page's value sums are merged at the warpgroup's next page (after its key
+  // codes and metadata), so that the value MMAs run behind that work; these
+  // hold the pending page's rescale factors (thread = dim position).
+  bool pend = false;
+  float p_crun = 1.f, p_pm = 0.f, p_fa = 0.f, p_fr = 0.f;
+
   PageIter it;
   seek(it, x0);
   int k = 0;
   int n_w = 0;  // pages this warpgroup has taken (phase of its per-warpgroup barriers)
+
+  auto merge_pending = [&]() {
+    wait_or_abort(&obar[wg], (n_w - 1) & 1);
+    tc::fence_after_sync();
+    if constexpr (ANCH) {
+      uint32_t v[3];
+#pragma unroll
+      for (int j = 0; j < 3; ++j)
+        tc::tmem_ld_n<1>(tl + C::T_OA + j * 4 + chunk, *reinterpret_cast<uint32_t(*)[1]>(&v[j]));
+      tc::tmem_wait_ld();
+      tc::reg_fence(v);
+      acc_ref = fmaf(acc_ref, p_crun, p_pm * p_fa * comb24(v[0], v[1], v[2]));
+    }
+    if constexpr (RB != 0) {
+      // a tensor-memory load takes one address for the whole warp: both
+      // parities' columns of 16-dim groups are loaded, then selected per thread
+      uint32_t v[C::NPAR][3];
+#pragma unroll
+      for (int p = 0; p < C::NPAR; ++p)
+#pragma unroll
+        for (int j = 0; j < 3; ++j)
+          tc::tmem_ld_n<1>(tl + C::T_OR + j * NGR + chunk * C::NPAR + p, *reinterpret_cast<uint32_t(*)[1]>(&v[p][j]));
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int p = 0; p < C::NPAR; ++p) tc::reg_fence(v[p]);
+      uint32_t b2 = v[0][0], b1 = v[0][1], b0 = v[0][2];
+      if constexpr (C::NPAR == 2) {
+        b2 = par_r ? v[1][0] : b2;
+        b1 = par_r ? v[1][1] : b1;
+        b0 = par_r ? v[1][2] : b0;
+      }
+      acc_res = fmaf(acc_res, p_crun, p_pm * p_fr * comb24(b2, b1, b0));
+    }
+    // the value sums are read: the next value MMAs may write them
+    tc::fence_before_sync();
+    pend = false;
+  };
   while (k < n_pages) {
     const int b = it.b, h = it.h;
     const int seg_pages = min(nt_of(b) - it.page, n_pages - k);
@@ -533,8 +548,10 @@ __global__ void __launch_bounds__(kPpNT, 1) decode_pp_kernel(const __grid_consta
           zAv[u] = valid ? c2.y : 0.f;
         }
       }
-      // ---- value codes into this warpgroup's shared tiles (its previous page's
-      // value MMAs have completed: it merged their sums); then the stage is free
+      // ---- the previous page's value sums (its MMAs have run meanwhile)
+      if (pend) merge_pending();
+      // ---- value codes into this warpgroup's shared tiles (the previous page's
+      // value MMAs have completed: its sums are merged); then the stage is free
       if constexpr (ANCH) expand_row<4>(st + C::O_REFV + r * 64, fw + C::F_URV, r);
       if constexpr (RB != 0) expand_row<RB>(st + C::O_RESV + r * C::CB, fw + C::F_UV, r);
       __syncwarp();
@@ -545,33 +562,42 @@ __global__ void __launch_bounds__(kPpNT, 1) decode_pp_kernel(const __grid_consta
       tc::fence_after_sync();
       float S = 0.f;
       {
-        float dotA = 0.f, offA = 0.f, dotR = 0.f, offR = 0.f;
+        // columns 3 g + k: byte plane k of group g (the residual's last four
+        // 16-dim groups are read after the first ones are folded)
+        uint32_t va[12], vr[12];
+        if constexpr (ANCH) tc::tmem_ld_n<12>(tl + C::T_SA, va);
+        if constexpr (RB != 0) tc::tmem_ld_n<12>(tl + C::T_SR, vr);
+        tc::tmem_wait_ld();
+        if constexpr (ANCH) {
+          tc::reg_fence(va);
+          float dotA = 0.f, offA = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t va[3], vr[C::NPAR][3];
-          if constexpr (ANCH) tc::tmem_ld_n<3>(tl + C::T_SA + C::N_SA * c, va);
-          if constexpr (RB != 0) {
-#pragma unroll
-            for (int p = 0; p < C::NPAR; ++p) tc::tmem_ld_n<3>(tl + C::T_SR + C::N_SR * c + 3 * p, vr[p]);
+          for (int g = 0; g < 4; ++g) {
+            dotA = fmaf(sAk[g], comb24(va[3 * g], va[3 * g + 1], va[3 * g + 2]), dotA);
+            offA = fmaf(zAk[g], q_sc[2 + g], offA);
           }
-          tc::tmem_wait_ld();
-          if constexpr (ANCH) {
-            tc::reg_fence(va);
-            dotA = fmaf(sAk[c], comb24(va[0], va[1], va[2]), dotA);
-            offA = fmaf(zAk[c], q_sc[2 + c], offA);
-          }
-          if constexpr (RB != 0) {
+          S = aK * fmaf(dotA, q_sc[0], offA);
+        }
+        if constexpr (RB != 0) {
+          tc::reg_fence(vr);
+          float dotR = 0.f, offR = 0.f;
 #pragma unroll
-            for (int p = 0; p < C::NPAR; ++p) {
-              tc::reg_fence(vr[p]);
-              const int g = c * C::NPAR + p;
-              dotR = fmaf(sK[g], comb24(vr[p][0], vr[p][1], vr[p][2]), dotR);
-              offR = fmaf(zK[g], q_sc[6 + g], offR);
+          for (int g = 0; g < 4; ++g) {
+            dotR = fmaf(sK[g], comb24(vr[3 * g], vr[3 * g + 1], vr[3 * g + 2]), dotR);
+            offR = fmaf(zK[g], q_sc[6 + g], offR);
+          }
+          if constexpr (NGR == 8) {
+            tc::tmem_ld_n<12>(tl + C::T_SR + 12, vr);
+            tc::tmem_wait_ld();
+            tc::reg_fence(vr);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              dotR = fmaf(sK[4 + g], comb24(vr[3 * g], vr[3 * g + 1], vr[3 * g + 2]), dotR);
+              offR = fmaf(zK[4 + g], q_sc[10 + g], offR);
             }
           }
+          S += fmaf(dotR, q_sc[1], offR);
         }
-        if constexpr (ANCH) S = aK * fmaf(dotA, q_sc[0], offA);
-        if constexpr (RB != 0) S += fmaf(dotR, q_sc[1], offR);
       }
       S = valid ? S : -INFINITY;
 
@@ -671,50 +697,27 @@ __global__ void __launch_bounds__(kPpNT, 1) decode_pp_kernel(const __grid_consta
         }
       }
 
-      // ---- merge the page's value sums (thread = dim position r)
-      wait_or_abort(&obar[wg], ph);
-      tc::fence_after_sync();
+      // ---- this page's value sums are merged at the next page (or the flush)
+      p_crun = crun;
+      p_pm = pm;
       if constexpr (ANCH) {
-        uint32_t v[3];
-        tc::tmem_ld_n<1>(tl + C::T_OA + 0 * 4 + chunk, *reinterpret_cast<uint32_t(*)[1]>(&v[0]));
-        tc::tmem_ld_n<1>(tl + C::T_OA + 1 * 4 + chunk, *reinterpret_cast<uint32_t(*)[1]>(&v[1]));
-        tc::tmem_ld_n<1>(tl + C::T_OA + 2 * 4 + chunk, *reinterpret_cast<uint32_t(*)[1]>(&v[2]));
-        tc::tmem_wait_ld();
-        tc::reg_fence(v);
         float sg = siga[0];
 #pragma unroll
         for (int g = 1; g < 4; ++g) sg = (chunk == g) ? siga[g] : sg;
-        acc_ref = fmaf(acc_ref, crun, pm * sg * (1.f / kQ3) * comb24(v[0], v[1], v[2]));
+        p_fa = sg * (1.f / kQ3);
       }
       if constexpr (RB != 0) {
-        // a tensor-memory load takes one address for the whole warp: both
-        // parities' columns of 16-dim groups are loaded, then selected per thread
-        uint32_t v[C::NPAR][3];
-#pragma unroll
-        for (int p = 0; p < C::NPAR; ++p)
-#pragma unroll
-          for (int j = 0; j < 3; ++j)
-            tc::tmem_ld_n<1>(tl + C::T_OR + j * NGR + chunk * C::NPAR + p, *reinterpret_cast<uint32_t(*)[1]>(&v[p][j]));
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int p = 0; p < C::NPAR; ++p) tc::reg_fence(v[p]);
-        uint32_t b2 = v[0][0], b1 = v[0][1], b0 = v[0][2];
-        if constexpr (C::NPAR == 2) {
-          b2 = par_r ? v[1][0] : b2;
-          b1 = par_r ? v[1][1] : b1;
-          b0 = par_r ? v[1][2] : b0;
-        }
         float sg = sig[0];
 #pragma unroll
         for (int g = 1; g < NGR; ++g) sg = (g_res == g) ? sig[g] : sg;
-        acc_res = fmaf(acc_res, crun, pm * sg * (1.f / kU3) * comb24(b2, b1, b0));
+        p_fr = sg * (1.f / kU3);
       }
-      // the value sums are read: the next page may write them
-      tc::fence_before_sync();
+      pend = true;
       ++n_w;
       advance(it);
     }
 
+    if (pend) merge_pending();
     // ---- flush this (b, h) segment: both warpgroups' states into their slots,
     // then added in a fixed order into the CTA's partial record
     {

@@ -141,6 +141,40 @@ __device__ __forceinline__ void put_q_s24(uint8_t* tile, const float (&x)[4], in
   if (lane == 0) *scale_out = m * (1.f / kQ3) * scale_log2;
 }
 
+// The same query quantisation, written for one MMA sequence over all 128 dims
+// whose output columns are (group, byte plane): row 3 g + k holds byte k of the
+// query's elements in group g (RGRP dims each) and zero at every other group's
+// K positions, so that accumulating the four 32-dim chunks gives each group's
+// dot product in columns 3 g .. 3 g + 2.
+template <int BITS, int RGRP>
+__device__ __forceinline__ void put_q_grouped(uint8_t* tile, const float (&x)[4], int lane, float* scale_out,
+                                              float* gsum_out, float scale_log2) {
+  constexpr int NGRP = 128 / RGRP;
+  float m = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+  m = warp_max_nonneg(m);
+  const float inv = m > 0.f ? kQ3 / m : 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int d = 4 * lane + e;
+    int qi = __float2int_rn(x[e] * inv);
+    qi = max(-8323072, min(8323072, qi));
+    int b[3];
+    split24(qi, b[0], b[1], b[2]);
+    const int j = 32 * (d >> 5) + dim_pos<BITS>(d & 31);
+    const int g = d / RGRP;
+#pragma unroll
+    for (int gg = 0; gg < NGRP; ++gg)
+#pragma unroll
+      for (int k = 0; k < 3; ++k) tile[kmaj_byte(3 * gg + k, j)] = gg == g ? static_cast<uint8_t>(b[k]) : 0;
+  }
+  float s = x[0] + x[1] + x[2] + x[3];
+  constexpr int LPG = RGRP / 4;  // lanes per group
+#pragma unroll
+  for (int o = 1; o < LPG; o <<= 1) s += __shfl_xor_sync(kFull, s, o);
+  if ((lane % LPG) == 0) gsum_out[lane / LPG] = s * scale_log2;
+  if (lane == 0) *scale_out = m * (1.f / kQ3) * scale_log2;
+}
+
 // Byte planes of NB 24-bit values v[] (byte 2 = top): out[j] holds byte 2 - j
 // of every value, value m at byte m of the plane.
 template <int NB>
