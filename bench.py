@@ -444,14 +444,29 @@ def measure_multi_query(wl, n_q, steps, warmup, world, rank):
     ms1 = time_steps(single_step, steps, warmup, world, stream)
     call_ms, _ = residual_call_ms(lambda: cache.decode_attention_multi(0, qm[0], ctx, kt[0], vt[0], out=outs[0]),
                                   stream, reps=10, warmup=3)
+    # the same rows as blocks of half the draft tokens, one cache pass each
+    # (the way rows beyond one pass run): the cost a single pass saves
+    half = n_q // 2
+    qh = [qm[0][:, :half].contiguous(), qm[0][:, half:].contiguous()]
+    oh = [outs[0][:, :half].contiguous(), outs[0][:, half:].contiguous()]
+
+    def two_calls():
+        for i in range(2):
+            cache.decode_attention_multi(0, qh[i], ctx, kt[0], vt[0], out=oh[i])
+
+    call2_ms, _ = residual_call_ms(two_calls, stream, reps=10, warmup=3)
     res_bytes = (tokens_total * Hkv * record_bytes(cache.layout, cfgd, 0) + B * n_q * Hq * 128 * (2 + 4) +
                  B * Hkv * n_q * 512)
     flags = cache.get_error()
+    kernel, rows_per_pass = cache.decode_plan(0, n_q)
     out = {"workload": f"{wl.name}_verify{n_q}", "n_q": n_q,
+           "rows_per_kv_head": n_q * wl.gqa, "rows_per_pass": rows_per_pass,
+           "passes": n_q * wl.gqa // rows_per_pass, "kernel": {1: "simt", 2: "tensor"}.get(kernel, kernel),
            "query_tokens_per_s": round(job_tokens_per_s(B * n_q, world, ms), 1), "ms_per_step": round(ms, 4),
            "single_query_tokens_per_s": round(job_tokens_per_s(B, world, ms1), 1),
            "single_query_ms_per_step": round(ms1, 4),
            "residual_loop_gbs": round(res_bytes / (call_ms * 1e-3) / 1e9, 1), "residual_loop_bytes": res_bytes,
+           "residual_loop_ms": round(call_ms, 4), "residual_loop_ms_as_two_calls_of_half": round(call2_ms, 4),
            "device_flags": flags}
     del cache, inp, outs, out1, qm
     torch.cuda.empty_cache()
@@ -846,7 +861,8 @@ def run_rq(args, world, rank):
                  measure_workload(synth.gqa_long(batch=8, q_heads=64), 30, 3, world, rank),
                  measure_workload(synth.ouro_8k_next_loop(), 30, 3, world, rank, per_loop=True),
                  measure_workload(synth.ouro_8k_next_loop_int4(), 30, 3, world, rank, per_loop=True),
-                 measure_multi_query(synth.ouro_8k(), 4, 30, 3, world, rank)]
+                 measure_multi_query(synth.ouro_8k(), 4, 30, 3, world, rank),
+                 measure_multi_query(synth.gqa_long(batch=8), 4, 20, 3, world, rank)]
     sweeps = None
     if not args.no_sweeps and args.workload == "ouro8k":
         # the mixed-precision [2,2,4,4] batch sweep and the 24-layer capacity

@@ -224,8 +224,10 @@ RQ_API rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const 
  *  RQ_DECODE_KERNEL_TENSOR  split kernel on the tensor cores (tcgen05), 128-token
  *                           pages: bf16 and int8 MMAs for the scores of all G
  *                           query heads of a kv-head at once and for the
- *                           probability-weighted value sums; G in {1, 2, 4, 8},
- *                           not for the residual loops of chained policies.
+ *                           probability-weighted value sums; G in {1, 2, 4, 8,
+ *                           16} (16 rows for some formats: see
+ *                           rq_decode_attention_multi), not for the residual
+ *                           loops of chained policies.
  *  RQ_DECODE_KERNEL_AUTO    the tensor-core kernel for G >= 4 where it has a
  *                           variant, else the CUDA-core kernel (the default). */
 typedef enum {
@@ -296,9 +298,12 @@ RQ_API rq_status rq_decode_multi_workspace_size(const rq_cache* cache, int32_t n
  * 0 .. n_tail - n_q + i: the last n_q tail tokens are the draft tokens' own
  * keys and values (bf16, not yet encoded), each visible to itself and to the
  * later ones, and any earlier tail tokens to all.  Up to 8 query rows per
- * kv-head (n_q * G) share every read of its cached pages; more rows run in
- * blocks of 8, one pass over the cache each.  With 4 or more rows in a block
- * the automatic kernel choice is the tensor-core kernel.
+ * kv-head (n_q * G) share every read of its cached pages, and 16 rows do where
+ * the tensor-core kernel has a 16-row variant for the loop's format (bf16
+ * anchor with INT2 g=32 residuals, an INT4 or bf16 anchor loop, no anchor with
+ * g=32 residuals) and the call takes that kernel; other rows run in blocks of 16
+ * or 8, one pass over the cache each.  With 4 or more rows in a block the
+ * automatic kernel choice is the tensor-core kernel.
  *  q        device bf16 [B][n_q][Hq][128]
  *  out      device fp32 [B][n_q][Hq][128]
  *  n_q      in [1, RQ_MAX_DRAFT] (else RQ_ERR_INVALID_ARG) with n_q * (Hq / Hkv)
@@ -310,6 +315,15 @@ RQ_API rq_status rq_decode_attention_multi(const rq_cache* cache, int32_t loop, 
                                            const int32_t* ctx_len, const void* k_tail, const void* v_tail,
                                            int32_t n_tail, float softmax_scale, float* out, void* workspace,
                                            int64_t workspace_bytes, rq_stream_t stream);
+
+/* How rq_decode_attention_multi (n_q draft tokens; rq_decode_attention is
+ * n_q = 1) would run `loop` on this handle, without running it: the kernel it
+ * takes (RQ_DECODE_KERNEL_SIMT or RQ_DECODE_KERNEL_TENSOR) and the query rows
+ * per kv-head of one pass over the cache; n_q * G / rows_per_pass passes read
+ * the loop's pages.  Returns what that call would return for an unsupported
+ * loop, n_q or kernel (RQ_ERR_INVALID_ARG, RQ_ERR_UNSUPPORTED).  Host only. */
+RQ_API rq_status rq_decode_plan(const rq_cache* cache, int32_t loop, int32_t n_q, int32_t* kernel_out,
+                                int32_t* rows_per_pass_out);
 
 /* rq_decode_attention of `loop`, plus the encode of n_new new tokens of every
  * loop into the cache in the same call: the per-step append of a decoding
@@ -347,8 +361,9 @@ RQ_API rq_status rq_decode_attention_append(rq_cache* cache, int32_t loop, const
  *  - It allocates nothing and calls no allocating routine.
  *  - Limit: the split-K partials of this decode must fit in
  *    RQ_STATIC_SCRATCH_BYTES: (batch*kv_heads + SMs) * G * 1040 bytes, with G
- *    the query rows of one pass over the cache (q_heads / kv_heads, or 4 where
- *    the default decode runs 8 rows as two passes of 4); otherwise it returns
+ *    the query rows of one pass over the cache (q_heads / kv_heads up to 8; 16
+ *    where a 16-row tensor-core pass takes them, else 8; 4 where the default
+ *    decode runs 8 rows as two passes of 4); otherwise it returns
  *    RQ_ERR_WORKSPACE before enqueuing anything.
  *  - Device: the device current at the call must be the one the cache was
  *    created on (RQ_ERR_INVALID_ARG otherwise).

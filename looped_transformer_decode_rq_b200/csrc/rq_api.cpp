@@ -430,11 +430,13 @@ int loop_chain(const rq_cache* cache, int loop, int (&chain)[RQ_MAX_CHAIN]) {
 }
 
 // Query rows per pass over the cache (G of the kernels) for a decode of `loop`
-// with n_q query tokens per sequence: all rows up to 8, else blocks of 8.  The
-// CUDA-core kernel has no 8-row variant (its registers would spill, at about a
-// tenth of the 4-row rate): 8 rows that land on the CUDA cores -- by the
-// automatic choice or a forced one -- run as two passes of 4 rows (each reads
-// the cache once more).
+// with n_q query tokens per sequence: all rows up to 8; 16 rows (and each block
+// of 16 of a multiple of 16) in one pass where the tensor-core kernel has a
+// 16-row variant for the loop's format and is the kernel the call takes; else
+// blocks of 8.  The CUDA-core kernel has no 8-row variant (its registers would
+// spill, at about a tenth of the 4-row rate): 8 rows that land on the CUDA
+// cores -- by the automatic choice or a forced one -- run as two passes of 4
+// rows (each reads the cache once more).
 rq_status block_rows(const rq_cache* cache, int loop, int n_q, int* G_out) {
   const rq_config& c = cache->cfg;
   if (loop < 0 || loop >= c.num_loops) return fail(RQ_ERR_INVALID_ARG, "loop %d outside [0, %d)", loop, c.num_loops);
@@ -450,8 +452,12 @@ rq_status block_rows(const rq_cache* cache, int loop, int n_q, int* G_out) {
   const int ref_kind = ref_kind_for(c, loop);
   const int res_bits = loop == a ? 0 : c.bits[loop];
   const int res_group = loop == a ? 32 : c.group[loop];
-  if (G == 8 && rq::decode_kernel_choice(ref_kind, res_bits, res_group, 8, cache->decode_kernel,
-                                         n_chain > 1 ? n_chain : 1) == rq::kKernelSimt)
+  const int nc = n_chain > 1 ? n_chain : 1;
+  if (rows % 16 == 0 &&
+      rq::decode_kernel_choice(ref_kind, res_bits, res_group, 16, cache->decode_kernel, nc) == rq::kKernelTensor &&
+      rq::decode_variant_supported(ref_kind, res_bits, res_group, 16, rq::kKernelTensor, nc))
+    G = 16;
+  if (G == 8 && rq::decode_kernel_choice(ref_kind, res_bits, res_group, 8, cache->decode_kernel, nc) == rq::kKernelSimt)
     G = 4;
   *G_out = G;
   return RQ_OK;
@@ -582,11 +588,35 @@ rq_status rq_decode_attention(const rq_cache* cache, int32_t loop, const void* q
                      workspace_bytes, stream, nullptr);
 }
 
+rq_status rq_decode_plan(const rq_cache* cache, int32_t loop, int32_t n_q, int32_t* kernel_out,
+                         int32_t* rows_per_pass_out) {
+  if (cache == nullptr || kernel_out == nullptr || rows_per_pass_out == nullptr)
+    return fail(RQ_ERR_INVALID_ARG, "null argument");
+  int G = 0;
+  const rq_status st = block_rows(cache, loop, n_q, &G);
+  if (st != RQ_OK) return st;
+  const rq_config& c = cache->cfg;
+  int chain[RQ_MAX_CHAIN];
+  const int n_chain = loop_chain(cache, loop, chain);
+  const int a = cache->lay.anchor_of[loop];
+  const int ref_kind = ref_kind_for(c, loop);
+  const int res_bits = loop == a ? 0 : c.bits[loop];
+  const int res_group = loop == a ? 32 : c.group[loop];
+  const int nc = n_chain > 1 ? n_chain : 1;
+  if (!rq::decode_variant_supported(ref_kind, res_bits, res_group, G, cache->decode_kernel, nc))
+    return fail(RQ_ERR_UNSUPPORTED, "no decode kernel for this loop format, G = %d and a chain of %d", G, n_chain);
+  const int k = rq::decode_kernel_choice(ref_kind, res_bits, res_group, G, cache->decode_kernel, nc);
+  *kernel_out = k == rq::kKernelTensor ? RQ_DECODE_KERNEL_TENSOR : RQ_DECODE_KERNEL_SIMT;
+  *rows_per_pass_out = G;
+  return RQ_OK;
+}
+
 rq_status rq_decode_multi_workspace_size(const rq_cache* cache, int32_t n_q, int64_t* bytes_out) {
   if (cache == nullptr || bytes_out == nullptr) return fail(RQ_ERR_INVALID_ARG, "null argument");
   if (n_q < 1 || n_q > RQ_MAX_DRAFT) return fail(RQ_ERR_INVALID_ARG, "n_q %d outside [1, %d]", n_q, RQ_MAX_DRAFT);
   const int rows = n_q * (cache->cfg.q_heads / cache->cfg.kv_heads);
-  const int G = rows < 8 ? rows : 8;
+  // the most rows one pass may take (any loop of the cache)
+  const int G = rows < 8 ? rows : (rows % 16 == 0 ? 16 : 8);
   *bytes_out = rq::decode_workspace_bytes(cache->cfg.batch, cache->cfg.kv_heads, G, cache->num_ctas);
   return RQ_OK;
 }

@@ -75,17 +75,25 @@ struct TcCfg {
   static constexpr int N_SR = round16(3 * G * NPAR);                   // residual score columns per chunk
   static constexpr int N_VA = round16(3 * 4 * G);                      // INT4 anchor value columns
   static constexpr int N_VR = round16(3 * NGR * G);                    // residual value columns
+  static constexpr int N_VB = round16(2 * G);                          // bf16 anchor value columns (hi, lo)
+  // With 16 query rows the integer key codes are widened into tensor memory
+  // (the score MMAs' A operand) instead of shared tiles, which the larger
+  // query and weight operands need.
+  static constexpr bool KTM = G == 16;
   // tensor-memory columns: scores, then value sums (separate, so that the next
-  // page's scores can be computed while this page's value sums are read)
+  // page's scores can be computed while this page's value sums are read), then
+  // the key codes of the 16-row variants
   static constexpr int S_REF = 0;
   static constexpr int S_REF_COLS = REF == kRefBf16 ? 16 : (REF == kRefInt4 ? 4 * N_SA : 0);
   static constexpr int S_RES = S_REF + S_REF_COLS;
   static constexpr int S_COLS = S_RES + (RB ? 4 * N_SR : 0);
   static constexpr int O_REF = S_COLS;
-  static constexpr int O_REF_COLS = REF == kRefBf16 ? 16 : (REF == kRefInt4 ? N_VA : 0);
+  static constexpr int O_REF_COLS = REF == kRefBf16 ? N_VB : (REF == kRefInt4 ? N_VA : 0);
   static constexpr int O_RES = O_REF + O_REF_COLS;
   static constexpr int O_COLS = O_RES + (RB ? N_VR : 0);
-  static constexpr int COLS = O_COLS;
+  static constexpr int TK_REF = O_COLS;                               // INT4 anchor key codes (KTM)
+  static constexpr int TK_RES = TK_REF + (REF == kRefInt4 ? 32 : 0);  // residual key codes (KTM)
+  static constexpr int COLS = O_COLS + (KTM ? (REF == kRefInt4 ? 32 : 0) + (RB ? 32 : 0) : 0);
   static constexpr int TMEM_COLS = COLS <= 32 ? 32 : COLS <= 64 ? 64 : COLS <= 128 ? 128 : COLS <= 256 ? 256 : 512;
   // stage layout (pieces 1024-byte aligned)
   static constexpr int al(int x) { return (x + 1023) & ~1023; }
@@ -101,26 +109,28 @@ struct TcCfg {
   static constexpr int STAGE_BYTES = O_AL + al(kTP * AL_REC);
   // operand tiles (after the stages)
   static constexpr int F_UK = 0;                                   // residual K codes, int8 [128 tok][128]
-  static constexpr int F_UV = F_UK + (RB ? 16384 : 0);             // residual V codes
+  static constexpr int F_UV = F_UK + (RB && !KTM ? 16384 : 0);     // residual V codes
   static constexpr int F_URK = F_UV + (RB ? 16384 : 0);            // INT4 anchor K codes
-  static constexpr int F_URV = F_URK + (REF == kRefInt4 ? 16384 : 0);
+  static constexpr int F_URV = F_URK + (REF == kRefInt4 && !KTM ? 16384 : 0);
   static constexpr int F_QB = F_URV + (REF == kRefInt4 ? 16384 : 0);  // bf16 q [16][128], K-major sw128
   static constexpr int F_QA = F_QB + (REF == kRefBf16 ? 4096 : 0);    // int8 q bytes [N_SA][128]
   static constexpr int F_HQ = F_QA + (REF == kRefInt4 ? al(N_SA * 128) : 0);  // int8 H q bytes [N_SR][128]
-  static constexpr int F_WB = F_HQ + (RB ? al(N_SR * 128) : 0);       // bf16 weights, MN-major [16 x 128 tok]
-  static constexpr int F_WA = F_WB + (REF == kRefBf16 ? 4096 : 0);    // int8 weights [N_VA x 128 tok]
+  static constexpr int F_WB = F_HQ + (RB ? al(N_SR * 128) : 0);       // bf16 weights, MN-major [N_VB x 128 tok]
+  static constexpr int F_WA = F_WB + (REF == kRefBf16 ? N_VB * 256 : 0);  // int8 weights [N_VA x 128 tok]
   static constexpr int F_WR = F_WA + (REF == kRefInt4 ? al(N_VA * 128) : 0);
   static constexpr int F_END = F_WR + (RB ? al(N_VR * 128) : 0);
   // small state (after the tiles; 4-byte words)
   static constexpr int NRED = 1 + 8 + 4;                 // l, residual offsets, anchor offsets
-  static constexpr int W_CS = 0;                         // [G] residual q scale * scale_log2
-  static constexpr int W_QS = W_CS + 8;                  // [G][8] residual group sums of H q
-  static constexpr int W_CA = W_QS + 64;                 // [G] anchor q scale * scale_log2
-  static constexpr int W_QA = W_CA + 8;                  // [G][4] anchor group sums of q
-  static constexpr int W_WM = W_QA + 32;                 // [2][4 warps][4] warp maxima of scores
-  static constexpr int W_SIG = W_WM + 32;                // [2][4 warps][12] warp maxima of scales
-  static constexpr int W_RED = W_SIG + 96;               // [4 warps][8 heads][NRED] flush sums
-  static constexpr int W_PRE = W_RED + 4 * 8 * NRED;     // [RQ_MAX_BATCH + 1] page prefix
+  static constexpr int GS = G > 8 ? G : 8;               // head slots of the small arrays
+  static constexpr int GHS = GH > 4 ? GH : 4;            // head slots per warpgroup
+  static constexpr int W_CS = 0;                         // [GS] residual q scale * scale_log2
+  static constexpr int W_QS = W_CS + GS;                 // [GS][8] residual group sums of H q
+  static constexpr int W_CA = W_QS + 8 * GS;             // [GS] anchor q scale * scale_log2
+  static constexpr int W_QA = W_CA + GS;                 // [GS][4] anchor group sums of q
+  static constexpr int W_WM = W_QA + 4 * GS;             // [2][4 warps][GHS] warp maxima of scores
+  static constexpr int W_SIG = W_WM + 8 * GHS;           // [2][4 warps][12] warp maxima of scales
+  static constexpr int W_RED = W_SIG + 96;               // [4 warps][GS heads][NRED] flush sums
+  static constexpr int W_PRE = W_RED + 4 * GS * NRED;    // [RQ_MAX_BATCH + 1] page prefix
   static constexpr int W_MISC = W_PRE + RQ_MAX_BATCH + 1;  // abort flag, tensor-memory base
   static constexpr int W_BAR = (W_MISC + 2 + 1) & ~1;    // 8-byte aligned mbarriers
   static constexpr int NBARS = 2 * 4 + 8;
@@ -128,17 +138,20 @@ struct TcCfg {
   static constexpr int FIXED = 1024 + F_END + SMALL_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT >= 4 ? 4 : (STAGES_FIT >= 2 ? STAGES_FIT : 2);
-  static constexpr bool FITS = STAGES_FIT >= 2 && COLS <= 512;
+  // 16 rows with an INT4 anchor and residual links would keep both offset sums
+  // of 8 heads per thread and spill registers: those run as two 8-row passes
+  static constexpr bool REGS_FIT = !(G == 16 && REF == kRefInt4 && RB != 0);
+  static constexpr bool FITS =
+      STAGES_FIT >= 2 && COLS <= 512 && N_VA <= 256 && N_VR <= 256 && N_SR <= 256 && REGS_FIT;
   static constexpr int SMEM_BYTES = FIXED + STAGES * STAGE_BYTES;
   // instruction descriptors
   static constexpr uint32_t ID_SB = tc::instr_desc(tc::kAccF32, tc::kFmtBf16, tc::kFmtBf16, 0, 0, 128, 16);
   static constexpr uint32_t ID_SA = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 0, 0, 128, N_SA);
   static constexpr uint32_t ID_SR = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 0, 0, 128, N_SR);
-  static constexpr uint32_t ID_VB = tc::instr_desc(tc::kAccF32, tc::kFmtBf16, tc::kFmtBf16, 1, 1, 128, 16);
+  static constexpr uint32_t ID_VB = tc::instr_desc(tc::kAccF32, tc::kFmtBf16, tc::kFmtBf16, 1, 1, 128, N_VB);
   static constexpr uint32_t ID_VA = tc::instr_desc(tc::kAccS32, tc::kFmtS8, tc::kFmtS8, 1, 1, 128, N_VA);
   static constexpr uint32_t ID_VR = tc::instr_desc(tc::kAccS32, 0, 0, 1, 1, 128, N_VR);  // unsigned bytes
-  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "query heads per kv-head");
-  static_assert(N_VA <= 256 && N_VR <= 256 && N_SR <= 256, "MMA width");
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8 || G == 16, "query heads per kv-head");
 };
 
 // ---------------------------------------------------------------------------
@@ -177,6 +190,22 @@ __device__ __forceinline__ void tc_issue_page(const DecodeParams& P, const CUten
     bulk_g2s(smem_u32(st + C::O_RESMV), P.res_meta[0][1] + rec0 * C::MB, nrec * C::MB, full);
   }
   if constexpr (C::HAS_ALPHA) bulk_g2s(smem_u32(st + C::O_AL), P.alpha[0] + rec0 * 4, nrec * 4, full);
+}
+
+// one token's (scale, offset) pairs of NG groups (fp16 pairs), zero past the context
+template <int NG>
+__device__ __forceinline__ void token_meta(const uint8_t* rec, bool valid, float (&sc)[NG], float (&zo)[NG]) {
+#pragma unroll
+  for (int g = 0; g < NG; g += 4) {
+    const uint4 m4 = *reinterpret_cast<const uint4*>(rec + 4 * g);
+    const uint32_t w4[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 a = half2_bits_to_f2(w4[u]);
+      sc[g + u] = valid ? a.x : 0.f;
+      zo[g + u] = valid ? a.y : 0.f;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -385,15 +414,25 @@ __global__ void __launch_bounds__(kNT, 1)
           tc::fence_after_sync();
           if constexpr (REF == kRefInt4) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-              tc::mma_s8(tbase + C::S_REF + C::N_SA * c, tc::desc_k_sw128(smem_u32(URKm + 32 * c)),
-                         tc::desc_k_sw128(smem_u32(QAm + 32 * c)), C::ID_SA, 0);
+            for (int c = 0; c < 4; ++c) {
+              if constexpr (C::KTM)
+                tc::mma_s8_ta(tbase + C::S_REF + C::N_SA * c, tbase + C::TK_REF + 8 * c,
+                              tc::desc_k_sw128(smem_u32(QAm + 32 * c)), C::ID_SA, 0);
+              else
+                tc::mma_s8(tbase + C::S_REF + C::N_SA * c, tc::desc_k_sw128(smem_u32(URKm + 32 * c)),
+                           tc::desc_k_sw128(smem_u32(QAm + 32 * c)), C::ID_SA, 0);
+            }
           }
           if constexpr (RB != 0) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-              tc::mma_s8(tbase + C::S_RES + C::N_SR * c, tc::desc_k_sw128(smem_u32(UKm + 32 * c)),
-                         tc::desc_k_sw128(smem_u32(HQm + 32 * c)), C::ID_SR, 0);
+            for (int c = 0; c < 4; ++c) {
+              if constexpr (C::KTM)
+                tc::mma_s8_ta(tbase + C::S_RES + C::N_SR * c, tbase + C::TK_RES + 8 * c,
+                              tc::desc_k_sw128(smem_u32(HQm + 32 * c)), C::ID_SR, 0);
+              else
+                tc::mma_s8(tbase + C::S_RES + C::N_SR * c, tc::desc_k_sw128(smem_u32(UKm + 32 * c)),
+                           tc::desc_k_sw128(smem_u32(HQm + 32 * c)), C::ID_SR, 0);
+            }
           }
         }
         tc::commit(smem_u32(sbar));
@@ -464,8 +503,7 @@ __global__ void __launch_bounds__(kNT, 1)
 
   // query operands of the G heads of (b, h), for the score MMAs
   auto setup = [&](int b, int h) {
-    if (warp < G) {
-      const int hq = warp;
+    for (int hq = warp; hq < G; hq += kNCW) {
       const uint2 raw = *reinterpret_cast<const uint2*>(P.q + q_row_offset(P, b, h, hq) + 4 * lane);
       const int d = 4 * lane;
       if constexpr (REF == kRefBf16) {
@@ -507,9 +545,25 @@ __global__ void __launch_bounds__(kNT, 1)
   };
   // warpgroup 0: key-side code tiles of the page in stage `st`
   auto expand_keys = [&](const uint8_t* st) {
-    if constexpr (RB != 0) expand_row<RB>(st + C::O_RESK + r * C::CB, UK, r);
-    if constexpr (REF == kRefInt4) expand_row<4>(st + C::O_REFK + r * 64, URK, r);
-    fence_proxy_async_smem();
+    if constexpr (C::KTM) {
+      // token r's codes into tensor-memory lane r (its warp's quarter)
+      if constexpr (REF == kRefInt4) {
+        uint32_t o[32];
+        widen_codes<4>(st + C::O_REFK + r * 64, o);
+        tc::tmem_st_x32(tl + C::TK_REF, o);
+      }
+      if constexpr (RB != 0) {
+        uint32_t o[32];
+        widen_codes<RB>(st + C::O_RESK + r * C::CB, o);
+        tc::tmem_st_x32(tl + C::TK_RES, o);
+      }
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+    } else {
+      if constexpr (RB != 0) expand_row<RB>(st + C::O_RESK + r * C::CB, UK, r);
+      if constexpr (REF == kRefInt4) expand_row<4>(st + C::O_REFK + r * 64, URK, r);
+      fence_proxy_async_smem();
+    }
     if constexpr (NEED_KREADY) {
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(kready));
@@ -569,35 +623,43 @@ __global__ void __launch_bounds__(kNT, 1)
       aV = a.y;
     }
     if (!valid) aK = aV = 0.f;
+    // with 16 rows the value-side metadata is read after the scores (the stage
+    // stays until the page's value MMAs complete), so that fewer registers are
+    // live across the score reads
     float sK[NGR > 0 ? NGR : 1], zK[NGR > 0 ? NGR : 1], sV[NGR > 0 ? NGR : 1], zV[NGR > 0 ? NGR : 1];
-    if constexpr (RB != 0) {
+    float sAk[4], zAk[4], sAv[4], zAv[4];
+    if constexpr (C::KTM) {
+      if constexpr (RB != 0) token_meta(st + C::O_RESMK + r * C::MB, valid, sK, zK);
+      if constexpr (REF == kRefInt4) token_meta(st + C::O_REFMK + r * 16, valid, sAk, zAk);
+    } else {
+      if constexpr (RB != 0) {
 #pragma unroll
-      for (int g = 0; g < NGR; g += 4) {
-        const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_RESMK + r * C::MB + 4 * g);
-        const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_RESMV + r * C::MB + 4 * g);
+        for (int g = 0; g < NGR; g += 4) {
+          const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_RESMK + r * C::MB + 4 * g);
+          const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_RESMV + r * C::MB + 4 * g);
+          const uint32_t wk[4] = {mk.x, mk.y, mk.z, mk.w}, wv[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 a = half2_bits_to_f2(wk[u]), c2 = half2_bits_to_f2(wv[u]);
+            sK[g + u] = valid ? a.x : 0.f;
+            zK[g + u] = valid ? a.y : 0.f;
+            sV[g + u] = valid ? c2.x : 0.f;
+            zV[g + u] = valid ? c2.y : 0.f;
+          }
+        }
+      }
+      if constexpr (REF == kRefInt4) {
+        const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_REFMK + r * 16);
+        const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_REFMV + r * 16);
         const uint32_t wk[4] = {mk.x, mk.y, mk.z, mk.w}, wv[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float2 a = half2_bits_to_f2(wk[u]), c2 = half2_bits_to_f2(wv[u]);
-          sK[g + u] = valid ? a.x : 0.f;
-          zK[g + u] = valid ? a.y : 0.f;
-          sV[g + u] = valid ? c2.x : 0.f;
-          zV[g + u] = valid ? c2.y : 0.f;
+          sAk[u] = valid ? a.x : 0.f;
+          zAk[u] = valid ? a.y : 0.f;
+          sAv[u] = valid ? c2.x : 0.f;
+          zAv[u] = valid ? c2.y : 0.f;
         }
-      }
-    }
-    float sAk[4], zAk[4], sAv[4], zAv[4];
-    if constexpr (REF == kRefInt4) {
-      const uint4 mk = *reinterpret_cast<const uint4*>(st + C::O_REFMK + r * 16);
-      const uint4 mv = *reinterpret_cast<const uint4*>(st + C::O_REFMV + r * 16);
-      const uint32_t wk[4] = {mk.x, mk.y, mk.z, mk.w}, wv[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float2 a = half2_bits_to_f2(wk[u]), c2 = half2_bits_to_f2(wv[u]);
-        sAk[u] = valid ? a.x : 0.f;
-        zAk[u] = valid ? a.y : 0.f;
-        sAv[u] = valid ? c2.x : 0.f;
-        zAv[u] = valid ? c2.y : 0.f;
       }
     }
 
@@ -618,37 +680,41 @@ __global__ void __launch_bounds__(kNT, 1)
       for (int i = 0; i < GH; ++i) S[i] = __uint_as_float(v[i]) * ak;
     }
     if constexpr (REF == kRefInt4 || RB != 0) {
+      constexpr int HB = GH > 4 ? 4 : GH;  // heads per tensor-memory read
       float dotA[GH], offA[GH], dotR[GH], offR[GH];
 #pragma unroll
       for (int i = 0; i < GH; ++i) dotA[i] = offA[i] = dotR[i] = offR[i] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t va[3 * GH], vr[C::NPAR][3 * GH];
-        if constexpr (REF == kRefInt4) tc::tmem_ld_n<3 * GH>(tl + C::S_REF + C::N_SA * c + 3 * hb, va);
-        if constexpr (RB != 0) {
 #pragma unroll
-          for (int p = 0; p < C::NPAR; ++p)
-            tc::tmem_ld_n<3 * GH>(tl + C::S_RES + C::N_SR * c + p * 3 * G + 3 * hb, vr[p]);
-        }
-        tc::tmem_wait_ld();
-        if constexpr (REF == kRefInt4) tc::reg_fence(va);
-        if constexpr (RB != 0) {
-#pragma unroll
-          for (int p = 0; p < C::NPAR; ++p) tc::reg_fence(vr[p]);
-        }
-#pragma unroll
-        for (int i = 0; i < GH; ++i) {
-          const int hq = hb + i;
-          if constexpr (REF == kRefInt4) {
-            dotA[i] = fmaf(sAk[c], comb24(va[3 * i], va[3 * i + 1], va[3 * i + 2]), dotA[i]);
-            offA[i] = fmaf(zAk[c], sQA[hq * 4 + c], offA[i]);
-          }
+        for (int h0 = 0; h0 < GH; h0 += HB) {
+          uint32_t va[3 * HB], vr[C::NPAR][3 * HB];
+          if constexpr (REF == kRefInt4) tc::tmem_ld_n<3 * HB>(tl + C::S_REF + C::N_SA * c + 3 * (hb + h0), va);
           if constexpr (RB != 0) {
 #pragma unroll
-            for (int p = 0; p < C::NPAR; ++p) {
-              const int g = c * C::NPAR + p;
-              dotR[i] = fmaf(sK[g], comb24(vr[p][3 * i], vr[p][3 * i + 1], vr[p][3 * i + 2]), dotR[i]);
-              offR[i] = fmaf(zK[g], sQS[hq * 8 + g], offR[i]);
+            for (int p = 0; p < C::NPAR; ++p)
+              tc::tmem_ld_n<3 * HB>(tl + C::S_RES + C::N_SR * c + p * 3 * G + 3 * (hb + h0), vr[p]);
+          }
+          tc::tmem_wait_ld();
+          if constexpr (REF == kRefInt4) tc::reg_fence(va);
+          if constexpr (RB != 0) {
+#pragma unroll
+            for (int p = 0; p < C::NPAR; ++p) tc::reg_fence(vr[p]);
+          }
+#pragma unroll
+          for (int i = 0; i < HB; ++i) {
+            const int hi = h0 + i, hq = hb + hi;
+            if constexpr (REF == kRefInt4) {
+              dotA[hi] = fmaf(sAk[c], comb24(va[3 * i], va[3 * i + 1], va[3 * i + 2]), dotA[hi]);
+              offA[hi] = fmaf(zAk[c], sQA[hq * 4 + c], offA[hi]);
+            }
+            if constexpr (RB != 0) {
+#pragma unroll
+              for (int p = 0; p < C::NPAR; ++p) {
+                const int g = c * C::NPAR + p;
+                dotR[hi] = fmaf(sK[g], comb24(vr[p][3 * i], vr[p][3 * i + 1], vr[p][3 * i + 2]), dotR[hi]);
+                offR[hi] = fmaf(zK[g], sQS[hq * 8 + g], offR[hi]);
+              }
             }
           }
         }
@@ -660,6 +726,10 @@ __global__ void __launch_bounds__(kNT, 1)
         if constexpr (RB != 0) S[i] += fmaf(dotR[i], sCS[hq], offR[i]);
       }
     }
+    if constexpr (C::KTM) {
+      if constexpr (RB != 0) token_meta(st + C::O_RESMV + r * C::MB, valid, sV, zV);
+      if constexpr (REF == kRefInt4) token_meta(st + C::O_REFMV + r * 16, valid, sAv, zAv);
+    }
 #pragma unroll
     for (int i = 0; i < GH; ++i) S[i] = valid ? S[i] : -INFINITY;
 
@@ -667,7 +737,7 @@ __global__ void __launch_bounds__(kNT, 1)
 #pragma unroll
     for (int i = 0; i < GH; ++i) {
       const float v = warp_max(S[i]);
-      if (lane == 0) sWM[(wg * 4 + (warp & 3)) * 4 + i] = v;
+      if (lane == 0) sWM[(wg * 4 + (warp & 3)) * C::GHS + i] = v;
     }
     if constexpr (RB != 0) {
 #pragma unroll
@@ -687,8 +757,8 @@ __global__ void __launch_bounds__(kNT, 1)
     float pm[GH], crun[GH], prel[GH];
 #pragma unroll
     for (int i = 0; i < GH; ++i) {
-      const float* wm = sWM + wg * 16 + i;
-      const float mp = fmaxf(fmaxf(wm[0], wm[4]), fmaxf(wm[8], wm[12]));
+      const float* wm = sWM + wg * (4 * C::GHS) + i;
+      const float mp = fmaxf(fmaxf(wm[0], wm[C::GHS]), fmaxf(wm[2 * C::GHS], wm[3 * C::GHS]));
       const float mn = fmaxf(m_run[i], mp);
       crun[i] = fast_exp2(m_run[i] - mn);
       pm[i] = fast_exp2(mp - mn);
@@ -726,7 +796,10 @@ __global__ void __launch_bounds__(kNT, 1)
         }
         const int n0 = wgo * G;  // rows n = 2 * head + (0: hi, 1: lo)
         uint8_t* dst = WB + (n0 >> 3) * 2048 + wrow + (n0 & 7) * 2;
-        if constexpr (GH == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if constexpr (GH == 8) {
+          *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(dst + 2048) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else if constexpr (GH == 4) *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         else if constexpr (GH == 2) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
         else *reinterpret_cast<uint32_t*>(dst) = pk[0];
       }
@@ -893,7 +966,7 @@ __global__ void __launch_bounds__(kNT, 1)
     if (seg_end) {
       // per-warp sums into their own slots, added in a fixed order below, so
       // that a decode is reproducible bit for bit from run to run
-      float* myred = sRed + (warp & 3) * 8 * C::NRED;
+      float* myred = sRed + (warp & 3) * C::GS * C::NRED;
 #pragma unroll
       for (int i = 0; i < GH; ++i) {
         const int hq = hb + i;
@@ -923,7 +996,8 @@ __global__ void __launch_bounds__(kNT, 1)
       named_bar_sync(kBarAll, kNCT);  // both warpgroups' sums (G == 1 splits them)
       auto red = [&](int hq, int slot) {
         const float* p = sRed + hq * C::NRED + slot;
-        return __fadd_rn(__fadd_rn(p[0], p[8 * C::NRED]), __fadd_rn(p[16 * C::NRED], p[24 * C::NRED]));
+        constexpr int WS = C::GS * C::NRED;  // one warp's slots
+        return __fadd_rn(__fadd_rn(p[0], p[WS]), __fadd_rn(p[2 * WS], p[3 * WS]));
       };
       const int pair = cur.b * Hkv + cur.h;
       const int d_ref = REF == kRefInt4 ? 32 * chunk + pos_dim<4>(r & 31) : r;
@@ -1006,6 +1080,7 @@ TcFn tc_pick_g(int G) {
     case 2: return tc_if_fits<REF, RB, RG, 2>();
     case 4: return tc_if_fits<REF, RB, RG, 4>();
     case 8: return tc_if_fits<REF, RB, RG, 8>();
+    case 16: return tc_if_fits<REF, RB, RG, 16>();
     default: return nullptr;
   }
 }

@@ -209,6 +209,28 @@ __device__ __forceinline__ void put_plane(uint8_t* tile, int n0, int wrow, const
   }
 }
 
+// One token's packed codes widened to int8, in 32-bit words, chunk-major: word
+// 8c + u holds bytes 4u .. 4u + 3 of 32-dim chunk c, in the order of
+// pos_dim / dim_pos (the layout expand_row writes into a shared tile).
+template <int BITS>
+__device__ __forceinline__ void widen_codes(const uint8_t* src, uint32_t (&o)[32]) {
+  constexpr int NW = BITS * 4;  // packed 32-bit words per token
+  uint32_t w[NW];
+#pragma unroll
+  for (int i = 0; i < NW / 4; ++i) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src + 16 * i);
+    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+  }
+  constexpr int WPC = BITS == 2 ? 2 : 4;  // words per 32-dim chunk
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int k = u / WPC, ww = u % WPC;
+      o[8 * c + u] = BITS == 2 ? ((w[WPC * c + ww] >> (2 * k)) & 0x03030303u) : ((w[WPC * c + ww] >> (4 * k)) & 0x0F0F0F0Fu);
+    }
+}
+
 // 65536 b2 + 256 b1 + b0 of three int32 byte-products (as fp32)
 __device__ __forceinline__ float comb24(uint32_t b2, uint32_t b1, uint32_t b0) {
   return fmaf(65536.f, static_cast<float>(static_cast<int>(b2)),

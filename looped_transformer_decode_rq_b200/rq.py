@@ -41,7 +41,7 @@ EXPORTED = ("rq_cache_layout", "rq_cache_create", "rq_cache_destroy", "rq_cache_
             "rq_bf16_decode_attention", "rq_reconstruct", "rq_get_error", "rq_status_string",
             "rq_last_error_message", "rq_decode_attention_static_scratch", "rq_cache_set_decode_kernel",
             "rq_cache_set_debug_stall", "rq_decode_attention_append", "rq_decode_multi_workspace_size",
-            "rq_decode_attention_multi")
+            "rq_decode_attention_multi", "rq_decode_plan")
 STATIC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 
@@ -72,6 +72,7 @@ _sig = {
     "rq_cache_set_debug_stall": (C.c_int, [_vp, _i32]),
     "rq_decode_workspace_size": (C.c_int, [_vp, C.POINTER(_i64)]),
     "rq_decode_multi_workspace_size": (C.c_int, [_vp, _i32, C.POINTER(_i64)]),
+    "rq_decode_plan": (C.c_int, [_vp, _i32, _i32, C.POINTER(_i32), C.POINTER(_i32)]),
     "rq_decode_attention_multi": (C.c_int, [_vp, _i32, _vp, _i32, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp]),
     "rq_decode_attention": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _i64, _vp]),
     "rq_decode_attention_static_scratch": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp]),
@@ -238,6 +239,13 @@ class Cache:
                                         _ptr(v_tail), n_tail, scale, out.data_ptr(), self.workspace.data_ptr(),
                                         self.workspace.numel(), _stream(stream)), "rq_decode_attention")
         return out
+
+    def decode_plan(self, loop: int, n_q: int = 1):
+        """(kernel, rows per pass over the cache) that a decode of `loop` with
+        n_q draft tokens takes on this handle (rq_decode_plan)."""
+        k, rows = _i32(0), _i32(0)
+        _check(_lib.rq_decode_plan(self._h, loop, n_q, C.byref(k), C.byref(rows)), "rq_decode_plan")
+        return k.value, rows.value
 
     def decode_attention_multi(self, loop: int, q: torch.Tensor, ctx_len: torch.Tensor,
                                k_tail: torch.Tensor, v_tail: torch.Tensor, softmax_scale: Optional[float] = None,

@@ -428,7 +428,7 @@ def test_any_workspace_contents_repeated_calls_and_graph_replay(librq, kernel):
     (1, 4, (2, 2, 2, 16), "simt"),
     (2, 4, (2, 2, 4, 4), None),           # GQA pairs x 4 drafts = 8 rows, INT4 anchor
     (1, 8, (2, 2, 2, 16), "simt"),
-    (4, 4, (2, 2, 2, 16), None),          # 16 rows: two blocks of 8, one cache pass each
+    (4, 4, (2, 2, 2, 16), None),          # 16 rows: one pass on the tensor cores
     (1, 16, (2, 2, 4, 4), None),
     (1, 4, (2, 2, 2, 16), "next_loop"),   # draft tokens on a Next-loop chained cache (CUDA cores)
     (2, 4, (2, 2, 2, 4), "next_loop"),    # 8 rows of a chain: two passes of 4 by default
@@ -457,6 +457,40 @@ def test_multi_query_decode(librq, gq, n_q, bits, kernel):
         want = O.decode_attention_multi_f64(enc, loop, to_np32(qm[loop]), ctx.numpy(), to_np32(kt), to_np32(vt))
         err = rel_err_rows(out.cpu().numpy(), want)
         assert err.max() <= ATTN_TOL, (loop, float(err.max()))
+    assert cache.get_error() == 0
+
+
+@pytest.mark.parametrize("bits,rows_of_loop", [
+    ((2, 2, 2, 16), {0: 16, 3: 16}),        # bf16 anchor, INT2 g=32: 16 rows in one pass
+    ((2, 2, 4, 4), {0: 8, 2: 8, 3: 16}),    # INT4 anchor: its own loop in one pass, residual loops in two
+])
+def test_sixteen_rows_per_pass(librq, bits, rows_of_loop):
+    """4 query heads per kv-head x 4 draft tokens: where the tensor-core kernel
+    has a 16-row variant the call reads each cached page once for all 16 rows
+    (rq_decode_plan), and every loop matches the float64 oracle."""
+    rq = librq
+    gq, n_q = 4, 4
+    wl = synth.Workload(name=f"rows16_{bits}", batch=2, kv_heads=2, q_heads=2 * gq, context=400, bits=bits,
+                        sigma=(0.3, 0.2, 0.1), outlier_p=0.01, n_tail=n_q, seed=170 + bits[2])
+    wl = wl.with_(lengths=(400, 131))
+    inp = synth.make_inputs(wl, "cpu")
+    qm = synth.draft_queries(wl, n_q, "cpu")
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
+    cache.encode(inp["k"].cuda(), inp["v"].cuda())
+    enc = oracle_encode(inp, cfgd)
+    ctx = inp["ctx_len"]
+    for loop, rows in rows_of_loop.items():
+        assert cache.decode_plan(loop, n_q) == (rq.DECODE_KERNEL_TENSOR, rows), loop
+        kt, vt = inp["k_tail"][loop], inp["v_tail"][loop]
+        out = cache.decode_attention_multi(loop, qm[loop].cuda(), ctx.cuda(), kt.cuda(), vt.cuda())
+        torch.cuda.synchronize()
+        want = O.decode_attention_multi_f64(enc, loop, to_np32(qm[loop]), ctx.numpy(), to_np32(kt), to_np32(vt))
+        err = rel_err_rows(out.cpu().numpy(), want)
+        assert err.max() <= ATTN_TOL, (loop, float(err.max()))
+    # forced onto the CUDA cores the same call runs in 4-row passes
+    cache.set_decode_kernel(rq.DECODE_KERNEL_SIMT)
+    assert cache.decode_plan(0, n_q) == (rq.DECODE_KERNEL_SIMT, 4)
     assert cache.get_error() == 0
 
 
