@@ -299,11 +299,11 @@ RQ_API rq_status rq_decode_multi_workspace_size(const rq_cache* cache, int32_t n
  * keys and values (bf16, not yet encoded), each visible to itself and to the
  * later ones, and any earlier tail tokens to all.  Up to 8 query rows per
  * kv-head (n_q * G) share every read of its cached pages, and 16 rows do where
- * the tensor-core kernel has a 16-row variant for the loop's format (bf16
- * anchor with INT2 g=32 residuals, an INT4 or bf16 anchor loop, no anchor with
- * g=32 residuals) and the call takes that kernel; other rows run in blocks of 16
- * or 8, one pass over the cache each.  With 4 or more rows in a block the
- * automatic kernel choice is the tensor-core kernel.
+ * the tensor-core kernel has a 16-row variant for the loop's format (residuals
+ * in 32-dim groups with an INT4 anchor or none, INT2 g=32 residuals with a bf16
+ * anchor, and both anchor loops) and the call takes that kernel; other rows run
+ * in blocks of 16 or 8, one pass over the cache each.  With 4 or more rows in a
+ * block the automatic kernel choice is the tensor-core kernel.
  *  q        device bf16 [B][n_q][Hq][128]
  *  out      device fp32 [B][n_q][Hq][128]
  *  n_q      in [1, RQ_MAX_DRAFT] (else RQ_ERR_INVALID_ARG) with n_q * (Hq / Hkv)

@@ -48,6 +48,15 @@ constexpr int kNCT = kNCW * 32;
 constexpr int kProducerWarp = kNCW;
 constexpr int kMmaWarp = kNCW + 1;
 constexpr int kNT = kNCT + 64; // + producer warp + MMA-issuing warp
+// Register split of the variants that need more than 168 registers per
+// consumer thread: a third warpgroup (producer, MMA issuer, two spare warps)
+// launched with the others at 168 registers a thread gives up all but kRegsAux,
+// and the two consumer warpgroups take them:
+//   384 threads x 168 = 128 x kRegsAux + 256 x kRegsConsumer.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsAux = 56;
+constexpr int kRegsConsumer = 224;
+static_assert(384 * kLaunchRegs == 128 * kRegsAux + 256 * kRegsConsumer, "register split");
 constexpr int kBarAll = 1;     // the 256 consumer threads
 constexpr int kBarWG = 2;      // warpgroup w uses kBarWG + w
 constexpr int kSmemLimit = 227 * 1024;
@@ -82,18 +91,23 @@ struct TcCfg {
   static constexpr bool KTM = G == 16;
   // tensor-memory columns: scores, then value sums (separate, so that the next
   // page's scores can be computed while this page's value sums are read), then
-  // the key codes of the 16-row variants
+  // the key codes of the 16-row variants.  Where that exceeds the 512 columns
+  // (16 rows with an INT4 anchor and residual links) the value sums overlay the
+  // scores, and the next page's score MMAs wait until this page's sums are read.
   static constexpr int S_REF = 0;
   static constexpr int S_REF_COLS = REF == kRefBf16 ? 16 : (REF == kRefInt4 ? 4 * N_SA : 0);
   static constexpr int S_RES = S_REF + S_REF_COLS;
   static constexpr int S_COLS = S_RES + (RB ? 4 * N_SR : 0);
-  static constexpr int O_REF = S_COLS;
   static constexpr int O_REF_COLS = REF == kRefBf16 ? N_VB : (REF == kRefInt4 ? N_VA : 0);
+  static constexpr int O_SIZE = O_REF_COLS + (RB ? N_VR : 0);
+  static constexpr int KT_COLS = KTM ? (REF == kRefInt4 ? 32 : 0) + (RB ? 32 : 0) : 0;
+  static constexpr bool ALIAS = KTM && S_COLS + O_SIZE + KT_COLS > 512;
+  static constexpr int O_REF = ALIAS ? 0 : S_COLS;
   static constexpr int O_RES = O_REF + O_REF_COLS;
   static constexpr int O_COLS = O_RES + (RB ? N_VR : 0);
-  static constexpr int TK_REF = O_COLS;                               // INT4 anchor key codes (KTM)
+  static constexpr int TK_REF = S_COLS > O_COLS ? S_COLS : O_COLS;   // INT4 anchor key codes (KTM)
   static constexpr int TK_RES = TK_REF + (REF == kRefInt4 ? 32 : 0);  // residual key codes (KTM)
-  static constexpr int COLS = O_COLS + (KTM ? (REF == kRefInt4 ? 32 : 0) + (RB ? 32 : 0) : 0);
+  static constexpr int COLS = TK_REF + KT_COLS;
   static constexpr int TMEM_COLS = COLS <= 32 ? 32 : COLS <= 64 ? 64 : COLS <= 128 ? 128 : COLS <= 256 ? 256 : 512;
   // stage layout (pieces 1024-byte aligned)
   static constexpr int al(int x) { return (x + 1023) & ~1023; }
@@ -138,11 +152,11 @@ struct TcCfg {
   static constexpr int FIXED = 1024 + F_END + SMALL_BYTES;
   static constexpr int STAGES_FIT = (kSmemLimit - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT >= 4 ? 4 : (STAGES_FIT >= 2 ? STAGES_FIT : 2);
-  // 16 rows with an INT4 anchor and residual links would keep both offset sums
-  // of 8 heads per thread and spill registers: those run as two 8-row passes
-  static constexpr bool REGS_FIT = !(G == 16 && REF == kRefInt4 && RB != 0);
-  static constexpr bool FITS =
-      STAGES_FIT >= 2 && COLS <= 512 && N_VA <= 256 && N_VR <= 256 && N_SR <= 256 && REGS_FIT;
+  // An INT4 anchor with residual links keeps both offset sums of its heads per
+  // thread: from 2 rows on those variants take the register split
+  static constexpr bool REGSPLIT = REF == kRefInt4 && RB != 0 && G >= 2;
+  static constexpr int NT = REGSPLIT ? kNCT + 128 : kNT;
+  static constexpr bool FITS = STAGES_FIT >= 2 && COLS <= 512 && N_VA <= 256 && N_VR <= 256 && N_SR <= 256;
   static constexpr int SMEM_BYTES = FIXED + STAGES * STAGE_BYTES;
   // instruction descriptors
   static constexpr uint32_t ID_SB = tc::instr_desc(tc::kAccF32, tc::kFmtBf16, tc::kFmtBf16, 0, 0, 128, 16);
@@ -212,7 +226,7 @@ __device__ __forceinline__ void token_meta(const uint8_t* rec, bool valid, float
 // split kernel
 // ---------------------------------------------------------------------------
 template <int REF, int RB, int RG, int G>
-__global__ void __launch_bounds__(kNT, 1)
+__global__ void __launch_bounds__(TcCfg<REF, RB, RG, G>::NT, 1)
     decode_tc_kernel(const __grid_constant__ DecodeParams P, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV) {
   using C = TcCfg<REF, RB, RG, G>;
@@ -348,6 +362,12 @@ __global__ void __launch_bounds__(kNT, 1)
   tc::fence_after_sync();
   const uint32_t tbase = *sTmem;
 
+  // the producer warpgroup: producer warp, MMA-issuing warp (and, with the
+  // register split, two spare warps); no path out of it reaches the consumers'
+  // code, so each side is compiled for its own register budget
+  if (warp >= kNCW) {
+  if constexpr (C::REGSPLIT) tc::setmaxnreg_dec<kRegsAux>();
+
   // ========================= producer warp =========================
   if (warp == kProducerWarp) {
     if (lane == 0) {
@@ -386,17 +406,21 @@ __global__ void __launch_bounds__(kNT, 1)
   // MMAs in two groups as their weight operands are written.
   if (warp == kMmaWarp) {
     if (lane == 0) {
-      uint8_t* UKm = fx + C::F_UK;
-      uint8_t* UVm = fx + C::F_UV;
-      uint8_t* URKm = fx + C::F_URK;
-      uint8_t* URVm = fx + C::F_URV;
-      uint8_t* QBm = fx + C::F_QB;
-      uint8_t* QAm = fx + C::F_QA;
-      uint8_t* HQm = fx + C::F_HQ;
-      uint8_t* WBm = fx + C::F_WB;
-      uint8_t* WAm = fx + C::F_WA;
-      uint8_t* WRm = fx + C::F_WR;
       for (int k = 0; k < n_pages; ++k) {
+        // with the register split this warp has few registers: the operand
+        // descriptors are recomputed every page rather than kept
+        uint8_t* fxk = fx;
+        if constexpr (C::REGSPLIT) asm volatile("" : "+l"(fxk));
+        uint8_t* UKm = fxk + C::F_UK;
+        uint8_t* UVm = fxk + C::F_UV;
+        uint8_t* URKm = fxk + C::F_URK;
+        uint8_t* URVm = fxk + C::F_URV;
+        uint8_t* QBm = fxk + C::F_QB;
+        uint8_t* QAm = fxk + C::F_QA;
+        uint8_t* HQm = fxk + C::F_HQ;
+        uint8_t* WBm = fxk + C::F_WB;
+        uint8_t* WAm = fxk + C::F_WA;
+        uint8_t* WRm = fxk + C::F_WR;
         const int s = k % C::STAGES;
         uint8_t* st = stages + s * C::STAGE_BYTES;
         const uint32_t ph = k & 1;
@@ -466,6 +490,9 @@ __global__ void __launch_bounds__(kNT, 1)
     }
     return;
   }
+  return;  // spare warps
+  }
+  if constexpr (C::REGSPLIT) tc::setmaxnreg_inc<kRegsConsumer>();
 
   // ========================= consumer warpgroups =========================
   // G >= 2: warpgroup wg scores and sums query heads [wg GH, wg GH + GH).
@@ -704,16 +731,17 @@ __global__ void __launch_bounds__(kNT, 1)
 #pragma unroll
           for (int i = 0; i < HB; ++i) {
             const int hi = h0 + i, hq = hb + hi;
+            // (16 rows: the offsets are summed after the chunks, in the same order)
             if constexpr (REF == kRefInt4) {
               dotA[hi] = fmaf(sAk[c], comb24(va[3 * i], va[3 * i + 1], va[3 * i + 2]), dotA[hi]);
-              offA[hi] = fmaf(zAk[c], sQA[hq * 4 + c], offA[hi]);
+              if constexpr (!C::KTM) offA[hi] = fmaf(zAk[c], sQA[hq * 4 + c], offA[hi]);
             }
             if constexpr (RB != 0) {
 #pragma unroll
               for (int p = 0; p < C::NPAR; ++p) {
                 const int g = c * C::NPAR + p;
                 dotR[hi] = fmaf(sK[g], comb24(vr[p][3 * i], vr[p][3 * i + 1], vr[p][3 * i + 2]), dotR[hi]);
-                offR[hi] = fmaf(zK[g], sQS[hq * 8 + g], offR[hi]);
+                if constexpr (!C::KTM) offR[hi] = fmaf(zK[g], sQS[hq * 8 + g], offR[hi]);
               }
             }
           }
@@ -722,6 +750,16 @@ __global__ void __launch_bounds__(kNT, 1)
 #pragma unroll
       for (int i = 0; i < GH; ++i) {
         const int hq = hb + i;
+        if constexpr (C::KTM) {
+          if constexpr (REF == kRefInt4) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) offA[i] = fmaf(zAk[c], sQA[hq * 4 + c], offA[i]);
+          }
+          if constexpr (RB != 0) {
+#pragma unroll
+            for (int g = 0; g < NGR; ++g) offR[i] = fmaf(zK[g], sQS[hq * 8 + g], offR[i]);
+          }
+        }
         if constexpr (REF == kRefInt4) S[i] = aK * fmaf(dotA[i], sCA[hq], offA[i]);
         if constexpr (RB != 0) S[i] += fmaf(dotR[i], sCS[hq], offR[i]);
       }
@@ -816,26 +854,33 @@ __global__ void __launch_bounds__(kNT, 1)
     }
     if constexpr (REF == kRefInt4) {
       if (own_ref) {
-        // signed weights (alpha may be negative): three signed bytes each
+        // signed weights (alpha may be negative): three signed bytes each;
+        // with 8 heads a warpgroup writes them in two halves of the groups
         constexpr int NB = 4 * GH;
-        uint32_t v[NB];
+        constexpr int NH = NB > 16 ? 2 : 1;
+        constexpr int GPH = 4 / NH;
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const float t = siga[g] > 0.f ? aV * sAv[g] * rcp_approx(siga[g]) * kQ3 : 0.f;
+        for (int hh = 0; hh < NH; ++hh) {
+          uint32_t v[NB / NH];
 #pragma unroll
-          for (int i = 0; i < GH; ++i) {
-            int qi = __float2int_rn(prel[i] * t);
-            qi = max(-8323072, min(8323072, qi));
-            int b2, b1, b0;
-            split24(qi, b2, b1, b0);
-            v[g * GH + i] = (static_cast<uint32_t>(b0) & 0xFFu) | ((static_cast<uint32_t>(b1) & 0xFFu) << 8) |
-                            ((static_cast<uint32_t>(b2) & 0xFFu) << 16);
+          for (int gg = 0; gg < GPH; ++gg) {
+            const int g = hh * GPH + gg;
+            const float t = siga[g] > 0.f ? aV * sAv[g] * rcp_approx(siga[g]) * kQ3 : 0.f;
+#pragma unroll
+            for (int i = 0; i < GH; ++i) {
+              int qi = __float2int_rn(prel[i] * t);
+              qi = max(-8323072, min(8323072, qi));
+              int b2, b1, b0;
+              split24(qi, b2, b1, b0);
+              v[gg * GH + i] = (static_cast<uint32_t>(b0) & 0xFFu) | ((static_cast<uint32_t>(b1) & 0xFFu) << 8) |
+                               ((static_cast<uint32_t>(b2) & 0xFFu) << 16);
+            }
           }
-        }
-        uint32_t planes[3][NB / 4];
-        byte_planes<NB>(v, planes);
+          uint32_t planes[3][NB / NH / 4];
+          byte_planes<NB / NH>(v, planes);
 #pragma unroll
-        for (int j = 0; j < 3; ++j) put_plane<NB>(WA, j * 4 * G + wgo * NB, wrow, planes[j]);
+          for (int j = 0; j < 3; ++j) put_plane<NB / NH>(WA, j * 4 * G + wgo * NB + hh * (NB / NH), wrow, planes[j]);
+        }
       }
     }
     // the scores are in registers: the value sums may now be written
@@ -849,17 +894,23 @@ __global__ void __launch_bounds__(kNT, 1)
       if (own_res) {
         // non-negative weights p * s_g / max_page(s_g) as unsigned 24-bit integers
         constexpr int NB = NGR * GH;
-        uint32_t v[NB];
+        constexpr int NH = (NB > 16 && GH == 8 && C::REGSPLIT) ? 2 : 1;  // halves, as for the anchor
+        constexpr int GPH = NGR / NH;
 #pragma unroll
-        for (int g = 0; g < NGR; ++g) {
-          const float t = sig[g] > 0.f ? sV[g] * rcp_approx(sig[g]) * kU3 : 0.f;
+        for (int hh = 0; hh < NH; ++hh) {
+          uint32_t v[NB / NH];
 #pragma unroll
-          for (int i = 0; i < GH; ++i) v[g * GH + i] = min(__float2uint_rn(prel[i] * t), 16777215u);
+          for (int gg = 0; gg < GPH; ++gg) {
+            const int g = hh * GPH + gg;
+            const float t = sig[g] > 0.f ? sV[g] * rcp_approx(sig[g]) * kU3 : 0.f;
+#pragma unroll
+            for (int i = 0; i < GH; ++i) v[gg * GH + i] = min(__float2uint_rn(prel[i] * t), 16777215u);
+          }
+          uint32_t planes[3][NB / NH / 4];
+          byte_planes<NB / NH>(v, planes);
+#pragma unroll
+          for (int j = 0; j < 3; ++j) put_plane<NB / NH>(WR, j * NGR * G + wgo * NB + hh * (NB / NH), wrow, planes[j]);
         }
-        uint32_t planes[3][NB / 4];
-        byte_planes<NB>(v, planes);
-#pragma unroll
-        for (int j = 0; j < 3; ++j) put_plane<NB>(WR, j * NGR * G + wgo * NB, wrow, planes[j]);
       }
     }
     if constexpr (HAS_V2) {
@@ -895,7 +946,7 @@ __global__ void __launch_bounds__(kNT, 1)
         len_nxt = seq_len(nxt.b);
         setup(nxt.b, nxt.h);
       }
-      release_scores();
+      if constexpr (!C::ALIAS) release_scores();
       if (wg == 0) {
         wait_or_abort(&full[s1], ((k + 1) / C::STAGES) & 1);
         expand_keys(st1);
@@ -960,6 +1011,11 @@ __global__ void __launch_bounds__(kNT, 1)
           acc_res[i] = fmaf(acc_res[i], crun[i], pm[i] * f * comb24(b2, b1, b0));
         }
       }
+    }
+
+    // the value sums overlay the scores: page k + 1 may be scored once they are read
+    if constexpr (C::ALIAS) {
+      if (!last) release_scores();
     }
 
     // ---- flush a finished (b, h) segment: one partial record per query head
@@ -1061,7 +1117,7 @@ cudaError_t launch_tc(const DecodeParams& p, const CUtensorMap* tk, const CUtens
       if (e != cudaSuccess) return e;
       attr_done = true;
     }
-    return launch_dependent(kern, p.num_ctas, kNT, C::SMEM_BYTES, s, p, *tk, *tv);
+    return launch_dependent(kern, p.num_ctas, C::NT, C::SMEM_BYTES, s, p, *tk, *tv);
   }
 }
 

@@ -462,7 +462,7 @@ def test_multi_query_decode(librq, gq, n_q, bits, kernel):
 
 @pytest.mark.parametrize("bits,rows_of_loop", [
     ((2, 2, 2, 16), {0: 16, 3: 16}),        # bf16 anchor, INT2 g=32: 16 rows in one pass
-    ((2, 2, 4, 4), {0: 8, 2: 8, 3: 16}),    # INT4 anchor: its own loop in one pass, residual loops in two
+    ((2, 2, 4, 4), {0: 16, 2: 16, 3: 16}),  # INT4 anchor, INT2 and INT4 g=32 residuals
 ])
 def test_sixteen_rows_per_pass(librq, bits, rows_of_loop):
     """4 query heads per kv-head x 4 draft tokens: where the tensor-core kernel
