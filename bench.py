@@ -51,9 +51,11 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["rq", "reference"], default="rq")
-    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "next_loop", "next_loop_int4", "tiny", "capacity",
-                                           "mixed_sweep"],
+    ap.add_argument("--workload", choices=["ouro8k", "mixed", "gqa", "gqa_int4", "next_loop", "next_loop_int4", "tiny",
+                                           "capacity", "mixed_sweep", "verify_gqa"],
                     default="ouro8k")
+    ap.add_argument("--decode-kernel", choices=["auto", "simt", "tensor"], default="auto",
+                    help="decode kernel of the RQ cache (the automatic choice by default)")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
@@ -72,6 +74,8 @@ def make_workload(args) -> synth.Workload:
         return synth.mixed_int4_anchor(batch=args.batch or 8)
     if args.workload == "gqa":
         return synth.gqa_long(batch=args.batch or 8)
+    if args.workload == "gqa_int4":
+        return synth.gqa_long(batch=args.batch or 8, int4_anchor=True)
     if args.workload == "next_loop":
         return synth.ouro_8k_next_loop(batch=args.batch or 16)
     if args.workload == "next_loop_int4":
@@ -671,6 +675,8 @@ def run_rq(args, world, rank):
     e2e_warm = 3
     cfgd = synth.cache_config_dict(wl, capacity=T + 1 + (0 if args.no_e2e else e2e_warm + args.steps))
     cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
+    cache.set_decode_kernel({"auto": rq.DECODE_KERNEL_AUTO, "simt": rq.DECODE_KERNEL_SIMT,
+                             "tensor": rq.DECODE_KERNEL_TENSOR}[args.decode_kernel])
     cache.encode(inp["k"], inp["v"])
     ctx = inp["ctx_len"]
     tokens_total = int(ctx.sum().item())
@@ -859,6 +865,7 @@ def run_rq(args, world, rank):
         extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 30, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8), 30, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8, q_heads=64), 30, 3, world, rank),
+                 measure_workload(synth.gqa_long(batch=8, int4_anchor=True), 30, 3, world, rank),
                  measure_workload(synth.ouro_8k_next_loop(), 30, 3, world, rank, per_loop=True),
                  measure_workload(synth.ouro_8k_next_loop_int4(), 30, 3, world, rank, per_loop=True),
                  measure_multi_query(synth.ouro_8k(), 4, 30, 3, world, rank),
@@ -942,6 +949,11 @@ def main():
             run_capacity(args, world, rank)
         elif args.workload == "mixed_sweep":
             run_mixed_sweep(args, world, rank)
+        elif args.workload == "verify_gqa":
+            out = measure_multi_query(synth.gqa_long(batch=args.batch or 8), 4, max(3, args.steps),
+                                      max(3, args.warmup), world, rank)
+            if rank == 0:
+                print(json.dumps(out))
         else:
             run_rq(args, world, rank)
     finally:

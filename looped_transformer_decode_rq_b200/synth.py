@@ -126,11 +126,13 @@ def capacity_24layer(batch: int = 1, context: int = 8192) -> Workload:
                     seed=3, layers=24)
 
 
-def gqa_long(batch: int = 8, context: int = 32768, q_heads: int = 32) -> Workload:
+def gqa_long(batch: int = 8, context: int = 32768, q_heads: int = 32, int4_anchor: bool = False) -> Workload:
     """4 loops, 32 (or `q_heads`) query heads / 8 KV heads, batch 8, ragged
-    lengths U{context/2 .. context}, INT2 loops 1-3 g=32, bf16 reference."""
-    return Workload(name=f"gqa_L4_Hq{q_heads}_Hkv8_B{batch}_T{context}_ragged", batch=batch,
-                    kv_heads=8, q_heads=q_heads, context=context,
+    lengths U{context/2 .. context}, INT2 loops 1-3 g=32, bf16 reference (or an
+    INT4 g=32 anchor: the [2,2,2,4] setting)."""
+    suffix = "_int4ref" if int4_anchor else ""
+    return Workload(name=f"gqa_L4_Hq{q_heads}_Hkv8_B{batch}_T{context}_ragged{suffix}", batch=batch,
+                    kv_heads=8, q_heads=q_heads, context=context, bits=(2, 2, 2, 4) if int4_anchor else (2, 2, 2, 16),
                     length_range=(context // 2, context), sigma=(0.3, 0.2, 0.1),
                     outlier_p=0.01, seed=4)
 
