@@ -185,25 +185,6 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
 
 __device__ __forceinline__ float bf16_bits_to_f(uint32_t lo16) { return __uint_as_float(lo16 << 16); }
 
-// The bits of 1.0f (0x3F800000) in a register the compiler cannot see
-// through.  An instruction carries at most one 32-bit immediate, so with both
-// the code mask and the exponent as immediates (w & mask) | exponent costs two
-// logic operations; with the exponent in this register it is one LOP3.
-__device__ __forceinline__ uint32_t opaque_one_bits() {
-  uint32_t lid;
-  asm volatile("mov.u32 %0, %%laneid;" : "=r"(lid));
-  return 0x3F800000u | (lid >> 5);  // lid < 32
-}
-
-// A b-bit code c sitting at bit p (p + b <= 23) of `w` becomes the float
-// 1 + c * 2^(p - 23) with one LOP3 ((w & mask) | one, one = opaque_one_bits());
-// subtracting 1 is then exact, and the 2^(p - 23) factor is folded into the
-// operand it multiplies.
-__device__ __forceinline__ float code_float(uint32_t w, uint32_t mask_at_p, uint32_t one) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "r"(mask_at_p), "r"(one));
-  return __uint_as_float(d);
-}
 
 // fp16 (scale, offset) pair packed in a 32-bit word
 __device__ __forceinline__ float2 half2_bits_to_f2(uint32_t w) {

@@ -24,8 +24,8 @@
 //     token t -- its softmax weight p, the products of the links' alpha_V,
 //     the weight of every (link, group) and the group offsets' sums -- and
 //     leaves the weights in shared memory;
-//   * values: 16 lanes per token, 8 dims per lane, one LOP3 per code into a
-//     float, fp32 pairs (FADD2/FFMA2);
+//   * values: 16 lanes per token, 8 dims per lane, one AND per code into a
+//     subnormal float (code_sub), fp32 pair FMAs;
 //   * at the end of a (b, kv-head) segment every warp leaves its state in a
 //     slot and the CTA adds the twelve slots in a fixed order into its partial
 //     record, so a decode is reproducible bit for bit.
@@ -107,7 +107,6 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int B = P.B, Hkv = P.Hkv;
-  const uint32_t one = opaque_one_bits();
   // a programmatic dependent of the previous kernel: nothing global is
   // touched before it has completed
   pdl_wait();
@@ -396,9 +395,11 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
             const uint4 mv = *reinterpret_cast<const uint4*>(st + S::O_REFMV + t * 16);
             const uint32_t m4[4] = {mv.x, mv.y, mv.z, mv.w};
 #pragma unroll
+            const float pas = pa * kSubScale;  // value weights carry the code scale (code_sub)
+#pragma unroll
             for (int g = 0; g < 4; ++g) {
               const float2 sz = half2_bits_to_f2(m4[g]);
-              wa[g] = pa * sz.x;
+              wa[g] = pas * sz.x;
               za[g] = fmaf(pa, sz.y, za[g]);
             }
           }
@@ -413,7 +414,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                   const float2 sz = half2_bits_to_f2(m4[u]);
-                  wr[ci][g4 + u] = wl[ci] * sz.x;
+                  wr[ci][g4 + u] = (wl[ci] * kSubScale) * sz.x;
                   zr[g4 + u] = fmaf(wl[ci], sz.y, zr[g4 + u]);
                 }
               }
@@ -463,7 +464,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
             const float2 ww = make_float2(w[0], w[0]);
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
-              const float2 f = f2sub1(make_float2(code_f<4>(cw1, e, one), code_f<4>(cw1, e + 1, one)));
+              const float2 f = make_float2(code_sub<4>(cw1, e), code_sub<4>(cw1, e + 1));
               acc_a[e / 2] = __ffma2_rn(ww, f, acc_a[e / 2]);
             }
             ++n;
@@ -477,7 +478,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
               const float2 ww = make_float2(wv, wv);
 #pragma unroll
               for (int e = 0; e < 8; e += 2) {
-                const float2 f = f2sub1(make_float2(code_f<RB>(cw, e, one), code_f<RB>(cw, e + 1, one)));
+                const float2 f = make_float2(code_sub<RB>(cw, e), code_sub<RB>(cw, e + 1));
                 acc_r[e / 2] = __ffma2_rn(ww, f, acc_r[e / 2]);
               }
             }
@@ -520,8 +521,8 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
         va = __fadd_rn(va, __shfl_xor_sync(kFull, va, 16));  // the two token parities
         vr = __fadd_rn(vr, __shfl_xor_sync(kFull, vr, 16));
         if (lane < 16) {
-          slot[4 + 8 * j2 + e] = ANCH ? fmaf(va, pow2i(23 - code_pos<4>(e)), zav) : 0.f;
-          slot[4 + kD + 8 * j2 + e] = RB ? fmaf(vr, pow2i(23 - code_pos<RB ? RB : 2>(e)), zrv) : 0.f;
+          slot[4 + 8 * j2 + e] = ANCH ? fmaf(va, pow2i(kSubExp - code_pos<4>(e)), zav) : 0.f;
+          slot[4 + kD + 8 * j2 + e] = RB ? fmaf(vr, pow2i(kSubExp - code_pos<RB ? RB : 2>(e)), zrv) : 0.f;
         }
       }
       if (lane == 0) {

@@ -24,9 +24,10 @@
 //     codes, shuffle reduction) and values (16 lanes per token row, 8 dims per
 //     lane, softmax weights recomputed per lane).  The groups merge once per
 //     segment, in a fixed order;
-//   * packed codes become floats with one LOP3 each (1 + c*2^(p-23)), the
-//     2^(p-23) factor being folded into the accumulators once per flush; fp32
-//     pairs use FFMA2.
+//   * packed codes become subnormal floats with one AND each (c * 2^(p-149),
+//     code_sub), against weights pre-multiplied by 2^100; the remaining power
+//     of two is folded into the accumulators once per flush; fp32 pairs use
+//     FFMA2.
 #pragma once
 
 #include "rq_common.cuh"
@@ -155,22 +156,26 @@ __device__ __forceinline__ void load_codes(const uint8_t* p, uint32_t (&w)[(NB +
   }
 }
 
-// code e of a thread's unit (bits per code BITS) as 1 + c*2^(p_e - 23)
-// (`one`: opaque_one_bits())
 template <int BITS>
-__device__ __forceinline__ float code_f(const uint32_t* w, int e, uint32_t one) {
+__device__ __forceinline__ int code_pos(int e) { return (e * BITS) & 15; }
+
+// Code e of a thread's unit as the subnormal float c * 2^(p_e - 149): one AND
+// leaves the code's bits in the mantissa under a zero exponent, so nothing has
+// to be subtracted.  The value weights are multiplied by kSubScale = 2^100
+// first, which keeps every product w * c a normal number (the FMA forms it
+// exactly), and an accumulator of code e is scaled by 2^(kSubExp - p_e) at the
+// end.  (Subnormals are kept: the library is built without flush-to-zero.)
+constexpr float kSubScale = 0x1p100f;
+constexpr int kSubExp = 49;
+template <int BITS>
+__device__ __forceinline__ float code_sub(const uint32_t* w, int e) {
   const int bit = e * BITS;
   const uint32_t word = w[bit >> 5];
   const int b32 = bit & 31;
   const uint32_t src = (b32 >= 16) ? (word >> 16) : word;
   const int p = b32 & 15;
-  return code_float(src, ((1u << BITS) - 1u) << p, one);
+  return __uint_as_float(src & (((1u << BITS) - 1u) << p));
 }
-
-template <int BITS>
-__device__ __forceinline__ int code_pos(int e) { return (e * BITS) & 15; }
-
-__device__ __forceinline__ float2 f2sub1(float2 f) { return __fadd2_rn(f, make_float2(-1.f, -1.f)); }
 
 // Integer-dot-product operands for a lane's D query values against BITS-bit
 // packed codes.  The values are quantised to int16 with one scale per lane
@@ -336,7 +341,6 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int B = P.B, Hkv = P.Hkv;
-  const uint32_t one = opaque_one_bits();
   // Launched as a programmatic dependent of the previous kernel on the stream
   // (typically the previous call's combine kernel, which reads the partials
   // this grid writes): everything above overlaps its tail; nothing global is
@@ -756,12 +760,13 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
           uint32_t cw[1];
           load_codes<C::D2 / 2>(st + C::O_REFV + t * 64 + (d2 >> 1), cw);
           const float2 sz = half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::O_REFMV + t * 16 + 4 * (d2 >> 5)));
+          const float sxs = sz.x * kSubScale;
 #pragma unroll
           for (int e = 0; e < C::D2; e += 2) {
-            const float2 f = f2sub1(make_float2(code_f<4>(cw, e, one), code_f<4>(cw, e + 1, one)));
+            const float2 f = make_float2(code_sub<4>(cw, e), code_sub<4>(cw, e + 1));
 #pragma unroll
             for (int gi = 0; gi < G; ++gi) {
-              const float w = pa[gi] * sz.x;
+              const float w = pa[gi] * sxs;
               acc_ref[gi][e / 2] = __ffma2_rn(make_float2(w, w), f, acc_ref[gi][e / 2]);
             }
           }
@@ -775,12 +780,13 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
             load_codes<C::D2 * RB / 8>(st + C::o_resv(ci) + t * C::CB + (d2 * RB >> 3), cw);
             const float2 sz =
                 half2_bits_to_f2(*reinterpret_cast<const uint32_t*>(st + C::o_resmv(ci) + t * C::MB + 4 * (d2 / RG)));
+            const float sxs = sz.x * kSubScale;
 #pragma unroll
             for (int e = 0; e < C::D2; e += 2) {
-              const float2 f = f2sub1(make_float2(code_f<RB>(cw, e, one), code_f<RB>(cw, e + 1, one)));
+              const float2 f = make_float2(code_sub<RB>(cw, e), code_sub<RB>(cw, e + 1));
 #pragma unroll
               for (int gi = 0; gi < G; ++gi) {
-                const float w = pw[ci][gi] * sz.x;
+                const float w = pw[ci][gi] * sxs;
                 acc_res[gi][e / 2] = __ffma2_rn(make_float2(w, w), f, acc_res[gi][e / 2]);
               }
             }
@@ -823,12 +829,12 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
       for (int e = 0; e < C::D2; ++e) {
         const float2 ar = acc_ref[gi][e >> 1];
         float vr = (e & 1) ? ar.y : ar.x;
-        if constexpr (REF == kRefInt4) vr = fmaf(vr, pow2i(23 - code_pos<4>(e)), z_ref[gi]);
+        if constexpr (REF == kRefInt4) vr = fmaf(vr, pow2i(kSubExp - code_pos<4>(e)), z_ref[gi]);
         cref[gi][e] = __fmul_rn(vr, f);
         float vs = 0.f;
         if constexpr (RB != 0) {
           const float2 as = acc_res[gi][e >> 1];
-          vs = fmaf((e & 1) ? as.y : as.x, pow2i(23 - code_pos<RB>(e)), z_res[gi]);
+          vs = fmaf((e & 1) ? as.y : as.x, pow2i(kSubExp - code_pos<RB>(e)), z_res[gi]);
         }
         cres[gi][e] = __fmul_rn(vs, f);
         if constexpr (SPW == 2) {
