@@ -277,21 +277,20 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
 #pragma unroll
     for (int g = 0; g < NGR1; ++g) zr[g] = 0.f;
 
-    for (int sp = 0; sp < seg_pages; ++sp, ++k) {
-      if ((k % NG) != grp) {  // another group's page
-        it.next(sNt, B, Hkv);
-        continue;
-      }
-      const int s = k % C::STAGES;
+    // this group's pages of the segment: every NG-th, from the first with
+    // (k + sp) % NG == grp
+    for (int sp = (grp - k % NG + NG) % NG; sp < seg_pages; sp += NG) {
+      const int kp = k + sp;  // the CTA's page index
+      const int s = kp % C::STAGES;
       const uint8_t* st = stages + s * S::STAGE_BYTES;
       if (!*sAbort) {
-        if (!mbar_wait_bounded(smem_u32(&bars[s]), (k / C::STAGES) & 1)) {
+        if (!mbar_wait_bounded(smem_u32(&bars[s]), (kp / C::STAGES) & 1)) {
           set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
           *sAbort = 1;
         }
       }
-      const int t0 = TW * gw;                            // first stage row of this warp's quarter
-      const int nv = min(TT, len_b - it.page * TT) - t0;  // its valid tokens (warp-uniform; may be <= 0)
+      const int t0 = TW * gw;                                   // first stage row of this warp's quarter
+      const int nv = min(TT, len_b - (it.page + sp) * TT) - t0;  // its valid tokens (warp-uniform; may be <= 0)
       if (nv > 0) {
         // ---------------- phase 1: scores of the quarter's 32 tokens
         float wmax = -INFINITY;
@@ -485,7 +484,10 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
           }
         };
         if (nv >= TW) {
-#pragma unroll 4
+          // fully unrolled with one link (constant offsets, no loop
+          // arithmetic); chained links keep the register budget of unroll 4
+          constexpr int UNROLL = NCH == 1 ? TW / 2 : 4;
+#pragma unroll UNROLL
           for (int i = 0; i < TW / 2; ++i) value_token(2 * i + half);
         } else {
           // a partial quarter: tokens past the context have zero weights, so
@@ -495,8 +497,11 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars[C::STAGES + s]));
-      it.next(sNt, B, Hkv);
     }
+    // past the segment: the next (b, h) (the loop ends when the CTA's pages do)
+    k += seg_pages;
+    it.page += seg_pages - 1;
+    it.next(sNt, B, Hkv);
 
     // ---- flush this (b, h) segment: every warp's state into its slot, then the
     // slots added in a fixed order into the CTA's partial record

@@ -534,21 +534,20 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
       for (int e = 0; e < C::D2 / 2; ++e) acc_ref[gi][e] = acc_res[gi][e] = make_float2(0.f, 0.f);
     }
 
-    for (int sp = 0; sp < seg_pages; ++sp, ++k) {
-      if ((k % NG) != grp) {  // another group's page
-        it.next(sNt, B, Hkv);
-        continue;
-      }
-      const int s = k % C::STAGES;
+    // this group's pages of the segment: every NG-th, from the first with
+    // (k + sp) % NG == grp
+    for (int sp = (grp - k % NG + NG) % NG; sp < seg_pages; sp += NG) {
+      const int kp = k + sp;  // the CTA's page index
+      const int s = kp % C::STAGES;
       const uint8_t* st = stages + s * C::STAGE_BYTES;
       if (!*sAbort) {
-        if (!mbar_wait_bounded(smem_u32(&bars[s]), (k / C::STAGES) & 1)) {
+        if (!mbar_wait_bounded(smem_u32(&bars[s]), (kp / C::STAGES) & 1)) {
           set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
           *sAbort = 1;
         }
       }
-      const int n_valid = min(TT, len_b - it.page * TT);
-      const int par = (k / NG) & 1;
+      const int n_valid = min(TT, len_b - (it.page + sp) * TT);
+      const int par = (kp / NG) & 1;
       float* pS = gS + par * G * TT;
       float* pWM = gWM + par * G * kGW;
 
@@ -806,8 +805,11 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars[C::STAGES + s]));
-      it.next(sNt, B, Hkv);
     }
+    // past the segment: the next (b, h) (the loop ends when the CTA's pages do)
+    k += seg_pages;
+    it.page += seg_pages - 1;
+    it.next(sNt, B, Hkv);
 
     // ---- flush this (b, h) segment: merge the two groups, write one partial
     if (gtid == 0) {
