@@ -191,9 +191,14 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
   const int gw = warp % kGW;    // quarter of the page: tokens [TW gw, TW gw + TW)
   const int j1 = lane & 3;      // phase 1: dims [32 j1, 32 j1 + 32) ...
   const int tq1 = lane >> 2;    // ... of token 8 ps + tq1 of the quarter
-  const int half = lane >> 4;   // phase 2: token parity ...
-  const int j2 = lane & 15;     // ... and dims [8 j2, 8 j2 + 8)
-  const int gwl = RB ? (8 * j2) / RG : (j2 >> 2);  // weight group of the phase-2 lane
+  // phase 2: VD value dims per lane, VL lanes per token, TPS tokens per step
+  // (16 dims per lane halves the per-token loads but measured slower: 4.81
+  // against 5.01 TB/s on the INT4-anchor INT2 loop)
+  constexpr int VD = 8;
+  constexpr int VL = kD / VD, TPS = 32 / VL;
+  const int tph = lane / VL;    // phase 2: token phase ...
+  const int j2 = lane % VL;     // ... and dims [VD j2, VD j2 + VD)
+  const int gwl = RB ? (VD * j2) / RG : (VD * j2) / 32;  // weight group of the phase-2 lane
   float* wbuf = sW + warp * TW * C::WSTRIDE;
   float* scb = sSC + warp * TW;
   constexpr int NG1 = RB ? (32 >= RG ? 32 / RG : 1) : 1;  // residual groups in a phase-1 lane's dims
@@ -268,10 +273,10 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
 
     // per-warp running state
     float m_run = -INFINITY, l_lane = 0.f;
-    float2 acc_a[4], acc_r[4];
+    float2 acc_a[VD / 2], acc_r[VD / 2];
     float za[4], zr[NGR1];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc_a[e] = acc_r[e] = make_float2(0.f, 0.f);
+    for (int e = 0; e < VD / 2; ++e) acc_a[e] = acc_r[e] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int g = 0; g < 4; ++g) za[g] = 0.f;
 #pragma unroll
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
           const float corr = fast_exp2(m_run - mp);
           const float2 c2 = make_float2(corr, corr);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
+          for (int e = 0; e < VD / 2; ++e) {
             acc_a[e] = __fmul2_rn(acc_a[e], c2);
             acc_r[e] = __fmul2_rn(acc_r[e], c2);
           }
@@ -442,7 +447,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
           for (int i = 0; i < C::WS; ++i) row[i] = 0.f;
         }
         __syncwarp();
-        // ---------------- phase 2: values, two tokens per step (token parity `half`)
+        // ---------------- phase 2: values, TPS tokens per step (token phase `tph`)
         auto value_token = [&](int tq) {
           const int t = t0 + tq;
           const float* wrow = wbuf + tq * C::WSTRIDE + gwl * C::P1P;
@@ -458,25 +463,26 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
           }
           int n = 0;
           if constexpr (ANCH) {
-            const uint32_t cw = *reinterpret_cast<const uint32_t*>(st + S::O_REFV + t * 64 + 4 * j2);
-            const uint32_t cw1[1] = {cw};
+            uint32_t cw[VD / 8];
+            load_codes<VD / 2>(st + S::O_REFV + t * 64 + (VD / 2) * j2, cw);
             const float2 ww = make_float2(w[0], w[0]);
 #pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const float2 f = make_float2(code_sub<4>(cw1, e), code_sub<4>(cw1, e + 1));
+            for (int e = 0; e < VD; e += 2) {
+              const float2 f = make_float2(code_sub<4>(cw, e), code_sub<4>(cw, e + 1));
               acc_a[e / 2] = __ffma2_rn(ww, f, acc_a[e / 2]);
             }
             ++n;
           }
           if constexpr (RB != 0) {
+            constexpr int NBV = RB * VD / 8;  // code bytes of the lane's dims
 #pragma unroll
             for (int ci = 0; ci < NCH; ++ci) {
-              uint32_t cw[1];
-              load_codes<RB>(st + S::o_resv(ci) + t * S::CB + RB * j2, cw);
+              uint32_t cw[NBV >= 4 ? NBV / 4 : 1];
+              load_codes<NBV>(st + S::o_resv(ci) + t * S::CB + NBV * j2, cw);
               const float wv = w[n + ci];
               const float2 ww = make_float2(wv, wv);
 #pragma unroll
-              for (int e = 0; e < 8; e += 2) {
+              for (int e = 0; e < VD; e += 2) {
                 const float2 f = make_float2(code_sub<RB>(cw, e), code_sub<RB>(cw, e + 1));
                 acc_r[e / 2] = __ffma2_rn(ww, f, acc_r[e / 2]);
               }
@@ -486,13 +492,13 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
         if (nv >= TW) {
           // fully unrolled with one link (constant offsets, no loop
           // arithmetic); chained links keep the register budget of unroll 4
-          constexpr int UNROLL = NCH == 1 ? TW / 2 : 4;
+          constexpr int UNROLL = NCH == 1 ? TW / TPS : 4;
 #pragma unroll UNROLL
-          for (int i = 0; i < TW / 2; ++i) value_token(2 * i + half);
+          for (int i = 0; i < TW / TPS; ++i) value_token(TPS * i + tph);
         } else {
           // a partial quarter: tokens past the context have zero weights, so
           // only the steps with a valid token are taken
-          for (int i = 0; 2 * i < nv; ++i) value_token(2 * i + half);
+          for (int i = 0; TPS * i < nv; ++i) value_token(TPS * i + tph);
         }
       }
       __syncwarp();
@@ -515,19 +521,22 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
       for (int g = 0; g < NGR1; ++g) zr[g] = bp_warp_sum(zr[g]);
       float zav = za[0], zrv = zr[0];
 #pragma unroll
-      for (int g = 1; g < 4; ++g) zav = (j2 >> 2) == g ? za[g] : zav;
+      for (int g = 1; g < 4; ++g) zav = (VD * j2) / 32 == g ? za[g] : zav;  // the lane's anchor group
 #pragma unroll
       for (int g = 1; g < NGR1; ++g) zrv = gwl == g ? zr[g] : zrv;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < VD; ++e) {
         const float2 aa = acc_a[e >> 1], ar = acc_r[e >> 1];
         float va = (e & 1) ? aa.y : aa.x;
         float vr = (e & 1) ? ar.y : ar.x;
-        va = __fadd_rn(va, __shfl_xor_sync(kFull, va, 16));  // the two token parities
-        vr = __fadd_rn(vr, __shfl_xor_sync(kFull, vr, 16));
-        if (lane < 16) {
-          slot[4 + 8 * j2 + e] = ANCH ? fmaf(va, pow2i(kSubExp - code_pos<4>(e)), zav) : 0.f;
-          slot[4 + kD + 8 * j2 + e] = RB ? fmaf(vr, pow2i(kSubExp - code_pos<RB ? RB : 2>(e)), zrv) : 0.f;
+#pragma unroll
+        for (int o = VL; o < 32; o <<= 1) {  // the token phases, in a fixed order
+          va = __fadd_rn(va, __shfl_xor_sync(kFull, va, o));
+          vr = __fadd_rn(vr, __shfl_xor_sync(kFull, vr, o));
+        }
+        if (lane < VL) {
+          slot[4 + VD * j2 + e] = ANCH ? fmaf(va, pow2i(kSubExp - code_pos<4>(e)), zav) : 0.f;
+          slot[4 + kD + VD * j2 + e] = RB ? fmaf(vr, pow2i(kSubExp - code_pos<RB ? RB : 2>(e)), zrv) : 0.f;
         }
       }
       if (lane == 0) {
