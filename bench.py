@@ -57,6 +57,7 @@ def parse_args():
     ap.add_argument("--decode-kernel", choices=["auto", "simt", "tensor"], default="auto",
                     help="decode kernel of the RQ cache (the automatic choice by default)")
     ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--q-heads", type=int, default=None, help="query heads of the workload (a multiple of its kv-heads)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
@@ -68,6 +69,13 @@ def parse_args():
 
 
 def make_workload(args) -> synth.Workload:
+    wl = _base_workload(args)
+    if args.q_heads:
+        wl = wl.with_(name=f"{wl.name}_Hq{args.q_heads}", q_heads=args.q_heads)
+    return wl
+
+
+def _base_workload(args) -> synth.Workload:
     if args.workload == "ouro8k":
         return synth.ouro_8k(batch=args.batch or 16)
     if args.workload == "mixed":
