@@ -870,7 +870,7 @@ def run_rq(args, world, rank):
         del cache, inp, outs
         torch.cuda.empty_cache()
     if not args.no_extra and args.workload == "ouro8k":
-        extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 30, 3, world, rank),
+        extra = [measure_workload(synth.mixed_int4_anchor(batch=32), 30, 3, world, rank, per_loop=True),
                  measure_workload(synth.gqa_long(batch=8), 30, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8, q_heads=64), 30, 3, world, rank),
                  measure_workload(synth.gqa_long(batch=8, int4_anchor=True), 30, 3, world, rank),

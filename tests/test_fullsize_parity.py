@@ -16,9 +16,12 @@ pytestmark = pytest.mark.gpu
 CASES = [
     (synth.ouro_8k(), [(0, 0), (7, 9), (15, 15)]),
     (synth.mixed_int4_anchor(batch=8), [(0, 3), (7, 15)]),
+    (synth.mixed_int4_anchor(batch=32), [(31, 15)]),
     (synth.gqa_long(batch=8), [(0, 0), (5, 7)]),
     (synth.gqa_long(batch=8, q_heads=64), [(3, 4)]),
+    (synth.gqa_long(batch=8, int4_anchor=True), [(0, 0), (6, 3)]),
     (synth.ouro_8k_next_loop(), [(0, 0), (15, 15)]),
+    (synth.ouro_8k_next_loop_int4(), [(0, 0), (9, 12)]),
 ]
 
 
@@ -110,5 +113,39 @@ def test_full_size_multi_query(librq):
             q = qm[l][b:b + 1, :, h:h + 1].float().cpu().numpy()
             want = O.decode_attention_multi_f64(enc, l, q, np.array([n]), kt[l], vt[l])
             got = outs[i][b:b + 1, :, h:h + 1].cpu().numpy()
+            err = rel_err_rows(got, want).max()
+            assert err <= ATTN_TOL, (b, h, l, float(err))
+
+
+def test_full_size_sixteen_rows_one_pass(librq):
+    """Four draft tokens on the full 32k GQA cache (4 query heads per kv-head):
+    16 rows per kv-head in one pass over the cache on the tensor cores, as the
+    bench's verify line times them."""
+    rq = librq
+    n_q = 4
+    wl = synth.gqa_long(batch=8).with_(n_tail=n_q)
+    dev = torch.device("cuda")
+    inp = synth.make_inputs(wl, dev)
+    qm = synth.draft_queries(wl, n_q, dev)
+    cfgd = synth.cache_config_dict(wl)
+    cache = rq.Cache(rq.config_from_dict(cfgd), device=dev)
+    cache.encode(inp["k"], inp["v"])
+    ctx = inp["ctx_len"]
+    G = wl.gqa
+    for l in (0, 3):
+        assert cache.decode_plan(l, n_q) == (rq.DECODE_KERNEL_TENSOR, n_q * G)
+    outs = [cache.decode_attention_multi(l, qm[l], ctx, inp["k_tail"][l], inp["v_tail"][l]) for l in (0, 3)]
+    torch.cuda.synchronize()
+    assert cache.get_error() == 0
+    ocfg = O.CacheConfig.from_dict(cfgd)
+    for b, h in [(1, 2), (7, 7)]:
+        n = int(ctx[b])
+        sl = lambda t: t[:, b:b + 1, h:h + 1].float().cpu().numpy()  # noqa: E731
+        enc = O.encode_fp32emu(sl(inp["k"])[:, :, :, :n], sl(inp["v"])[:, :, :, :n], ocfg)
+        kt, vt = sl(inp["k_tail"]), sl(inp["v_tail"])
+        for i, l in enumerate((0, 3)):
+            q = qm[l][b:b + 1, :, h * G:(h + 1) * G].float().cpu().numpy()
+            want = O.decode_attention_multi_f64(enc, l, q, np.array([n]), kt[l], vt[l])
+            got = outs[i][b:b + 1, :, h * G:(h + 1) * G].cpu().numpy()
             err = rel_err_rows(got, want).max()
             assert err <= ATTN_TOL, (b, h, l, float(err))
