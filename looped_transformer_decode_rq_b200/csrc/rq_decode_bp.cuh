@@ -42,10 +42,10 @@ __device__ __forceinline__ float bp_warp_sum(float v) {
   return v;
 }
 
-template <int REF, int RB, int RG, int NCH>
-struct BpCfg {
+template <int REF, int RB, int RG, int NCH, int NG_>
+struct BpCfgN {
   static constexpr int TT = 2 * kPage;  // tokens per page (stage)
-  static constexpr int NG = 3;          // consumer groups of kGW warps
+  static constexpr int NG = NG_;        // consumer groups of kGW warps
   using S = Cfg<REF, RB, RG, 1, TT, NCH, NG>;  // stage layout, record sizes, copy bytes
   static constexpr int NCW = S::NCW, NCT = S::NCT, NT = S::NT;
   static constexpr int TW = TT / kGW;   // tokens of a warp's quarter of a page
@@ -77,6 +77,16 @@ struct BpCfg {
   static constexpr int SMEM_BYTES = 1024 + STAGES * S::STAGE_BYTES + MISC_BYTES;
   static_assert((W_QS % 4) == 0 && (W_QT % 4) == 0 && (WSTRIDE % P1P) == 0, "alignment");
 };
+
+// Three consumer groups where two stages per group fit (six stages), else two
+// groups where two stages each fit (a group with a single stage cannot have
+// its next page in flight while it works on one), else three groups of one.
+template <int REF, int RB, int RG, int NCH>
+constexpr int bp_groups() {
+  return BpCfgN<REF, RB, RG, NCH, 3>::STAGES_MAX >= 6 ? 3 : (BpCfgN<REF, RB, RG, NCH, 2>::STAGES_MAX >= 4 ? 2 : 3);
+}
+template <int REF, int RB, int RG, int NCH>
+using BpCfg = BpCfgN<REF, RB, RG, NCH, bp_groups<REF, RB, RG, NCH>()>;
 
 template <int REF, int RB, int RG, int NCH>
 __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
