@@ -69,10 +69,16 @@ struct BpCfgN {
   static constexpr int W_NT = W_PRE + RQ_MAX_BATCH + 1;         // [RQ_MAX_BATCH]
   static constexpr int W_MISC = W_NT + RQ_MAX_BATCH;            // abort flag
   static constexpr int W_BAR = (W_MISC + 2 + 1) & ~1;           // 8-byte aligned mbarriers
-  static constexpr int MISC_BYTES = 4 * W_BAR + 16 * 8;
+  static constexpr int NBARS = 20;                              // full[9], empty[9], -, never
+  static constexpr int BAR_NEVER = NBARS - 1;
+  static constexpr int MISC_BYTES = 4 * W_BAR + NBARS * 8;
   static constexpr int STAGES_MAX = (S::kSmemLimit - 1024 - MISC_BYTES) / S::STAGE_BYTES;
-  // a multiple of NG stages: each stage always serves the same group
-  static constexpr int STAGES = STAGES_MAX >= 2 * NG ? 2 * NG : NG;
+  // a multiple of NG stages, so that each stage always serves the same group:
+  // up to three per group, as many as fit (small records keep more pages in
+  // flight per SM)
+  static constexpr int PER_GROUP = STAGES_MAX / NG >= 3 ? 3 : (STAGES_MAX / NG >= 2 ? 2 : 1);
+  static constexpr int STAGES = NG * PER_GROUP;
+  static_assert(2 * 9 < BAR_NEVER + 1, "barrier slots");
   static constexpr bool FITS = STAGES_MAX >= NG;
   static constexpr int SMEM_BYTES = 1024 + STAGES * S::STAGE_BYTES + MISC_BYTES;
   static_assert((W_QS % 4) == 0 && (W_QT % 4) == 0 && (WSTRIDE % P1P) == 0, "alignment");
@@ -153,7 +159,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
       mbar_init(smem_u32(&bars[s]), 1);                // full: the producer's expect_tx
       mbar_init(smem_u32(&bars[C::STAGES + s]), kGW);  // empty: the page's four warps
     }
-    mbar_init(smem_u32(&bars[15]), 1);  // never arrived at: the wait of the stall test hook
+    mbar_init(smem_u32(&bars[C::BAR_NEVER]), 1);  // never arrived at: the wait of the stall test hook
     fence_barrier_init();
   }
   __syncthreads();
@@ -179,7 +185,8 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
           *sAbort = 1;
           break;
         }
-        if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[15]), 0)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+        if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[C::BAR_NEVER]), 0))
+          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
         if (*sAbort) break;
         issue_page<REF, RB, RG, 1, TT, NCH, NG>(P, &tmK, &tmV, stages + s * S::STAGE_BYTES, smem_u32(&bars[s]), it,
                                                 Hkv);
