@@ -886,12 +886,14 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
 // Pages of 64 tokens for a bf16 anchor (one tensor-copy tile); 128 for the
 // byte-plane formats, whose 64-token pages are too small to amortise the
 // per-page synchronisation, when four stages still fit.
-// Three consumer groups (12 warps) for the byte-plane formats at G <= 2, which
+// Three consumer groups (12 warps) for the byte-plane formats at G = 1, which
 // are bound by instruction latency with two; two elsewhere (the bf16-anchor
-// formats are bound by HBM, and larger G or chains need the registers).
+// formats are bound by HBM, and larger G or chains need the registers: at
+// G = 2 two groups run as fast as three, 2.70 against 2.71 TB/s on the
+// INT4-anchor [2,2,4,4] loop, without the spills of the 128-register limit).
 template <int REF, int RB, int RG, int G, int NCH>
 constexpr int groups_of() {
-  return (REF != kRefBf16 && (G == 1 || (G == 2 && NCH == 1))) ? 3 : 2;
+  return (REF != kRefBf16 && G == 1) ? 3 : 2;
 }
 
 template <int REF, int RB, int RG, int G, int NCH>
