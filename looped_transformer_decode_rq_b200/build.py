@@ -25,11 +25,11 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
               "--expt-relaxed-constexpr", "-I", INCLUDE]
 
-CU_SOURCES = ["rq_encode.cu", "rq_decode.cu", "rq_decode_chain.cu", "rq_decode_tc.cu", "rq_decode_pp.cu",
-              "rq_static_scratch.cu"]
+CU_SOURCES = ["rq_encode.cu", "rq_decode.cu", "rq_decode_chain.cu", "rq_decode_tc.cu", "rq_decode_tc_chain.cu",
+              "rq_decode_pp.cu", "rq_static_scratch.cu"]
 CPP_SOURCES = ["rq_api.cpp"]
 HEADERS = ["rq_common.cuh", "rq_internal.h", "rq_tcgen05.cuh", "rq_encode_dev.cuh", "rq_decode_split.cuh",
-           "rq_decode_bp.cuh", "rq_tc_ops.cuh"]
+           "rq_decode_bp.cuh", "rq_tc_ops.cuh", "rq_decode_tc.cuh"]
 
 
 def _sources():

@@ -13,7 +13,7 @@
 // combine kernel.  No bf16 copy of loop l is ever formed.
 //
 // This file holds the combine kernel and the dispatch; the CUDA-core split
-// kernel is in rq_decode_split.cuh, the tensor-core one in rq_decode_tc.cu.
+// kernel is in rq_decode_split.cuh, the tensor-core one in rq_decode_tc.cuh.
 // Combine kernel: one warp per (b, query row) merges the CTA partials with the
 // max-rescale rule, adds the bf16 tail tokens (a draft token of a multi-query
 // call sees the tail up to itself), applies the inverse rotation and
@@ -198,7 +198,7 @@ bool pp_case(int ref_kind, int res_bits, int res_group, int G, int n_chain) {
 // [2,2,4,4] residual loop).
 int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int kernel, int n_chain) {
   if (kernel == kKernelAuto)
-    return (G >= 4 && n_chain <= 1 && tc_variant_supported(ref_kind, res_bits, res_group, G)) ? kKernelTensor
+    return (G >= 4 && tc_variant_supported(ref_kind, res_bits, res_group, G, n_chain)) ? kKernelTensor
                                                                                               : kKernelSimt;
   return kernel;
 }
@@ -207,8 +207,8 @@ bool decode_variant_supported(int ref_kind, int res_bits, int res_group, int G, 
   if (res_bits != 0 && res_group != 16 && res_group != 32) return false;
   kernel = decode_kernel_choice(ref_kind, res_bits, res_group, G, kernel, n_chain);
   if (kernel == kKernelTensor)
-    return n_chain <= 1 && (pp_case(ref_kind, res_bits, res_group, G, n_chain) ||
-                            tc_variant_supported(ref_kind, res_bits, res_group, G));
+    return pp_case(ref_kind, res_bits, res_group, G, n_chain) ||
+           tc_variant_supported(ref_kind, res_bits, res_group, G, n_chain);
   if (kernel == kKernelSimt) return pick(ref_kind, res_bits, res_group, G, n_chain) != nullptr;
   return false;
 }
@@ -231,12 +231,11 @@ cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_gr
   kernel = decode_kernel_choice(ref_kind, res_bits, res_group, p.G, kernel, n_chain);
   cudaError_t e;
   if (kernel == kKernelTensor) {
-    if (n_chain > 1) return cudaErrorInvalidValue;
     p.page_tokens = kTcPage;
     if (pp_case(ref_kind, res_bits, res_group, p.G, n_chain))
       e = launch_split_pp(p, ref_kind, res_bits, res_group, s);
     else
-      e = launch_split_tc(p, ref_kind, res_bits, res_group, tmap_k, tmap_v, s);
+      e = launch_split_tc(p, ref_kind, res_bits, res_group, n_chain, tmap_k, tmap_v, s);
   } else {
     SplitFn fn = pick(ref_kind, res_bits, res_group, p.G, n_chain);
     if (fn == nullptr) return cudaErrorInvalidValue;

@@ -26,7 +26,7 @@
 //   * at the end of a (b, kv-head) segment the two warpgroups' states are
 //     added in a fixed order into the CTA's partial record.
 //
-// Numerics are those of the tensor-core kernel in rq_decode_tc.cu: queries and
+// Numerics are those of the tensor-core kernel in rq_decode_tc.cuh: queries and
 // weights as 24-bit integers in byte planes, exact int32 sums.
 #include "rq_common.cuh"
 #include "rq_internal.h"

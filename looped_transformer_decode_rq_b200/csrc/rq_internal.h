@@ -104,8 +104,9 @@ int decode_grid_ctas(int device);  // persistent grid size for this device
 
 cudaError_t launch_encode(const EncodeParams& p, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconstructParams& p, cudaStream_t s);
-// Decode kernels: the CUDA-core split kernel (64-token pages, any G) and the
-// tensor-core split kernel (128-token pages, G in {2, 4, 8}).
+// Decode kernels: the CUDA-core split kernels (64- or 128-token pages, G in
+// {1, 2, 4}) and the tensor-core split kernels (128-token pages, G in {1, 2, 4,
+// 8, 16}; chained INT4-anchor loops at G in {2, 4, 8}).
 enum DecodeKernel : int { kKernelAuto = RQ_DECODE_KERNEL_AUTO, kKernelSimt = RQ_DECODE_KERNEL_SIMT,
                           kKernelTensor = RQ_DECODE_KERNEL_TENSOR };
 
@@ -125,10 +126,14 @@ int decode_kernel_choice(int ref_kind, int res_bits, int res_group, int G, int k
 using SplitLaunchFn = cudaError_t (*)(DecodeParams&, const CUtensorMap*, const CUtensorMap*, cudaStream_t);
 SplitLaunchFn pick_chain(int ref_kind, int res_bits, int res_group, int G, int n_chain);
 
-// tensor-core split kernel (rq_decode_tc.cu)
-bool tc_variant_supported(int ref_kind, int res_bits, int res_group, int G);
-cudaError_t launch_split_tc(const DecodeParams& p, int ref_kind, int res_bits, int res_group,
+// tensor-core split kernel (rq_decode_tc.cuh; dispatch in rq_decode_tc.cu)
+bool tc_variant_supported(int ref_kind, int res_bits, int res_group, int G, int n_chain = 1);
+cudaError_t launch_split_tc(const DecodeParams& p, int ref_kind, int res_bits, int res_group, int n_chain,
                             const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
+// chained loops (2 or 3 residual links, INT4 anchor) on the tensor cores
+bool tc_chain_variant_supported(int ref_kind, int res_bits, int res_group, int G, int n_chain);
+cudaError_t launch_split_tc_chain(const DecodeParams& p, int ref_kind, int res_bits, int res_group, int n_chain,
+                                  const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s);
 constexpr int kTcPage = 128;
 // tensor-core split kernel for the byte-plane formats at one query row per
 // kv-head, two warpgroups on alternate pages (rq_decode_pp.cu)

@@ -1,5 +1,5 @@
 // rq_tc_ops.cuh -- per-thread operations shared by the tensor-core decode
-// kernels (rq_decode_tc.cu, rq_decode_pp.cu): warp reductions, the expansion of
+// kernels (rq_decode_tc.cuh, rq_decode_pp.cu): warp reductions, the expansion of
 // packed 2/4-bit codes into int8 rows in the byte order the MMAs' other
 // operands use, and the 24-bit byte-plane operands that carry queries and
 // softmax weights to the int8 tensor cores.

@@ -162,10 +162,38 @@ def test_chained_policies(librq, policy, bits, group, G):
     run_case(librq, wl, lengths=[300, 129, 1])
 
 
+@pytest.mark.parametrize("policy,bits,group,G,loops", [
+    (4, (2, 2, 2, 4), (32,) * 4, 4, [0, 1, 2, 3]),    # Next-loop [2,2,2,4]: 3, 2 and 1 links, and the anchor
+    (4, (2, 2, 2, 4), (32,) * 4, 8, [1, 2, 3]),       # 8 rows: two links (value sums over the scores)
+    (3, (4, 2, 2, 2), (32, 16, 16, 16), 4, [1, 2]),   # Previous-loop, INT2 g=16 links: 1 and 2 links
+    (4, (4, 4, 4, 4), (32,) * 4, 4, [1, 2]),          # INT4 links: 2 and 1 links
+])
+def test_chained_loops_on_the_tensor_cores(librq, policy, bits, group, G, loops):
+    """Chained (Previous-/Next-loop) INT4-anchor loops on the tensor-core
+    kernel: every link's keys are scored against the one rotated query and
+    combined by Horner's rule from the anchor outward, every link's values go
+    into the one rotated accumulator with signed weights.  Forced onto the
+    tensor cores against the float64 oracle; the automatic choice takes them
+    from 4 rows (three links at 8 rows as two 4-row passes)."""
+    rq = librq
+    anchor = 0 if policy == 3 else 3
+    rot = tuple(0 if l == anchor else 1 for l in range(4))
+    wl = synth.Workload(name=f"chain_tc_{policy}_{G}", batch=3, kv_heads=2, q_heads=2 * G, context=300, bits=bits,
+                        group=group, rotate=rot, sigma=(0.3, 0.2, 0.1), outlier_p=0.01, anchor_policy=policy,
+                        seed=90 + policy + G)
+    run_case(rq, wl, lengths=[300, 129, 1], loops=loops, kernel=rq.DECODE_KERNEL_TENSOR)
+    cache = rq.Cache(rq.config_from_dict(synth.cache_config_dict(wl)), device="cuda")
+    for l in loops:
+        kernel, rows = cache.decode_plan(l, 1)
+        assert kernel == rq.DECODE_KERNEL_TENSOR and rows == G, (l, kernel, rows)
+    if G == 8 and anchor == 3:
+        assert cache.decode_plan(0, 1) == (rq.DECODE_KERNEL_TENSOR, 4)  # three links: two 4-row passes
+
+
 def test_chained_loops_run_on_the_cuda_core_kernel(librq):
-    """The tensor-core kernel decodes the anchor and the loop next to it (one
-    link) but reports a longer chain as unsupported; the default then picks the
-    CUDA-core kernel."""
+    """With a bf16 anchor the tensor-core kernel decodes the anchor and the
+    loop next to it (one link) but reports a longer chain as unsupported; the
+    default then picks the CUDA-core kernel."""
     rq = librq
     wl = synth.Workload(name="chain_tc", batch=2, kv_heads=2, q_heads=8, context=260, sigma=(0.3, 0.2, 0.1),
                         anchor_policy=4, seed=66)
