@@ -296,18 +296,25 @@ def test_tensor_kernel_rejects_unimplemented(librq):
     assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
 
 
-@pytest.mark.parametrize("kernel", ["simt", "tensor", "simt_int4_anchor_g1", "tensor_int4_anchor_g1"])
+@pytest.mark.parametrize("kernel", ["simt", "tensor", "simt_int4_anchor_g1", "tensor_int4_anchor_g1",
+                                    "tensor_int4_anchor_g4", "tensor_chain_g4"])
 def test_wait_limit_sets_flag_and_context_recovers(librq, kernel):
     """Failure path without a fault: the producers wait on a barrier nothing
     arrives at (test hook); every wait gives up after its limit, the call sets
     FLAG_PIPE_TIMEOUT and returns, and the next call on the same context is
-    correct.  The last two cases are the byte-plane kernels (INT4 anchor, one
-    query row per kv-head) on the CUDA cores and on the tensor cores."""
+    correct.  The int4_anchor_g1 cases are the byte-plane kernels (INT4 anchor,
+    one query row per kv-head) on the CUDA cores and on the tensor cores; the
+    last two the tensor-core kernel with its register split (INT4 anchor, 4 rows)
+    and with a three-link chain."""
     import time
     rq = librq
     wl = synth.Workload(name="stall", batch=2, kv_heads=2, q_heads=8, context=300, seed=90)
     if kernel.endswith("int4_anchor_g1"):
         wl = wl.with_(q_heads=2, bits=(2, 2, 4, 4))
+    elif kernel.endswith("int4_anchor_g4"):
+        wl = wl.with_(bits=(2, 2, 4, 4))
+    elif kernel.endswith("chain_g4"):
+        wl = wl.with_(bits=(2, 2, 2, 4), anchor_policy=4)  # loop 0 is three links from the anchor
     inp = synth.make_inputs(wl, "cpu")
     cfgd = synth.cache_config_dict(wl)
     cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
