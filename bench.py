@@ -876,6 +876,10 @@ def run_rq(args, world, rank):
                  measure_workload(synth.gqa_long(batch=8, int4_anchor=True), 30, 3, world, rank),
                  measure_workload(synth.ouro_8k_next_loop(), 30, 3, world, rank, per_loop=True),
                  measure_workload(synth.ouro_8k_next_loop_int4(), 30, 3, world, rank, per_loop=True),
+                 # the same chain with 4 query heads per kv-head (chained loops on the tensor cores)
+                 measure_workload(synth.ouro_8k_next_loop_int4(batch=8).with_(
+                     name="ouro_L4_Hq64_H16_B8_T8192_2224_int4ref_next_loop", q_heads=64), 20, 3, world, rank,
+                     per_loop=True),
                  measure_multi_query(synth.ouro_8k(), 4, 30, 3, world, rank),
                  measure_multi_query(synth.gqa_long(batch=8), 4, 20, 3, world, rank)]
     sweeps = None
