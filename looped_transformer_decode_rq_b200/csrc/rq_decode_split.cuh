@@ -17,7 +17,7 @@
 //     tensor copies with the 128-byte swizzle for bf16 anchor tiles, bulk
 //     copies for code, metadata and alpha records -- completing on mbarriers;
 //   * the consumer warps form NG groups of four (2, or 3 for the byte-plane
-//     formats at G <= 2) that take pages in turn, each with its own online
+//     formats at G = 1) that take pages in turn, each with its own online
 //     softmax and group-local barriers, so that one group's barrier and
 //     reduction latency overlaps the others' math.  Within a group a page is
 //     processed in two phases: scores (4G lanes per token, dp4a on the packed
