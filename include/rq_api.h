@@ -226,8 +226,9 @@ RQ_API rq_status rq_encode(rq_cache* cache, const void* k, const void* v, const 
  *                           query heads of a kv-head at once and for the
  *                           probability-weighted value sums; G in {1, 2, 4, 8,
  *                           16} (16 rows for some formats: see
- *                           rq_decode_attention_multi), not for the residual
- *                           loops of chained policies.
+ *                           rq_decode_attention_multi); the residual loops of
+ *                           chained policies at G in {4, 8} with an INT4
+ *                           anchor only.
  *  RQ_DECODE_KERNEL_AUTO    the tensor-core kernel for G >= 4 where it has a
  *                           variant, else the CUDA-core kernel (the default). */
 typedef enum {

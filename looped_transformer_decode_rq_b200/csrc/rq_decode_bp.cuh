@@ -47,7 +47,16 @@ struct BpCfgN {
   static constexpr int TT = 2 * kPage;  // tokens per page (stage)
   static constexpr int NG = NG_;        // consumer groups of kGW warps
   using S = Cfg<REF, RB, RG, 1, TT, NCH, NG>;  // stage layout, record sizes, copy bytes
-  static constexpr int NCW = S::NCW, NCT = S::NCT, NT = S::NT;
+  static constexpr int NCW = S::NCW, NCT = S::NCT;
+  // Three links in three groups hold more than the 128 registers a thread of
+  // 416 gets (warps take registers in fours): launched as four warpgroups of
+  // 128 registers a thread, the producer's (the producer warp and three idle
+  // warps) keeps kSplitRegsAux and the three consumer warpgroups take the rest.
+  static constexpr bool REGSPLIT = NCH == 3 && NG == 3;
+  static constexpr int REGS_CONSUMER = (512 * 128 - 128 * kSplitRegsAux) / NCT;
+  static_assert(!REGSPLIT || (REGS_CONSUMER % 8 == 0 && 128 * kSplitRegsAux + NCT * REGS_CONSUMER == 512 * 128),
+                "register split");
+  static constexpr int NT = REGSPLIT ? NCT + 128 : S::NT;
   static constexpr int TW = TT / kGW;   // tokens of a warp's quarter of a page
   static_assert(TW == 32, "phase 1.5 takes one token per lane");
   static constexpr bool ANCH = REF == kRefInt4;
@@ -173,8 +182,9 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
   const int n_pages = static_cast<int>(x1 - x0);
 
   // ========================= producer warp =========================
-  if (warp == NCW) {
-    if (lane == 0) {
+  if (warp >= NCW) {
+    if constexpr (C::REGSPLIT) tc::setmaxnreg_dec<kSplitRegsAux>();
+    if (warp == NCW && lane == 0) {
       PageIter it;
       it.seek(x0, sPre, sNt, B, Hkv);
       int k = 0;
@@ -202,6 +212,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
     }
     return;
   }
+  if constexpr (C::REGSPLIT) tc::setmaxnreg_inc<C::REGS_CONSUMER>();
 
   // ========================= consumer warps =========================
   const int grp = warp / kGW;   // pages k with k % NG == grp

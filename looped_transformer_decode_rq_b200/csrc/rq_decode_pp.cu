@@ -788,7 +788,9 @@ PpFn pp_pick(int ref_kind, int res_bits, int res_group) {
   const bool g16 = res_group == 16;
   if (ref_kind == kRefInt4) {
     if (res_bits == 0) return pp_if_fits<kRefInt4, 0, 32>();
-    if (res_bits == 2) return g16 ? pp_if_fits<kRefInt4, 2, 16>() : pp_if_fits<kRefInt4, 2, 32>();
+    // INT2 with 16-dim groups needs more registers than the kernel's 168 a
+    // thread: that format's one-row tensor-core decode is decode_tc_kernel's
+    if (res_bits == 2) return g16 ? nullptr : pp_if_fits<kRefInt4, 2, 32>();
     if (res_bits == 4) return g16 ? pp_if_fits<kRefInt4, 4, 16>() : pp_if_fits<kRefInt4, 4, 32>();
   } else if (ref_kind == kRefNone) {
     if (res_bits == 2) return g16 ? pp_if_fits<kRefNone, 2, 16>() : pp_if_fits<kRefNone, 2, 32>();

@@ -32,6 +32,7 @@
 
 #include "rq_common.cuh"
 #include "rq_internal.h"
+#include "rq_tcgen05.cuh"
 
 // Internal linkage: each including translation unit has its own copy.
 namespace rq {
@@ -44,6 +45,14 @@ constexpr int kGT = kGW * 32;  // threads per consumer group
 constexpr int kConsumerBar = 1;  // all consumers
 constexpr int kGroupBar0 = 2;    // group g uses kGroupBar0 + g (128 threads)
 constexpr unsigned kFull = 0xffffffffu;
+// Register split of the variants that need more than the 168 registers a
+// thread of a 288-thread CTA gets (warps take registers in fours): the producer
+// warp comes with three idle warps, a warpgroup that keeps kSplitRegsAux of the
+// 168 registers a thread and gives the rest to the two consumer warpgroups:
+//   384 x 168 = 128 x kSplitRegsAux + 256 x kSplitRegsConsumer.
+constexpr int kSplitRegsAux = 56;
+constexpr int kSplitRegsConsumer = 224;
+static_assert(384 * 168 == 128 * kSplitRegsAux + 256 * kSplitRegsConsumer, "register split");
 
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
@@ -73,7 +82,10 @@ struct Cfg {
   static_assert(NG == 2 || NG == 3, "consumer groups");
   static constexpr int NCW = kGW * NG;   // consumer warps
   static constexpr int NCT = NCW * 32;   // consumer threads
-  static constexpr int NT = NCT + 32;    // + producer warp
+  // four query rows with residual links hold more than 168 registers a
+  // consumer thread: those variants take the register split
+  static constexpr bool REGSPLIT = NG == 2 && G >= 4 && RB != 0 && REF != kRefNone;
+  static constexpr int NT = NCT + (REGSPLIT ? 128 : 32);  // + producer warp (+ three idle warps)
   static_assert(G <= NCW, "one warp per query head in the segment set-up");
   static constexpr int PAGE = TT;  // tokens per page / stage
   // phase 1 (scores): 4G lanes per token, D1 = 32/G dims per lane
@@ -395,8 +407,9 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
   const int n_pages = static_cast<int>(x1 - x0);
 
   // ========================= producer warp =========================
-  if (warp == kNCW) {
-    if (lane == 0) {
+  if (warp >= kNCW) {
+    if constexpr (C::REGSPLIT) tc::setmaxnreg_dec<kSplitRegsAux>();
+    if (warp == kNCW && lane == 0) {
       if constexpr (REF == kRefBf16) {
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
@@ -426,6 +439,7 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
     }
     return;
   }
+  if constexpr (C::REGSPLIT) tc::setmaxnreg_inc<kSplitRegsConsumer>();
 
   // ========================= consumer groups =========================
   const int grp = warp / kGW;        // pages k with k % NG == grp

@@ -1,6 +1,8 @@
 // rq_decode_tc_chain.cu -- the tensor-core split kernel's instantiations for
 // loops of a chained (Previous-/Next-loop) policy with an INT4 anchor: 2 or 3
-// residual links, G in {2, 4, 8} where they fit (the kernel: rq_decode_tc.cuh).
+// residual links, G in {4, 8} where they fit (the kernel: rq_decode_tc.cuh).
+// Two rows stay on the CUDA cores: there some of these variants would need more
+// than the 224 registers a consumer thread has.
 #include "rq_decode_tc.cuh"
 
 namespace rq {
@@ -9,7 +11,6 @@ namespace {
 template <int RB, int RG, int NCH>
 TcFn tc_chain_pick_g(int G) {
   switch (G) {
-    case 2: return tc_if_fits<kRefInt4, RB, RG, 2, NCH>();
     case 4: return tc_if_fits<kRefInt4, RB, RG, 4, NCH>();
     case 8: return tc_if_fits<kRefInt4, RB, RG, 8, NCH>();
     default: return nullptr;

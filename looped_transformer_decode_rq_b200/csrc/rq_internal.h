@@ -106,14 +106,15 @@ cudaError_t launch_encode(const EncodeParams& p, cudaStream_t s);
 cudaError_t launch_reconstruct(const ReconstructParams& p, cudaStream_t s);
 // Decode kernels: the CUDA-core split kernels (64- or 128-token pages, G in
 // {1, 2, 4}) and the tensor-core split kernels (128-token pages, G in {1, 2, 4,
-// 8, 16}; chained INT4-anchor loops at G in {2, 4, 8}).
+// 8, 16}; chained INT4-anchor loops at G in {4, 8}).
 enum DecodeKernel : int { kKernelAuto = RQ_DECODE_KERNEL_AUTO, kKernelSimt = RQ_DECODE_KERNEL_SIMT,
                           kKernelTensor = RQ_DECODE_KERNEL_TENSOR };
 
 // ref_kind: RefKind; res_bits: 0 | 2 | 4; res_group: 16 | 32
 // `append` (or null): tokens to encode into the cache in the same launch as
 // the combine kernel (positions past every context of this decode).
-// p.n_chain > 1 (a chained loop) is CUDA-core only.
+// p.n_chain > 1 (a chained loop): the tensor cores for an INT4 anchor at G in
+// {4, 8}, else the CUDA cores.
 cudaError_t launch_decode(DecodeParams p, int ref_kind, int res_bits, int res_group, int kernel,
                           const CUtensorMap* tmap_k, const CUtensorMap* tmap_v, cudaStream_t s,
                           const EncodeParams* append = nullptr);

@@ -296,16 +296,19 @@ def test_tensor_kernel_rejects_unimplemented(librq):
     assert rel_err_rows(out.cpu().numpy(), want).max() <= ATTN_TOL
 
 
-@pytest.mark.parametrize("kernel", ["simt", "tensor", "simt_int4_anchor_g1", "tensor_int4_anchor_g1",
-                                    "tensor_int4_anchor_g4", "tensor_chain_g4"])
+@pytest.mark.parametrize("kernel", ["simt", "tensor", "tensor_g8", "simt_int4_anchor_g1", "tensor_int4_anchor_g1",
+                                    "tensor_int4_anchor_g4", "tensor_chain_g4", "simt_chain_g1"])
 def test_wait_limit_sets_flag_and_context_recovers(librq, kernel):
     """Failure path without a fault: the producers wait on a barrier nothing
     arrives at (test hook); every wait gives up after its limit, the call sets
     FLAG_PIPE_TIMEOUT and returns, and the next call on the same context is
     correct.  The int4_anchor_g1 cases are the byte-plane kernels (INT4 anchor,
     one query row per kv-head) on the CUDA cores and on the tensor cores; the
-    last two the tensor-core kernel with its register split (INT4 anchor, 4 rows)
-    and with a three-link chain."""
+    two after them the tensor-core kernel with its register split (INT4 anchor,
+    4 rows) and with a three-link chain; tensor_g8 the tensor-core kernel whose
+    stages refill their key and value halves separately (bf16 anchor, 8 rows);
+    simt_chain_g1 the byte-plane CUDA-core kernel with its register split (one
+    row, three links)."""
     import time
     rq = librq
     wl = synth.Workload(name="stall", batch=2, kv_heads=2, q_heads=8, context=300, seed=90)
@@ -315,6 +318,10 @@ def test_wait_limit_sets_flag_and_context_recovers(librq, kernel):
         wl = wl.with_(bits=(2, 2, 4, 4))
     elif kernel.endswith("chain_g4"):
         wl = wl.with_(bits=(2, 2, 2, 4), anchor_policy=4)  # loop 0 is three links from the anchor
+    elif kernel.endswith("chain_g1"):
+        wl = wl.with_(q_heads=2, bits=(2, 2, 2, 4), anchor_policy=4)
+    elif kernel.endswith("_g8"):
+        wl = wl.with_(q_heads=16)
     inp = synth.make_inputs(wl, "cpu")
     cfgd = synth.cache_config_dict(wl)
     cache = rq.Cache(rq.config_from_dict(cfgd), device="cuda")
