@@ -426,7 +426,6 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
           if constexpr (ANCH) {
             const uint4 mv = *reinterpret_cast<const uint4*>(st + S::O_REFMV + t * 16);
             const uint32_t m4[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
             const float pas = pa * kSubScale;  // value weights carry the code scale (code_sub)
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
