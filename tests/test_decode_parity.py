@@ -236,7 +236,7 @@ def test_recent_window_bf16_tail(librq, n_tail):
 
 # ---------------------------------------------------------------------------
 # both decode kernels on the same cases: the CUDA-core kernel (64-token pages)
-# and the tensor-core kernel (128-token pages, G in {2, 4, 8})
+# and the tensor-core kernel (128-token pages, G in {1, 2, 4, 8})
 # ---------------------------------------------------------------------------
 TC_FORMATS = {
     # name: (bits, group, rotate, alpha_mode, G values)
