@@ -56,7 +56,10 @@ struct BpCfgN {
   static constexpr int REGS_CONSUMER = (512 * 128 - 128 * kSplitRegsAux) / NCT;
   static_assert(!REGSPLIT || (REGS_CONSUMER % 8 == 0 && 128 * kSplitRegsAux + NCT * REGS_CONSUMER == 512 * 128),
                 "register split");
-  static constexpr int NT = REGSPLIT ? NCT + 128 : S::NT;
+  // two producer warps (see the kernel) for up to two links; with the
+  // register split the second is one of the producer warpgroup's idle warps
+  static constexpr int NPROD = NCH <= 2 ? 2 : 1;
+  static constexpr int NT = REGSPLIT ? NCT + 128 : NCT + 32 * NPROD;
   static constexpr int TW = TT / kGW;   // tokens of a warp's quarter of a page
   static_assert(TW == 32, "phase 1.5 takes one token per lane");
   static constexpr bool ANCH = REF == kRefInt4;
@@ -181,29 +184,38 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
   const int64_t x1 = static_cast<int64_t>(blockIdx.x + 1) * total / P_eff;
   const int n_pages = static_cast<int>(x1 - x0);
 
-  // ========================= producer warp =========================
+  // ========================= producer warps =========================
+  // Two producer threads: the first fills the even stages, the second the odd
+  // ones, so that a stage is always filled by the same thread.  A page's copy
+  // instructions take a producer thread long enough that one thread alone held
+  // the consumers back on these small-record formats.
   if (warp >= NCW) {
     if constexpr (C::REGSPLIT) tc::setmaxnreg_dec<kSplitRegsAux>();
-    if (warp == NCW && lane == 0) {
+    const int pw = warp - NCW;
+    if (pw < C::NPROD && lane == 0) {
       PageIter it;
       it.seek(x0, sPre, sNt, B, Hkv);
       int k = 0;
       for (; k < n_pages; ++k) {
         const int s = k % C::STAGES;
-        if (!mbar_wait_bounded(smem_u32(&bars[C::STAGES + s]), ((k / C::STAGES) & 1) ^ 1)) {
-          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-          *sAbort = 1;
-          break;
+        if (C::NPROD == 1 || (s & 1) == pw) {
+          if (!mbar_wait_bounded(smem_u32(&bars[C::STAGES + s]), ((k / C::STAGES) & 1) ^ 1)) {
+            set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+            *sAbort = 1;
+            break;
+          }
+          if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[C::BAR_NEVER]), 0))
+            set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+          if (*sAbort) break;
+          issue_page<REF, RB, RG, 1, TT, NCH, NG>(P, &tmK, &tmV, stages + s * S::STAGE_BYTES, smem_u32(&bars[s]), it,
+                                                  Hkv);
         }
-        if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[C::BAR_NEVER]), 0))
-          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-        if (*sAbort) break;
-        issue_page<REF, RB, RG, 1, TT, NCH, NG>(P, &tmK, &tmV, stages + s * S::STAGE_BYTES, smem_u32(&bars[s]), it,
-                                                Hkv);
         it.next(sNt, B, Hkv);
       }
-      // drain: no copy this CTA issued may still be landing when it exits
+      // drain: no copy this thread issued may still be landing when it exits
+      // (each of its stages' last page: nothing later went into those stages)
       for (int kk = (k > C::STAGES ? k - C::STAGES : 0); kk < k; ++kk) {
+        if (C::NPROD == 2 && ((kk % C::STAGES) & 1) != pw) continue;
         if (!mbar_wait_bounded(smem_u32(&bars[kk % C::STAGES]), (kk / C::STAGES) & 1)) {
           set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
           break;

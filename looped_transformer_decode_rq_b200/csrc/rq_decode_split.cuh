@@ -12,7 +12,8 @@
 //     contiguous ranges of equal length, so ragged batches balance to within
 //     one page; a CTA emits one partial (m, l, acc) per (b, kv-head) segment
 //     it touches;
-//   * the last warp is the producer: one lane streams pages into a ring of
+//   * two warps after the consumers are the producers: one lane of each
+//     (the even stages, the odd stages) streams pages into a ring of
 //     shared-memory stages through the Tensor Memory Accelerator -- tiled
 //     tensor copies with the 128-byte swizzle for bf16 anchor tiles, bulk
 //     copies for code, metadata and alpha records -- completing on mbarriers;
@@ -85,7 +86,8 @@ struct Cfg {
   // four query rows with residual links hold more than 168 registers a
   // consumer thread: those variants take the register split
   static constexpr bool REGSPLIT = NG == 2 && G >= 4 && RB != 0 && REF != kRefNone;
-  static constexpr int NT = NCT + (REGSPLIT ? 128 : 32);  // + producer warp (+ three idle warps)
+  // + two producer warps (+ two idle warps with the register split)
+  static constexpr int NT = NCT + (REGSPLIT ? 128 : 64);
   static_assert(G <= NCW, "one warp per query head in the segment set-up");
   static constexpr int PAGE = TT;  // tokens per page / stage
   // phase 1 (scores): 4G lanes per token, D1 = 32/G dims per lane
@@ -407,9 +409,13 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
   const int n_pages = static_cast<int>(x1 - x0);
 
   // ========================= producer warp =========================
+  // Two producer threads: the first fills the even stages, the second the odd
+  // ones (a stage is always filled by the same thread).  A page's copy
+  // instructions keep a producer thread busy for most of a page's time.
   if (warp >= kNCW) {
     if constexpr (C::REGSPLIT) tc::setmaxnreg_dec<kSplitRegsAux>();
-    if (warp == kNCW && lane == 0) {
+    const int pw = warp - kNCW;
+    if (pw < 2 && lane == 0) {
       if constexpr (REF == kRefBf16) {
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
@@ -419,18 +425,23 @@ __global__ void __launch_bounds__(Cfg<REF, RB, RG, G, TT, NCH, NG>::NT, 1)
       int k = 0;
       for (; k < n_pages; ++k) {
         const int s = k % C::STAGES;
-        if (!mbar_wait_bounded(smem_u32(&bars[C::STAGES + s]), ((k / C::STAGES) & 1) ^ 1)) {
-          set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-          *sAbort = 1;
-          break;
+        if ((s & 1) == pw) {
+          if (!mbar_wait_bounded(smem_u32(&bars[C::STAGES + s]), ((k / C::STAGES) & 1) ^ 1)) {
+            set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+            *sAbort = 1;
+            break;
+          }
+          if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[15]), 0)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
+          if (*sAbort) break;
+          issue_page<REF, RB, RG, G, TT, NCH, NG>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it,
+                                                  Hkv);
         }
-        if (k == P.stall_page && !mbar_wait_bounded(smem_u32(&bars[15]), 0)) set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
-        if (*sAbort) break;
-        issue_page<REF, RB, RG, G, TT, NCH, NG>(P, &tmK, &tmV, stages + s * C::STAGE_BYTES, smem_u32(&bars[s]), it, Hkv);
         it.next(sNt, B, Hkv);
       }
-      // Drain: no copy this CTA issued may still be landing when it exits.
+      // Drain: no copy this thread issued may still be landing when it exits
+      // (each of its stages' last page: nothing later went into those stages).
       for (int kk = (k > C::STAGES ? k - C::STAGES : 0); kk < k; ++kk) {
+        if (((kk % C::STAGES) & 1) != pw) continue;
         if (!mbar_wait_bounded(smem_u32(&bars[kk % C::STAGES]), (kk / C::STAGES) & 1)) {
           set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
           break;
