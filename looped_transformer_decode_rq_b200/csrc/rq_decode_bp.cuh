@@ -56,9 +56,10 @@ struct BpCfgN {
   static constexpr int REGS_CONSUMER = (512 * 128 - 128 * kSplitRegsAux) / NCT;
   static_assert(!REGSPLIT || (REGS_CONSUMER % 8 == 0 && 128 * kSplitRegsAux + NCT * REGS_CONSUMER == 512 * 128),
                 "register split");
-  // two producer warps (see the kernel) for up to two links; with the
-  // register split the second is one of the producer warpgroup's idle warps
-  static constexpr int NPROD = NCH <= 2 ? 2 : 1;
+  // three producer warps (see the kernel) for up to two links (two measured
+  // 1.3% slower on the [2,2,4,4] step, one 7.5%); the three-link variant keeps
+  // one (two measured 10% slower there)
+  static constexpr int NPROD = NCH <= 2 ? 3 : 1;
   static constexpr int NT = REGSPLIT ? NCT + 128 : NCT + 32 * NPROD;
   static constexpr int TW = TT / kGW;   // tokens of a warp's quarter of a page
   static_assert(TW == 32, "phase 1.5 takes one token per lane");
@@ -185,8 +186,8 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
   const int n_pages = static_cast<int>(x1 - x0);
 
   // ========================= producer warps =========================
-  // Two producer threads: the first fills the even stages, the second the odd
-  // ones, so that a stage is always filled by the same thread.  A page's copy
+  // NPROD producer threads: producer p fills the stages s with s % NPROD == p,
+  // so that a stage is always filled by the same thread.  A page's copy
   // instructions take a producer thread long enough that one thread alone held
   // the consumers back on these small-record formats.
   if (warp >= NCW) {
@@ -198,7 +199,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
       int k = 0;
       for (; k < n_pages; ++k) {
         const int s = k % C::STAGES;
-        if (C::NPROD == 1 || (s & 1) == pw) {
+        if (s % C::NPROD == pw) {
           if (!mbar_wait_bounded(smem_u32(&bars[C::STAGES + s]), ((k / C::STAGES) & 1) ^ 1)) {
             set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
             *sAbort = 1;
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(BpCfg<REF, RB, RG, NCH>::NT, 1)
       // drain: no copy this thread issued may still be landing when it exits
       // (each of its stages' last page: nothing later went into those stages)
       for (int kk = (k > C::STAGES ? k - C::STAGES : 0); kk < k; ++kk) {
-        if (C::NPROD == 2 && ((kk % C::STAGES) & 1) != pw) continue;
+        if ((kk % C::STAGES) % C::NPROD != pw) continue;
         if (!mbar_wait_bounded(smem_u32(&bars[kk % C::STAGES]), (kk / C::STAGES) & 1)) {
           set_flag(P.status, RQ_FLAG_PIPE_TIMEOUT);
           break;
