@@ -10,7 +10,8 @@
 // per-token arithmetic, not HBM, sets the pace; this kernel is organised to
 // spend as few instructions per token as it can:
 //   * pages of 128 tokens stream into a shared ring exactly as for the other
-//     kernel (one TMA producer warp, three groups of four consumer warps, a
+//     kernel (TMA producer warps -- three, each filling its own stages, or one
+//     with three links -- three groups of four consumer warps, a
 //     page per group in turn), but each warp owns a 32-token quarter of its
 //     group's pages and keeps its own online softmax: no barrier is taken per
 //     page, only the stage's release counts the four warps;
